@@ -1,0 +1,77 @@
+"""The seeded input generator (CPU only): known-answer values of its random
+number generator and the structure of the five decode workloads."""
+import numpy as np
+import pytest
+
+import synth
+from synth.workloads import bf16_bits_to_f32, f32_to_bf16_bits, normals, philox4x32_10
+
+
+def test_philox_known_answers():
+    # Known-answer vectors of Philox4x32-10 (Salmon et al., SC 2011).
+    assert list(philox4x32_10([0, 0, 0, 0], [0, 0])) == [0x6627E8D5, 0xE169C58D, 0xBC57AC4C, 0x9B00DBD8]
+    ff = 0xFFFFFFFF
+    assert list(philox4x32_10([ff] * 4, [ff] * 2)) == [0x408F276D, 0x41C83B0E, 0xA20BC7C6, 0x6D5451FD]
+
+
+def test_normals_moments_and_determinism():
+    a = normals(123, 0, (1 << 20,), "f32")
+    b = normals(123, 0, (1 << 20,), "f32")
+    c = normals(123, 1, (1 << 20,), "f32")
+    assert np.array_equal(a, b) and not np.array_equal(a, c)
+    assert abs(a.mean()) < 5e-3 and abs(a.std() - 1.0) < 5e-3
+    assert abs((np.abs(a) < 1.0).mean() - 0.6827) < 3e-3
+
+
+def test_bf16_rounding_nearest_even():
+    x = np.array([1.0, 1.0 + 2**-8, 1.0 + 3 * 2**-8, -2.5, 1.0 + 2**-9, 1.0 + 2**-8 + 2**-20], np.float32)
+    back = bf16_bits_to_f32(f32_to_bf16_bits(x))
+    # bf16 spacing at 1.0 is 2^-7: exact halves go to the even mantissa
+    expect = np.array([1.0, 1.0, 1.0 + 2**-6, -2.5, 1.0, 1.0 + 2**-7], np.float32)
+    assert np.array_equal(back, expect)
+    assert normals(5, 0, (64,), "bf16").dtype == np.uint16
+
+
+@pytest.mark.parametrize("cid", [1, 2, 3, 4, 5])
+def test_config_structure(cid):
+    c = synth.make_config(cid, values=False)
+    lo, hi = {1: (17, 33), 2: (128, 2048), 3: (512, 4096), 4: (32768, 131072), 5: (16, 16384)}[cid]
+    assert c.context_lens.min() >= lo and c.context_lens.max() <= hi
+    assert c.B == {1: 2, 2: 32, 3: 128, 4: 8, 5: 256}[cid]
+    bs = c.block_size
+    used = []
+    for b in range(c.B):
+        L = int(c.context_lens[b])
+        n = -(-L // bs)
+        row = c.block_tables[b]
+        assert np.all(row[:n] >= 0) and np.all(row[:n] < c.num_blocks)
+        assert np.all(row[n:] == -1)
+        pos = L - 1
+        assert c.slot_mapping[b] == row[pos // bs] * bs + pos % bs
+        used.extend(int(x) for x in row[:n])
+    if cid == 5:
+        # first full blocks are shared inside each group of 8; append slots stay private
+        for gk in range(0, c.B, 8):
+            for b in range(gk, gk + 8):
+                ns = min(4, (int(c.context_lens[b]) - 1) // bs)
+                ref = [b2 for b2 in range(gk, gk + 8) if min(4, (int(c.context_lens[b2]) - 1) // bs) >= ns]
+                for b2 in ref:
+                    assert np.array_equal(c.block_tables[b, :ns], c.block_tables[b2, :ns])
+        slots_blocks = set(int(s) // bs for s in c.slot_mapping)
+        assert len(slots_blocks) == c.B
+        assert c.unique_blocks() < c.blocks_used()
+    else:
+        assert len(set(used)) == len(used)        # no block is shared
+    if cid == 3:
+        assert c.num_blocks == int(np.ceil(1.5 * c.blocks_used()))
+    if cid == 1:
+        assert c.num_blocks == 8 and c.dtype == "f32"
+    if cid == 4:
+        assert c.partition_tokens == 512 and c.Hkv == 1 and c.block_size == 256
+
+
+def test_config_is_deterministic():
+    a = synth.make_config(1)
+    b = synth.make_config(1)
+    for f in ("q", "k_new", "v_new", "k_cache", "v_cache", "block_tables", "slot_mapping", "context_lens"):
+        assert np.array_equal(getattr(a, f), getattr(b, f))
