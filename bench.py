@@ -1,0 +1,328 @@
+"""Benchmark: one decode step = pa_kv_append + pa_decode over one batch.
+
+Default workload: the Qwen3-0.6B-shaped decode batch (B=32, Hq=16, Hkv=8,
+D=128, block_size=16, context lengths ~ U[128, 2048], bf16, shuffled pool).
+Metric: paged-decode attention HBM GB/s (algorithmic bytes of the step /
+device time of the step) and us per decode step.
+
+  python bench.py [--gpus N] [--steps K] [--warmup W] [--config 1..5] [--impl reference]
+
+Timing: inputs resident in HBM; R copies of the whole step's inputs are used
+in rotation so that the working set of consecutive steps exceeds the L2
+cache; the K timed steps are bracketed by a barrier and a device synchronise
+and measured with CUDA events on the launching stream (max over ranks).  The
+decode kernel's own duration is taken with events around every launch.
+Under torchrun each rank runs its own batch (weak scaling, no collective on
+the data path).
+"""
+from __future__ import annotations
+
+import argparse
+import hashlib
+import json
+import math
+import os
+import statistics
+import sys
+import threading
+import time
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+import numpy as np  # noqa: E402
+
+FALLBACK_HBM_GBS = 6650.0
+
+
+def parse():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=4000)
+    ap.add_argument("--warmup", type=int, default=50)
+    ap.add_argument("--config", type=int, default=2)
+    ap.add_argument("--partition", type=int, default=-1, help="-1: the workload's own (0 = balanced)")
+    ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--cpu-seconds", type=float, default=10.0)
+    ap.add_argument("--e2e-steps", type=int, default=200)
+    return ap.parse_args()
+
+
+def csrc_hash() -> str:
+    h = hashlib.sha256()
+    d = os.path.join(ROOT, "paged_kv_cache_472_b200", "csrc")
+    for fn in sorted(os.listdir(d)):
+        h.update(fn.encode())
+        h.update(open(os.path.join(d, fn), "rb").read())
+    return h.hexdigest()[:16]
+
+
+def measured_peak():
+    try:
+        with open(os.path.join(ROOT, "MEASURED_PEAKS.json")) as f:
+            return float(json.load(f)["hbm_gbs"]), "measured"
+    except Exception:
+        return FALLBACK_HBM_GBS, "fallback"
+
+
+def profiled_traffic(workload: str):
+    """DRAM bytes per decode launch from the committed ncu summary, if it was
+    taken on the current kernel sources."""
+    path = os.path.join(ROOT, "profiles", "decode_traffic.json")
+    try:
+        with open(path) as f:
+            rec = json.load(f)
+        ent = rec.get(workload)
+        if ent and ent.get("csrc_hash") == csrc_hash():
+            return float(ent["dram_bytes_per_launch"])
+    except Exception:
+        pass
+    return None
+
+
+class ClockSampler:
+    """SM clock and throttle reasons sampled with NVML while the timed region runs."""
+
+    REASONS = {0x1: "gpu_idle", 0x2: "applications_clocks_setting", 0x4: "sw_power_cap", 0x8: "hw_slowdown",
+               0x10: "sync_boost", 0x20: "sw_thermal_slowdown", 0x40: "hw_thermal_slowdown",
+               0x80: "hw_power_brake_slowdown", 0x100: "display_clock_setting"}
+
+    def __init__(self, index: int, period_s: float = 0.01):
+        self.samples, self.reasons, self.ok = [], 0, False
+        self.period, self.stop_ev = period_s, threading.Event()
+        try:
+            import pynvml
+            pynvml.nvmlInit()
+            self.nv = pynvml
+            self.h = pynvml.nvmlDeviceGetHandleByIndex(index)
+            self.max_mhz = pynvml.nvmlDeviceGetMaxClockInfo(self.h, pynvml.NVML_CLOCK_SM)
+            self.ok = True
+        except Exception:
+            self.max_mhz = None
+
+    def _run(self):
+        nv = self.nv
+        while not self.stop_ev.is_set():
+            try:
+                self.samples.append(nv.nvmlDeviceGetClockInfo(self.h, nv.NVML_CLOCK_SM))
+                self.reasons |= nv.nvmlDeviceGetCurrentClocksEventReasons(self.h)
+            except Exception:
+                pass
+            time.sleep(self.period)
+
+    def __enter__(self):
+        if self.ok:
+            self.t = threading.Thread(target=self._run, daemon=True)
+            self.t.start()
+        return self
+
+    def __exit__(self, *a):
+        if self.ok:
+            self.stop_ev.set()
+            self.t.join()
+
+    def summary(self):
+        if not self.ok or not self.samples:
+            return {"sm_mhz": None, "sm_max_mhz": self.max_mhz, "reasons": ["unavailable"]}
+        names = [n for bit, n in self.REASONS.items() if self.reasons & bit and n != "gpu_idle"]
+        return {"sm_mhz": float(statistics.median(self.samples)), "sm_max_mhz": self.max_mhz, "reasons": names,
+                "samples": len(self.samples)}
+
+
+# ---------------------------------------------------------------------------
+def cpu_baseline(case, seconds: float):
+    """The float64 oracle as it stands (append + decode of the whole batch),
+    repeated for about `seconds` on the host cores."""
+    import oracle
+    from synth import algorithmic_bytes
+    orc = oracle.default()
+    nbytes = algorithmic_bytes(case)["step_total"]
+    steps, t0 = 0, time.perf_counter()
+    while True:
+        kc, vc = orc.kv_append(case)
+        orc.decode(case, kc, vc)
+        steps += 1
+        el = time.perf_counter() - t0
+        if el >= seconds:
+            break
+    cores = orc.max_threads()
+    return {"value": nbytes * steps / el / 1e9, "unit": "GB/s", "cores": cores, "kind": "oracle",
+            "sample": f"{steps} full steps (append + decode of all {case.B} requests) of {case.name} in {el:.1f} s",
+            "ms_per_step": el / steps * 1e3}
+
+
+def run_reference(args):
+    import synth
+    rank = int(os.environ.get("RANK", "0"))
+    if rank != 0:
+        return
+    case = synth.make_config(args.config)
+    from synth import algorithmic_bytes
+    base = cpu_baseline(case, max(args.cpu_seconds, 1.0) if args.steps else args.cpu_seconds)
+    line = {"impl": "reference", "metric": "paged-decode attention HBM GB/s (% of B200 peak); us/decode step",
+            "value": base["value"], "unit": "GB/s", "n_gpus": args.gpus, "steps": args.steps,
+            "warmup": args.warmup, "ms_per_step": base["ms_per_step"], "higher_is_better": True,
+            "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic",
+            "config": {"workload": case.name, "B": case.B, "Hq": case.Hq, "Hkv": case.Hkv, "D": case.D,
+                       "block_size": case.block_size, "bytes_per_step": algorithmic_bytes(case)["step_total"]},
+            "cpu_baseline": {k: base[k] for k in ("kind", "cores", "sample", "value", "unit")},
+            "e2e": {"value": base["value"], "unit": "GB/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
+            "gpu_launches": 0}
+    print(json.dumps(line), flush=True)
+
+
+# ---------------------------------------------------------------------------
+def main():
+    args = parse()
+    if args.impl == "reference":
+        return run_reference(args)
+
+    import torch
+    import torch.distributed as dist
+
+    import synth
+    from synth import algorithmic_bytes
+    from paged_kv_cache_472_b200 import build as libbuild
+    libbuild.build()
+    import paged_kv_cache_472_b200 as pa
+    from paged_kv_cache_472_b200.session import PagedDecoder
+    from tests import gpu_harness as H
+
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    torch.cuda.set_device(local)
+    if world > 1:
+        from datetime import timedelta
+        dist.init_process_group("nccl", timeout=timedelta(seconds=120))
+
+    # each rank decodes its own batch of the workload (distinct seed per rank)
+    base_case = synth.make_config(args.config, seed=None if rank == 0 else 1000 + args.config + 7919 * rank)
+    pt = base_case.partition_tokens if args.partition < 0 else args.partition
+    ab = algorithmic_bytes(base_case)
+    step_bytes = ab["step_total"]
+    decode_bytes = ab["decode_total"]
+    l2 = torch.cuda.get_device_properties(local).L2_cache_size
+    R = max(3, math.ceil(3 * l2 / max(step_bytes, 1)))
+    copies = [H.upload(base_case) for _ in range(R)]
+    shape = H.shape_of(base_case)
+    dec = PagedDecoder(shape, int(base_case.max_blocks_per_seq * base_case.block_size), pt)
+    stream = torch.cuda.current_stream()
+    sp = stream.cuda_stream
+
+    # raw pointers, so the launch loop is two plain C calls
+    lib, byref = pa.lib, __import__("ctypes").byref
+    shp, pln = byref(dec.shape), byref(dec.plan)
+    ws, wsb = dec.workspace.data_ptr(), dec.workspace.numel()
+    ptrs = [(c.k_new.data_ptr(), c.v_new.data_ptr(), c.slot_mapping.data_ptr(), c.k_cache.data_ptr(),
+             c.v_cache.data_ptr(), c.q.data_ptr(), c.block_tables.data_ptr(), c.context_lens.data_ptr(),
+             c.out.data_ptr()) for c in copies]
+    scale = float(base_case.scale)
+
+    def step(i, ev=None):
+        kn, vn, sm, kc, vc, q, bt, cl, out = ptrs[i % R]
+        st = lib.pa_kv_append(kn, vn, sm, kc, vc, shp, ws, sp)
+        if ev is not None:
+            ev[0].record(stream)
+        st |= lib.pa_decode(q, kc, vc, bt, cl, scale, out, shp, pln, ws, wsb, sp)
+        if ev is not None:
+            ev[1].record(stream)
+        return st
+
+    for i in range(args.warmup):
+        if step(i):
+            raise RuntimeError(pa.pa_last_error_message())
+    torch.cuda.synchronize()
+    if world > 1:
+        dist.barrier()
+    torch.cuda.synchronize()
+
+    K = args.steps
+    kev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)) for _ in range(K)]
+    start, end = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    with ClockSampler(local) as clk:
+        torch.cuda._sleep(20_000_000)          # keep the queue ahead of the GPU (not timed)
+        start.record(stream)
+        for i in range(K):
+            step(i, kev[i])
+        end.record(stream)
+        torch.cuda.synchronize()
+    if world > 1:
+        dist.barrier()
+    ms_total = start.elapsed_time(end)
+    dec_ms = [a.elapsed_time(b) for a, b in kev]
+    t = torch.tensor([ms_total], device="cuda", dtype=torch.float64)
+    if world > 1:
+        dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    ms_total = float(t.item())
+    ms_step = ms_total / K
+    err = dec.device_error()
+    if err:
+        raise RuntimeError(f"device error word {err:#x}")
+
+    # ---- end to end: host buffers through the same C calls ----
+    E = args.e2e_steps
+    c0 = copies[0]
+    host_in = {n: getattr(c0, n).cpu().pin_memory() for n in ("q", "k_new", "v_new", "slot_mapping",
+                                                               "block_tables", "context_lens")}
+    host_out = torch.empty(c0.out.shape, dtype=c0.out.dtype).pin_memory()
+    h2d = sum(v.numel() * v.element_size() for v in host_in.values())
+    d2h = host_out.numel() * host_out.element_size()
+    kn, vn, sm, kc, vc, q, bt, cl, out = ptrs[0]
+    torch.cuda.synchronize()
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    e0.record(stream)
+    for i in range(E):
+        for n, hv in host_in.items():
+            getattr(c0, n).copy_(hv, non_blocking=True)
+        lib.pa_kv_append(kn, vn, sm, kc, vc, shp, ws, sp)
+        lib.pa_decode(q, kc, vc, bt, cl, scale, out, shp, pln, ws, wsb, sp)
+        host_out.copy_(c0.out, non_blocking=True)
+    e1.record(stream)
+    torch.cuda.synchronize()
+    e2e_ms = e0.elapsed_time(e1) / E
+    te = torch.tensor([e2e_ms], device="cuda", dtype=torch.float64)
+    if world > 1:
+        dist.all_reduce(te, op=dist.ReduceOp.MAX)
+    e2e_ms = float(te.item())
+
+    if rank == 0:
+        peak, peak_kind = measured_peak()
+        dec_avg_ms = sum(dec_ms) / len(dec_ms)
+        achieved = decode_bytes / (dec_avg_ms * 1e-3) / 1e9
+        value = world * step_bytes / (ms_step * 1e-3) / 1e9
+        line = {
+            "metric": "paged-decode attention HBM GB/s (% of B200 peak); us/decode step",
+            "value": round(value, 2), "unit": "GB/s", "n_gpus": world, "steps": K, "warmup": args.warmup,
+            "ms_per_step": round(ms_step, 6), "us_per_step": round(ms_step * 1e3, 3),
+            "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": base_case.dtype,
+            "data": "synthetic",
+            "config": {"workload": base_case.name, "B": base_case.B, "Hq": base_case.Hq, "Hkv": base_case.Hkv,
+                       "D": base_case.D, "block_size": base_case.block_size,
+                       "context_tokens": int(base_case.context_lens.sum()), "partition_tokens": pt,
+                       "bytes_per_step": step_bytes, "decode_bytes_per_step": decode_bytes,
+                       "l2": f"{R} rotating input copies, {R * step_bytes / 1e6:.0f} MB > L2 {l2 / 1e6:.0f} MB",
+                       "parallelism": f"replicas x{world}" if world > 1 else "1 GPU",
+                       "tokens_per_s": round(world * base_case.B / (ms_step * 1e-3), 1),
+                       "pct_of_peak": round(100 * value / world / peak, 2)},
+            "roofline": {"bound": "hbm", "achieved": round(achieved, 2), "peak": peak, "unit": "GB/s",
+                         "frac": round(achieved / peak, 4), "traffic": profiled_traffic(base_case.name),
+                         "kernel": "paged_decode_kernel", "peak_kind": peak_kind,
+                         "decode_us": round(dec_avg_ms * 1e3, 3)},
+            "e2e": {"value": round(world * step_bytes / (e2e_ms * 1e-3) / 1e9, 2), "unit": "GB/s",
+                    "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h, "us_per_step": round(e2e_ms * 1e3, 3)},
+            "gpu_launches": 2 * K,
+            "clocks": clk.summary(),
+        }
+        if not args.no_cpu_baseline:
+            cb = cpu_baseline(base_case, args.cpu_seconds)
+            line["cpu_baseline"] = {k: cb[k] for k in ("value", "unit", "cores", "kind", "sample")}
+        print(json.dumps(line), flush=True)
+    if world > 1:
+        dist.barrier()
+        dist.destroy_process_group()
+
+
+if __name__ == "__main__":
+    main()

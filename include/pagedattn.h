@@ -1,0 +1,177 @@
+/*
+ * libpagedattn -- one-token batched decode attention read directly from a
+ * paged KV cache, and the per-step KV append that feeds it (NVIDIA B200,
+ * sm_100a).
+ *
+ * The operations follow the pages on mini vLLM-style engines:
+ *   - paged storage: per layer, K and V tensors shaped
+ *     [num_blocks, block_size, Hkv, D] in token-before-head (NHD) order, one
+ *     fixed-size physical block per block-table entry (BareLLM README, cache
+ *     section and "Cache layers" bullets);
+ *   - address translation: position t of request b lives in physical block
+ *     block_tables[b][t / block_size] at row t % block_size (BareLLM README,
+ *     cache section; Nano-vLLM overview, "Kernmodul: Sequence");
+ *   - decode: for every request and query head, softmax(q . K^T * scale) . V
+ *     over that request's own context length, for MHA, GQA and MQA
+ *     (BareLLM README feature list), computed with a running max and sum
+ *     (MinivLLM review, engine layout section; LLAISYS self-attention bullet)
+ *     and, for long contexts, split over context partitions whose partial
+ *     results are combined by log-sum-exp;
+ *   - append: PagedKVCache's logical-to-physical write of each request's new
+ *     token (BareLLM README component list).
+ *
+ * Conventions for every entry point:
+ *   - All device pointers are caller-owned; the library never allocates,
+ *     frees or synchronises inside pa_kv_append / pa_decode.  Work is queued
+ *     on `stream` (a cudaStream_t; NULL = the legacy default stream).
+ *   - Errors are returned as pa_status; nothing throws across the ABI.
+ *     pa_last_error_message() gives a one-line reason for the last non-OK
+ *     status returned on the calling host thread.
+ *   - Value tensors (q, k/v cache, k/v new, out) have dtype s->dtype and must
+ *     be 16-byte aligned.  Index tensors are int32.
+ *   - Nothing falls back silently: shapes outside the supported set return
+ *     PA_ERR_UNSUPPORTED.
+ */
+#ifndef PAGEDATTN_H
+#define PAGEDATTN_H
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef enum {
+    PA_OK = 0,
+    PA_ERR_INVALID_ARG = 1,  /* null/misaligned pointer, inconsistent shape or plan */
+    PA_ERR_UNSUPPORTED = 2,  /* a valid shape this build does not implement */
+    PA_ERR_CUDA = 3,         /* a CUDA runtime call or kernel launch failed */
+    PA_ERR_WORKSPACE = 4     /* workspace missing or smaller than the plan needs */
+} pa_status;
+
+typedef enum { PA_DTYPE_F32 = 0, PA_DTYPE_BF16 = 1 } pa_dtype;
+
+/* Bits of the device error word (see pa_get_device_error).  Kernels never
+ * trap: an out-of-range index is recorded here and the access is skipped. */
+#define PA_DEVERR_BLOCK_ID    0x1  /* a block-table entry outside [0, num_blocks) */
+#define PA_DEVERR_CONTEXT_LEN 0x2  /* context_lens[b] < 0 or > max_blocks_per_seq*block_size */
+#define PA_DEVERR_TIMEOUT     0x4  /* a pipeline wait gave up (internal error) */
+#define PA_DEVERR_WORKSPACE   0x8  /* more partitions than the plan provided for */
+#define PA_DEVERR_SLOT        0x10 /* an append slot >= num_blocks*block_size */
+
+/* Problem shape.  B requests, Hq query heads, Hkv KV heads (Hq % Hkv == 0;
+ * query head h reads KV head h / (Hq/Hkv)), head dim D, block_size tokens per
+ * physical block, num_blocks blocks in the pool, max_blocks_per_seq columns
+ * in the block table. */
+typedef struct {
+    int32_t B, Hq, Hkv, D;
+    int32_t block_size, num_blocks, max_blocks_per_seq;
+    int32_t dtype; /* pa_dtype */
+} pa_shape;
+
+/* How a decode call splits its work (filled by pa_plan; treat as opaque). */
+typedef enum {
+    PA_SPLIT_BALANCED = 0, /* persistent CTAs, equal token share each, split anywhere */
+    PA_SPLIT_FIXED = 1     /* fixed partitions of partition_tokens tokens per request */
+} pa_split_mode;
+
+typedef struct {
+    int32_t mode;             /* pa_split_mode */
+    int32_t partition_tokens; /* PA_SPLIT_FIXED: tokens per partition */
+    int32_t num_ctas;         /* persistent CTAs launched */
+    int32_t tile_tokens;      /* tokens staged per pipeline stage */
+    int32_t stages;           /* pipeline depth */
+    int32_t head_group;       /* KV heads handled per work item */
+    int32_t heads_per_unit;   /* query heads one warp carries */
+    int32_t units_per_warp;
+    int32_t warps_per_unit;   /* >1: a warp team splits the tokens of one unit */
+    int32_t max_context_len;  /* the bound the workspace was sized for */
+    int32_t smem_bytes;
+    int32_t reserved;
+    int64_t max_slots;        /* partial-result slots in the workspace */
+    pa_shape shape;           /* the shape this plan was made for */
+    size_t workspace_bytes;   /* bytes pa_decode needs at `workspace` */
+} pa_plan_t;
+
+/* Library version: major*10000 + minor*100 + patch. */
+int32_t pa_version(void);
+
+const char *pa_status_str(pa_status st);
+
+/* One-line reason for the last non-OK status on this host thread ("" if none). */
+const char *pa_last_error_message(void);
+
+/*
+ * KV append (BareLLM README: PagedKVCache's logical-to-physical writes).
+ * For each i < s->B with slot = slot_mapping[i] >= 0:
+ *     k_cache[slot / block_size][slot % block_size][:][:] = k_new[i][:][:]
+ * and the same for V; slot < 0 skips request i.
+ *   k_new, v_new : device, [B, Hkv, D], dtype s->dtype
+ *   slot_mapping : device, [B] int32, slot = physical_block*block_size + row
+ *   k_cache, v_cache : device, [num_blocks, block_size, Hkv, D], updated in place
+ *   device_error : device int32 or NULL; a slot >= num_blocks*block_size is
+ *                  skipped and, if non-NULL, PA_DEVERR_SLOT is OR-ed in.
+ * Non-negative slots must be distinct (two writes to one slot race).
+ * Only s->B, Hkv, D, block_size, num_blocks and dtype are read from s.
+ */
+pa_status pa_kv_append(const void *k_new, const void *v_new, const int32_t *slot_mapping, void *k_cache,
+                       void *v_cache, const pa_shape *s, int32_t *device_error, void *stream);
+
+/*
+ * Host-only planner (no device work, no allocation).
+ *   max_context_len : the largest context_lens[b] any later call will pass;
+ *                     bounds the workspace of PA_SPLIT_FIXED.
+ *   partition_tokens: 0 = PA_SPLIT_BALANCED (persistent CTAs with an equal
+ *                     share of all requests' tokens each); > 0 =
+ *                     PA_SPLIT_FIXED with partitions of that many tokens (a
+ *                     multiple of 16); >= max_context_len gives one partition
+ *                     per request (no split).
+ *   num_sms         : SM count to size the grid for; 0 = query the current
+ *                     CUDA device.
+ * Returns PA_ERR_UNSUPPORTED for shapes the kernels do not cover:
+ * D not in {64, 128}; block_size not a power of two in [16, 256]; a GQA
+ * group Hq/Hkv that is not a power of two <= 64; more query heads than one
+ * CTA can carry.
+ */
+pa_status pa_plan(const pa_shape *s, int32_t max_context_len, int32_t partition_tokens, int32_t num_sms,
+                  pa_plan_t *plan_out);
+
+/* Bytes of device workspace pa_decode needs for `plan` (== plan->workspace_bytes). */
+size_t pa_decode_workspace_size(const pa_plan_t *plan);
+
+/* Zero a workspace before its first pa_decode (the kernels leave it ready
+ * for the next call afterwards).  Queued on `stream`. */
+pa_status pa_workspace_init(void *workspace, size_t workspace_bytes, void *stream);
+
+/*
+ * Decode attention over the paged cache.
+ *   q            : device, [B, Hq, D] (NHD), dtype s->dtype
+ *   k_cache/v_cache : device, [num_blocks, block_size, Hkv, D]
+ *   block_tables : device, [B, max_blocks_per_seq] int32; entries past
+ *                  ceil(context_lens[b]/block_size) are never read
+ *   context_lens : device, [B] int32, tokens of request b (0 gives out = 0)
+ *   scale        : softmax scale (typically 1/sqrt(D))
+ *   out          : device, [B, Hq, D], dtype s->dtype (fp32 results rounded
+ *                  to nearest-even for bf16)
+ *   plan         : from pa_plan for the same *s
+ *   workspace    : device, >= plan->workspace_bytes, 256-byte aligned,
+ *                  zeroed once by pa_workspace_init; holds partial results,
+ *                  merge counters and the device error word.  Two calls that
+ *                  overlap on the GPU must not share a workspace.
+ * out[b][h] = sum_t softmax_t(scale * q[b][h] . K[t]) V[t], t < context_lens[b],
+ * with K[t], V[t] the rows of KV head h / (Hq/Hkv) found through the table.
+ */
+pa_status pa_decode(const void *q, const void *k_cache, const void *v_cache, const int32_t *block_tables,
+                    const int32_t *context_lens, float scale, void *out, const pa_shape *s,
+                    const pa_plan_t *plan, void *workspace, size_t workspace_bytes, void *stream);
+
+/* Copy the device error word of `workspace` to *err_out (synchronises
+ * `stream`; not for the hot path).  clear != 0 resets it to 0 afterwards. */
+pa_status pa_get_device_error(void *workspace, int32_t clear, int32_t *err_out, void *stream);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* PAGEDATTN_H */

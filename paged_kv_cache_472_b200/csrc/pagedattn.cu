@@ -1,0 +1,358 @@
+// C ABI of libpagedattn: argument validation, the host-side planner and
+// kernel dispatch.  Declarations and contracts live in include/pagedattn.h.
+#include <cmath>
+#include <cstdarg>
+#include <cstdio>
+#include <cstring>
+#include <mutex>
+
+#include "append.cuh"
+#include "decode.cuh"
+
+namespace {
+
+thread_local char g_msg[256] = "";
+
+pa_status fail(pa_status st, const char *fmt, ...) {
+    va_list ap;
+    va_start(ap, fmt);
+    vsnprintf(g_msg, sizeof g_msg, fmt, ap);
+    va_end(ap);
+    return st;
+}
+
+pa_status ok() {
+    g_msg[0] = '\0';
+    return PA_OK;
+}
+
+bool aligned16(const void *p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
+bool pow2(int x) { return x > 0 && (x & (x - 1)) == 0; }
+int elem_bytes(int dtype) { return dtype == PA_DTYPE_F32 ? 4 : 2; }
+size_t round_up(size_t x, size_t a) { return (x + a - 1) / a * a; }
+
+constexpr int kSmemLimit = 232448;     // opt-in dynamic shared memory per CTA on sm_100
+constexpr size_t kWsHeader = 256;      // error word + reserved
+constexpr int kStageTargetBytes = 32768;  // K bytes per stage (V the same)
+constexpr int kMaxStages = 4;
+
+pa_status check_shape(const pa_shape *s) {
+    if (!s) return fail(PA_ERR_INVALID_ARG, "shape is NULL");
+    if (s->B < 0) return fail(PA_ERR_INVALID_ARG, "B=%d < 0", s->B);
+    if (s->Hq <= 0 || s->Hkv <= 0) return fail(PA_ERR_INVALID_ARG, "Hq=%d Hkv=%d must be > 0", s->Hq, s->Hkv);
+    if (s->Hq % s->Hkv) return fail(PA_ERR_INVALID_ARG, "Hq=%d is not a multiple of Hkv=%d", s->Hq, s->Hkv);
+    if (s->D <= 0 || s->block_size <= 0 || s->num_blocks <= 0 || s->max_blocks_per_seq <= 0)
+        return fail(PA_ERR_INVALID_ARG, "D, block_size, num_blocks, max_blocks_per_seq must be > 0");
+    if (s->dtype != PA_DTYPE_F32 && s->dtype != PA_DTYPE_BF16)
+        return fail(PA_ERR_INVALID_ARG, "dtype=%d is not a pa_dtype", s->dtype);
+    if ((int64_t)s->num_blocks * s->block_size > INT32_MAX)
+        return fail(PA_ERR_UNSUPPORTED, "num_blocks*block_size exceeds the int32 slot range");
+    if ((int64_t)s->max_blocks_per_seq * s->block_size > INT32_MAX)
+        return fail(PA_ERR_UNSUPPORTED, "max_blocks_per_seq*block_size exceeds int32");
+    return PA_OK;
+}
+
+// ---------------------------------------------------------------------------
+// decode kernel variants: (dtype, D, HC, UPW)
+using KernelFn = void (*)(const pa::DecodeParams);
+
+template <typename T, int D>
+KernelFn pick_hc_upw(int hc, int upw) {
+#define PA_CASE(H, U) \
+    if (hc == H && upw == U) return pa::paged_decode_kernel<T, D, H, U>;
+    PA_CASE(1, 1) PA_CASE(2, 1) PA_CASE(4, 1) PA_CASE(1, 2) PA_CASE(2, 2) PA_CASE(4, 2) PA_CASE(1, 4) PA_CASE(2, 4)
+#undef PA_CASE
+    return nullptr;
+}
+
+KernelFn pick_kernel(int dtype, int D, int hc, int upw) {
+    if (dtype == PA_DTYPE_BF16) {
+        if (D == 64) return pick_hc_upw<__nv_bfloat16, 64>(hc, upw);
+        if (D == 128) return pick_hc_upw<__nv_bfloat16, 128>(hc, upw);
+    } else {
+        if (D == 64) return pick_hc_upw<float, 64>(hc, upw);
+        if (D == 128) return pick_hc_upw<float, 128>(hc, upw);
+    }
+    return nullptr;
+}
+
+std::mutex g_attr_mu;
+
+pa_status ensure_smem_attr(KernelFn fn, int bytes) {
+    // cudaFuncSetAttribute is cheap but not free; remember the largest size set per kernel.
+    static struct {
+        KernelFn fn;
+        int bytes;
+    } seen[64];
+    static int nseen = 0;
+    std::lock_guard<std::mutex> lk(g_attr_mu);
+    for (int i = 0; i < nseen; ++i)
+        if (seen[i].fn == fn && seen[i].bytes >= bytes) return PA_OK;
+    cudaError_t e = cudaFuncSetAttribute(fn, cudaFuncAttributeMaxDynamicSharedMemorySize, bytes);
+    if (e != cudaSuccess) return fail(PA_ERR_CUDA, "cudaFuncSetAttribute: %s", cudaGetErrorString(e));
+    for (int i = 0; i < nseen; ++i)
+        if (seen[i].fn == fn) {
+            seen[i].bytes = bytes;
+            return PA_OK;
+        }
+    if (nseen < 64) seen[nseen++] = {fn, bytes};
+    return PA_OK;
+}
+
+struct Layout {
+    uint32_t off_bar, off_q, off_stage, off_scratch, off_comb, total;
+};
+
+Layout smem_layout(int stages, uint32_t q_bytes, uint32_t half_bytes, int hc, int D, int tsplit) {
+    Layout l;
+    l.off_bar = 0;
+    const uint32_t bar_bytes = (uint32_t)round_up((2 * stages + 4) * 8, 128);
+    l.off_q = bar_bytes;
+    l.off_stage = (uint32_t)round_up(l.off_q + 2 * q_bytes, 128);
+    l.off_scratch = (uint32_t)round_up(l.off_stage + (size_t)stages * 2 * half_bytes, 128);
+    const uint32_t scratch = pa::kConsumerWarps * 2 * pa::kSubTile * hc * 4;
+    l.off_comb = (uint32_t)round_up(l.off_scratch + scratch, 128);
+    const uint32_t comb = tsplit > 1 ? pa::kConsumerWarps * (uint32_t)(hc * D + 8) * 4 : 0;
+    l.total = (uint32_t)round_up(l.off_comb + comb, 128);
+    return l;
+}
+
+}  // namespace
+
+extern "C" {
+
+int32_t pa_version(void) { return 100; }
+
+const char *pa_status_str(pa_status st) {
+    switch (st) {
+        case PA_OK: return "PA_OK";
+        case PA_ERR_INVALID_ARG: return "PA_ERR_INVALID_ARG";
+        case PA_ERR_UNSUPPORTED: return "PA_ERR_UNSUPPORTED";
+        case PA_ERR_CUDA: return "PA_ERR_CUDA";
+        case PA_ERR_WORKSPACE: return "PA_ERR_WORKSPACE";
+    }
+    return "PA_ERR_UNKNOWN";
+}
+
+const char *pa_last_error_message(void) { return g_msg; }
+
+pa_status pa_kv_append(const void *k_new, const void *v_new, const int32_t *slot_mapping, void *k_cache,
+                       void *v_cache, const pa_shape *s, int32_t *device_error, void *stream) {
+    if (pa_status st = check_shape(s)) return st;
+    if (s->B == 0) return ok();
+    if (!k_new || !v_new || !slot_mapping || !k_cache || !v_cache)
+        return fail(PA_ERR_INVALID_ARG, "NULL tensor pointer");
+    if (!aligned16(k_new) || !aligned16(v_new) || !aligned16(k_cache) || !aligned16(v_cache))
+        return fail(PA_ERR_INVALID_ARG, "value tensors must be 16-byte aligned");
+    const int64_t token_bytes = (int64_t)s->Hkv * s->D * elem_bytes(s->dtype);
+    if (token_bytes % 16) return fail(PA_ERR_UNSUPPORTED, "Hkv*D*elem=%lld is not a multiple of 16", (long long)token_bytes);
+    const int vec = (int)(token_bytes / 16);
+    const int64_t total = (int64_t)s->B * vec;
+    const int threads = 256;
+    int64_t blocks = (total + threads - 1) / threads;
+    if (blocks > 148 * 16) blocks = 148 * 16;
+    pa::kv_append_kernel<<<(unsigned)blocks, threads, 0, (cudaStream_t)stream>>>(
+        (const uint4 *)k_new, (const uint4 *)v_new, slot_mapping, (uint4 *)k_cache, (uint4 *)v_cache, s->B, vec,
+        (int64_t)s->num_blocks * s->block_size, device_error);
+    cudaError_t e = cudaGetLastError();
+    if (e != cudaSuccess) return fail(PA_ERR_CUDA, "append launch: %s", cudaGetErrorString(e));
+    return ok();
+}
+
+pa_status pa_plan(const pa_shape *s, int32_t max_context_len, int32_t partition_tokens, int32_t num_sms,
+                  pa_plan_t *plan) {
+    if (!plan) return fail(PA_ERR_INVALID_ARG, "plan_out is NULL");
+    if (pa_status st = check_shape(s)) return st;
+    const int cap = s->max_blocks_per_seq * s->block_size;
+    if (max_context_len < 0 || max_context_len > cap)
+        return fail(PA_ERR_INVALID_ARG, "max_context_len=%d outside [0, %d]", max_context_len, cap);
+    if (partition_tokens < 0) return fail(PA_ERR_INVALID_ARG, "partition_tokens=%d < 0", partition_tokens);
+    if (s->D != 64 && s->D != 128) return fail(PA_ERR_UNSUPPORTED, "D=%d (supported: 64, 128)", s->D);
+    if (!pow2(s->block_size) || s->block_size < 16 || s->block_size > 256)
+        return fail(PA_ERR_UNSUPPORTED, "block_size=%d (supported: powers of two in [16, 256])", s->block_size);
+    const int G = s->Hq / s->Hkv;
+    if (!pow2(G) || G > 64) return fail(PA_ERR_UNSUPPORTED, "GQA group %d (supported: powers of two <= 64)", G);
+    const int e = elem_bytes(s->dtype);
+
+    if (num_sms <= 0) {
+        int dev = 0;
+        cudaError_t ce = cudaGetDevice(&dev);
+        if (ce == cudaSuccess) ce = cudaDeviceGetAttribute(&num_sms, cudaDevAttrMultiProcessorCount, dev);
+        if (ce != cudaSuccess) return fail(PA_ERR_CUDA, "querying the SM count: %s", cudaGetErrorString(ce));
+    }
+
+    // Head group HG (KV heads per work item), heads per warp unit HC, units
+    // per warp UPW and warps per unit (token split).
+    int HG = 0, HC = 0, UPW = 0, TS = 0;
+    for (int hg = s->Hkv; hg >= 1 && !HG; --hg) {
+        if (s->Hkv % hg || hg * s->D * e > 2048) continue;
+        for (int hc = 4; hc >= 1; hc >>= 1) {
+            if (G % hc) continue;
+            const int U = hg * (G / hc);
+            if (U >= 8) {
+                if (U % 8) continue;
+                const int upw = U / 8;
+                if (upw > 4 || upw * hc > 8 || (upw == 4 && hc > 2)) continue;
+                HG = hg, HC = hc, UPW = upw, TS = 1;
+                break;
+            }
+        }
+        if (!HG && s->Hkv % hg == 0 && hg * s->D * e <= 2048) {
+            const int U = hg * G;  // HC = 1
+            if (U < 8 && 8 % U == 0) HG = hg, HC = 1, UPW = 1, TS = 8 / U;
+        }
+    }
+    if (!HG) return fail(PA_ERR_UNSUPPORTED, "no warp mapping for Hq=%d Hkv=%d D=%d", s->Hq, s->Hkv, s->D);
+    const int NHvr = HG * G;
+    const int NHG = s->Hkv / HG;
+    const uint32_t row_bytes = (uint32_t)(HG * s->D * e);
+    const uint32_t q_bytes = (uint32_t)(NHvr * s->D * e);
+
+    int ST = 16;
+    while (ST * 2 <= 256 && (uint32_t)(ST * 2) * row_bytes <= (uint32_t)kStageTargetBytes) ST *= 2;
+    int mode = PA_SPLIT_BALANCED, part_tiles = 1;
+    if (partition_tokens > 0) {
+        if (partition_tokens % 16) return fail(PA_ERR_INVALID_ARG, "partition_tokens=%d is not a multiple of 16", partition_tokens);
+        mode = PA_SPLIT_FIXED;
+        while (partition_tokens % ST) ST /= 2;  // tiles must not straddle partitions
+        part_tiles = partition_tokens / ST;
+    }
+    int stages = 0;
+    Layout lay{};
+    for (;;) {
+        const uint32_t half = (uint32_t)ST * row_bytes;
+        for (stages = kMaxStages; stages >= 2; --stages) {
+            lay = smem_layout(stages, q_bytes, half, HC, s->D, TS);
+            if (lay.total + 256 <= (uint32_t)kSmemLimit) break;
+        }
+        if (stages >= 2) break;
+        if (ST == 16 || mode == PA_SPLIT_FIXED) return fail(PA_ERR_UNSUPPORTED, "shared memory too small for this shape");
+        ST /= 2;
+    }
+
+    memset(plan, 0, sizeof *plan);
+    plan->mode = mode;
+    plan->partition_tokens = mode == PA_SPLIT_FIXED ? partition_tokens : 0;
+    plan->num_ctas = num_sms;
+    plan->tile_tokens = ST;
+    plan->stages = stages;
+    plan->head_group = HG;
+    plan->heads_per_unit = HC;
+    plan->units_per_warp = UPW;
+    plan->warps_per_unit = TS;
+    plan->max_context_len = max_context_len;
+    plan->smem_bytes = (int32_t)lay.total;
+    plan->shape = *s;
+    if (mode == PA_SPLIT_BALANCED) {
+        plan->max_slots = 2LL * num_sms;
+    } else {
+        const int64_t parts = (max_context_len + partition_tokens - 1) / partition_tokens;
+        plan->max_slots = (int64_t)NHG * s->B * (parts > 1 ? parts : 0);
+    }
+    const size_t slot_floats = (size_t)NHvr * s->D + round_up(2 * NHvr, 4);
+    const size_t counters = round_up((size_t)s->B * NHG * 4, 256);
+    plan->workspace_bytes = kWsHeader + counters + (size_t)plan->max_slots * slot_floats * 4;
+    return ok();
+}
+
+size_t pa_decode_workspace_size(const pa_plan_t *plan) { return plan ? plan->workspace_bytes : 0; }
+
+pa_status pa_workspace_init(void *workspace, size_t workspace_bytes, void *stream) {
+    if (!workspace) return fail(PA_ERR_INVALID_ARG, "workspace is NULL");
+    cudaError_t e = cudaMemsetAsync(workspace, 0, workspace_bytes, (cudaStream_t)stream);
+    if (e != cudaSuccess) return fail(PA_ERR_CUDA, "cudaMemsetAsync: %s", cudaGetErrorString(e));
+    return ok();
+}
+
+pa_status pa_decode(const void *q, const void *k_cache, const void *v_cache, const int32_t *block_tables,
+                    const int32_t *context_lens, float scale, void *out, const pa_shape *s, const pa_plan_t *plan,
+                    void *workspace, size_t workspace_bytes, void *stream) {
+    if (pa_status st = check_shape(s)) return st;
+    if (!plan) return fail(PA_ERR_INVALID_ARG, "plan is NULL");
+    if (memcmp(&plan->shape, s, sizeof *s) != 0) return fail(PA_ERR_INVALID_ARG, "plan was made for another shape");
+    if (!std::isfinite(scale)) return fail(PA_ERR_INVALID_ARG, "scale is not finite");
+    if (!workspace) return fail(PA_ERR_WORKSPACE, "workspace is NULL");
+    if (workspace_bytes < plan->workspace_bytes)
+        return fail(PA_ERR_WORKSPACE, "workspace %zu bytes < %zu needed", workspace_bytes, plan->workspace_bytes);
+    if ((reinterpret_cast<uintptr_t>(workspace) & 255u) != 0) return fail(PA_ERR_INVALID_ARG, "workspace must be 256-byte aligned");
+    if (s->B == 0) return ok();
+    if (!q || !k_cache || !v_cache || !block_tables || !context_lens || !out)
+        return fail(PA_ERR_INVALID_ARG, "NULL tensor pointer");
+    if (!aligned16(q) || !aligned16(k_cache) || !aligned16(v_cache) || !aligned16(out))
+        return fail(PA_ERR_INVALID_ARG, "value tensors must be 16-byte aligned");
+
+    const int HC = plan->heads_per_unit, UPW = plan->units_per_warp, TS = plan->warps_per_unit;
+    const int G = s->Hq / s->Hkv;
+    const int e = elem_bytes(s->dtype);
+    KernelFn fn = pick_kernel(s->dtype, s->D, HC, UPW);
+    if (!fn) return fail(PA_ERR_INVALID_ARG, "plan names no kernel variant");
+    const int HG = plan->head_group;
+    const int NHvr = HG * G;
+    const uint32_t row_bytes = (uint32_t)(HG * s->D * e);
+    const uint32_t half = (uint32_t)plan->tile_tokens * row_bytes;
+    const uint32_t q_bytes = (uint32_t)(NHvr * s->D * e);
+    const Layout lay = smem_layout(plan->stages, q_bytes, half, HC, s->D, TS);
+    if ((int)lay.total != plan->smem_bytes) return fail(PA_ERR_INVALID_ARG, "plan is inconsistent");
+
+    pa::DecodeParams p{};
+    p.q = q;
+    p.k_cache = k_cache;
+    p.v_cache = v_cache;
+    p.block_tables = block_tables;
+    p.context_lens = context_lens;
+    p.out = out;
+    unsigned char *ws = static_cast<unsigned char *>(workspace);
+    const size_t counters = round_up((size_t)s->B * (s->Hkv / HG) * 4, 256);
+    p.error = reinterpret_cast<int32_t *>(ws);
+    p.counters = reinterpret_cast<int32_t *>(ws + kWsHeader);
+    p.partials = reinterpret_cast<float *>(ws + kWsHeader + counters);
+    p.qscale = scale * 1.4426950408889634f;
+    p.B = s->B;
+    p.Hq = s->Hq;
+    p.Hkv = s->Hkv;
+    p.bs = s->block_size;
+    p.num_blocks = s->num_blocks;
+    p.max_blocks = s->max_blocks_per_seq;
+    p.G = G;
+    p.HG = HG;
+    p.NHG = s->Hkv / HG;
+    p.NHvr = NHvr;
+    p.ST = plan->tile_tokens;
+    p.stages = plan->stages;
+    p.mode = plan->mode;
+    p.part_tiles = plan->mode == PA_SPLIT_FIXED ? plan->partition_tokens / plan->tile_tokens : 1;
+    p.num_ctas = plan->num_ctas;
+    p.tsplit = TS;
+    p.units = HG * (G / HC);
+    p.max_slots = plan->max_slots;
+    p.slot_floats = (int64_t)NHvr * s->D + (int64_t)round_up(2 * NHvr, 4);
+    p.off_bar = lay.off_bar;
+    p.off_q = lay.off_q;
+    p.off_stage = lay.off_stage;
+    p.off_scratch = lay.off_scratch;
+    p.off_comb = lay.off_comb;
+    p.row_bytes = row_bytes;
+    p.half_bytes = half;
+    p.q_bytes = q_bytes;
+
+    if (pa_status st = ensure_smem_attr(fn, plan->smem_bytes)) return st;
+    fn<<<plan->num_ctas, pa::kDecodeThreads, plan->smem_bytes, (cudaStream_t)stream>>>(p);
+    cudaError_t ce = cudaGetLastError();
+    if (ce != cudaSuccess) return fail(PA_ERR_CUDA, "decode launch: %s", cudaGetErrorString(ce));
+    return ok();
+}
+
+pa_status pa_get_device_error(void *workspace, int32_t clear, int32_t *err_out, void *stream) {
+    if (!workspace || !err_out) return fail(PA_ERR_INVALID_ARG, "NULL pointer");
+    cudaStream_t st = (cudaStream_t)stream;
+    cudaError_t e = cudaMemcpyAsync(err_out, workspace, sizeof(int32_t), cudaMemcpyDeviceToHost, st);
+    if (e == cudaSuccess) e = cudaStreamSynchronize(st);
+    if (e == cudaSuccess && clear) {
+        e = cudaMemsetAsync(workspace, 0, sizeof(int32_t), st);
+        if (e == cudaSuccess) e = cudaStreamSynchronize(st);
+    }
+    if (e != cudaSuccess) return fail(PA_ERR_CUDA, "reading the error word: %s", cudaGetErrorString(e));
+    return ok();
+}
+
+}  // extern "C"

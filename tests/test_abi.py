@@ -1,0 +1,148 @@
+"""The C ABI without a GPU: the library loads, exports every declared symbol,
+plans the five workloads, and rejects bad arguments with a status (never a
+crash).  No call here launches a kernel."""
+import ctypes
+import os
+import re
+
+import pytest
+
+from paged_kv_cache_472_b200 import build as _build
+
+_build.build()
+import paged_kv_cache_472_b200 as pa  # noqa: E402
+import synth  # noqa: E402
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+
+
+def declared_symbols():
+    names = set()
+    for fn in os.listdir(os.path.join(ROOT, "include")):
+        if fn.endswith(".h"):
+            src = open(os.path.join(ROOT, "include", fn)).read()
+            src = re.sub(r"/\*.*?\*/", "", src, flags=re.S)
+            names.update(re.findall(r"\b(pa_[a-z0-9_]+)\s*\(", src))
+    return sorted(names)
+
+
+def test_every_declared_symbol_is_exported():
+    names = declared_symbols()
+    assert len(names) >= 9, names
+    for n in names:
+        assert hasattr(pa.lib, n), n
+
+
+def test_status_strings_and_version():
+    assert pa.pa_status_str(0) == "PA_OK"
+    assert pa.pa_status_str(4) == "PA_ERR_WORKSPACE"
+    assert pa.pa_version() >= 100
+
+
+def shape_of(case):
+    return pa.Shape(case.B, case.Hq, case.Hkv, case.D, case.block_size, case.num_blocks,
+                    case.max_blocks_per_seq, pa.DTYPE_F32 if case.dtype == "f32" else pa.DTYPE_BF16)
+
+
+@pytest.mark.parametrize("cid", [1, 2, 3, 4, 5])
+def test_plan_workloads(cid):
+    c = synth.make_config(cid, values=False)
+    s = shape_of(c)
+    plan = pa.pa_plan(s, int(c.max_blocks_per_seq * c.block_size), c.partition_tokens, 148)
+    G = c.Hq // c.Hkv
+    assert plan.num_ctas == 148
+    assert plan.smem_bytes <= 232448 - 256
+    assert plan.stages >= 2
+    assert plan.head_group * plan.heads_per_unit >= 1
+    units = plan.head_group * G // plan.heads_per_unit
+    assert units == 8 * plan.units_per_warp or units * plan.warps_per_unit == 8
+    assert plan.tile_tokens >= 16 and plan.tile_tokens & (plan.tile_tokens - 1) == 0
+    assert pa.pa_decode_workspace_size(plan) == plan.workspace_bytes
+    if c.partition_tokens:
+        assert plan.mode == pa.SPLIT_FIXED and plan.partition_tokens % plan.tile_tokens == 0
+    else:
+        assert plan.mode == pa.SPLIT_BALANCED and plan.max_slots == 2 * 148
+    expect = {1: (2, 1, 2), 2: (8, 2, 1), 3: (8, 4, 1), 4: (1, 4, 1), 5: (8, 4, 1)}[cid]
+    assert (plan.head_group, plan.heads_per_unit, plan.warps_per_unit) == expect
+
+
+@pytest.mark.parametrize("Hq,Hkv,D,upw,hc,hg,ts", [
+    (32, 32, 128, 1, 1, 8, 1), (16, 16, 64, 2, 1, 16, 1), (64, 16, 64, 2, 4, 16, 1), (32, 16, 64, 2, 2, 16, 1),
+    (64, 16, 128, 1, 4, 8, 1), (4, 1, 128, 1, 1, 1, 2), (8, 1, 128, 1, 1, 1, 1), (64, 1, 128, 2, 4, 1, 1),
+    (2, 2, 64, 1, 1, 2, 4), (1, 1, 64, 1, 1, 1, 8)])
+def test_plan_head_mappings(Hq, Hkv, D, upw, hc, hg, ts):
+    s = pa.Shape(3, Hq, Hkv, D, 16, 64, 8, pa.DTYPE_BF16)
+    plan = pa.pa_plan(s, 128, 0, 148)
+    assert (plan.units_per_warp, plan.heads_per_unit, plan.head_group, plan.warps_per_unit) == (upw, hc, hg, ts)
+
+
+@pytest.mark.parametrize("mut,status", [
+    (dict(D=96), pa.PA_ERR_UNSUPPORTED), (dict(block_size=8), pa.PA_ERR_UNSUPPORTED),
+    (dict(block_size=48), pa.PA_ERR_UNSUPPORTED), (dict(Hq=12, Hkv=4), pa.PA_ERR_UNSUPPORTED),
+    (dict(Hq=10, Hkv=4), pa.PA_ERR_INVALID_ARG), (dict(dtype=7), pa.PA_ERR_INVALID_ARG),
+    (dict(B=-1), pa.PA_ERR_INVALID_ARG), (dict(num_blocks=0), pa.PA_ERR_INVALID_ARG),
+])
+def test_plan_rejects(mut, status):
+    base = dict(B=2, Hq=8, Hkv=2, D=128, block_size=16, num_blocks=8, max_blocks_per_seq=4, dtype=pa.DTYPE_BF16)
+    base.update(mut)
+    s = pa.Shape(**base)
+    with pytest.raises(pa.PagedAttnError) as ei:
+        pa.pa_plan(s, 32, 0, 148)
+    assert ei.value.status == status
+
+
+def test_plan_rejects_bad_partition_and_context():
+    s = pa.Shape(2, 8, 2, 128, 16, 8, 4, pa.DTYPE_BF16)
+    with pytest.raises(pa.PagedAttnError) as ei:
+        pa.pa_plan(s, 32, 10, 148)
+    assert ei.value.status == pa.PA_ERR_INVALID_ARG
+    with pytest.raises(pa.PagedAttnError) as ei:
+        pa.pa_plan(s, 65, 0, 148)          # > max_blocks_per_seq * block_size
+    assert ei.value.status == pa.PA_ERR_INVALID_ARG
+
+
+def test_fixed_plan_workspace_formula():
+    s = pa.Shape(8, 32, 1, 128, 256, 4096, 512, pa.DTYPE_BF16)
+    plan = pa.pa_plan(s, 131072, 512, 148)
+    assert plan.max_slots == 8 * 256
+    slot_floats = 32 * 128 + 64
+    assert plan.workspace_bytes == 256 + 256 + plan.max_slots * slot_floats * 4
+
+
+FAKE = 1 << 20  # aligned, never dereferenced: every call below fails validation first
+
+
+def _decode(s, plan, **kw):
+    args = dict(q=FAKE, k=FAKE, v=FAKE, tables=FAKE, lens=FAKE, scale=0.1, out=FAKE, ws=FAKE,
+                ws_bytes=plan.workspace_bytes if plan else 0)
+    args.update(kw)
+    return pa.lib.pa_decode(args["q"], args["k"], args["v"], args["tables"], args["lens"], args["scale"], args["out"],
+                            ctypes.byref(s), ctypes.byref(plan) if plan else None, args["ws"], args["ws_bytes"], None)
+
+
+def test_decode_validation_paths():
+    s = pa.Shape(2, 8, 2, 128, 16, 8, 4, pa.DTYPE_BF16)
+    plan = pa.pa_plan(s, 64, 0, 148)
+    assert _decode(s, None) == pa.PA_ERR_INVALID_ARG
+    assert _decode(s, plan, ws_bytes=plan.workspace_bytes - 1) == pa.PA_ERR_WORKSPACE
+    assert _decode(s, plan, ws=0) == pa.PA_ERR_WORKSPACE
+    assert _decode(s, plan, ws=FAKE + 16) == pa.PA_ERR_INVALID_ARG        # not 256-aligned
+    assert _decode(s, plan, q=FAKE + 2) == pa.PA_ERR_INVALID_ARG          # not 16-aligned
+    assert _decode(s, plan, out=0) == pa.PA_ERR_INVALID_ARG
+    assert _decode(s, plan, scale=float("nan")) == pa.PA_ERR_INVALID_ARG
+    s2 = pa.Shape(2, 8, 2, 128, 16, 9, 4, pa.DTYPE_BF16)                 # plan made for another shape
+    assert _decode(s2, plan) == pa.PA_ERR_INVALID_ARG
+    s0 = pa.Shape(0, 8, 2, 128, 16, 8, 4, pa.DTYPE_BF16)
+    plan0 = pa.pa_plan(s0, 64, 0, 148)
+    assert _decode(s0, plan0) == pa.PA_OK                                 # empty batch: nothing to launch
+    assert "plan" in pa.pa_last_error_message() or pa.pa_last_error_message() == ""
+
+
+def test_append_validation_paths():
+    s = pa.Shape(2, 8, 2, 128, 16, 8, 4, pa.DTYPE_BF16)
+    f = pa.lib.pa_kv_append
+    assert f(FAKE, FAKE, FAKE, FAKE, 0, ctypes.byref(s), None, None) == pa.PA_ERR_INVALID_ARG
+    assert f(FAKE + 4, FAKE, FAKE, FAKE, FAKE, ctypes.byref(s), None, None) == pa.PA_ERR_INVALID_ARG
+    s0 = pa.Shape(0, 8, 2, 128, 16, 8, 4, pa.DTYPE_BF16)
+    assert f(0, 0, 0, 0, 0, ctypes.byref(s0), None, None) == pa.PA_OK
+    assert f(FAKE, FAKE, FAKE, FAKE, FAKE, None, None, None) == pa.PA_ERR_INVALID_ARG

@@ -1,0 +1,176 @@
+"""pa_decode against the float64 oracle on the same seeded inputs.
+
+Full outputs at sizes the oracle finishes in seconds (several tiles, ragged
+tails, every split mode); sampled (request, head) outputs at the full sizes
+of the five workloads, in the launch configuration the benchmark times
+(balanced split, one CTA per SM)."""
+import zlib
+
+import numpy as np
+import pytest
+import torch
+
+import synth
+from paged_kv_cache_472_b200 import DEVERR_BLOCK_ID, DEVERR_CONTEXT_LEN
+from tests import gpu_harness as H
+
+pytestmark = pytest.mark.gpu
+
+
+_REF = {}
+
+
+def oracle_out(orc, case):
+    key = (case.name, case.seed)
+    if key not in _REF:
+        _REF[key] = orc.decode(case)
+    return _REF[key]
+
+
+def check_full(orc, case, partition_tokens=0, what=""):
+    dev, dec, err = H.run(case, partition_tokens)
+    assert err == 0, f"device error word {err:#x}"
+    ref = oracle_out(orc, case)
+    H.assert_close(H.out_f64(dev), ref, case.dtype, what or case.name)
+    return dev
+
+
+# ---- the five workloads, full outputs (smaller batches where the oracle needs it) ----
+@pytest.mark.parametrize("cid,batch", [(1, None), (2, None), (3, 32), (4, 2), (5, 48)])
+@pytest.mark.parametrize("partition", ["balanced", "fixed", "none"])
+def test_workloads_full_output(orc, cid, batch, partition):
+    case = synth.make_config(cid, batch=batch)
+    pt = {"balanced": 0, "fixed": case.partition_tokens or 256,
+          "none": int(case.max_blocks_per_seq * case.block_size)}[partition]
+    check_full(orc, case, pt, f"{case.name}/{partition}")
+
+
+# ---- full sizes, sampled outputs, launch configuration of the benchmark ----
+@pytest.mark.parametrize("cid", [2, 3, 4, 5])
+def test_workloads_full_size_sampled(orc, cid):
+    case = synth.make_config(cid)
+    dev, dec, err = H.run(case, case.partition_tokens)
+    assert err == 0
+    pairs = H.sample_pairs(case, 48, seed=cid)
+    kc, vc = orc.kv_append(case)
+    ref = orc.decode_pairs(case, pairs, kc, vc)
+    got = H.out_f64(dev)[pairs[:, 0], pairs[:, 1]]
+    H.assert_close(got, ref, case.dtype, f"{case.name} sampled")
+    assert np.all(np.isfinite(H.out_f64(dev)))
+    if case.partition_tokens:   # also the balanced split on the same inputs
+        dev2, _, err2 = H.run(case, 0, dev=H.upload(case))
+        assert err2 == 0
+        got2 = H.out_f64(dev2)[pairs[:, 0], pairs[:, 1]]
+        H.assert_close(got2, ref, case.dtype, f"{case.name} sampled balanced")
+
+
+def test_split_equals_unsplit(orc):
+    """Balanced, fixed and unsplit launches agree with each other (and the oracle)."""
+    case = synth.make_config(4, batch=2)
+    outs = []
+    for pt in (0, 512, 2048, int(case.max_blocks_per_seq * case.block_size)):
+        dev, _, err = H.run(case, pt)
+        assert err == 0
+        outs.append(H.out_f64(dev))
+    for o in outs[1:]:
+        H.assert_close(o, outs[0], case.dtype, "split vs split")
+
+
+# ---- edge shapes ----
+EDGE = [
+    # name, dtype, Hq, Hkv, D, bs, lens
+    ("len1", "bf16", 16, 8, 128, 16, [1, 1, 2, 1]),
+    ("exact_blocks", "bf16", 32, 8, 64, 16, [16, 32, 48, 256]),
+    ("block_pm1", "bf16", 16, 8, 128, 16, [15, 17, 31, 33, 47, 49]),
+    ("mha8", "bf16", 8, 8, 128, 16, [5, 100, 300]),
+    ("mha32_headgroups", "bf16", 32, 32, 128, 16, [40, 333, 17]),
+    ("mha16_d64_two_units", "bf16", 16, 16, 64, 16, [77, 250, 1]),
+    ("gqa4_d64_hkv16", "bf16", 64, 16, 64, 32, [300, 65, 2]),
+    ("mqa8", "bf16", 8, 1, 128, 16, [1000, 3, 129]),
+    ("mqa4_tsplit", "bf16", 4, 1, 128, 64, [700, 64, 65]),
+    ("mqa32", "bf16", 32, 1, 128, 256, [3000, 257, 1]),
+    ("mqa64", "bf16", 64, 1, 64, 128, [1500, 130]),
+    ("gqa16", "bf16", 32, 2, 128, 32, [900, 31, 2]),
+    ("tiny_heads", "bf16", 2, 2, 64, 16, [50, 3]),
+    ("one_head", "f32", 1, 1, 64, 16, [33, 80]),
+    ("f32_gqa4", "f32", 16, 4, 128, 32, [129, 500, 31]),
+    ("f32_d64_bs256", "f32", 8, 2, 64, 256, [600, 256, 257]),
+    ("bs128_d128", "bf16", 16, 8, 128, 128, [129, 1024, 383]),
+    ("single_request", "bf16", 16, 8, 128, 16, [4000]),
+]
+
+
+@pytest.mark.parametrize("name,dtype,Hq,Hkv,D,bs,lens", EDGE, ids=[e[0] for e in EDGE])
+@pytest.mark.parametrize("pt", [0, 64])
+def test_edge_shapes(orc, name, dtype, Hq, Hkv, D, bs, lens, pt):
+    case = synth.build_case(name, dtype=dtype, Hq=Hq, Hkv=Hkv, D=D, block_size=bs, context_lens=lens,
+                            seed=zlib.crc32(name.encode()) % 100000, pool="factor", pool_factor=1.25)
+    check_full(orc, case, pt, f"{name}/pt{pt}")
+
+
+def test_many_short_requests(orc):
+    """More requests than CTAs; many requests inside one CTA's range."""
+    rng = np.random.default_rng(9)
+    lens = rng.integers(1, 40, size=700)
+    case = synth.build_case("many_short", dtype="bf16", Hq=16, Hkv=8, D=128, block_size=16, context_lens=lens,
+                            seed=9)
+    check_full(orc, case, 0)
+
+
+def test_fewer_tiles_than_ctas(orc):
+    case = synth.build_case("few", dtype="bf16", Hq=16, Hkv=8, D=128, block_size=16, context_lens=[20, 3],
+                            seed=10)
+    check_full(orc, case, 0)
+
+
+def test_zero_length_requests_give_zero(orc):
+    case = synth.build_case("zeros", dtype="bf16", Hq=16, Hkv=8, D=128, block_size=16, context_lens=[50, 1, 70],
+                            seed=11)
+    dev = H.upload(case)
+    lens = case.context_lens.copy()
+    lens[1] = 0
+    dev.context_lens = torch.from_numpy(lens).cuda()
+    dev, dec, err = H.run(case, 0, dev=dev, append=False)
+    assert err == 0
+    got = H.out_f64(dev)
+    assert np.all(got[1] == 0.0)
+    ref = orc.decode(case, case.k_cache, case.v_cache, context_lens=lens)
+    H.assert_close(got, ref, "bf16", "zeros")
+
+
+def test_bad_block_id_is_flagged_not_faulted():
+    case = synth.build_case("badid", dtype="bf16", Hq=16, Hkv=8, D=128, block_size=16, context_lens=[40, 70],
+                            seed=12)
+    dev = H.upload(case)
+    tables = case.block_tables.copy()
+    tables[1, 2] = case.num_blocks + 5          # outside the pool
+    dev.block_tables = torch.from_numpy(tables).cuda()
+    dev, dec, err = H.run(case, 0, dev=dev)
+    assert err & DEVERR_BLOCK_ID
+    torch.cuda.synchronize()                      # the context is still usable
+
+
+def test_context_longer_than_table_is_flagged():
+    case = synth.build_case("badlen", dtype="bf16", Hq=16, Hkv=8, D=128, block_size=16, context_lens=[40, 70],
+                            seed=13, max_blocks_per_seq=5)
+    dev = H.upload(case)
+    lens = case.context_lens.copy()
+    lens[1] = 5 * 16 + 7
+    dev.context_lens = torch.from_numpy(lens).cuda()
+    dev, dec, err = H.run(case, 0, dev=dev, max_context_len=80)
+    assert err & DEVERR_CONTEXT_LEN
+
+
+def test_repeated_calls_reuse_workspace(orc):
+    """The merge counters return to zero: the same workspace serves call after call."""
+    case = synth.make_config(2, batch=8)
+    dev, dec, err = H.run(case, 0)
+    first = dev.out.clone()
+    for _ in range(3):
+        dev.out.fill_(float("nan"))
+        dec.decode(dev.q, dev.k_cache, dev.v_cache, dev.block_tables, dev.context_lens, case.scale, dev.out)
+    torch.cuda.synchronize()
+    assert torch.equal(first, dev.out)
+    assert dec.device_error() == 0
+    counters = dec.workspace[256:256 + 4 * case.B * case.Hkv].view(torch.int32)
+    assert int(counters.abs().sum()) == 0
