@@ -166,6 +166,20 @@ pa_status pa_decode(const void *q, const void *k_cache, const void *v_cache, con
                     const int32_t *context_lens, float scale, void *out, const pa_shape *s,
                     const pa_plan_t *plan, void *workspace, size_t workspace_bytes, void *stream);
 
+/*
+ * One decode step: pa_kv_append followed by pa_decode on the same stream,
+ * the decode grid launched as a programmatic dependent of the append grid so
+ * that its prologue (lengths, block table, q) overlaps the append; every K/V
+ * row is read only after the append grid has completed.  Arguments as in the
+ * two calls; the append's slot errors land in the workspace error word.
+ * Requires that nothing but the append writes q, block_tables and
+ * context_lens between the two launches (true by construction here).
+ */
+pa_status pa_kv_append_decode(const void *k_new, const void *v_new, const int32_t *slot_mapping, const void *q,
+                              void *k_cache, void *v_cache, const int32_t *block_tables,
+                              const int32_t *context_lens, float scale, void *out, const pa_shape *s,
+                              const pa_plan_t *plan, void *workspace, size_t workspace_bytes, void *stream);
+
 /* Copy the device error word of `workspace` to *err_out (synchronises
  * `stream`; not for the hot path).  clear != 0 resets it to 0 afterwards. */
 pa_status pa_get_device_error(void *workspace, int32_t clear, int32_t *err_out, void *stream);

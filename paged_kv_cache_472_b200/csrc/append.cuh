@@ -16,6 +16,9 @@ __global__ void __launch_bounds__(256) kv_append_kernel(const uint4 *__restrict_
                                                         uint4 *__restrict__ k_cache, uint4 *__restrict__ v_cache,
                                                         int32_t B, int32_t vec_per_token, int64_t num_slots,
                                                         int32_t *error) {
+    // a decode grid launched after this one may run its prologue meanwhile; it
+    // waits for this grid's completion before reading any K/V row
+    grid_launch_dependents();
     const int64_t total = (int64_t)B * vec_per_token;
     for (int64_t i = (int64_t)blockIdx.x * blockDim.x + threadIdx.x; i < total;
          i += (int64_t)gridDim.x * blockDim.x) {

@@ -1,14 +1,14 @@
-// Paged decode attention for sm_100a (CUDA-core path).
+// Paged decode attention for sm_100a.
 //
 // What it computes (BareLLM README: paged KV cache, block table, one-token
 // batched decode over unequal histories; MHA/GQA/MQA): for every request b
 // and query head h,
 //     out[b][h] = sum_t softmax_t(scale * q[b][h] . K_t) V_t ,  t < L_b,
 // where K_t / V_t is row t % bs of physical block block_tables[b][t / bs] for
-// KV head h / (Hq/Hkv).  The softmax is evaluated with a running maximum and
-// sum (the online softmax of the MinivLLM review and the LLAISYS
-// self-attention bullet), in fp32, in the base-2 domain (q is pre-scaled by
-// scale * log2 e so that every weight is one exp2).
+// KV head h / (Hq/Hkv).  The softmax runs with a running maximum and sum
+// (the online softmax of the MinivLLM review and the LLAISYS self-attention
+// bullet), in fp32, in the base-2 domain (scores are scaled by scale*log2 e
+// so every weight is one exp2).
 //
 // Work decomposition.  A "virtual request" (vr) is one request restricted to
 // a group of HG KV heads (HG = Hkv unless one token of all KV heads is too
@@ -24,20 +24,22 @@
 // the pieces by log-sum-exp and restores the counter to zero (no CTA ever
 // waits for another).
 //
-// Inside a CTA: warp 8 is a producer that walks the block table and issues
-// one bulk asynchronous copy (cp.async.bulk, completion on an mbarrier) per
-// block piece into a ring of `stages` shared-memory stages; a tile of a full
-// head group is one contiguous run of [ST, HG, D] elements per block, so the
-// copy engine moves whole rows and no thread computes addresses per element.
-// Warps 0-7 consume: each owns one (KV head, HC query heads) unit, stages the
-// q slice of its heads in registers, and for every 16 tokens
-//   QK  : lane (slice, token-group) forms 8-element partial dots with packed
-//         fp32x2 FMAs; a reduce-scatter across the D/8 slice lanes finishes
-//         the dots and leaves each lane a few whole scores;
-//   softmax: lanes of each head reduce the tile maximum and sum by shuffles;
-//   PV  : every lane accumulates its 8 output elements of all HC heads.
-// Shared-memory reads are 16-byte row slices of consecutive lanes, so every
-// phase of a warp's load hits 32 distinct banks.
+// Inside a CTA: warp 8 is a producer that walks the block table (a window of
+// 32 entries held in registers, the next window prefetched) and issues bulk
+// asynchronous copies (cp.async.bulk, completion counted on an mbarrier) of
+// whole K/V rows into a ring of shared-memory stages.  Warps 0-7 consume;
+// each owns (KV head, query heads) units of the vr and runs one of two
+// engines over every 16 tokens:
+//   * MmaEngine (bf16): warp-level tensor-core tiles with tokens as the M
+//     dimension: S^T = K Q^T (m16n8k16, K from shared memory by ldmatrix,
+//     Q fragments in registers), online softmax on the accumulator
+//     fragments, then O^T += V^T P^T (V by transposing ldmatrix, P moved into
+//     operand layout by movmatrix).  Stage rows are padded by 16 bytes so the
+//     8 rows of every ldmatrix hit 8 different bank groups.
+//   * CoreEngine (fp32, or any dtype): lanes own 8-element slices of a token
+//     row; packed fp32x2 FMAs form partial dots, a reduce-scatter across the
+//     slice lanes finishes them, and every lane accumulates its 8 output
+//     elements of all its heads.
 #pragma once
 
 #include "common.cuh"
@@ -46,7 +48,8 @@ namespace pa {
 
 constexpr int kConsumerWarps = 8;
 constexpr int kDecodeThreads = (kConsumerWarps + 1) * 32;
-constexpr int kSubTile = 16;  // tokens per online-softmax update
+constexpr int kSubTile = 16;     // tokens per online-softmax update
+constexpr int kMergeParts = 64;  // pieces the shared-memory merge path handles
 
 struct DecodeParams {
     const void *q;
@@ -67,13 +70,17 @@ struct DecodeParams {
     int32_t part_tiles;   // fixed mode: tiles per partition
     int32_t num_ctas;
     int32_t tsplit;       // warps sharing one unit (token split)
-    int32_t units;        // units per vr = HG * G / HC
+    int32_t units;        // units per vr
+    int32_t heads_per_unit;
+    int32_t pdl;          // 1: wait for the preceding grid before the first K/V copy
     int64_t max_slots;
     int64_t slot_floats;  // NHvr * D + (2 * NHvr rounded up to a multiple of 4)
-    uint32_t off_bar, off_q, off_stage, off_scratch, off_comb;
-    uint32_t row_bytes;   // HG * D * elem
-    uint32_t half_bytes;  // ST * row_bytes (K part of a stage; V part follows)
+    uint32_t off_bar, off_q, off_stage, off_scratch, off_comb, off_merge;
+    uint32_t row_bytes;   // HG * D * elem: one token of the head group
+    uint32_t row_pitch;   // bytes between token rows in a stage (row_bytes, or + 16 for ldmatrix)
+    uint32_t half_bytes;  // ST * row_pitch (K part of a stage; V part follows)
     uint32_t q_bytes;     // NHvr * D * elem
+    uint32_t comb_stride; // bytes per warp in the token-split combine area
 };
 
 // ---------------------------------------------------------------------------
@@ -84,7 +91,6 @@ struct Elem;
 template <>
 struct Elem<__nv_bfloat16> {
     static constexpr int kBytes = 2;
-    // 8 consecutive elements -> 4 float2 pairs
     static __device__ __forceinline__ void load8(const void *p, float2 (&v)[4]) {
         const uint4 w = *reinterpret_cast<const uint4 *>(p);
         v[0] = bf16x2_to_float2(w.x);
@@ -94,16 +100,17 @@ struct Elem<__nv_bfloat16> {
     }
     static __device__ __forceinline__ void store8(void *p, const float2 (&v)[4]) {
         uint4 w;
-        __nv_bfloat162 t;
-        t = __floats2bfloat162_rn(v[0].x, v[0].y);
-        w.x = *reinterpret_cast<uint32_t *>(&t);
-        t = __floats2bfloat162_rn(v[1].x, v[1].y);
-        w.y = *reinterpret_cast<uint32_t *>(&t);
-        t = __floats2bfloat162_rn(v[2].x, v[2].y);
-        w.z = *reinterpret_cast<uint32_t *>(&t);
-        t = __floats2bfloat162_rn(v[3].x, v[3].y);
-        w.w = *reinterpret_cast<uint32_t *>(&t);
+        w.x = pack_bf16x2(v[0].x, v[0].y);
+        w.y = pack_bf16x2(v[1].x, v[1].y);
+        w.z = pack_bf16x2(v[2].x, v[2].y);
+        w.w = pack_bf16x2(v[3].x, v[3].y);
         *reinterpret_cast<uint4 *>(p) = w;
+    }
+    static __device__ __forceinline__ void store2(void *p, float a, float b) {
+        *reinterpret_cast<uint32_t *>(p) = pack_bf16x2(a, b);
+    }
+    static __device__ __forceinline__ void store1(void *p, float a) {
+        *reinterpret_cast<__nv_bfloat16 *>(p) = __float2bfloat16_rn(a);
     }
     static __device__ __forceinline__ void store_zero8(void *p) {
         *reinterpret_cast<uint4 *>(p) = make_uint4(0, 0, 0, 0);
@@ -125,6 +132,10 @@ struct Elem<float> {
         reinterpret_cast<float4 *>(p)[0] = make_float4(v[0].x, v[0].y, v[1].x, v[1].y);
         reinterpret_cast<float4 *>(p)[1] = make_float4(v[2].x, v[2].y, v[3].x, v[3].y);
     }
+    static __device__ __forceinline__ void store2(void *p, float a, float b) {
+        *reinterpret_cast<float2 *>(p) = make_float2(a, b);
+    }
+    static __device__ __forceinline__ void store1(void *p, float a) { *reinterpret_cast<float *>(p) = a; }
     static __device__ __forceinline__ void store_zero8(void *p) {
         reinterpret_cast<float4 *>(p)[0] = make_float4(0.f, 0.f, 0.f, 0.f);
         reinterpret_cast<float4 *>(p)[1] = make_float4(0.f, 0.f, 0.f, 0.f);
@@ -171,9 +182,9 @@ struct SegIter {
                 if (++hg == p.NHG) {
                     hg = 0;
                     ++b;
-                    L = (b < p.B) ? clamped_len(p, b) : 0;
-                    units = (b < p.B) ? units_of_len(p, L) : 0;
                     if (b >= p.B) return false;
+                    L = clamped_len(p, b);
+                    units = units_of_len(p, L);
                 }
                 continue;
             }
@@ -184,17 +195,21 @@ struct SegIter {
             s.L = L;
             s.vr_start = vr_start;
             s.units = units;
-            const int tiles = (L + p.ST - 1) / p.ST;
             if (p.mode == PA_SPLIT_BALANCED) {
                 const int64_t end = vr_start + units < hi ? vr_start + units : hi;
                 u1 = (int)(end - vr_start);
                 s.t_begin = u0;
                 s.t_end = u1;
-                const int64_t c0 = cta_of(vr_start, NT, C);
-                const int64_t c1 = cta_of(vr_start + units - 1, NT, C);
-                s.nparts = (int)(c1 - c0 + 1);
+                if (u0 == 0 && u1 == units) {
+                    s.nparts = 1;
+                } else {
+                    const int64_t c0 = cta_of(vr_start, NT, C);
+                    const int64_t c1 = cta_of(vr_start + units - 1, NT, C);
+                    s.nparts = (int)(c1 - c0 + 1);
+                }
                 s.slot = 2 * (int64_t)blockIdx.x + (cur == lo ? 0 : 1);
             } else {
+                const int tiles = (L + p.ST - 1) / p.ST;
                 u1 = u0 + 1;
                 s.t_begin = u0 * p.part_tiles;
                 s.t_end = min(tiles, (u0 + 1) * p.part_tiles);
@@ -216,27 +231,33 @@ struct __align__(16) DecodeCtl {
     int merge_flag;
 };
 
+// slot of piece i of a split vr
+__device__ __forceinline__ int64_t piece_slot(const DecodeParams &p, const Seg &s, int i, int64_t NT, int64_t C) {
+    if (p.mode == PA_SPLIT_BALANCED) {
+        const int64_t c = cta_of(s.vr_start, NT, C) + i;
+        return 2 * c + (s.vr_start <= range_lo(c, NT, C) ? 0 : 1);
+    }
+    return s.vr_start + i;
+}
+
 // ---------------------------------------------------------------------------
-// reduce-scatter of N per-lane values across the RL lanes of a slice group
-// (lane bits below log2(RL)).  Afterwards lane `sl` holds value indices
-// [sl*N/RL, (sl+1)*N/RL) in v[0..), or, when N < RL, index sl / (RL/N) in v[0].
+// reduce-scatter of N per-lane values across the slice lanes (lane bits below
+// log2 of the group).  Each lane stores its values in an order permuted by
+// its own lane bits, so that at every step both partners keep v[0..H) and
+// send v[H..2H): no selects.  Afterwards v[0..) holds value indices
+// [sl*N/RL, (sl+1)*N/RL), or index sl / (RL/N) when N < RL.
 template <int N, int M>
 struct ReduceScatter {
-    static __device__ __forceinline__ void run(float *v, int lane) {
+    static __device__ __forceinline__ void run(float *v) {
         if constexpr (M >= 1) {
             if constexpr (N > 1) {
                 constexpr int H = N / 2;
-                const bool upper = (lane & M) != 0;
 #pragma unroll
-                for (int i = 0; i < H; ++i) {
-                    const float send = upper ? v[i] : v[i + H];
-                    const float keep = upper ? v[i + H] : v[i];
-                    v[i] = keep + __shfl_xor_sync(0xffffffffu, send, M);
-                }
-                ReduceScatter<H, M / 2>::run(v, lane);
+                for (int i = 0; i < H; ++i) v[i] += __shfl_xor_sync(0xffffffffu, v[i + H], M);
+                ReduceScatter<H, M / 2>::run(v);
             } else {
                 v[0] += __shfl_xor_sync(0xffffffffu, v[0], M);
-                ReduceScatter<1, M / 2>::run(v, lane);
+                ReduceScatter<1, M / 2>::run(v);
             }
         }
     }
@@ -244,12 +265,14 @@ struct ReduceScatter {
 
 template <int N>
 struct ReduceScatter<N, 0> {
-    static __device__ __forceinline__ void run(float *, int) {}
+    static __device__ __forceinline__ void run(float *) {}
 };
 
-// ---------------------------------------------------------------------------
+// ===========================================================================
+// CUDA-core engine
+// ===========================================================================
 template <typename T, int D, int HC, int UPW>
-struct Consumer {
+struct CoreEngine {
     static constexpr int RL = D / 8;          // lanes per token row (8 elements each)
     static constexpr int TG = 32 / RL;        // token rows per warp load
     static constexpr int R = kSubTile / TG;   // rounds per sub-tile
@@ -258,6 +281,16 @@ struct Consumer {
     static constexpr int LPH = (32 / HC) < 16 ? (32 / HC) : 16;  // softmax lanes per head
     static constexpr int TPL = kSubTile / LPH;                   // tokens per softmax lane
     static constexpr int E = Elem<T>::kBytes;
+    static constexpr bool kPaddedRows = false;
+    static constexpr int kUnitsPerWarp = UPW;
+    static constexpr int kCombFloats = HC * D + 8;
+    static constexpr int kScratchFloats = 2 * kSubTile * HC;
+
+    // value index = h*R + r; bits flipped per lane by the reduce-scatter order
+    static constexpr int kLogR = R == 8 ? 3 : (R == 4 ? 2 : (R == 2 ? 1 : 0));
+    static constexpr int kLogNV = NV >= 32 ? 5 : NV >= 16 ? 4 : NV >= 8 ? 3 : NV >= 4 ? 2 : NV >= 2 ? 1 : 0;
+    static constexpr int kLogRL = RL == 16 ? 4 : 3;
+    static constexpr int kScatter = kLogNV < kLogRL ? kLogNV : kLogRL;
 
     struct Unit {
         float2 q2[HC][4];
@@ -265,23 +298,49 @@ struct Consumer {
         float m_own, l_own;  // running max / sum of head (lane / LPH), base-2 domain
     };
 
-    // One 16-token sub-tile of one unit.  kst/vst point at token 0 of the
-    // sub-tile in the stage; rows are HG*D elements apart.
-    static __device__ __forceinline__ void subtile(Unit &u, const unsigned char *kst, const unsigned char *vst,
-                                                   int g_local, int nvalid, uint32_t row_bytes, float *s_sm,
-                                                   float *p_sm, int lane) {
-        const int sl = lane % RL;
-        const int tg = lane / RL;
+    int sl, tg, perm, head_flip, round_flip;
+
+    __device__ __forceinline__ void setup(int lane) {
+        sl = lane % RL;
+        tg = lane / RL;
+        perm = 0;
+#pragma unroll
+        for (int k = 0; k < kScatter; ++k) {
+            const int lane_bit = (sl >> (kLogRL - 1 - k)) & 1;
+            perm |= lane_bit << (kLogNV - 1 - k);
+        }
+        head_flip = perm >> kLogR;
+        round_flip = perm & (R - 1);
+    }
+
+    __device__ __forceinline__ void init_unit(Unit &u, const unsigned char *qs, int h0, float qscale) const {
+#pragma unroll
+        for (int h = 0; h < HC; ++h) {
+            float2 q2[4];
+            Elem<T>::load8(qs + ((size_t)(h0 + (h ^ head_flip)) * D + sl * 8) * E, q2);
+            const float2 sc = make_float2(qscale, qscale);
+#pragma unroll
+            for (int i = 0; i < 4; ++i) {
+                u.q2[h][i] = fmul2(q2[i], sc);
+                u.o2[h][i] = make_float2(0.f, 0.f);
+            }
+        }
+        u.m_own = -INFINITY;
+        u.l_own = 0.f;
+    }
+
+    __device__ __forceinline__ void subtile(Unit &u, const unsigned char *kst, const unsigned char *vst, int g_local,
+                                            int nvalid, uint32_t pitch, float *s_sm, float *p_sm, int lane) const {
         const uint32_t col = (uint32_t)(g_local * D + sl * 8) * E;
 
-        // ---- QK: partial dots over this lane's 8 elements ----
+        // ---- QK: partial dots over this lane's 8 elements (rounds permuted per lane) ----
         float acc[NV];
 #pragma unroll
         for (int r = 0; r < R; ++r) {
-            const int tok = r * TG + tg;
+            const int tok = (r ^ round_flip) * TG + tg;
             float2 k2[4];
             if (tok < nvalid) {
-                Elem<T>::load8(kst + tok * row_bytes + col, k2);
+                Elem<T>::load8(kst + tok * pitch + col, k2);
             } else {
 #pragma unroll
                 for (int i = 0; i < 4; ++i) k2[i] = make_float2(0.f, 0.f);
@@ -295,8 +354,7 @@ struct Consumer {
                 acc[h * R + r] = a.x + a.y;
             }
         }
-        ReduceScatter<NV, RL / 2>::run(acc, lane);
-        // value j of this lane is (head, round) index i = h*R + r
+        ReduceScatter<NV, RL / 2>::run(acc);
 #pragma unroll
         for (int j = 0; j < NVL; ++j) {
             const int i = (NV >= RL) ? sl * NVL + j : sl / (RL / NV);
@@ -306,7 +364,7 @@ struct Consumer {
         __syncwarp();
 
         // ---- online softmax per head ----
-        const int hs = lane / LPH;  // head served by this lane (HC*LPH <= 32)
+        const int hs = lane / LPH;
         const int li = lane % LPH;
         const bool active = hs < HC;
         float sc[TPL];
@@ -320,11 +378,11 @@ struct Consumer {
 #pragma unroll
         for (int m = 1; m < LPH; m <<= 1) tmax = fmaxf(tmax, __shfl_xor_sync(0xffffffffu, tmax, m));
         const float m_new = fmaxf(u.m_own, tmax);
-        const float alpha = exp2f(u.m_own - m_new);  // m_own = -inf at start -> 0
+        const float alpha = exp2f(u.m_own - m_new);
         float psum = 0.f;
 #pragma unroll
         for (int k = 0; k < TPL; ++k) {
-            const float pk = exp2f(sc[k] - m_new);  // masked: exp2(-inf) = 0
+            const float pk = exp2f(sc[k] - m_new);
             psum += pk;
             if (active) p_sm[(li * TPL + k) * HC + hs] = pk;
         }
@@ -349,7 +407,7 @@ struct Consumer {
             const int tok = r * TG + tg;
             if (tok < nvalid) {
                 float2 v2[4];
-                Elem<T>::load8(vst + tok * row_bytes + col, v2);
+                Elem<T>::load8(vst + tok * pitch + col, v2);
                 float pv[HC];
                 if constexpr (HC == 4) {
                     const float4 t = *reinterpret_cast<const float4 *>(p_sm + tok * HC);
@@ -372,8 +430,12 @@ struct Consumer {
         __syncwarp();
     }
 
+    // running max / sum of head h, broadcast to every lane
+    __device__ __forceinline__ float head_m(const Unit &u, int h) const { return __shfl_sync(0xffffffffu, u.m_own, h * LPH); }
+    __device__ __forceinline__ float head_l(const Unit &u, int h) const { return __shfl_sync(0xffffffffu, u.l_own, h * LPH); }
+
     // sum the output partials of the TG token-groups (lanes with equal slice)
-    static __device__ __forceinline__ void reduce_token_groups(Unit &u) {
+    __device__ __forceinline__ void finish_unit(Unit &u) const {
 #pragma unroll
         for (int m = RL; m < 32; m <<= 1) {
 #pragma unroll
@@ -385,14 +447,525 @@ struct Consumer {
                 }
         }
     }
+
+    // hand the unit's state to another warp of the same unit (token split)
+    __device__ __forceinline__ void save(const Unit &u, float *comb, int lane) const {
+#pragma unroll
+        for (int h = 0; h < HC; ++h) {
+            const float mh = head_m(u, h), lh = head_l(u, h);
+            if (tg == 0) {
+                Elem<float>::store8(comb + h * D + sl * 8, u.o2[h]);
+                if (sl == 0) {
+                    comb[HC * D + h] = mh;
+                    comb[HC * D + HC + h] = lh;
+                }
+            }
+        }
+    }
+
+    __device__ __forceinline__ void absorb(Unit &u, const float *oc, int lane) const {
+#pragma unroll
+        for (int h = 0; h < HC; ++h) {
+            const float m1 = head_m(u, h), l1 = head_l(u, h);
+            const float m2 = oc[HC * D + h], l2 = oc[HC * D + HC + h];
+            const float M = fmaxf(m1, m2);
+            const float a1 = exp2f(m1 - M), a2 = exp2f(m2 - M);
+            float2 o2[4];
+            Elem<float>::load8(oc + h * D + sl * 8, o2);
+#pragma unroll
+            for (int i = 0; i < 4; ++i) {
+                u.o2[h][i].x = u.o2[h][i].x * a1 + o2[i].x * a2;
+                u.o2[h][i].y = u.o2[h][i].y * a1 + o2[i].y * a2;
+            }
+            if (lane / LPH == h) {
+                u.m_own = M;
+                u.l_own = l1 * a1 + l2 * a2;
+            }
+        }
+    }
+
+    // normalised output of the unit's heads (h_out0 = first head's index in out)
+    __device__ __forceinline__ void write_out(const Unit &u, unsigned char *outb, size_t h_out0) const {
+#pragma unroll
+        for (int h = 0; h < HC; ++h) {
+            const float lh = head_l(u, h);
+            if (tg == 0) {
+                const float inv = 1.f / lh;
+                float2 r[4];
+#pragma unroll
+                for (int i = 0; i < 4; ++i) r[i] = make_float2(u.o2[h][i].x * inv, u.o2[h][i].y * inv);
+                Elem<T>::store8(outb + ((h_out0 + h) * D + sl * 8) * E, r);
+            }
+        }
+    }
+
+    __device__ __forceinline__ void write_partial(const Unit &u, float *slot, int NHvr, int hl0) const {
+#pragma unroll
+        for (int h = 0; h < HC; ++h) {
+            const float mh = head_m(u, h), lh = head_l(u, h);
+            if (tg == 0) {
+                Elem<float>::store8(slot + (size_t)(hl0 + h) * D + sl * 8, u.o2[h]);
+                if (sl == 0) {
+                    slot[NHvr * D + hl0 + h] = mh;
+                    slot[NHvr * D + NHvr + hl0 + h] = lh;
+                }
+            }
+        }
+    }
 };
 
-// ---------------------------------------------------------------------------
-template <typename T, int D, int HC, int UPW>
-__global__ void __launch_bounds__(kDecodeThreads, 1) paged_decode_kernel(const DecodeParams p) {
-    using C = Consumer<T, D, HC, UPW>;
+// ===========================================================================
+// tensor-core engine (bf16): tokens are the M dimension of every tile
+// ===========================================================================
+template <int D, int UPW>
+struct MmaEngine {
+    static constexpr int KS = D / 16;  // k-steps of QK (over d) = m-tiles of PV (over d)
+    static constexpr int E = 2;
+    static constexpr bool kPaddedRows = true;
+    static constexpr int kUnitsPerWarp = UPW;
+    static constexpr int kCombFloats = 4 * KS * 32 + 4 * 32;  // fragment-ordered o, then m, l
+    static constexpr int kScratchFloats = 0;
+
+    struct Unit {
+        uint32_t qb[KS][2];  // B fragments of Q: head g4, d pairs
+        float o[KS][4];      // O^T: rows d = mt*16 + g4 (+8), cols heads 2*t4, 2*t4+1
+        float m[2], l[2];    // heads 2*t4, 2*t4+1 of the unit, base-2 domain
+    };
+
+    int g4, t4;
+    int a_tok, a_col;  // this lane's ldmatrix row for QK (K tile)
+    int v_tok, v_col;  // and for PV (V tile, transposed load)
+    float qscale;
+    int nreal;         // real heads in a unit (<= 8)
+
+    __device__ __forceinline__ void setup(int lane) {
+        g4 = lane >> 2;
+        t4 = lane & 3;
+        a_tok = (lane & 7) + ((lane >> 3) & 1) * 8;
+        a_col = (lane >> 4) * 8;
+        v_tok = (lane & 7) + ((lane >> 4) & 1) * 8;
+        v_col = ((lane >> 3) & 1) * 8;
+    }
+
+    __device__ __forceinline__ void init_unit(Unit &u, const unsigned char *qs, int h0, float qs_) {
+        qscale = qs_;
+        // head g4 of the unit (rows past the real heads are zero)
+        const bool real = g4 < nreal;
+        const uint32_t *qrow = reinterpret_cast<const uint32_t *>(qs + (size_t)(h0 + g4) * D * E);
+#pragma unroll
+        for (int ks = 0; ks < KS; ++ks) {
+            u.qb[ks][0] = real ? qrow[ks * 8 + t4] : 0u;
+            u.qb[ks][1] = real ? qrow[ks * 8 + 4 + t4] : 0u;
+        }
+#pragma unroll
+        for (int mt = 0; mt < KS; ++mt)
+#pragma unroll
+            for (int i = 0; i < 4; ++i) u.o[mt][i] = 0.f;
+        u.m[0] = u.m[1] = -INFINITY;
+        u.l[0] = u.l[1] = 0.f;
+    }
+
+    __device__ __forceinline__ void subtile(Unit &u, const unsigned char *kst, unsigned char *vst, int g_local,
+                                            int nvalid, uint32_t pitch, float *, float *, int lane) const {
+        const uint32_t colb = (uint32_t)g_local * D * E;
+        // ---- S^T[16 tok x 8 heads] = K Q^T ----
+        float s[4] = {0.f, 0.f, 0.f, 0.f};
+        const unsigned char *ka = kst + a_tok * pitch + colb + a_col * E;
+#pragma unroll
+        for (int ks = 0; ks < KS; ++ks) {
+            uint32_t a[4];
+            ldmatrix_x4(a, ka + ks * 16 * E);
+            mma_bf16_16816(s, a, u.qb[ks][0], u.qb[ks][1]);
+        }
+        // ---- online softmax over the 16 tokens, per head column ----
+        const bool v0 = g4 < nvalid, v1 = g4 + 8 < nvalid;
+        const float s0 = v0 ? s[0] * qscale : -INFINITY;
+        const float s1 = v0 ? s[1] * qscale : -INFINITY;
+        const float s2 = v1 ? s[2] * qscale : -INFINITY;
+        const float s3 = v1 ? s[3] * qscale : -INFINITY;
+        float mx0 = fmaxf(s0, s2), mx1 = fmaxf(s1, s3);
+#pragma unroll
+        for (int m = 4; m < 32; m <<= 1) {
+            mx0 = fmaxf(mx0, __shfl_xor_sync(0xffffffffu, mx0, m));
+            mx1 = fmaxf(mx1, __shfl_xor_sync(0xffffffffu, mx1, m));
+        }
+        const float mn0 = fmaxf(u.m[0], mx0), mn1 = fmaxf(u.m[1], mx1);
+        const float al0 = exp2f(u.m[0] - mn0), al1 = exp2f(u.m[1] - mn1);
+        const uint32_t pb0 = pack_bf16x2(exp2f(s0 - mn0), exp2f(s1 - mn1));  // token g4
+        const uint32_t pb1 = pack_bf16x2(exp2f(s2 - mn0), exp2f(s3 - mn1));  // token g4 + 8
+        // the denominator sums the same (rounded) weights the PV product uses
+        const float2 f0 = bf16x2_to_float2(pb0), f1 = bf16x2_to_float2(pb1);
+        float r0 = f0.x + f1.x, r1 = f0.y + f1.y;
+#pragma unroll
+        for (int m = 4; m < 32; m <<= 1) {
+            r0 += __shfl_xor_sync(0xffffffffu, r0, m);
+            r1 += __shfl_xor_sync(0xffffffffu, r1, m);
+        }
+        u.l[0] = u.l[0] * al0 + r0;
+        u.l[1] = u.l[1] * al1 + r1;
+        u.m[0] = mn0;
+        u.m[1] = mn1;
+        // P^T fragments (k = token, n = head)
+        const uint32_t b0 = movmatrix_trans(pb0);
+        const uint32_t b1 = movmatrix_trans(pb1);
+        if (al0 != 1.f || al1 != 1.f) {
+#pragma unroll
+            for (int mt = 0; mt < KS; ++mt) {
+                u.o[mt][0] *= al0;
+                u.o[mt][1] *= al1;
+                u.o[mt][2] *= al0;
+                u.o[mt][3] *= al1;
+            }
+        }
+        // rows past nvalid may hold stale data: zero this unit's columns there
+        if (nvalid < kSubTile) {
+            for (int r = nvalid; r < kSubTile; ++r)
+                for (int c = lane; c < D * E / 16; c += 32)
+                    *reinterpret_cast<uint4 *>(vst + r * pitch + colb + c * 16) = make_uint4(0, 0, 0, 0);
+            __syncwarp();
+        }
+        // ---- O^T[d x heads] += V^T P^T ----
+        const unsigned char *va = vst + v_tok * pitch + colb + v_col * E;
+#pragma unroll
+        for (int mt = 0; mt < KS; ++mt) {
+            uint32_t a[4];
+            ldmatrix_x4_trans(a, va + mt * 16 * E);
+            mma_bf16_16816(u.o[mt], a, b0, b1);
+        }
+    }
+
+    __device__ __forceinline__ void finish_unit(Unit &) const {}
+
+    __device__ __forceinline__ void save(const Unit &u, float *comb, int lane) const {
+#pragma unroll
+        for (int mt = 0; mt < KS; ++mt)
+#pragma unroll
+            for (int i = 0; i < 4; ++i) comb[(mt * 4 + i) * 32 + lane] = u.o[mt][i];
+        comb[(4 * KS + 0) * 32 + lane] = u.m[0];
+        comb[(4 * KS + 1) * 32 + lane] = u.m[1];
+        comb[(4 * KS + 2) * 32 + lane] = u.l[0];
+        comb[(4 * KS + 3) * 32 + lane] = u.l[1];
+    }
+
+    __device__ __forceinline__ void absorb(Unit &u, const float *oc, int lane) const {
+        float a1[2], a2[2];
+#pragma unroll
+        for (int j = 0; j < 2; ++j) {
+            const float m2 = oc[(4 * KS + j) * 32 + lane], l2 = oc[(4 * KS + 2 + j) * 32 + lane];
+            const float M = fmaxf(u.m[j], m2);
+            a1[j] = exp2f(u.m[j] - M);
+            a2[j] = exp2f(m2 - M);
+            u.l[j] = u.l[j] * a1[j] + l2 * a2[j];
+            u.m[j] = M;
+        }
+#pragma unroll
+        for (int mt = 0; mt < KS; ++mt)
+#pragma unroll
+            for (int i = 0; i < 4; ++i)
+                u.o[mt][i] = u.o[mt][i] * a1[i & 1] + oc[(mt * 4 + i) * 32 + lane] * a2[i & 1];
+    }
+
+    __device__ __forceinline__ void write_out(const Unit &u, unsigned char *outb, size_t h_out0) const {
+#pragma unroll
+        for (int j = 0; j < 2; ++j) {
+            const int h = 2 * t4 + j;
+            if (h >= nreal) continue;
+            const float inv = 1.f / u.l[j];
+            unsigned char *row = outb + (h_out0 + h) * D * E;
+#pragma unroll
+            for (int mt = 0; mt < KS; ++mt) {
+                Elem<__nv_bfloat16>::store1(row + (mt * 16 + g4) * E, u.o[mt][j] * inv);
+                Elem<__nv_bfloat16>::store1(row + (mt * 16 + g4 + 8) * E, u.o[mt][2 + j] * inv);
+            }
+        }
+    }
+
+    __device__ __forceinline__ void write_partial(const Unit &u, float *slot, int NHvr, int hl0) const {
+#pragma unroll
+        for (int j = 0; j < 2; ++j) {
+            const int h = 2 * t4 + j;
+            if (h >= nreal) continue;
+            float *row = slot + (size_t)(hl0 + h) * D;
+#pragma unroll
+            for (int mt = 0; mt < KS; ++mt) {
+                row[mt * 16 + g4] = u.o[mt][j];
+                row[mt * 16 + g4 + 8] = u.o[mt][2 + j];
+            }
+            if (g4 == 0) {
+                slot[NHvr * D + hl0 + h] = u.m[j];
+                slot[NHvr * D + NHvr + hl0 + h] = u.l[j];
+            }
+        }
+    }
+};
+
+// ===========================================================================
+// producer warp
+// ===========================================================================
+template <int D, int E>
+__device__ __forceinline__ void run_producer(const DecodeParams &p, SegIter it, uint64_t *full, uint64_t *empty,
+                                             uint64_t *qfull, uint64_t *qempty, unsigned char *qarea,
+                                             unsigned char *stage_base, volatile int *abort_flag, int lane) {
+    const uint64_t policy = policy_evict_first();
+    const unsigned char *kc = reinterpret_cast<const unsigned char *>(p.k_cache);
+    const unsigned char *vc = reinterpret_cast<const unsigned char *>(p.v_cache);
+    const unsigned char *qg = reinterpret_cast<const unsigned char *>(p.q);
+    const uint32_t row_bytes = p.row_bytes, pitch = p.row_pitch;
+    const size_t tok_stride = (size_t)p.Hkv * D * E;  // bytes between token rows in the pool
+    const bool contiguous = (p.HG == p.Hkv) && (pitch == row_bytes);
+    const int S = p.stages;
+    int stage = 0;
+    uint32_t phase = 0;
+    int qslot = 0;
+    uint32_t qphase = 0;
+    uint32_t issued = 0, issued_par = 0;  // per stage: filled at least once / parity of the last fill
+    bool dep_done = (p.pdl == 0);
+    bool ok = true;
+    Seg s;
+    while (ok && it.next(p, s)) {
+        if (!mbar_wait(&qempty[qslot], qphase ^ 1u, abort_flag)) {
+            ok = false;
+            break;
+        }
+        if (lane == 0) {
+            mbar_arrive_expect_tx(&qfull[qslot], p.q_bytes);
+            bulk_g2s(qarea + qslot * p.q_bytes, qg + ((size_t)s.b * p.Hq + (size_t)s.hg * p.NHvr) * D * E, p.q_bytes,
+                     &qfull[qslot]);
+        }
+        qslot ^= 1;
+        if (qslot == 0) qphase ^= 1u;
+
+        const int32_t *table = p.block_tables + (size_t)s.b * p.max_blocks;
+        const int nblk = (s.L + p.bs - 1) / p.bs;
+        int cur_base = -1, cur_val = -1, nxt_base = -1, nxt_val = -1;
+        for (int t = s.t_begin; t < s.t_end; ++t) {
+            if (!mbar_wait(&empty[stage], phase ^ 1u, abort_flag)) {
+                ok = false;
+                break;
+            }
+            const int tok0 = t * p.ST;
+            const int ntok = min(p.ST, s.L - tok0);
+            const int jb0 = tok0 / p.bs;
+            const int wb = jb0 & ~31;
+            if (wb != cur_base) {
+                if (wb == nxt_base) {
+                    cur_val = nxt_val;
+                } else {
+                    cur_val = (wb + lane < nblk) ? table[wb + lane] : -1;
+                }
+                cur_base = wb;
+                nxt_base = wb + 32;
+                nxt_val = (nxt_base + lane < nblk) ? table[nxt_base + lane] : -1;  // prefetch
+            }
+            if (!dep_done) {
+                grid_dependency_wait();  // K/V may have just been appended by the preceding grid
+                dep_done = true;
+            }
+            unsigned char *kdst = stage_base + (size_t)stage * 2 * p.half_bytes;
+            unsigned char *vdst = kdst + p.half_bytes;
+            uint32_t bytes = 0;
+            if (contiguous) {
+                // one copy per block piece: rows of all KV heads are contiguous in both places
+                const int np = (tok0 + ntok - 1) / p.bs - jb0 + 1;
+                const int j = jb0 + lane;
+                const int phys = __shfl_sync(0xffffffffu, cur_val, (j - cur_base) & 31);
+                int tlo = 0, nrows = 0;
+                bool valid = false;
+                if (lane < np) {
+                    tlo = max(tok0, j * p.bs);
+                    nrows = min(tok0 + ntok, (j + 1) * p.bs) - tlo;
+                    valid = phys >= 0 && phys < p.num_blocks;
+                    if (!valid) set_error(p.error, PA_DEVERR_BLOCK_ID);
+                    else bytes = 2u * (uint32_t)nrows * row_bytes;
+                }
+#pragma unroll
+                for (int m = 16; m >= 1; m >>= 1) bytes += __shfl_xor_sync(0xffffffffu, bytes, m);
+                if (lane == 0) mbar_arrive_expect_tx(&full[stage], bytes);
+                __syncwarp();
+                if (valid) {
+                    const size_t src = ((size_t)phys * p.bs + (tlo - j * p.bs)) * tok_stride;
+                    const uint32_t n = (uint32_t)nrows * row_bytes;
+                    bulk_g2s_hint(kdst + (tlo - tok0) * pitch, kc + src, n, &full[stage], policy);
+                    bulk_g2s_hint(vdst + (tlo - tok0) * pitch, vc + src, n, &full[stage], policy);
+                }
+            } else {
+                // one copy per token row (padded rows, or a head group narrower than the pool row)
+                for (int i0 = 0; i0 < ntok; i0 += 32) {
+                    const int i = i0 + lane;
+                    const int tt = tok0 + i;
+                    const int j = tt / p.bs;
+                    const int phys = __shfl_sync(0xffffffffu, cur_val, (j - cur_base) & 31);
+                    if (i < ntok) {
+                        if (phys < 0 || phys >= p.num_blocks) set_error(p.error, PA_DEVERR_BLOCK_ID);
+                        else bytes += 2u * row_bytes;
+                    }
+                }
+#pragma unroll
+                for (int m = 16; m >= 1; m >>= 1) bytes += __shfl_xor_sync(0xffffffffu, bytes, m);
+                if (lane == 0) mbar_arrive_expect_tx(&full[stage], bytes);
+                __syncwarp();
+                for (int i0 = 0; i0 < ntok; i0 += 32) {
+                    const int i = i0 + lane;
+                    const int tt = tok0 + i;
+                    const int j = tt / p.bs;
+                    const int phys = __shfl_sync(0xffffffffu, cur_val, (j - cur_base) & 31);
+                    if (i < ntok && phys >= 0 && phys < p.num_blocks) {
+                        const size_t src = ((size_t)phys * p.bs + (tt - j * p.bs)) * tok_stride + (size_t)s.hg * row_bytes;
+                        bulk_g2s_hint(kdst + i * pitch, kc + src, row_bytes, &full[stage], policy);
+                        bulk_g2s_hint(vdst + i * pitch, vc + src, row_bytes, &full[stage], policy);
+                    }
+                }
+            }
+            issued |= 1u << stage;
+            issued_par = (issued_par & ~(1u << stage)) | (phase << stage);
+            if (++stage == S) {
+                stage = 0;
+                phase ^= 1u;
+            }
+        }
+    }
+    if (!ok) {
+        *abort_flag = 1;
+        if (lane == 0) set_error(p.error, PA_DEVERR_TIMEOUT);
+    }
+    // every copy this warp issued lands before the CTA can retire
+    volatile int never = 0;
+    for (int st = 0; st < S; ++st)
+        if (issued & (1u << st)) mbar_wait(&full[st], (issued_par >> st) & 1u, &never);
+}
+
+// ===========================================================================
+// merge of a split vr by log-sum-exp (run by the consumer warps of the CTA
+// that delivered the last piece)
+// ===========================================================================
+template <typename T, int D>
+__device__ __forceinline__ void merge_vr(const DecodeParams &p, const Seg &s, int64_t NT, int64_t C, float *msm,
+                                         int tid) {
     constexpr int E = Elem<T>::kBytes;
-    constexpr int kCombStride = HC * D + 8;  // floats per warp in the token-split combine area
+    constexpr int NTH = kConsumerWarps * 32;
+    const int NH = p.NHvr;
+    const int nparts = s.nparts;
+    const int warp = tid >> 5, lane = tid & 31;
+    const size_t out_head0 = (size_t)s.b * p.Hq + (size_t)s.hg * NH;
+    if (nparts <= kMergeParts) {
+        // weights w[i][h] = exp2(m_i - M_h) and 1 / sum_i w l into shared memory
+        float *w = msm;                    // [nparts][NH]
+        float *inv_den = msm + kMergeParts * NH;
+        for (int h = warp; h < NH; h += kConsumerWarps) {
+            float mi[2], li[2];
+            float M = -INFINITY;
+#pragma unroll
+            for (int k = 0; k < 2; ++k) {
+                const int i = lane + 32 * k;
+                mi[k] = -INFINITY;
+                li[k] = 0.f;
+                if (i < nparts) {
+                    const int64_t slot = piece_slot(p, s, i, NT, C);
+                    if (slot < p.max_slots) {
+                        const float *base = p.partials + slot * p.slot_floats;
+                        mi[k] = __ldcg(base + NH * D + h);
+                        li[k] = __ldcg(base + NH * D + NH + h);
+                    }
+                }
+                M = fmaxf(M, mi[k]);
+            }
+#pragma unroll
+            for (int m = 16; m >= 1; m >>= 1) M = fmaxf(M, __shfl_xor_sync(0xffffffffu, M, m));
+            float den = 0.f;
+#pragma unroll
+            for (int k = 0; k < 2; ++k) {
+                const int i = lane + 32 * k;
+                const float wi = (mi[k] == -INFINITY) ? 0.f : exp2f(mi[k] - M);
+                den += wi * li[k];
+                if (i < nparts) w[i * NH + h] = wi;
+            }
+#pragma unroll
+            for (int m = 16; m >= 1; m >>= 1) den += __shfl_xor_sync(0xffffffffu, den, m);
+            if (lane == 0) inv_den[h] = 1.f / den;
+        }
+        named_barrier(1, NTH);
+        const int nq = NH * (D / 4);
+        for (int idx = tid; idx < nq; idx += NTH) {
+            const int h = idx / (D / 4);
+            const int d4 = idx % (D / 4);
+            float4 num = make_float4(0.f, 0.f, 0.f, 0.f);
+            int i = 0;
+            for (; i + 4 <= nparts; i += 4) {
+                float4 o[4];
+                float wi[4];
+#pragma unroll
+                for (int k = 0; k < 4; ++k) {
+                    const int64_t slot = piece_slot(p, s, i + k, NT, C);
+                    const bool okk = slot < p.max_slots;
+                    o[k] = okk ? __ldcg(reinterpret_cast<const float4 *>(p.partials + slot * p.slot_floats +
+                                                                           (size_t)h * D) + d4)
+                               : make_float4(0.f, 0.f, 0.f, 0.f);
+                    wi[k] = w[(i + k) * NH + h];
+                }
+#pragma unroll
+                for (int k = 0; k < 4; ++k) {
+                    num.x += wi[k] * o[k].x;
+                    num.y += wi[k] * o[k].y;
+                    num.z += wi[k] * o[k].z;
+                    num.w += wi[k] * o[k].w;
+                }
+            }
+            for (; i < nparts; ++i) {
+                const int64_t slot = piece_slot(p, s, i, NT, C);
+                if (slot >= p.max_slots) continue;
+                const float4 o =
+                    __ldcg(reinterpret_cast<const float4 *>(p.partials + slot * p.slot_floats + (size_t)h * D) + d4);
+                const float wi = w[i * NH + h];
+                num.x += wi * o.x;
+                num.y += wi * o.y;
+                num.z += wi * o.z;
+                num.w += wi * o.w;
+            }
+            const float inv = inv_den[h];
+            unsigned char *dst =
+                reinterpret_cast<unsigned char *>(p.out) + ((out_head0 + h) * D + d4 * 4) * E;
+            Elem<T>::store2(dst, num.x * inv, num.y * inv);
+            Elem<T>::store2(dst + 2 * E, num.z * inv, num.w * inv);
+        }
+        named_barrier(1, NTH);  // the weights area is free again
+        return;
+    }
+    // many pieces (fixed partitions of a very long context): direct two-pass form
+    const int nq = NH * (D / 4);
+    for (int idx = tid; idx < nq; idx += NTH) {
+        const int h = idx / (D / 4);
+        const int d4 = idx % (D / 4);
+        float M = -INFINITY;
+        for (int i = 0; i < nparts; ++i) {
+            const int64_t slot = piece_slot(p, s, i, NT, C);
+            if (slot < p.max_slots) M = fmaxf(M, __ldcg(p.partials + slot * p.slot_floats + NH * D + h));
+        }
+        float4 num = make_float4(0.f, 0.f, 0.f, 0.f);
+        float den = 0.f;
+        for (int i = 0; i < nparts; ++i) {
+            const int64_t slot = piece_slot(p, s, i, NT, C);
+            if (slot >= p.max_slots) continue;
+            const float *base = p.partials + slot * p.slot_floats;
+            const float wi = exp2f(__ldcg(base + NH * D + h) - M);
+            den += wi * __ldcg(base + NH * D + NH + h);
+            const float4 o = __ldcg(reinterpret_cast<const float4 *>(base + (size_t)h * D) + d4);
+            num.x += wi * o.x;
+            num.y += wi * o.y;
+            num.z += wi * o.z;
+            num.w += wi * o.w;
+        }
+        const float inv = 1.f / den;
+        unsigned char *dst = reinterpret_cast<unsigned char *>(p.out) + ((out_head0 + h) * D + d4 * 4) * E;
+        Elem<T>::store2(dst, num.x * inv, num.y * inv);
+        Elem<T>::store2(dst + 2 * E, num.z * inv, num.w * inv);
+    }
+}
+
+// ===========================================================================
+template <typename T, int D, class Engine>
+__global__ void __launch_bounds__(kDecodeThreads, 1) paged_decode_kernel(const DecodeParams p) {
+    constexpr int E = Elem<T>::kBytes;
+    constexpr int UPW = Engine::kUnitsPerWarp;
     extern __shared__ __align__(128) unsigned char smem[];
     __shared__ DecodeCtl ctl;
 
@@ -497,108 +1070,7 @@ __global__ void __launch_bounds__(kDecodeThreads, 1) paged_decode_kernel(const D
     }
 
     if (warp == kConsumerWarps) {
-        // ================= producer warp =================
-        const uint64_t policy = policy_evict_first();
-        const unsigned char *kc = reinterpret_cast<const unsigned char *>(p.k_cache);
-        const unsigned char *vc = reinterpret_cast<const unsigned char *>(p.v_cache);
-        const unsigned char *qg = reinterpret_cast<const unsigned char *>(p.q);
-        const uint32_t row_bytes = p.row_bytes;
-        const size_t tok_stride = (size_t)p.Hkv * D * E;  // bytes between token rows in the pool
-        Seg s;
-        int64_t fill = 0;
-        int segk = 0;
-        bool ok = true;
-        while (ok && it.next(p, s)) {
-            const int qb = segk & 1;
-            if (!mbar_wait(&qempty[qb], ((segk >> 1) & 1) ^ 1, abort_flag)) {
-                ok = false;
-                break;
-            }
-            if (lane == 0) {
-                mbar_arrive_expect_tx(&qfull[qb], p.q_bytes);
-                bulk_g2s(qarea + qb * p.q_bytes, qg + ((size_t)s.b * p.Hq + (size_t)s.hg * p.NHvr) * D * E,
-                         p.q_bytes, &qfull[qb]);
-            }
-            const int32_t *table = p.block_tables + (size_t)s.b * p.max_blocks;
-            for (int t = s.t_begin; t < s.t_end; ++t) {
-                const int stage = (int)(fill % S);
-                if (!mbar_wait(&empty[stage], (uint32_t)((fill / S) & 1) ^ 1u, abort_flag)) {
-                    ok = false;
-                    break;
-                }
-                unsigned char *kdst = stage_base + (size_t)stage * 2 * p.half_bytes;
-                unsigned char *vdst = kdst + p.half_bytes;
-                const int tok0 = t * p.ST;
-                const int ntok = min(p.ST, s.L - tok0);
-                if (p.HG == p.Hkv) {
-                    // one copy per block piece: rows of all KV heads are contiguous
-                    const int jb0 = tok0 / p.bs;
-                    const int np = (tok0 + ntok - 1) / p.bs - jb0 + 1;
-                    uint32_t bytes = 0;
-                    int phys = -1, r0 = 0, nrows = 0, dtok = 0;
-                    if (lane < np) {
-                        const int j = jb0 + lane;
-                        const int tlo = max(tok0, j * p.bs);
-                        const int thi = min(tok0 + ntok, (j + 1) * p.bs);
-                        phys = table[j];
-                        r0 = tlo - j * p.bs;
-                        nrows = thi - tlo;
-                        dtok = tlo - tok0;
-                        if (phys < 0 || phys >= p.num_blocks) {
-                            set_error(p.error, PA_DEVERR_BLOCK_ID);
-                            phys = -1;
-                        } else {
-                            bytes = 2u * (uint32_t)nrows * row_bytes;
-                        }
-                    }
-#pragma unroll
-                    for (int m = 16; m >= 1; m >>= 1) bytes += __shfl_xor_sync(0xffffffffu, bytes, m);
-                    if (lane == 0) mbar_arrive_expect_tx(&full[stage], bytes);
-                    __syncwarp();
-                    if (phys >= 0) {
-                        const size_t src = ((size_t)phys * p.bs + r0) * tok_stride;
-                        const uint32_t n = (uint32_t)nrows * row_bytes;
-                        bulk_g2s_hint(kdst + dtok * row_bytes, kc + src, n, &full[stage], policy);
-                        bulk_g2s_hint(vdst + dtok * row_bytes, vc + src, n, &full[stage], policy);
-                    }
-                } else {
-                    // head group narrower than the pool row: one copy per token
-                    uint32_t bytes = 0;
-                    for (int i = lane; i < ntok; i += 32) {
-                        const int tt = tok0 + i;
-                        const int ph = table[tt / p.bs];
-                        if (ph < 0 || ph >= p.num_blocks)
-                            set_error(p.error, PA_DEVERR_BLOCK_ID);
-                        else
-                            bytes += 2u * row_bytes;
-                    }
-#pragma unroll
-                    for (int m = 16; m >= 1; m >>= 1) bytes += __shfl_xor_sync(0xffffffffu, bytes, m);
-                    if (lane == 0) mbar_arrive_expect_tx(&full[stage], bytes);
-                    __syncwarp();
-                    for (int i = lane; i < ntok; i += 32) {
-                        const int tt = tok0 + i;
-                        const int ph = table[tt / p.bs];
-                        if (ph < 0 || ph >= p.num_blocks) continue;
-                        const size_t src =
-                            ((size_t)ph * p.bs + (tt % p.bs)) * tok_stride + (size_t)s.hg * row_bytes;
-                        bulk_g2s_hint(kdst + i * row_bytes, kc + src, row_bytes, &full[stage], policy);
-                        bulk_g2s_hint(vdst + i * row_bytes, vc + src, row_bytes, &full[stage], policy);
-                    }
-                }
-                ++fill;
-            }
-            ++segk;
-        }
-        if (!ok) {
-            *abort_flag = 1;
-            if (lane == 0) set_error(p.error, PA_DEVERR_TIMEOUT);
-        }
-        // Let every copy this warp issued land before the CTA can retire.
-        volatile int never = 0;
-        for (int64_t k = fill - S > 0 ? fill - S : 0; k < fill; ++k)
-            mbar_wait(&full[k % S], (uint32_t)((k / S) & 1), &never);
-        for (int k = segk - 2 > 0 ? segk - 2 : 0; k < segk; ++k) mbar_wait(&qfull[k & 1], (k >> 1) & 1, &never);
+        run_producer<D, E>(p, it, full, empty, qfull, qempty, qarea, stage_base, abort_flag, lane);
         return;
     }
 
@@ -613,147 +1085,94 @@ __global__ void __launch_bounds__(kDecodeThreads, 1) paged_decode_kernel(const D
     const int U = p.units;
     const int tsplit = p.tsplit;
     const int split = (tsplit > 1) ? warp / U : 0;
-    const int units_per_g = p.G / HC;
-    float *s_sm = reinterpret_cast<float *>(smem + p.off_scratch) + warp * (2 * kSubTile * HC);
-    float *p_sm = s_sm + kSubTile * HC;
+    const int HC = p.heads_per_unit;
+    const int units_per_g = p.G / HC < 1 ? 1 : p.G / HC;
+    float *s_sm = reinterpret_cast<float *>(smem + p.off_scratch) + warp * Engine::kScratchFloats;
+    float *p_sm = s_sm + kSubTile * (Engine::kScratchFloats / (2 * kSubTile));
+    float *msm = reinterpret_cast<float *>(smem + p.off_merge);
 
-    typename C::Unit unit[UPW];
+    Engine eng;
+    eng.setup(lane);
+    if constexpr (Engine::kPaddedRows) eng.nreal = p.G < 8 ? p.G : 8;
+    typename Engine::Unit unit[UPW];
     int u_g[UPW], u_h0[UPW];
 #pragma unroll
     for (int k = 0; k < UPW; ++k) {
         const int uid = (tsplit > 1) ? warp % U : warp + k * kConsumerWarps;
-        u_g[k] = uid / units_per_g;                            // KV head within the group
-        u_h0[k] = u_g[k] * p.G + (uid % units_per_g) * HC;     // first query head within the vr
+        u_g[k] = uid / units_per_g;                          // KV head within the group
+        u_h0[k] = u_g[k] * p.G + (uid % units_per_g) * HC;   // first query head within the vr
     }
-    const int sl = lane % C::RL;
-    const int tg = lane / C::RL;
 
+    int stage = 0;
+    uint32_t phase = 0;
+    int qslot = 0;
+    uint32_t qphase = 0;
     Seg s;
-    int64_t fill = 0;
-    int segk = 0;
     while (it.next(p, s)) {
         // -- q of this vr --
-        const int qb = segk & 1;
-        if (!*abort_flag && !mbar_wait(&qfull[qb], (segk >> 1) & 1, abort_flag)) {
+        if (!*abort_flag && !mbar_wait(&qfull[qslot], qphase, abort_flag)) {
             *abort_flag = 1;
             set_error(p.error, PA_DEVERR_TIMEOUT);
         }
-        const unsigned char *qs = qarea + qb * p.q_bytes;
+        const unsigned char *qs = qarea + qslot * p.q_bytes;
 #pragma unroll
-        for (int k = 0; k < UPW; ++k) {
-#pragma unroll
-            for (int h = 0; h < HC; ++h) {
-                float2 q2[4];
-                Elem<T>::load8(qs + ((size_t)(u_h0[k] + h) * D + sl * 8) * E, q2);
-                const float2 sc = make_float2(p.qscale, p.qscale);
-#pragma unroll
-                for (int i = 0; i < 4; ++i) {
-                    unit[k].q2[h][i] = fmul2(q2[i], sc);
-                    unit[k].o2[h][i] = make_float2(0.f, 0.f);
-                }
-            }
-            unit[k].m_own = -INFINITY;
-            unit[k].l_own = 0.f;
-        }
+        for (int k = 0; k < UPW; ++k) eng.init_unit(unit[k], qs, u_h0[k], p.qscale);
         __syncwarp();
-        if (lane == 0) mbar_arrive(&qempty[qb]);
+        if (lane == 0) mbar_arrive(&qempty[qslot]);
+        qslot ^= 1;
+        if (qslot == 0) qphase ^= 1u;
 
         // -- tiles --
         for (int t = s.t_begin; t < s.t_end; ++t) {
-            const int stage = (int)(fill % S);
-            if (!*abort_flag && !mbar_wait(&full[stage], (uint32_t)((fill / S) & 1), abort_flag)) {
+            if (!*abort_flag && !mbar_wait(&full[stage], phase, abort_flag)) {
                 *abort_flag = 1;
                 set_error(p.error, PA_DEVERR_TIMEOUT);
             }
             if (!*abort_flag) {
-                const unsigned char *kst = stage_base + (size_t)stage * 2 * p.half_bytes;
-                const unsigned char *vst = kst + p.half_bytes;
+                unsigned char *kst = stage_base + (size_t)stage * 2 * p.half_bytes;
+                unsigned char *vst = kst + p.half_bytes;
                 const int ntok = min(p.ST, s.L - t * p.ST);
                 for (int st = split; st * kSubTile < ntok; st += tsplit) {
                     const int nvalid = min(kSubTile, ntok - st * kSubTile);
 #pragma unroll
                     for (int k = 0; k < UPW; ++k)
-                        C::subtile(unit[k], kst + (size_t)st * kSubTile * p.row_bytes,
-                                   vst + (size_t)st * kSubTile * p.row_bytes, u_g[k], nvalid, p.row_bytes, s_sm,
-                                   p_sm, lane);
+                        eng.subtile(unit[k], kst + (size_t)st * kSubTile * p.row_pitch,
+                                    vst + (size_t)st * kSubTile * p.row_pitch, u_g[k], nvalid, p.row_pitch, s_sm,
+                                    p_sm, lane);
                 }
             }
             __syncwarp();
             if (lane == 0) mbar_arrive(&empty[stage]);
-            ++fill;
+            if (++stage == S) {
+                stage = 0;
+                phase ^= 1u;
+            }
         }
-        ++segk;
 
         // -- finish the piece --
 #pragma unroll
-        for (int k = 0; k < UPW; ++k) C::reduce_token_groups(unit[k]);
+        for (int k = 0; k < UPW; ++k) eng.finish_unit(unit[k]);
 
         if (tsplit > 1) {
             // warps of split > 0 hand their state to the split-0 warp of the same unit
-            float *comb = reinterpret_cast<float *>(smem + p.off_comb) + warp * kCombStride;
-            if (split > 0) {
-#pragma unroll
-                for (int h = 0; h < HC; ++h) {
-                    const float mh = __shfl_sync(0xffffffffu, unit[0].m_own, h * C::LPH);
-                    const float lh = __shfl_sync(0xffffffffu, unit[0].l_own, h * C::LPH);
-                    if (tg == 0) {
-                        Elem<float>::store8(comb + h * D + sl * 8, unit[0].o2[h]);
-                        if (sl == 0) {
-                            comb[HC * D + h] = mh;
-                            comb[HC * D + HC + h] = lh;
-                        }
-                    }
-                }
-            }
+            float *comb = reinterpret_cast<float *>(smem + p.off_comb + warp * p.comb_stride);
+            if (split > 0) eng.save(unit[0], comb, lane);
             named_barrier(1, kConsumerWarps * 32);
-            if (split == 0) {
-                for (int s2 = 1; s2 < tsplit; ++s2) {
-                    const float *oc = reinterpret_cast<const float *>(smem + p.off_comb) + (warp + s2 * U) * kCombStride;
-#pragma unroll
-                    for (int h = 0; h < HC; ++h) {
-                        const float m1 = __shfl_sync(0xffffffffu, unit[0].m_own, h * C::LPH);
-                        const float l1 = __shfl_sync(0xffffffffu, unit[0].l_own, h * C::LPH);
-                        const float m2 = oc[HC * D + h];
-                        const float l2 = oc[HC * D + HC + h];
-                        const float M = fmaxf(m1, m2);
-                        const float a1 = exp2f(m1 - M), a2 = exp2f(m2 - M);
-                        float2 o2[4];
-                        Elem<float>::load8(oc + h * D + sl * 8, o2);
-#pragma unroll
-                        for (int i = 0; i < 4; ++i) {
-                            unit[0].o2[h][i].x = unit[0].o2[h][i].x * a1 + o2[i].x * a2;
-                            unit[0].o2[h][i].y = unit[0].o2[h][i].y * a1 + o2[i].y * a2;
-                        }
-                        if (lane / C::LPH == h) {
-                            unit[0].m_own = M;
-                            unit[0].l_own = l1 * a1 + l2 * a2;
-                        }
-                    }
-                }
-            }
+            if (split == 0)
+                for (int s2 = 1; s2 < tsplit; ++s2)
+                    eng.absorb(unit[0],
+                               reinterpret_cast<const float *>(smem + p.off_comb + (warp + s2 * U) * p.comb_stride),
+                               lane);
             named_barrier(1, kConsumerWarps * 32);
         }
 
         const bool writer = (split == 0);
         if (s.nparts == 1) {
             if (writer && !*abort_flag) {
+                unsigned char *outb = reinterpret_cast<unsigned char *>(p.out);
 #pragma unroll
                 for (int k = 0; k < UPW; ++k)
-#pragma unroll
-                    for (int h = 0; h < HC; ++h) {
-                        const float lh = __shfl_sync(0xffffffffu, unit[k].l_own, h * C::LPH);
-                        if (tg == 0) {
-                            const float inv = 1.f / lh;
-                            float2 r[4];
-#pragma unroll
-                            for (int i = 0; i < 4; ++i)
-                                r[i] = make_float2(unit[k].o2[h][i].x * inv, unit[k].o2[h][i].y * inv);
-                            const size_t hgl = (size_t)s.hg * p.NHvr + u_h0[k] + h;
-                            Elem<T>::store8(reinterpret_cast<unsigned char *>(p.out) +
-                                                (((size_t)s.b * p.Hq + hgl) * D + sl * 8) * E,
-                                            r);
-                        }
-                    }
+                    eng.write_out(unit[k], outb, (size_t)s.b * p.Hq + (size_t)s.hg * p.NHvr + u_h0[k]);
             }
             continue;
         }
@@ -763,20 +1182,7 @@ __global__ void __launch_bounds__(kDecodeThreads, 1) paged_decode_kernel(const D
         if (writer && slot_ok) {
             float *base = p.partials + s.slot * p.slot_floats;
 #pragma unroll
-            for (int k = 0; k < UPW; ++k)
-#pragma unroll
-                for (int h = 0; h < HC; ++h) {
-                    const float mh = __shfl_sync(0xffffffffu, unit[k].m_own, h * C::LPH);
-                    const float lh = __shfl_sync(0xffffffffu, unit[k].l_own, h * C::LPH);
-                    const int hl = u_h0[k] + h;
-                    if (tg == 0) {
-                        Elem<float>::store8(base + (size_t)hl * D + sl * 8, unit[k].o2[h]);
-                        if (sl == 0) {
-                            base[p.NHvr * D + hl] = mh;
-                            base[p.NHvr * D + p.NHvr + hl] = lh;
-                        }
-                    }
-                }
+            for (int k = 0; k < UPW; ++k) eng.write_partial(unit[k], base, p.NHvr, u_h0[k]);
         }
         if (!slot_ok && tid == 0) set_error(p.error, PA_DEVERR_WORKSPACE);
         __threadfence();
@@ -789,61 +1195,7 @@ __global__ void __launch_bounds__(kDecodeThreads, 1) paged_decode_kernel(const D
         named_barrier(1, kConsumerWarps * 32);
         if (ctl.merge_flag) {
             __threadfence();
-            // combine every piece of this vr by log-sum-exp
-            const int64_t NTc = NT;
-            const int64_t c0 = cta_of(s.vr_start, NTc, Cn);
-            const int nq = p.NHvr * (D / 4);
-            for (int idx = tid; idx < nq; idx += kConsumerWarps * 32) {
-                const int h = idx / (D / 4);
-                const int d4 = idx % (D / 4);
-                float M = -INFINITY;
-                for (int i = 0; i < s.nparts; ++i) {
-                    int64_t slot;
-                    if (p.mode == PA_SPLIT_BALANCED) {
-                        const int64_t c = c0 + i;
-                        slot = 2 * c + (s.vr_start <= range_lo(c, NTc, Cn) ? 0 : 1);
-                    } else {
-                        slot = s.vr_start + i;
-                    }
-                    if (slot >= p.max_slots) continue;
-                    const float *base = p.partials + slot * p.slot_floats;
-                    M = fmaxf(M, __ldcg(base + p.NHvr * D + h));
-                }
-                float4 num = make_float4(0.f, 0.f, 0.f, 0.f);
-                float den = 0.f;
-                for (int i = 0; i < s.nparts; ++i) {
-                    int64_t slot;
-                    if (p.mode == PA_SPLIT_BALANCED) {
-                        const int64_t c = c0 + i;
-                        slot = 2 * c + (s.vr_start <= range_lo(c, NTc, Cn) ? 0 : 1);
-                    } else {
-                        slot = s.vr_start + i;
-                    }
-                    if (slot >= p.max_slots) continue;
-                    const float *base = p.partials + slot * p.slot_floats;
-                    const float w = exp2f(__ldcg(base + p.NHvr * D + h) - M);
-                    den += w * __ldcg(base + p.NHvr * D + p.NHvr + h);
-                    const float4 o = __ldcg(reinterpret_cast<const float4 *>(base + (size_t)h * D) + d4);
-                    num.x += w * o.x;
-                    num.y += w * o.y;
-                    num.z += w * o.z;
-                    num.w += w * o.w;
-                }
-                const float inv = 1.f / den;
-                const size_t hgl = (size_t)s.hg * p.NHvr + h;
-                unsigned char *dst =
-                    reinterpret_cast<unsigned char *>(p.out) + (((size_t)s.b * p.Hq + hgl) * D + d4 * 4) * E;
-                if constexpr (E == 2) {
-                    __nv_bfloat162 a = __floats2bfloat162_rn(num.x * inv, num.y * inv);
-                    __nv_bfloat162 c = __floats2bfloat162_rn(num.z * inv, num.w * inv);
-                    uint2 w2;
-                    w2.x = *reinterpret_cast<uint32_t *>(&a);
-                    w2.y = *reinterpret_cast<uint32_t *>(&c);
-                    *reinterpret_cast<uint2 *>(dst) = w2;
-                } else {
-                    *reinterpret_cast<float4 *>(dst) = make_float4(num.x * inv, num.y * inv, num.z * inv, num.w * inv);
-                }
-            }
+            merge_vr<T, D>(p, s, NT, Cn, msm, tid);
             if (tid == 0) p.counters[vr] = 0;
         }
     }

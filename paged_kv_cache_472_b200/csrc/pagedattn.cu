@@ -53,27 +53,29 @@ pa_status check_shape(const pa_shape *s) {
 }
 
 // ---------------------------------------------------------------------------
-// decode kernel variants: (dtype, D, HC, UPW)
+// decode kernel variants.  bf16: tensor-core engine (D, units per warp);
+// fp32: CUDA-core engine (D, heads per unit, units per warp).
 using KernelFn = void (*)(const pa::DecodeParams);
 
-template <typename T, int D>
-KernelFn pick_hc_upw(int hc, int upw) {
+template <int D>
+KernelFn pick_core(int hc, int upw) {
 #define PA_CASE(H, U) \
-    if (hc == H && upw == U) return pa::paged_decode_kernel<T, D, H, U>;
+    if (hc == H && upw == U) return pa::paged_decode_kernel<float, D, pa::CoreEngine<float, D, H, U>>;
     PA_CASE(1, 1) PA_CASE(2, 1) PA_CASE(4, 1) PA_CASE(1, 2) PA_CASE(2, 2) PA_CASE(4, 2) PA_CASE(1, 4) PA_CASE(2, 4)
 #undef PA_CASE
     return nullptr;
 }
 
-KernelFn pick_kernel(int dtype, int D, int hc, int upw) {
-    if (dtype == PA_DTYPE_BF16) {
-        if (D == 64) return pick_hc_upw<__nv_bfloat16, 64>(hc, upw);
-        if (D == 128) return pick_hc_upw<__nv_bfloat16, 128>(hc, upw);
-    } else {
-        if (D == 64) return pick_hc_upw<float, 64>(hc, upw);
-        if (D == 128) return pick_hc_upw<float, 128>(hc, upw);
-    }
+template <int D>
+KernelFn pick_mma(int upw) {
+    if (upw == 1) return pa::paged_decode_kernel<__nv_bfloat16, D, pa::MmaEngine<D, 1>>;
+    if (upw == 2) return pa::paged_decode_kernel<__nv_bfloat16, D, pa::MmaEngine<D, 2>>;
     return nullptr;
+}
+
+KernelFn pick_kernel(int dtype, int D, int hc, int upw) {
+    if (dtype == PA_DTYPE_BF16) return D == 64 ? pick_mma<64>(upw) : (D == 128 ? pick_mma<128>(upw) : nullptr);
+    return D == 64 ? pick_core<64>(hc, upw) : (D == 128 ? pick_core<128>(hc, upw) : nullptr);
 }
 
 std::mutex g_attr_mu;
@@ -100,28 +102,204 @@ pa_status ensure_smem_attr(KernelFn fn, int bytes) {
 }
 
 struct Layout {
-    uint32_t off_bar, off_q, off_stage, off_scratch, off_comb, total;
+    uint32_t off_bar, off_q, off_stage, off_scratch, off_comb, off_merge, total;
+    uint32_t comb_stride;
 };
 
-Layout smem_layout(int stages, uint32_t q_bytes, uint32_t half_bytes, int hc, int D, int tsplit) {
+// shared-memory layout of one decode CTA
+Layout smem_layout(int dtype, int D, int stages, uint32_t q_bytes, uint32_t half_bytes, int hc, int tsplit,
+                   int nhvr) {
     Layout l;
+    const bool mma = dtype == PA_DTYPE_BF16;
     l.off_bar = 0;
     const uint32_t bar_bytes = (uint32_t)round_up((2 * stages + 4) * 8, 128);
     l.off_q = bar_bytes;
     l.off_stage = (uint32_t)round_up(l.off_q + 2 * q_bytes, 128);
     l.off_scratch = (uint32_t)round_up(l.off_stage + (size_t)stages * 2 * half_bytes, 128);
-    const uint32_t scratch = pa::kConsumerWarps * 2 * pa::kSubTile * hc * 4;
+    const uint32_t scratch = mma ? 0u : (uint32_t)(pa::kConsumerWarps * 2 * pa::kSubTile * hc * 4);
     l.off_comb = (uint32_t)round_up(l.off_scratch + scratch, 128);
-    const uint32_t comb = tsplit > 1 ? pa::kConsumerWarps * (uint32_t)(hc * D + 8) * 4 : 0;
-    l.total = (uint32_t)round_up(l.off_comb + comb, 128);
+    const uint32_t comb_floats = mma ? (uint32_t)(4 * (D / 16) * 32 + 4 * 32) : (uint32_t)(hc * D + 8);
+    l.comb_stride = comb_floats * 4;
+    const uint32_t comb = tsplit > 1 ? pa::kConsumerWarps * l.comb_stride : 0;
+    l.off_merge = (uint32_t)round_up(l.off_comb + comb, 128);
+    const uint32_t merge = (uint32_t)(2 * pa::kMergeParts + pa::kMergeParts * nhvr + nhvr) * 4;
+    l.total = (uint32_t)round_up(l.off_merge + merge, 128);
     return l;
+}
+
+// ---------------------------------------------------------------------------
+pa_status launch_append(const void *k_new, const void *v_new, const int32_t *slot_mapping, void *k_cache,
+                        void *v_cache, const pa_shape *s, int32_t *device_error, cudaStream_t stream) {
+    if (!k_new || !v_new || !slot_mapping || !k_cache || !v_cache)
+        return fail(PA_ERR_INVALID_ARG, "NULL tensor pointer");
+    if (!aligned16(k_new) || !aligned16(v_new) || !aligned16(k_cache) || !aligned16(v_cache))
+        return fail(PA_ERR_INVALID_ARG, "value tensors must be 16-byte aligned");
+    const int64_t token_bytes = (int64_t)s->Hkv * s->D * elem_bytes(s->dtype);
+    if (token_bytes % 16)
+        return fail(PA_ERR_UNSUPPORTED, "Hkv*D*elem=%lld is not a multiple of 16", (long long)token_bytes);
+    const int vec = (int)(token_bytes / 16);
+    const int64_t total = (int64_t)s->B * vec;
+    const int threads = 256;
+    int64_t blocks = (total + threads - 1) / threads;
+    if (blocks > 148 * 16) blocks = 148 * 16;
+    pa::kv_append_kernel<<<(unsigned)blocks, threads, 0, stream>>>(
+        (const uint4 *)k_new, (const uint4 *)v_new, slot_mapping, (uint4 *)k_cache, (uint4 *)v_cache, s->B, vec,
+        (int64_t)s->num_blocks * s->block_size, device_error);
+    cudaError_t e = cudaGetLastError();
+    if (e != cudaSuccess) return fail(PA_ERR_CUDA, "append launch: %s", cudaGetErrorString(e));
+    return PA_OK;
+}
+
+struct Mapping {
+    int HG, HC, UPW, TS;
+};
+
+// Head group HG (KV heads per work item), heads per warp unit HC, units per
+// warp UPW and warps per unit TS (token split) for one shape and engine.
+bool choose_mapping(const pa_shape *s, Mapping &m) {
+    const int G = s->Hq / s->Hkv;
+    const int e = elem_bytes(s->dtype);
+    const bool mma = s->dtype == PA_DTYPE_BF16;
+    for (int hg = s->Hkv; hg >= 1; --hg) {
+        if (s->Hkv % hg || hg * s->D * e > 2048) continue;
+        if (mma) {
+            // a unit is one KV head and up to 8 of its query heads (one n=8 tile)
+            const int hc = G < 8 ? G : 8;
+            const int U = hg * (G / hc);
+            if (U >= 8 && U % 8 == 0 && U / 8 <= 2) {
+                m = {hg, hc, U / 8, 1};
+                return true;
+            }
+            if (U < 8 && 8 % U == 0) {
+                m = {hg, hc, 1, 8 / U};
+                return true;
+            }
+            continue;
+        }
+        for (int hc = 4; hc >= 1; hc >>= 1) {
+            if (G % hc) continue;
+            const int U = hg * (G / hc);
+            if (U >= 8) {
+                if (U % 8) continue;
+                const int upw = U / 8;
+                if (upw > 4 || upw * hc > 8 || (upw == 4 && hc > 2)) continue;
+                m = {hg, hc, upw, 1};
+                return true;
+            }
+        }
+        const int U = hg * G;  // HC = 1
+        if (U < 8 && 8 % U == 0) {
+            m = {hg, 1, 1, 8 / U};
+            return true;
+        }
+    }
+    return false;
+}
+
+uint32_t row_pitch_of(const pa_shape *s, uint32_t row_bytes) {
+    return s->dtype == PA_DTYPE_BF16 ? row_bytes + 16 : row_bytes;  // padded rows for ldmatrix
+}
+
+pa_status launch_decode(const void *q, const void *k_cache, const void *v_cache, const int32_t *block_tables,
+                        const int32_t *context_lens, float scale, void *out, const pa_shape *s,
+                        const pa_plan_t *plan, void *workspace, size_t workspace_bytes, cudaStream_t stream,
+                        bool pdl) {
+    if (!plan) return fail(PA_ERR_INVALID_ARG, "plan is NULL");
+    if (memcmp(&plan->shape, s, sizeof *s) != 0) return fail(PA_ERR_INVALID_ARG, "plan was made for another shape");
+    if (!std::isfinite(scale)) return fail(PA_ERR_INVALID_ARG, "scale is not finite");
+    if (!workspace) return fail(PA_ERR_WORKSPACE, "workspace is NULL");
+    if (workspace_bytes < plan->workspace_bytes)
+        return fail(PA_ERR_WORKSPACE, "workspace %zu bytes < %zu needed", workspace_bytes, plan->workspace_bytes);
+    if ((reinterpret_cast<uintptr_t>(workspace) & 255u) != 0)
+        return fail(PA_ERR_INVALID_ARG, "workspace must be 256-byte aligned");
+    if (s->B == 0) return PA_OK;
+    if (!q || !k_cache || !v_cache || !block_tables || !context_lens || !out)
+        return fail(PA_ERR_INVALID_ARG, "NULL tensor pointer");
+    if (!aligned16(q) || !aligned16(k_cache) || !aligned16(v_cache) || !aligned16(out))
+        return fail(PA_ERR_INVALID_ARG, "value tensors must be 16-byte aligned");
+
+    const int HC = plan->heads_per_unit, UPW = plan->units_per_warp, TS = plan->warps_per_unit;
+    const int G = s->Hq / s->Hkv;
+    const int e = elem_bytes(s->dtype);
+    KernelFn fn = pick_kernel(s->dtype, s->D, HC, UPW);
+    if (!fn) return fail(PA_ERR_INVALID_ARG, "plan names no kernel variant");
+    const int HG = plan->head_group;
+    const int NHvr = HG * G;
+    const uint32_t row_bytes = (uint32_t)(HG * s->D * e);
+    const uint32_t pitch = row_pitch_of(s, row_bytes);
+    const uint32_t half = (uint32_t)plan->tile_tokens * pitch;
+    const uint32_t q_bytes = (uint32_t)(NHvr * s->D * e);
+    const Layout lay = smem_layout(s->dtype, s->D, plan->stages, q_bytes, half, HC, TS, NHvr);
+    if ((int)lay.total != plan->smem_bytes) return fail(PA_ERR_INVALID_ARG, "plan is inconsistent");
+
+    pa::DecodeParams p{};
+    p.q = q;
+    p.k_cache = k_cache;
+    p.v_cache = v_cache;
+    p.block_tables = block_tables;
+    p.context_lens = context_lens;
+    p.out = out;
+    unsigned char *ws = static_cast<unsigned char *>(workspace);
+    const size_t counters = round_up((size_t)s->B * (s->Hkv / HG) * 4, 256);
+    p.error = reinterpret_cast<int32_t *>(ws);
+    p.counters = reinterpret_cast<int32_t *>(ws + kWsHeader);
+    p.partials = reinterpret_cast<float *>(ws + kWsHeader + counters);
+    p.qscale = scale * 1.4426950408889634f;
+    p.B = s->B;
+    p.Hq = s->Hq;
+    p.Hkv = s->Hkv;
+    p.bs = s->block_size;
+    p.num_blocks = s->num_blocks;
+    p.max_blocks = s->max_blocks_per_seq;
+    p.G = G;
+    p.HG = HG;
+    p.NHG = s->Hkv / HG;
+    p.NHvr = NHvr;
+    p.ST = plan->tile_tokens;
+    p.stages = plan->stages;
+    p.mode = plan->mode;
+    p.part_tiles = plan->mode == PA_SPLIT_FIXED ? plan->partition_tokens / plan->tile_tokens : 1;
+    p.num_ctas = plan->num_ctas;
+    p.tsplit = TS;
+    p.units = HG * (G / HC);
+    p.heads_per_unit = HC;
+    p.pdl = pdl ? 1 : 0;
+    p.max_slots = plan->max_slots;
+    p.slot_floats = (int64_t)NHvr * s->D + (int64_t)round_up(2 * NHvr, 4);
+    p.off_bar = lay.off_bar;
+    p.off_q = lay.off_q;
+    p.off_stage = lay.off_stage;
+    p.off_scratch = lay.off_scratch;
+    p.off_comb = lay.off_comb;
+    p.off_merge = lay.off_merge;
+    p.row_bytes = row_bytes;
+    p.row_pitch = pitch;
+    p.half_bytes = half;
+    p.q_bytes = q_bytes;
+    p.comb_stride = lay.comb_stride;
+
+    if (pa_status st = ensure_smem_attr(fn, plan->smem_bytes)) return st;
+    cudaLaunchConfig_t cfg = {};
+    cfg.gridDim = dim3((unsigned)plan->num_ctas);
+    cfg.blockDim = dim3(pa::kDecodeThreads);
+    cfg.dynamicSmemBytes = (size_t)plan->smem_bytes;
+    cfg.stream = stream;
+    cudaLaunchAttribute attr[1];
+    attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+    attr[0].val.programmaticStreamSerializationAllowed = 1;
+    cfg.attrs = attr;
+    cfg.numAttrs = pdl ? 1 : 0;
+    cudaError_t ce = cudaLaunchKernelEx(&cfg, fn, p);
+    if (ce == cudaSuccess) ce = cudaGetLastError();
+    if (ce != cudaSuccess) return fail(PA_ERR_CUDA, "decode launch: %s", cudaGetErrorString(ce));
+    return PA_OK;
 }
 
 }  // namespace
 
 extern "C" {
 
-int32_t pa_version(void) { return 100; }
+int32_t pa_version(void) { return 200; }
 
 const char *pa_status_str(pa_status st) {
     switch (st) {
@@ -140,22 +318,9 @@ pa_status pa_kv_append(const void *k_new, const void *v_new, const int32_t *slot
                        void *v_cache, const pa_shape *s, int32_t *device_error, void *stream) {
     if (pa_status st = check_shape(s)) return st;
     if (s->B == 0) return ok();
-    if (!k_new || !v_new || !slot_mapping || !k_cache || !v_cache)
-        return fail(PA_ERR_INVALID_ARG, "NULL tensor pointer");
-    if (!aligned16(k_new) || !aligned16(v_new) || !aligned16(k_cache) || !aligned16(v_cache))
-        return fail(PA_ERR_INVALID_ARG, "value tensors must be 16-byte aligned");
-    const int64_t token_bytes = (int64_t)s->Hkv * s->D * elem_bytes(s->dtype);
-    if (token_bytes % 16) return fail(PA_ERR_UNSUPPORTED, "Hkv*D*elem=%lld is not a multiple of 16", (long long)token_bytes);
-    const int vec = (int)(token_bytes / 16);
-    const int64_t total = (int64_t)s->B * vec;
-    const int threads = 256;
-    int64_t blocks = (total + threads - 1) / threads;
-    if (blocks > 148 * 16) blocks = 148 * 16;
-    pa::kv_append_kernel<<<(unsigned)blocks, threads, 0, (cudaStream_t)stream>>>(
-        (const uint4 *)k_new, (const uint4 *)v_new, slot_mapping, (uint4 *)k_cache, (uint4 *)v_cache, s->B, vec,
-        (int64_t)s->num_blocks * s->block_size, device_error);
-    cudaError_t e = cudaGetLastError();
-    if (e != cudaSuccess) return fail(PA_ERR_CUDA, "append launch: %s", cudaGetErrorString(e));
+    if (pa_status st = launch_append(k_new, v_new, slot_mapping, k_cache, v_cache, s, device_error,
+                                     (cudaStream_t)stream))
+        return st;
     return ok();
 }
 
@@ -181,52 +346,35 @@ pa_status pa_plan(const pa_shape *s, int32_t max_context_len, int32_t partition_
         if (ce != cudaSuccess) return fail(PA_ERR_CUDA, "querying the SM count: %s", cudaGetErrorString(ce));
     }
 
-    // Head group HG (KV heads per work item), heads per warp unit HC, units
-    // per warp UPW and warps per unit (token split).
-    int HG = 0, HC = 0, UPW = 0, TS = 0;
-    for (int hg = s->Hkv; hg >= 1 && !HG; --hg) {
-        if (s->Hkv % hg || hg * s->D * e > 2048) continue;
-        for (int hc = 4; hc >= 1; hc >>= 1) {
-            if (G % hc) continue;
-            const int U = hg * (G / hc);
-            if (U >= 8) {
-                if (U % 8) continue;
-                const int upw = U / 8;
-                if (upw > 4 || upw * hc > 8 || (upw == 4 && hc > 2)) continue;
-                HG = hg, HC = hc, UPW = upw, TS = 1;
-                break;
-            }
-        }
-        if (!HG && s->Hkv % hg == 0 && hg * s->D * e <= 2048) {
-            const int U = hg * G;  // HC = 1
-            if (U < 8 && 8 % U == 0) HG = hg, HC = 1, UPW = 1, TS = 8 / U;
-        }
-    }
-    if (!HG) return fail(PA_ERR_UNSUPPORTED, "no warp mapping for Hq=%d Hkv=%d D=%d", s->Hq, s->Hkv, s->D);
+    Mapping mp;
+    if (!choose_mapping(s, mp))
+        return fail(PA_ERR_UNSUPPORTED, "no warp mapping for Hq=%d Hkv=%d D=%d", s->Hq, s->Hkv, s->D);
+    const int HG = mp.HG, HC = mp.HC, UPW = mp.UPW, TS = mp.TS;
     const int NHvr = HG * G;
     const int NHG = s->Hkv / HG;
     const uint32_t row_bytes = (uint32_t)(HG * s->D * e);
+    const uint32_t pitch = row_pitch_of(s, row_bytes);
     const uint32_t q_bytes = (uint32_t)(NHvr * s->D * e);
 
     int ST = 16;
     while (ST * 2 <= 256 && (uint32_t)(ST * 2) * row_bytes <= (uint32_t)kStageTargetBytes) ST *= 2;
-    int mode = PA_SPLIT_BALANCED, part_tiles = 1;
+    int mode = PA_SPLIT_BALANCED;
     if (partition_tokens > 0) {
-        if (partition_tokens % 16) return fail(PA_ERR_INVALID_ARG, "partition_tokens=%d is not a multiple of 16", partition_tokens);
+        if (partition_tokens % 16)
+            return fail(PA_ERR_INVALID_ARG, "partition_tokens=%d is not a multiple of 16", partition_tokens);
         mode = PA_SPLIT_FIXED;
         while (partition_tokens % ST) ST /= 2;  // tiles must not straddle partitions
-        part_tiles = partition_tokens / ST;
     }
     int stages = 0;
     Layout lay{};
     for (;;) {
-        const uint32_t half = (uint32_t)ST * row_bytes;
+        const uint32_t half = (uint32_t)ST * pitch;
         for (stages = kMaxStages; stages >= 2; --stages) {
-            lay = smem_layout(stages, q_bytes, half, HC, s->D, TS);
+            lay = smem_layout(s->dtype, s->D, stages, q_bytes, half, HC, TS, NHvr);
             if (lay.total + 256 <= (uint32_t)kSmemLimit) break;
         }
         if (stages >= 2) break;
-        if (ST == 16 || mode == PA_SPLIT_FIXED) return fail(PA_ERR_UNSUPPORTED, "shared memory too small for this shape");
+        if (ST == 16) return fail(PA_ERR_UNSUPPORTED, "shared memory too small for this shape");
         ST /= 2;
     }
 
@@ -268,77 +416,27 @@ pa_status pa_decode(const void *q, const void *k_cache, const void *v_cache, con
                     const int32_t *context_lens, float scale, void *out, const pa_shape *s, const pa_plan_t *plan,
                     void *workspace, size_t workspace_bytes, void *stream) {
     if (pa_status st = check_shape(s)) return st;
-    if (!plan) return fail(PA_ERR_INVALID_ARG, "plan is NULL");
-    if (memcmp(&plan->shape, s, sizeof *s) != 0) return fail(PA_ERR_INVALID_ARG, "plan was made for another shape");
-    if (!std::isfinite(scale)) return fail(PA_ERR_INVALID_ARG, "scale is not finite");
-    if (!workspace) return fail(PA_ERR_WORKSPACE, "workspace is NULL");
-    if (workspace_bytes < plan->workspace_bytes)
-        return fail(PA_ERR_WORKSPACE, "workspace %zu bytes < %zu needed", workspace_bytes, plan->workspace_bytes);
-    if ((reinterpret_cast<uintptr_t>(workspace) & 255u) != 0) return fail(PA_ERR_INVALID_ARG, "workspace must be 256-byte aligned");
+    if (pa_status st = launch_decode(q, k_cache, v_cache, block_tables, context_lens, scale, out, s, plan, workspace,
+                                     workspace_bytes, (cudaStream_t)stream, false))
+        return st;
+    return ok();
+}
+
+pa_status pa_kv_append_decode(const void *k_new, const void *v_new, const int32_t *slot_mapping, const void *q,
+                              void *k_cache, void *v_cache, const int32_t *block_tables,
+                              const int32_t *context_lens, float scale, void *out, const pa_shape *s,
+                              const pa_plan_t *plan, void *workspace, size_t workspace_bytes, void *stream) {
+    if (pa_status st = check_shape(s)) return st;
     if (s->B == 0) return ok();
-    if (!q || !k_cache || !v_cache || !block_tables || !context_lens || !out)
-        return fail(PA_ERR_INVALID_ARG, "NULL tensor pointer");
-    if (!aligned16(q) || !aligned16(k_cache) || !aligned16(v_cache) || !aligned16(out))
-        return fail(PA_ERR_INVALID_ARG, "value tensors must be 16-byte aligned");
-
-    const int HC = plan->heads_per_unit, UPW = plan->units_per_warp, TS = plan->warps_per_unit;
-    const int G = s->Hq / s->Hkv;
-    const int e = elem_bytes(s->dtype);
-    KernelFn fn = pick_kernel(s->dtype, s->D, HC, UPW);
-    if (!fn) return fail(PA_ERR_INVALID_ARG, "plan names no kernel variant");
-    const int HG = plan->head_group;
-    const int NHvr = HG * G;
-    const uint32_t row_bytes = (uint32_t)(HG * s->D * e);
-    const uint32_t half = (uint32_t)plan->tile_tokens * row_bytes;
-    const uint32_t q_bytes = (uint32_t)(NHvr * s->D * e);
-    const Layout lay = smem_layout(plan->stages, q_bytes, half, HC, s->D, TS);
-    if ((int)lay.total != plan->smem_bytes) return fail(PA_ERR_INVALID_ARG, "plan is inconsistent");
-
-    pa::DecodeParams p{};
-    p.q = q;
-    p.k_cache = k_cache;
-    p.v_cache = v_cache;
-    p.block_tables = block_tables;
-    p.context_lens = context_lens;
-    p.out = out;
-    unsigned char *ws = static_cast<unsigned char *>(workspace);
-    const size_t counters = round_up((size_t)s->B * (s->Hkv / HG) * 4, 256);
-    p.error = reinterpret_cast<int32_t *>(ws);
-    p.counters = reinterpret_cast<int32_t *>(ws + kWsHeader);
-    p.partials = reinterpret_cast<float *>(ws + kWsHeader + counters);
-    p.qscale = scale * 1.4426950408889634f;
-    p.B = s->B;
-    p.Hq = s->Hq;
-    p.Hkv = s->Hkv;
-    p.bs = s->block_size;
-    p.num_blocks = s->num_blocks;
-    p.max_blocks = s->max_blocks_per_seq;
-    p.G = G;
-    p.HG = HG;
-    p.NHG = s->Hkv / HG;
-    p.NHvr = NHvr;
-    p.ST = plan->tile_tokens;
-    p.stages = plan->stages;
-    p.mode = plan->mode;
-    p.part_tiles = plan->mode == PA_SPLIT_FIXED ? plan->partition_tokens / plan->tile_tokens : 1;
-    p.num_ctas = plan->num_ctas;
-    p.tsplit = TS;
-    p.units = HG * (G / HC);
-    p.max_slots = plan->max_slots;
-    p.slot_floats = (int64_t)NHvr * s->D + (int64_t)round_up(2 * NHvr, 4);
-    p.off_bar = lay.off_bar;
-    p.off_q = lay.off_q;
-    p.off_stage = lay.off_stage;
-    p.off_scratch = lay.off_scratch;
-    p.off_comb = lay.off_comb;
-    p.row_bytes = row_bytes;
-    p.half_bytes = half;
-    p.q_bytes = q_bytes;
-
-    if (pa_status st = ensure_smem_attr(fn, plan->smem_bytes)) return st;
-    fn<<<plan->num_ctas, pa::kDecodeThreads, plan->smem_bytes, (cudaStream_t)stream>>>(p);
-    cudaError_t ce = cudaGetLastError();
-    if (ce != cudaSuccess) return fail(PA_ERR_CUDA, "decode launch: %s", cudaGetErrorString(ce));
+    if (!workspace || workspace_bytes < (plan ? plan->workspace_bytes : 0) ||
+        (reinterpret_cast<uintptr_t>(workspace) & 255u) != 0)
+        return fail(PA_ERR_WORKSPACE, "workspace missing, too small or not 256-byte aligned");
+    if (pa_status st = launch_append(k_new, v_new, slot_mapping, k_cache, v_cache, s,
+                                     static_cast<int32_t *>(workspace), (cudaStream_t)stream))
+        return st;
+    if (pa_status st = launch_decode(q, k_cache, v_cache, block_tables, context_lens, scale, out, s, plan, workspace,
+                                     workspace_bytes, (cudaStream_t)stream, true))
+        return st;
     return ok();
 }
 

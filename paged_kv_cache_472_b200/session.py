@@ -5,8 +5,8 @@ from __future__ import annotations
 
 import torch
 
-from . import (DTYPE_BF16, DTYPE_F32, Plan, Shape, pa_decode, pa_get_device_error, pa_kv_append, pa_plan,
-               pa_workspace_init)
+from . import (DTYPE_BF16, DTYPE_F32, Plan, Shape, pa_decode, pa_get_device_error, pa_kv_append,
+               pa_kv_append_decode, pa_plan, pa_workspace_init)
 
 TORCH_DTYPE = {DTYPE_F32: torch.float32, DTYPE_BF16: torch.bfloat16}
 PA_DTYPE = {torch.float32: DTYPE_F32, torch.bfloat16: DTYPE_BF16}
@@ -43,6 +43,12 @@ class PagedDecoder:
 
     def append(self, k_new, v_new, slot_mapping, k_cache, v_cache, stream=None):
         pa_kv_append(k_new, v_new, slot_mapping, k_cache, v_cache, self.shape, self.workspace, stream)
+
+    def append_decode(self, k_new, v_new, slot_mapping, q, k_cache, v_cache, block_tables, context_lens, scale, out,
+                      stream=None):
+        pa_kv_append_decode(k_new, v_new, slot_mapping, q, k_cache, v_cache, block_tables, context_lens, scale, out,
+                            self.shape, self.plan, self.workspace, self.workspace.numel(), stream)
+        return out
 
     def device_error(self, clear: bool = False) -> int:
         return pa_get_device_error(self.workspace, clear)

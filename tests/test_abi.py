@@ -28,7 +28,7 @@ def declared_symbols():
 
 def test_every_declared_symbol_is_exported():
     names = declared_symbols()
-    assert len(names) >= 9, names
+    assert len(names) >= 10, names
     for n in names:
         assert hasattr(pa.lib, n), n
 
@@ -62,16 +62,27 @@ def test_plan_workloads(cid):
         assert plan.mode == pa.SPLIT_FIXED and plan.partition_tokens % plan.tile_tokens == 0
     else:
         assert plan.mode == pa.SPLIT_BALANCED and plan.max_slots == 2 * 148
-    expect = {1: (2, 1, 2), 2: (8, 2, 1), 3: (8, 4, 1), 4: (1, 4, 1), 5: (8, 4, 1)}[cid]
+    expect = {1: (2, 1, 2), 2: (8, 2, 1), 3: (8, 4, 1), 4: (1, 8, 2), 5: (8, 4, 1)}[cid]
     assert (plan.head_group, plan.heads_per_unit, plan.warps_per_unit) == expect
 
 
 @pytest.mark.parametrize("Hq,Hkv,D,upw,hc,hg,ts", [
     (32, 32, 128, 1, 1, 8, 1), (16, 16, 64, 2, 1, 16, 1), (64, 16, 64, 2, 4, 16, 1), (32, 16, 64, 2, 2, 16, 1),
-    (64, 16, 128, 1, 4, 8, 1), (4, 1, 128, 1, 1, 1, 2), (8, 1, 128, 1, 1, 1, 1), (64, 1, 128, 2, 4, 1, 1),
-    (2, 2, 64, 1, 1, 2, 4), (1, 1, 64, 1, 1, 1, 8)])
+    (64, 16, 128, 1, 4, 8, 1), (4, 1, 128, 1, 4, 1, 8), (8, 1, 128, 1, 8, 1, 8), (64, 1, 128, 1, 8, 1, 1),
+    (2, 2, 64, 1, 1, 2, 4), (1, 1, 64, 1, 1, 1, 8), (32, 1, 128, 1, 8, 1, 2)])
 def test_plan_head_mappings(Hq, Hkv, D, upw, hc, hg, ts):
+    """bf16 shapes use the tensor-core engine: a unit is one KV head with up to 8 query heads."""
     s = pa.Shape(3, Hq, Hkv, D, 16, 64, 8, pa.DTYPE_BF16)
+    plan = pa.pa_plan(s, 128, 0, 148)
+    assert (plan.units_per_warp, plan.heads_per_unit, plan.head_group, plan.warps_per_unit) == (upw, hc, hg, ts)
+
+
+@pytest.mark.parametrize("Hq,Hkv,D,upw,hc,hg,ts", [
+    (4, 2, 64, 1, 1, 2, 2), (16, 4, 128, 1, 2, 4, 1), (8, 2, 64, 1, 1, 2, 1), (1, 1, 64, 1, 1, 1, 8),
+    (32, 32, 64, 1, 1, 8, 1)])
+def test_plan_head_mappings_fp32(Hq, Hkv, D, upw, hc, hg, ts):
+    """fp32 shapes use the CUDA-core engine."""
+    s = pa.Shape(3, Hq, Hkv, D, 16, 64, 8, pa.DTYPE_F32)
     plan = pa.pa_plan(s, 128, 0, 148)
     assert (plan.units_per_warp, plan.heads_per_unit, plan.head_group, plan.warps_per_unit) == (upw, hc, hg, ts)
 

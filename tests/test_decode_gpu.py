@@ -174,3 +174,21 @@ def test_repeated_calls_reuse_workspace(orc):
     assert dec.device_error() == 0
     counters = dec.workspace[256:256 + 4 * case.B * case.Hkv].view(torch.int32)
     assert int(counters.abs().sum()) == 0
+
+
+@pytest.mark.parametrize("cid,batch", [(2, None), (3, 32), (5, 48), (1, None)])
+def test_fused_append_decode_matches_separate_calls(orc, cid, batch):
+    """pa_kv_append_decode (decode chained to the append by programmatic
+    dependent launch) gives bit-identical results to the two separate calls."""
+    case = synth.make_config(cid, batch=batch)
+    dev_a, dec_a, err_a = H.run(case, 0)
+    dev_b = H.upload(case)
+    dec_b = H.PagedDecoder(H.shape_of(case), int(case.context_lens.max()), 0)
+    for _ in range(3):   # repeated steps: the append is idempotent, the result must not change
+        dec_b.append_decode(dev_b.k_new, dev_b.v_new, dev_b.slot_mapping, dev_b.q, dev_b.k_cache, dev_b.v_cache,
+                            dev_b.block_tables, dev_b.context_lens, case.scale, dev_b.out)
+    torch.cuda.synchronize()
+    assert err_a == 0 and dec_b.device_error() == 0
+    assert torch.equal(dev_a.k_cache, dev_b.k_cache) and torch.equal(dev_a.v_cache, dev_b.v_cache)
+    assert torch.equal(dev_a.out, dev_b.out)
+    H.assert_close(H.out_f64(dev_b), oracle_out(orc, case), case.dtype, "fused")
