@@ -591,11 +591,9 @@ struct MmaEngine {
         }
         const float mn0 = fmaxf(u.m[0], mx0), mn1 = fmaxf(u.m[1], mx1);
         const float al0 = exp2f(u.m[0] - mn0), al1 = exp2f(u.m[1] - mn1);
-        const uint32_t pb0 = pack_bf16x2(exp2f(s0 - mn0), exp2f(s1 - mn1));  // token g4
-        const uint32_t pb1 = pack_bf16x2(exp2f(s2 - mn0), exp2f(s3 - mn1));  // token g4 + 8
-        // the denominator sums the same (rounded) weights the PV product uses
-        const float2 f0 = bf16x2_to_float2(pb0), f1 = bf16x2_to_float2(pb1);
-        float r0 = f0.x + f1.x, r1 = f0.y + f1.y;
+        const float p0 = exp2f(s0 - mn0), p1 = exp2f(s1 - mn1);  // token g4
+        const float p2 = exp2f(s2 - mn0), p3 = exp2f(s3 - mn1);  // token g4 + 8
+        float r0 = p0 + p2, r1 = p1 + p3;
 #pragma unroll
         for (int m = 4; m < 32; m <<= 1) {
             r0 += __shfl_xor_sync(0xffffffffu, r0, m);
@@ -605,9 +603,15 @@ struct MmaEngine {
         u.l[1] = u.l[1] * al1 + r1;
         u.m[0] = mn0;
         u.m[1] = mn1;
+        // P = hi + lo, both bf16: the PV product then carries ~16 bits of each
+        // weight instead of 8 (one bf16 P alone misses the tolerance on very
+        // short, peaked contexts)
+        const uint32_t ph0 = pack_bf16x2(p0, p1), ph1 = pack_bf16x2(p2, p3);
+        const float2 h0 = bf16x2_to_float2(ph0), h1 = bf16x2_to_float2(ph1);
+        const uint32_t pl0 = pack_bf16x2(p0 - h0.x, p1 - h0.y), pl1 = pack_bf16x2(p2 - h1.x, p3 - h1.y);
         // P^T fragments (k = token, n = head)
-        const uint32_t b0 = movmatrix_trans(pb0);
-        const uint32_t b1 = movmatrix_trans(pb1);
+        const uint32_t bh0 = movmatrix_trans(ph0), bh1 = movmatrix_trans(ph1);
+        const uint32_t bl0 = movmatrix_trans(pl0), bl1 = movmatrix_trans(pl1);
         if (al0 != 1.f || al1 != 1.f) {
 #pragma unroll
             for (int mt = 0; mt < KS; ++mt) {
@@ -630,7 +634,8 @@ struct MmaEngine {
         for (int mt = 0; mt < KS; ++mt) {
             uint32_t a[4];
             ldmatrix_x4_trans(a, va + mt * 16 * E);
-            mma_bf16_16816(u.o[mt], a, b0, b1);
+            mma_bf16_16816(u.o[mt], a, bh0, bh1);
+            mma_bf16_16816(u.o[mt], a, bl0, bl1);
         }
     }
 
