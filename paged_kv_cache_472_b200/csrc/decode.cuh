@@ -42,6 +42,8 @@
 //     elements of all its heads.
 #pragma once
 
+#include <cstddef>
+
 #include "common.cuh"
 
 namespace pa {
@@ -52,6 +54,8 @@ constexpr int kSubTile = 16;     // tokens per online-softmax update
 constexpr int kMergeParts = 64;  // pieces the shared-memory merge path handles
 
 struct DecodeParams {
+    CUtensorMap tmap_k;   // bf16 path: [d, token row, head] view of the pools, 128B swizzle,
+    CUtensorMap tmap_v;   // box {64, br, HG}: one block piece of one head group, head-major in smem
     const void *q;
     const void *k_cache;
     const void *v_cache;
@@ -81,7 +85,13 @@ struct DecodeParams {
     uint32_t half_bytes;  // ST * row_pitch (K part of a stage; V part follows)
     uint32_t q_bytes;     // NHvr * D * elem
     uint32_t comb_stride; // bytes per warp in the token-split combine area
+    int32_t use_tmap;     // 1: stages are filled by tensor-map boxes (swizzled, head-major)
+    int32_t br_log2;      // rows of one box = min(ST, bs) = 1 << br_log2
+    int32_t bs_log2;
+    int32_t lens_cached;  // context lengths were copied into shared memory
 };
+static_assert(offsetof(DecodeParams, tmap_k) % 64 == 0 && offsetof(DecodeParams, tmap_v) % 64 == 0,
+              "tensor maps must be 64-byte aligned");
 
 // ---------------------------------------------------------------------------
 // element access
@@ -144,8 +154,10 @@ struct Elem<float> {
 
 // ---------------------------------------------------------------------------
 // work list (identical sequence in every warp of a CTA)
-__device__ __forceinline__ int clamped_len(const DecodeParams &p, int b) {
-    int L = p.context_lens[b];
+constexpr int kLensCache = 1024;  // requests whose lengths are kept in shared memory
+
+__device__ __forceinline__ int clamped_len(const DecodeParams &p, const int *lens_s, int b) {
+    int L = p.lens_cached ? lens_s[b] : p.context_lens[b];
     const int cap = p.max_blocks * p.bs;
     return L < 0 ? 0 : (L > cap ? cap : L);
 }
@@ -174,6 +186,7 @@ struct SegIter {
     int64_t cur, hi, lo, NT, C;
     int64_t vr_start;
     int b, hg, L, units;
+    const int *lens_s;
 
     __device__ __forceinline__ bool next(const DecodeParams &p, Seg &s) {
         while (cur < hi) {
@@ -183,7 +196,7 @@ struct SegIter {
                     hg = 0;
                     ++b;
                     if (b >= p.B) return false;
-                    L = clamped_len(p, b);
+                    L = clamped_len(p, lens_s, b);
                     units = units_of_len(p, L);
                 }
                 continue;
@@ -329,8 +342,12 @@ struct CoreEngine {
         u.l_own = 0.f;
     }
 
-    __device__ __forceinline__ void subtile(Unit &u, const unsigned char *kst, const unsigned char *vst, int g_local,
-                                            int nvalid, uint32_t pitch, float *s_sm, float *p_sm, int lane) const {
+    __device__ __forceinline__ void subtile(Unit &u, const unsigned char *tile_k, const unsigned char *tile_v, int st,
+                                            int g_local, int nvalid, const DecodeParams &p, float *s_sm, float *p_sm,
+                                            int lane) const {
+        const uint32_t pitch = p.row_pitch;
+        const unsigned char *kst = tile_k + (size_t)st * kSubTile * pitch;
+        const unsigned char *vst = tile_v + (size_t)st * kSubTile * pitch;
         const uint32_t col = (uint32_t)(g_local * D + sl * 8) * E;
 
         // ---- QK: partial dots over this lane's 8 elements (rounds permuted per lane) ----
@@ -565,16 +582,31 @@ struct MmaEngine {
         u.l[0] = u.l[1] = 0.f;
     }
 
-    __device__ __forceinline__ void subtile(Unit &u, const unsigned char *kst, unsigned char *vst, int g_local,
-                                            int nvalid, uint32_t pitch, float *, float *, int lane) const {
-        const uint32_t colb = (uint32_t)g_local * D * E;
+    // Stage layout (filled by tensor-map boxes): [piece][d-chunk of 64][head][row][128 B],
+    // each 128-byte row stored with the 128B swizzle (16-byte chunk c of row r at c ^ (r & 7)).
+    // Address of 16-byte chunk `cid` (0..15 over the head's D) of row `tok` of the tile.
+    static __device__ __forceinline__ const unsigned char *row_ptr(const unsigned char *tile, int tok, int g_local,
+                                                                  const DecodeParams &p) {
+        const int piece = tok >> p.br_log2, r = tok & ((1 << p.br_log2) - 1);
+        const uint32_t head_bytes = 128u << p.br_log2;
+        return tile + ((size_t)piece * (D / 64) * p.HG + g_local) * head_bytes + r * 128;
+    }
+    static __device__ __forceinline__ uint32_t chunk_off(int cid, int swz, const DecodeParams &p) {
+        // d-chunk (cid / 8) selects the 64-element half; within it the swizzled 16-byte slot
+        return (uint32_t)(cid >> 3) * ((uint32_t)p.HG << (7 + p.br_log2)) + (uint32_t)(((cid & 7) ^ swz) << 4);
+    }
+
+    __device__ __forceinline__ void subtile(Unit &u, const unsigned char *tile_k, unsigned char *tile_v, int st,
+                                            int g_local, int nvalid, const DecodeParams &p, float *, float *,
+                                            int lane) const {
         // ---- S^T[16 tok x 8 heads] = K Q^T ----
         float s[4] = {0.f, 0.f, 0.f, 0.f};
-        const unsigned char *ka = kst + a_tok * pitch + colb + a_col * E;
+        const unsigned char *ka = row_ptr(tile_k, st * kSubTile + a_tok, g_local, p);
+        const int swz = a_tok & 7;
 #pragma unroll
         for (int ks = 0; ks < KS; ++ks) {
             uint32_t a[4];
-            ldmatrix_x4(a, ka + ks * 16 * E);
+            ldmatrix_x4(a, ka + chunk_off(ks * 2 + (a_col >> 3), swz, p));
             mma_bf16_16816(s, a, u.qb[ks][0], u.qb[ks][1]);
         }
         // ---- online softmax over the 16 tokens, per head column ----
@@ -621,19 +653,23 @@ struct MmaEngine {
                 u.o[mt][3] *= al1;
             }
         }
-        // rows past nvalid may hold stale data: zero this unit's columns there
+        // rows past nvalid may hold stale data: zero this head's rows there
         if (nvalid < kSubTile) {
-            for (int r = nvalid; r < kSubTile; ++r)
-                for (int c = lane; c < D * E / 16; c += 32)
-                    *reinterpret_cast<uint4 *>(vst + r * pitch + colb + c * 16) = make_uint4(0, 0, 0, 0);
+            for (int i = lane; i < (kSubTile - nvalid) * (D / 8); i += 32) {
+                const int tok = st * kSubTile + nvalid + i / (D / 8);
+                const int cid = i % (D / 8);
+                unsigned char *row = const_cast<unsigned char *>(row_ptr(tile_v, tok, g_local, p));
+                *reinterpret_cast<uint4 *>(row + chunk_off(cid, 0, p)) = make_uint4(0, 0, 0, 0);
+            }
             __syncwarp();
         }
         // ---- O^T[d x heads] += V^T P^T ----
-        const unsigned char *va = vst + v_tok * pitch + colb + v_col * E;
+        const unsigned char *va = row_ptr(tile_v, st * kSubTile + v_tok, g_local, p);
+        const int vswz = v_tok & 7;
 #pragma unroll
         for (int mt = 0; mt < KS; ++mt) {
             uint32_t a[4];
-            ldmatrix_x4_trans(a, va + mt * 16 * E);
+            ldmatrix_x4_trans(a, va + chunk_off(mt * 2 + (v_col >> 3), vswz, p));
             mma_bf16_16816(u.o[mt], a, bh0, bh1);
             mma_bf16_16816(u.o[mt], a, bl0, bl1);
         }
@@ -769,7 +805,36 @@ __device__ __forceinline__ void run_producer(const DecodeParams &p, SegIter it, 
             unsigned char *kdst = stage_base + (size_t)stage * 2 * p.half_bytes;
             unsigned char *vdst = kdst + p.half_bytes;
             uint32_t bytes = 0;
-            if (contiguous) {
+            if (p.use_tmap) {
+                // one box {64 d, br rows, HG heads} per (block piece, 64-wide d-chunk), for K and V
+                const int br = 1 << p.br_log2;
+                const int npc = (ntok + br - 1) >> p.br_log2;  // pieces holding valid tokens
+                const uint32_t box_bytes = (uint32_t)p.HG << (7 + p.br_log2);
+                constexpr int NDC = D / 64;
+                const int tp = tok0 + lane * br;                 // first token of this lane's piece
+                const int j = tp >> p.bs_log2;
+                const int phys = __shfl_sync(0xffffffffu, cur_val, (j - cur_base) & 31);
+                bool valid = false;
+                if (lane < npc) {
+                    valid = phys >= 0 && phys < p.num_blocks;
+                    if (!valid) set_error(p.error, PA_DEVERR_BLOCK_ID);
+                    else bytes = 2u * NDC * box_bytes;
+                }
+#pragma unroll
+                for (int m = 16; m >= 1; m >>= 1) bytes += __shfl_xor_sync(0xffffffffu, bytes, m);
+                if (lane == 0) mbar_arrive_expect_tx(&full[stage], bytes);
+                __syncwarp();
+                if (valid) {
+                    const int32_t row = phys * p.bs + (tp & (p.bs - 1));
+                    const int32_t head0 = s.hg * p.HG;
+#pragma unroll
+                    for (int c2 = 0; c2 < NDC; ++c2) {
+                        const size_t off = (size_t)(lane * NDC + c2) * box_bytes;
+                        tma_load_3d(kdst + off, &p.tmap_k, c2 * 64, row, head0, &full[stage], policy);
+                        tma_load_3d(vdst + off, &p.tmap_v, c2 * 64, row, head0, &full[stage], policy);
+                    }
+                }
+            } else if (contiguous) {
                 // one copy per block piece: rows of all KV heads are contiguous in both places
                 const int np = (tok0 + ntok - 1) / p.bs - jb0 + 1;
                 const int j = jb0 + lane;
@@ -853,9 +918,15 @@ __device__ __forceinline__ void merge_vr(const DecodeParams &p, const Seg &s, in
     const int warp = tid >> 5, lane = tid & 31;
     const size_t out_head0 = (size_t)s.b * p.Hq + (size_t)s.hg * NH;
     if (nparts <= kMergeParts) {
-        // weights w[i][h] = exp2(m_i - M_h) and 1 / sum_i w l into shared memory
-        float *w = msm;                    // [nparts][NH]
-        float *inv_den = msm + kMergeParts * NH;
+        // slots of the pieces (once), then w[i][h] = exp2(m_i - M_h) and 1 / sum_i w l
+        int64_t *slot_s = reinterpret_cast<int64_t *>(msm);  // [kMergeParts]
+        float *w = msm + 2 * kMergeParts;                      // [nparts][NH]
+        float *inv_den = w + kMergeParts * NH;
+        for (int i = tid; i < nparts; i += NTH) {
+            const int64_t slot = piece_slot(p, s, i, NT, C);
+            slot_s[i] = slot < p.max_slots ? slot : -1;
+        }
+        named_barrier(1, NTH);
         for (int h = warp; h < NH; h += kConsumerWarps) {
             float mi[2], li[2];
             float M = -INFINITY;
@@ -864,13 +935,11 @@ __device__ __forceinline__ void merge_vr(const DecodeParams &p, const Seg &s, in
                 const int i = lane + 32 * k;
                 mi[k] = -INFINITY;
                 li[k] = 0.f;
-                if (i < nparts) {
-                    const int64_t slot = piece_slot(p, s, i, NT, C);
-                    if (slot < p.max_slots) {
-                        const float *base = p.partials + slot * p.slot_floats;
-                        mi[k] = __ldcg(base + NH * D + h);
-                        li[k] = __ldcg(base + NH * D + NH + h);
-                    }
+                const int64_t slot = i < nparts ? slot_s[i] : -1;
+                if (slot >= 0) {
+                    const float *base = p.partials + slot * p.slot_floats;
+                    mi[k] = __ldcg(base + NH * D + h);
+                    li[k] = __ldcg(base + NH * D + NH + h);
                 }
                 M = fmaxf(M, mi[k]);
             }
@@ -894,37 +963,23 @@ __device__ __forceinline__ void merge_vr(const DecodeParams &p, const Seg &s, in
             const int h = idx / (D / 4);
             const int d4 = idx % (D / 4);
             float4 num = make_float4(0.f, 0.f, 0.f, 0.f);
-            int i = 0;
-            for (; i + 4 <= nparts; i += 4) {
-                float4 o[4];
-                float wi[4];
+            for (int i0 = 0; i0 < nparts; i0 += 8) {
+                float4 o[8];
 #pragma unroll
-                for (int k = 0; k < 4; ++k) {
-                    const int64_t slot = piece_slot(p, s, i + k, NT, C);
-                    const bool okk = slot < p.max_slots;
-                    o[k] = okk ? __ldcg(reinterpret_cast<const float4 *>(p.partials + slot * p.slot_floats +
-                                                                           (size_t)h * D) + d4)
-                               : make_float4(0.f, 0.f, 0.f, 0.f);
-                    wi[k] = w[(i + k) * NH + h];
+                for (int k = 0; k < 8; ++k) {  // eight loads in flight
+                    const int64_t slot = (i0 + k < nparts) ? slot_s[i0 + k] : -1;
+                    o[k] = slot >= 0 ? __ldcg(reinterpret_cast<const float4 *>(p.partials + slot * p.slot_floats +
+                                                                                (size_t)h * D) + d4)
+                                     : make_float4(0.f, 0.f, 0.f, 0.f);
                 }
 #pragma unroll
-                for (int k = 0; k < 4; ++k) {
-                    num.x += wi[k] * o[k].x;
-                    num.y += wi[k] * o[k].y;
-                    num.z += wi[k] * o[k].z;
-                    num.w += wi[k] * o[k].w;
+                for (int k = 0; k < 8; ++k) {
+                    const float wi = (i0 + k < nparts) ? w[(i0 + k) * NH + h] : 0.f;
+                    num.x += wi * o[k].x;
+                    num.y += wi * o[k].y;
+                    num.z += wi * o[k].z;
+                    num.w += wi * o[k].w;
                 }
-            }
-            for (; i < nparts; ++i) {
-                const int64_t slot = piece_slot(p, s, i, NT, C);
-                if (slot >= p.max_slots) continue;
-                const float4 o =
-                    __ldcg(reinterpret_cast<const float4 *>(p.partials + slot * p.slot_floats + (size_t)h * D) + d4);
-                const float wi = w[i * NH + h];
-                num.x += wi * o.x;
-                num.y += wi * o.y;
-                num.z += wi * o.z;
-                num.w += wi * o.w;
             }
             const float inv = inv_den[h];
             unsigned char *dst =
@@ -932,7 +987,7 @@ __device__ __forceinline__ void merge_vr(const DecodeParams &p, const Seg &s, in
             Elem<T>::store2(dst, num.x * inv, num.y * inv);
             Elem<T>::store2(dst + 2 * E, num.z * inv, num.w * inv);
         }
-        named_barrier(1, NTH);  // the weights area is free again
+        named_barrier(1, NTH);  // the shared area is free again
         return;
     }
     // many pieces (fixed partitions of a very long context): direct two-pass form
@@ -968,11 +1023,14 @@ __device__ __forceinline__ void merge_vr(const DecodeParams &p, const Seg &s, in
 
 // ===========================================================================
 template <typename T, int D, class Engine>
-__global__ void __launch_bounds__(kDecodeThreads, 1) paged_decode_kernel(const DecodeParams p) {
+__global__ void __launch_bounds__(kDecodeThreads, 1) paged_decode_kernel(const __grid_constant__ DecodeParams p) {
     constexpr int E = Elem<T>::kBytes;
     constexpr int UPW = Engine::kUnitsPerWarp;
-    extern __shared__ __align__(128) unsigned char smem[];
+    extern __shared__ __align__(1024) unsigned char smem_raw[];
     __shared__ DecodeCtl ctl;
+    __shared__ int lens_s[kLensCache];
+    // swizzled tensor-map boxes need 1024-byte aligned destinations
+    unsigned char *smem = smem_raw + ((1024u - (smem_u32(smem_raw) & 1023u)) & 1023u);
 
     const int tid = threadIdx.x;
     const int warp = tid >> 5;
@@ -1005,7 +1063,9 @@ __global__ void __launch_bounds__(kDecodeThreads, 1) paged_decode_kernel(const D
     for (int b = tid; b < p.B; b += kDecodeThreads) {
         const int raw = p.context_lens[b];
         if (blockIdx.x == 0 && (raw < 0 || raw > p.max_blocks * p.bs)) set_error(p.error, PA_DEVERR_CONTEXT_LEN);
-        local += units_of_len(p, clamped_len(p, b));
+        if (p.lens_cached) lens_s[b] = raw;
+        const int cap = p.max_blocks * p.bs;
+        local += units_of_len(p, raw < 0 ? 0 : (raw > cap ? cap : raw));
     }
 #pragma unroll
     for (int m = 16; m >= 1; m >>= 1) local += __shfl_xor_sync(0xffffffffu, local, m);
@@ -1027,7 +1087,7 @@ __global__ void __launch_bounds__(kDecodeThreads, 1) paged_decode_kernel(const D
         int64_t running = 0;
         for (int base = 0; base < p.B; base += kDecodeThreads) {
             const int b = base + tid;
-            const int64_t u = (b < p.B) ? (int64_t)p.NHG * units_of_len(p, clamped_len(p, b)) : 0;
+            const int64_t u = (b < p.B) ? (int64_t)p.NHG * units_of_len(p, clamped_len(p, lens_s, b)) : 0;
             int64_t x = u;
 #pragma unroll
             for (int m = 1; m < 32; m <<= 1) {
@@ -1060,9 +1120,10 @@ __global__ void __launch_bounds__(kDecodeThreads, 1) paged_decode_kernel(const D
     it.lo = lo;
     it.NT = NT;
     it.C = Cn;
+    it.lens_s = lens_s;
     if (lo < hi) {
         it.b = (int)ctl.found_b;
-        it.L = clamped_len(p, it.b);
+        it.L = clamped_len(p, lens_s, it.b);
         it.units = units_of_len(p, it.L);
         it.hg = (int)((lo - ctl.found_excl) / it.units);
         it.vr_start = ctl.found_excl + (int64_t)it.hg * it.units;
@@ -1082,7 +1143,7 @@ __global__ void __launch_bounds__(kDecodeThreads, 1) paged_decode_kernel(const D
     // ================= consumer warps =================
     // requests with no tokens: out = 0
     for (int b = blockIdx.x; b < p.B; b += p.num_ctas) {
-        if (clamped_len(p, b) != 0) continue;
+        if (clamped_len(p, lens_s, b) != 0) continue;
         unsigned char *o = reinterpret_cast<unsigned char *>(p.out) + (size_t)b * p.Hq * D * E;
         for (int i = tid; i < p.Hq * D / 8; i += kConsumerWarps * 32) Elem<T>::store_zero8(o + (size_t)i * 8 * E);
     }
@@ -1141,9 +1202,7 @@ __global__ void __launch_bounds__(kDecodeThreads, 1) paged_decode_kernel(const D
                     const int nvalid = min(kSubTile, ntok - st * kSubTile);
 #pragma unroll
                     for (int k = 0; k < UPW; ++k)
-                        eng.subtile(unit[k], kst + (size_t)st * kSubTile * p.row_pitch,
-                                    vst + (size_t)st * kSubTile * p.row_pitch, u_g[k], nvalid, p.row_pitch, s_sm,
-                                    p_sm, lane);
+                        eng.subtile(unit[k], kst, vst, st, u_g[k], nvalid, p, s_sm, p_sm, lane);
                 }
             }
             __syncwarp();

@@ -1,5 +1,7 @@
 // C ABI of libpagedattn: argument validation, the host-side planner and
 // kernel dispatch.  Declarations and contracts live in include/pagedattn.h.
+#include <cudaTypedefs.h>
+
 #include <cmath>
 #include <cstdarg>
 #include <cstdio>
@@ -31,7 +33,8 @@ bool pow2(int x) { return x > 0 && (x & (x - 1)) == 0; }
 int elem_bytes(int dtype) { return dtype == PA_DTYPE_F32 ? 4 : 2; }
 size_t round_up(size_t x, size_t a) { return (x + a - 1) / a * a; }
 
-constexpr int kSmemLimit = 232448;     // opt-in dynamic shared memory per CTA on sm_100
+constexpr int kSmemLimit = 232448;     // opt-in shared memory per CTA on sm_100 (static + dynamic)
+constexpr int kStaticSmem = 4096 + 256;  // lengths cache and control block
 constexpr size_t kWsHeader = 256;      // error word + reserved
 constexpr int kStageTargetBytes = 32768;  // K bytes per stage (V the same)
 constexpr int kMaxStages = 4;
@@ -114,7 +117,7 @@ Layout smem_layout(int dtype, int D, int stages, uint32_t q_bytes, uint32_t half
     l.off_bar = 0;
     const uint32_t bar_bytes = (uint32_t)round_up((2 * stages + 4) * 8, 128);
     l.off_q = bar_bytes;
-    l.off_stage = (uint32_t)round_up(l.off_q + 2 * q_bytes, 128);
+    l.off_stage = (uint32_t)round_up(l.off_q + 2 * q_bytes, 1024);
     l.off_scratch = (uint32_t)round_up(l.off_stage + (size_t)stages * 2 * half_bytes, 128);
     const uint32_t scratch = mma ? 0u : (uint32_t)(pa::kConsumerWarps * 2 * pa::kSubTile * hc * 4);
     l.off_comb = (uint32_t)round_up(l.off_scratch + scratch, 128);
@@ -123,7 +126,8 @@ Layout smem_layout(int dtype, int D, int stages, uint32_t q_bytes, uint32_t half
     const uint32_t comb = tsplit > 1 ? pa::kConsumerWarps * l.comb_stride : 0;
     l.off_merge = (uint32_t)round_up(l.off_comb + comb, 128);
     const uint32_t merge = (uint32_t)(2 * pa::kMergeParts + pa::kMergeParts * nhvr + nhvr) * 4;
-    l.total = (uint32_t)round_up(l.off_merge + merge, 128);
+    // + 1024: the kernel rounds its dynamic base up to a 1024-byte boundary
+    l.total = (uint32_t)round_up(l.off_merge + merge, 128) + 1024;
     return l;
 }
 
@@ -196,8 +200,42 @@ bool choose_mapping(const pa_shape *s, Mapping &m) {
     return false;
 }
 
-uint32_t row_pitch_of(const pa_shape *s, uint32_t row_bytes) {
-    return s->dtype == PA_DTYPE_BF16 ? row_bytes + 16 : row_bytes;  // padded rows for ldmatrix
+uint32_t row_pitch_of(const pa_shape *, uint32_t row_bytes) { return row_bytes; }
+
+// cuTensorMapEncodeTiled through the runtime's driver entry point (no libcuda link)
+PFN_cuTensorMapEncodeTiled encode_fn() {
+    static PFN_cuTensorMapEncodeTiled fn = nullptr;
+    static std::once_flag once;
+    std::call_once(once, [] {
+        void *f = nullptr;
+        cudaDriverEntryPointQueryResult q;
+        if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &f, cudaEnableDefault, &q) == cudaSuccess &&
+            q == cudaDriverEntryPointSuccess)
+            fn = reinterpret_cast<PFN_cuTensorMapEncodeTiled>(f);
+    });
+    return fn;
+}
+
+// [d, token row, head] view of a bf16 pool [num_blocks, bs, Hkv, D]; the box
+// {64, br, HG} lands head-major ([head][row][64]) with the 128-byte swizzle.
+pa_status encode_pool_map(CUtensorMap *map, const void *pool, const pa_shape *s, int br, int hg) {
+    PFN_cuTensorMapEncodeTiled enc = encode_fn();
+    if (!enc) return fail(PA_ERR_CUDA, "cuTensorMapEncodeTiled is not available");
+    cuuint64_t dims[3] = {(cuuint64_t)s->D, (cuuint64_t)s->num_blocks * (cuuint64_t)s->block_size, (cuuint64_t)s->Hkv};
+    cuuint64_t strides[2] = {(cuuint64_t)s->Hkv * s->D * 2, (cuuint64_t)s->D * 2};
+    cuuint32_t box[3] = {64, (cuuint32_t)br, (cuuint32_t)hg};
+    cuuint32_t estr[3] = {1, 1, 1};
+    CUresult r = enc(map, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3, const_cast<void *>(pool), dims, strides, box, estr,
+                     CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+                     CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+    if (r != CUDA_SUCCESS) return fail(PA_ERR_CUDA, "cuTensorMapEncodeTiled failed (%d)", (int)r);
+    return PA_OK;
+}
+
+int log2i(int x) {
+    int l = 0;
+    while ((1 << l) < x) ++l;
+    return l;
 }
 
 pa_status launch_decode(const void *q, const void *k_cache, const void *v_cache, const int32_t *block_tables,
@@ -277,6 +315,15 @@ pa_status launch_decode(const void *q, const void *k_cache, const void *v_cache,
     p.half_bytes = half;
     p.q_bytes = q_bytes;
     p.comb_stride = lay.comb_stride;
+    p.bs_log2 = log2i(s->block_size);
+    p.lens_cached = s->B <= pa::kLensCache ? 1 : 0;
+    if (s->dtype == PA_DTYPE_BF16) {
+        const int br = plan->tile_tokens < s->block_size ? plan->tile_tokens : s->block_size;
+        p.use_tmap = 1;
+        p.br_log2 = log2i(br);
+        if (pa_status st = encode_pool_map(&p.tmap_k, k_cache, s, br, HG)) return st;
+        if (pa_status st = encode_pool_map(&p.tmap_v, v_cache, s, br, HG)) return st;
+    }
 
     if (pa_status st = ensure_smem_attr(fn, plan->smem_bytes)) return st;
     cudaLaunchConfig_t cfg = {};
@@ -371,7 +418,7 @@ pa_status pa_plan(const pa_shape *s, int32_t max_context_len, int32_t partition_
         const uint32_t half = (uint32_t)ST * pitch;
         for (stages = kMaxStages; stages >= 2; --stages) {
             lay = smem_layout(s->dtype, s->D, stages, q_bytes, half, HC, TS, NHvr);
-            if (lay.total + 256 <= (uint32_t)kSmemLimit) break;
+            if (lay.total + kStaticSmem <= (uint32_t)kSmemLimit) break;
         }
         if (stages >= 2) break;
         if (ST == 16) return fail(PA_ERR_UNSUPPORTED, "shared memory too small for this shape");
