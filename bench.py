@@ -183,8 +183,12 @@ def main():
 
     import synth
     from synth import algorithmic_bytes
-    from paged_kv_cache_472_b200 import build as libbuild
-    libbuild.build()
+    import importlib.util
+    spec = importlib.util.spec_from_file_location(
+        "_pagedattn_build", os.path.join(ROOT, "paged_kv_cache_472_b200", "build.py"))
+    libbuild = importlib.util.module_from_spec(spec)
+    spec.loader.exec_module(libbuild)
+    libbuild.build()   # before the package import loads the library
     import paged_kv_cache_472_b200 as pa
     from paged_kv_cache_472_b200.session import PagedDecoder
     from tests import gpu_harness as H

@@ -7,9 +7,9 @@ import re
 
 import pytest
 
-from paged_kv_cache_472_b200 import build as _build
+import __graft_entry__
 
-_build.build()
+__graft_entry__.build()
 import paged_kv_cache_472_b200 as pa  # noqa: E402
 import synth  # noqa: E402
 
