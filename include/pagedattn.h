@@ -180,6 +180,27 @@ pa_status pa_kv_append_decode(const void *k_new, const void *v_new, const int32_
                               const int32_t *context_lens, float scale, void *out, const pa_shape *s,
                               const pa_plan_t *plan, void *workspace, size_t workspace_bytes, void *stream);
 
+/*
+ * pa_decode for callers that cannot allocate device memory: a caller whose
+ * host framework owns every device allocation and gives it none, or code
+ * that runs where cudaMalloc is not allowed.  It takes no workspace; it uses
+ * a 16 MiB array compiled into the library instead (every GPU that loads
+ * the library holds it until the process exits).  There is no counterpart
+ * of this call in the pages: it only changes where the scratch lives.
+ *   Arguments as in pa_decode, minus workspace and workspace_bytes.
+ *   plan->workspace_bytes above 16 MiB returns PA_ERR_WORKSPACE.
+ *   Allocates nothing: no cudaMalloc, no cudaFree, no allocating library call.
+ *   The first call on a device looks up the array's device address for that
+ *   device (with it current); make that first call before any stream capture.
+ *   Every call clears the array's error word and merge counters first (one
+ *   cudaMemsetAsync on `stream`), so index errors recorded by one call are
+ *   gone at the next and cannot be read back through this entry point.
+ *   All calls share the one array: two calls that overlap on the GPU race.
+ */
+pa_status pa_decode_no_alloc(const void *q, const void *k_cache, const void *v_cache, const int32_t *block_tables,
+                             const int32_t *context_lens, float scale, void *out, const pa_shape *s,
+                             const pa_plan_t *plan, void *stream);
+
 /* Copy the device error word of `workspace` to *err_out (synchronises
  * `stream`; not for the hot path).  clear != 0 resets it to 0 afterwards. */
 pa_status pa_get_device_error(void *workspace, int32_t clear, int32_t *err_out, void *stream);

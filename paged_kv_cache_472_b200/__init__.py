@@ -17,7 +17,7 @@ __all__ = ["PagedAttnError", "Shape", "Plan", "DTYPE_F32", "DTYPE_BF16", "SPLIT_
            "DEVERR_BLOCK_ID", "DEVERR_CONTEXT_LEN", "DEVERR_TIMEOUT", "DEVERR_WORKSPACE", "DEVERR_SLOT",
            "pa_version", "pa_status_str", "pa_last_error_message", "pa_kv_append", "pa_plan",
            "pa_decode_workspace_size", "pa_workspace_init", "pa_decode", "pa_kv_append_decode", "pa_get_device_error",
-           "lib"]
+           "pa_decode_no_alloc", "lib"]
 
 PA_OK, PA_ERR_INVALID_ARG, PA_ERR_UNSUPPORTED, PA_ERR_CUDA, PA_ERR_WORKSPACE = range(5)
 DTYPE_F32, DTYPE_BF16 = 0, 1
@@ -73,8 +73,9 @@ lib.pa_decode.argtypes = [_vp, _vp, _vp, _vp, _vp, ctypes.c_float, _vp, _P(Shape
 lib.pa_get_device_error.argtypes = [_vp, _i32, _P(_i32), _vp]
 lib.pa_kv_append_decode.argtypes = [_vp, _vp, _vp, _vp, _vp, _vp, _vp, _vp, ctypes.c_float, _vp, _P(Shape), _P(Plan),
                                     _vp, _sz, _vp]
+lib.pa_decode_no_alloc.argtypes = [_vp, _vp, _vp, _vp, _vp, ctypes.c_float, _vp, _P(Shape), _P(Plan), _vp]
 for _f in ("pa_kv_append", "pa_plan", "pa_workspace_init", "pa_decode", "pa_get_device_error",
-           "pa_kv_append_decode"):
+           "pa_kv_append_decode", "pa_decode_no_alloc"):
     getattr(lib, _f).restype = ctypes.c_int
 
 
@@ -145,6 +146,13 @@ def pa_kv_append_decode(k_new, v_new, slot_mapping, q, k_cache, v_cache, block_t
                                    _ptr(v_cache), _ptr(block_tables), _ptr(context_lens), float(scale), _ptr(out),
                                    ctypes.byref(shape), ctypes.byref(plan), _ptr(workspace), int(workspace_bytes),
                                    _stream(stream)), "pa_kv_append_decode")
+
+
+def pa_decode_no_alloc(q, k_cache, v_cache, block_tables, context_lens, scale: float, out, shape: Shape, plan: Plan,
+                       stream=None):
+    _check(lib.pa_decode_no_alloc(_ptr(q), _ptr(k_cache), _ptr(v_cache), _ptr(block_tables), _ptr(context_lens),
+                                  float(scale), _ptr(out), ctypes.byref(shape), ctypes.byref(plan), _stream(stream)),
+           "pa_decode_no_alloc")
 
 
 def pa_get_device_error(workspace, clear: bool = False, stream=None) -> int:

@@ -501,3 +501,57 @@ pa_status pa_get_device_error(void *workspace, int32_t clear, int32_t *err_out, 
 }
 
 }  // extern "C"
+
+// ---------------------------------------------------------------------------
+// Decode for callers that cannot allocate device memory: the workspace is a
+// fixed array compiled into this library instead of caller-provided memory.
+static constexpr size_t kNoAllocWorkspaceBytes = 16u << 20;  // 16 MiB, held by every GPU that loads the library
+static __device__ __align__(256) unsigned char g_no_alloc_workspace[kNoAllocWorkspaceBytes];
+
+namespace {
+constexpr int kNoAllocMaxDevices = 64;
+std::mutex g_no_alloc_mu;
+void *g_no_alloc_ptr[kNoAllocMaxDevices] = {};
+
+// Device address of the array on the current device.  The host-side name
+// g_no_alloc_workspace is only a stand-in, so the address is looked up once
+// per device (with that device current) and remembered.
+pa_status no_alloc_workspace(void **out) {
+    int dev = 0;
+    cudaError_t e = cudaGetDevice(&dev);
+    if (e != cudaSuccess) return fail(PA_ERR_CUDA, "cudaGetDevice: %s", cudaGetErrorString(e));
+    if (dev < 0 || dev >= kNoAllocMaxDevices) return fail(PA_ERR_UNSUPPORTED, "device ordinal %d", dev);
+    std::lock_guard<std::mutex> lk(g_no_alloc_mu);
+    if (!g_no_alloc_ptr[dev]) {
+        void *ptr = nullptr;
+        e = cudaGetSymbolAddress(&ptr, g_no_alloc_workspace);
+        if (e != cudaSuccess) return fail(PA_ERR_CUDA, "cudaGetSymbolAddress: %s", cudaGetErrorString(e));
+        g_no_alloc_ptr[dev] = ptr;
+    }
+    *out = g_no_alloc_ptr[dev];
+    return PA_OK;
+}
+}  // namespace
+
+extern "C" pa_status pa_decode_no_alloc(const void *q, const void *k_cache, const void *v_cache,
+                                        const int32_t *block_tables, const int32_t *context_lens, float scale,
+                                        void *out, const pa_shape *s, const pa_plan_t *plan, void *stream) {
+    if (pa_status st = check_shape(s)) return st;
+    if (!plan) return fail(PA_ERR_INVALID_ARG, "plan is NULL");
+    if (plan->workspace_bytes > kNoAllocWorkspaceBytes)
+        return fail(PA_ERR_WORKSPACE, "this plan needs %zu workspace bytes; the built-in workspace holds %zu",
+                    plan->workspace_bytes, kNoAllocWorkspaceBytes);
+    if (s->B == 0) return ok();
+    void *ws = nullptr;
+    if (pa_status st = no_alloc_workspace(&ws)) return st;
+    // the array keeps the previous call's contents: the error word and the
+    // merge counters must start at zero
+    const size_t counters = round_up((size_t)s->B * (s->Hkv / (plan->head_group > 0 ? plan->head_group : 1)) * 4, 256);
+    cudaError_t e = cudaMemsetAsync(ws, 0, kWsHeader + counters, (cudaStream_t)stream);
+    if (e != cudaSuccess) return fail(PA_ERR_CUDA, "cudaMemsetAsync: %s", cudaGetErrorString(e));
+    if (pa_status st = launch_decode(q, k_cache, v_cache, block_tables, context_lens, scale, out, s, plan, ws,
+                                     kNoAllocWorkspaceBytes, (cudaStream_t)stream, false))
+        return st;
+    return ok();
+}
+
