@@ -131,6 +131,27 @@ class ClockSampler:
 
 
 # ---------------------------------------------------------------------------
+# multi-rank host logic (replicas: each rank decodes its own batch, no exchange)
+def rank_seed(cid: int, rank: int):
+    """Seed of rank `rank`'s batch: rank 0 runs the workload's own seed."""
+    return None if rank == 0 else 1000 + cid + 7919 * rank
+
+
+def max_over_ranks(value: float, world: int, device) -> float:
+    import torch
+    t = torch.tensor([value], dtype=torch.float64, device=device)
+    if world > 1:
+        import torch.distributed as dist
+        dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return float(t.item())
+
+
+def job_throughput_gbs(step_bytes: int, world: int, ms_step: float) -> float:
+    """Whole-job GB/s: every rank moved step_bytes per step."""
+    return world * step_bytes / (ms_step * 1e-3) / 1e9
+
+
+# ---------------------------------------------------------------------------
 def cpu_baseline(case, seconds: float):
     """The float64 oracle as it stands (append + decode of the whole batch),
     repeated for about `seconds` on the host cores."""
@@ -202,7 +223,7 @@ def main():
         dist.init_process_group("nccl", timeout=timedelta(seconds=120))
 
     # each rank decodes its own batch of the workload (distinct seed per rank)
-    base_case = synth.make_config(args.config, seed=None if rank == 0 else 1000 + args.config + 7919 * rank)
+    base_case = synth.make_config(args.config, seed=rank_seed(args.config, rank))
     pt = base_case.partition_tokens if args.partition < 0 else args.partition
     ab = algorithmic_bytes(base_case)
     step_bytes = ab["step_total"]
@@ -252,7 +273,7 @@ def main():
         torch.cuda.synchronize()
     if world > 1:
         dist.barrier()
-    ms_total = start.elapsed_time(end)
+    ms_total = max_over_ranks(start.elapsed_time(end), world, "cuda")
 
     # the decode kernel alone, CUDA events around every launch on its stream
     KD = max(min(K, 2000), 1)
@@ -264,10 +285,6 @@ def main():
         kev[i][1].record(stream)
     torch.cuda.synchronize()
     dec_ms = [a.elapsed_time(b) for a, b in kev]
-    t = torch.tensor([ms_total], device="cuda", dtype=torch.float64)
-    if world > 1:
-        dist.all_reduce(t, op=dist.ReduceOp.MAX)
-    ms_total = float(t.item())
     ms_step = ms_total / K
     err = dec.device_error()
     if err:
@@ -292,17 +309,13 @@ def main():
         host_out.copy_(c0.out, non_blocking=True)
     e1.record(stream)
     torch.cuda.synchronize()
-    e2e_ms = e0.elapsed_time(e1) / E
-    te = torch.tensor([e2e_ms], device="cuda", dtype=torch.float64)
-    if world > 1:
-        dist.all_reduce(te, op=dist.ReduceOp.MAX)
-    e2e_ms = float(te.item())
+    e2e_ms = max_over_ranks(e0.elapsed_time(e1) / E, world, "cuda")
 
     if rank == 0:
         peak, peak_kind = measured_peak()
         dec_avg_ms = sum(dec_ms) / len(dec_ms)
         achieved = decode_bytes / (dec_avg_ms * 1e-3) / 1e9
-        value = world * step_bytes / (ms_step * 1e-3) / 1e9
+        value = job_throughput_gbs(step_bytes, world, ms_step)
         line = {
             "metric": "paged-decode attention HBM GB/s (% of B200 peak); us/decode step",
             "value": round(value, 2), "unit": "GB/s", "n_gpus": world, "steps": K, "warmup": args.warmup,
@@ -322,7 +335,7 @@ def main():
                          "kernel": "paged_decode_kernel", "peak_kind": peak_kind,
                          "decode_us": round(dec_avg_ms * 1e3, 3), "decode_launches_timed": KD,
                          "engine": "tensor-core mma" if base_case.dtype == "bf16" else "cuda-core fp32"},
-            "e2e": {"value": round(world * step_bytes / (e2e_ms * 1e-3) / 1e9, 2), "unit": "GB/s",
+            "e2e": {"value": round(job_throughput_gbs(step_bytes, world, e2e_ms), 2), "unit": "GB/s",
                     "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h, "us_per_step": round(e2e_ms * 1e3, 3)},
             "gpu_launches": 2 * K,
             "clocks": clk.summary(),
