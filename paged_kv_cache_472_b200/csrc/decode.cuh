@@ -236,12 +236,16 @@ struct SegIter {
     }
 };
 
+constexpr int kMaxPending = 16;  // split pieces whose arrival a CTA counts at once
+
 struct __align__(16) DecodeCtl {
     int64_t red[kConsumerWarps + 1];
     int64_t total;
     int64_t found_b, found_excl;
     int abort;
     int merge_flag;
+    Seg pending[kMaxPending];   // pieces written to the workspace, arrival not yet counted
+    int last[kMaxPending];      // this CTA delivered the vr's last piece
 };
 
 // slot of piece i of a split vr
@@ -747,6 +751,10 @@ template <int D, int E>
 __device__ __forceinline__ void run_producer(const DecodeParams &p, SegIter it, uint64_t *full, uint64_t *empty,
                                              uint64_t *qfull, uint64_t *qempty, unsigned char *qarea,
                                              unsigned char *stage_base, volatile int *abort_flag, int lane) {
+    if (p.use_tmap && lane == 0) {
+        prefetch_tensormap(&p.tmap_k);
+        prefetch_tensormap(&p.tmap_v);
+    }
     const uint64_t policy = policy_evict_first();
     const unsigned char *kc = reinterpret_cast<const unsigned char *>(p.k_cache);
     const unsigned char *vc = reinterpret_cast<const unsigned char *>(p.v_cache);
@@ -906,119 +914,126 @@ __device__ __forceinline__ void run_producer(const DecodeParams &p, SegIter it, 
 
 // ===========================================================================
 // merge of a split vr by log-sum-exp (run by the consumer warps of the CTA
-// that delivered the last piece)
+// that delivered the last piece).  One pass per output element keeps a
+// running maximum, so any number of pieces is combined with eight pieces'
+// loads (o, m, l) in flight at a time.
 // ===========================================================================
 template <typename T, int D>
 __device__ __forceinline__ void merge_vr(const DecodeParams &p, const Seg &s, int64_t NT, int64_t C, float *msm,
                                          int tid) {
     constexpr int E = Elem<T>::kBytes;
     constexpr int NTH = kConsumerWarps * 32;
+    constexpr int KF = 8;  // pieces per batch of loads
     const int NH = p.NHvr;
     const int nparts = s.nparts;
-    const int warp = tid >> 5, lane = tid & 31;
     const size_t out_head0 = (size_t)s.b * p.Hq + (size_t)s.hg * NH;
-    if (nparts <= kMergeParts) {
-        // slots of the pieces (once), then w[i][h] = exp2(m_i - M_h) and 1 / sum_i w l
-        int64_t *slot_s = reinterpret_cast<int64_t *>(msm);  // [kMergeParts]
-        float *w = msm + 2 * kMergeParts;                      // [nparts][NH]
-        float *inv_den = w + kMergeParts * NH;
+    int64_t *slot_s = reinterpret_cast<int64_t *>(msm);  // [kMergeParts]
+    const bool cached = nparts <= kMergeParts;
+    if (cached) {
         for (int i = tid; i < nparts; i += NTH) {
             const int64_t slot = piece_slot(p, s, i, NT, C);
             slot_s[i] = slot < p.max_slots ? slot : -1;
         }
         named_barrier(1, NTH);
-        for (int h = warp; h < NH; h += kConsumerWarps) {
-            float mi[2], li[2];
-            float M = -INFINITY;
-#pragma unroll
-            for (int k = 0; k < 2; ++k) {
-                const int i = lane + 32 * k;
-                mi[k] = -INFINITY;
-                li[k] = 0.f;
-                const int64_t slot = i < nparts ? slot_s[i] : -1;
-                if (slot >= 0) {
-                    const float *base = p.partials + slot * p.slot_floats;
-                    mi[k] = __ldcg(base + NH * D + h);
-                    li[k] = __ldcg(base + NH * D + NH + h);
-                }
-                M = fmaxf(M, mi[k]);
-            }
-#pragma unroll
-            for (int m = 16; m >= 1; m >>= 1) M = fmaxf(M, __shfl_xor_sync(0xffffffffu, M, m));
-            float den = 0.f;
-#pragma unroll
-            for (int k = 0; k < 2; ++k) {
-                const int i = lane + 32 * k;
-                const float wi = (mi[k] == -INFINITY) ? 0.f : exp2f(mi[k] - M);
-                den += wi * li[k];
-                if (i < nparts) w[i * NH + h] = wi;
-            }
-#pragma unroll
-            for (int m = 16; m >= 1; m >>= 1) den += __shfl_xor_sync(0xffffffffu, den, m);
-            if (lane == 0) inv_den[h] = 1.f / den;
-        }
-        named_barrier(1, NTH);
-        const int nq = NH * (D / 4);
-        for (int idx = tid; idx < nq; idx += NTH) {
-            const int h = idx / (D / 4);
-            const int d4 = idx % (D / 4);
-            float4 num = make_float4(0.f, 0.f, 0.f, 0.f);
-            for (int i0 = 0; i0 < nparts; i0 += 8) {
-                float4 o[8];
-#pragma unroll
-                for (int k = 0; k < 8; ++k) {  // eight loads in flight
-                    const int64_t slot = (i0 + k < nparts) ? slot_s[i0 + k] : -1;
-                    o[k] = slot >= 0 ? __ldcg(reinterpret_cast<const float4 *>(p.partials + slot * p.slot_floats +
-                                                                                (size_t)h * D) + d4)
-                                     : make_float4(0.f, 0.f, 0.f, 0.f);
-                }
-#pragma unroll
-                for (int k = 0; k < 8; ++k) {
-                    const float wi = (i0 + k < nparts) ? w[(i0 + k) * NH + h] : 0.f;
-                    num.x += wi * o[k].x;
-                    num.y += wi * o[k].y;
-                    num.z += wi * o[k].z;
-                    num.w += wi * o[k].w;
-                }
-            }
-            const float inv = inv_den[h];
-            unsigned char *dst =
-                reinterpret_cast<unsigned char *>(p.out) + ((out_head0 + h) * D + d4 * 4) * E;
-            Elem<T>::store2(dst, num.x * inv, num.y * inv);
-            Elem<T>::store2(dst + 2 * E, num.z * inv, num.w * inv);
-        }
-        named_barrier(1, NTH);  // the shared area is free again
-        return;
     }
-    // many pieces (fixed partitions of a very long context): direct two-pass form
     const int nq = NH * (D / 4);
-    for (int idx = tid; idx < nq; idx += NTH) {
-        const int h = idx / (D / 4);
-        const int d4 = idx % (D / 4);
-        float M = -INFINITY;
-        for (int i = 0; i < nparts; ++i) {
-            const int64_t slot = piece_slot(p, s, i, NT, C);
-            if (slot < p.max_slots) M = fmaxf(M, __ldcg(p.partials + slot * p.slot_floats + NH * D + h));
+    for (int idx0 = tid; idx0 < nq; idx0 += 2 * NTH) {
+        constexpr int IT = 2;  // output items per thread per batch
+        int hh[IT], dd[IT];
+        bool act[IT];
+        float M[IT], den[IT];
+        float4 num[IT];
+#pragma unroll
+        for (int j = 0; j < IT; ++j) {
+            const int idx = idx0 + j * NTH;
+            act[j] = idx < nq;
+            hh[j] = act[j] ? idx / (D / 4) : 0;
+            dd[j] = act[j] ? idx % (D / 4) : 0;
+            M[j] = -INFINITY;
+            den[j] = 0.f;
+            num[j] = make_float4(0.f, 0.f, 0.f, 0.f);
         }
-        float4 num = make_float4(0.f, 0.f, 0.f, 0.f);
-        float den = 0.f;
-        for (int i = 0; i < nparts; ++i) {
-            const int64_t slot = piece_slot(p, s, i, NT, C);
-            if (slot >= p.max_slots) continue;
-            const float *base = p.partials + slot * p.slot_floats;
-            const float wi = exp2f(__ldcg(base + NH * D + h) - M);
-            den += wi * __ldcg(base + NH * D + NH + h);
-            const float4 o = __ldcg(reinterpret_cast<const float4 *>(base + (size_t)h * D) + d4);
-            num.x += wi * o.x;
-            num.y += wi * o.y;
-            num.z += wi * o.z;
-            num.w += wi * o.w;
+        for (int i0 = 0; i0 < nparts; i0 += KF) {
+            int64_t sl[KF];
+#pragma unroll
+            for (int k = 0; k < KF; ++k) {
+                const int i = i0 + k;
+                int64_t slot = -1;
+                if (i < nparts) {
+                    slot = cached ? slot_s[i] : piece_slot(p, s, i, NT, C);
+                    if (slot >= p.max_slots) slot = -1;
+                }
+                sl[k] = slot;
+            }
+            float4 o[IT][KF];
+            float mi[IT][KF], li[IT][KF];
+#pragma unroll
+            for (int j = 0; j < IT; ++j)
+#pragma unroll
+                for (int k = 0; k < KF; ++k) {
+                    if (act[j] && sl[k] >= 0) {
+                        const float *base = p.partials + sl[k] * p.slot_floats;
+                        o[j][k] = __ldcg(reinterpret_cast<const float4 *>(base + (size_t)hh[j] * D) + dd[j]);
+                        mi[j][k] = __ldcg(base + NH * D + hh[j]);
+                        li[j][k] = __ldcg(base + NH * D + NH + hh[j]);
+                    } else {
+                        o[j][k] = make_float4(0.f, 0.f, 0.f, 0.f);
+                        mi[j][k] = -INFINITY;
+                        li[j][k] = 0.f;
+                    }
+                }
+#pragma unroll
+            for (int j = 0; j < IT; ++j) {
+                float cm = M[j];
+#pragma unroll
+                for (int k = 0; k < KF; ++k) cm = fmaxf(cm, mi[j][k]);
+                if (cm == -INFINITY) continue;
+                const float a = exp2f(M[j] - cm);  // M = -inf before the first piece: 0
+                num[j].x *= a;
+                num[j].y *= a;
+                num[j].z *= a;
+                num[j].w *= a;
+                den[j] *= a;
+#pragma unroll
+                for (int k = 0; k < KF; ++k) {
+                    const float w = exp2f(mi[j][k] - cm);  // missing pieces: exp2(-inf) = 0
+                    den[j] += w * li[j][k];
+                    num[j].x += w * o[j][k].x;
+                    num[j].y += w * o[j][k].y;
+                    num[j].z += w * o[j][k].z;
+                    num[j].w += w * o[j][k].w;
+                }
+                M[j] = cm;
+            }
         }
-        const float inv = 1.f / den;
-        unsigned char *dst = reinterpret_cast<unsigned char *>(p.out) + ((out_head0 + h) * D + d4 * 4) * E;
-        Elem<T>::store2(dst, num.x * inv, num.y * inv);
-        Elem<T>::store2(dst + 2 * E, num.z * inv, num.w * inv);
+#pragma unroll
+        for (int j = 0; j < IT; ++j) {
+            if (!act[j]) continue;
+            const float inv = 1.f / den[j];
+            unsigned char *dst =
+                reinterpret_cast<unsigned char *>(p.out) + ((out_head0 + hh[j]) * D + dd[j] * 4) * E;
+            Elem<T>::store2(dst, num[j].x * inv, num[j].y * inv);
+            Elem<T>::store2(dst + 2 * E, num[j].z * inv, num[j].w * inv);
+        }
     }
+    if (cached) named_barrier(1, NTH);  // the slot list is free again
+}
+
+// Merge every vr for which this CTA delivered the last piece (arrivals were
+// already counted by thread 0 as the pieces were stored).
+template <typename T, int D>
+__device__ __forceinline__ void flush_pending(const DecodeParams &p, DecodeCtl &ctl, int npend, int64_t NT,
+                                              int64_t C, float *msm, int tid) {
+    constexpr int NTH = kConsumerWarps * 32;
+    named_barrier(1, NTH);
+    for (int k = 0; k < npend; ++k) {
+        if (!ctl.last[k]) continue;
+        __threadfence();
+        const Seg sk = ctl.pending[k];
+        merge_vr<T, D>(p, sk, NT, C, msm, tid);
+        if (tid == 0) p.counters[(int64_t)sk.b * p.NHG + sk.hg] = 0;
+    }
+    named_barrier(1, NTH);  // pending list free again
 }
 
 // ===========================================================================
@@ -1173,6 +1188,7 @@ __global__ void __launch_bounds__(kDecodeThreads, 1) paged_decode_kernel(const _
     uint32_t phase = 0;
     int qslot = 0;
     uint32_t qphase = 0;
+    int npend = 0;
     Seg s;
     while (it.next(p, s)) {
         // -- q of this vr --
@@ -1241,7 +1257,10 @@ __global__ void __launch_bounds__(kDecodeThreads, 1) paged_decode_kernel(const _
             continue;
         }
 
-        // partial piece: leave (m, l, o) in the slot, then count arrivals
+        // partial piece: leave (m, l, o) in the slot and count its arrival.
+        // Only thread 0 fences and bumps the counter (after a barrier, as a
+        // grid-wide sync does); the other warps go on with the next tile.  A
+        // vr whose last piece this was is merged when the CTA is done.
         const bool slot_ok = s.slot < p.max_slots;
         if (writer && slot_ok) {
             float *base = p.partials + s.slot * p.slot_floats;
@@ -1249,20 +1268,19 @@ __global__ void __launch_bounds__(kDecodeThreads, 1) paged_decode_kernel(const _
             for (int k = 0; k < UPW; ++k) eng.write_partial(unit[k], base, p.NHvr, u_h0[k]);
         }
         if (!slot_ok && tid == 0) set_error(p.error, PA_DEVERR_WORKSPACE);
-        __threadfence();
         named_barrier(1, kConsumerWarps * 32);
-        const int64_t vr = (int64_t)s.b * p.NHG + s.hg;
         if (tid == 0) {
-            const int prev = atomicAdd(&p.counters[vr], 1);
-            ctl.merge_flag = (prev == s.nparts - 1);
-        }
-        named_barrier(1, kConsumerWarps * 32);
-        if (ctl.merge_flag) {
             __threadfence();
-            merge_vr<T, D>(p, s, NT, Cn, msm, tid);
-            if (tid == 0) p.counters[vr] = 0;
+            const int prev = atomicAdd(&p.counters[(int64_t)s.b * p.NHG + s.hg], 1);
+            ctl.pending[npend] = s;
+            ctl.last[npend] = (prev == s.nparts - 1);
+        }
+        if (++npend == kMaxPending) {
+            flush_pending<T, D>(p, ctl, npend, NT, Cn, msm, tid);
+            npend = 0;
         }
     }
+    if (npend) flush_pending<T, D>(p, ctl, npend, NT, Cn, msm, tid);
 }
 
 }  // namespace pa

@@ -34,7 +34,7 @@ int elem_bytes(int dtype) { return dtype == PA_DTYPE_F32 ? 4 : 2; }
 size_t round_up(size_t x, size_t a) { return (x + a - 1) / a * a; }
 
 constexpr int kSmemLimit = 232448;     // opt-in shared memory per CTA on sm_100 (static + dynamic)
-constexpr int kStaticSmem = 4096 + 256;  // lengths cache and control block
+constexpr int kStaticSmem = 4096 + 1536;  // lengths cache and control block (pending list)
 constexpr size_t kWsHeader = 256;      // error word + reserved
 constexpr int kStageTargetBytes = 32768;  // K bytes per stage (V the same)
 constexpr int kMaxStages = 4;
