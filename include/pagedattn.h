@@ -50,7 +50,7 @@ typedef enum {
     PA_ERR_WORKSPACE = 4     /* workspace missing or smaller than the plan needs */
 } pa_status;
 
-typedef enum { PA_DTYPE_F32 = 0, PA_DTYPE_BF16 = 1 } pa_dtype;
+typedef enum { PA_DTYPE_F32 = 0, PA_DTYPE_BF16 = 1, PA_DTYPE_F16 = 2 } pa_dtype;
 
 /* Bits of the device error word (see pa_get_device_error).  Kernels never
  * trap: an out-of-range index is recorded here and the access is skipped. */

@@ -65,7 +65,7 @@ class Oracle:
     # -- helpers ---------------------------------------------------------
     @staticmethod
     def _dtype_code(dtype: str) -> int:
-        return {"f32": 0, "bf16": 1}[dtype]
+        return {"f32": 0, "bf16": 1, "f16": 2}[dtype]
 
     @staticmethod
     def _c(a: np.ndarray, dt) -> np.ndarray:

@@ -41,6 +41,7 @@
 
 #define ORACLE_F32 0
 #define ORACLE_BF16 1
+#define ORACLE_F16 2
 
 typedef struct {
     const void *q;              /* [B, Hq, D] */
@@ -51,8 +52,23 @@ typedef struct {
     double scale;
     int32_t B, Hq, Hkv, D;
     int32_t block_size, num_blocks, max_blocks_per_seq;
-    int32_t dtype;              /* ORACLE_F32 or ORACLE_BF16 */
+    int32_t dtype;              /* ORACLE_F32, ORACLE_BF16 or ORACLE_F16 */
 } oracle_problem;
+
+/* IEEE 754 binary16 -> double (exact): sign, 5 exponent bits (bias 15),
+ * 10 fraction bits; exponent 0 is subnormal, 31 is infinity / NaN. */
+static double half_to_double(uint16_t h)
+{
+    int sign = h >> 15, e = (h >> 10) & 0x1F, f = h & 0x3FF;
+    double v;
+    if (e == 0)
+        v = ldexp((double)f, -24);
+    else if (e == 31)
+        v = f ? NAN : INFINITY;
+    else
+        v = ldexp((double)(1024 + f), e - 25);
+    return sign ? -v : v;
+}
 
 /* One stored value, widened to double.  bf16 is the upper half of an IEEE
  * binary32, so shifting its 16 bits up gives the float exactly. */
@@ -60,6 +76,8 @@ static double value_at(const void *base, int64_t i, int dtype)
 {
     if (dtype == ORACLE_F32)
         return (double)((const float *)base)[i];
+    if (dtype == ORACLE_F16)
+        return half_to_double(((const uint16_t *)base)[i]);
     uint32_t bits = ((uint32_t)((const uint16_t *)base)[i]) << 16;
     float f;
     memcpy(&f, &bits, sizeof f);
@@ -74,7 +92,7 @@ static int check_problem(const oracle_problem *p)
         return -2;
     if (p->block_size <= 0 || p->num_blocks < 0 || p->max_blocks_per_seq < 0)
         return -3;
-    if (p->dtype != ORACLE_F32 && p->dtype != ORACLE_BF16)
+    if (p->dtype != ORACLE_F32 && p->dtype != ORACLE_BF16 && p->dtype != ORACLE_F16)
         return -4;
     for (int b = 0; b < p->B; ++b) {
         int32_t L = p->context_lens[b];

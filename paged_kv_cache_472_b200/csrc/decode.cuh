@@ -128,6 +128,35 @@ struct Elem<__nv_bfloat16> {
 };
 
 template <>
+struct Elem<__half> {
+    static constexpr int kBytes = 2;
+    static __device__ __forceinline__ void load8(const void *p, float2 (&v)[4]) {
+        const uint4 w = *reinterpret_cast<const uint4 *>(p);
+        v[0] = f16x2_to_float2(w.x);
+        v[1] = f16x2_to_float2(w.y);
+        v[2] = f16x2_to_float2(w.z);
+        v[3] = f16x2_to_float2(w.w);
+    }
+    static __device__ __forceinline__ void store8(void *p, const float2 (&v)[4]) {
+        uint4 w;
+        w.x = pack_f16x2(v[0].x, v[0].y);
+        w.y = pack_f16x2(v[1].x, v[1].y);
+        w.z = pack_f16x2(v[2].x, v[2].y);
+        w.w = pack_f16x2(v[3].x, v[3].y);
+        *reinterpret_cast<uint4 *>(p) = w;
+    }
+    static __device__ __forceinline__ void store2(void *p, float a, float b) {
+        *reinterpret_cast<uint32_t *>(p) = pack_f16x2(a, b);
+    }
+    static __device__ __forceinline__ void store1(void *p, float a) {
+        *reinterpret_cast<__half *>(p) = __float2half_rn(a);
+    }
+    static __device__ __forceinline__ void store_zero8(void *p) {
+        *reinterpret_cast<uint4 *>(p) = make_uint4(0, 0, 0, 0);
+    }
+};
+
+template <>
 struct Elem<float> {
     static constexpr int kBytes = 4;
     static __device__ __forceinline__ void load8(const void *p, float2 (&v)[4]) {
@@ -536,10 +565,11 @@ struct CoreEngine {
 };
 
 // ===========================================================================
-// tensor-core engine (bf16): tokens are the M dimension of every tile
+// tensor-core engine (bf16 / fp16): tokens are the M dimension of every tile
 // ===========================================================================
-template <int D, int UPW>
+template <typename T, int D, int UPW>
 struct MmaEngine {
+    using Op = Mma16<T>;
     static constexpr int KS = D / 16;  // k-steps of QK (over d) = m-tiles of PV (over d)
     static constexpr int E = 2;
     static constexpr bool kPaddedRows = true;
@@ -611,7 +641,7 @@ struct MmaEngine {
         for (int ks = 0; ks < KS; ++ks) {
             uint32_t a[4];
             ldmatrix_x4(a, ka + chunk_off(ks * 2 + (a_col >> 3), swz, p));
-            mma_bf16_16816(s, a, u.qb[ks][0], u.qb[ks][1]);
+            Op::mma(s, a, u.qb[ks][0], u.qb[ks][1]);
         }
         // ---- online softmax over the 16 tokens, per head column ----
         const bool v0 = g4 < nvalid, v1 = g4 + 8 < nvalid;
@@ -642,9 +672,9 @@ struct MmaEngine {
         // P = hi + lo, both bf16: the PV product then carries ~16 bits of each
         // weight instead of 8 (one bf16 P alone misses the tolerance on very
         // short, peaked contexts)
-        const uint32_t ph0 = pack_bf16x2(p0, p1), ph1 = pack_bf16x2(p2, p3);
-        const float2 h0 = bf16x2_to_float2(ph0), h1 = bf16x2_to_float2(ph1);
-        const uint32_t pl0 = pack_bf16x2(p0 - h0.x, p1 - h0.y), pl1 = pack_bf16x2(p2 - h1.x, p3 - h1.y);
+        const uint32_t ph0 = Op::pack(p0, p1), ph1 = Op::pack(p2, p3);
+        const float2 h0 = Op::unpack(ph0), h1 = Op::unpack(ph1);
+        const uint32_t pl0 = Op::pack(p0 - h0.x, p1 - h0.y), pl1 = Op::pack(p2 - h1.x, p3 - h1.y);
         // P^T fragments (k = token, n = head)
         const uint32_t bh0 = movmatrix_trans(ph0), bh1 = movmatrix_trans(ph1);
         const uint32_t bl0 = movmatrix_trans(pl0), bl1 = movmatrix_trans(pl1);
@@ -674,8 +704,8 @@ struct MmaEngine {
         for (int mt = 0; mt < KS; ++mt) {
             uint32_t a[4];
             ldmatrix_x4_trans(a, va + chunk_off(mt * 2 + (v_col >> 3), vswz, p));
-            mma_bf16_16816(u.o[mt], a, bh0, bh1);
-            mma_bf16_16816(u.o[mt], a, bl0, bl1);
+            Op::mma(u.o[mt], a, bh0, bh1);
+            Op::mma(u.o[mt], a, bl0, bl1);
         }
     }
 
@@ -719,8 +749,8 @@ struct MmaEngine {
             unsigned char *row = outb + (h_out0 + h) * D * E;
 #pragma unroll
             for (int mt = 0; mt < KS; ++mt) {
-                Elem<__nv_bfloat16>::store1(row + (mt * 16 + g4) * E, u.o[mt][j] * inv);
-                Elem<__nv_bfloat16>::store1(row + (mt * 16 + g4 + 8) * E, u.o[mt][2 + j] * inv);
+                Elem<T>::store1(row + (mt * 16 + g4) * E, u.o[mt][j] * inv);
+                Elem<T>::store1(row + (mt * 16 + g4 + 8) * E, u.o[mt][2 + j] * inv);
             }
         }
     }

@@ -31,6 +31,7 @@ pa_status ok() {
 bool aligned16(const void *p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
 bool pow2(int x) { return x > 0 && (x & (x - 1)) == 0; }
 int elem_bytes(int dtype) { return dtype == PA_DTYPE_F32 ? 4 : 2; }
+bool tensor_core_dtype(int dtype) { return dtype == PA_DTYPE_BF16 || dtype == PA_DTYPE_F16; }
 size_t round_up(size_t x, size_t a) { return (x + a - 1) / a * a; }
 
 constexpr int kSmemLimit = 232448;     // opt-in shared memory per CTA on sm_100 (static + dynamic)
@@ -46,7 +47,7 @@ pa_status check_shape(const pa_shape *s) {
     if (s->Hq % s->Hkv) return fail(PA_ERR_INVALID_ARG, "Hq=%d is not a multiple of Hkv=%d", s->Hq, s->Hkv);
     if (s->D <= 0 || s->block_size <= 0 || s->num_blocks <= 0 || s->max_blocks_per_seq <= 0)
         return fail(PA_ERR_INVALID_ARG, "D, block_size, num_blocks, max_blocks_per_seq must be > 0");
-    if (s->dtype != PA_DTYPE_F32 && s->dtype != PA_DTYPE_BF16)
+    if (s->dtype != PA_DTYPE_F32 && s->dtype != PA_DTYPE_BF16 && s->dtype != PA_DTYPE_F16)
         return fail(PA_ERR_INVALID_ARG, "dtype=%d is not a pa_dtype", s->dtype);
     if ((int64_t)s->num_blocks * s->block_size > INT32_MAX)
         return fail(PA_ERR_UNSUPPORTED, "num_blocks*block_size exceeds the int32 slot range");
@@ -69,15 +70,18 @@ KernelFn pick_core(int hc, int upw) {
     return nullptr;
 }
 
-template <int D>
+template <typename T, int D>
 KernelFn pick_mma(int upw) {
-    if (upw == 1) return pa::paged_decode_kernel<__nv_bfloat16, D, pa::MmaEngine<D, 1>>;
-    if (upw == 2) return pa::paged_decode_kernel<__nv_bfloat16, D, pa::MmaEngine<D, 2>>;
+    if (upw == 1) return pa::paged_decode_kernel<T, D, pa::MmaEngine<T, D, 1>>;
+    if (upw == 2) return pa::paged_decode_kernel<T, D, pa::MmaEngine<T, D, 2>>;
     return nullptr;
 }
 
 KernelFn pick_kernel(int dtype, int D, int hc, int upw) {
-    if (dtype == PA_DTYPE_BF16) return D == 64 ? pick_mma<64>(upw) : (D == 128 ? pick_mma<128>(upw) : nullptr);
+    if (dtype == PA_DTYPE_BF16)
+        return D == 64 ? pick_mma<__nv_bfloat16, 64>(upw) : (D == 128 ? pick_mma<__nv_bfloat16, 128>(upw) : nullptr);
+    if (dtype == PA_DTYPE_F16)
+        return D == 64 ? pick_mma<__half, 64>(upw) : (D == 128 ? pick_mma<__half, 128>(upw) : nullptr);
     return D == 64 ? pick_core<64>(hc, upw) : (D == 128 ? pick_core<128>(hc, upw) : nullptr);
 }
 
@@ -113,7 +117,7 @@ struct Layout {
 Layout smem_layout(int dtype, int D, int stages, uint32_t q_bytes, uint32_t half_bytes, int hc, int tsplit,
                    int nhvr) {
     Layout l;
-    const bool mma = dtype == PA_DTYPE_BF16;
+    const bool mma = tensor_core_dtype(dtype);
     l.off_bar = 0;
     const uint32_t bar_bytes = (uint32_t)round_up((2 * stages + 4) * 8, 128);
     l.off_q = bar_bytes;
@@ -163,7 +167,7 @@ struct Mapping {
 bool choose_mapping(const pa_shape *s, Mapping &m) {
     const int G = s->Hq / s->Hkv;
     const int e = elem_bytes(s->dtype);
-    const bool mma = s->dtype == PA_DTYPE_BF16;
+    const bool mma = tensor_core_dtype(s->dtype);
     for (int hg = s->Hkv; hg >= 1; --hg) {
         if (s->Hkv % hg || hg * s->D * e > 2048) continue;
         if (mma) {
@@ -225,7 +229,9 @@ pa_status encode_pool_map(CUtensorMap *map, const void *pool, const pa_shape *s,
     cuuint64_t strides[2] = {(cuuint64_t)s->Hkv * s->D * 2, (cuuint64_t)s->D * 2};
     cuuint32_t box[3] = {64, (cuuint32_t)br, (cuuint32_t)hg};
     cuuint32_t estr[3] = {1, 1, 1};
-    CUresult r = enc(map, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3, const_cast<void *>(pool), dims, strides, box, estr,
+    const CUtensorMapDataType dt =
+        s->dtype == PA_DTYPE_F16 ? CU_TENSOR_MAP_DATA_TYPE_FLOAT16 : CU_TENSOR_MAP_DATA_TYPE_BFLOAT16;
+    CUresult r = enc(map, dt, 3, const_cast<void *>(pool), dims, strides, box, estr,
                      CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
                      CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
     if (r != CUDA_SUCCESS) return fail(PA_ERR_CUDA, "cuTensorMapEncodeTiled failed (%d)", (int)r);
@@ -317,7 +323,7 @@ pa_status launch_decode(const void *q, const void *k_cache, const void *v_cache,
     p.comb_stride = lay.comb_stride;
     p.bs_log2 = log2i(s->block_size);
     p.lens_cached = s->B <= pa::kLensCache ? 1 : 0;
-    if (s->dtype == PA_DTYPE_BF16) {
+    if (tensor_core_dtype(s->dtype)) {
         const int br = plan->tile_tokens < s->block_size ? plan->tile_tokens : s->block_size;
         p.use_tmap = 1;
         p.br_log2 = log2i(br);

@@ -5,11 +5,11 @@ from __future__ import annotations
 
 import torch
 
-from . import (DTYPE_BF16, DTYPE_F32, Plan, Shape, pa_decode, pa_get_device_error, pa_kv_append,
+from . import (DTYPE_BF16, DTYPE_F16, DTYPE_F32, Plan, Shape, pa_decode, pa_get_device_error, pa_kv_append,
                pa_kv_append_decode, pa_plan, pa_workspace_init)
 
-TORCH_DTYPE = {DTYPE_F32: torch.float32, DTYPE_BF16: torch.bfloat16}
-PA_DTYPE = {torch.float32: DTYPE_F32, torch.bfloat16: DTYPE_BF16}
+TORCH_DTYPE = {DTYPE_F32: torch.float32, DTYPE_BF16: torch.bfloat16, DTYPE_F16: torch.float16}
+PA_DTYPE = {torch.float32: DTYPE_F32, torch.bfloat16: DTYPE_BF16, torch.float16: DTYPE_F16}
 
 
 def shape_of(q: torch.Tensor, k_cache: torch.Tensor, block_tables: torch.Tensor) -> Shape:

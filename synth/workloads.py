@@ -81,11 +81,13 @@ def philox4x32_10(ctr, key) -> np.ndarray:
 
 
 def normals(seed: int, stream: int, shape, dtype: str) -> np.ndarray:
-    """N(0,1) values of the given shape: float32, or bf16 bit patterns (uint16)."""
+    """N(0,1) values of the given shape: float32, or bf16 / fp16 bit patterns (uint16)."""
     n = int(np.prod(shape))
-    if dtype == DTYPE_F32:
+    if dtype in (DTYPE_F32, DTYPE_F16):
         out = np.empty(n, dtype=np.float32)
         _lib().synth_normals(seed, stream, n, out.ctypes.data, None)
+        if dtype == DTYPE_F16:  # nearest-even, as numpy's float32 -> float16 cast
+            out = out.astype(np.float16).view(np.uint16)
     else:
         out = np.empty(n, dtype=np.uint16)
         _lib().synth_normals(seed, stream, n, None, out.ctypes.data)
@@ -93,6 +95,7 @@ def normals(seed: int, stream: int, shape, dtype: str) -> np.ndarray:
 
 DTYPE_F32 = "f32"
 DTYPE_BF16 = "bf16"
+DTYPE_F16 = "f16"
 
 
 def f32_to_bf16_bits(x: np.ndarray) -> np.ndarray:
@@ -148,8 +151,12 @@ class PagedDecodeCase:
         return self.Hq // self.Hkv
 
     def as_float32(self, a: np.ndarray) -> np.ndarray:
-        """Value array widened to float32 (exact for both dtypes)."""
-        return bf16_bits_to_f32(a) if self.dtype == DTYPE_BF16 else np.asarray(a, np.float32)
+        """Value array widened to float32 (exact for every dtype)."""
+        if self.dtype == DTYPE_BF16:
+            return bf16_bits_to_f32(a)
+        if self.dtype == DTYPE_F16:
+            return np.asarray(a, np.uint16).view(np.float16).astype(np.float32)
+        return np.asarray(a, np.float32)
 
     def blocks_used(self) -> int:
         return int(sum(-(-int(L) // self.block_size) for L in self.context_lens))

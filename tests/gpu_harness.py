@@ -8,7 +8,7 @@ import numpy as np
 import torch
 
 import synth
-from paged_kv_cache_472_b200 import DTYPE_BF16, DTYPE_F32, Shape
+from paged_kv_cache_472_b200 import DTYPE_BF16, DTYPE_F16, DTYPE_F32, Shape
 from paged_kv_cache_472_b200.session import PagedDecoder
 
 # Tolerances of the decode parity check, per element:
@@ -16,13 +16,17 @@ from paged_kv_cache_472_b200.session import PagedDecoder
 # bf16 inputs with fp32 accumulation: 2e-3 absolute / 1e-2 relative.  The
 # bf16 output rounding alone is up to 2^-9 relative, so the two bounds are
 # combined as allclose rather than required together.  fp32 inputs: 1e-5.
-TOL = {"bf16": (2e-3, 1e-2), "f32": (1e-5, 1e-5)}
+# fp16 inputs (no bound is stated for them): the bf16 bound, which the fp16
+# output rounding (2^-11 relative) sits well inside.
+TOL = {"bf16": (2e-3, 1e-2), "f16": (2e-3, 1e-2), "f32": (1e-5, 1e-5)}
 
 
 def _vals(a: np.ndarray, dtype: str, device) -> torch.Tensor:
     a = np.ascontiguousarray(a)
     if dtype == "bf16":
         return torch.from_numpy(a.view(np.int16)).view(torch.bfloat16).to(device)
+    if dtype == "f16":
+        return torch.from_numpy(a.view(np.int16)).view(torch.float16).to(device)
     return torch.from_numpy(a).to(device)
 
 
@@ -50,7 +54,7 @@ def upload(case, device="cuda") -> DeviceCase:
 
 def shape_of(case) -> Shape:
     return Shape(case.B, case.Hq, case.Hkv, case.D, case.block_size, case.num_blocks, case.max_blocks_per_seq,
-                 DTYPE_F32 if case.dtype == "f32" else DTYPE_BF16)
+                 {"f32": DTYPE_F32, "bf16": DTYPE_BF16, "f16": DTYPE_F16}[case.dtype])
 
 
 def run(case, partition_tokens: int = 0, max_context_len: int | None = None, dev: DeviceCase | None = None,
@@ -86,8 +90,8 @@ def assert_close(got: np.ndarray, ref: np.ndarray, dtype: str, what: str = ""):
 
 def pool_equal(dev_pool: torch.Tensor, ref_pool: np.ndarray, dtype: str) -> bool:
     ref = _vals(ref_pool, dtype, dev_pool.device)
-    return bool(torch.equal(dev_pool.view(torch.int16 if dtype == "bf16" else torch.int32),
-                            ref.view(torch.int16 if dtype == "bf16" else torch.int32)))
+    iv = torch.int32 if dtype == "f32" else torch.int16
+    return bool(torch.equal(dev_pool.view(iv), ref.view(iv)))
 
 
 def sample_pairs(case, n: int, seed: int = 0) -> np.ndarray:

@@ -97,6 +97,9 @@ EDGE = [
     ("f32_d64_bs256", "f32", 8, 2, 64, 256, [600, 256, 257]),
     ("bs128_d128", "bf16", 16, 8, 128, 128, [129, 1024, 383]),
     ("single_request", "bf16", 16, 8, 128, 16, [4000]),
+    ("f16_gqa2", "f16", 16, 8, 128, 16, [300, 17, 1, 1100]),
+    ("f16_d64_gqa4", "f16", 32, 8, 64, 32, [513, 64, 2]),
+    ("f16_mqa32", "f16", 32, 1, 128, 256, [2000, 255]),
 ]
 
 
@@ -174,6 +177,15 @@ def test_repeated_calls_reuse_workspace(orc):
     assert dec.device_error() == 0
     counters = dec.workspace[256:256 + 4 * case.B * case.Hkv].view(torch.int32)
     assert int(counters.abs().sum()) == 0
+
+
+def test_fp16_workload_shape(orc):
+    """The Qwen3-0.6B-shaped batch with fp16 values instead of bf16."""
+    rng = np.random.default_rng(2002)
+    lens = rng.integers(128, 2048, size=32, endpoint=True)
+    case = synth.build_case("qwen3-0.6b-fp16", dtype="f16", Hq=16, Hkv=8, D=128, block_size=16,
+                            context_lens=lens, seed=2002)
+    check_full(orc, case, 0)
 
 
 @pytest.mark.parametrize("cid,batch", [(2, None), (3, 32), (5, 48), (1, None)])

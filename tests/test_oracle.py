@@ -59,3 +59,21 @@ def test_thread_count_does_not_change_result(orc):
     case = synth.make_config(1)
     kc, vc = orc.kv_append(case)
     assert np.array_equal(orc.decode(case, kc, vc, nthreads=1), orc.decode(case, kc, vc, nthreads=4))
+
+
+def test_fp16_values_widen_exactly(orc):
+    """Every finite fp16 bit pattern reaches the oracle's arithmetic exactly:
+    with one token, out = V, compared with numpy's float16 -> float64."""
+    bits = np.arange(65536, dtype=np.uint32).astype(np.uint16)
+    finite = bits[np.isfinite(bits.view(np.float16))]
+    D = 256
+    n = -(-finite.size // D) * D
+    vals = np.zeros(n, np.uint16)
+    vals[:finite.size] = finite
+    rows = n // D
+    case = synth.build_case("f16bits", dtype="f16", Hq=1, Hkv=1, D=D, block_size=16,
+                            context_lens=[1] * rows, seed=4)
+    case.v_new = vals.reshape(rows, 1, D)
+    out = orc.decode(case)
+    want = vals.view(np.float16).astype(np.float64).reshape(rows, 1, D)
+    assert np.array_equal(out, want)
