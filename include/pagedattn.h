@@ -88,7 +88,10 @@ typedef struct {
     int32_t warps_per_unit;   /* >1: a warp team splits the tokens of one unit */
     int32_t max_context_len;  /* the bound the workspace was sized for */
     int32_t smem_bytes;
-    int32_t reserved;
+    int32_t dynamic_share;    /* PA_SPLIT_BALANCED: share of each request's tiles handed out
+                                 at run time to whichever CTA is free, in 1/256.  pa_plan
+                                 sets 0; a caller may set 1..64 when B <= 512 (the
+                                 workspace is sized for 64) */
     int64_t max_slots;        /* partial-result slots in the workspace */
     pa_shape shape;           /* the shape this plan was made for */
     size_t workspace_bytes;   /* bytes pa_decode needs at `workspace` */

@@ -39,11 +39,11 @@ class Plan(ctypes.Structure):
                 ("tile_tokens", ctypes.c_int32), ("stages", ctypes.c_int32), ("head_group", ctypes.c_int32),
                 ("heads_per_unit", ctypes.c_int32), ("units_per_warp", ctypes.c_int32),
                 ("warps_per_unit", ctypes.c_int32), ("max_context_len", ctypes.c_int32),
-                ("smem_bytes", ctypes.c_int32), ("reserved", ctypes.c_int32), ("max_slots", ctypes.c_int64),
+                ("smem_bytes", ctypes.c_int32), ("dynamic_share", ctypes.c_int32), ("max_slots", ctypes.c_int64),
                 ("shape", Shape), ("workspace_bytes", ctypes.c_size_t)]
 
     def as_dict(self):
-        d = {n: getattr(self, n) for n, _ in self._fields_ if n not in ("shape", "reserved")}
+        d = {n: getattr(self, n) for n, _ in self._fields_ if n != "shape"}
         d["shape"] = {n: getattr(self.shape, n) for n, _ in Shape._fields_}
         return d
 

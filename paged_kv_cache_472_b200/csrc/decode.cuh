@@ -12,34 +12,45 @@
 //
 // Work decomposition.  A "virtual request" (vr) is one request restricted to
 // a group of HG KV heads (HG = Hkv unless one token of all KV heads is too
-// large to stage).  Its tokens are cut into tiles of ST tokens.  The tiles of
-// all vrs, laid end to end, are divided among persistent CTAs:
-//   * balanced mode: CTA c takes tiles [c*NT/C, (c+1)*NT/C) of the flat list,
-//     so every CTA moves the same number of bytes whatever the length mix;
-//   * fixed mode: the flat list is of partitions of `part_tiles` tiles (the
-//     classic flash-decoding split), divided the same way.
-// A vr that lies wholly inside one CTA's range is written straight to `out`.
-// Otherwise each covering CTA leaves (m, l, o) for its piece in the
-// workspace and bumps the vr's counter; the CTA that arrives last combines
-// the pieces by log-sum-exp and restores the counter to zero (no CTA ever
-// waits for another).
+// large to stage).  Its tokens are cut into tiles of ST tokens.
+//   * balanced mode: the first tiles of every vr form a static list, its last
+//     share (a quarter, for batches large enough) a dynamic list.  CTA c takes
+//     slice c of the static list; the dynamic list is cut into grains of about
+//     an eighth of a CTA's share, handed out at run time through a global
+//     counter to whichever CTA is free, so that fast and slow SMs finish
+//     together.  The cut itself depends only on the lengths, so every CTA can
+//     name all pieces of a vr and their partial slots.
+//   * fixed mode: the static list is of partitions of `part_tiles` tiles (the
+//     classic flash-decoding split), divided the same way; nothing dynamic.
+// A vr that lies wholly inside one piece is written straight to `out`.
+// Otherwise each piece leaves (m, l, o) in its workspace slot and bumps the
+// vr's counter; the CTA that arrives last combines the pieces by log-sum-exp
+// and restores the counter to zero (no CTA ever waits for another).
 //
-// Inside a CTA: warp 8 is a producer that walks the block table (a window of
-// 32 entries held in registers, the next window prefetched) and issues bulk
-// asynchronous copies (cp.async.bulk, completion counted on an mbarrier) of
-// whole K/V rows into a ring of shared-memory stages.  Warps 0-7 consume;
+// Inside a CTA: warp 8 is the producer.  It alone walks the work, publishes
+// one descriptor per piece (with q) to the consumers, walks the block table (a
+// window of 32 entries held in registers, the next window prefetched) and
+// fills a ring of shared-memory stages with tensor-map boxes (bf16 / fp16) or
+// bulk copies (fp32), completion counted on mbarriers.  Warps 0-7 consume;
 // each owns (KV head, query heads) units of the vr and runs one of two
 // engines over every 16 tokens:
-//   * MmaEngine (bf16): warp-level tensor-core tiles with tokens as the M
-//     dimension: S^T = K Q^T (m16n8k16, K from shared memory by ldmatrix,
+//   * MmaEngine (bf16 / fp16): warp-level tensor-core tiles with tokens as the
+//     M dimension: S^T = K Q^T (m16n8k16, K from shared memory by ldmatrix,
 //     Q fragments in registers), online softmax on the accumulator
 //     fragments, then O^T += V^T P^T (V by transposing ldmatrix, P moved into
-//     operand layout by movmatrix).  Stage rows are padded by 16 bytes so the
-//     8 rows of every ldmatrix hit 8 different bank groups.
+//     operand layout by movmatrix).
 //   * CoreEngine (fp32, or any dtype): lanes own 8-element slices of a token
 //     row; packed fp32x2 FMAs form partial dots, a reduce-scatter across the
 //     slice lanes finishes them, and every lane accumulates its 8 output
 //     elements of all its heads.
+// Warp 9 counts arrivals: after the consumers have stored a piece's partial it
+// fences and bumps the vr's counter, so no consumer stalls on a global atomic.
+//
+// Fused step (append + decode in one launch): the piece holding a request's
+// last position also writes the request's new K/V token to its cache slot, and
+// the consumers overwrite that row of the staged tile with the new values
+// before reading it, so the decode sees the appended token without waiting
+// for the cache write.
 #pragma once
 
 #include <cstddef>
@@ -49,9 +60,12 @@
 namespace pa {
 
 constexpr int kConsumerWarps = 8;
-constexpr int kDecodeThreads = (kConsumerWarps + 1) * 32;
+constexpr int kProducerWarp = kConsumerWarps;
+constexpr int kArrivalWarp = kConsumerWarps + 1;
+constexpr int kDecodeThreads = (kConsumerWarps + 2) * 32;
 constexpr int kSubTile = 16;     // tokens per online-softmax update
 constexpr int kMergeParts = 64;  // pieces the shared-memory merge path handles
+constexpr int kPrefixCache = 512;  // requests whose static / dynamic prefix sums live in shared memory
 
 struct DecodeParams {
     CUtensorMap tmap_k;   // bf16 path: [d, token row, head] view of the pools, 128B swizzle,
@@ -65,6 +79,11 @@ struct DecodeParams {
     float *partials;      // [slots][slot_floats] fp32: o[NHvr][D], m[NHvr], l[NHvr], padding
     int32_t *counters;    // [B * NHG]
     int32_t *error;       // device error word
+    int32_t *grab;        // dynamic grains handed out so far (reset by the last CTA)
+    int32_t *grab_done;   // CTAs that found the dynamic list empty
+    const void *k_new;    // fused step: [B, Hkv, D] new token per request
+    const void *v_new;
+    const int32_t *slot_mapping;  // fused step: [B] cache slot of the new token (< 0: none)
     float qscale;         // scale * log2(e)
     int32_t B, Hq, Hkv, bs, num_blocks, max_blocks;
     int32_t G, HG, NHG, NHvr;
@@ -76,7 +95,8 @@ struct DecodeParams {
     int32_t tsplit;       // warps sharing one unit (token split)
     int32_t units;        // units per vr
     int32_t heads_per_unit;
-    int32_t pdl;          // 1: wait for the preceding grid before the first K/V copy
+    int32_t fused;        // 1: append the new tokens in this launch
+    int32_t dyn_num;      // balanced mode: dynamic share of each vr, in 1/256 (0: all static)
     int64_t max_slots;
     int64_t slot_floats;  // NHvr * D + (2 * NHvr rounded up to a multiple of 4)
     uint32_t off_bar, off_q, off_stage, off_scratch, off_comb, off_merge;
@@ -182,7 +202,7 @@ struct Elem<float> {
 };
 
 // ---------------------------------------------------------------------------
-// work list (identical sequence in every warp of a CTA)
+// work list
 constexpr int kLensCache = 1024;  // requests whose lengths are kept in shared memory
 
 __device__ __forceinline__ int clamped_len(const DecodeParams &p, const int *lens_s, int b) {
@@ -197,36 +217,76 @@ __device__ __forceinline__ int units_of_len(const DecodeParams &p, int L) {
     return p.mode == PA_SPLIT_BALANCED ? tiles : (tiles + p.part_tiles - 1) / p.part_tiles;
 }
 
-__device__ __forceinline__ int64_t range_lo(int64_t c, int64_t NT, int64_t C) { return c * NT / C; }
+// units of a vr of T units that go to the dynamic list
+__device__ __forceinline__ int dyn_units(int T, int dyn_num) { return (int)(((int64_t)T * dyn_num) >> 8); }
 
-// CTA whose range contains flat unit x
-__device__ __forceinline__ int64_t cta_of(int64_t x, int64_t NT, int64_t C) { return ((x + 1) * C - 1) / NT; }
-
-struct Seg {
-    int b, hg, L;
-    int t_begin, t_end;  // tiles of the vr
-    int nparts;          // pieces this vr is split into (1 = whole vr here)
-    int64_t slot;        // partial slot when nparts > 1
-    int64_t vr_start;    // flat index of the vr's first unit
-    int units;           // units of the vr
+// The cut of the work (identical in every CTA): the static list (every vr's
+// first units, vr after vr) in Cn slices, and the dynamic list (every vr's
+// remaining units, vr after vr) in J grains of g units.
+struct Cut {
+    int64_t S, Dn;  // units in the static / dynamic list
+    int64_t Cn;     // CTAs with a static slice
+    int64_t g, J;
+    int dyn;        // the dynamic list is in use
 };
 
+__device__ __forceinline__ int64_t slice_lo(int64_t r, const Cut &k) { return r * k.S / k.Cn; }
+// static slice holding static-list position x
+__device__ __forceinline__ int64_t slice_of(int64_t x, const Cut &k) { return ((x + 1) * k.Cn - 1) / k.S; }
+
+struct Seg {
+    int b, hg, L;         // b < 0: no more work
+    int t_begin, t_end;   // tiles of the vr this piece covers
+    int nparts;           // pieces of the vr (1: the whole vr is in this piece)
+    int s_len, d_len;     // static / dynamic units of the vr
+    int64_t slot;         // partial slot when nparts > 1
+    int64_t ss, ds;       // list positions of the vr's first static / dynamic unit
+    int32_t patch;        // fused step: vr token that is the new token (-1: none)
+    int32_t append_slot;  // fused step: cache slot the new token goes to (-1: none)
+};
+
+// Pieces of a vr in balanced mode: one per static slice and one per grain its
+// units fall in.  Static piece (vr v, slice r) owns slot v + r and dynamic
+// piece (vr v, grain j) slot NV + C + v + j: a later vr never lies in an
+// earlier slice or grain, so no two pieces share a slot.
+__device__ __forceinline__ int balanced_parts(const Cut &k, int64_t ss, int s_len, int64_t ds, int d_len) {
+    const int ns = (int)(slice_of(ss + s_len - 1, k) - slice_of(ss, k) + 1);
+    const int nd = d_len > 0 ? (int)((ds + d_len - 1) / k.g - ds / k.g + 1) : 0;
+    return ns + nd;
+}
+
+__device__ __forceinline__ int64_t piece_slot(const DecodeParams &p, const Cut &k, const Seg &s, int i) {
+    if (p.mode != PA_SPLIT_BALANCED) return s.ss + i;
+    const int64_t v = (int64_t)s.b * p.NHG + s.hg;
+    const int64_t r0 = slice_of(s.ss, k);
+    const int ns = (int)(slice_of(s.ss + s.s_len - 1, k) - r0 + 1);
+    if (i < ns) return v + r0 + i;
+    return (int64_t)p.B * p.NHG + p.num_ctas + v + s.ds / k.g + (i - ns);
+}
+
+// pieces of this CTA's static slice, in list order
 struct SegIter {
-    int64_t cur, hi, lo, NT, C;
-    int64_t vr_start;
-    int b, hg, L, units;
+    int64_t cur, hi;
+    int64_t vr_start, ds;  // list positions of the current vr's first static / dynamic unit
+    int b, hg, L, su, du;  // current vr: request, head group, length, static / dynamic units
     const int *lens_s;
 
-    __device__ __forceinline__ bool next(const DecodeParams &p, Seg &s) {
+    __device__ __forceinline__ void load_request(const DecodeParams &p, const Cut &k) {
+        L = clamped_len(p, lens_s, b);
+        const int T = units_of_len(p, L);
+        du = k.dyn ? dyn_units(T, p.dyn_num) : 0;
+        su = T - du;
+    }
+
+    __device__ __forceinline__ bool next(const DecodeParams &p, const Cut &k, Seg &s) {
         while (cur < hi) {
-            if (cur >= vr_start + units) {
-                vr_start += units;
+            if (cur >= vr_start + su) {
+                vr_start += su;
+                ds += du;
                 if (++hg == p.NHG) {
                     hg = 0;
-                    ++b;
-                    if (b >= p.B) return false;
-                    L = clamped_len(p, lens_s, b);
-                    units = units_of_len(p, L);
+                    if (++b >= p.B) return false;
+                    load_request(p, k);
                 }
                 continue;
             }
@@ -235,27 +295,25 @@ struct SegIter {
             s.b = b;
             s.hg = hg;
             s.L = L;
-            s.vr_start = vr_start;
-            s.units = units;
+            s.s_len = su;
+            s.d_len = du;
+            s.ss = vr_start;
+            s.ds = ds;
+            s.patch = -1;
+            s.append_slot = -1;
             if (p.mode == PA_SPLIT_BALANCED) {
-                const int64_t end = vr_start + units < hi ? vr_start + units : hi;
+                const int64_t end = vr_start + su < hi ? vr_start + su : hi;
                 u1 = (int)(end - vr_start);
                 s.t_begin = u0;
                 s.t_end = u1;
-                if (u0 == 0 && u1 == units) {
-                    s.nparts = 1;
-                } else {
-                    const int64_t c0 = cta_of(vr_start, NT, C);
-                    const int64_t c1 = cta_of(vr_start + units - 1, NT, C);
-                    s.nparts = (int)(c1 - c0 + 1);
-                }
-                s.slot = 2 * (int64_t)blockIdx.x + (cur == lo ? 0 : 1);
+                s.nparts = balanced_parts(k, vr_start, su, ds, du);
+                s.slot = (int64_t)b * p.NHG + hg + blockIdx.x;
             } else {
                 const int tiles = (L + p.ST - 1) / p.ST;
                 u1 = u0 + 1;
                 s.t_begin = u0 * p.part_tiles;
                 s.t_end = min(tiles, (u0 + 1) * p.part_tiles);
-                s.nparts = units;
+                s.nparts = su;
                 s.slot = vr_start + u0;
             }
             cur = vr_start + u1;
@@ -265,26 +323,78 @@ struct SegIter {
     }
 };
 
-constexpr int kMaxPending = 16;  // split pieces whose arrival a CTA counts at once
+// pieces of grain j of the dynamic list (balanced mode, prefix sums in shared memory)
+struct GrainIter {
+    int64_t y, y1, j;
 
-struct __align__(16) DecodeCtl {
-    int64_t red[kConsumerWarps + 1];
-    int64_t total;
-    int64_t found_b, found_excl;
-    int abort;
-    int merge_flag;
-    Seg pending[kMaxPending];   // pieces written to the workspace, arrival not yet counted
-    int last[kMaxPending];      // this CTA delivered the vr's last piece
+    __device__ __forceinline__ bool next(const DecodeParams &p, const Cut &k, const int *lens_s, const int *pre_s,
+                                         const int *pre_d, Seg &s) {
+        if (y >= y1) return false;
+        // request holding dynamic position y: pre_d[b] <= y < pre_d[b + 1]
+        int lo = 0, hi = p.B;
+        while (hi - lo > 1) {
+            const int mid = (lo + hi) >> 1;
+            if (pre_d[mid] <= y) lo = mid;
+            else hi = mid;
+        }
+        const int b = lo;
+        const int L = clamped_len(p, lens_s, b);
+        const int T = units_of_len(p, L);
+        const int du = dyn_units(T, p.dyn_num);
+        const int su = T - du;
+        const int64_t off = y - pre_d[b];
+        if (du <= 0 || off < 0 || off >= (int64_t)du * p.NHG) {  // inconsistent tables: stop, never index past them
+            set_error(p.error, PA_DEVERR_TIMEOUT);
+            y = y1;
+            return false;
+        }
+        const int hg = (int)(off / du);
+        const int w = (int)(off - (int64_t)hg * du);
+        const int n = (int)(du - w < y1 - y ? du - w : y1 - y);
+        s.b = b;
+        s.hg = hg;
+        s.L = L;
+        s.t_begin = su + w;
+        s.t_end = su + w + n;
+        s.s_len = su;
+        s.d_len = du;
+        s.ss = pre_s[b] + (int64_t)hg * su;
+        s.ds = pre_d[b] + (int64_t)hg * du;
+        s.nparts = balanced_parts(k, s.ss, su, s.ds, du);
+        s.slot = (int64_t)p.B * p.NHG + p.num_ctas + (int64_t)b * p.NHG + hg + j;
+        s.patch = -1;
+        s.append_slot = -1;
+        y += n;
+        return true;
+    }
 };
 
-// slot of piece i of a split vr
-__device__ __forceinline__ int64_t piece_slot(const DecodeParams &p, const Seg &s, int i, int64_t NT, int64_t C) {
-    if (p.mode == PA_SPLIT_BALANCED) {
-        const int64_t c = cta_of(s.vr_start, NT, C) + i;
-        return 2 * c + (s.vr_start <= range_lo(c, NT, C) ? 0 : 1);
+constexpr int kMaxPending = 16;  // split pieces a CTA holds before it merges
+
+struct __align__(16) DecodeCtl {
+    int64_t red[kConsumerWarps + 2][2];
+    Cut cut;
+    int64_t found_b, found_excl, found_dexcl;
+    int abort;
+    Seg segs[2];               // published by the producer together with q
+    Seg pending[kMaxPending];  // pieces whose partial is stored; b < 0 ends the list
+    int last[kMaxPending];     // set by the arrival warp: this CTA completed the vr
+};
+
+// Barrier of the eight consumer warps on an mbarrier, so that every wait is
+// bounded (a warp that gave up after a timeout cannot leave the others
+// waiting for good, as a named barrier could).
+struct ConsumerBarrier {
+    uint64_t *bar;
+    uint32_t par;
+    __device__ __forceinline__ bool sync(volatile int *abort_flag, int lane) {
+        __syncwarp();
+        if (lane == 0) mbar_arrive(bar);
+        const bool ok = mbar_wait(bar, par, abort_flag);
+        par ^= 1u;
+        return ok;
     }
-    return s.vr_start + i;
-}
+};
 
 // ---------------------------------------------------------------------------
 // reduce-scatter of N per-lane values across the slice lanes (lane bits below
@@ -695,6 +805,7 @@ struct MmaEngine {
                 unsigned char *row = const_cast<unsigned char *>(row_ptr(tile_v, tok, g_local, p));
                 *reinterpret_cast<uint4 *>(row + chunk_off(cid, 0, p)) = make_uint4(0, 0, 0, 0);
             }
+            fence_async_smem();  // ordered before the next tensor-map fill of this stage
             __syncwarp();
         }
         // ---- O^T[d x heads] += V^T P^T ----
@@ -777,169 +888,251 @@ struct MmaEngine {
 // ===========================================================================
 // producer warp
 // ===========================================================================
-template <int D, int E>
-__device__ __forceinline__ void run_producer(const DecodeParams &p, SegIter it, uint64_t *full, uint64_t *empty,
-                                             uint64_t *qfull, uint64_t *qempty, unsigned char *qarea,
-                                             unsigned char *stage_base, volatile int *abort_flag, int lane) {
-    if (p.use_tmap && lane == 0) {
-        prefetch_tensormap(&p.tmap_k);
-        prefetch_tensormap(&p.tmap_v);
-    }
-    const uint64_t policy = policy_evict_first();
-    const unsigned char *kc = reinterpret_cast<const unsigned char *>(p.k_cache);
-    const unsigned char *vc = reinterpret_cast<const unsigned char *>(p.v_cache);
-    const unsigned char *qg = reinterpret_cast<const unsigned char *>(p.q);
-    const uint32_t row_bytes = p.row_bytes, pitch = p.row_pitch;
-    const size_t tok_stride = (size_t)p.Hkv * D * E;  // bytes between token rows in the pool
-    const bool contiguous = (p.HG == p.Hkv) && (pitch == row_bytes);
-    const int S = p.stages;
+struct ProducerState {
     int stage = 0;
     uint32_t phase = 0;
     int qslot = 0;
     uint32_t qphase = 0;
     uint32_t issued = 0, issued_par = 0;  // per stage: filled at least once / parity of the last fill
-    bool dep_done = (p.pdl == 0);
     bool ok = true;
-    Seg s;
-    while (ok && it.next(p, s)) {
-        if (!mbar_wait(&qempty[qslot], qphase ^ 1u, abort_flag)) {
-            ok = false;
-            break;
-        }
-        if (lane == 0) {
-            mbar_arrive_expect_tx(&qfull[qslot], p.q_bytes);
-            bulk_g2s(qarea + qslot * p.q_bytes, qg + ((size_t)s.b * p.Hq + (size_t)s.hg * p.NHvr) * D * E, p.q_bytes,
-                     &qfull[qslot]);
-        }
-        qslot ^= 1;
-        if (qslot == 0) qphase ^= 1u;
+    bool grab_issued = false;
+    int grab_val = 0;  // lane 0: result of the pending grab
+};
 
-        const int32_t *table = p.block_tables + (size_t)s.b * p.max_blocks;
-        const int nblk = (s.L + p.bs - 1) / p.bs;
-        int cur_base = -1, cur_val = -1, nxt_base = -1, nxt_val = -1;
-        for (int t = s.t_begin; t < s.t_end; ++t) {
-            if (!mbar_wait(&empty[stage], phase ^ 1u, abort_flag)) {
-                ok = false;
-                break;
-            }
-            const int tok0 = t * p.ST;
-            const int ntok = min(p.ST, s.L - tok0);
-            const int jb0 = tok0 / p.bs;
-            const int wb = jb0 & ~31;
-            if (wb != cur_base) {
-                if (wb == nxt_base) {
-                    cur_val = nxt_val;
-                } else {
-                    cur_val = (wb + lane < nblk) ? table[wb + lane] : -1;
-                }
-                cur_base = wb;
-                nxt_base = wb + 32;
-                nxt_val = (nxt_base + lane < nblk) ? table[nxt_base + lane] : -1;  // prefetch
-            }
-            if (!dep_done) {
-                grid_dependency_wait();  // K/V may have just been appended by the preceding grid
-                dep_done = true;
-            }
-            unsigned char *kdst = stage_base + (size_t)stage * 2 * p.half_bytes;
-            unsigned char *vdst = kdst + p.half_bytes;
-            uint32_t bytes = 0;
-            if (p.use_tmap) {
-                // one box {64 d, br rows, HG heads} per (block piece, 64-wide d-chunk), for K and V
-                const int br = 1 << p.br_log2;
-                const int npc = (ntok + br - 1) >> p.br_log2;  // pieces holding valid tokens
-                const uint32_t box_bytes = (uint32_t)p.HG << (7 + p.br_log2);
-                constexpr int NDC = D / 64;
-                const int tp = tok0 + lane * br;                 // first token of this lane's piece
-                const int j = tp >> p.bs_log2;
-                const int phys = __shfl_sync(0xffffffffu, cur_val, (j - cur_base) & 31);
-                bool valid = false;
-                if (lane < npc) {
-                    valid = phys >= 0 && phys < p.num_blocks;
-                    if (!valid) set_error(p.error, PA_DEVERR_BLOCK_ID);
-                    else bytes = 2u * NDC * box_bytes;
-                }
-#pragma unroll
-                for (int m = 16; m >= 1; m >>= 1) bytes += __shfl_xor_sync(0xffffffffu, bytes, m);
-                if (lane == 0) mbar_arrive_expect_tx(&full[stage], bytes);
-                __syncwarp();
-                if (valid) {
-                    const int32_t row = phys * p.bs + (tp & (p.bs - 1));
-                    const int32_t head0 = s.hg * p.HG;
-#pragma unroll
-                    for (int c2 = 0; c2 < NDC; ++c2) {
-                        const size_t off = (size_t)(lane * NDC + c2) * box_bytes;
-                        tma_load_3d(kdst + off, &p.tmap_k, c2 * 64, row, head0, &full[stage], policy);
-                        tma_load_3d(vdst + off, &p.tmap_v, c2 * 64, row, head0, &full[stage], policy);
-                    }
-                }
-            } else if (contiguous) {
-                // one copy per block piece: rows of all KV heads are contiguous in both places
-                const int np = (tok0 + ntok - 1) / p.bs - jb0 + 1;
-                const int j = jb0 + lane;
-                const int phys = __shfl_sync(0xffffffffu, cur_val, (j - cur_base) & 31);
-                int tlo = 0, nrows = 0;
-                bool valid = false;
-                if (lane < np) {
-                    tlo = max(tok0, j * p.bs);
-                    nrows = min(tok0 + ntok, (j + 1) * p.bs) - tlo;
-                    valid = phys >= 0 && phys < p.num_blocks;
-                    if (!valid) set_error(p.error, PA_DEVERR_BLOCK_ID);
-                    else bytes = 2u * (uint32_t)nrows * row_bytes;
-                }
-#pragma unroll
-                for (int m = 16; m >= 1; m >>= 1) bytes += __shfl_xor_sync(0xffffffffu, bytes, m);
-                if (lane == 0) mbar_arrive_expect_tx(&full[stage], bytes);
-                __syncwarp();
-                if (valid) {
-                    const size_t src = ((size_t)phys * p.bs + (tlo - j * p.bs)) * tok_stride;
-                    const uint32_t n = (uint32_t)nrows * row_bytes;
-                    bulk_g2s_hint(kdst + (tlo - tok0) * pitch, kc + src, n, &full[stage], policy);
-                    bulk_g2s_hint(vdst + (tlo - tok0) * pitch, vc + src, n, &full[stage], policy);
-                }
+// Fused step: if this piece holds the vr's last token, find where the new
+// token goes.  It is patched into the staged tile only when its slot is the
+// request's own last position; any other slot is reported.
+__device__ __forceinline__ void fused_info(const DecodeParams &p, Seg &s, int lane) {
+    if (!p.fused || s.t_end != (s.L + p.ST - 1) / p.ST) return;
+    int sm = -1, expect = -1;
+    if (lane == 0) {
+        sm = p.slot_mapping[s.b];
+        const int t = s.L - 1;
+        const int phys = p.block_tables[(size_t)s.b * p.max_blocks + t / p.bs];
+        expect = (phys >= 0 && phys < p.num_blocks) ? phys * p.bs + (t & (p.bs - 1)) : -1;
+    }
+    sm = __shfl_sync(0xffffffffu, sm, 0);
+    expect = __shfl_sync(0xffffffffu, expect, 0);
+    if (sm < 0) return;
+    if ((int64_t)sm >= (int64_t)p.num_blocks * p.bs) {
+        if (lane == 0) set_error(p.error, PA_DEVERR_SLOT);
+        return;
+    }
+    s.append_slot = sm;
+    if (sm == expect) s.patch = s.L - 1;
+    else if (lane == 0) set_error(p.error, PA_DEVERR_SLOT);
+}
+
+// Hand a piece (or the end marker, b < 0) and its q to the consumers.
+__device__ __forceinline__ void publish(const DecodeParams &p, ProducerState &ps, const Seg &s, DecodeCtl &ctl,
+                                        uint64_t *qfull, uint64_t *qempty, unsigned char *qarea,
+                                        volatile int *abort_flag, int D, int E, int lane) {
+    if (!mbar_wait(&qempty[ps.qslot], ps.qphase ^ 1u, abort_flag)) {
+        ps.ok = false;
+        return;
+    }
+    if (lane == 0) {
+        ctl.segs[ps.qslot] = s;
+        if (s.b >= 0) {
+            mbar_arrive_expect_tx(&qfull[ps.qslot], p.q_bytes);
+            const unsigned char *qg = reinterpret_cast<const unsigned char *>(p.q);
+            bulk_g2s(qarea + ps.qslot * p.q_bytes, qg + ((size_t)s.b * p.Hq + (size_t)s.hg * p.NHvr) * D * E,
+                     p.q_bytes, &qfull[ps.qslot]);
+        } else {
+            mbar_arrive(&qfull[ps.qslot]);
+        }
+    }
+    __syncwarp();
+    ps.qslot ^= 1;
+    if (ps.qslot == 0) ps.qphase ^= 1u;
+}
+
+// Fill one stage per tile of the piece.  With `grab_at_last`, the next grain
+// is requested while the piece's last tile is being issued.
+template <int D, int E>
+__device__ __forceinline__ void issue_tiles(const DecodeParams &p, ProducerState &ps, const Seg &s, bool grab_at_last,
+                                            uint64_t *full, uint64_t *empty, unsigned char *stage_base,
+                                            volatile int *abort_flag, uint64_t policy, int lane) {
+    const unsigned char *kc = reinterpret_cast<const unsigned char *>(p.k_cache);
+    const unsigned char *vc = reinterpret_cast<const unsigned char *>(p.v_cache);
+    const uint32_t row_bytes = p.row_bytes, pitch = p.row_pitch;
+    const size_t tok_stride = (size_t)p.Hkv * D * E;  // bytes between token rows in the pool
+    const bool contiguous = (p.HG == p.Hkv) && (pitch == row_bytes);
+    const int32_t *table = p.block_tables + (size_t)s.b * p.max_blocks;
+    const int nblk = (s.L + p.bs - 1) / p.bs;
+    int cur_base = -1, cur_val = -1, nxt_base = -1, nxt_val = -1;
+    for (int t = s.t_begin; t < s.t_end; ++t) {
+        if (!mbar_wait(&empty[ps.stage], ps.phase ^ 1u, abort_flag)) {
+            ps.ok = false;
+            return;
+        }
+        if (grab_at_last && t == s.t_end - 1 && !ps.grab_issued) {
+            if (lane == 0) ps.grab_val = atomicAdd(p.grab, 1);
+            ps.grab_issued = true;
+        }
+        const int tok0 = t * p.ST;
+        const int ntok = min(p.ST, s.L - tok0);
+        const int jb0 = tok0 / p.bs;
+        const int wb = jb0 & ~31;
+        if (wb != cur_base) {
+            if (wb == nxt_base) {
+                cur_val = nxt_val;
             } else {
-                // one copy per token row (padded rows, or a head group narrower than the pool row)
-                for (int i0 = 0; i0 < ntok; i0 += 32) {
-                    const int i = i0 + lane;
-                    const int tt = tok0 + i;
-                    const int j = tt / p.bs;
-                    const int phys = __shfl_sync(0xffffffffu, cur_val, (j - cur_base) & 31);
-                    if (i < ntok) {
-                        if (phys < 0 || phys >= p.num_blocks) set_error(p.error, PA_DEVERR_BLOCK_ID);
-                        else bytes += 2u * row_bytes;
-                    }
-                }
+                cur_val = (wb + lane < nblk) ? table[wb + lane] : -1;
+            }
+            cur_base = wb;
+            nxt_base = wb + 32;
+            nxt_val = (nxt_base + lane < nblk) ? table[nxt_base + lane] : -1;  // prefetch
+        }
+        unsigned char *kdst = stage_base + (size_t)ps.stage * 2 * p.half_bytes;
+        unsigned char *vdst = kdst + p.half_bytes;
+        uint32_t bytes = 0;
+        if (p.use_tmap) {
+            // one box {64 d, br rows, HG heads} per (block piece, 64-wide d-chunk), for K and V
+            const int br = 1 << p.br_log2;
+            const int npc = (ntok + br - 1) >> p.br_log2;  // pieces holding valid tokens
+            const uint32_t box_bytes = (uint32_t)p.HG << (7 + p.br_log2);
+            constexpr int NDC = D / 64;
+            const int tp = tok0 + lane * br;  // first token of this lane's piece
+            const int j = tp >> p.bs_log2;
+            const int phys = __shfl_sync(0xffffffffu, cur_val, (j - cur_base) & 31);
+            bool valid = false;
+            if (lane < npc) {
+                valid = phys >= 0 && phys < p.num_blocks;
+                if (!valid) set_error(p.error, PA_DEVERR_BLOCK_ID);
+                else bytes = 2u * NDC * box_bytes;
+            }
 #pragma unroll
-                for (int m = 16; m >= 1; m >>= 1) bytes += __shfl_xor_sync(0xffffffffu, bytes, m);
-                if (lane == 0) mbar_arrive_expect_tx(&full[stage], bytes);
-                __syncwarp();
-                for (int i0 = 0; i0 < ntok; i0 += 32) {
-                    const int i = i0 + lane;
-                    const int tt = tok0 + i;
-                    const int j = tt / p.bs;
-                    const int phys = __shfl_sync(0xffffffffu, cur_val, (j - cur_base) & 31);
-                    if (i < ntok && phys >= 0 && phys < p.num_blocks) {
-                        const size_t src = ((size_t)phys * p.bs + (tt - j * p.bs)) * tok_stride + (size_t)s.hg * row_bytes;
-                        bulk_g2s_hint(kdst + i * pitch, kc + src, row_bytes, &full[stage], policy);
-                        bulk_g2s_hint(vdst + i * pitch, vc + src, row_bytes, &full[stage], policy);
-                    }
+            for (int m = 16; m >= 1; m >>= 1) bytes += __shfl_xor_sync(0xffffffffu, bytes, m);
+            if (lane == 0) mbar_arrive_expect_tx(&full[ps.stage], bytes);
+            __syncwarp();
+            if (valid) {
+                const int32_t row = phys * p.bs + (tp & (p.bs - 1));
+                const int32_t head0 = s.hg * p.HG;
+#pragma unroll
+                for (int c2 = 0; c2 < NDC; ++c2) {
+                    const size_t off = (size_t)(lane * NDC + c2) * box_bytes;
+                    tma_load_3d(kdst + off, &p.tmap_k, c2 * 64, row, head0, &full[ps.stage], policy);
+                    tma_load_3d(vdst + off, &p.tmap_v, c2 * 64, row, head0, &full[ps.stage], policy);
                 }
             }
-            issued |= 1u << stage;
-            issued_par = (issued_par & ~(1u << stage)) | (phase << stage);
-            if (++stage == S) {
-                stage = 0;
-                phase ^= 1u;
+        } else if (contiguous) {
+            // one copy per block piece: rows of all KV heads are contiguous in both places
+            const int np = (tok0 + ntok - 1) / p.bs - jb0 + 1;
+            const int j = jb0 + lane;
+            const int phys = __shfl_sync(0xffffffffu, cur_val, (j - cur_base) & 31);
+            int tlo = 0, nrows = 0;
+            bool valid = false;
+            if (lane < np) {
+                tlo = max(tok0, j * p.bs);
+                nrows = min(tok0 + ntok, (j + 1) * p.bs) - tlo;
+                valid = phys >= 0 && phys < p.num_blocks;
+                if (!valid) set_error(p.error, PA_DEVERR_BLOCK_ID);
+                else bytes = 2u * (uint32_t)nrows * row_bytes;
+            }
+#pragma unroll
+            for (int m = 16; m >= 1; m >>= 1) bytes += __shfl_xor_sync(0xffffffffu, bytes, m);
+            if (lane == 0) mbar_arrive_expect_tx(&full[ps.stage], bytes);
+            __syncwarp();
+            if (valid) {
+                const size_t src = ((size_t)phys * p.bs + (tlo - j * p.bs)) * tok_stride;
+                const uint32_t n = (uint32_t)nrows * row_bytes;
+                bulk_g2s_hint(kdst + (tlo - tok0) * pitch, kc + src, n, &full[ps.stage], policy);
+                bulk_g2s_hint(vdst + (tlo - tok0) * pitch, vc + src, n, &full[ps.stage], policy);
+            }
+        } else {
+            // one copy per token row (a head group narrower than the pool row)
+            for (int i0 = 0; i0 < ntok; i0 += 32) {
+                const int i = i0 + lane;
+                const int tt = tok0 + i;
+                const int j = tt / p.bs;
+                const int phys = __shfl_sync(0xffffffffu, cur_val, (j - cur_base) & 31);
+                if (i < ntok) {
+                    if (phys < 0 || phys >= p.num_blocks) set_error(p.error, PA_DEVERR_BLOCK_ID);
+                    else bytes += 2u * row_bytes;
+                }
+            }
+#pragma unroll
+            for (int m = 16; m >= 1; m >>= 1) bytes += __shfl_xor_sync(0xffffffffu, bytes, m);
+            if (lane == 0) mbar_arrive_expect_tx(&full[ps.stage], bytes);
+            __syncwarp();
+            for (int i0 = 0; i0 < ntok; i0 += 32) {
+                const int i = i0 + lane;
+                const int tt = tok0 + i;
+                const int j = tt / p.bs;
+                const int phys = __shfl_sync(0xffffffffu, cur_val, (j - cur_base) & 31);
+                if (i < ntok && phys >= 0 && phys < p.num_blocks) {
+                    const size_t src = ((size_t)phys * p.bs + (tt - j * p.bs)) * tok_stride + (size_t)s.hg * row_bytes;
+                    bulk_g2s_hint(kdst + i * pitch, kc + src, row_bytes, &full[ps.stage], policy);
+                    bulk_g2s_hint(vdst + i * pitch, vc + src, row_bytes, &full[ps.stage], policy);
+                }
+            }
+        }
+        ps.issued |= 1u << ps.stage;
+        ps.issued_par = (ps.issued_par & ~(1u << ps.stage)) | (ps.phase << ps.stage);
+        if (++ps.stage == p.stages) {
+            ps.stage = 0;
+            ps.phase ^= 1u;
+        }
+    }
+}
+
+template <int D, int E>
+__device__ __forceinline__ void run_producer(const DecodeParams &p, const Cut &k, SegIter it, DecodeCtl &ctl,
+                                             const int *lens_s, const int *pre_s, const int *pre_d, uint64_t *full,
+                                             uint64_t *empty, uint64_t *qfull, uint64_t *qempty,
+                                             unsigned char *qarea, unsigned char *stage_base,
+                                             volatile int *abort_flag, int lane) {
+    const uint64_t policy = policy_evict_first();
+    ProducerState ps;
+    Seg s;
+    // this CTA's static slice
+    while (ps.ok && it.next(p, k, s)) {
+        fused_info(p, s, lane);
+        publish(p, ps, s, ctl, qfull, qempty, qarea, abort_flag, D, E, lane);
+        if (!ps.ok) break;
+        issue_tiles<D, E>(p, ps, s, k.dyn && it.cur >= it.hi, full, empty, stage_base, abort_flag, policy, lane);
+    }
+    // grains of the dynamic list, one at a time, to whichever CTA asks first
+    if (k.dyn) {
+        for (;;) {
+            if (!ps.grab_issued && lane == 0) ps.grab_val = atomicAdd(p.grab, 1);
+            const int64_t j = __shfl_sync(0xffffffffu, ps.grab_val, 0);
+            ps.grab_issued = false;
+            if (j >= k.J) break;
+            GrainIter gi;
+            gi.j = j;
+            gi.y = j * k.g;
+            gi.y1 = gi.y + k.g < k.Dn ? gi.y + k.g : k.Dn;
+            while (ps.ok && gi.next(p, k, lens_s, pre_s, pre_d, s)) {
+                fused_info(p, s, lane);
+                publish(p, ps, s, ctl, qfull, qempty, qarea, abort_flag, D, E, lane);
+                if (!ps.ok) break;
+                issue_tiles<D, E>(p, ps, s, gi.y >= gi.y1, full, empty, stage_base, abort_flag, policy, lane);
+            }
+        }
+        // the last CTA to find the list empty leaves the counters at zero for the next launch
+        if (lane == 0) {
+            const int d = atomicAdd(p.grab_done, 1);
+            if (d == p.num_ctas - 1) {
+                atomicExch(p.grab, 0);
+                atomicExch(p.grab_done, 0);
             }
         }
     }
-    if (!ok) {
+    if (ps.ok) {
+        Seg end;
+        end.b = -1;
+        publish(p, ps, end, ctl, qfull, qempty, qarea, abort_flag, D, E, lane);
+    }
+    if (!ps.ok) {
         *abort_flag = 1;
         if (lane == 0) set_error(p.error, PA_DEVERR_TIMEOUT);
     }
     // every copy this warp issued lands before the CTA can retire
     volatile int never = 0;
-    for (int st = 0; st < S; ++st)
-        if (issued & (1u << st)) mbar_wait(&full[st], (issued_par >> st) & 1u, &never);
+    for (int st = 0; st < p.stages; ++st)
+        if (ps.issued & (1u << st)) mbar_wait(&full[st], (ps.issued_par >> st) & 1u, &never);
 }
 
 // ===========================================================================
@@ -949,8 +1142,8 @@ __device__ __forceinline__ void run_producer(const DecodeParams &p, SegIter it, 
 // loads (o, m, l) in flight at a time.
 // ===========================================================================
 template <typename T, int D>
-__device__ __forceinline__ void merge_vr(const DecodeParams &p, const Seg &s, int64_t NT, int64_t C, float *msm,
-                                         int tid) {
+__device__ __forceinline__ void merge_vr(const DecodeParams &p, const Cut &cut, const Seg &s, float *msm,
+                                         ConsumerBarrier &cb, volatile int *abort_flag, int tid) {
     constexpr int E = Elem<T>::kBytes;
     constexpr int NTH = kConsumerWarps * 32;
     constexpr int KF = 8;  // pieces per batch of loads
@@ -961,10 +1154,10 @@ __device__ __forceinline__ void merge_vr(const DecodeParams &p, const Seg &s, in
     const bool cached = nparts <= kMergeParts;
     if (cached) {
         for (int i = tid; i < nparts; i += NTH) {
-            const int64_t slot = piece_slot(p, s, i, NT, C);
+            const int64_t slot = piece_slot(p, cut, s, i);
             slot_s[i] = slot < p.max_slots ? slot : -1;
         }
-        named_barrier(1, NTH);
+        cb.sync(abort_flag, tid & 31);
     }
     const int nq = NH * (D / 4);
     for (int idx0 = tid; idx0 < nq; idx0 += 2 * NTH) {
@@ -990,8 +1183,8 @@ __device__ __forceinline__ void merge_vr(const DecodeParams &p, const Seg &s, in
                 const int i = i0 + k;
                 int64_t slot = -1;
                 if (i < nparts) {
-                    slot = cached ? slot_s[i] : piece_slot(p, s, i, NT, C);
-                    if (slot >= p.max_slots) slot = -1;
+                    slot = cached ? slot_s[i] : piece_slot(p, cut, s, i);
+                    if (slot < 0 || slot >= p.max_slots) slot = -1;
                 }
                 sl[k] = slot;
             }
@@ -1046,34 +1239,133 @@ __device__ __forceinline__ void merge_vr(const DecodeParams &p, const Seg &s, in
             Elem<T>::store2(dst + 2 * E, num[j].z * inv, num[j].w * inv);
         }
     }
-    if (cached) named_barrier(1, NTH);  // the slot list is free again
+    if (cached) cb.sync(abort_flag, tid & 31);  // the slot list is free again
 }
 
-// Merge every vr for which this CTA delivered the last piece (arrivals were
-// already counted by thread 0 as the pieces were stored).
+// Merge every vr for which this CTA delivered the last piece.  The arrival
+// warp has counted the arrivals of pieces [0, npend) and signals `adone`
+// once it has; it fenced after every counter it found complete, so the other
+// CTAs' partials are visible to the loads below.
 template <typename T, int D>
-__device__ __forceinline__ void flush_pending(const DecodeParams &p, DecodeCtl &ctl, int npend, int64_t NT,
-                                              int64_t C, float *msm, int tid) {
-    constexpr int NTH = kConsumerWarps * 32;
-    named_barrier(1, NTH);
-    for (int k = 0; k < npend; ++k) {
-        if (!ctl.last[k]) continue;
-        __threadfence();
-        const Seg sk = ctl.pending[k];
-        merge_vr<T, D>(p, sk, NT, C, msm, tid);
-        if (tid == 0) p.counters[(int64_t)sk.b * p.NHG + sk.hg] = 0;
+__device__ __forceinline__ bool flush_pending(const DecodeParams &p, DecodeCtl &ctl, int npend, uint64_t *adone,
+                                              uint32_t adone_par, volatile int *abort_flag, float *msm,
+                                              ConsumerBarrier &cb, int tid) {
+    const bool ok = mbar_wait(adone, adone_par, abort_flag);
+    if (ok) {
+        const Cut cut = ctl.cut;
+        for (int k = 0; k < npend; ++k) {
+            if (!ctl.last[k]) continue;
+            const Seg sk = ctl.pending[k];
+            merge_vr<T, D>(p, cut, sk, msm, cb, abort_flag, tid);
+            if (tid == 0) p.counters[(int64_t)sk.b * p.NHG + sk.hg] = 0;
+        }
     }
-    named_barrier(1, NTH);  // pending list free again
+    cb.sync(abort_flag, tid & 31);  // pending list free again
+    return ok;
 }
+
+// Arrival warp: for each stored piece, in order, fence and count it on the
+// vr's counter; the piece that completes the vr is marked for merging.
+__device__ __forceinline__ void run_arrivals(const DecodeParams &p, DecodeCtl &ctl, uint64_t *pdone, uint64_t *adone,
+                                             volatile int *abort_flag, int lane) {
+    uint32_t pdone_par = 0;  // bit k: parity of pdone[k]'s next phase
+    int k = 0;
+    for (;;) {
+        if (!mbar_wait(&pdone[k], (pdone_par >> k) & 1u, abort_flag)) {
+            *abort_flag = 1;
+            if (lane == 0) set_error(p.error, PA_DEVERR_TIMEOUT);
+            return;
+        }
+        pdone_par ^= 1u << k;
+        const Seg s = ctl.pending[k];
+        if (s.b < 0) break;
+        if (lane == 0) {
+            __threadfence();  // the consumers' partial stores, seen through pdone, before the count
+            const int prev = atomicAdd(&p.counters[(int64_t)s.b * p.NHG + s.hg], 1);
+            const int last = prev == s.nparts - 1;
+            if (last) __threadfence();  // every other piece's partial before the merge reads them
+            ctl.last[k] = last;
+        }
+        __syncwarp();
+        if (++k == kMaxPending) {
+            if (lane == 0) mbar_arrive(adone);
+            k = 0;
+        }
+    }
+    __syncwarp();
+    if (lane == 0) mbar_arrive(adone);
+}
+
+// ===========================================================================
+// the fused step's new token, one KV head: lane i holds 16-byte chunks
+// i, i + 32, ... of [K row | V row]
+template <int D, int E>
+__device__ __forceinline__ unsigned char *stage_chunk(unsigned char *tile, int tok, int g_local, int c,
+                                                      const DecodeParams &p) {
+    if (p.use_tmap) {
+        // [piece][d-chunk][head][row][128 B], 16-byte slots swizzled by row
+        const int piece = tok >> p.br_log2, r = tok & ((1 << p.br_log2) - 1);
+        const uint32_t head_bytes = 128u << p.br_log2;
+        const int c2 = c >> 3, cc = c & 7;
+        return tile + ((size_t)(piece * (D / 64) + c2) * p.HG + g_local) * head_bytes + r * 128 +
+               ((cc ^ (r & 7)) << 4);
+    }
+    return tile + (size_t)tok * p.row_pitch + (size_t)g_local * D * E + c * 16;
+}
+
+template <int D, int E>
+struct NewToken {
+    static constexpr int CH = D * E / 16;           // 16-byte chunks in one head's row
+    static constexpr int NCH = (2 * CH + 31) / 32;  // chunks per lane
+    uint4 v[NCH];
+
+    __device__ __forceinline__ void load(const DecodeParams &p, int b, int head, int lane) {
+        const size_t base = ((size_t)b * p.Hkv + head) * D * E;
+#pragma unroll
+        for (int i = 0; i < NCH; ++i) {
+            const int c = lane + 32 * i;
+            if (c < 2 * CH) {
+                const unsigned char *src = reinterpret_cast<const unsigned char *>(c < CH ? p.k_new : p.v_new);
+                v[i] = __ldg(reinterpret_cast<const uint4 *>(src + base + (size_t)(c % CH) * 16));
+            }
+        }
+    }
+    // the append proper: the new token into its cache slot
+    __device__ __forceinline__ void store(const DecodeParams &p, int slot, int head, int lane) const {
+        const size_t base = ((size_t)slot * p.Hkv + head) * D * E;
+#pragma unroll
+        for (int i = 0; i < NCH; ++i) {
+            const int c = lane + 32 * i;
+            if (c < 2 * CH) {
+                unsigned char *dst = reinterpret_cast<unsigned char *>(const_cast<void *>(c < CH ? p.k_cache : p.v_cache));
+                *reinterpret_cast<uint4 *>(dst + base + (size_t)(c % CH) * 16) = v[i];
+            }
+        }
+    }
+    // row `tok` of the staged tile takes the new token's values
+    __device__ __forceinline__ void patch(unsigned char *tk, unsigned char *tv, int tok, int g_local,
+                                          const DecodeParams &p, int lane) const {
+#pragma unroll
+        for (int i = 0; i < NCH; ++i) {
+            const int c = lane + 32 * i;
+            if (c < 2 * CH)
+                *reinterpret_cast<uint4 *>(stage_chunk<D, E>(c < CH ? tk : tv, tok, g_local, c % CH, p)) = v[i];
+        }
+        fence_async_smem();  // ordered before the next tensor-map fill of this stage
+        __syncwarp();
+    }
+};
 
 // ===========================================================================
 template <typename T, int D, class Engine>
 __global__ void __launch_bounds__(kDecodeThreads, 1) paged_decode_kernel(const __grid_constant__ DecodeParams p) {
     constexpr int E = Elem<T>::kBytes;
     constexpr int UPW = Engine::kUnitsPerWarp;
+    constexpr int NWARPS = kConsumerWarps + 2;
     extern __shared__ __align__(1024) unsigned char smem_raw[];
     __shared__ DecodeCtl ctl;
     __shared__ int lens_s[kLensCache];
+    __shared__ int pre_s[kPrefixCache + 1], pre_d[kPrefixCache + 1];
     // swizzled tensor-map boxes need 1024-byte aligned destinations
     unsigned char *smem = smem_raw + ((1024u - (smem_u32(smem_raw) & 1023u)) & 1023u);
 
@@ -1085,6 +1377,9 @@ __global__ void __launch_bounds__(kDecodeThreads, 1) paged_decode_kernel(const _
     uint64_t *empty = full + S;
     uint64_t *qfull = empty + S;
     uint64_t *qempty = qfull + 2;
+    uint64_t *pdone = qempty + 2;
+    uint64_t *adone = pdone + kMaxPending;
+    uint64_t *cbar = adone + 1;
     volatile int *abort_flag = &ctl.abort;
     unsigned char *qarea = smem + p.off_q;
     unsigned char *stage_base = smem + p.off_stage;
@@ -1098,63 +1393,125 @@ __global__ void __launch_bounds__(kDecodeThreads, 1) paged_decode_kernel(const _
             mbar_init(&qfull[i], 1);
             mbar_init(&qempty[i], kConsumerWarps);
         }
+        for (int i = 0; i < kMaxPending; ++i) mbar_init(&pdone[i], kConsumerWarps);
+        mbar_init(adone, 1);
+        mbar_init(cbar, kConsumerWarps);
         ctl.abort = 0;
         ctl.found_b = -1;
         fence_mbarrier_init();
     }
+    if (warp == kProducerWarp && lane == 0 && p.use_tmap) {
+        prefetch_tensormap(&p.tmap_k);
+        prefetch_tensormap(&p.tmap_v);
+    }
+    // everything below may read what the preceding grid on the stream wrote;
+    // the next grid may start its own prologue as soon as SMs free up
+    grid_dependency_wait();
+    grid_launch_dependents();
 
-    // ---- prologue: total units and this CTA's starting point ----
-    int64_t local = 0;
+    // ---- prologue: the cut of the work and this CTA's static slice ----
+    const int cap = p.max_blocks * p.bs;
+    const bool may_dyn = p.mode == PA_SPLIT_BALANCED && p.dyn_num > 0 && p.B <= kPrefixCache && p.lens_cached;
+    int64_t t_local = 0, d_local = 0;
     for (int b = tid; b < p.B; b += kDecodeThreads) {
         const int raw = p.context_lens[b];
-        if (blockIdx.x == 0 && (raw < 0 || raw > p.max_blocks * p.bs)) set_error(p.error, PA_DEVERR_CONTEXT_LEN);
+        if (blockIdx.x == 0 && (raw < 0 || raw > cap)) set_error(p.error, PA_DEVERR_CONTEXT_LEN);
         if (p.lens_cached) lens_s[b] = raw;
-        const int cap = p.max_blocks * p.bs;
-        local += units_of_len(p, raw < 0 ? 0 : (raw > cap ? cap : raw));
+        const int nu = units_of_len(p, raw < 0 ? 0 : (raw > cap ? cap : raw));
+        t_local += nu;
+        if (may_dyn) d_local += dyn_units(nu, p.dyn_num);
     }
 #pragma unroll
-    for (int m = 16; m >= 1; m >>= 1) local += __shfl_xor_sync(0xffffffffu, local, m);
-    if (lane == 0) ctl.red[warp] = local;
+    for (int m = 16; m >= 1; m >>= 1) {
+        t_local += __shfl_xor_sync(0xffffffffu, t_local, m);
+        d_local += __shfl_xor_sync(0xffffffffu, d_local, m);
+    }
+    if (lane == 0) {
+        ctl.red[warp][0] = t_local;
+        ctl.red[warp][1] = d_local;
+    }
     __syncthreads();
     if (tid == 0) {
-        int64_t t = 0;
-        for (int w = 0; w <= kConsumerWarps; ++w) t += ctl.red[w];
-        ctl.total = t * p.NHG;
+        int64_t tq = 0, dq = 0;
+        for (int w = 0; w < NWARPS; ++w) {
+            tq += ctl.red[w][0];
+            dq += ctl.red[w][1];
+        }
+        const int64_t NT = tq * p.NHG;
+        const int64_t C = p.num_ctas;
+        Cut k;
+        k.dyn = may_dyn && dq > 0 && NT >= 4 * C && NT < (int64_t(1) << 30);
+        k.Dn = k.dyn ? dq * p.NHG : 0;
+        k.S = NT - k.Dn;
+        k.Cn = k.S < C ? (k.S > 0 ? k.S : 1) : C;
+        k.g = (NT + 8 * C - 1) / (8 * C);
+        if (k.g < 1) k.g = 1;
+        k.J = k.dyn ? (k.Dn + k.g - 1) / k.g : 0;
+        ctl.cut = k;
     }
     __syncthreads();
-    const int64_t NT = ctl.total;
-    // ranges are cut among min(num_ctas, NT) CTAs so none is empty; the rest idle
-    const int64_t Cn = NT < p.num_ctas ? (NT > 0 ? NT : 1) : p.num_ctas;
-    const int64_t lo = (NT > 0 && blockIdx.x < Cn) ? range_lo(blockIdx.x, NT, Cn) : 0;
-    const int64_t hi = (NT > 0 && blockIdx.x < Cn) ? range_lo(blockIdx.x + 1, NT, Cn) : 0;
+    const Cut cut = ctl.cut;
+    const bool has_slice = cut.S > 0 && blockIdx.x < cut.Cn;
+    const int64_t lo = has_slice ? slice_lo(blockIdx.x, cut) : 0;
+    const int64_t hi = has_slice ? slice_lo(blockIdx.x + 1, cut) : 0;
 
-    if (lo < hi) {
-        int64_t running = 0;
+    // exclusive prefix sums of static / dynamic units over requests: the
+    // request holding this CTA's first unit, and (dynamic list) the tables
+    // the grains are located with
+    if (lo < hi || cut.dyn) {
+        int64_t run_s = 0, run_d = 0;
         for (int base = 0; base < p.B; base += kDecodeThreads) {
             const int b = base + tid;
-            const int64_t u = (b < p.B) ? (int64_t)p.NHG * units_of_len(p, clamped_len(p, lens_s, b)) : 0;
-            int64_t x = u;
+            int64_t us = 0, ud = 0;
+            if (b < p.B) {
+                const int nu = units_of_len(p, clamped_len(p, lens_s, b));
+                const int d = cut.dyn ? dyn_units(nu, p.dyn_num) : 0;
+                us = (int64_t)p.NHG * (nu - d);
+                ud = (int64_t)p.NHG * d;
+            }
+            int64_t xs = us, xd = ud;
 #pragma unroll
             for (int m = 1; m < 32; m <<= 1) {
-                const int64_t y = __shfl_up_sync(0xffffffffu, x, m);
-                if (lane >= m) x += y;
+                const int64_t ys = __shfl_up_sync(0xffffffffu, xs, m);
+                const int64_t yd = __shfl_up_sync(0xffffffffu, xd, m);
+                if (lane >= m) {
+                    xs += ys;
+                    xd += yd;
+                }
             }
             __syncthreads();  // ctl.red free to overwrite
-            if (lane == 31) ctl.red[warp] = x;
-            __syncthreads();
-            int64_t before = 0, chunk = 0;
-            for (int w = 0; w <= kConsumerWarps; ++w) {
-                if (w < warp) before += ctl.red[w];
-                chunk += ctl.red[w];
+            if (lane == 31) {
+                ctl.red[warp][0] = xs;
+                ctl.red[warp][1] = xd;
             }
-            const int64_t excl = running + before + x - u;
-            if (u > 0 && excl <= lo && lo < excl + u) {
+            __syncthreads();
+            int64_t bs_ = 0, bd_ = 0, cs = 0, cd = 0;
+            for (int w = 0; w < NWARPS; ++w) {
+                if (w < warp) {
+                    bs_ += ctl.red[w][0];
+                    bd_ += ctl.red[w][1];
+                }
+                cs += ctl.red[w][0];
+                cd += ctl.red[w][1];
+            }
+            const int64_t es = run_s + bs_ + xs - us, ed = run_d + bd_ + xd - ud;
+            if (cut.dyn && b < p.B) {
+                pre_s[b] = (int)es;
+                pre_d[b] = (int)ed;
+            }
+            if (us > 0 && es <= lo && lo < es + us) {
                 ctl.found_b = b;
-                ctl.found_excl = excl;
+                ctl.found_excl = es;
+                ctl.found_dexcl = ed;
             }
-            running += chunk;
+            run_s += cs;
+            run_d += cd;
             __syncthreads();
-            if (ctl.found_b >= 0) break;
+            if (!cut.dyn && ctl.found_b >= 0) break;
+        }
+        if (cut.dyn && tid == 0) {
+            pre_s[p.B] = (int)cut.S;
+            pre_d[p.B] = (int)cut.Dn;
         }
     }
     __syncthreads();
@@ -1162,35 +1519,55 @@ __global__ void __launch_bounds__(kDecodeThreads, 1) paged_decode_kernel(const _
     SegIter it;
     it.cur = lo;
     it.hi = hi;
-    it.lo = lo;
-    it.NT = NT;
-    it.C = Cn;
     it.lens_s = lens_s;
     if (lo < hi) {
         it.b = (int)ctl.found_b;
-        it.L = clamped_len(p, lens_s, it.b);
-        it.units = units_of_len(p, it.L);
-        it.hg = (int)((lo - ctl.found_excl) / it.units);
-        it.vr_start = ctl.found_excl + (int64_t)it.hg * it.units;
+        it.load_request(p, cut);
+        it.hg = (int)((lo - ctl.found_excl) / it.su);
+        it.vr_start = ctl.found_excl + (int64_t)it.hg * it.su;
+        it.ds = ctl.found_dexcl + (int64_t)it.hg * it.du;
     } else {
         it.b = 0;
         it.hg = 0;
         it.L = 0;
-        it.units = 0;
+        it.su = 0;
+        it.du = 0;
         it.vr_start = 0;
+        it.ds = 0;
     }
 
-    if (warp == kConsumerWarps) {
-        run_producer<D, E>(p, it, full, empty, qfull, qempty, qarea, stage_base, abort_flag, lane);
+    if (warp == kProducerWarp) {
+        run_producer<D, E>(p, cut, it, ctl, lens_s, pre_s, pre_d, full, empty, qfull, qempty, qarea, stage_base,
+                           abort_flag, lane);
+        return;
+    }
+    if (warp == kArrivalWarp) {
+        run_arrivals(p, ctl, pdone, adone, abort_flag, lane);
         return;
     }
 
     // ================= consumer warps =================
-    // requests with no tokens: out = 0
+    constexpr int NTH = kConsumerWarps * 32;
+    // requests with no tokens: out = 0 (a fused step still appends their token)
     for (int b = blockIdx.x; b < p.B; b += p.num_ctas) {
         if (clamped_len(p, lens_s, b) != 0) continue;
         unsigned char *o = reinterpret_cast<unsigned char *>(p.out) + (size_t)b * p.Hq * D * E;
-        for (int i = tid; i < p.Hq * D / 8; i += kConsumerWarps * 32) Elem<T>::store_zero8(o + (size_t)i * 8 * E);
+        for (int i = tid; i < p.Hq * D / 8; i += NTH) Elem<T>::store_zero8(o + (size_t)i * 8 * E);
+        if (p.fused) {
+            const int sm = p.slot_mapping[b];
+            if (sm >= 0 && (int64_t)sm >= (int64_t)p.num_blocks * p.bs) {
+                if (tid == 0) set_error(p.error, PA_DEVERR_SLOT);
+            } else if (sm >= 0) {
+                const int nvec = p.Hkv * D * E / 16;
+                for (int i = tid; i < 2 * nvec; i += NTH) {
+                    const bool kk = i < nvec;
+                    const uint4 *src = reinterpret_cast<const uint4 *>(kk ? p.k_new : p.v_new) + (size_t)b * nvec;
+                    uint4 *dst = reinterpret_cast<uint4 *>(const_cast<void *>(kk ? p.k_cache : p.v_cache)) +
+                                 (size_t)sm * nvec;
+                    dst[i % nvec] = __ldg(src + i % nvec);
+                }
+            }
+        }
     }
 
     const int U = p.units;
@@ -1206,33 +1583,46 @@ __global__ void __launch_bounds__(kDecodeThreads, 1) paged_decode_kernel(const _
     eng.setup(lane);
     if constexpr (Engine::kPaddedRows) eng.nreal = p.G < 8 ? p.G : 8;
     typename Engine::Unit unit[UPW];
+    NewToken<D, E> nt[UPW];
     int u_g[UPW], u_h0[UPW];
+    bool u_writer[UPW];  // this warp stores the new token of the unit's KV head
 #pragma unroll
     for (int k = 0; k < UPW; ++k) {
         const int uid = (tsplit > 1) ? warp % U : warp + k * kConsumerWarps;
         u_g[k] = uid / units_per_g;                          // KV head within the group
         u_h0[k] = u_g[k] * p.G + (uid % units_per_g) * HC;   // first query head within the vr
+        u_writer[k] = split == 0 && uid % units_per_g == 0;
     }
 
+    ConsumerBarrier cb{cbar, 0u};
     int stage = 0;
     uint32_t phase = 0;
     int qslot = 0;
     uint32_t qphase = 0;
     int npend = 0;
-    Seg s;
-    while (it.next(p, s)) {
-        // -- q of this vr --
-        if (!*abort_flag && !mbar_wait(&qfull[qslot], qphase, abort_flag)) {
+    uint32_t adone_par = 0;
+    for (;;) {
+        // -- the next piece and its q --
+        if (!mbar_wait(&qfull[qslot], qphase, abort_flag)) {
             *abort_flag = 1;
             set_error(p.error, PA_DEVERR_TIMEOUT);
+            break;
         }
+        const Seg s = ctl.segs[qslot];
+        if (s.b < 0) break;
         const unsigned char *qs = qarea + qslot * p.q_bytes;
 #pragma unroll
         for (int k = 0; k < UPW; ++k) eng.init_unit(unit[k], qs, u_h0[k], p.qscale);
+        if (s.append_slot >= 0) {
+#pragma unroll
+            for (int k = 0; k < UPW; ++k) nt[k].load(p, s.b, s.hg * p.HG + u_g[k], lane);
+        }
         __syncwarp();
         if (lane == 0) mbar_arrive(&qempty[qslot]);
         qslot ^= 1;
         if (qslot == 0) qphase ^= 1u;
+        const int patch_tile = s.patch >= 0 ? s.patch / p.ST : -1;
+        const int patch_tok = s.patch - patch_tile * p.ST;
 
         // -- tiles --
         for (int t = s.t_begin; t < s.t_end; ++t) {
@@ -1246,6 +1636,10 @@ __global__ void __launch_bounds__(kDecodeThreads, 1) paged_decode_kernel(const _
                 const int ntok = min(p.ST, s.L - t * p.ST);
                 for (int st = split; st * kSubTile < ntok; st += tsplit) {
                     const int nvalid = min(kSubTile, ntok - st * kSubTile);
+                    if (t == patch_tile && st == patch_tok / kSubTile) {
+#pragma unroll
+                        for (int k = 0; k < UPW; ++k) nt[k].patch(kst, vst, patch_tok, u_g[k], p, lane);
+                    }
 #pragma unroll
                     for (int k = 0; k < UPW; ++k)
                         eng.subtile(unit[k], kst, vst, st, u_g[k], nvalid, p, s_sm, p_sm, lane);
@@ -1262,18 +1656,23 @@ __global__ void __launch_bounds__(kDecodeThreads, 1) paged_decode_kernel(const _
         // -- finish the piece --
 #pragma unroll
         for (int k = 0; k < UPW; ++k) eng.finish_unit(unit[k]);
+        if (s.append_slot >= 0 && !*abort_flag) {
+#pragma unroll
+            for (int k = 0; k < UPW; ++k)
+                if (u_writer[k]) nt[k].store(p, s.append_slot, s.hg * p.HG + u_g[k], lane);
+        }
 
         if (tsplit > 1) {
             // warps of split > 0 hand their state to the split-0 warp of the same unit
             float *comb = reinterpret_cast<float *>(smem + p.off_comb + warp * p.comb_stride);
             if (split > 0) eng.save(unit[0], comb, lane);
-            named_barrier(1, kConsumerWarps * 32);
+            cb.sync(abort_flag, lane);
             if (split == 0)
                 for (int s2 = 1; s2 < tsplit; ++s2)
                     eng.absorb(unit[0],
                                reinterpret_cast<const float *>(smem + p.off_comb + (warp + s2 * U) * p.comb_stride),
                                lane);
-            named_barrier(1, kConsumerWarps * 32);
+            cb.sync(abort_flag, lane);
         }
 
         const bool writer = (split == 0);
@@ -1287,10 +1686,8 @@ __global__ void __launch_bounds__(kDecodeThreads, 1) paged_decode_kernel(const _
             continue;
         }
 
-        // partial piece: leave (m, l, o) in the slot and count its arrival.
-        // Only thread 0 fences and bumps the counter (after a barrier, as a
-        // grid-wide sync does); the other warps go on with the next tile.  A
-        // vr whose last piece this was is merged when the CTA is done.
+        // partial piece: leave (m, l, o) in the slot; the arrival warp counts
+        // it once every consumer warp has stored its part
         const bool slot_ok = s.slot < p.max_slots;
         if (writer && slot_ok) {
             float *base = p.partials + s.slot * p.slot_floats;
@@ -1298,19 +1695,20 @@ __global__ void __launch_bounds__(kDecodeThreads, 1) paged_decode_kernel(const _
             for (int k = 0; k < UPW; ++k) eng.write_partial(unit[k], base, p.NHvr, u_h0[k]);
         }
         if (!slot_ok && tid == 0) set_error(p.error, PA_DEVERR_WORKSPACE);
-        named_barrier(1, kConsumerWarps * 32);
-        if (tid == 0) {
-            __threadfence();
-            const int prev = atomicAdd(&p.counters[(int64_t)s.b * p.NHG + s.hg], 1);
-            ctl.pending[npend] = s;
-            ctl.last[npend] = (prev == s.nparts - 1);
-        }
+        __syncwarp();
+        if (tid == 0) ctl.pending[npend] = s;
+        if (lane == 0) mbar_arrive(&pdone[npend]);
         if (++npend == kMaxPending) {
-            flush_pending<T, D>(p, ctl, npend, NT, Cn, msm, tid);
+            flush_pending<T, D>(p, ctl, npend, adone, adone_par, abort_flag, msm, cb, tid);
+            adone_par ^= 1u;
             npend = 0;
         }
     }
-    if (npend) flush_pending<T, D>(p, ctl, npend, NT, Cn, msm, tid);
+    // close the list for the arrival warp, then merge what this CTA completed
+    if (tid == 0) ctl.pending[npend].b = -1;
+    __syncwarp();
+    if (lane == 0) mbar_arrive(&pdone[npend]);
+    flush_pending<T, D>(p, ctl, npend, adone, adone_par, abort_flag, msm, cb, tid);
 }
 
 }  // namespace pa

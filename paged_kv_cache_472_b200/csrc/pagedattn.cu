@@ -35,8 +35,17 @@ bool tensor_core_dtype(int dtype) { return dtype == PA_DTYPE_BF16 || dtype == PA
 size_t round_up(size_t x, size_t a) { return (x + a - 1) / a * a; }
 
 constexpr int kSmemLimit = 232448;     // opt-in shared memory per CTA on sm_100 (static + dynamic)
-constexpr int kStaticSmem = 4096 + 1536;  // lengths cache and control block (pending list)
-constexpr size_t kWsHeader = 256;      // error word + reserved
+// the decode kernel's static shared memory: control block, lengths and prefix-sum caches
+constexpr int kStaticSmem = (int)sizeof(pa::DecodeCtl) + 4 * pa::kLensCache + 8 * (pa::kPrefixCache + 1) + 256;
+constexpr size_t kWsHeader = 256;      // error word, dynamic-list counters
+constexpr size_t kWsGrab = 64;         // header offset of the grains-handed-out counter
+constexpr size_t kWsGrabDone = 128;    // header offset of the finished-CTA counter
+// Balanced mode: share of each vr's tiles handed out at run time (0 = none).
+// Grains of ~1/8 of a CTA's share cost a cold block-table fetch and a partial
+// each; measured on the Qwen3-0.6B-shaped batch they lose more than the
+// balance gains, so the planner leaves the list static unless asked.
+constexpr int kDynamicShare = 0;
+constexpr int kMaxDynamicShare = 64;
 constexpr int kStageTargetBytes = 32768;  // K bytes per stage (V the same)
 constexpr int kMaxStages = 4;
 
@@ -119,7 +128,7 @@ Layout smem_layout(int dtype, int D, int stages, uint32_t q_bytes, uint32_t half
     Layout l;
     const bool mma = tensor_core_dtype(dtype);
     l.off_bar = 0;
-    const uint32_t bar_bytes = (uint32_t)round_up((2 * stages + 4) * 8, 128);
+    const uint32_t bar_bytes = (uint32_t)round_up((2 * stages + 4 + pa::kMaxPending + 2) * 8, 128);
     l.off_q = bar_bytes;
     l.off_stage = (uint32_t)round_up(l.off_q + 2 * q_bytes, 1024);
     l.off_scratch = (uint32_t)round_up(l.off_stage + (size_t)stages * 2 * half_bytes, 128);
@@ -129,7 +138,7 @@ Layout smem_layout(int dtype, int D, int stages, uint32_t q_bytes, uint32_t half
     l.comb_stride = comb_floats * 4;
     const uint32_t comb = tsplit > 1 ? pa::kConsumerWarps * l.comb_stride : 0;
     l.off_merge = (uint32_t)round_up(l.off_comb + comb, 128);
-    const uint32_t merge = (uint32_t)(2 * pa::kMergeParts + pa::kMergeParts * nhvr + nhvr) * 4;
+    const uint32_t merge = (uint32_t)pa::kMergeParts * 8;  // slot list of the vr being merged
     // + 1024: the kernel rounds its dynamic base up to a 1024-byte boundary
     l.total = (uint32_t)round_up(l.off_merge + merge, 128) + 1024;
     return l;
@@ -244,12 +253,20 @@ int log2i(int x) {
     return l;
 }
 
+// The fused step (k_new != NULL) appends each request's new token in the
+// same launch.  Every launch may start while the preceding grid on the stream
+// finishes (programmatic dependent launch): the kernel waits for that grid
+// before its first global memory access.
 pa_status launch_decode(const void *q, const void *k_cache, const void *v_cache, const int32_t *block_tables,
                         const int32_t *context_lens, float scale, void *out, const pa_shape *s,
                         const pa_plan_t *plan, void *workspace, size_t workspace_bytes, cudaStream_t stream,
-                        bool pdl) {
+                        const void *k_new, const void *v_new, const int32_t *slot_mapping) {
     if (!plan) return fail(PA_ERR_INVALID_ARG, "plan is NULL");
     if (memcmp(&plan->shape, s, sizeof *s) != 0) return fail(PA_ERR_INVALID_ARG, "plan was made for another shape");
+    if (plan->dynamic_share < 0 || plan->dynamic_share > kMaxDynamicShare ||
+        (plan->dynamic_share > 0 && (plan->mode != PA_SPLIT_BALANCED || s->B > pa::kPrefixCache)))
+        return fail(PA_ERR_INVALID_ARG, "dynamic_share=%d outside [0, %d] or not available for this plan",
+                    plan->dynamic_share, kMaxDynamicShare);
     if (!std::isfinite(scale)) return fail(PA_ERR_INVALID_ARG, "scale is not finite");
     if (!workspace) return fail(PA_ERR_WORKSPACE, "workspace is NULL");
     if (workspace_bytes < plan->workspace_bytes)
@@ -286,6 +303,13 @@ pa_status launch_decode(const void *q, const void *k_cache, const void *v_cache,
     unsigned char *ws = static_cast<unsigned char *>(workspace);
     const size_t counters = round_up((size_t)s->B * (s->Hkv / HG) * 4, 256);
     p.error = reinterpret_cast<int32_t *>(ws);
+    p.grab = reinterpret_cast<int32_t *>(ws + kWsGrab);
+    p.grab_done = reinterpret_cast<int32_t *>(ws + kWsGrabDone);
+    p.fused = k_new ? 1 : 0;
+    p.k_new = k_new;
+    p.v_new = v_new;
+    p.slot_mapping = slot_mapping;
+    p.dyn_num = plan->mode == PA_SPLIT_BALANCED ? plan->dynamic_share : 0;
     p.counters = reinterpret_cast<int32_t *>(ws + kWsHeader);
     p.partials = reinterpret_cast<float *>(ws + kWsHeader + counters);
     p.qscale = scale * 1.4426950408889634f;
@@ -307,7 +331,6 @@ pa_status launch_decode(const void *q, const void *k_cache, const void *v_cache,
     p.tsplit = TS;
     p.units = HG * (G / HC);
     p.heads_per_unit = HC;
-    p.pdl = pdl ? 1 : 0;
     p.max_slots = plan->max_slots;
     p.slot_floats = (int64_t)NHvr * s->D + (int64_t)round_up(2 * NHvr, 4);
     p.off_bar = lay.off_bar;
@@ -341,7 +364,7 @@ pa_status launch_decode(const void *q, const void *k_cache, const void *v_cache,
     attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
     attr[0].val.programmaticStreamSerializationAllowed = 1;
     cfg.attrs = attr;
-    cfg.numAttrs = pdl ? 1 : 0;
+    cfg.numAttrs = 1;
     cudaError_t ce = cudaLaunchKernelEx(&cfg, fn, p);
     if (ce == cudaSuccess) ce = cudaGetLastError();
     if (ce != cudaSuccess) return fail(PA_ERR_CUDA, "decode launch: %s", cudaGetErrorString(ce));
@@ -445,7 +468,14 @@ pa_status pa_plan(const pa_shape *s, int32_t max_context_len, int32_t partition_
     plan->smem_bytes = (int32_t)lay.total;
     plan->shape = *s;
     if (mode == PA_SPLIT_BALANCED) {
-        plan->max_slots = 2LL * num_sms;
+        // static piece (vr v, slice r): slot v + r; dynamic piece (vr v, grain j):
+        // NV + C + v + j with j < J <= 8*C*share/256 + 1
+        const int64_t NV = (int64_t)s->B * NHG, C = num_sms;
+        const bool dyn = s->B <= pa::kPrefixCache && s->B <= pa::kLensCache;
+        plan->dynamic_share = dyn ? kDynamicShare : 0;
+        // slots for the largest share a caller may set in the plan
+        const int64_t Jmax = 8 * C * kMaxDynamicShare / 256 + 1;
+        plan->max_slots = dyn ? 2 * NV + C + Jmax : NV + C;
     } else {
         const int64_t parts = (max_context_len + partition_tokens - 1) / partition_tokens;
         plan->max_slots = (int64_t)NHG * s->B * (parts > 1 ? parts : 0);
@@ -470,7 +500,7 @@ pa_status pa_decode(const void *q, const void *k_cache, const void *v_cache, con
                     void *workspace, size_t workspace_bytes, void *stream) {
     if (pa_status st = check_shape(s)) return st;
     if (pa_status st = launch_decode(q, k_cache, v_cache, block_tables, context_lens, scale, out, s, plan, workspace,
-                                     workspace_bytes, (cudaStream_t)stream, false))
+                                     workspace_bytes, (cudaStream_t)stream, nullptr, nullptr, nullptr))
         return st;
     return ok();
 }
@@ -484,11 +514,10 @@ pa_status pa_kv_append_decode(const void *k_new, const void *v_new, const int32_
     if (!workspace || workspace_bytes < (plan ? plan->workspace_bytes : 0) ||
         (reinterpret_cast<uintptr_t>(workspace) & 255u) != 0)
         return fail(PA_ERR_WORKSPACE, "workspace missing, too small or not 256-byte aligned");
-    if (pa_status st = launch_append(k_new, v_new, slot_mapping, k_cache, v_cache, s,
-                                     static_cast<int32_t *>(workspace), (cudaStream_t)stream))
-        return st;
+    if (!k_new || !v_new || !slot_mapping) return fail(PA_ERR_INVALID_ARG, "NULL tensor pointer");
+    if (!aligned16(k_new) || !aligned16(v_new)) return fail(PA_ERR_INVALID_ARG, "value tensors must be 16-byte aligned");
     if (pa_status st = launch_decode(q, k_cache, v_cache, block_tables, context_lens, scale, out, s, plan, workspace,
-                                     workspace_bytes, (cudaStream_t)stream, true))
+                                     workspace_bytes, (cudaStream_t)stream, k_new, v_new, slot_mapping))
         return st;
     return ok();
 }
@@ -556,7 +585,7 @@ extern "C" pa_status pa_decode_no_alloc(const void *q, const void *k_cache, cons
     cudaError_t e = cudaMemsetAsync(ws, 0, kWsHeader + counters, (cudaStream_t)stream);
     if (e != cudaSuccess) return fail(PA_ERR_CUDA, "cudaMemsetAsync: %s", cudaGetErrorString(e));
     if (pa_status st = launch_decode(q, k_cache, v_cache, block_tables, context_lens, scale, out, s, plan, ws,
-                                     kNoAllocWorkspaceBytes, (cudaStream_t)stream, false))
+                                     kNoAllocWorkspaceBytes, (cudaStream_t)stream, nullptr, nullptr, nullptr))
         return st;
     return ok();
 }

@@ -61,7 +61,11 @@ def test_plan_workloads(cid):
     if c.partition_tokens:
         assert plan.mode == pa.SPLIT_FIXED and plan.partition_tokens % plan.tile_tokens == 0
     else:
-        assert plan.mode == pa.SPLIT_BALANCED and plan.max_slots == 2 * 148
+        # static piece (vr v, slice r) -> slot v + r; dynamic piece (vr v, grain j) -> NV + C + v + j,
+        # with at most 8*C*share/256 + 1 grains
+        NV = c.B * (c.Hkv // plan.head_group)
+        assert plan.mode == pa.SPLIT_BALANCED and plan.dynamic_share == 0
+        assert plan.max_slots == 2 * NV + 148 + 8 * 148 * 64 // 256 + 1
     expect = {1: (2, 1, 2), 2: (8, 2, 1), 3: (8, 4, 1), 4: (1, 8, 2), 5: (8, 4, 1)}[cid]
     assert (plan.head_group, plan.heads_per_unit, plan.warps_per_unit) == expect
 
@@ -157,3 +161,14 @@ def test_append_validation_paths():
     s0 = pa.Shape(0, 8, 2, 128, 16, 8, 4, pa.DTYPE_BF16)
     assert f(0, 0, 0, 0, 0, ctypes.byref(s0), None, None) == pa.PA_OK
     assert f(FAKE, FAKE, FAKE, FAKE, FAKE, None, None, None) == pa.PA_ERR_INVALID_ARG
+
+
+@pytest.mark.parametrize("share,mode_fixed", [(-1, False), (65, False), (16, True)])
+def test_decode_rejects_bad_dynamic_share(share, mode_fixed):
+    """The plan's dynamic share is checked before anything reaches the GPU."""
+    s = pa.Shape(2, 8, 2, 128, 16, 8, 4, pa.DTYPE_BF16)
+    plan = pa.pa_plan(s, 64, 16 if mode_fixed else 0, 148)
+    plan.dynamic_share = share
+    with pytest.raises(pa.PagedAttnError) as ei:
+        pa.pa_decode(0, 0, 0, 0, 0, 0.1, 0, s, plan, 0, 0, stream=0)
+    assert ei.value.status == pa.PA_ERR_INVALID_ARG

@@ -4,6 +4,7 @@ Full outputs at sizes the oracle finishes in seconds (several tiles, ragged
 tails, every split mode); sampled (request, head) outputs at the full sizes
 of the five workloads, in the launch configuration the benchmark times
 (balanced split, one CTA per SM)."""
+import dataclasses
 import zlib
 
 import numpy as np
@@ -11,7 +12,7 @@ import pytest
 import torch
 
 import synth
-from paged_kv_cache_472_b200 import DEVERR_BLOCK_ID, DEVERR_CONTEXT_LEN
+from paged_kv_cache_472_b200 import DEVERR_BLOCK_ID, DEVERR_CONTEXT_LEN, DEVERR_SLOT
 from tests import gpu_harness as H
 
 pytestmark = pytest.mark.gpu
@@ -177,6 +178,35 @@ def test_repeated_calls_reuse_workspace(orc):
     assert dec.device_error() == 0
     counters = dec.workspace[256:256 + 4 * case.B * case.Hkv].view(torch.int32)
     assert int(counters.abs().sum()) == 0
+    header = dec.workspace[:256].view(torch.int32)   # error word, dynamic-list counters
+    assert int(header.abs().sum()) == 0
+
+
+def test_dynamic_grains_match_static_split(orc):
+    """The same batch with a quarter of every request's tiles handed out at run
+    time and with a purely static split: both match the oracle, and repeated
+    calls (different CTAs taking different grains) are bit-identical."""
+    case = synth.make_config(2)
+    ref = oracle_out(orc, case)
+    outs = []
+    for share in (64, 0):
+        dev = H.upload(case)
+        dec = H.PagedDecoder(H.shape_of(case), int(case.context_lens.max()), 0)
+        assert dec.plan.dynamic_share == 0
+        dec.plan.dynamic_share = share
+        dec.append(dev.k_new, dev.v_new, dev.slot_mapping, dev.k_cache, dev.v_cache)
+        first = None
+        for _ in range(4):
+            dev.out.fill_(float("nan"))
+            dec.decode(dev.q, dev.k_cache, dev.v_cache, dev.block_tables, dev.context_lens, case.scale, dev.out)
+            torch.cuda.synchronize()
+            if first is None:
+                first = dev.out.clone()
+            assert torch.equal(first, dev.out)
+        assert dec.device_error() == 0
+        assert int(dec.workspace[:256].view(torch.int32).abs().sum()) == 0
+        H.assert_close(H.out_f64(dev), ref, case.dtype, f"dynamic share {share}")
+        outs.append(H.out_f64(dev))
 
 
 def test_fp16_workload_shape(orc):
@@ -190,8 +220,9 @@ def test_fp16_workload_shape(orc):
 
 @pytest.mark.parametrize("cid,batch", [(2, None), (3, 32), (5, 48), (1, None)])
 def test_fused_append_decode_matches_separate_calls(orc, cid, batch):
-    """pa_kv_append_decode (decode chained to the append by programmatic
-    dependent launch) gives bit-identical results to the two separate calls."""
+    """pa_kv_append_decode (one launch: the new token is written to its slot
+    and patched into the staged tile) gives bit-identical results to the two
+    separate calls."""
     case = synth.make_config(cid, batch=batch)
     dev_a, dec_a, err_a = H.run(case, 0)
     dev_b = H.upload(case)
@@ -204,3 +235,74 @@ def test_fused_append_decode_matches_separate_calls(orc, cid, batch):
     assert torch.equal(dev_a.k_cache, dev_b.k_cache) and torch.equal(dev_a.v_cache, dev_b.v_cache)
     assert torch.equal(dev_a.out, dev_b.out)
     H.assert_close(H.out_f64(dev_b), oracle_out(orc, case), case.dtype, "fused")
+
+
+def _free_slot(case) -> int:
+    used = set(int(x) for x in case.block_tables.ravel() if x >= 0)
+    free = [b for b in range(case.num_blocks) if b not in used]
+    assert free, "the pool has no unused block"
+    return free[0] * case.block_size + 3
+
+
+def test_fused_step_flags_a_slot_that_is_not_the_last_position(orc):
+    """A new token sent to another slot than its request's last position: the
+    fused step still writes it there, decodes from the cache as it stands and
+    reports PA_DEVERR_SLOT (its contract); nothing faults."""
+    base = synth.build_case("foreign_slot", dtype="bf16", Hq=16, Hkv=8, D=128, block_size=16,
+                            context_lens=[300, 41, 900], seed=21, pool="factor", pool_factor=1.5)
+    sm = base.slot_mapping.copy()
+    sm[1] = _free_slot(base)
+    case = dataclasses.replace(base, slot_mapping=sm)
+    dev = H.upload(case)
+    dec = H.PagedDecoder(H.shape_of(case), int(case.context_lens.max()), 0)
+    dec.append_decode(dev.k_new, dev.v_new, dev.slot_mapping, dev.q, dev.k_cache, dev.v_cache, dev.block_tables,
+                      dev.context_lens, case.scale, dev.out)
+    torch.cuda.synchronize()
+    assert dec.device_error() & DEVERR_SLOT
+    kc, vc = orc.kv_append(case)
+    assert H.pool_equal(dev.k_cache, kc, case.dtype) and H.pool_equal(dev.v_cache, vc, case.dtype)
+    H.assert_close(H.out_f64(dev), orc.decode(case, kc, vc), case.dtype, "foreign slot")
+
+
+def test_fused_step_appends_for_zero_length_requests(orc):
+    """context_lens[b] = 0 with a slot: out[b] = 0 and the token still lands."""
+    base = synth.build_case("zero_append", dtype="bf16", Hq=16, Hkv=8, D=128, block_size=16,
+                            context_lens=[70, 1, 200], seed=22, pool="factor", pool_factor=1.5)
+    lens = base.context_lens.copy()
+    lens[1] = 0
+    sm = base.slot_mapping.copy()
+    sm[1] = _free_slot(base)
+    case = dataclasses.replace(base, context_lens=lens, slot_mapping=sm)
+    dev = H.upload(case)
+    dec = H.PagedDecoder(H.shape_of(case), 200, 0)
+    dec.append_decode(dev.k_new, dev.v_new, dev.slot_mapping, dev.q, dev.k_cache, dev.v_cache, dev.block_tables,
+                      dev.context_lens, case.scale, dev.out)
+    torch.cuda.synchronize()
+    assert dec.device_error() == 0
+    kc, vc = orc.kv_append(case)
+    assert H.pool_equal(dev.k_cache, kc, case.dtype) and H.pool_equal(dev.v_cache, vc, case.dtype)
+    got = H.out_f64(dev)
+    assert np.all(got[1] == 0.0)
+    H.assert_close(got, orc.decode(case, kc, vc), case.dtype, "zero-length append")
+
+
+@pytest.mark.parametrize("name,dtype,Hq,Hkv,D,bs,lens,pt", [
+    ("fused_f32", "f32", 16, 4, 128, 32, [129, 500, 31, 1], 0),
+    ("fused_mqa32", "bf16", 32, 1, 128, 256, [3000, 257, 1], 0),
+    ("fused_tsplit", "bf16", 4, 1, 128, 64, [700, 64, 65], 0),
+    ("fused_fixed", "bf16", 16, 8, 128, 16, [1000, 17, 513], 256),
+    ("fused_f16_d64", "f16", 32, 8, 64, 32, [513, 64, 2], 0),
+])
+def test_fused_step_edge_shapes(orc, name, dtype, Hq, Hkv, D, bs, lens, pt):
+    """The fused step on engines, layouts and splits the workloads do not reach."""
+    case = synth.build_case(name, dtype=dtype, Hq=Hq, Hkv=Hkv, D=D, block_size=bs, context_lens=lens,
+                            seed=zlib.crc32(name.encode()) % 100000, pool="factor", pool_factor=1.25)
+    dev = H.upload(case)
+    dec = H.PagedDecoder(H.shape_of(case), int(max(lens)), pt)
+    dec.append_decode(dev.k_new, dev.v_new, dev.slot_mapping, dev.q, dev.k_cache, dev.v_cache, dev.block_tables,
+                      dev.context_lens, case.scale, dev.out)
+    torch.cuda.synchronize()
+    assert dec.device_error() == 0
+    kc, vc = orc.kv_append(case)
+    assert H.pool_equal(dev.k_cache, kc, case.dtype) and H.pool_equal(dev.v_cache, vc, case.dtype)
+    H.assert_close(H.out_f64(dev), oracle_out(orc, case), case.dtype, name)
