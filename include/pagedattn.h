@@ -86,7 +86,7 @@ typedef struct {
     int32_t heads_per_unit;   /* query heads one warp carries */
     int32_t units_per_warp;
     int32_t warps_per_unit;   /* >1: a warp team splits the tokens of one unit */
-    int32_t max_context_len;  /* the bound the workspace was sized for */
+    int32_t max_context_len;  /* the longest context the plan was made for */
     int32_t smem_bytes;
     int32_t dynamic_share;    /* PA_SPLIT_BALANCED: share of each request's tiles handed out
                                  at run time to whichever CTA is free, in 1/256.  pa_plan
@@ -123,15 +123,21 @@ pa_status pa_kv_append(const void *k_new, const void *v_new, const int32_t *slot
 
 /*
  * Host-only planner (no device work, no allocation).
- *   max_context_len : the largest context_lens[b] any later call will pass;
- *                     bounds the workspace of PA_SPLIT_FIXED.
+ *   max_context_len : the largest context_lens[b] any later call will pass
+ *                     (at most max_blocks_per_seq*block_size); recorded in
+ *                     the plan.
  *   partition_tokens: 0 = PA_SPLIT_BALANCED (persistent CTAs with an equal
  *                     share of all requests' tokens each); > 0 =
  *                     PA_SPLIT_FIXED with partitions of that many tokens (a
- *                     multiple of 16); >= max_context_len gives one partition
- *                     per request (no split).
+ *                     multiple of 16), dealt to the CTAs in equal shares of
+ *                     whole partitions; the partitions of a request that one
+ *                     CTA takes are combined as they stream, the others by
+ *                     log-sum-exp; >= max_context_len gives one partition per
+ *                     request (no split).
  *   num_sms         : SM count to size the grid for; 0 = query the current
  *                     CUDA device.
+ * The workspace holds one partial result per (request, CTA) pair that can
+ * share a request, so its size does not depend on the context lengths.
  * Returns PA_ERR_UNSUPPORTED for shapes the kernels do not cover:
  * D not in {64, 128}; block_size not a power of two in [16, 256]; a GQA
  * group Hq/Hkv that is not a power of two <= 64; more query heads than one

@@ -162,6 +162,36 @@ __device__ __forceinline__ void set_error(int32_t *err, int32_t bits) {
     if (err) atomicOr(err, bits);
 }
 
+// Pull one line into L2.  A prefetch returns nothing to the thread, so it is
+// correct even on memory another grid is still writing.
+__device__ __forceinline__ void prefetch_l2(const void *p) {
+    asm volatile("prefetch.global.L2 [%0];" ::"l"(p));
+}
+
+// L2 prefetch of lines first, first + stride, ... of a buffer, at most `cap` of them.
+__device__ __forceinline__ void prefetch_l2_share(const void *base, size_t bytes, size_t first, size_t stride,
+                                                  int cap) {
+    const size_t lines = (bytes + 127) / 128;
+    const unsigned char *b = static_cast<const unsigned char *>(base);
+    for (size_t l = first; l < lines && cap > 0; l += stride, --cap) prefetch_l2(b + l * 128);
+}
+
+// atomicAdd with release and acquire semantics at GPU scope: the caller's
+// earlier writes (and those it has observed) are visible before the add, and
+// what other threads released before their adds is visible after it.
+__device__ __forceinline__ int atomic_add_acq_rel(int *p, int v) {
+    int old;
+    asm volatile("atom.acq_rel.gpu.global.add.s32 %0, [%1], %2;" : "=r"(old) : "l"(p), "r"(v) : "memory");
+    return old;
+}
+
+// floor(n / d) for 0 <= n < 2^53 and d >= 1, in double precision.  Exact: the
+// rounded quotient of n / d = k - delta (k an integer, delta >= 1/d) could
+// reach k only if delta were within half an ulp of k, i.e. d*k >= 2^53 > n.
+__device__ __forceinline__ int64_t floor_div_exact(int64_t n, int64_t d) {
+    return (int64_t)__double2ll_rz(__ddiv_rn((double)n, (double)d));
+}
+
 }  // namespace pa
 
 namespace pa {

@@ -20,8 +20,12 @@
 //     counter to whichever CTA is free, so that fast and slow SMs finish
 //     together.  The cut itself depends only on the lengths, so every CTA can
 //     name all pieces of a vr and their partial slots.
-//   * fixed mode: the static list is of partitions of `part_tiles` tiles (the
-//     classic flash-decoding split), divided the same way; nothing dynamic.
+//   * fixed mode: the units of the static list are partitions of `part_tiles`
+//     tiles (the classic flash-decoding split), divided the same way; nothing
+//     dynamic.  The partitions of a vr that fall in one CTA's slice are
+//     combined as they stream (the online softmax carried across the
+//     partition boundary is the log-sum-exp combination of the two), so a vr
+//     leaves one partial per CTA it touches, not one per partition.
 // A vr that lies wholly inside one piece is written straight to `out`.
 // Otherwise each piece leaves (m, l, o) in its workspace slot and bumps the
 // vr's counter; the CTA that arrives last combines the pieces by log-sum-exp
@@ -64,7 +68,6 @@ constexpr int kProducerWarp = kConsumerWarps;
 constexpr int kArrivalWarp = kConsumerWarps + 1;
 constexpr int kDecodeThreads = (kConsumerWarps + 2) * 32;
 constexpr int kSubTile = 16;     // tokens per online-softmax update
-constexpr int kMergeParts = 64;  // pieces the shared-memory merge path handles
 constexpr int kPrefixCache = 512;  // requests whose static / dynamic prefix sums live in shared memory
 
 struct DecodeParams {
@@ -99,7 +102,7 @@ struct DecodeParams {
     int32_t dyn_num;      // balanced mode: dynamic share of each vr, in 1/256 (0: all static)
     int64_t max_slots;
     int64_t slot_floats;  // NHvr * D + (2 * NHvr rounded up to a multiple of 4)
-    uint32_t off_bar, off_q, off_stage, off_scratch, off_comb, off_merge;
+    uint32_t off_bar, off_q, off_stage, off_scratch, off_comb;
     uint32_t row_bytes;   // HG * D * elem: one token of the head group
     uint32_t row_pitch;   // bytes between token rows in a stage (row_bytes, or + 16 for ldmatrix)
     uint32_t half_bytes;  // ST * row_pitch (K part of a stage; V part follows)
@@ -201,6 +204,21 @@ struct Elem<float> {
     }
 };
 
+// Read every scalar launch parameter once, so that the constant cache holds
+// them before the prologue's dependent chain starts.
+__device__ __forceinline__ void warm_params(const DecodeParams &p) {
+    asm volatile("" ::"l"(p.q), "l"(p.k_cache), "l"(p.v_cache), "l"(p.block_tables), "l"(p.context_lens),
+                 "l"(p.out), "l"(p.partials), "l"(p.counters));
+    asm volatile("" ::"l"(p.error), "l"(p.grab), "l"(p.grab_done), "l"(p.k_new), "l"(p.v_new), "l"(p.slot_mapping),
+                 "f"(p.qscale), "l"(p.max_slots), "l"(p.slot_floats));
+    asm volatile("" ::"r"(p.B), "r"(p.Hq), "r"(p.Hkv), "r"(p.bs), "r"(p.num_blocks), "r"(p.max_blocks), "r"(p.G),
+                 "r"(p.HG), "r"(p.NHG), "r"(p.NHvr), "r"(p.ST), "r"(p.stages), "r"(p.mode), "r"(p.part_tiles),
+                 "r"(p.num_ctas), "r"(p.tsplit), "r"(p.units), "r"(p.heads_per_unit), "r"(p.fused), "r"(p.dyn_num));
+    asm volatile("" ::"r"(p.off_bar), "r"(p.off_q), "r"(p.off_stage), "r"(p.off_scratch), "r"(p.off_comb),
+                 "r"(p.row_bytes), "r"(p.row_pitch), "r"(p.half_bytes), "r"(p.q_bytes), "r"(p.comb_stride),
+                 "r"(p.use_tmap), "r"(p.br_log2), "r"(p.bs_log2), "r"(p.lens_cached));
+}
+
 // ---------------------------------------------------------------------------
 // work list
 constexpr int kLensCache = 1024;  // requests whose lengths are kept in shared memory
@@ -230,9 +248,27 @@ struct Cut {
     int dyn;        // the dynamic list is in use
 };
 
-__device__ __forceinline__ int64_t slice_lo(int64_t r, const Cut &k) { return r * k.S / k.Cn; }
+// (positions and products stay far below 2^53, so the double quotients are exact)
+__device__ __forceinline__ int64_t slice_lo(int64_t r, const Cut &k) { return floor_div_exact(r * k.S, k.Cn); }
 // static slice holding static-list position x
-__device__ __forceinline__ int64_t slice_of(int64_t x, const Cut &k) { return ((x + 1) * k.Cn - 1) / k.S; }
+__device__ __forceinline__ int64_t slice_of(int64_t x, const Cut &k) {
+    return floor_div_exact((x + 1) * k.Cn - 1, k.S);
+}
+
+// The cut from the totals: tq units over all requests (one head group), dq of
+// them dynamic.
+__device__ __forceinline__ Cut make_cut(int64_t tq, int64_t dq, int NHG, int64_t C, bool may_dyn) {
+    const int64_t NT = tq * NHG;
+    Cut k;
+    k.dyn = may_dyn && dq > 0 && NT >= 4 * C && NT < (int64_t(1) << 30);
+    k.Dn = k.dyn ? dq * NHG : 0;
+    k.S = NT - k.Dn;
+    k.Cn = k.S < C ? (k.S > 0 ? k.S : 1) : C;
+    k.g = floor_div_exact(NT + 8 * C - 1, 8 * C);
+    if (k.g < 1) k.g = 1;
+    k.J = k.dyn ? floor_div_exact(k.Dn + k.g - 1, k.g) : 0;
+    return k;
+}
 
 struct Seg {
     int b, hg, L;         // b < 0: no more work
@@ -251,17 +287,26 @@ struct Seg {
 // earlier slice or grain, so no two pieces share a slot.
 __device__ __forceinline__ int balanced_parts(const Cut &k, int64_t ss, int s_len, int64_t ds, int d_len) {
     const int ns = (int)(slice_of(ss + s_len - 1, k) - slice_of(ss, k) + 1);
-    const int nd = d_len > 0 ? (int)((ds + d_len - 1) / k.g - ds / k.g + 1) : 0;
+    const int nd = d_len > 0 ? (int)(floor_div_exact(ds + d_len - 1, k.g) - floor_div_exact(ds, k.g) + 1) : 0;
     return ns + nd;
 }
 
-__device__ __forceinline__ int64_t piece_slot(const DecodeParams &p, const Cut &k, const Seg &s, int i) {
-    if (p.mode != PA_SPLIT_BALANCED) return s.ss + i;
+// Partial slots of the pieces of a vr: piece i < ns at a + i, the others at
+// b + (i - ns).
+struct PieceSlots {
+    int64_t a, b;
+    int ns;
+    __device__ __forceinline__ int64_t operator()(int i) const { return i < ns ? a + i : b + (i - ns); }
+};
+
+__device__ __forceinline__ PieceSlots piece_slots(const DecodeParams &p, const Cut &k, const Seg &s) {
+    PieceSlots r;
     const int64_t v = (int64_t)s.b * p.NHG + s.hg;
     const int64_t r0 = slice_of(s.ss, k);
-    const int ns = (int)(slice_of(s.ss + s.s_len - 1, k) - r0 + 1);
-    if (i < ns) return v + r0 + i;
-    return (int64_t)p.B * p.NHG + p.num_ctas + v + s.ds / k.g + (i - ns);
+    r.ns = (int)(slice_of(s.ss + s.s_len - 1, k) - r0 + 1);
+    r.a = v + r0;
+    r.b = (int64_t)p.B * p.NHG + p.num_ctas + v + (s.d_len > 0 ? floor_div_exact(s.ds, k.g) : 0);
+    return r;
 }
 
 // pieces of this CTA's static slice, in list order
@@ -301,21 +346,19 @@ struct SegIter {
             s.ds = ds;
             s.patch = -1;
             s.append_slot = -1;
+            // the run of this vr's units inside the slice is one piece
+            const int64_t end = vr_start + su < hi ? vr_start + su : hi;
+            u1 = (int)(end - vr_start);
             if (p.mode == PA_SPLIT_BALANCED) {
-                const int64_t end = vr_start + su < hi ? vr_start + su : hi;
-                u1 = (int)(end - vr_start);
                 s.t_begin = u0;
                 s.t_end = u1;
-                s.nparts = balanced_parts(k, vr_start, su, ds, du);
-                s.slot = (int64_t)b * p.NHG + hg + blockIdx.x;
             } else {
                 const int tiles = (L + p.ST - 1) / p.ST;
-                u1 = u0 + 1;
                 s.t_begin = u0 * p.part_tiles;
-                s.t_end = min(tiles, (u0 + 1) * p.part_tiles);
-                s.nparts = su;
-                s.slot = vr_start + u0;
+                s.t_end = min(tiles, u1 * p.part_tiles);
             }
+            s.nparts = balanced_parts(k, vr_start, su, ds, du);
+            s.slot = (int64_t)b * p.NHG + hg + blockIdx.x;
             cur = vr_start + u1;
             return true;
         }
@@ -899,6 +942,38 @@ struct ProducerState {
     int grab_val = 0;  // lane 0: result of the pending grab
 };
 
+// The block-table entries a piece reads, 32 at a time: lane i holds entry
+// base + i of the current window, and the next window is loaded one window
+// ahead.
+struct TableWindow {
+    const int32_t *table;
+    int nblk;
+    int cur_base, cur_val, nxt_base, nxt_val;
+
+    // load the window holding the piece's first tile (and the one after it)
+    __device__ __forceinline__ void prime(const DecodeParams &p, const Seg &s, int lane) {
+        table = p.block_tables + (size_t)s.b * p.max_blocks;
+        nblk = (s.L + p.bs - 1) >> p.bs_log2;
+        cur_base = ((s.t_begin * p.ST) >> p.bs_log2) & ~31;
+        cur_val = (cur_base + lane < nblk) ? table[cur_base + lane] : -1;
+        nxt_base = cur_base + 32;
+        nxt_val = (nxt_base + lane < nblk) ? table[nxt_base + lane] : -1;
+    }
+    // make the window holding block-table column jb current
+    __device__ __forceinline__ void advance(int jb, int lane) {
+        const int wb = jb & ~31;
+        if (wb == cur_base) return;
+        if (wb == nxt_base) {
+            cur_val = nxt_val;
+        } else {
+            cur_val = (wb + lane < nblk) ? table[wb + lane] : -1;
+        }
+        cur_base = wb;
+        nxt_base = wb + 32;
+        nxt_val = (nxt_base + lane < nblk) ? table[nxt_base + lane] : -1;  // one window ahead
+    }
+};
+
 // Fused step: if this piece holds the vr's last token, find where the new
 // token goes.  It is patched into the staged tile only when its slot is the
 // request's own last position; any other slot is reported.
@@ -908,7 +983,7 @@ __device__ __forceinline__ void fused_info(const DecodeParams &p, Seg &s, int la
     if (lane == 0) {
         sm = p.slot_mapping[s.b];
         const int t = s.L - 1;
-        const int phys = p.block_tables[(size_t)s.b * p.max_blocks + t / p.bs];
+        const int phys = p.block_tables[(size_t)s.b * p.max_blocks + (t >> p.bs_log2)];
         expect = (phys >= 0 && phys < p.num_blocks) ? phys * p.bs + (t & (p.bs - 1)) : -1;
     }
     sm = __shfl_sync(0xffffffffu, sm, 0);
@@ -950,17 +1025,15 @@ __device__ __forceinline__ void publish(const DecodeParams &p, ProducerState &ps
 // Fill one stage per tile of the piece.  With `grab_at_last`, the next grain
 // is requested while the piece's last tile is being issued.
 template <int D, int E>
-__device__ __forceinline__ void issue_tiles(const DecodeParams &p, ProducerState &ps, const Seg &s, bool grab_at_last,
-                                            uint64_t *full, uint64_t *empty, unsigned char *stage_base,
-                                            volatile int *abort_flag, uint64_t policy, int lane) {
+__device__ __forceinline__ void issue_tiles(const DecodeParams &p, ProducerState &ps, const Seg &s, TableWindow &win,
+                                            bool grab_at_last, uint64_t *full, uint64_t *empty,
+                                            unsigned char *stage_base, volatile int *abort_flag, uint64_t policy,
+                                            int lane) {
     const unsigned char *kc = reinterpret_cast<const unsigned char *>(p.k_cache);
     const unsigned char *vc = reinterpret_cast<const unsigned char *>(p.v_cache);
     const uint32_t row_bytes = p.row_bytes, pitch = p.row_pitch;
     const size_t tok_stride = (size_t)p.Hkv * D * E;  // bytes between token rows in the pool
     const bool contiguous = (p.HG == p.Hkv) && (pitch == row_bytes);
-    const int32_t *table = p.block_tables + (size_t)s.b * p.max_blocks;
-    const int nblk = (s.L + p.bs - 1) / p.bs;
-    int cur_base = -1, cur_val = -1, nxt_base = -1, nxt_val = -1;
     for (int t = s.t_begin; t < s.t_end; ++t) {
         if (!mbar_wait(&empty[ps.stage], ps.phase ^ 1u, abort_flag)) {
             ps.ok = false;
@@ -972,18 +1045,9 @@ __device__ __forceinline__ void issue_tiles(const DecodeParams &p, ProducerState
         }
         const int tok0 = t * p.ST;
         const int ntok = min(p.ST, s.L - tok0);
-        const int jb0 = tok0 / p.bs;
-        const int wb = jb0 & ~31;
-        if (wb != cur_base) {
-            if (wb == nxt_base) {
-                cur_val = nxt_val;
-            } else {
-                cur_val = (wb + lane < nblk) ? table[wb + lane] : -1;
-            }
-            cur_base = wb;
-            nxt_base = wb + 32;
-            nxt_val = (nxt_base + lane < nblk) ? table[nxt_base + lane] : -1;  // prefetch
-        }
+        const int jb0 = tok0 >> p.bs_log2;
+        win.advance(jb0, lane);
+        const int cur_base = win.cur_base, cur_val = win.cur_val;
         unsigned char *kdst = stage_base + (size_t)ps.stage * 2 * p.half_bytes;
         unsigned char *vdst = kdst + p.half_bytes;
         uint32_t bytes = 0;
@@ -1087,11 +1151,14 @@ __device__ __forceinline__ void run_producer(const DecodeParams &p, const Cut &k
     ProducerState ps;
     Seg s;
     // this CTA's static slice
+    TableWindow win;
     while (ps.ok && it.next(p, k, s)) {
+        win.prime(p, s, lane);  // in flight while q is published
         fused_info(p, s, lane);
         publish(p, ps, s, ctl, qfull, qempty, qarea, abort_flag, D, E, lane);
         if (!ps.ok) break;
-        issue_tiles<D, E>(p, ps, s, k.dyn && it.cur >= it.hi, full, empty, stage_base, abort_flag, policy, lane);
+        issue_tiles<D, E>(p, ps, s, win, k.dyn && it.cur >= it.hi, full, empty, stage_base, abort_flag, policy,
+                          lane);
     }
     // grains of the dynamic list, one at a time, to whichever CTA asks first
     if (k.dyn) {
@@ -1105,10 +1172,11 @@ __device__ __forceinline__ void run_producer(const DecodeParams &p, const Cut &k
             gi.y = j * k.g;
             gi.y1 = gi.y + k.g < k.Dn ? gi.y + k.g : k.Dn;
             while (ps.ok && gi.next(p, k, lens_s, pre_s, pre_d, s)) {
+                win.prime(p, s, lane);
                 fused_info(p, s, lane);
                 publish(p, ps, s, ctl, qfull, qempty, qarea, abort_flag, D, E, lane);
                 if (!ps.ok) break;
-                issue_tiles<D, E>(p, ps, s, gi.y >= gi.y1, full, empty, stage_base, abort_flag, policy, lane);
+                issue_tiles<D, E>(p, ps, s, win, gi.y >= gi.y1, full, empty, stage_base, abort_flag, policy, lane);
             }
         }
         // the last CTA to find the list empty leaves the counters at zero for the next launch
@@ -1137,28 +1205,22 @@ __device__ __forceinline__ void run_producer(const DecodeParams &p, const Cut &k
 
 // ===========================================================================
 // merge of a split vr by log-sum-exp (run by the consumer warps of the CTA
-// that delivered the last piece).  One pass per output element keeps a
-// running maximum, so any number of pieces is combined with eight pieces'
-// loads (o, m, l) in flight at a time.
+// that delivered the last piece):
+//     out[h] = sum_i 2^(m_i[h] - M[h]) o_i[h] / sum_i 2^(m_i[h] - M[h]) l_i[h],
+//     M[h] = max_i m_i[h]  (base-2 domain; pieces with m = -inf contribute 0).
 // ===========================================================================
+
+// From registers: one pass per output element keeps a running maximum, so any
+// number of pieces is combined with eight pieces' loads (o, m, l) in flight.
 template <typename T, int D>
-__device__ __forceinline__ void merge_vr(const DecodeParams &p, const Cut &cut, const Seg &s, float *msm,
-                                         ConsumerBarrier &cb, volatile int *abort_flag, int tid) {
+__device__ __forceinline__ void merge_vr(const DecodeParams &p, const Cut &cut, const Seg &s, int tid) {
     constexpr int E = Elem<T>::kBytes;
     constexpr int NTH = kConsumerWarps * 32;
     constexpr int KF = 8;  // pieces per batch of loads
     const int NH = p.NHvr;
     const int nparts = s.nparts;
     const size_t out_head0 = (size_t)s.b * p.Hq + (size_t)s.hg * NH;
-    int64_t *slot_s = reinterpret_cast<int64_t *>(msm);  // [kMergeParts]
-    const bool cached = nparts <= kMergeParts;
-    if (cached) {
-        for (int i = tid; i < nparts; i += NTH) {
-            const int64_t slot = piece_slot(p, cut, s, i);
-            slot_s[i] = slot < p.max_slots ? slot : -1;
-        }
-        cb.sync(abort_flag, tid & 31);
-    }
+    const PieceSlots slots = piece_slots(p, cut, s);
     const int nq = NH * (D / 4);
     for (int idx0 = tid; idx0 < nq; idx0 += 2 * NTH) {
         constexpr int IT = 2;  // output items per thread per batch
@@ -1183,7 +1245,7 @@ __device__ __forceinline__ void merge_vr(const DecodeParams &p, const Cut &cut, 
                 const int i = i0 + k;
                 int64_t slot = -1;
                 if (i < nparts) {
-                    slot = cached ? slot_s[i] : piece_slot(p, cut, s, i);
+                    slot = slots(i);
                     if (slot < 0 || slot >= p.max_slots) slot = -1;
                 }
                 sl[k] = slot;
@@ -1239,28 +1301,28 @@ __device__ __forceinline__ void merge_vr(const DecodeParams &p, const Cut &cut, 
             Elem<T>::store2(dst + 2 * E, num[j].z * inv, num[j].w * inv);
         }
     }
-    if (cached) cb.sync(abort_flag, tid & 31);  // the slot list is free again
 }
 
 // Merge every vr for which this CTA delivered the last piece.  The arrival
 // warp has counted the arrivals of pieces [0, npend) and signals `adone`
-// once it has; it fenced after every counter it found complete, so the other
-// CTAs' partials are visible to the loads below.
+// once it has; its counting atomics acquire what the other pieces' CTAs
+// released, so their partials are visible to the loads below.  `more`: more
+// pieces follow, so the pending list is handed back afterwards.
 template <typename T, int D>
 __device__ __forceinline__ bool flush_pending(const DecodeParams &p, DecodeCtl &ctl, int npend, uint64_t *adone,
-                                              uint32_t adone_par, volatile int *abort_flag, float *msm,
-                                              ConsumerBarrier &cb, int tid) {
+                                              uint32_t adone_par, volatile int *abort_flag, ConsumerBarrier &cb,
+                                              bool more, int tid) {
     const bool ok = mbar_wait(adone, adone_par, abort_flag);
     if (ok) {
         const Cut cut = ctl.cut;
         for (int k = 0; k < npend; ++k) {
             if (!ctl.last[k]) continue;
             const Seg sk = ctl.pending[k];
-            merge_vr<T, D>(p, cut, sk, msm, cb, abort_flag, tid);
+            merge_vr<T, D>(p, cut, sk, tid);
             if (tid == 0) p.counters[(int64_t)sk.b * p.NHG + sk.hg] = 0;
         }
     }
-    cb.sync(abort_flag, tid & 31);  // pending list free again
+    if (more) cb.sync(abort_flag, tid & 31);  // pending list free again
     return ok;
 }
 
@@ -1280,10 +1342,10 @@ __device__ __forceinline__ void run_arrivals(const DecodeParams &p, DecodeCtl &c
         const Seg s = ctl.pending[k];
         if (s.b < 0) break;
         if (lane == 0) {
-            __threadfence();  // the consumers' partial stores, seen through pdone, before the count
-            const int prev = atomicAdd(&p.counters[(int64_t)s.b * p.NHG + s.hg], 1);
+            // release: the consumers' partial stores, seen through pdone, before the
+            // count; acquire: every other piece's partial before the merge reads them
+            const int prev = atomic_add_acq_rel(&p.counters[(int64_t)s.b * p.NHG + s.hg], 1);
             const int last = prev == s.nparts - 1;
-            if (last) __threadfence();  // every other piece's partial before the merge reads them
             ctl.last[k] = last;
         }
         __syncwarp();
@@ -1404,6 +1466,23 @@ __global__ void __launch_bounds__(kDecodeThreads, 1) paged_decode_kernel(const _
         prefetch_tensormap(&p.tmap_k);
         prefetch_tensormap(&p.tmap_v);
     }
+    // ---- while the preceding grid may still run: nothing here reads its output ----
+    // Warm the constant cache with the launch parameters, and pull the first
+    // metadata reads of the prologue into L2: every CTA the lengths, and each
+    // CTA its share of the block tables, q and (fused step) the new tokens.
+    {
+        if (tid == 0) warm_params(p);
+        prefetch_l2_share(p.context_lens, (size_t)p.B * 4, tid, kDecodeThreads, 4);
+        const size_t first = (size_t)blockIdx.x * kDecodeThreads + tid;
+        const size_t stride = (size_t)gridDim.x * kDecodeThreads;
+        prefetch_l2_share(p.block_tables, (size_t)p.B * p.max_blocks * 4, first, stride, 2);
+        prefetch_l2_share(p.q, (size_t)p.B * p.Hq * D * E, first, stride, 2);
+        if (p.fused) {
+            prefetch_l2_share(p.slot_mapping, (size_t)p.B * 4, tid, kDecodeThreads, 4);
+            prefetch_l2_share(p.k_new, (size_t)p.B * p.Hkv * D * E, first, stride, 1);
+            prefetch_l2_share(p.v_new, (size_t)p.B * p.Hkv * D * E, first, stride, 1);
+        }
+    }
     // everything below may read what the preceding grid on the stream wrote;
     // the next grid may start its own prologue as soon as SMs free up
     grid_dependency_wait();
@@ -1412,90 +1491,56 @@ __global__ void __launch_bounds__(kDecodeThreads, 1) paged_decode_kernel(const _
     // ---- prologue: the cut of the work and this CTA's static slice ----
     const int cap = p.max_blocks * p.bs;
     const bool may_dyn = p.mode == PA_SPLIT_BALANCED && p.dyn_num > 0 && p.B <= kPrefixCache && p.lens_cached;
-    int64_t t_local = 0, d_local = 0;
-    for (int b = tid; b < p.B; b += kDecodeThreads) {
-        const int raw = p.context_lens[b];
-        if (blockIdx.x == 0 && (raw < 0 || raw > cap)) set_error(p.error, PA_DEVERR_CONTEXT_LEN);
-        if (p.lens_cached) lens_s[b] = raw;
-        const int nu = units_of_len(p, raw < 0 ? 0 : (raw > cap ? cap : raw));
-        t_local += nu;
-        if (may_dyn) d_local += dyn_units(nu, p.dyn_num);
-    }
-#pragma unroll
-    for (int m = 16; m >= 1; m >>= 1) {
-        t_local += __shfl_xor_sync(0xffffffffu, t_local, m);
-        d_local += __shfl_xor_sync(0xffffffffu, d_local, m);
-    }
-    if (lane == 0) {
-        ctl.red[warp][0] = t_local;
-        ctl.red[warp][1] = d_local;
-    }
-    __syncthreads();
-    if (tid == 0) {
-        int64_t tq = 0, dq = 0;
-        for (int w = 0; w < NWARPS; ++w) {
-            tq += ctl.red[w][0];
-            dq += ctl.red[w][1];
+    Cut cut;
+    int64_t lo = 0, hi = 0;
+    if (p.B <= kDecodeThreads) {
+        // one request per thread: lengths, units, and one block-wide scan that
+        // yields the totals (the cut) and each request's list positions
+        const int b = tid;
+        int nu = 0, du = 0;
+        if (b < p.B) {
+            const int raw = p.context_lens[b];
+            if (blockIdx.x == 0 && (raw < 0 || raw > cap)) set_error(p.error, PA_DEVERR_CONTEXT_LEN);
+            lens_s[b] = raw;  // B <= kDecodeThreads <= kLensCache: lens_cached
+            nu = units_of_len(p, raw < 0 ? 0 : (raw > cap ? cap : raw));
+            du = may_dyn ? dyn_units(nu, p.dyn_num) : 0;
         }
-        const int64_t NT = tq * p.NHG;
-        const int64_t C = p.num_ctas;
-        Cut k;
-        k.dyn = may_dyn && dq > 0 && NT >= 4 * C && NT < (int64_t(1) << 30);
-        k.Dn = k.dyn ? dq * p.NHG : 0;
-        k.S = NT - k.Dn;
-        k.Cn = k.S < C ? (k.S > 0 ? k.S : 1) : C;
-        k.g = (NT + 8 * C - 1) / (8 * C);
-        if (k.g < 1) k.g = 1;
-        k.J = k.dyn ? (k.Dn + k.g - 1) / k.g : 0;
-        ctl.cut = k;
-    }
-    __syncthreads();
-    const Cut cut = ctl.cut;
-    const bool has_slice = cut.S > 0 && blockIdx.x < cut.Cn;
-    const int64_t lo = has_slice ? slice_lo(blockIdx.x, cut) : 0;
-    const int64_t hi = has_slice ? slice_lo(blockIdx.x + 1, cut) : 0;
-
-    // exclusive prefix sums of static / dynamic units over requests: the
-    // request holding this CTA's first unit, and (dynamic list) the tables
-    // the grains are located with
-    if (lo < hi || cut.dyn) {
-        int64_t run_s = 0, run_d = 0;
-        for (int base = 0; base < p.B; base += kDecodeThreads) {
-            const int b = base + tid;
-            int64_t us = 0, ud = 0;
-            if (b < p.B) {
-                const int nu = units_of_len(p, clamped_len(p, lens_s, b));
-                const int d = cut.dyn ? dyn_units(nu, p.dyn_num) : 0;
-                us = (int64_t)p.NHG * (nu - d);
-                ud = (int64_t)p.NHG * d;
-            }
-            int64_t xs = us, xd = ud;
+        int64_t xa = nu, xb = du;  // inclusive scan within the warp
 #pragma unroll
-            for (int m = 1; m < 32; m <<= 1) {
-                const int64_t ys = __shfl_up_sync(0xffffffffu, xs, m);
-                const int64_t yd = __shfl_up_sync(0xffffffffu, xd, m);
-                if (lane >= m) {
-                    xs += ys;
-                    xd += yd;
-                }
+        for (int m = 1; m < 32; m <<= 1) {
+            const int64_t ya = __shfl_up_sync(0xffffffffu, xa, m);
+            const int64_t yb = __shfl_up_sync(0xffffffffu, xb, m);
+            if (lane >= m) {
+                xa += ya;
+                xb += yb;
             }
-            __syncthreads();  // ctl.red free to overwrite
-            if (lane == 31) {
-                ctl.red[warp][0] = xs;
-                ctl.red[warp][1] = xd;
+        }
+        if (lane == 31) {
+            ctl.red[warp][0] = xa;
+            ctl.red[warp][1] = xb;
+        }
+        __syncthreads();
+        int64_t ta = 0, tb = 0, pa = 0, pb = 0;
+        for (int w = 0; w < NWARPS; ++w) {
+            const int64_t wa = ctl.red[w][0], wb = ctl.red[w][1];
+            if (w < warp) {
+                pa += wa;
+                pb += wb;
             }
-            __syncthreads();
-            int64_t bs_ = 0, bd_ = 0, cs = 0, cd = 0;
-            for (int w = 0; w < NWARPS; ++w) {
-                if (w < warp) {
-                    bs_ += ctl.red[w][0];
-                    bd_ += ctl.red[w][1];
-                }
-                cs += ctl.red[w][0];
-                cd += ctl.red[w][1];
-            }
-            const int64_t es = run_s + bs_ + xs - us, ed = run_d + bd_ + xd - ud;
-            if (cut.dyn && b < p.B) {
+            ta += wa;
+            tb += wb;
+        }
+        cut = make_cut(ta, tb, p.NHG, p.num_ctas, may_dyn);
+        const bool has_slice = cut.S > 0 && blockIdx.x < cut.Cn;
+        lo = has_slice ? slice_lo(blockIdx.x, cut) : 0;
+        hi = has_slice ? slice_lo(blockIdx.x + 1, cut) : 0;
+        // request b's first static / dynamic list positions and unit counts
+        const int64_t ea = pa + xa - nu, eb = pb + xb - du;
+        const int64_t es = (int64_t)p.NHG * (cut.dyn ? ea - eb : ea);
+        const int64_t ed = cut.dyn ? (int64_t)p.NHG * eb : 0;
+        const int64_t us = (int64_t)p.NHG * (cut.dyn ? nu - du : nu);
+        if (b < p.B) {
+            if (cut.dyn) {
                 pre_s[b] = (int)es;
                 pre_d[b] = (int)ed;
             }
@@ -1504,14 +1549,107 @@ __global__ void __launch_bounds__(kDecodeThreads, 1) paged_decode_kernel(const _
                 ctl.found_excl = es;
                 ctl.found_dexcl = ed;
             }
-            run_s += cs;
-            run_d += cd;
-            __syncthreads();
-            if (!cut.dyn && ctl.found_b >= 0) break;
         }
-        if (cut.dyn && tid == 0) {
-            pre_s[p.B] = (int)cut.S;
-            pre_d[p.B] = (int)cut.Dn;
+        if (tid == 0) {
+            ctl.cut = cut;
+            if (cut.dyn) {
+                pre_s[p.B] = (int)cut.S;
+                pre_d[p.B] = (int)cut.Dn;
+            }
+        }
+    } else {
+        // any batch size: the totals first, then the prefix sums chunk by chunk
+        int64_t t_local = 0, d_local = 0;
+        for (int b = tid; b < p.B; b += kDecodeThreads) {
+            const int raw = p.context_lens[b];
+            if (blockIdx.x == 0 && (raw < 0 || raw > cap)) set_error(p.error, PA_DEVERR_CONTEXT_LEN);
+            if (p.lens_cached) lens_s[b] = raw;
+            const int nu = units_of_len(p, raw < 0 ? 0 : (raw > cap ? cap : raw));
+            t_local += nu;
+            if (may_dyn) d_local += dyn_units(nu, p.dyn_num);
+        }
+#pragma unroll
+        for (int m = 16; m >= 1; m >>= 1) {
+            t_local += __shfl_xor_sync(0xffffffffu, t_local, m);
+            d_local += __shfl_xor_sync(0xffffffffu, d_local, m);
+        }
+        if (lane == 0) {
+            ctl.red[warp][0] = t_local;
+            ctl.red[warp][1] = d_local;
+        }
+        __syncthreads();
+        if (tid == 0) {
+            int64_t tq = 0, dq = 0;
+            for (int w = 0; w < NWARPS; ++w) {
+                tq += ctl.red[w][0];
+                dq += ctl.red[w][1];
+            }
+            ctl.cut = make_cut(tq, dq, p.NHG, p.num_ctas, may_dyn);
+        }
+        __syncthreads();
+        cut = ctl.cut;
+        const bool has_slice = cut.S > 0 && blockIdx.x < cut.Cn;
+        lo = has_slice ? slice_lo(blockIdx.x, cut) : 0;
+        hi = has_slice ? slice_lo(blockIdx.x + 1, cut) : 0;
+
+        // exclusive prefix sums of static / dynamic units over requests: the
+        // request holding this CTA's first unit, and (dynamic list) the tables
+        // the grains are located with
+        if (lo < hi || cut.dyn) {
+            int64_t run_s = 0, run_d = 0;
+            for (int base = 0; base < p.B; base += kDecodeThreads) {
+                const int b = base + tid;
+                int64_t us = 0, ud = 0;
+                if (b < p.B) {
+                    const int nu = units_of_len(p, clamped_len(p, lens_s, b));
+                    const int d = cut.dyn ? dyn_units(nu, p.dyn_num) : 0;
+                    us = (int64_t)p.NHG * (nu - d);
+                    ud = (int64_t)p.NHG * d;
+                }
+                int64_t xs = us, xd = ud;
+#pragma unroll
+                for (int m = 1; m < 32; m <<= 1) {
+                    const int64_t ys = __shfl_up_sync(0xffffffffu, xs, m);
+                    const int64_t yd = __shfl_up_sync(0xffffffffu, xd, m);
+                    if (lane >= m) {
+                        xs += ys;
+                        xd += yd;
+                    }
+                }
+                __syncthreads();  // ctl.red free to overwrite
+                if (lane == 31) {
+                    ctl.red[warp][0] = xs;
+                    ctl.red[warp][1] = xd;
+                }
+                __syncthreads();
+                int64_t bs_ = 0, bd_ = 0, cs = 0, cd = 0;
+                for (int w = 0; w < NWARPS; ++w) {
+                    if (w < warp) {
+                        bs_ += ctl.red[w][0];
+                        bd_ += ctl.red[w][1];
+                    }
+                    cs += ctl.red[w][0];
+                    cd += ctl.red[w][1];
+                }
+                const int64_t es = run_s + bs_ + xs - us, ed = run_d + bd_ + xd - ud;
+                if (cut.dyn && b < p.B) {
+                    pre_s[b] = (int)es;
+                    pre_d[b] = (int)ed;
+                }
+                if (us > 0 && es <= lo && lo < es + us) {
+                    ctl.found_b = b;
+                    ctl.found_excl = es;
+                    ctl.found_dexcl = ed;
+                }
+                run_s += cs;
+                run_d += cd;
+                __syncthreads();
+                if (!cut.dyn && ctl.found_b >= 0) break;
+            }
+            if (cut.dyn && tid == 0) {
+                pre_s[p.B] = (int)cut.S;
+                pre_d[p.B] = (int)cut.Dn;
+            }
         }
     }
     __syncthreads();
@@ -1523,7 +1661,7 @@ __global__ void __launch_bounds__(kDecodeThreads, 1) paged_decode_kernel(const _
     if (lo < hi) {
         it.b = (int)ctl.found_b;
         it.load_request(p, cut);
-        it.hg = (int)((lo - ctl.found_excl) / it.su);
+        it.hg = (int)floor_div_exact(lo - ctl.found_excl, it.su);
         it.vr_start = ctl.found_excl + (int64_t)it.hg * it.su;
         it.ds = ctl.found_dexcl + (int64_t)it.hg * it.du;
     } else {
@@ -1577,7 +1715,6 @@ __global__ void __launch_bounds__(kDecodeThreads, 1) paged_decode_kernel(const _
     const int units_per_g = p.G / HC < 1 ? 1 : p.G / HC;
     float *s_sm = reinterpret_cast<float *>(smem + p.off_scratch) + warp * Engine::kScratchFloats;
     float *p_sm = s_sm + kSubTile * (Engine::kScratchFloats / (2 * kSubTile));
-    float *msm = reinterpret_cast<float *>(smem + p.off_merge);
 
     Engine eng;
     eng.setup(lane);
@@ -1699,7 +1836,7 @@ __global__ void __launch_bounds__(kDecodeThreads, 1) paged_decode_kernel(const _
         if (tid == 0) ctl.pending[npend] = s;
         if (lane == 0) mbar_arrive(&pdone[npend]);
         if (++npend == kMaxPending) {
-            flush_pending<T, D>(p, ctl, npend, adone, adone_par, abort_flag, msm, cb, tid);
+            flush_pending<T, D>(p, ctl, npend, adone, adone_par, abort_flag, cb, true, tid);
             adone_par ^= 1u;
             npend = 0;
         }
@@ -1708,7 +1845,7 @@ __global__ void __launch_bounds__(kDecodeThreads, 1) paged_decode_kernel(const _
     if (tid == 0) ctl.pending[npend].b = -1;
     __syncwarp();
     if (lane == 0) mbar_arrive(&pdone[npend]);
-    flush_pending<T, D>(p, ctl, npend, adone, adone_par, abort_flag, msm, cb, tid);
+    flush_pending<T, D>(p, ctl, npend, adone, adone_par, abort_flag, cb, false, tid);
 }
 
 }  // namespace pa

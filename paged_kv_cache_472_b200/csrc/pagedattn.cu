@@ -118,7 +118,7 @@ pa_status ensure_smem_attr(KernelFn fn, int bytes) {
 }
 
 struct Layout {
-    uint32_t off_bar, off_q, off_stage, off_scratch, off_comb, off_merge, total;
+    uint32_t off_bar, off_q, off_stage, off_scratch, off_comb, total;
     uint32_t comb_stride;
 };
 
@@ -128,6 +128,8 @@ Layout smem_layout(int dtype, int D, int stages, uint32_t q_bytes, uint32_t half
     Layout l;
     const bool mma = tensor_core_dtype(dtype);
     l.off_bar = 0;
+    // full/empty per stage, q full/empty, piece-done per pending piece, arrivals done,
+    // consumer barrier
     const uint32_t bar_bytes = (uint32_t)round_up((2 * stages + 4 + pa::kMaxPending + 2) * 8, 128);
     l.off_q = bar_bytes;
     l.off_stage = (uint32_t)round_up(l.off_q + 2 * q_bytes, 1024);
@@ -137,10 +139,8 @@ Layout smem_layout(int dtype, int D, int stages, uint32_t q_bytes, uint32_t half
     const uint32_t comb_floats = mma ? (uint32_t)(4 * (D / 16) * 32 + 4 * 32) : (uint32_t)(hc * D + 8);
     l.comb_stride = comb_floats * 4;
     const uint32_t comb = tsplit > 1 ? pa::kConsumerWarps * l.comb_stride : 0;
-    l.off_merge = (uint32_t)round_up(l.off_comb + comb, 128);
-    const uint32_t merge = (uint32_t)pa::kMergeParts * 8;  // slot list of the vr being merged
     // + 1024: the kernel rounds its dynamic base up to a 1024-byte boundary
-    l.total = (uint32_t)round_up(l.off_merge + merge, 128) + 1024;
+    l.total = (uint32_t)round_up(l.off_comb + comb, 128) + 1024;
     return l;
 }
 
@@ -338,7 +338,6 @@ pa_status launch_decode(const void *q, const void *k_cache, const void *v_cache,
     p.off_stage = lay.off_stage;
     p.off_scratch = lay.off_scratch;
     p.off_comb = lay.off_comb;
-    p.off_merge = lay.off_merge;
     p.row_bytes = row_bytes;
     p.row_pitch = pitch;
     p.half_bytes = half;
@@ -477,8 +476,8 @@ pa_status pa_plan(const pa_shape *s, int32_t max_context_len, int32_t partition_
         const int64_t Jmax = 8 * C * kMaxDynamicShare / 256 + 1;
         plan->max_slots = dyn ? 2 * NV + C + Jmax : NV + C;
     } else {
-        const int64_t parts = (max_context_len + partition_tokens - 1) / partition_tokens;
-        plan->max_slots = (int64_t)NHG * s->B * (parts > 1 ? parts : 0);
+        // one partial per (vr, slice) it touches, as in the static list above
+        plan->max_slots = (int64_t)s->B * NHG + num_sms;
     }
     const size_t slot_floats = (size_t)NHvr * s->D + round_up(2 * NHvr, 4);
     const size_t counters = round_up((size_t)s->B * NHG * 4, 256);

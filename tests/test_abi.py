@@ -119,7 +119,7 @@ def test_plan_rejects_bad_partition_and_context():
 def test_fixed_plan_workspace_formula():
     s = pa.Shape(8, 32, 1, 128, 256, 4096, 512, pa.DTYPE_BF16)
     plan = pa.pa_plan(s, 131072, 512, 148)
-    assert plan.max_slots == 8 * 256
+    assert plan.max_slots == 8 + 148          # one partial per (request, slice)
     slot_floats = 32 * 128 + 64
     assert plan.workspace_bytes == 256 + 256 + plan.max_slots * slot_floats * 4
 

@@ -41,8 +41,8 @@ def test_no_alloc_matches_workspace_decode(cid, batch, partition):
 
 
 def test_no_alloc_rejects_plans_beyond_its_array():
-    # fixed partitions of 16 tokens over long contexts need far more than 16 MiB
-    s = pa.Shape(64, 32, 8, 128, 16, 70000, 1024, pa.DTYPE_BF16)
+    # a batch of 1024 requests needs one 16.6 KB partial per request, more than 16 MiB
+    s = pa.Shape(1024, 32, 8, 128, 16, 70000, 1024, pa.DTYPE_BF16)
     plan = pa.pa_plan(s, 16384, 16, 148)
     assert plan.workspace_bytes > 16 << 20
     st = pa.lib.pa_decode_no_alloc(1 << 20, 1 << 20, 1 << 20, 1 << 20, 1 << 20, ctypes.c_float(0.1), 1 << 20,
