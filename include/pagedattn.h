@@ -92,10 +92,25 @@ typedef struct {
                                  at run time to whichever CTA is free, in 1/256.  pa_plan
                                  sets 0; a caller may set 1..64 when B <= 512 (the
                                  workspace is sized for 64) */
+    int32_t flags;            /* PA_PLAN_* bits; pa_plan sets 0, a caller may set them */
+    int32_t reserved;
     int64_t max_slots;        /* partial-result slots in the workspace */
     pa_shape shape;           /* the shape this plan was made for */
     size_t workspace_bytes;   /* bytes pa_decode needs at `workspace` */
 } pa_plan_t;
+
+/* pa_plan_t.flags.  By default a decode grid launched behind another grid on
+ * the same stream (programmatic dependent launch) reads context_lens and the
+ * block table as they are while that grid still runs, plans its work from
+ * them and pulls its first K/V blocks into L2.  Once that grid has
+ * completed it reads both again and keeps the plan only if nothing changed
+ * (otherwise it plans again), so the result never depends on the early
+ * reads.  PA_PLAN_NO_SPECULATION turns the early reads off (useful when the
+ * preceding kernel rewrites the metadata every step).  PA_PLAN_TEST_MISGUESS
+ * makes every early guess wrong, so that the plan-again path runs (for
+ * tests; slower). */
+#define PA_PLAN_NO_SPECULATION 0x1
+#define PA_PLAN_TEST_MISGUESS  0x2
 
 /* Library version: major*10000 + minor*100 + patch. */
 int32_t pa_version(void);

@@ -15,6 +15,7 @@ from .build import LIB as _LIB_PATH
 
 __all__ = ["PagedAttnError", "Shape", "Plan", "DTYPE_F32", "DTYPE_BF16", "DTYPE_F16", "SPLIT_BALANCED", "SPLIT_FIXED",
            "DEVERR_BLOCK_ID", "DEVERR_CONTEXT_LEN", "DEVERR_TIMEOUT", "DEVERR_WORKSPACE", "DEVERR_SLOT",
+           "PLAN_NO_SPECULATION", "PLAN_TEST_MISGUESS",
            "pa_version", "pa_status_str", "pa_last_error_message", "pa_kv_append", "pa_plan",
            "pa_decode_workspace_size", "pa_workspace_init", "pa_decode", "pa_kv_append_decode", "pa_get_device_error",
            "pa_decode_no_alloc", "lib"]
@@ -23,6 +24,7 @@ PA_OK, PA_ERR_INVALID_ARG, PA_ERR_UNSUPPORTED, PA_ERR_CUDA, PA_ERR_WORKSPACE = r
 DTYPE_F32, DTYPE_BF16, DTYPE_F16 = 0, 1, 2
 SPLIT_BALANCED, SPLIT_FIXED = 0, 1
 DEVERR_BLOCK_ID, DEVERR_CONTEXT_LEN, DEVERR_TIMEOUT, DEVERR_WORKSPACE, DEVERR_SLOT = 0x1, 0x2, 0x4, 0x8, 0x10
+PLAN_NO_SPECULATION, PLAN_TEST_MISGUESS = 0x1, 0x2
 
 
 class Shape(ctypes.Structure):
@@ -39,7 +41,8 @@ class Plan(ctypes.Structure):
                 ("tile_tokens", ctypes.c_int32), ("stages", ctypes.c_int32), ("head_group", ctypes.c_int32),
                 ("heads_per_unit", ctypes.c_int32), ("units_per_warp", ctypes.c_int32),
                 ("warps_per_unit", ctypes.c_int32), ("max_context_len", ctypes.c_int32),
-                ("smem_bytes", ctypes.c_int32), ("dynamic_share", ctypes.c_int32), ("max_slots", ctypes.c_int64),
+                ("smem_bytes", ctypes.c_int32), ("dynamic_share", ctypes.c_int32), ("flags", ctypes.c_int32),
+                ("reserved", ctypes.c_int32), ("max_slots", ctypes.c_int64),
                 ("shape", Shape), ("workspace_bytes", ctypes.c_size_t)]
 
     def as_dict(self):

@@ -116,6 +116,23 @@ __device__ __forceinline__ void tma_load_3d(void *dst, const CUtensorMap *map, i
         : "memory");
 }
 
+// Pull the box a tma_load_3d with the same map and coordinates would copy
+// into L2 (no shared memory written, no completion to wait for).
+__device__ __forceinline__ void tma_prefetch_3d(const CUtensorMap *map, int32_t c0, int32_t c1, int32_t c2) {
+    asm volatile("cp.async.bulk.prefetch.tensor.3d.L2.global.tile [%0, {%1, %2, %3}];" ::"l"(
+                     reinterpret_cast<uint64_t>(map)),
+                 "r"(c0), "r"(c1), "r"(c2)
+                 : "memory");
+}
+
+// Load that may see memory another grid is still writing (the value is only
+// a hint; nothing derived from it is trusted without a later re-read).
+__device__ __forceinline__ int ld_hint(const int32_t *p) {
+    int v;
+    asm volatile("ld.relaxed.gpu.global.b32 %0, [%1];" : "=r"(v) : "l"(p) : "memory");
+    return v;
+}
+
 // Pull a tensor map into the descriptor cache ahead of its first use.
 __device__ __forceinline__ void prefetch_tensormap(const CUtensorMap *map) {
     asm volatile("prefetch.tensormap [%0];" ::"l"(reinterpret_cast<uint64_t>(map)) : "memory");
@@ -190,6 +207,17 @@ __device__ __forceinline__ int atomic_add_acq_rel(int *p, int v) {
 // reach k only if delta were within half an ulp of k, i.e. d*k >= 2^53 > n.
 __device__ __forceinline__ int64_t floor_div_exact(int64_t n, int64_t d) {
     return (int64_t)__double2ll_rz(__ddiv_rn((double)n, (double)d));
+}
+
+// floor(n / d) for 0 <= n, n / d < 2^52, d >= 1, given inv = 1/d rounded to
+// nearest: n * inv is within (n / d) * 2^-52 < 1 of n / d, so its truncation
+// is off by at most one, which the remainder check corrects.
+__device__ __forceinline__ int64_t floor_div_inv(int64_t n, int64_t d, double inv) {
+    int64_t q = (int64_t)__double2ll_rz((double)n * inv);
+    const int64_t r = n - q * d;
+    if (r < 0) --q;
+    else if (r >= d) ++q;
+    return q;
 }
 
 }  // namespace pa

@@ -111,6 +111,8 @@ struct DecodeParams {
     int32_t use_tmap;     // 1: stages are filled by tensor-map boxes (swizzled, head-major)
     int32_t br_log2;      // rows of one box = min(ST, bs) = 1 << br_log2
     int32_t bs_log2;
+    int32_t st_log2;      // ST = 1 << st_log2
+    int32_t spec;         // 0: no speculation; 1: speculate; 2: speculate on wrong guesses (tests)
     int32_t lens_cached;  // context lengths were copied into shared memory
 };
 static_assert(offsetof(DecodeParams, tmap_k) % 64 == 0 && offsetof(DecodeParams, tmap_v) % 64 == 0,
@@ -216,7 +218,7 @@ __device__ __forceinline__ void warm_params(const DecodeParams &p) {
                  "r"(p.num_ctas), "r"(p.tsplit), "r"(p.units), "r"(p.heads_per_unit), "r"(p.fused), "r"(p.dyn_num));
     asm volatile("" ::"r"(p.off_bar), "r"(p.off_q), "r"(p.off_stage), "r"(p.off_scratch), "r"(p.off_comb),
                  "r"(p.row_bytes), "r"(p.row_pitch), "r"(p.half_bytes), "r"(p.q_bytes), "r"(p.comb_stride),
-                 "r"(p.use_tmap), "r"(p.br_log2), "r"(p.bs_log2), "r"(p.lens_cached));
+                 "r"(p.use_tmap), "r"(p.br_log2), "r"(p.bs_log2), "r"(p.st_log2), "r"(p.spec), "r"(p.lens_cached));
 }
 
 // ---------------------------------------------------------------------------
@@ -231,7 +233,7 @@ __device__ __forceinline__ int clamped_len(const DecodeParams &p, const int *len
 
 // work units of a request: tiles (balanced) or partitions (fixed)
 __device__ __forceinline__ int units_of_len(const DecodeParams &p, int L) {
-    const int tiles = (L + p.ST - 1) / p.ST;
+    const int tiles = (L + p.ST - 1) >> p.st_log2;
     return p.mode == PA_SPLIT_BALANCED ? tiles : (tiles + p.part_tiles - 1) / p.part_tiles;
 }
 
@@ -246,13 +248,14 @@ struct Cut {
     int64_t Cn;     // CTAs with a static slice
     int64_t g, J;
     int dyn;        // the dynamic list is in use
+    double inv_S, inv_Cn, inv_g;  // 1/S, 1/Cn, 1/g rounded to nearest (for floor_div_inv)
 };
 
-// (positions and products stay far below 2^53, so the double quotients are exact)
-__device__ __forceinline__ int64_t slice_lo(int64_t r, const Cut &k) { return floor_div_exact(r * k.S, k.Cn); }
+// (positions and products stay far below 2^52, so these quotients are exact)
+__device__ __forceinline__ int64_t slice_lo(int64_t r, const Cut &k) { return floor_div_inv(r * k.S, k.Cn, k.inv_Cn); }
 // static slice holding static-list position x
 __device__ __forceinline__ int64_t slice_of(int64_t x, const Cut &k) {
-    return floor_div_exact((x + 1) * k.Cn - 1, k.S);
+    return floor_div_inv((x + 1) * k.Cn - 1, k.S, k.inv_S);
 }
 
 // The cut from the totals: tq units over all requests (one head group), dq of
@@ -267,6 +270,9 @@ __device__ __forceinline__ Cut make_cut(int64_t tq, int64_t dq, int NHG, int64_t
     k.g = floor_div_exact(NT + 8 * C - 1, 8 * C);
     if (k.g < 1) k.g = 1;
     k.J = k.dyn ? floor_div_exact(k.Dn + k.g - 1, k.g) : 0;
+    k.inv_S = __drcp_rn((double)(k.S > 0 ? k.S : 1));
+    k.inv_Cn = __drcp_rn((double)k.Cn);
+    k.inv_g = __drcp_rn((double)k.g);
     return k;
 }
 
@@ -287,7 +293,7 @@ struct Seg {
 // earlier slice or grain, so no two pieces share a slot.
 __device__ __forceinline__ int balanced_parts(const Cut &k, int64_t ss, int s_len, int64_t ds, int d_len) {
     const int ns = (int)(slice_of(ss + s_len - 1, k) - slice_of(ss, k) + 1);
-    const int nd = d_len > 0 ? (int)(floor_div_exact(ds + d_len - 1, k.g) - floor_div_exact(ds, k.g) + 1) : 0;
+    const int nd = d_len > 0 ? (int)(floor_div_inv(ds + d_len - 1, k.g, k.inv_g) - floor_div_inv(ds, k.g, k.inv_g) + 1) : 0;
     return ns + nd;
 }
 
@@ -305,7 +311,7 @@ __device__ __forceinline__ PieceSlots piece_slots(const DecodeParams &p, const C
     const int64_t r0 = slice_of(s.ss, k);
     r.ns = (int)(slice_of(s.ss + s.s_len - 1, k) - r0 + 1);
     r.a = v + r0;
-    r.b = (int64_t)p.B * p.NHG + p.num_ctas + v + (s.d_len > 0 ? floor_div_exact(s.ds, k.g) : 0);
+    r.b = (int64_t)p.B * p.NHG + p.num_ctas + v + (s.d_len > 0 ? floor_div_inv(s.ds, k.g, k.inv_g) : 0);
     return r;
 }
 
@@ -353,7 +359,7 @@ struct SegIter {
                 s.t_begin = u0;
                 s.t_end = u1;
             } else {
-                const int tiles = (L + p.ST - 1) / p.ST;
+                const int tiles = (L + p.ST - 1) >> p.st_log2;
                 s.t_begin = u0 * p.part_tiles;
                 s.t_end = min(tiles, u1 * p.part_tiles);
             }
@@ -955,8 +961,8 @@ struct TableWindow {
         table = p.block_tables + (size_t)s.b * p.max_blocks;
         nblk = (s.L + p.bs - 1) >> p.bs_log2;
         cur_base = ((s.t_begin * p.ST) >> p.bs_log2) & ~31;
-        cur_val = (cur_base + lane < nblk) ? table[cur_base + lane] : -1;
         nxt_base = cur_base + 32;
+        cur_val = (cur_base + lane < nblk) ? table[cur_base + lane] : -1;
         nxt_val = (nxt_base + lane < nblk) ? table[nxt_base + lane] : -1;
     }
     // make the window holding block-table column jb current
@@ -978,7 +984,7 @@ struct TableWindow {
 // token goes.  It is patched into the staged tile only when its slot is the
 // request's own last position; any other slot is reported.
 __device__ __forceinline__ void fused_info(const DecodeParams &p, Seg &s, int lane) {
-    if (!p.fused || s.t_end != (s.L + p.ST - 1) / p.ST) return;
+    if (!p.fused || s.t_end != (s.L + p.ST - 1) >> p.st_log2) return;
     int sm = -1, expect = -1;
     if (lane == 0) {
         sm = p.slot_mapping[s.b];
@@ -1022,19 +1028,19 @@ __device__ __forceinline__ void publish(const DecodeParams &p, ProducerState &ps
     if (ps.qslot == 0) ps.qphase ^= 1u;
 }
 
-// Fill one stage per tile of the piece.  With `grab_at_last`, the next grain
-// is requested while the piece's last tile is being issued.
+// Fill one stage per tile t_lo..t_hi-1 of the piece.  With `grab_at_last`, the
+// next grain is requested while the piece's last tile is being issued.
 template <int D, int E>
-__device__ __forceinline__ void issue_tiles(const DecodeParams &p, ProducerState &ps, const Seg &s, TableWindow &win,
-                                            bool grab_at_last, uint64_t *full, uint64_t *empty,
-                                            unsigned char *stage_base, volatile int *abort_flag, uint64_t policy,
-                                            int lane) {
+__device__ __forceinline__ void issue_tiles(const DecodeParams &p, ProducerState &ps, const Seg &s, int t_lo,
+                                            int t_hi, TableWindow &win, bool grab_at_last, uint64_t *full,
+                                            uint64_t *empty, unsigned char *stage_base, volatile int *abort_flag,
+                                            uint64_t policy, int lane) {
     const unsigned char *kc = reinterpret_cast<const unsigned char *>(p.k_cache);
     const unsigned char *vc = reinterpret_cast<const unsigned char *>(p.v_cache);
     const uint32_t row_bytes = p.row_bytes, pitch = p.row_pitch;
     const size_t tok_stride = (size_t)p.Hkv * D * E;  // bytes between token rows in the pool
     const bool contiguous = (p.HG == p.Hkv) && (pitch == row_bytes);
-    for (int t = s.t_begin; t < s.t_end; ++t) {
+    for (int t = t_lo; t < t_hi; ++t) {
         if (!mbar_wait(&empty[ps.stage], ps.phase ^ 1u, abort_flag)) {
             ps.ok = false;
             return;
@@ -1082,7 +1088,7 @@ __device__ __forceinline__ void issue_tiles(const DecodeParams &p, ProducerState
             }
         } else if (contiguous) {
             // one copy per block piece: rows of all KV heads are contiguous in both places
-            const int np = (tok0 + ntok - 1) / p.bs - jb0 + 1;
+            const int np = ((tok0 + ntok - 1) >> p.bs_log2) - jb0 + 1;
             const int j = jb0 + lane;
             const int phys = __shfl_sync(0xffffffffu, cur_val, (j - cur_base) & 31);
             int tlo = 0, nrows = 0;
@@ -1109,7 +1115,7 @@ __device__ __forceinline__ void issue_tiles(const DecodeParams &p, ProducerState
             for (int i0 = 0; i0 < ntok; i0 += 32) {
                 const int i = i0 + lane;
                 const int tt = tok0 + i;
-                const int j = tt / p.bs;
+                const int j = tt >> p.bs_log2;
                 const int phys = __shfl_sync(0xffffffffu, cur_val, (j - cur_base) & 31);
                 if (i < ntok) {
                     if (phys < 0 || phys >= p.num_blocks) set_error(p.error, PA_DEVERR_BLOCK_ID);
@@ -1123,7 +1129,7 @@ __device__ __forceinline__ void issue_tiles(const DecodeParams &p, ProducerState
             for (int i0 = 0; i0 < ntok; i0 += 32) {
                 const int i = i0 + lane;
                 const int tt = tok0 + i;
-                const int j = tt / p.bs;
+                const int j = tt >> p.bs_log2;
                 const int phys = __shfl_sync(0xffffffffu, cur_val, (j - cur_base) & 31);
                 if (i < ntok && phys >= 0 && phys < p.num_blocks) {
                     const size_t src = ((size_t)phys * p.bs + (tt - j * p.bs)) * tok_stride + (size_t)s.hg * row_bytes;
@@ -1150,15 +1156,15 @@ __device__ __forceinline__ void run_producer(const DecodeParams &p, const Cut &k
     const uint64_t policy = policy_evict_first();
     ProducerState ps;
     Seg s;
-    // this CTA's static slice
     TableWindow win;
+    // this CTA's static slice
     while (ps.ok && it.next(p, k, s)) {
         win.prime(p, s, lane);  // in flight while q is published
         fused_info(p, s, lane);
         publish(p, ps, s, ctl, qfull, qempty, qarea, abort_flag, D, E, lane);
         if (!ps.ok) break;
-        issue_tiles<D, E>(p, ps, s, win, k.dyn && it.cur >= it.hi, full, empty, stage_base, abort_flag, policy,
-                          lane);
+        issue_tiles<D, E>(p, ps, s, s.t_begin, s.t_end, win, k.dyn && it.cur >= it.hi, full, empty, stage_base,
+                          abort_flag, policy, lane);
     }
     // grains of the dynamic list, one at a time, to whichever CTA asks first
     if (k.dyn) {
@@ -1176,7 +1182,8 @@ __device__ __forceinline__ void run_producer(const DecodeParams &p, const Cut &k
                 fused_info(p, s, lane);
                 publish(p, ps, s, ctl, qfull, qempty, qarea, abort_flag, D, E, lane);
                 if (!ps.ok) break;
-                issue_tiles<D, E>(p, ps, s, win, gi.y >= gi.y1, full, empty, stage_base, abort_flag, policy, lane);
+                issue_tiles<D, E>(p, ps, s, s.t_begin, s.t_end, win, gi.y >= gi.y1, full, empty, stage_base,
+                                  abort_flag, policy, lane);
             }
         }
         // the last CTA to find the list empty leaves the counters at zero for the next launch
@@ -1419,6 +1426,152 @@ struct NewToken {
 };
 
 // ===========================================================================
+// prologue helpers
+// ===========================================================================
+
+// One request per thread (B <= kDecodeThreads): `raw` is request tid's
+// length (any value past B).  One block-wide scan yields the totals (the
+// cut), this CTA's static slice [lo, hi), each request's list positions and
+// the request holding the slice's first unit (ctl.found_*, which must be -1
+// on entry).  Contains one __syncthreads; the caller synchronises before
+// reading ctl.
+__device__ __forceinline__ Cut scan_requests(const DecodeParams &p, int raw, DecodeCtl &ctl, int *lens_s, int *pre_s,
+                                             int *pre_d, bool may_dyn, int64_t &lo, int64_t &hi, int tid, int lane,
+                                             int warp) {
+    constexpr int NWARPS = kConsumerWarps + 2;
+    const int cap = p.max_blocks * p.bs;
+    const int b = tid;
+    int nu = 0, du = 0;
+    if (b < p.B) {
+        lens_s[b] = raw;  // B <= kDecodeThreads <= kLensCache: lens_cached
+        nu = units_of_len(p, raw < 0 ? 0 : (raw > cap ? cap : raw));
+        du = may_dyn ? dyn_units(nu, p.dyn_num) : 0;
+    }
+    int64_t xa = nu, xb = du;  // inclusive scan within the warp
+#pragma unroll
+    for (int m = 1; m < 32; m <<= 1) {
+        const int64_t ya = __shfl_up_sync(0xffffffffu, xa, m);
+        const int64_t yb = __shfl_up_sync(0xffffffffu, xb, m);
+        if (lane >= m) {
+            xa += ya;
+            xb += yb;
+        }
+    }
+    if (lane == 31) {
+        ctl.red[warp][0] = xa;
+        ctl.red[warp][1] = xb;
+    }
+    __syncthreads();
+    int64_t ta = 0, tb = 0, pa = 0, pb = 0;
+    for (int w = 0; w < NWARPS; ++w) {
+        const int64_t wa = ctl.red[w][0], wb = ctl.red[w][1];
+        if (w < warp) {
+            pa += wa;
+            pb += wb;
+        }
+        ta += wa;
+        tb += wb;
+    }
+    const Cut cut = make_cut(ta, tb, p.NHG, p.num_ctas, may_dyn);
+    const bool has_slice = cut.S > 0 && blockIdx.x < cut.Cn;
+    lo = has_slice ? slice_lo(blockIdx.x, cut) : 0;
+    hi = has_slice ? slice_lo(blockIdx.x + 1, cut) : 0;
+    // request b's first static / dynamic list positions and unit counts
+    const int64_t ea = pa + xa - nu, eb = pb + xb - du;
+    const int64_t es = (int64_t)p.NHG * (cut.dyn ? ea - eb : ea);
+    const int64_t ed = cut.dyn ? (int64_t)p.NHG * eb : 0;
+    const int64_t us = (int64_t)p.NHG * (cut.dyn ? nu - du : nu);
+    if (b < p.B) {
+        if (cut.dyn) {
+            pre_s[b] = (int)es;
+            pre_d[b] = (int)ed;
+        }
+        if (us > 0 && es <= lo && lo < es + us) {
+            ctl.found_b = b;
+            ctl.found_excl = es;
+            ctl.found_dexcl = ed;
+        }
+    }
+    if (tid == 0) {
+        ctl.cut = cut;
+        if (cut.dyn) {
+            pre_s[p.B] = (int)cut.S;
+            pre_d[p.B] = (int)cut.Dn;
+        }
+    }
+    return cut;
+}
+
+// The iterator over this CTA's static slice [lo, hi), positioned by ctl.found_*.
+__device__ __forceinline__ SegIter slice_iter(const DecodeParams &p, const DecodeCtl &ctl, const Cut &cut, int64_t lo,
+                                              int64_t hi, const int *lens_s) {
+    SegIter it;
+    it.cur = lo;
+    it.hi = hi;
+    it.lens_s = lens_s;
+    if (lo < hi && ctl.found_b >= 0) {
+        it.b = (int)ctl.found_b;
+        it.load_request(p, cut);
+        it.hg = p.NHG == 1 ? 0 : (int)floor_div_exact(lo - ctl.found_excl, it.su);
+        it.vr_start = ctl.found_excl + (int64_t)it.hg * it.su;
+        it.ds = ctl.found_dexcl + (int64_t)it.hg * it.du;
+    } else {
+        it.cur = it.hi = 0;
+        it.b = 0;
+        it.hg = 0;
+        it.L = 0;
+        it.su = 0;
+        it.du = 0;
+        it.vr_start = 0;
+        it.ds = 0;
+    }
+    return it;
+}
+
+// Speculative warm-up (producer warp, tensor-map path): the first blocks
+// this CTA would stream with the guessed lengths (as far as kSpecBytes of K
+// and V) pulled into L2.  It runs before the grid-dependency wait, on lengths
+// and block-table entries the preceding grid may still change: nothing read
+// here is used for the decode itself (the plan is kept only if every length
+// read after the wait matches its guess, and the block tables are read again
+// after the wait), and a wrong guess only costs bandwidth.
+constexpr uint32_t kSpecBytes = 256u << 10;
+
+template <int D>
+__device__ __forceinline__ void prefetch_block(const DecodeParams &p, const Seg &s, int phys) {
+    constexpr int NDC = D / 64;
+    if (phys < 0 || phys >= p.num_blocks) return;
+    const int32_t head0 = s.hg * p.HG;
+    const int boxes = p.bs >> p.br_log2;  // boxes per block (tiles shorter than a block: several)
+    for (int x = 0; x < boxes; ++x) {
+        const int32_t row = phys * p.bs + (x << p.br_log2);
+#pragma unroll
+        for (int c2 = 0; c2 < NDC; ++c2) {
+            tma_prefetch_3d(&p.tmap_k, c2 * 64, row, head0);
+            tma_prefetch_3d(&p.tmap_v, c2 * 64, row, head0);
+        }
+    }
+}
+
+template <int D>
+__device__ __forceinline__ void speculative_prefetch(const DecodeParams &p, const DecodeCtl &ctl, const Cut &cut,
+                                                     int64_t lo, int64_t hi, const int *lens_s, int lane) {
+    constexpr int E = 2;
+    SegIter it = slice_iter(p, ctl, cut, lo, hi, lens_s);
+    const uint32_t block_bytes = 2u * (uint32_t)p.bs * p.HG * D * E;
+    int budget = (int)(kSpecBytes / block_bytes);
+    budget = budget < 1 ? 1 : (budget > 32 ? 32 : budget);
+    Seg s;
+    while (budget > 0 && it.next(p, cut, s)) {  // one guessed table entry per lane and block
+        const int jb0 = (s.t_begin * p.ST) >> p.bs_log2;
+        const int jb1 = (min(s.t_end * p.ST, s.L) - 1) >> p.bs_log2;
+        const int n = min(jb1 - jb0 + 1, budget);
+        if (lane < n) prefetch_block<D>(p, s, ld_hint(p.block_tables + (size_t)s.b * p.max_blocks + jb0 + lane));
+        budget -= n;
+    }
+}
+
+// ===========================================================================
 template <typename T, int D, class Engine>
 __global__ void __launch_bounds__(kDecodeThreads, 1) paged_decode_kernel(const __grid_constant__ DecodeParams p) {
     constexpr int E = Elem<T>::kBytes;
@@ -1483,79 +1636,37 @@ __global__ void __launch_bounds__(kDecodeThreads, 1) paged_decode_kernel(const _
             prefetch_l2_share(p.v_new, (size_t)p.B * p.Hkv * D * E, first, stride, 1);
         }
     }
+    // Speculative plan (batches of up to kDecodeThreads requests): the slice
+    // this CTA would take with the lengths as they are now, and its first
+    // blocks pulled into L2 while the preceding grid finishes.
+    const int cap = p.max_blocks * p.bs;
+    const bool may_dyn = p.mode == PA_SPLIT_BALANCED && p.dyn_num > 0 && p.B <= kPrefixCache && p.lens_cached;
+    const bool one_pass = p.B <= kDecodeThreads;
+    const bool speculate = one_pass && p.spec != 0;
+    Cut cut;
+    int64_t lo = 0, hi = 0;
+    int guess = 0;
+    if (speculate) {
+        if (tid < p.B) guess = ld_hint(p.context_lens + tid) + (p.spec == 2 ? 1 + (tid & 1) : 0);
+        cut = scan_requests(p, guess, ctl, lens_s, pre_s, pre_d, may_dyn, lo, hi, tid, lane, warp);
+        __syncthreads();
+        if (warp == kProducerWarp && p.use_tmap) speculative_prefetch<D>(p, ctl, cut, lo, hi, lens_s, lane);
+    }
+
     // everything below may read what the preceding grid on the stream wrote;
     // the next grid may start its own prologue as soon as SMs free up
     grid_dependency_wait();
     grid_launch_dependents();
 
     // ---- prologue: the cut of the work and this CTA's static slice ----
-    const int cap = p.max_blocks * p.bs;
-    const bool may_dyn = p.mode == PA_SPLIT_BALANCED && p.dyn_num > 0 && p.B <= kPrefixCache && p.lens_cached;
-    Cut cut;
-    int64_t lo = 0, hi = 0;
-    if (p.B <= kDecodeThreads) {
-        // one request per thread: lengths, units, and one block-wide scan that
-        // yields the totals (the cut) and each request's list positions
-        const int b = tid;
-        int nu = 0, du = 0;
-        if (b < p.B) {
-            const int raw = p.context_lens[b];
-            if (blockIdx.x == 0 && (raw < 0 || raw > cap)) set_error(p.error, PA_DEVERR_CONTEXT_LEN);
-            lens_s[b] = raw;  // B <= kDecodeThreads <= kLensCache: lens_cached
-            nu = units_of_len(p, raw < 0 ? 0 : (raw > cap ? cap : raw));
-            du = may_dyn ? dyn_units(nu, p.dyn_num) : 0;
-        }
-        int64_t xa = nu, xb = du;  // inclusive scan within the warp
-#pragma unroll
-        for (int m = 1; m < 32; m <<= 1) {
-            const int64_t ya = __shfl_up_sync(0xffffffffu, xa, m);
-            const int64_t yb = __shfl_up_sync(0xffffffffu, xb, m);
-            if (lane >= m) {
-                xa += ya;
-                xb += yb;
-            }
-        }
-        if (lane == 31) {
-            ctl.red[warp][0] = xa;
-            ctl.red[warp][1] = xb;
-        }
-        __syncthreads();
-        int64_t ta = 0, tb = 0, pa = 0, pb = 0;
-        for (int w = 0; w < NWARPS; ++w) {
-            const int64_t wa = ctl.red[w][0], wb = ctl.red[w][1];
-            if (w < warp) {
-                pa += wa;
-                pb += wb;
-            }
-            ta += wa;
-            tb += wb;
-        }
-        cut = make_cut(ta, tb, p.NHG, p.num_ctas, may_dyn);
-        const bool has_slice = cut.S > 0 && blockIdx.x < cut.Cn;
-        lo = has_slice ? slice_lo(blockIdx.x, cut) : 0;
-        hi = has_slice ? slice_lo(blockIdx.x + 1, cut) : 0;
-        // request b's first static / dynamic list positions and unit counts
-        const int64_t ea = pa + xa - nu, eb = pb + xb - du;
-        const int64_t es = (int64_t)p.NHG * (cut.dyn ? ea - eb : ea);
-        const int64_t ed = cut.dyn ? (int64_t)p.NHG * eb : 0;
-        const int64_t us = (int64_t)p.NHG * (cut.dyn ? nu - du : nu);
-        if (b < p.B) {
-            if (cut.dyn) {
-                pre_s[b] = (int)es;
-                pre_d[b] = (int)ed;
-            }
-            if (us > 0 && es <= lo && lo < es + us) {
-                ctl.found_b = b;
-                ctl.found_excl = es;
-                ctl.found_dexcl = ed;
-            }
-        }
-        if (tid == 0) {
-            ctl.cut = cut;
-            if (cut.dyn) {
-                pre_s[p.B] = (int)cut.S;
-                pre_d[p.B] = (int)cut.Dn;
-            }
+    if (one_pass) {
+        // the lengths again, now that the preceding grid has completed: the
+        // early plan stands only if every one is unchanged
+        const int raw = tid < p.B ? p.context_lens[tid] : 0;
+        if (blockIdx.x == 0 && tid < p.B && (raw < 0 || raw > cap)) set_error(p.error, PA_DEVERR_CONTEXT_LEN);
+        if (!__syncthreads_and(speculate && raw == guess)) {
+            if (tid == 0) ctl.found_b = -1;
+            cut = scan_requests(p, raw, ctl, lens_s, pre_s, pre_d, may_dyn, lo, hi, tid, lane, warp);
         }
     } else {
         // any batch size: the totals first, then the prefix sums chunk by chunk
@@ -1654,25 +1765,7 @@ __global__ void __launch_bounds__(kDecodeThreads, 1) paged_decode_kernel(const _
     }
     __syncthreads();
 
-    SegIter it;
-    it.cur = lo;
-    it.hi = hi;
-    it.lens_s = lens_s;
-    if (lo < hi) {
-        it.b = (int)ctl.found_b;
-        it.load_request(p, cut);
-        it.hg = (int)floor_div_exact(lo - ctl.found_excl, it.su);
-        it.vr_start = ctl.found_excl + (int64_t)it.hg * it.su;
-        it.ds = ctl.found_dexcl + (int64_t)it.hg * it.du;
-    } else {
-        it.b = 0;
-        it.hg = 0;
-        it.L = 0;
-        it.su = 0;
-        it.du = 0;
-        it.vr_start = 0;
-        it.ds = 0;
-    }
+    const SegIter it = slice_iter(p, ctl, cut, lo, hi, lens_s);
 
     if (warp == kProducerWarp) {
         run_producer<D, E>(p, cut, it, ctl, lens_s, pre_s, pre_d, full, empty, qfull, qempty, qarea, stage_base,
@@ -1758,7 +1851,7 @@ __global__ void __launch_bounds__(kDecodeThreads, 1) paged_decode_kernel(const _
         if (lane == 0) mbar_arrive(&qempty[qslot]);
         qslot ^= 1;
         if (qslot == 0) qphase ^= 1u;
-        const int patch_tile = s.patch >= 0 ? s.patch / p.ST : -1;
+        const int patch_tile = s.patch >= 0 ? s.patch >> p.st_log2 : -1;
         const int patch_tok = s.patch - patch_tile * p.ST;
 
         // -- tiles --

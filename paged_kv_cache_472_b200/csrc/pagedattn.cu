@@ -268,6 +268,8 @@ pa_status launch_decode(const void *q, const void *k_cache, const void *v_cache,
         return fail(PA_ERR_INVALID_ARG, "dynamic_share=%d outside [0, %d] or not available for this plan",
                     plan->dynamic_share, kMaxDynamicShare);
     if (!std::isfinite(scale)) return fail(PA_ERR_INVALID_ARG, "scale is not finite");
+    if (plan->flags & ~(PA_PLAN_NO_SPECULATION | PA_PLAN_TEST_MISGUESS))
+        return fail(PA_ERR_INVALID_ARG, "unknown plan flags %#x", plan->flags);
     if (!workspace) return fail(PA_ERR_WORKSPACE, "workspace is NULL");
     if (workspace_bytes < plan->workspace_bytes)
         return fail(PA_ERR_WORKSPACE, "workspace %zu bytes < %zu needed", workspace_bytes, plan->workspace_bytes);
@@ -344,6 +346,8 @@ pa_status launch_decode(const void *q, const void *k_cache, const void *v_cache,
     p.q_bytes = q_bytes;
     p.comb_stride = lay.comb_stride;
     p.bs_log2 = log2i(s->block_size);
+    p.st_log2 = log2i(plan->tile_tokens);
+    p.spec = (plan->flags & PA_PLAN_NO_SPECULATION) ? 0 : ((plan->flags & PA_PLAN_TEST_MISGUESS) ? 2 : 1);
     p.lens_cached = s->B <= pa::kLensCache ? 1 : 0;
     if (tensor_core_dtype(s->dtype)) {
         const int br = plan->tile_tokens < s->block_size ? plan->tile_tokens : s->block_size;

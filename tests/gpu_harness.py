@@ -58,11 +58,13 @@ def shape_of(case) -> Shape:
 
 
 def run(case, partition_tokens: int = 0, max_context_len: int | None = None, dev: DeviceCase | None = None,
-        append: bool = True, num_sms: int = 0):
-    """Append then decode on the GPU; returns (device case, decoder, device error word)."""
+        append: bool = True, num_sms: int = 0, flags: int = 0):
+    """Append then decode on the GPU; returns (device case, decoder, device error word).
+    `flags`: pa_plan_t.flags for the decode."""
     dev = dev or upload(case)
     mc = max_context_len if max_context_len is not None else max(int(case.context_lens.max()), 1)
     dec = PagedDecoder(shape_of(case), mc, partition_tokens, num_sms)
+    dec.plan.flags = flags
     if append:
         dec.append(dev.k_new, dev.v_new, dev.slot_mapping, dev.k_cache, dev.v_cache)
     dec.decode(dev.q, dev.k_cache, dev.v_cache, dev.block_tables, dev.context_lens, case.scale, dev.out)

@@ -143,6 +143,11 @@ def test_decode_validation_paths():
     assert _decode(s, plan, ws=0) == pa.PA_ERR_WORKSPACE
     assert _decode(s, plan, ws=FAKE + 16) == pa.PA_ERR_INVALID_ARG        # not 256-aligned
     assert _decode(s, plan, q=FAKE + 2) == pa.PA_ERR_INVALID_ARG          # not 16-aligned
+    plan.flags = 0x100                                                    # unknown flag bit
+    assert _decode(s, plan) == pa.PA_ERR_INVALID_ARG
+    plan.flags = pa.PLAN_NO_SPECULATION | pa.PLAN_TEST_MISGUESS
+    assert _decode(s, plan, ws=0) == pa.PA_ERR_WORKSPACE                  # known bits pass on to later checks
+    plan.flags = 0
     assert _decode(s, plan, out=0) == pa.PA_ERR_INVALID_ARG
     assert _decode(s, plan, scale=float("nan")) == pa.PA_ERR_INVALID_ARG
     s2 = pa.Shape(2, 8, 2, 128, 16, 9, 4, pa.DTYPE_BF16)                 # plan made for another shape

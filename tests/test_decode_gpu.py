@@ -12,7 +12,8 @@ import pytest
 import torch
 
 import synth
-from paged_kv_cache_472_b200 import DEVERR_BLOCK_ID, DEVERR_CONTEXT_LEN, DEVERR_SLOT
+from paged_kv_cache_472_b200 import (DEVERR_BLOCK_ID, DEVERR_CONTEXT_LEN, DEVERR_SLOT, PLAN_NO_SPECULATION,
+                                     PLAN_TEST_MISGUESS)
 from tests import gpu_harness as H
 
 pytestmark = pytest.mark.gpu
@@ -235,6 +236,40 @@ def test_fused_append_decode_matches_separate_calls(orc, cid, batch):
     assert torch.equal(dev_a.k_cache, dev_b.k_cache) and torch.equal(dev_a.v_cache, dev_b.v_cache)
     assert torch.equal(dev_a.out, dev_b.out)
     H.assert_close(H.out_f64(dev_b), oracle_out(orc, case), case.dtype, "fused")
+
+
+# ---- the early (speculative) plan: off, and always wrong (the start-over path) ----
+@pytest.mark.parametrize("flags", [PLAN_NO_SPECULATION, PLAN_TEST_MISGUESS])
+@pytest.mark.parametrize("cid,batch,pt", [(1, None, 0), (2, None, 0), (3, 32, 0), (4, 2, 512), (5, 48, 0)])
+def test_speculation_off_and_misguessed(orc, flags, cid, batch, pt):
+    """With the early plan turned off, or with every early guess made wrong on
+    purpose (so each CTA plans again after the grid-dependency wait), the
+    output still matches the oracle and nothing is flagged."""
+    case = synth.make_config(cid, batch=batch)
+    dev, dec, err = H.run(case, pt, flags=flags)
+    assert err == 0, f"device error word {err:#x}"
+    H.assert_close(H.out_f64(dev), oracle_out(orc, case), case.dtype, f"{case.name} flags={flags}")
+
+
+@pytest.mark.parametrize("cid,batch", [(2, None), (5, 48)])
+def test_fused_step_misguessed_matches(orc, cid, batch):
+    """The fused step with every early guess wrong: bit-identical to the fused
+    step that guessed right, over repeated steps on one workspace."""
+    case = synth.make_config(cid, batch=batch)
+    outs = []
+    for flags in (0, PLAN_TEST_MISGUESS):
+        dev = H.upload(case)
+        dec = H.PagedDecoder(H.shape_of(case), int(case.context_lens.max()), 0)
+        dec.plan.flags = flags
+        for _ in range(3):
+            dec.append_decode(dev.k_new, dev.v_new, dev.slot_mapping, dev.q, dev.k_cache, dev.v_cache,
+                              dev.block_tables, dev.context_lens, case.scale, dev.out)
+        torch.cuda.synchronize()
+        assert dec.device_error() == 0
+        outs.append(dev)
+    assert torch.equal(outs[0].out, outs[1].out)
+    assert torch.equal(outs[0].k_cache, outs[1].k_cache) and torch.equal(outs[0].v_cache, outs[1].v_cache)
+    H.assert_close(H.out_f64(outs[1]), oracle_out(orc, case), case.dtype, "fused misguessed")
 
 
 def _free_slot(case) -> int:
