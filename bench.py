@@ -1,4 +1,4 @@
-"""Benchmark: one decode step = pa_kv_append + pa_decode over one batch.
+"""Benchmark: one decode step = one pa_kv_append_decode launch (append + decode) over one batch.
 
 Default workload: the Qwen3-0.6B-shaped decode batch (B=32, Hq=16, Hkv=8,
 D=128, block_size=16, context lengths ~ U[128, 2048], bf16, shuffled pool).
@@ -13,7 +13,9 @@ cache; the K timed steps are bracketed by a barrier and a device synchronise
 and measured with CUDA events on the launching stream (max over ranks).  The
 decode kernel's own duration is taken with events around every launch.
 Under torchrun each rank runs its own batch (weak scaling, no collective on
-the data path).
+the data path).  The end-to-end leg stages each step's inputs in one pinned
+host buffer (one copy in) and reads the output back (one copy out) around the
+same C call.
 """
 from __future__ import annotations
 
@@ -298,22 +300,27 @@ def main():
         raise RuntimeError(f"device error word {err:#x}")
 
     # ---- end to end: host buffers through the same C calls ----
+    # the step's inputs staged in one pinned host buffer, uploaded with one
+    # copy; the result read back with one copy; the KV pool is resident state
+    from paged_kv_cache_472_b200.session import StepStaging
     E = args.e2e_steps
     c0 = copies[0]
-    host_in = {n: getattr(c0, n).cpu().pin_memory() for n in ("q", "k_new", "v_new", "slot_mapping",
-                                                               "block_tables", "context_lens")}
-    host_out = torch.empty(c0.out.shape, dtype=c0.out.dtype).pin_memory()
-    h2d = sum(v.numel() * v.element_size() for v in host_in.values())
-    d2h = host_out.numel() * host_out.element_size()
-    kn, vn, sm, kc, vc, q, bt, cl, out = ptrs[0]
+    names = StepStaging.ORDER
+    stg = StepStaging({n: (tuple(getattr(c0, n).shape), getattr(c0, n).dtype) for n in names},
+                      tuple(c0.out.shape), c0.out.dtype)
+    for n in names:
+        stg.host[n].copy_(getattr(c0, n).cpu())
+    h2d = stg.upload_bytes
+    d2h = stg.out.numel() * stg.out.element_size()
+    sq, skn, svn, ssm, scl, sbt = (stg.dev[n].data_ptr() for n in names)
+    kc, vc, out = c0.k_cache.data_ptr(), c0.v_cache.data_ptr(), c0.out.data_ptr()
     torch.cuda.synchronize()
     e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
     e0.record(stream)
     for i in range(E):
-        for n, hv in host_in.items():
-            getattr(c0, n).copy_(hv, non_blocking=True)
-        lib.pa_kv_append_decode(kn, vn, sm, q, kc, vc, bt, cl, scale, out, shp, pln, ws, wsb, sp)
-        host_out.copy_(c0.out, non_blocking=True)
+        stg.upload(stream)
+        lib.pa_kv_append_decode(skn, svn, ssm, sq, kc, vc, sbt, scl, scale, out, shp, pln, ws, wsb, sp)
+        stg.download(c0.out, stream)
     e1.record(stream)
     torch.cuda.synchronize()
     e2e_ms = max_over_ranks(e0.elapsed_time(e1) / E, world, "cuda")

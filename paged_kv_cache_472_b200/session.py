@@ -52,3 +52,48 @@ class PagedDecoder:
 
     def device_error(self, clear: bool = False) -> int:
         return pa_get_device_error(self.workspace, clear)
+
+
+class StepStaging:
+    """One decode step's per-step inputs (q, new K/V, slot mapping, context
+    lengths, block tables) packed in one pinned host buffer and one device
+    buffer, so a step uploads them with a single copy.  Each named view is a
+    tensor aligned to 256 bytes; write a step's values into ``host[name]``
+    and call ``upload()``; the library calls take ``dev[name]``.  ``out`` is
+    a pinned host tensor for the step's result (``download(out_dev)``)."""
+
+    ORDER = ("q", "k_new", "v_new", "slot_mapping", "context_lens", "block_tables")
+
+    def __init__(self, specs: dict, out_shape, out_dtype, device="cuda"):
+        # specs: name -> (shape, dtype)
+        offs, off = {}, 0
+        for name in self.ORDER:
+            shape, dtype = specs[name]
+            n = 1
+            for d in shape:
+                n *= int(d)
+            nbytes = n * torch.empty((), dtype=dtype).element_size()
+            offs[name] = (off, nbytes, shape, dtype)
+            off += (nbytes + 255) // 256 * 256
+        self.nbytes = off
+        self.host_buf = torch.empty(off, dtype=torch.uint8).pin_memory()
+        self.dev_buf = torch.empty(off, dtype=torch.uint8, device=device)
+        self.host, self.dev = {}, {}
+        for name, (o, nb, shape, dtype) in offs.items():
+            self.host[name] = self.host_buf[o:o + nb].view(dtype).view(*shape)
+            self.dev[name] = self.dev_buf[o:o + nb].view(dtype).view(*shape)
+        self.out = torch.empty(out_shape, dtype=out_dtype).pin_memory()
+
+    @property
+    def upload_bytes(self) -> int:
+        return self.nbytes
+
+    def upload(self, stream=None):
+        s = stream or torch.cuda.current_stream()
+        with torch.cuda.stream(s):
+            self.dev_buf.copy_(self.host_buf, non_blocking=True)
+
+    def download(self, out_dev: torch.Tensor, stream=None):
+        s = stream or torch.cuda.current_stream()
+        with torch.cuda.stream(s):
+            self.out.copy_(out_dev, non_blocking=True)

@@ -341,3 +341,31 @@ def test_fused_step_edge_shapes(orc, name, dtype, Hq, Hkv, D, bs, lens, pt):
     kc, vc = orc.kv_append(case)
     assert H.pool_equal(dev.k_cache, kc, case.dtype) and H.pool_equal(dev.v_cache, vc, case.dtype)
     H.assert_close(H.out_f64(dev), oracle_out(orc, case), case.dtype, name)
+
+
+def test_step_staging_one_copy_matches(orc):
+    """Inputs staged in one pinned buffer and uploaded with one copy (the
+    end-to-end path of the benchmark) give the same bytes as separate device
+    tensors."""
+    from paged_kv_cache_472_b200.session import StepStaging
+    case = synth.make_config(2, batch=6)
+    dev = H.upload(case)
+    names = StepStaging.ORDER
+    stg = StepStaging({n: (tuple(getattr(dev, n).shape), getattr(dev, n).dtype) for n in names},
+                      tuple(dev.out.shape), dev.out.dtype)
+    for n in names:
+        stg.host[n].copy_(getattr(dev, n).cpu())
+        assert stg.dev[n].data_ptr() % 256 == 0
+    stg.upload()
+    ref = H.upload(case)
+    dec = H.PagedDecoder(H.shape_of(case), int(case.context_lens.max()), 0)
+    dec.append_decode(stg.dev["k_new"], stg.dev["v_new"], stg.dev["slot_mapping"], stg.dev["q"], dev.k_cache,
+                      dev.v_cache, stg.dev["block_tables"], stg.dev["context_lens"], case.scale, dev.out)
+    stg.download(dev.out)
+    dec.append_decode(ref.k_new, ref.v_new, ref.slot_mapping, ref.q, ref.k_cache, ref.v_cache, ref.block_tables,
+                      ref.context_lens, case.scale, ref.out)
+    torch.cuda.synchronize()
+    assert dec.device_error() == 0
+    assert torch.equal(stg.out, ref.out.cpu())
+    assert torch.equal(dev.k_cache, ref.k_cache) and torch.equal(dev.v_cache, ref.v_cache)
+    H.assert_close(stg.out.float().numpy().astype(np.float64), oracle_out(orc, case), case.dtype, "staged")
