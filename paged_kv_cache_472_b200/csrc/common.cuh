@@ -292,6 +292,12 @@ struct Mma16<__nv_bfloat16> {
         mma_bf16_16816(d, a, b0, b1);
     }
     static __device__ __forceinline__ uint32_t pack(float lo, float hi) { return pack_bf16x2(lo, hi); }
+    // Softmax weights (finite, >= 0) rounded to nearest-even with integer
+    // operations: the same bits as pack(), off the conversion pipe.
+    static __device__ __forceinline__ uint32_t pack_p(float lo, float hi) {
+        const uint32_t a = __float_as_uint(lo), b = __float_as_uint(hi);
+        return __byte_perm(a + 0x7FFFu + ((a >> 16) & 1u), b + 0x7FFFu + ((b >> 16) & 1u), 0x7632);
+    }
     static __device__ __forceinline__ float2 unpack(uint32_t w) { return bf16x2_to_float2(w); }
 };
 
@@ -301,6 +307,7 @@ struct Mma16<__half> {
         mma_f16_16816(d, a, b0, b1);
     }
     static __device__ __forceinline__ uint32_t pack(float lo, float hi) { return pack_f16x2(lo, hi); }
+    static __device__ __forceinline__ uint32_t pack_p(float lo, float hi) { return pack_f16x2(lo, hi); }
     static __device__ __forceinline__ float2 unpack(uint32_t w) { return f16x2_to_float2(w); }
 };
 

@@ -792,16 +792,20 @@ struct MmaEngine {
     __device__ __forceinline__ void subtile(Unit &u, const unsigned char *tile_k, unsigned char *tile_v, int st,
                                             int g_local, int nvalid, const DecodeParams &p, float *, float *,
                                             int lane) const {
-        // ---- S^T[16 tok x 8 heads] = K Q^T ----
-        float s[4] = {0.f, 0.f, 0.f, 0.f};
+        // ---- S^T[16 tok x 8 heads] = K Q^T (two accumulation chains) ----
+        float s[4] = {0.f, 0.f, 0.f, 0.f}, sb[4] = {0.f, 0.f, 0.f, 0.f};
         const unsigned char *ka = row_ptr(tile_k, st * kSubTile + a_tok, g_local, p);
         const int swz = a_tok & 7;
 #pragma unroll
-        for (int ks = 0; ks < KS; ++ks) {
-            uint32_t a[4];
+        for (int ks = 0; ks < KS; ks += 2) {
+            uint32_t a[4], b[4];
             ldmatrix_x4(a, ka + chunk_off(ks * 2 + (a_col >> 3), swz, p));
+            ldmatrix_x4(b, ka + chunk_off((ks + 1) * 2 + (a_col >> 3), swz, p));
             Op::mma(s, a, u.qb[ks][0], u.qb[ks][1]);
+            Op::mma(sb, b, u.qb[ks + 1][0], u.qb[ks + 1][1]);
         }
+#pragma unroll
+        for (int i = 0; i < 4; ++i) s[i] += sb[i];
         // ---- online softmax over the 16 tokens, per head column ----
         const bool v0 = g4 < nvalid, v1 = g4 + 8 < nvalid;
         const float s0 = v0 ? s[0] * qscale : -INFINITY;
@@ -831,9 +835,9 @@ struct MmaEngine {
         // P = hi + lo, both bf16: the PV product then carries ~16 bits of each
         // weight instead of 8 (one bf16 P alone misses the tolerance on very
         // short, peaked contexts)
-        const uint32_t ph0 = Op::pack(p0, p1), ph1 = Op::pack(p2, p3);
+        const uint32_t ph0 = Op::pack_p(p0, p1), ph1 = Op::pack_p(p2, p3);
         const float2 h0 = Op::unpack(ph0), h1 = Op::unpack(ph1);
-        const uint32_t pl0 = Op::pack(p0 - h0.x, p1 - h0.y), pl1 = Op::pack(p2 - h1.x, p3 - h1.y);
+        const uint32_t pl0 = Op::pack_p(p0 - h0.x, p1 - h0.y), pl1 = Op::pack_p(p2 - h1.x, p3 - h1.y);
         // P^T fragments (k = token, n = head)
         const uint32_t bh0 = movmatrix_trans(ph0), bh1 = movmatrix_trans(ph1);
         const uint32_t bl0 = movmatrix_trans(pl0), bl1 = movmatrix_trans(pl1);
