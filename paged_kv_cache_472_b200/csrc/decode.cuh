@@ -954,20 +954,30 @@ struct ProducerState {
 
 // The block-table entries a piece reads, 32 at a time: lane i holds entry
 // base + i of the current window, and the next window is loaded one window
-// ahead.
+// ahead.  In the first window (where prefix-cached blocks sit) nb_val holds
+// the following request's entry in the same column: a block both rows name
+// (a prefix block the next request shares) is worth keeping in L2 until that
+// request reads it.
 struct TableWindow {
     const int32_t *table;
-    int nblk;
-    int cur_base, cur_val, nxt_base, nxt_val;
+    const int32_t *next_table;  // the following request's row (nullptr: none)
+    int nblk, next_nblk;
+    int cur_base, cur_val, nxt_base, nxt_val, nb_val;
 
+    __device__ __forceinline__ int next_row(int col) const {
+        return (next_table && col < 32 && col < next_nblk) ? next_table[col] : -2;
+    }
     // load the window holding the piece's first tile (and the one after it)
-    __device__ __forceinline__ void prime(const DecodeParams &p, const Seg &s, int lane) {
+    __device__ __forceinline__ void prime(const DecodeParams &p, const Seg &s, const int *lens_s, int lane) {
         table = p.block_tables + (size_t)s.b * p.max_blocks;
         nblk = (s.L + p.bs - 1) >> p.bs_log2;
+        next_table = s.b + 1 < p.B ? table + p.max_blocks : nullptr;
+        next_nblk = next_table ? (clamped_len(p, lens_s, s.b + 1) + p.bs - 1) >> p.bs_log2 : 0;
         cur_base = ((s.t_begin * p.ST) >> p.bs_log2) & ~31;
         nxt_base = cur_base + 32;
         cur_val = (cur_base + lane < nblk) ? table[cur_base + lane] : -1;
         nxt_val = (nxt_base + lane < nblk) ? table[nxt_base + lane] : -1;
+        nb_val = next_row(cur_base + lane);
     }
     // make the window holding block-table column jb current
     __device__ __forceinline__ void advance(int jb, int lane) {
@@ -981,6 +991,7 @@ struct TableWindow {
         cur_base = wb;
         nxt_base = wb + 32;
         nxt_val = (nxt_base + lane < nblk) ? table[nxt_base + lane] : -1;  // one window ahead
+        nb_val = next_row(wb + lane);
     }
 };
 
@@ -1038,7 +1049,7 @@ template <int D, int E>
 __device__ __forceinline__ void issue_tiles(const DecodeParams &p, ProducerState &ps, const Seg &s, int t_lo,
                                             int t_hi, TableWindow &win, bool grab_at_last, uint64_t *full,
                                             uint64_t *empty, unsigned char *stage_base, volatile int *abort_flag,
-                                            uint64_t policy, int lane) {
+                                            uint64_t policy, uint64_t policy_keep, int lane) {
     const unsigned char *kc = reinterpret_cast<const unsigned char *>(p.k_cache);
     const unsigned char *vc = reinterpret_cast<const unsigned char *>(p.v_cache);
     const uint32_t row_bytes = p.row_bytes, pitch = p.row_pitch;
@@ -1057,7 +1068,7 @@ __device__ __forceinline__ void issue_tiles(const DecodeParams &p, ProducerState
         const int ntok = min(p.ST, s.L - tok0);
         const int jb0 = tok0 >> p.bs_log2;
         win.advance(jb0, lane);
-        const int cur_base = win.cur_base, cur_val = win.cur_val;
+        const int cur_base = win.cur_base, cur_val = win.cur_val, nb_val = win.nb_val;
         unsigned char *kdst = stage_base + (size_t)ps.stage * 2 * p.half_bytes;
         unsigned char *vdst = kdst + p.half_bytes;
         uint32_t bytes = 0;
@@ -1070,6 +1081,8 @@ __device__ __forceinline__ void issue_tiles(const DecodeParams &p, ProducerState
             const int tp = tok0 + lane * br;  // first token of this lane's piece
             const int j = tp >> p.bs_log2;
             const int phys = __shfl_sync(0xffffffffu, cur_val, (j - cur_base) & 31);
+            const int next_phys = __shfl_sync(0xffffffffu, nb_val, (j - cur_base) & 31);
+            const uint64_t pol = next_phys == phys ? policy_keep : policy;
             bool valid = false;
             if (lane < npc) {
                 valid = phys >= 0 && phys < p.num_blocks;
@@ -1086,8 +1099,8 @@ __device__ __forceinline__ void issue_tiles(const DecodeParams &p, ProducerState
 #pragma unroll
                 for (int c2 = 0; c2 < NDC; ++c2) {
                     const size_t off = (size_t)(lane * NDC + c2) * box_bytes;
-                    tma_load_3d(kdst + off, &p.tmap_k, c2 * 64, row, head0, &full[ps.stage], policy);
-                    tma_load_3d(vdst + off, &p.tmap_v, c2 * 64, row, head0, &full[ps.stage], policy);
+                    tma_load_3d(kdst + off, &p.tmap_k, c2 * 64, row, head0, &full[ps.stage], pol);
+                    tma_load_3d(vdst + off, &p.tmap_v, c2 * 64, row, head0, &full[ps.stage], pol);
                 }
             }
         } else if (contiguous) {
@@ -1157,18 +1170,19 @@ __device__ __forceinline__ void run_producer(const DecodeParams &p, const Cut &k
                                              uint64_t *empty, uint64_t *qfull, uint64_t *qempty,
                                              unsigned char *qarea, unsigned char *stage_base,
                                              volatile int *abort_flag, int lane) {
-    const uint64_t policy = policy_evict_first();
+    const uint64_t policy = policy_evict_first();        // K/V read once per step
+    const uint64_t policy_keep = policy_evict_normal();  // blocks the next request shares
     ProducerState ps;
     Seg s;
     TableWindow win;
     // this CTA's static slice
     while (ps.ok && it.next(p, k, s)) {
-        win.prime(p, s, lane);  // in flight while q is published
+        win.prime(p, s, lens_s, lane);  // in flight while q is published
         fused_info(p, s, lane);
         publish(p, ps, s, ctl, qfull, qempty, qarea, abort_flag, D, E, lane);
         if (!ps.ok) break;
         issue_tiles<D, E>(p, ps, s, s.t_begin, s.t_end, win, k.dyn && it.cur >= it.hi, full, empty, stage_base,
-                          abort_flag, policy, lane);
+                          abort_flag, policy, policy_keep, lane);
     }
     // grains of the dynamic list, one at a time, to whichever CTA asks first
     if (k.dyn) {
@@ -1182,12 +1196,12 @@ __device__ __forceinline__ void run_producer(const DecodeParams &p, const Cut &k
             gi.y = j * k.g;
             gi.y1 = gi.y + k.g < k.Dn ? gi.y + k.g : k.Dn;
             while (ps.ok && gi.next(p, k, lens_s, pre_s, pre_d, s)) {
-                win.prime(p, s, lane);
+                win.prime(p, s, lens_s, lane);
                 fused_info(p, s, lane);
                 publish(p, ps, s, ctl, qfull, qempty, qarea, abort_flag, D, E, lane);
                 if (!ps.ok) break;
                 issue_tiles<D, E>(p, ps, s, s.t_begin, s.t_end, win, gi.y >= gi.y1, full, empty, stage_base,
-                                  abort_flag, policy, lane);
+                                  abort_flag, policy, policy_keep, lane);
             }
         }
         // the last CTA to find the list empty leaves the counters at zero for the next launch
