@@ -57,8 +57,9 @@ class Oracle:
         lib.oracle_decode_pairs.argtypes = [pp, vp, i32, vp, i32]
         lib.oracle_decode_partitioned.argtypes = [pp, i32, vp, i32]
         lib.oracle_kv_append.argtypes = [vp, vp, vp, vp, vp, i32, i32, i32, i32, i32, i32]
+        lib.oracle_prefill.argtypes = [pp, vp, vp, i32]
         for f in (lib.oracle_decode, lib.oracle_decode_pairs, lib.oracle_decode_partitioned,
-                  lib.oracle_kv_append, lib.oracle_max_threads):
+                  lib.oracle_kv_append, lib.oracle_max_threads, lib.oracle_prefill):
             f.restype = ctypes.c_int
         self.lib = lib
 
@@ -136,6 +137,35 @@ class Oracle:
         rc = self.lib.oracle_decode_partitioned(ctypes.byref(p), partition_tokens, out.ctypes.data, nthreads)
         if rc:
             raise ValueError(f"oracle_decode_partitioned rejected the input ({rc})")
+        return out
+
+
+    # -- chunked prefill ---------------------------------------------------
+    def prefill_append(self, pcase, k_cache=None, v_cache=None):
+        """(k_cache, v_cache) after writing every new token's K/V to its slot."""
+        vdt = np.float32 if pcase.dtype == "f32" else np.uint16
+        kc = np.array(pcase.k_cache if k_cache is None else k_cache, dtype=vdt, copy=True)
+        vc = np.array(pcase.v_cache if v_cache is None else v_cache, dtype=vdt, copy=True)
+        kn, vn = self._c(pcase.k_new, vdt), self._c(pcase.v_new, vdt)
+        sm = self._c(pcase.slot_mapping, np.int32)
+        rc = self.lib.oracle_kv_append(kn.ctypes.data, vn.ctypes.data, sm.ctypes.data, kc.ctypes.data,
+                                       vc.ctypes.data, pcase.T, pcase.Hkv, pcase.D, pcase.block_size,
+                                       kc.shape[0], self._dtype_code(pcase.dtype))
+        if rc < 0:
+            raise ValueError(f"oracle_kv_append rejected the input ({rc})")
+        return kc, vc
+
+    def prefill(self, pcase, k_cache=None, v_cache=None, *, q=None, nthreads: int = 0) -> np.ndarray:
+        """out[T, Hq, D] (float64) of the chunked prefill over the given pool
+        (default: the case's pool after its new tokens are written)."""
+        if k_cache is None or v_cache is None:
+            k_cache, v_cache = self.prefill_append(pcase)
+        p, keep = self._problem(pcase, pcase.q if q is None else q, k_cache, v_cache)
+        qs = self._c(pcase.query_start, np.int32)
+        out = np.zeros((pcase.T, pcase.Hq, pcase.D), dtype=np.float64)
+        rc = self.lib.oracle_prefill(ctypes.byref(p), qs.ctypes.data, out.ctypes.data, nthreads)
+        if rc:
+            raise ValueError(f"oracle_prefill rejected the input ({rc})")
         return out
 
 

@@ -22,6 +22,8 @@
  *   - the grouped-query head map is contiguous: query head h reads KV head
  *     h / (Hq / Hkv), the "repeat each KV head Hq/Hkv times" form of GQA
  *     (MQA is Hkv = 1, MHA is Hkv = Hq);
+ *   - chunked prefill (oracle_prefill) applies the same definition to every
+ *     new token of a request over the positions up to its own (causal);
  *   - the partitioned form (oracle_decode_partitioned) splits each context
  *     into fixed token partitions, keeps (max, sum of weights, weighted sum
  *     of V) per partition and combines them by log-sum-exp; it exists only
@@ -305,6 +307,102 @@ int oracle_decode_partitioned(const oracle_problem *p, int partition_tokens, dou
         free(pm);
         free(pl);
         free(po);
+    }
+    return err;
+}
+
+/* Chunked prefill: the step before decode, in which a request's new tokens
+ * attend to its cached history and to each other, causally (the MinivLLM
+ * review's prefill path, read over the paged cache).  Request b owns rows
+ * query_start[b] .. query_start[b+1]-1 of q and of out: n_b new tokens, the
+ * last n_b of its context_lens[b] positions, whose K/V are already in the
+ * cache (written by the append, one slot per token).  New token j sits at
+ * position pos = context_lens[b] - n_b + j and attends to positions
+ * 0 .. pos: the decode definition above applied to that prefix, with q row
+ * query_start[b] + j. */
+static double score_prefill(const oracle_problem *p, int64_t row, int b, int h, int t)
+{
+    int g = h / (p->Hq / p->Hkv);
+    double dot = 0.0;
+    for (int d = 0; d < p->D; ++d) {
+        double qd = value_at(p->q, (row * p->Hq + h) * p->D + d, p->dtype);
+        double kd = value_at(p->k_cache, kv_index(p, b, t, g, d), p->dtype);
+        dot += qd * kd;
+    }
+    return p->scale * dot;
+}
+
+static void attend_prefill(const oracle_problem *p, int64_t row, int b, int h, int visible, double *s,
+                           double *out)
+{
+    int g = h / (p->Hq / p->Hkv);
+    for (int d = 0; d < p->D; ++d)
+        out[d] = 0.0;
+    if (visible <= 0)
+        return;
+    for (int t = 0; t < visible; ++t)
+        s[t] = score_prefill(p, row, b, h, t);
+    double m = s[0];
+    for (int t = 1; t < visible; ++t)
+        if (s[t] > m)
+            m = s[t];
+    double den = 0.0;
+    for (int t = 0; t < visible; ++t) {
+        double w = exp(s[t] - m);
+        den += w;
+        for (int d = 0; d < p->D; ++d)
+            out[d] += w * value_at(p->v_cache, kv_index(p, b, t, g, d), p->dtype);
+    }
+    for (int d = 0; d < p->D; ++d)
+        out[d] /= den;
+}
+
+/* out[T, Hq, D] for the T = query_start[B] new tokens.  Returns 0, or a
+ * negative code for a malformed problem (query_start not starting at 0,
+ * decreasing, or giving a request more new tokens than its context holds). */
+int oracle_prefill(const oracle_problem *p, const int32_t *query_start, double *out, int nthreads)
+{
+    int rc = check_problem(p);
+    if (rc)
+        return rc;
+    if (!query_start || query_start[0] != 0)
+        return -10;
+    for (int b = 0; b < p->B; ++b) {
+        int32_t n = query_start[b + 1] - query_start[b];
+        if (n < 0 || n > p->context_lens[b])
+            return -10;
+    }
+    int64_t T = query_start[p->B];
+    int64_t pairs = T * p->Hq;
+    int Lmax = max_context(p);
+    int err = 0;
+#pragma omp parallel num_threads(nthreads > 0 ? nthreads : omp_get_max_threads())
+    {
+        double *s = (double *)malloc(sizeof(double) * (size_t)Lmax);
+        if (!s) {
+#pragma omp atomic write
+            err = -7;
+        }
+#pragma omp for schedule(dynamic, 1)
+        for (int64_t i = 0; i < pairs; ++i) {
+            if (!s)
+                continue;
+            int64_t row = i / p->Hq;
+            int h = (int)(i % p->Hq);
+            int lo = 0, hi = p->B;  /* request owning the row: query_start[b] <= row < query_start[b+1] */
+            while (hi - lo > 1) {
+                int mid = (lo + hi) / 2;
+                if (query_start[mid] <= row)
+                    lo = mid;
+                else
+                    hi = mid;
+            }
+            int b = lo;
+            int n = query_start[b + 1] - query_start[b];
+            int pos = p->context_lens[b] - n + (int)(row - query_start[b]);
+            attend_prefill(p, row, b, h, pos + 1, s, out + i * p->D);
+        }
+        free(s);
     }
     return err;
 }

@@ -322,6 +322,152 @@ def make_config(cid: int, seed: int | None = None, batch: int | None = None,
     raise ValueError(cid)
 
 
+# ----------------------------------------------------------------------------
+# Chunked prefill: several new tokens per request.
+# ----------------------------------------------------------------------------
+@dataclass
+class PagedPrefillCase:
+    """One chunked-prefill step's inputs (host numpy arrays, value arrays as in
+    PagedDecodeCase).  Request b owns rows query_start[b] .. query_start[b+1]-1
+    of q / k_new / v_new / slot_mapping: its n_b new tokens, the last n_b of
+    its context_lens[b] positions.  ``k_cache``/``v_cache`` hold the history
+    (and stale values at the new tokens' slots, overwritten by the append)."""
+    name: str
+    dtype: str
+    B: int
+    T: int
+    Hq: int
+    Hkv: int
+    D: int
+    block_size: int
+    num_blocks: int
+    max_blocks_per_seq: int
+    context_lens: np.ndarray      # [B] int32, history + new tokens
+    query_start: np.ndarray       # [B + 1] int32
+    block_tables: np.ndarray      # [B, max_blocks_per_seq] int32
+    slot_mapping: np.ndarray      # [T] int32
+    q: np.ndarray                 # [T, Hq, D]
+    k_new: np.ndarray             # [T, Hkv, D]
+    v_new: np.ndarray             # [T, Hkv, D]
+    k_cache: np.ndarray
+    v_cache: np.ndarray
+    scale: float
+    seed: int = 0
+    notes: dict = field(default_factory=dict)
+
+    @property
+    def elem_bytes(self) -> int:
+        return 4 if self.dtype == DTYPE_F32 else 2
+
+    @property
+    def group(self) -> int:
+        return self.Hq // self.Hkv
+
+    def as_float32(self, a: np.ndarray) -> np.ndarray:
+        if self.dtype == DTYPE_BF16:
+            return bf16_bits_to_f32(a)
+        if self.dtype == DTYPE_F16:
+            return np.asarray(a, np.uint16).view(np.float16).astype(np.float32)
+        return np.asarray(a, np.float32)
+
+    def new_tokens(self) -> np.ndarray:
+        return np.diff(self.query_start.astype(np.int64))
+
+    def positions(self) -> np.ndarray:
+        """[T] position of every new token in its request's context."""
+        pos = np.empty(self.T, dtype=np.int64)
+        for b in range(self.B):
+            q0, q1 = int(self.query_start[b]), int(self.query_start[b + 1])
+            pos[q0:q1] = int(self.context_lens[b]) - (q1 - q0) + np.arange(q1 - q0)
+        return pos
+
+    def visible_pairs(self) -> int:
+        """(query token, key position) pairs the causal prefill computes."""
+        return int((self.positions() + 1).sum())
+
+
+_STREAM_PQ, _STREAM_PKNEW, _STREAM_PVNEW = 5, 6, 7
+
+
+def build_prefill_case(name: str, *, dtype: str, Hq: int, Hkv: int, D: int, block_size: int, context_lens,
+                       new_tokens, seed: int, values: bool = True, **pool) -> PagedPrefillCase:
+    """A seeded prefill step: the pool, tables and history as build_case makes
+    them for ``context_lens`` (history + new tokens), the new tokens' slots,
+    and q / new K / new V for every new token."""
+    lens = np.asarray(context_lens, dtype=np.int64)
+    n = np.asarray(new_tokens, dtype=np.int64)
+    assert lens.shape == n.shape and np.all(n >= 0) and np.all(n <= lens)
+    base = build_case(name, dtype=dtype, Hq=Hq, Hkv=Hkv, D=D, block_size=block_size, context_lens=lens,
+                      seed=seed, values=values, **pool)
+    B, bs = base.B, block_size
+    qs = np.zeros(B + 1, dtype=np.int32)
+    qs[1:] = np.cumsum(n)
+    T = int(qs[-1])
+    slots = np.empty(T, dtype=np.int32)
+    for b in range(B):
+        for j in range(int(n[b])):
+            pos = int(lens[b]) - int(n[b]) + j
+            slots[qs[b] + j] = int(base.block_tables[b, pos // bs]) * bs + pos % bs
+    if values:
+        vseed = int(np.random.default_rng(seed ^ 0x5DEECE66D).integers(0, 2**63 - 1))
+        q = normals(vseed, _STREAM_PQ, (T, Hq, D), dtype)
+        k_new = normals(vseed, _STREAM_PKNEW, (T, Hkv, D), dtype)
+        v_new = normals(vseed, _STREAM_PVNEW, (T, Hkv, D), dtype)
+    else:
+        shp = lambda *s_: np.zeros(s_, dtype=np.float32 if dtype == DTYPE_F32 else np.uint16)
+        q, k_new, v_new = shp(T, Hq, D), shp(T, Hkv, D), shp(T, Hkv, D)
+    return PagedPrefillCase(name=name, dtype=dtype, B=B, T=T, Hq=Hq, Hkv=Hkv, D=D, block_size=bs,
+                            num_blocks=base.num_blocks, max_blocks_per_seq=base.max_blocks_per_seq,
+                            context_lens=base.context_lens, query_start=qs, block_tables=base.block_tables,
+                            slot_mapping=slots, q=q, k_new=k_new, v_new=v_new, k_cache=base.k_cache,
+                            v_cache=base.v_cache, scale=1.0 / math.sqrt(D), seed=seed, notes=base.notes)
+
+
+PREFILL_NAMES = {
+    1: "qwen3-8b-prefill-chunk512-b8",
+    2: "llama-3.2-1b-prefill-mixed-b16",
+}
+
+
+def make_prefill_config(pid: int, seed: int | None = None, batch: int | None = None, chunk: int | None = None,
+                        values: bool = True) -> PagedPrefillCase:
+    """Chunked-prefill workloads (seed 2000 + pid unless given):
+      1. Qwen3-8B-shaped chunk: B=8, 32/8/128, bs=16, history ~ U[0, 3584],
+         512 new tokens per request (a 4096-token chunk);
+      2. Llama-3.2-1B-shaped mixed: B=16, 32/8/64, bs=16, history ~ U[0, 2048],
+         new tokens ~ U[1, 512] (some requests fresh, some continuing).
+    ``batch`` / ``chunk`` shrink the batch / the new tokens per request."""
+    seed = 2000 + pid if seed is None else seed
+    rng = np.random.default_rng(seed)
+    sub = int(rng.integers(0, 2**31 - 1))
+    name = PREFILL_NAMES[pid] + ("" if batch is None and chunk is None else f"-subset{batch}x{chunk}")
+    if pid == 1:
+        B = batch or 8
+        n = np.full(B, chunk or 512, dtype=np.int64)
+        hist = rng.integers(0, 3584, size=B, endpoint=True)
+        return build_prefill_case(name, dtype=DTYPE_BF16, Hq=32, Hkv=8, D=128, block_size=16,
+                                  context_lens=hist + n, new_tokens=n, seed=sub, values=values, pool="exact")
+    if pid == 2:
+        B = batch or 16
+        n = rng.integers(1, chunk or 512, size=B, endpoint=True)
+        hist = rng.integers(0, 2048, size=B, endpoint=True)
+        hist[::4] = 0  # every fourth request starts fresh
+        return build_prefill_case(name, dtype=DTYPE_BF16, Hq=32, Hkv=8, D=64, block_size=16,
+                                  context_lens=hist + n, new_tokens=n, seed=sub, values=values,
+                                  pool="factor", pool_factor=1.25)
+    raise ValueError(pid)
+
+
+def prefill_algorithmic(pc: PagedPrefillCase) -> dict:
+    """Flops of the causal prefill (QK^T and PV over the visible pairs) and
+    the bytes it must move at least (each request's K/V once, q in, out)."""
+    e = pc.elem_bytes
+    flops = 4 * pc.visible_pairs() * pc.Hq * pc.D
+    kv = int(pc.context_lens.astype(np.int64).sum()) * pc.Hkv * pc.D * e * 2
+    qo = 2 * pc.T * pc.Hq * pc.D * e
+    return {"flops": flops, "bytes": kv + qo}
+
+
 def algorithmic_bytes(case: PagedDecodeCase) -> dict:
     """Bytes one decode step must move: K+V each request reads, q in, out
     written, block-table entries and lengths read.  Append bytes (read

@@ -8,7 +8,10 @@ oracle disagrees with something that does not come from the oracle itself:
   * invariants the pages state or imply: paged == contiguous storage,
     GQA/MQA == MHA with repeated KV heads, physical block ids can be permuted,
     one token returns V, identical keys return the mean of V,
-    partition + log-sum-exp merge == unsplit.
+    partition + log-sum-exp merge == unsplit;
+  * for chunked prefill: brute force, one new token == decode, a fresh
+    request's first token returns its own V, causality (a later token's K/V
+    never reaches an earlier token).
 The same pins run against deliberately broken copies of the oracle
 (tests/test_oracle_mutants.py), so each plausible slip fails at least one.
 """
@@ -279,10 +282,115 @@ def pin_append_matches_index_assignment(orc):
         assert np.array_equal(vc.reshape(ev.shape).view(np.uint8), ev.view(np.uint8)), case.name
 
 
+# ---- chunked prefill ----------------------------------------------------
+def tiny_prefill_cases():
+    """Small prefill steps: fresh requests (no history), continuing ones,
+    one new token, MHA/GQA/MQA, block sizes 1..16, fp32 and bf16."""
+    specs = [
+        dict(dtype=DTYPE_F32, Hq=4, Hkv=2, D=8, block_size=4, context_lens=[5, 9, 3], new_tokens=[5, 3, 1], seed=31),
+        dict(dtype=DTYPE_BF16, Hq=4, Hkv=1, D=8, block_size=2, context_lens=[7, 4], new_tokens=[2, 4], seed=32),
+        dict(dtype=DTYPE_F32, Hq=3, Hkv=3, D=4, block_size=1, context_lens=[6, 2], new_tokens=[6, 1], seed=33),
+        dict(dtype=DTYPE_BF16, Hq=8, Hkv=2, D=16, block_size=16, context_lens=[17, 40], new_tokens=[17, 9],
+             seed=34, pool="factor", pool_factor=1.5),
+    ]
+    return [synth.build_prefill_case(f"ptiny{i}", **sp) for i, sp in enumerate(specs)]
+
+
+def prefill_brute_force(pc, k_cache, v_cache):
+    """Plain-Python causal attention: new token j of request b at position
+    L_b - n_b + j over positions 0..that position."""
+    q = _f64(pc, pc.q)
+    K = _f64(pc, k_cache)
+    V = _f64(pc, v_cache)
+    G = pc.Hq // pc.Hkv
+    out = np.zeros((pc.T, pc.Hq, pc.D))
+    for b in range(pc.B):
+        L = int(pc.context_lens[b])
+        q0, q1 = int(pc.query_start[b]), int(pc.query_start[b + 1])
+        n = q1 - q0
+        for j in range(n):
+            pos = L - n + j
+            rows = [(int(pc.block_tables[b][t // pc.block_size]), t % pc.block_size) for t in range(pos + 1)]
+            for h in range(pc.Hq):
+                g = h // G
+                s_ = [pc.scale * sum(float(q[q0 + j, h, d]) * float(K[p_, o, g, d]) for d in range(pc.D))
+                      for (p_, o) in rows]
+                m = max(s_)
+                w = [math.exp(x - m) for x in s_]
+                tot = sum(w)
+                for d in range(pc.D):
+                    out[q0 + j, h, d] = sum(w[i] * float(V[p_, o, g, d]) for i, (p_, o) in enumerate(rows)) / tot
+    return out
+
+
+def pin_prefill_brute_force(orc):
+    for pc in tiny_prefill_cases():
+        kc, vc = orc.prefill_append(pc)
+        np.testing.assert_allclose(orc.prefill(pc, kc, vc), prefill_brute_force(pc, kc, vc), rtol=1e-12,
+                                   atol=1e-13, err_msg=pc.name)
+
+
+def pin_prefill_one_token_is_decode(orc):
+    """One new token per request: prefill is exactly the decode step."""
+    for dc in tiny_cases() + [synth.make_config(1)]:
+        kc, vc = orc.kv_append(dc)
+        pc = synth.PagedPrefillCase(
+            name=dc.name + "-as-prefill", dtype=dc.dtype, B=dc.B, T=dc.B, Hq=dc.Hq, Hkv=dc.Hkv, D=dc.D,
+            block_size=dc.block_size, num_blocks=dc.num_blocks, max_blocks_per_seq=dc.max_blocks_per_seq,
+            context_lens=dc.context_lens, query_start=np.arange(dc.B + 1, dtype=np.int32),
+            block_tables=dc.block_tables, slot_mapping=dc.slot_mapping, q=dc.q, k_new=dc.k_new, v_new=dc.v_new,
+            k_cache=kc, v_cache=vc, scale=dc.scale)
+        assert np.array_equal(orc.prefill(pc, kc, vc), orc.decode(dc, kc, vc)), dc.name
+
+
+def pin_prefill_fresh_first_token_is_v(orc):
+    """A request with no history: its first new token sees only itself, so
+    its output is its own V row, exactly."""
+    for pc in tiny_prefill_cases():
+        kc, vc = orc.prefill_append(pc)
+        out = orc.prefill(pc, kc, vc)
+        vnew = _f64(pc, pc.v_new)
+        G = pc.Hq // pc.Hkv
+        for b in range(pc.B):
+            q0, q1 = int(pc.query_start[b]), int(pc.query_start[b + 1])
+            if q1 - q0 != int(pc.context_lens[b]) or q1 == q0:
+                continue
+            for h in range(pc.Hq):
+                assert np.array_equal(out[q0, h], vnew[q0, h // G]), (pc.name, b, h)
+
+
+def pin_prefill_causal(orc):
+    """Changing the K/V of a request's last new token changes only that
+    token's output: no earlier token sees a later one."""
+    for pc in tiny_prefill_cases():
+        kc, vc = orc.prefill_append(pc)
+        out = orc.prefill(pc, kc, vc)
+        pos = pc.positions()
+        for b in range(pc.B):
+            q0, q1 = int(pc.query_start[b]), int(pc.query_start[b + 1])
+            if q1 - q0 < 2:
+                continue
+            last = q1 - 1
+            slot = int(pc.slot_mapping[last])
+            k2, v2 = kc.copy(), vc.copy()
+            blk, row = slot // pc.block_size, slot % pc.block_size
+            if k2.dtype == np.uint16:                      # flip the sign of every value of that token
+                k2[blk, row] ^= np.uint16(0x8000)
+                v2[blk, row] ^= np.uint16(0x8000)
+            else:
+                k2[blk, row] = -k2[blk, row]
+                v2[blk, row] = -v2[blk, row]
+            out2 = orc.prefill(pc, k2, v2)
+            assert np.array_equal(out[q0:last], out2[q0:last]), (pc.name, b, "earlier tokens changed")
+            assert not np.array_equal(out[last], out2[last]), (pc.name, b, "the last token did not see itself")
+            assert pos[last] == int(pc.context_lens[b]) - 1
+
+
 ALL_PINS = [pin_golden_decode, pin_golden_append, pin_brute_force, pin_dense_numpy,
             pin_paged_equals_contiguous, pin_gqa_equals_repeated_mha, pin_block_permutation,
             pin_single_token_returns_v, pin_identical_keys_mean_v, pin_partitioned_equals_unsplit,
-            pin_append_matches_index_assignment]
+            pin_append_matches_index_assignment, pin_prefill_brute_force, pin_prefill_one_token_is_decode,
+            pin_prefill_fresh_first_token_is_v, pin_prefill_causal]
 
 
 if __name__ == "__main__":

@@ -31,6 +31,16 @@ MUTANTS = {
     "append_offset_dropped": ("int64_t offset = s % block_size;", "int64_t offset = 0;"),
     "append_v_from_k": ("memcpy((char *)v_cache + dst, (const char *)v_new",
                         "memcpy((char *)v_cache + dst, (const char *)k_new"),
+    "prefill_sees_one_future_token": ("attend_prefill(p, row, b, h, pos + 1, s, out + i * p->D);",
+                                      "attend_prefill(p, row, b, h, pos + 2 <= p->context_lens[b] ? pos + 2 : pos + 1, s, out + i * p->D);"),
+    "prefill_misses_itself": ("attend_prefill(p, row, b, h, pos + 1, s, out + i * p->D);",
+                              "attend_prefill(p, row, b, h, pos > 0 ? pos : 1, s, out + i * p->D);"),
+    "prefill_positions_from_zero": ("int pos = p->context_lens[b] - n + (int)(row - query_start[b]);",
+                                    "int pos = (int)(row - query_start[b]);"),
+    "prefill_not_causal": ("attend_prefill(p, row, b, h, pos + 1, s, out + i * p->D);",
+                           "attend_prefill(p, row, b, h, p->context_lens[b], s, out + i * p->D);"),
+    "prefill_q_row_of_request": ("double qd = value_at(p->q, (row * p->Hq + h) * p->D + d, p->dtype);",
+                                 "double qd = value_at(p->q, ((int64_t)b * p->Hq + h) * p->D + d, p->dtype);"),
 }
 
 

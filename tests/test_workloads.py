@@ -75,3 +75,23 @@ def test_config_is_deterministic():
     b = synth.make_config(1)
     for f in ("q", "k_new", "v_new", "k_cache", "v_cache", "block_tables", "slot_mapping", "context_lens"):
         assert np.array_equal(getattr(a, f), getattr(b, f))
+
+
+@pytest.mark.parametrize("pid", [1, 2])
+def test_prefill_config_structure(pid):
+    pc = synth.make_prefill_config(pid, values=False)
+    qs = pc.query_start.astype(np.int64)
+    n = np.diff(qs)
+    assert qs[0] == 0 and qs[-1] == pc.T and np.all(n >= 1) and np.all(n <= pc.context_lens)
+    pos = pc.positions()
+    for b in range(pc.B):
+        L = int(pc.context_lens[b])
+        nblk = -(-L // pc.block_size)
+        assert np.all((pc.block_tables[b, :nblk] >= 0) & (pc.block_tables[b, :nblk] < pc.num_blocks))
+        for i in range(qs[b], qs[b + 1]):
+            assert pos[i] == L - n[b] + (i - qs[b])
+            p_ = int(pos[i])
+            assert pc.slot_mapping[i] == pc.block_tables[b, p_ // pc.block_size] * pc.block_size + p_ % pc.block_size
+    assert len(set(pc.slot_mapping.tolist())) == pc.T          # distinct slots
+    again = synth.make_prefill_config(pid, values=False)
+    assert np.array_equal(again.context_lens, pc.context_lens) and np.array_equal(again.slot_mapping, pc.slot_mapping)
