@@ -225,6 +225,50 @@ pa_status pa_decode_no_alloc(const void *q, const void *k_cache, const void *v_c
                              const int32_t *context_lens, float scale, void *out, const pa_shape *s,
                              const pa_plan_t *plan, void *stream);
 
+/*
+ * Chunked prefill over the paged cache (the step before decode: a request's
+ * new tokens attend to its cached history and to each other, causally; the
+ * MinivLLM review's prefill path, read straight from the pages).
+ *
+ * Host-only planner.  s->B is the number of requests; max_new_tokens bounds
+ * query_start[b+1] - query_start[b] for every later call.  Supported: bf16
+ * and fp16; D in {64, 128}; block_size a power of two in [16, 256]; a GQA
+ * group Hq/Hkv that is a power of two <= 128.
+ */
+typedef struct {
+    int32_t q_tile;          /* new tokens per CTA (q_tile * Hq/Hkv rows) */
+    int32_t kv_tile;         /* keys per pipeline stage */
+    int32_t stages;
+    int32_t num_qtiles;      /* tiles of q_tile tokens per request the grid covers */
+    int32_t max_new_tokens;
+    int32_t smem_bytes;
+    pa_shape shape;
+} pa_prefill_plan_t;
+
+pa_status pa_prefill_plan(const pa_shape *s, int32_t max_new_tokens, pa_prefill_plan_t *plan_out);
+
+/*
+ * Prefill attention.  Request b owns rows query_start[b] .. query_start[b+1]-1
+ * of q and out: its n_b new tokens, the last n_b of its context_lens[b]
+ * positions, whose K/V must already be in the cache (pa_kv_append with one
+ * row per new token: a shape whose B is the number of new tokens).  New
+ * token j of request b sits at position context_lens[b] - n_b + j and
+ * attends to positions 0 .. that position:
+ *     out[row][h] = sum_{t <= pos} softmax_t(scale * q[row][h] . K[t]) V[t].
+ *   q, out       : device, [T, Hq, D], T = query_start[B], dtype s->dtype
+ *   query_start  : device, [B + 1] int32, query_start[0] = 0, non-decreasing
+ *   context_lens : device, [B] int32 (history + new tokens)
+ *   block_tables, k_cache, v_cache : as for pa_decode
+ *   device_error : device int32 or NULL; a request with a length outside
+ *                  [0, max_blocks_per_seq*block_size], more new tokens than
+ *                  its length or than the plan covers is skipped and sets
+ *                  PA_DEVERR_CONTEXT_LEN; a bad block id sets PA_DEVERR_BLOCK_ID.
+ * No workspace; nothing is allocated.  Queued on `stream`.
+ */
+pa_status pa_prefill(const void *q, const void *k_cache, const void *v_cache, const int32_t *block_tables,
+                     const int32_t *context_lens, const int32_t *query_start, float scale, void *out,
+                     const pa_shape *s, const pa_prefill_plan_t *plan, int32_t *device_error, void *stream);
+
 /* Copy the device error word of `workspace` to *err_out (synchronises
  * `stream`; not for the hot path).  clear != 0 resets it to 0 afterwards. */
 pa_status pa_get_device_error(void *workspace, int32_t clear, int32_t *err_out, void *stream);

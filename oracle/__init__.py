@@ -58,8 +58,9 @@ class Oracle:
         lib.oracle_decode_partitioned.argtypes = [pp, i32, vp, i32]
         lib.oracle_kv_append.argtypes = [vp, vp, vp, vp, vp, i32, i32, i32, i32, i32, i32]
         lib.oracle_prefill.argtypes = [pp, vp, vp, i32]
+        lib.oracle_prefill_rows.argtypes = [pp, vp, vp, i32, vp, i32]
         for f in (lib.oracle_decode, lib.oracle_decode_pairs, lib.oracle_decode_partitioned,
-                  lib.oracle_kv_append, lib.oracle_max_threads, lib.oracle_prefill):
+                  lib.oracle_kv_append, lib.oracle_max_threads, lib.oracle_prefill, lib.oracle_prefill_rows):
             f.restype = ctypes.c_int
         self.lib = lib
 
@@ -166,6 +167,20 @@ class Oracle:
         rc = self.lib.oracle_prefill(ctypes.byref(p), qs.ctypes.data, out.ctypes.data, nthreads)
         if rc:
             raise ValueError(f"oracle_prefill rejected the input ({rc})")
+        return out
+
+    def prefill_rows(self, pcase, rows, k_cache=None, v_cache=None, nthreads: int = 0) -> np.ndarray:
+        """out[len(rows), Hq, D] of the prefill for the listed q rows only."""
+        if k_cache is None or v_cache is None:
+            k_cache, v_cache = self.prefill_append(pcase)
+        p, keep = self._problem(pcase, pcase.q, k_cache, v_cache)
+        qs = self._c(pcase.query_start, np.int32)
+        r = self._c(np.asarray(rows).reshape(-1), np.int64)
+        out = np.zeros((r.shape[0], pcase.Hq, pcase.D), dtype=np.float64)
+        rc = self.lib.oracle_prefill_rows(ctypes.byref(p), qs.ctypes.data, r.ctypes.data, r.shape[0],
+                                          out.ctypes.data, nthreads)
+        if rc:
+            raise ValueError(f"oracle_prefill_rows rejected the input ({rc})")
         return out
 
 

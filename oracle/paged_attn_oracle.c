@@ -407,6 +407,58 @@ int oracle_prefill(const oracle_problem *p, const int32_t *query_start, double *
     return err;
 }
 
+/* oracle_prefill for the listed rows only (all heads): out[nrows, Hq, D].
+ * Used to check sampled rows of large prefill steps. */
+int oracle_prefill_rows(const oracle_problem *p, const int32_t *query_start, const int64_t *rows, int nrows,
+                        double *out, int nthreads)
+{
+    int rc = check_problem(p);
+    if (rc)
+        return rc;
+    if (!query_start || query_start[0] != 0)
+        return -10;
+    for (int b = 0; b < p->B; ++b) {
+        int32_t n = query_start[b + 1] - query_start[b];
+        if (n < 0 || n > p->context_lens[b])
+            return -10;
+    }
+    for (int i = 0; i < nrows; ++i)
+        if (rows[i] < 0 || rows[i] >= query_start[p->B])
+            return -11;
+    int Lmax = max_context(p);
+    int64_t pairs = (int64_t)nrows * p->Hq;
+    int err = 0;
+#pragma omp parallel num_threads(nthreads > 0 ? nthreads : omp_get_max_threads())
+    {
+        double *s = (double *)malloc(sizeof(double) * (size_t)Lmax);
+        if (!s) {
+#pragma omp atomic write
+            err = -7;
+        }
+#pragma omp for schedule(dynamic, 1)
+        for (int64_t i = 0; i < pairs; ++i) {
+            if (!s)
+                continue;
+            int64_t row = rows[i / p->Hq];
+            int h = (int)(i % p->Hq);
+            int lo = 0, hi = p->B;
+            while (hi - lo > 1) {
+                int mid = (lo + hi) / 2;
+                if (query_start[mid] <= row)
+                    lo = mid;
+                else
+                    hi = mid;
+            }
+            int b = lo;
+            int n = query_start[b + 1] - query_start[b];
+            int pos = p->context_lens[b] - n + (int)(row - query_start[b]);
+            attend_prefill(p, row, b, h, pos + 1, s, out + i * p->D);
+        }
+        free(s);
+    }
+    return err;
+}
+
 /* KV append: for each request i with slot s = slot_mapping[i] >= 0, copy the
  * new token's K (all KV heads) into block s / block_size, offset
  * s % block_size, and the same for V (the BareLLM README's "logical-to-

@@ -18,7 +18,7 @@ __all__ = ["PagedAttnError", "Shape", "Plan", "DTYPE_F32", "DTYPE_BF16", "DTYPE_
            "PLAN_NO_SPECULATION", "PLAN_TEST_MISGUESS",
            "pa_version", "pa_status_str", "pa_last_error_message", "pa_kv_append", "pa_plan",
            "pa_decode_workspace_size", "pa_workspace_init", "pa_decode", "pa_kv_append_decode", "pa_get_device_error",
-           "pa_decode_no_alloc", "lib"]
+           "pa_decode_no_alloc", "PrefillPlan", "pa_prefill_plan", "pa_prefill", "lib"]
 
 PA_OK, PA_ERR_INVALID_ARG, PA_ERR_UNSUPPORTED, PA_ERR_CUDA, PA_ERR_WORKSPACE = range(5)
 DTYPE_F32, DTYPE_BF16, DTYPE_F16 = 0, 1, 2
@@ -51,6 +51,12 @@ class Plan(ctypes.Structure):
         return d
 
 
+class PrefillPlan(ctypes.Structure):
+    _fields_ = [("q_tile", ctypes.c_int32), ("kv_tile", ctypes.c_int32), ("stages", ctypes.c_int32),
+                ("num_qtiles", ctypes.c_int32), ("max_new_tokens", ctypes.c_int32), ("smem_bytes", ctypes.c_int32),
+                ("shape", Shape)]
+
+
 class PagedAttnError(RuntimeError):
     def __init__(self, status: int, where: str, message: str):
         self.status = status
@@ -77,8 +83,10 @@ lib.pa_get_device_error.argtypes = [_vp, _i32, _P(_i32), _vp]
 lib.pa_kv_append_decode.argtypes = [_vp, _vp, _vp, _vp, _vp, _vp, _vp, _vp, ctypes.c_float, _vp, _P(Shape), _P(Plan),
                                     _vp, _sz, _vp]
 lib.pa_decode_no_alloc.argtypes = [_vp, _vp, _vp, _vp, _vp, ctypes.c_float, _vp, _P(Shape), _P(Plan), _vp]
+lib.pa_prefill_plan.argtypes = [_P(Shape), _i32, _P(PrefillPlan)]
+lib.pa_prefill.argtypes = [_vp, _vp, _vp, _vp, _vp, _vp, ctypes.c_float, _vp, _P(Shape), _P(PrefillPlan), _vp, _vp]
 for _f in ("pa_kv_append", "pa_plan", "pa_workspace_init", "pa_decode", "pa_get_device_error",
-           "pa_kv_append_decode", "pa_decode_no_alloc"):
+           "pa_kv_append_decode", "pa_decode_no_alloc", "pa_prefill_plan", "pa_prefill"):
     getattr(lib, _f).restype = ctypes.c_int
 
 
@@ -163,3 +171,16 @@ def pa_get_device_error(workspace, clear: bool = False, stream=None) -> int:
     _check(lib.pa_get_device_error(_ptr(workspace), int(bool(clear)), ctypes.byref(err), _stream(stream)),
            "pa_get_device_error")
     return err.value
+
+
+def pa_prefill_plan(shape: Shape, max_new_tokens: int) -> PrefillPlan:
+    plan = PrefillPlan()
+    _check(lib.pa_prefill_plan(ctypes.byref(shape), max_new_tokens, ctypes.byref(plan)), "pa_prefill_plan")
+    return plan
+
+
+def pa_prefill(q, k_cache, v_cache, block_tables, context_lens, query_start, scale, out, shape: Shape,
+               plan: PrefillPlan, device_error=None, stream=None):
+    _check(lib.pa_prefill(_ptr(q), _ptr(k_cache), _ptr(v_cache), _ptr(block_tables), _ptr(context_lens),
+                          _ptr(query_start), ctypes.c_float(scale), _ptr(out), ctypes.byref(shape),
+                          ctypes.byref(plan), _ptr(device_error), _stream(stream)), "pa_prefill")

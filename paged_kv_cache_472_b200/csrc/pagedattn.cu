@@ -10,6 +10,7 @@
 
 #include "append.cuh"
 #include "decode.cuh"
+#include "prefill.cuh"
 
 namespace {
 
@@ -522,6 +523,102 @@ pa_status pa_kv_append_decode(const void *k_new, const void *v_new, const int32_
     if (pa_status st = launch_decode(q, k_cache, v_cache, block_tables, context_lens, scale, out, s, plan, workspace,
                                      workspace_bytes, (cudaStream_t)stream, k_new, v_new, slot_mapping))
         return st;
+    return ok();
+}
+
+// ---------------------------------------------------------------------------
+// chunked prefill
+pa_status pa_prefill_plan(const pa_shape *s, int32_t max_new_tokens, pa_prefill_plan_t *plan) {
+    if (!plan) return fail(PA_ERR_INVALID_ARG, "plan_out is NULL");
+    if (pa_status st = check_shape(s)) return st;
+    if (max_new_tokens < 0 || max_new_tokens > s->max_blocks_per_seq * s->block_size)
+        return fail(PA_ERR_INVALID_ARG, "max_new_tokens=%d outside [0, %d]", max_new_tokens,
+                    s->max_blocks_per_seq * s->block_size);
+    if (!tensor_core_dtype(s->dtype)) return fail(PA_ERR_UNSUPPORTED, "prefill supports bf16 and fp16");
+    if (s->D != 64 && s->D != 128) return fail(PA_ERR_UNSUPPORTED, "D=%d (supported: 64, 128)", s->D);
+    if (!pow2(s->block_size) || s->block_size < 16 || s->block_size > 256)
+        return fail(PA_ERR_UNSUPPORTED, "block_size=%d (supported: powers of two in [16, 256])", s->block_size);
+    const int G = s->Hq / s->Hkv;
+    if (!pow2(G) || G > pa::kPrefillRows)
+        return fail(PA_ERR_UNSUPPORTED, "GQA group %d (supported: powers of two <= %d)", G, pa::kPrefillRows);
+    if (s->Hkv > 65535 || s->B > 65535) return fail(PA_ERR_UNSUPPORTED, "Hkv or B above 65535");
+    const int QT = pa::kPrefillRows / G;
+    const int KT = 64;
+    const uint32_t q_bytes = (uint32_t)pa::kPrefillRows * s->D * 2;
+    const uint32_t half = (uint32_t)KT * s->D * 2;
+    int stages = 4;
+    uint32_t total = 0;
+    for (; stages >= 2; --stages) {
+        total = (uint32_t)round_up(q_bytes, 1024) + (uint32_t)stages * 2 * half + 1024;
+        if (total + 1024 <= (uint32_t)kSmemLimit) break;
+    }
+    memset(plan, 0, sizeof *plan);
+    plan->q_tile = QT;
+    plan->kv_tile = KT;
+    plan->stages = stages;
+    plan->max_new_tokens = max_new_tokens;
+    plan->num_qtiles = (max_new_tokens + QT - 1) / QT;
+    plan->smem_bytes = (int32_t)total;
+    plan->shape = *s;
+    return ok();
+}
+
+pa_status pa_prefill(const void *q, const void *k_cache, const void *v_cache, const int32_t *block_tables,
+                     const int32_t *context_lens, const int32_t *query_start, float scale, void *out,
+                     const pa_shape *s, const pa_prefill_plan_t *plan, int32_t *device_error, void *stream) {
+    if (pa_status st = check_shape(s)) return st;
+    if (!plan) return fail(PA_ERR_INVALID_ARG, "plan is NULL");
+    if (memcmp(&plan->shape, s, sizeof *s) != 0) return fail(PA_ERR_INVALID_ARG, "plan was made for another shape");
+    if (!std::isfinite(scale)) return fail(PA_ERR_INVALID_ARG, "scale is not finite");
+    if (s->B == 0 || plan->num_qtiles == 0) return ok();
+    if (!q || !k_cache || !v_cache || !block_tables || !context_lens || !query_start || !out)
+        return fail(PA_ERR_INVALID_ARG, "NULL tensor pointer");
+    if (!aligned16(q) || !aligned16(k_cache) || !aligned16(v_cache) || !aligned16(out))
+        return fail(PA_ERR_INVALID_ARG, "value tensors must be 16-byte aligned");
+    const int G = s->Hq / s->Hkv;
+    if (plan->q_tile * G != pa::kPrefillRows || plan->kv_tile != 64 || plan->stages < 2 || plan->stages > 8)
+        return fail(PA_ERR_INVALID_ARG, "plan is inconsistent");
+    pa::PrefillParams p{};
+    p.q = q;
+    p.out = out;
+    p.block_tables = block_tables;
+    p.context_lens = context_lens;
+    p.query_start = query_start;
+    p.error = device_error;
+    p.qscale = scale * 1.4426950408889634f;
+    p.B = s->B;
+    p.Hq = s->Hq;
+    p.Hkv = s->Hkv;
+    p.G = G;
+    p.bs = s->block_size;
+    p.bs_log2 = log2i(s->block_size);
+    p.num_blocks = s->num_blocks;
+    p.max_blocks = s->max_blocks_per_seq;
+    p.QT = plan->q_tile;
+    p.KT = plan->kv_tile;
+    p.kt_log2 = log2i(plan->kv_tile);
+    const int br = plan->kv_tile < s->block_size ? plan->kv_tile : s->block_size;
+    p.br_log2 = log2i(br);
+    p.stages = plan->stages;
+    p.num_qtiles = plan->num_qtiles;
+    p.off_q = 0;
+    p.off_stage = (uint32_t)round_up((size_t)pa::kPrefillRows * s->D * 2, 1024);
+    p.half_bytes = (uint32_t)plan->kv_tile * s->D * 2;
+    if (pa_status st = encode_pool_map(&p.tmap_k, k_cache, s, br, 1)) return st;
+    if (pa_status st = encode_pool_map(&p.tmap_v, v_cache, s, br, 1)) return st;
+    using PrefillFn = void (*)(const pa::PrefillParams);
+    PrefillFn fn = nullptr;
+    if (s->dtype == PA_DTYPE_BF16) fn = s->D == 64 ? pa::paged_prefill_kernel<__nv_bfloat16, 64>
+                                                   : pa::paged_prefill_kernel<__nv_bfloat16, 128>;
+    else fn = s->D == 64 ? pa::paged_prefill_kernel<__half, 64> : pa::paged_prefill_kernel<__half, 128>;
+    {
+        cudaError_t e = cudaFuncSetAttribute(fn, cudaFuncAttributeMaxDynamicSharedMemorySize, plan->smem_bytes);
+        if (e != cudaSuccess) return fail(PA_ERR_CUDA, "cudaFuncSetAttribute: %s", cudaGetErrorString(e));
+    }
+    dim3 grid((unsigned)plan->num_qtiles, (unsigned)s->Hkv, (unsigned)s->B);
+    fn<<<grid, pa::kPrefillThreads, (size_t)plan->smem_bytes, (cudaStream_t)stream>>>(p);
+    cudaError_t e = cudaGetLastError();
+    if (e != cudaSuccess) return fail(PA_ERR_CUDA, "prefill launch: %s", cudaGetErrorString(e));
     return ok();
 }
 

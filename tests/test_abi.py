@@ -177,3 +177,20 @@ def test_decode_rejects_bad_dynamic_share(share, mode_fixed):
     with pytest.raises(pa.PagedAttnError) as ei:
         pa.pa_decode(0, 0, 0, 0, 0, 0.1, 0, s, plan, 0, 0, stream=0)
     assert ei.value.status == pa.PA_ERR_INVALID_ARG
+
+
+def test_prefill_plan_shapes_and_rejections():
+    s = pa.Shape(8, 32, 8, 128, 16, 4096, 256, pa.DTYPE_BF16)
+    plan = pa.pa_prefill_plan(s, 512)
+    assert plan.q_tile * 4 == 128 and plan.num_qtiles == 512 // plan.q_tile and plan.stages >= 2
+    assert plan.smem_bytes <= 232448
+    for bad, status in ((pa.Shape(2, 8, 2, 128, 16, 64, 8, pa.DTYPE_F32), pa.PA_ERR_UNSUPPORTED),
+                        (pa.Shape(2, 8, 2, 96, 16, 64, 8, pa.DTYPE_BF16), pa.PA_ERR_UNSUPPORTED),
+                        (pa.Shape(2, 8, 2, 128, 8, 64, 8, pa.DTYPE_BF16), pa.PA_ERR_UNSUPPORTED),
+                        (pa.Shape(2, 6, 2, 128, 16, 64, 8, pa.DTYPE_BF16), pa.PA_ERR_UNSUPPORTED)):
+        with pytest.raises(pa.PagedAttnError) as ei:
+            pa.pa_prefill_plan(bad, 16)
+        assert ei.value.status == status
+    with pytest.raises(pa.PagedAttnError) as ei:
+        pa.pa_prefill_plan(s, 256 * 16 + 1)            # more new tokens than a table row holds
+    assert ei.value.status == pa.PA_ERR_INVALID_ARG

@@ -77,3 +77,10 @@ def test_fp16_values_widen_exactly(orc):
     out = orc.decode(case)
     want = vals.view(np.float16).astype(np.float64).reshape(rows, 1, D)
     assert np.array_equal(out, want)
+
+
+def test_prefill_rows_match_full_prefill(orc):
+    pc = synth.make_prefill_config(2, batch=3, chunk=40)
+    full = orc.prefill(pc)
+    rows = [0, 5, pc.T - 1, int(pc.query_start[1])]
+    assert np.array_equal(orc.prefill_rows(pc, rows), full[rows])
