@@ -48,6 +48,8 @@ def parse():
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--cpu-seconds", type=float, default=10.0)
     ap.add_argument("--e2e-steps", type=int, default=200)
+    ap.add_argument("--prefill", type=int, default=0,
+                    help="time the chunked prefill step of prefill workload N (1, 2) instead of the decode step")
     ap.add_argument("--dynamic-share", type=int, default=-1,
                     help="balanced split: share of each request's tiles handed out at run time, in 1/256 "
                          "(-1: the planner's choice)")
@@ -69,6 +71,18 @@ def measured_peak():
             return float(json.load(f)["hbm_gbs"]), "measured"
     except Exception:
         return FALLBACK_HBM_GBS, "fallback"
+
+
+FALLBACK_BF16_TFLOPS = 1590.0
+
+
+def measured_tensor_peak():
+    """Dense bf16 TFLOP/s (cuBLAS, burst: the kernel is timed on its own)."""
+    try:
+        with open(os.path.join(ROOT, "MEASURED_PEAKS.json")) as f:
+            return float(json.load(f)["bf16_tflops"]), "measured"
+    except Exception:
+        return FALLBACK_BF16_TFLOPS, "fallback"
 
 
 def profiled_traffic(workload: str):
@@ -199,10 +213,112 @@ def run_reference(args):
 
 
 # ---------------------------------------------------------------------------
+def run_prefill(args):
+    """The chunked prefill step of a prefill workload: pa_kv_append of every
+    new token, then pa_prefill.  value = algorithmic causal FLOPs per second."""
+    import torch
+    import synth
+    import importlib.util
+    spec = importlib.util.spec_from_file_location(
+        "_pagedattn_build", os.path.join(ROOT, "paged_kv_cache_472_b200", "build.py"))
+    libbuild = importlib.util.module_from_spec(spec)
+    spec.loader.exec_module(libbuild)
+    libbuild.build()
+    import ctypes
+    import paged_kv_cache_472_b200 as pa
+    from tests import gpu_harness as H
+
+    torch.cuda.set_device(0)
+    pc = synth.make_prefill_config(args.prefill)
+    alg = synth.prefill_algorithmic(pc)
+    dt = {"bf16": pa.DTYPE_BF16, "f16": pa.DTYPE_F16}[pc.dtype]
+    shape = pa.Shape(pc.B, pc.Hq, pc.Hkv, pc.D, pc.block_size, pc.num_blocks, pc.max_blocks_per_seq, dt)
+    ashape = pa.Shape(pc.T, pc.Hq, pc.Hkv, pc.D, pc.block_size, pc.num_blocks, pc.max_blocks_per_seq, dt)
+    plan = pa.pa_prefill_plan(shape, int(pc.new_tokens().max()))
+    R = 3
+    v = lambda a: H._vals(a, pc.dtype, "cuda")
+    i32 = lambda a: torch.from_numpy(np.ascontiguousarray(a, dtype=np.int32)).cuda()
+    copies = []
+    for _ in range(R):
+        q = v(pc.q)
+        copies.append(dict(q=q, kn=v(pc.k_new), vn=v(pc.v_new), kc=v(pc.k_cache), vc=v(pc.v_cache),
+                           bt=i32(pc.block_tables), cl=i32(pc.context_lens), qs=i32(pc.query_start),
+                           sm=i32(pc.slot_mapping), out=torch.empty_like(q)))
+    err = torch.zeros(1, dtype=torch.int32, device="cuda")
+    lib, byref = pa.lib, ctypes.byref
+    stream = torch.cuda.current_stream()
+    sp = stream.cuda_stream
+
+    def step(i, append=True):
+        c = copies[i % R]
+        if append:
+            lib.pa_kv_append(c["kn"].data_ptr(), c["vn"].data_ptr(), c["sm"].data_ptr(), c["kc"].data_ptr(),
+                             c["vc"].data_ptr(), byref(ashape), err.data_ptr(), sp)
+        return lib.pa_prefill(c["q"].data_ptr(), c["kc"].data_ptr(), c["vc"].data_ptr(), c["bt"].data_ptr(),
+                              c["cl"].data_ptr(), c["qs"].data_ptr(), ctypes.c_float(pc.scale), c["out"].data_ptr(),
+                              byref(shape), byref(plan), err.data_ptr(), sp)
+
+    for i in range(max(args.warmup, 3)):
+        if step(i):
+            raise RuntimeError(pa.pa_last_error_message())
+    torch.cuda.synchronize()
+    K = args.steps
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    with ClockSampler(0) as clk:
+        torch.cuda._sleep(20_000_000)
+        e0.record(stream)
+        for i in range(K):
+            step(i)
+        e1.record(stream)
+        torch.cuda.synchronize()
+    ms_step = e0.elapsed_time(e1) / K
+    # the prefill kernel alone, back to back
+    torch.cuda._sleep(20_000_000)
+    e0.record(stream)
+    for i in range(K):
+        step(i, append=False)
+    e1.record(stream)
+    torch.cuda.synchronize()
+    ms_kernel = e0.elapsed_time(e1) / K
+    if int(err.item()):
+        raise RuntimeError(f"device error word {int(err.item()):#x}")
+    peak, kind = measured_tensor_peak()
+    tflops = alg["flops"] / (ms_step * 1e-3) / 1e12
+    k_tflops = alg["flops"] / (ms_kernel * 1e-3) / 1e12
+    line = {"metric": "paged chunked-prefill attention TFLOP/s (causal, algorithmic)", "value": round(tflops, 2),
+            "unit": "TFLOP/s", "n_gpus": 1, "steps": K, "warmup": args.warmup, "ms_per_step": round(ms_step, 6),
+            "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": pc.dtype, "data": "synthetic",
+            "config": {"workload": pc.name, "B": pc.B, "new_tokens": pc.T, "Hq": pc.Hq, "Hkv": pc.Hkv, "D": pc.D,
+                       "block_size": pc.block_size, "context_tokens": int(pc.context_lens.sum()),
+                       "flops_per_step": alg["flops"], "min_bytes_per_step": alg["bytes"],
+                       "l2": f"{R} rotating input copies"},
+            "roofline": {"bound": "tensor", "achieved": round(k_tflops, 2), "peak": peak, "unit": "TFLOP/s",
+                         "frac": round(k_tflops / peak, 4), "traffic": None, "kernel": "paged_prefill_kernel",
+                         "peak_kind": kind, "kernel_us": round(ms_kernel * 1e3, 3),
+                         "engine": "mma.sync m16n8k16, P split into two 16-bit parts"},
+            "gpu_launches": 2 * K, "clocks": clk.summary()}
+    if not args.no_cpu_baseline:
+        import oracle
+        orc = oracle.default()
+        rng = np.random.default_rng(0)
+        rows = np.sort(rng.choice(pc.T, size=min(pc.T, 64), replace=False))
+        kc, vc = orc.prefill_append(pc)
+        t0 = time.perf_counter()
+        orc.prefill_rows(pc, rows, kc, vc)
+        el = time.perf_counter() - t0
+        pos = pc.positions()
+        flops = 4 * int((pos[rows] + 1).sum()) * pc.Hq * pc.D
+        line["cpu_baseline"] = {"value": flops / el / 1e12, "unit": "TFLOP/s", "cores": orc.max_threads(),
+                                "kind": "oracle", "sample": f"{len(rows)} of {pc.T} new tokens, all heads, {el:.1f} s"}
+    print(json.dumps(line), flush=True)
+
+
 def main():
     args = parse()
     if args.impl == "reference":
         return run_reference(args)
+    if args.prefill:
+        return run_prefill(args)
 
     import torch
     import torch.distributed as dist

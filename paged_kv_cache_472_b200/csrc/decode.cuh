@@ -819,9 +819,9 @@ struct MmaEngine {
             mx1 = fmaxf(mx1, __shfl_xor_sync(0xffffffffu, mx1, m));
         }
         const float mn0 = fmaxf(u.m[0], mx0), mn1 = fmaxf(u.m[1], mx1);
-        const float al0 = exp2f(u.m[0] - mn0), al1 = exp2f(u.m[1] - mn1);
-        const float p0 = exp2f(s0 - mn0), p1 = exp2f(s1 - mn1);  // token g4
-        const float p2 = exp2f(s2 - mn0), p3 = exp2f(s3 - mn1);  // token g4 + 8
+        const float al0 = exp2_fast(u.m[0] - mn0), al1 = exp2_fast(u.m[1] - mn1);
+        const float p0 = exp2_fast(s0 - mn0), p1 = exp2_fast(s1 - mn1);  // token g4
+        const float p2 = exp2_fast(s2 - mn0), p3 = exp2_fast(s3 - mn1);  // token g4 + 8
         float r0 = p0 + p2, r1 = p1 + p3;
 #pragma unroll
         for (int m = 4; m < 32; m <<= 1) {

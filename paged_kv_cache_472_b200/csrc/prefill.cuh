@@ -29,6 +29,8 @@
 //                    the decode; V as the B operand by transposing ldmatrix).
 #pragma once
 
+#include <type_traits>
+
 #include "common.cuh"
 
 namespace pa {
@@ -249,50 +251,64 @@ __global__ void __launch_bounds__(kPrefillThreads, 1) paged_prefill_kernel(const
                 fence_async_smem();  // ordered before the next tensor-map fill of this stage
                 __syncwarp();
             }
-            for (int kg = 0; kg < nk16; ++kg) {
-                // ---- S[16 rows x 16 keys] = Q K^T, two n-tiles of 8 keys ----
-                float s0[4] = {0.f, 0.f, 0.f, 0.f}, s1[4] = {0.f, 0.f, 0.f, 0.f};
-                const int key = kg * 16 + kb_key;
+            // One online-softmax step over NG groups of 16 keys (groups kg0 ..
+            // kg0 + NG - 1, all loaded): S, mask, one max / rescale / sum, P V.
+            auto step = [&](auto ng, int kg0) {
+                constexpr int NG = decltype(ng)::value;
+                // ---- S[16 rows x 16 NG keys] = Q K^T, one accumulation chain per 8 keys ----
+                float sc[2 * NG][4];
+#pragma unroll
+                for (int nt = 0; nt < 2 * NG; ++nt) sc[nt][0] = sc[nt][1] = sc[nt][2] = sc[nt][3] = 0.f;
 #pragma unroll
                 for (int ks = 0; ks < KS; ++ks) {
-                    uint32_t bf[4];
-                    ldmatrix_x4(bf, kv_chunk<D>(kst, key, ks * 2 + kb_col, p.br_log2));
-                    Op::mma(s0, qa[ks], bf[0], bf[1]);
-                    Op::mma(s1, qa[ks], bf[2], bf[3]);
-                }
-                // ---- causal mask; scores in the base-2 domain ----
-                const int kc = k0 + kg * 16 + 2 * t4;  // key of s0[0]; s0[1] is kc+1, s1[*] kc+8, kc+9
-                float x[8] = {s0[0], s0[1], s1[0], s1[1], s0[2], s0[3], s1[2], s1[3]};
-                const int kk[4] = {kc, kc + 1, kc + 8, kc + 9};
 #pragma unroll
-                for (int i = 0; i < 4; ++i) {
-                    x[i] = kk[i] <= qpos_lo ? x[i] * p.qscale : -INFINITY;
-                    x[4 + i] = kk[i] <= qpos_hi ? x[4 + i] * p.qscale : -INFINITY;
+                    for (int gi = 0; gi < NG; ++gi) {
+                        uint32_t bf[4];
+                        ldmatrix_x4(bf, kv_chunk<D>(kst, (kg0 + gi) * 16 + kb_key, ks * 2 + kb_col, p.br_log2));
+                        Op::mma(sc[2 * gi], qa[ks], bf[0], bf[1]);
+                        Op::mma(sc[2 * gi + 1], qa[ks], bf[2], bf[3]);
+                    }
                 }
-                float mx_lo = fmaxf(fmaxf(x[0], x[1]), fmaxf(x[2], x[3]));
-                float mx_hi = fmaxf(fmaxf(x[4], x[5]), fmaxf(x[6], x[7]));
+                // ---- causal mask, scores in the base-2 domain ----
+                // sc[nt][0..1]: row lo, keys kc, kc+1 with kc = k0 + kg0*16 + nt*8 + 2*t4; [2..3]: row hi
+                float mx_lo = -INFINITY, mx_hi = -INFINITY;
+#pragma unroll
+                for (int nt = 0; nt < 2 * NG; ++nt) {
+                    const int kc = k0 + kg0 * 16 + nt * 8 + 2 * t4;
+#pragma unroll
+                    for (int i = 0; i < 2; ++i) {
+                        sc[nt][i] = kc + i <= qpos_lo ? sc[nt][i] * p.qscale : -INFINITY;
+                        sc[nt][2 + i] = kc + i <= qpos_hi ? sc[nt][2 + i] * p.qscale : -INFINITY;
+                        mx_lo = fmaxf(mx_lo, sc[nt][i]);
+                        mx_hi = fmaxf(mx_hi, sc[nt][2 + i]);
+                    }
+                }
                 mx_lo = fmaxf(mx_lo, __shfl_xor_sync(0xffffffffu, mx_lo, 1));
                 mx_lo = fmaxf(mx_lo, __shfl_xor_sync(0xffffffffu, mx_lo, 2));
                 mx_hi = fmaxf(mx_hi, __shfl_xor_sync(0xffffffffu, mx_hi, 1));
                 mx_hi = fmaxf(mx_hi, __shfl_xor_sync(0xffffffffu, mx_hi, 2));
                 const float mn_lo = fmaxf(m_lo, mx_lo), mn_hi = fmaxf(m_hi, mx_hi);
                 // a row with no visible key yet keeps m = -inf: its weights are 0
-                const float al_lo = mn_lo == -INFINITY ? 1.f : exp2f(m_lo - mn_lo);
-                const float al_hi = mn_hi == -INFINITY ? 1.f : exp2f(m_hi - mn_hi);
-                float pw[8];
+                const float al_lo = mn_lo == -INFINITY ? 1.f : exp2_fast(m_lo - mn_lo);
+                const float al_hi = mn_hi == -INFINITY ? 1.f : exp2_fast(m_hi - mn_hi);
+                const float sub_lo = mn_lo == -INFINITY ? 0.f : mn_lo, sub_hi = mn_hi == -INFINITY ? 0.f : mn_hi;
+                float sum_lo = 0.f, sum_hi = 0.f;
 #pragma unroll
-                for (int i = 0; i < 4; ++i) {
-                    pw[i] = mn_lo == -INFINITY ? 0.f : exp2f(x[i] - mn_lo);
-                    pw[4 + i] = mn_hi == -INFINITY ? 0.f : exp2f(x[4 + i] - mn_hi);
+                for (int nt = 0; nt < 2 * NG; ++nt) {
+#pragma unroll
+                    for (int i = 0; i < 2; ++i) {
+                        sc[nt][i] = exp2_fast(sc[nt][i] - sub_lo);  // masked: 2^-inf = 0
+                        sc[nt][2 + i] = exp2_fast(sc[nt][2 + i] - sub_hi);
+                        sum_lo += sc[nt][i];
+                        sum_hi += sc[nt][2 + i];
+                    }
                 }
-                float r_lo_sum = (pw[0] + pw[1]) + (pw[2] + pw[3]);
-                float r_hi_sum = (pw[4] + pw[5]) + (pw[6] + pw[7]);
-                r_lo_sum += __shfl_xor_sync(0xffffffffu, r_lo_sum, 1);
-                r_lo_sum += __shfl_xor_sync(0xffffffffu, r_lo_sum, 2);
-                r_hi_sum += __shfl_xor_sync(0xffffffffu, r_hi_sum, 1);
-                r_hi_sum += __shfl_xor_sync(0xffffffffu, r_hi_sum, 2);
-                l_lo = l_lo * al_lo + r_lo_sum;
-                l_hi = l_hi * al_hi + r_hi_sum;
+                sum_lo += __shfl_xor_sync(0xffffffffu, sum_lo, 1);
+                sum_lo += __shfl_xor_sync(0xffffffffu, sum_lo, 2);
+                sum_hi += __shfl_xor_sync(0xffffffffu, sum_hi, 1);
+                sum_hi += __shfl_xor_sync(0xffffffffu, sum_hi, 2);
+                l_lo = l_lo * al_lo + sum_lo;
+                l_hi = l_hi * al_hi + sum_hi;
                 m_lo = mn_lo;
                 m_hi = mn_hi;
                 if (al_lo != 1.f || al_hi != 1.f) {
@@ -304,32 +320,39 @@ __global__ void __launch_bounds__(kPrefillThreads, 1) paged_prefill_kernel(const
                         o[j][3] *= al_hi;
                     }
                 }
-                // ---- P as the A operand (m16 x k16 keys), high and low parts ----
-                uint32_t ph[4], pl[4];
-                ph[0] = Op::pack_p(pw[0], pw[1]);  // row lo, keys kc, kc+1
-                ph[1] = Op::pack_p(pw[4], pw[5]);  // row hi
-                ph[2] = Op::pack_p(pw[2], pw[3]);  // row lo, keys kc+8, kc+9
-                ph[3] = Op::pack_p(pw[6], pw[7]);  // row hi
-                {
-                    const float2 h0 = Op::unpack(ph[0]), h1 = Op::unpack(ph[1]);
-                    const float2 h2 = Op::unpack(ph[2]), h3 = Op::unpack(ph[3]);
-                    pl[0] = Op::pack_p(pw[0] - h0.x, pw[1] - h0.y);
-                    pl[1] = Op::pack_p(pw[4] - h1.x, pw[5] - h1.y);
-                    pl[2] = Op::pack_p(pw[2] - h2.x, pw[3] - h2.y);
-                    pl[3] = Op::pack_p(pw[6] - h3.x, pw[7] - h3.y);
-                }
-                // ---- O[16 rows x D] += P V: V rows kg*16.. as the B operand (k = key, n = d) ----
-                const int vkey = kg * 16 + vb_key;
+                // ---- O[16 rows x D] += P V, one 16-key group at a time ----
 #pragma unroll
-                for (int j2 = 0; j2 < NO / 2; ++j2) {
-                    uint32_t vf[4];
-                    ldmatrix_x4_trans(vf, kv_chunk<D>(vst, vkey, j2 * 2 + vb_col, p.br_log2));
-                    Op::mma(o[2 * j2], ph, vf[0], vf[1]);
-                    Op::mma(o[2 * j2], pl, vf[0], vf[1]);
-                    Op::mma(o[2 * j2 + 1], ph, vf[2], vf[3]);
-                    Op::mma(o[2 * j2 + 1], pl, vf[2], vf[3]);
+                for (int gi = 0; gi < NG; ++gi) {
+                    // P as the A operand (m16 x k16), high and low 16-bit parts
+                    const float *c0 = sc[2 * gi], *c1 = sc[2 * gi + 1];
+                    uint32_t ph[4], pl[4];
+                    ph[0] = Op::pack_p(c0[0], c0[1]);  // row lo, keys +2*t4
+                    ph[1] = Op::pack_p(c0[2], c0[3]);  // row hi
+                    ph[2] = Op::pack_p(c1[0], c1[1]);  // row lo, keys +8+2*t4
+                    ph[3] = Op::pack_p(c1[2], c1[3]);  // row hi
+                    {
+                        const float2 h0 = Op::unpack(ph[0]), h1 = Op::unpack(ph[1]);
+                        const float2 h2 = Op::unpack(ph[2]), h3 = Op::unpack(ph[3]);
+                        pl[0] = Op::pack_p(c0[0] - h0.x, c0[1] - h0.y);
+                        pl[1] = Op::pack_p(c0[2] - h1.x, c0[3] - h1.y);
+                        pl[2] = Op::pack_p(c1[0] - h2.x, c1[1] - h2.y);
+                        pl[3] = Op::pack_p(c1[2] - h3.x, c1[3] - h3.y);
+                    }
+                    const int vkey = (kg0 + gi) * 16 + vb_key;
+#pragma unroll
+                    for (int j2 = 0; j2 < NO / 2; ++j2) {
+                        uint32_t vf[4];
+                        ldmatrix_x4_trans(vf, kv_chunk<D>(vst, vkey, j2 * 2 + vb_col, p.br_log2));
+                        Op::mma(o[2 * j2], ph, vf[0], vf[1]);
+                        Op::mma(o[2 * j2 + 1], ph, vf[2], vf[3]);
+                        Op::mma(o[2 * j2], pl, vf[0], vf[1]);
+                        Op::mma(o[2 * j2 + 1], pl, vf[2], vf[3]);
+                    }
                 }
-            }
+            };
+            int kg = 0;
+            for (; kg + 1 < nk16; kg += 2) step(std::integral_constant<int, 2>{}, kg);
+            if (kg < nk16) step(std::integral_constant<int, 1>{}, kg);
         }
         __syncwarp();
         if (lane == 0) mbar_arrive(&empty[stage]);
