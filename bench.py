@@ -295,7 +295,7 @@ def run_prefill(args):
             "roofline": {"bound": "tensor", "achieved": round(k_tflops, 2), "peak": peak, "unit": "TFLOP/s",
                          "frac": round(k_tflops / peak, 4), "traffic": None, "kernel": "paged_prefill_kernel",
                          "peak_kind": kind, "kernel_us": round(ms_kernel * 1e3, 3),
-                         "engine": "mma.sync m16n8k16, P split into two 16-bit parts"},
+                         "engine": "tcgen05.mma, S and O in tensor memory, P split into two 16-bit parts"},
             "gpu_launches": 2 * K, "clocks": clk.summary()}
     if not args.no_cpu_baseline:
         import oracle

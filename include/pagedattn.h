@@ -59,6 +59,7 @@ typedef enum { PA_DTYPE_F32 = 0, PA_DTYPE_BF16 = 1, PA_DTYPE_F16 = 2 } pa_dtype;
 #define PA_DEVERR_TIMEOUT     0x4  /* a pipeline wait gave up (internal error) */
 #define PA_DEVERR_WORKSPACE   0x8  /* more partitions than the plan provided for */
 #define PA_DEVERR_SLOT        0x10 /* an append slot >= num_blocks*block_size */
+#define PA_DEVERR_SMEM        0x20 /* dynamic shared memory not 1024-byte aligned (internal error) */
 
 /* Problem shape.  B requests, Hq query heads, Hkv KV heads (Hq % Hkv == 0;
  * query head h reads KV head h / (Hq/Hkv)), head dim D, block_size tokens per

@@ -14,7 +14,7 @@ import os
 from .build import LIB as _LIB_PATH
 
 __all__ = ["PagedAttnError", "Shape", "Plan", "DTYPE_F32", "DTYPE_BF16", "DTYPE_F16", "SPLIT_BALANCED", "SPLIT_FIXED",
-           "DEVERR_BLOCK_ID", "DEVERR_CONTEXT_LEN", "DEVERR_TIMEOUT", "DEVERR_WORKSPACE", "DEVERR_SLOT",
+           "DEVERR_BLOCK_ID", "DEVERR_CONTEXT_LEN", "DEVERR_TIMEOUT", "DEVERR_WORKSPACE", "DEVERR_SLOT", "DEVERR_SMEM",
            "PLAN_NO_SPECULATION", "PLAN_TEST_MISGUESS",
            "pa_version", "pa_status_str", "pa_last_error_message", "pa_kv_append", "pa_plan",
            "pa_decode_workspace_size", "pa_workspace_init", "pa_decode", "pa_kv_append_decode", "pa_get_device_error",
@@ -23,7 +23,8 @@ __all__ = ["PagedAttnError", "Shape", "Plan", "DTYPE_F32", "DTYPE_BF16", "DTYPE_
 PA_OK, PA_ERR_INVALID_ARG, PA_ERR_UNSUPPORTED, PA_ERR_CUDA, PA_ERR_WORKSPACE = range(5)
 DTYPE_F32, DTYPE_BF16, DTYPE_F16 = 0, 1, 2
 SPLIT_BALANCED, SPLIT_FIXED = 0, 1
-DEVERR_BLOCK_ID, DEVERR_CONTEXT_LEN, DEVERR_TIMEOUT, DEVERR_WORKSPACE, DEVERR_SLOT = 0x1, 0x2, 0x4, 0x8, 0x10
+DEVERR_BLOCK_ID, DEVERR_CONTEXT_LEN, DEVERR_TIMEOUT, DEVERR_WORKSPACE, DEVERR_SLOT, DEVERR_SMEM = (
+    0x1, 0x2, 0x4, 0x8, 0x10, 0x20)
 PLAN_NO_SPECULATION, PLAN_TEST_MISGUESS = 0x1, 0x2
 
 

@@ -313,6 +313,18 @@ struct Mma16<__nv_bfloat16> {
         return __byte_perm(a + 0x7FFFu + ((a >> 16) & 1u), b + 0x7FFFu + ((b >> 16) & 1u), 0x7632);
     }
     static __device__ __forceinline__ float2 unpack(uint32_t w) { return bf16x2_to_float2(w); }
+    // Two weights (finite, >= 0, below 2^24) as a high and a low bf16 part
+    // on the FMA pipe.  Veltkamp's splitting (Dekker, "A floating-point
+    // technique for extending the available precision", 1971): with
+    // c = (2^16 + 1) x, hi = c - (c - x) keeps the leading 8 significant bits
+    // of x (so hi is a bf16 value: its low 16 bits are zero) and x - hi is
+    // exact; the low part is then truncated to bf16, an error below 2^-15 x.
+    static __device__ __forceinline__ void split_p(float a, float b, uint32_t &hi, uint32_t &lo) {
+        const float ca = __fmul_rn(a, 65537.f), cb = __fmul_rn(b, 65537.f);
+        const float ha = __fsub_rn(ca, __fsub_rn(ca, a)), hb = __fsub_rn(cb, __fsub_rn(cb, b));
+        hi = __byte_perm(__float_as_uint(ha), __float_as_uint(hb), 0x7632);
+        lo = __byte_perm(__float_as_uint(__fsub_rn(a, ha)), __float_as_uint(__fsub_rn(b, hb)), 0x7632);
+    }
 };
 
 template <>
@@ -323,6 +335,12 @@ struct Mma16<__half> {
     static __device__ __forceinline__ uint32_t pack(float lo, float hi) { return pack_f16x2(lo, hi); }
     static __device__ __forceinline__ uint32_t pack_p(float lo, float hi) { return pack_f16x2(lo, hi); }
     static __device__ __forceinline__ float2 unpack(uint32_t w) { return f16x2_to_float2(w); }
+    // Two weights as a high and a low fp16 part, each rounded to nearest.
+    static __device__ __forceinline__ void split_p(float a, float b, uint32_t &hi, uint32_t &lo) {
+        hi = pack_f16x2(a, b);
+        const float2 h = f16x2_to_float2(hi);
+        lo = pack_f16x2(a - h.x, b - h.y);
+    }
 };
 
 }  // namespace pa
@@ -390,6 +408,40 @@ __device__ __forceinline__ void tmem_st16(uint32_t taddr, const float (&v)[16]) 
         "r"(__float_as_uint(v[9])), "r"(__float_as_uint(v[10])), "r"(__float_as_uint(v[11])),
         "r"(__float_as_uint(v[12])), "r"(__float_as_uint(v[13])), "r"(__float_as_uint(v[14])),
         "r"(__float_as_uint(v[15]))
+        : "memory");
+}
+
+// 32 consecutive 32-bit TMEM columns of this thread's lane.
+__device__ __forceinline__ void tmem_ld32(uint32_t taddr, float *v) {
+    uint32_t r[32];
+    asm volatile(
+        "tcgen05.ld.sync.aligned.32x32b.x32.b32 {%0,%1,%2,%3,%4,%5,%6,%7,%8,%9,%10,%11,%12,%13,%14,%15,"
+        "%16,%17,%18,%19,%20,%21,%22,%23,%24,%25,%26,%27,%28,%29,%30,%31}, [%32];"
+        : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3]), "=r"(r[4]), "=r"(r[5]), "=r"(r[6]), "=r"(r[7]),
+          "=r"(r[8]), "=r"(r[9]), "=r"(r[10]), "=r"(r[11]), "=r"(r[12]), "=r"(r[13]), "=r"(r[14]), "=r"(r[15]),
+          "=r"(r[16]), "=r"(r[17]), "=r"(r[18]), "=r"(r[19]), "=r"(r[20]), "=r"(r[21]), "=r"(r[22]), "=r"(r[23]),
+          "=r"(r[24]), "=r"(r[25]), "=r"(r[26]), "=r"(r[27]), "=r"(r[28]), "=r"(r[29]), "=r"(r[30]), "=r"(r[31])
+        : "r"(taddr)
+        : "memory");
+#pragma unroll
+    for (int i = 0; i < 32; ++i) v[i] = __uint_as_float(r[i]);
+}
+
+__device__ __forceinline__ void tmem_st32(uint32_t taddr, const float *v) {
+    asm volatile(
+        "tcgen05.st.sync.aligned.32x32b.x32.b32 [%0], {%1,%2,%3,%4,%5,%6,%7,%8,%9,%10,%11,%12,%13,%14,%15,%16,"
+        "%17,%18,%19,%20,%21,%22,%23,%24,%25,%26,%27,%28,%29,%30,%31,%32};" ::"r"(taddr),
+        "r"(__float_as_uint(v[0])), "r"(__float_as_uint(v[1])), "r"(__float_as_uint(v[2])),
+        "r"(__float_as_uint(v[3])), "r"(__float_as_uint(v[4])), "r"(__float_as_uint(v[5])),
+        "r"(__float_as_uint(v[6])), "r"(__float_as_uint(v[7])), "r"(__float_as_uint(v[8])),
+        "r"(__float_as_uint(v[9])), "r"(__float_as_uint(v[10])), "r"(__float_as_uint(v[11])),
+        "r"(__float_as_uint(v[12])), "r"(__float_as_uint(v[13])), "r"(__float_as_uint(v[14])),
+        "r"(__float_as_uint(v[15])), "r"(__float_as_uint(v[16])), "r"(__float_as_uint(v[17])),
+        "r"(__float_as_uint(v[18])), "r"(__float_as_uint(v[19])), "r"(__float_as_uint(v[20])),
+        "r"(__float_as_uint(v[21])), "r"(__float_as_uint(v[22])), "r"(__float_as_uint(v[23])),
+        "r"(__float_as_uint(v[24])), "r"(__float_as_uint(v[25])), "r"(__float_as_uint(v[26])),
+        "r"(__float_as_uint(v[27])), "r"(__float_as_uint(v[28])), "r"(__float_as_uint(v[29])),
+        "r"(__float_as_uint(v[30])), "r"(__float_as_uint(v[31]))
         : "memory");
 }
 

@@ -37,6 +37,7 @@ size_t round_up(size_t x, size_t a) { return (x + a - 1) / a * a; }
 
 constexpr int kSmemLimit = 232448;     // opt-in shared memory per CTA on sm_100 (static + dynamic)
 // the decode kernel's static shared memory: control block, lengths and prefix-sum caches
+constexpr int kPrefillStaticSmem = 3072;  // barriers, row exchange, tensor-memory address, abort flag
 constexpr int kStaticSmem = (int)sizeof(pa::DecodeCtl) + 4 * pa::kLensCache + 8 * (pa::kPrefixCache + 1) + 256;
 constexpr size_t kWsHeader = 256;      // error word, dynamic-list counters
 constexpr size_t kWsGrab = 64;         // header offset of the grains-handed-out counter
@@ -543,19 +544,20 @@ pa_status pa_prefill_plan(const pa_shape *s, int32_t max_new_tokens, pa_prefill_
         return fail(PA_ERR_UNSUPPORTED, "GQA group %d (supported: powers of two <= %d)", G, pa::kPrefillRows);
     if (s->Hkv > 65535 || s->B > 65535) return fail(PA_ERR_UNSUPPORTED, "Hkv or B above 65535");
     const int QT = pa::kPrefillRows / G;
-    const int KT = 64;
+    const int KT = pa::kPrefillKT;
     const uint32_t q_bytes = (uint32_t)pa::kPrefillRows * s->D * 2;
-    const uint32_t half = (uint32_t)KT * s->D * 2;
-    int stages = 4;
+    const uint32_t p_bytes = 2u * pa::kPrefillRows * KT * 2;  // P, high and low parts
+    const uint32_t slot = (uint32_t)KT * s->D * 2;
+    int nslots = pa::kPrefillMaxSlots;
     uint32_t total = 0;
-    for (; stages >= 2; --stages) {
-        total = (uint32_t)round_up(q_bytes, 1024) + (uint32_t)stages * 2 * half + 1024;
-        if (total + 1024 <= (uint32_t)kSmemLimit) break;
+    for (; nslots >= 2; nslots -= 2) {
+        total = q_bytes + p_bytes + (uint32_t)nslots * slot;  // the kernel checks its base is 1024-aligned
+        if (total + kPrefillStaticSmem <= (uint32_t)kSmemLimit) break;
     }
     memset(plan, 0, sizeof *plan);
     plan->q_tile = QT;
     plan->kv_tile = KT;
-    plan->stages = stages;
+    plan->stages = nslots / 2;
     plan->max_new_tokens = max_new_tokens;
     plan->num_qtiles = (max_new_tokens + QT - 1) / QT;
     plan->smem_bytes = (int32_t)total;
@@ -576,7 +578,8 @@ pa_status pa_prefill(const void *q, const void *k_cache, const void *v_cache, co
     if (!aligned16(q) || !aligned16(k_cache) || !aligned16(v_cache) || !aligned16(out))
         return fail(PA_ERR_INVALID_ARG, "value tensors must be 16-byte aligned");
     const int G = s->Hq / s->Hkv;
-    if (plan->q_tile * G != pa::kPrefillRows || plan->kv_tile != 64 || plan->stages < 2 || plan->stages > 8)
+    if (plan->q_tile * G != pa::kPrefillRows || plan->kv_tile != pa::kPrefillKT || plan->stages < 1 ||
+        2 * plan->stages > pa::kPrefillMaxSlots)
         return fail(PA_ERR_INVALID_ARG, "plan is inconsistent");
     pa::PrefillParams p{};
     p.q = q;
@@ -585,25 +588,25 @@ pa_status pa_prefill(const void *q, const void *k_cache, const void *v_cache, co
     p.context_lens = context_lens;
     p.query_start = query_start;
     p.error = device_error;
-    p.qscale = scale * 1.4426950408889634f;
+    p.qscale = std::fabs(scale) * 1.4426950408889634f;
+    p.qflip = scale < 0.f ? 0x80008000u : 0u;
     p.B = s->B;
     p.Hq = s->Hq;
     p.Hkv = s->Hkv;
     p.G = G;
+    p.g_log2 = log2i(G);
     p.bs = s->block_size;
     p.bs_log2 = log2i(s->block_size);
     p.num_blocks = s->num_blocks;
     p.max_blocks = s->max_blocks_per_seq;
     p.QT = plan->q_tile;
-    p.KT = plan->kv_tile;
-    p.kt_log2 = log2i(plan->kv_tile);
     const int br = plan->kv_tile < s->block_size ? plan->kv_tile : s->block_size;
     p.br_log2 = log2i(br);
-    p.stages = plan->stages;
+    p.nslots = 2 * plan->stages;
     p.num_qtiles = plan->num_qtiles;
-    p.off_q = 0;
-    p.off_stage = (uint32_t)round_up((size_t)pa::kPrefillRows * s->D * 2, 1024);
-    p.half_bytes = (uint32_t)plan->kv_tile * s->D * 2;
+    p.off_p = (uint32_t)pa::kPrefillRows * s->D * 2;
+    p.off_ring = p.off_p + 2u * pa::kPrefillRows * pa::kPrefillKT * 2;
+    p.slot_bytes = (uint32_t)pa::kPrefillKT * s->D * 2;
     if (pa_status st = encode_pool_map(&p.tmap_k, k_cache, s, br, 1)) return st;
     if (pa_status st = encode_pool_map(&p.tmap_v, v_cache, s, br, 1)) return st;
     using PrefillFn = void (*)(const pa::PrefillParams);

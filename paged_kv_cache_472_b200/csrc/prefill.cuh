@@ -10,23 +10,34 @@
 // prefill path), read straight from the pages like the decode.
 //
 // Work decomposition: one CTA per (request, KV head, tile of QT new tokens).
-// Its rows are the QT tokens x G query heads of that KV head (row r = token
-// r / G, head r % G), at most 128, sixteen per consumer warp.  Every row of a
-// CTA sees keys 0 .. pos of its own token, so the CTA streams keys
-// 0 .. pos(last token) once and each warp masks the keys past its rows'
-// positions.  Tiles holding the latest tokens see the most keys; the grid
-// runs them first.
+// Its 128 rows are the QT tokens x G query heads of that KV head (row r =
+// token r / G, head r % G), so every K/V tile staged in shared memory serves
+// the whole head group.  The CTA streams keys 0 .. pos(last token) in tiles
+// of 128 and masks, per row, the keys past the row's own position.  Tiles
+// holding the latest tokens see the most keys; the grid runs them first.
 //
-// Inside a CTA: warp 8 is the producer.  It copies the q rows into shared
-// memory once and fills a ring of stages with tensor-map boxes of KT keys of
-// K and V (the same [d, token row, head] view of the pool as the decode,
-// 128-byte swizzle).  Warps 0-7 compute, per stage:
-//   S = Q K^T       (m16n8k16 tiles: Q as the A operand from registers, K as
-//                    the B operand by ldmatrix from the swizzled stage)
-//   causal mask, fp32 online softmax per row in the base-2 domain,
-//   O += P V        (P reused from the S accumulator fragments as the A
-//                    operand, split into a high and a low 16-bit part as in
-//                    the decode; V as the B operand by transposing ldmatrix).
+// Inside a CTA (5th-generation tensor cores, accumulators in tensor memory):
+//   warp 0     producer: walks the block table and fills a ring of K and V
+//              slots with tensor-map boxes ([d-block][key][128 B], 128-byte
+//              swizzle: the canonical K-major layout for K, MN-major for V);
+//   warp 1     allocates tensor memory; one lane issues every tcgen05.mma:
+//                S_j = Q K_j^T   (M 128 rows, N 128 keys, into one of two S
+//                                 buffers, so S_{j+1} runs while the softmax
+//                                 works on S_j),
+//                O  += P_j V_j   (M 128 rows, N = D, K = keys; P in two
+//                                 16-bit parts, high and low, as in decode);
+//   warps 2-9  softmax: two threads per row (tensor-memory lane = row), one
+//              for each half of the key columns (and of the O columns).  They
+//              copy the q rows into the swizzled Q tile, then per key tile
+//              read their half of the S row, mask, exchange the row maximum
+//              with the partner (a two-warp mbarrier), run the fp32 online
+//              softmax in the base-2 domain, write P (high and low parts) to
+//              shared memory, and at the end combine the two row sums, read
+//              O, divide and store the output row.
+// The running maximum is moved only when a tile's maximum exceeds it by more
+// than 2^8 (weights stay below 256, exact in fp32 and safe in 16 bits); the
+// rescale of O in tensor memory is then rare.  The final division uses the
+// same maximum as every weight, so the result is the plain softmax.
 #pragma once
 
 #include <type_traits>
@@ -35,9 +46,13 @@
 
 namespace pa {
 
-constexpr int kPrefillConsumerWarps = 8;
-constexpr int kPrefillThreads = (kPrefillConsumerWarps + 1) * 32;
-constexpr int kPrefillRows = kPrefillConsumerWarps * 16;  // rows per CTA (tokens x heads)
+constexpr int kPrefillRows = 128;     // rows per CTA: M of every tensor-core product
+constexpr int kPrefillKT = 128;       // keys per tile: N of S, K of P V
+constexpr int kPrefillSoftmaxWarps = 8;
+constexpr int kPrefillThreads = (2 + kPrefillSoftmaxWarps) * 32;  // producer, MMA, softmax
+constexpr int kPrefillTmemCols = 512; // S buffers (2 x 128 columns) + O (D columns), power of two
+constexpr int kPrefillMaxSlots = 8;   // K / V ring slots
+constexpr float kPrefillRescaleLog2 = 8.f;
 
 struct PrefillParams {
     CUtensorMap tmap_k;  // box {64 d, br rows, 1 head} on [d, token row, head] views of the pools
@@ -48,47 +63,50 @@ struct PrefillParams {
     const int32_t *context_lens;
     const int32_t *query_start;
     int32_t *error;      // device error word or nullptr
-    float qscale;        // scale * log2(e)
-    int32_t B, Hq, Hkv, G, bs, bs_log2, num_blocks, max_blocks;
-    int32_t QT;          // new tokens per CTA (QT * G <= kPrefillRows)
-    int32_t KT, kt_log2; // keys per stage
-    int32_t br_log2;     // rows of one box = min(KT, bs)
-    int32_t stages;
+    float qscale;        // |scale| * log2(e)
+    uint32_t qflip;      // 0x80008000 when scale < 0: q enters negated, so scores keep their order
+    int32_t B, Hq, Hkv, G, g_log2, bs, bs_log2, num_blocks, max_blocks;
+    int32_t QT;          // new tokens per CTA (QT * G = kPrefillRows)
+    int32_t br_log2;     // rows of one box = min(kPrefillKT, bs)
+    int32_t nslots;      // ring slots, even: K of tile j in slot 2j mod nslots, V in the next
     int32_t num_qtiles;  // tiles of QT tokens the grid covers per request
-    uint32_t off_q, off_stage, half_bytes;  // shared-memory layout (from the 1024-aligned base)
+    uint32_t off_p, off_ring, slot_bytes;  // shared-memory layout (from the 1024-aligned base; Q at 0)
 };
 static_assert(offsetof(PrefillParams, tmap_k) % 64 == 0 && offsetof(PrefillParams, tmap_v) % 64 == 0,
               "tensor maps must be 64-byte aligned");
-
-// Address of the 16-byte chunk holding d-columns 8*cid .. 8*cid+7 of key row
-// `tok` of a stage filled by {64 d, br rows, 1 head} boxes: [piece][d-chunk of
-// 64][row][128 B], each 128-byte row swizzled (chunk c of row r at c ^ (r & 7)).
-template <int D>
-__device__ __forceinline__ unsigned char *kv_chunk(unsigned char *tile, int tok, int cid, int br_log2) {
-    constexpr int NDC = D / 64;
-    const int piece = tok >> br_log2, r = tok & ((1 << br_log2) - 1);
-    const uint32_t box = 128u << br_log2;  // one {64 d, br rows} box
-    return tile + ((size_t)piece * NDC + (cid >> 3)) * box + (uint32_t)r * 128u +
-           ((uint32_t)((cid & 7) ^ (r & 7)) << 4);
-}
 
 template <typename T, int D>
 __global__ void __launch_bounds__(kPrefillThreads, 1) paged_prefill_kernel(const __grid_constant__ PrefillParams p) {
     using Op = Mma16<T>;
     constexpr int E = 2;
-    constexpr int KS = D / 16;   // k-steps of S over d
-    constexpr int NDC = D / 64;  // 64-wide d-chunks (one box each)
-    constexpr int NO = D / 8;    // n-tiles of O over d
+    constexpr int KT = kPrefillKT;
+    constexpr int KS = D / 16;                         // k-steps of S over d
+    constexpr int NDC = D / 64;                        // 64-wide d-blocks
+    constexpr uint32_t kBlk = kPrefillRows * 128u;     // one 64-column block of a 128-row operand: 16 KB
+    constexpr uint32_t kPPart = kPrefillRows * KT * E; // one 16-bit part of P
+    constexpr uint32_t kSlotBlk = KT * 128u;           // one d-block of a K / V slot
+    constexpr bool kBf16 = std::is_same<T, __nv_bfloat16>::value;
+    constexpr uint32_t kIdescPV = umma_idesc(kPrefillRows, D, false, true, kBf16);
+    constexpr uint32_t kColO = 2 * KT;                 // tensor-memory column of O
     extern __shared__ __align__(1024) unsigned char smem_raw[];
-    unsigned char *smem = smem_raw + ((1024u - (smem_u32(smem_raw) & 1023u)) & 1023u);
-    __shared__ uint64_t bars[2 * 8 + 1];
+    unsigned char *smem = smem_raw;  // the plan leaves no room to realign: checked below
+    __shared__ uint64_t bars[2 * kPrefillMaxSlots + 16];
+    __shared__ float red_s[2][2][kPrefillRows];  // [tile parity][column half][row]: row max / row sum
+    __shared__ uint32_t tmem_base_s;
     __shared__ volatile int abort_s;
 
     const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
-    const int S = p.stages;
-    uint64_t *full = bars, *empty = bars + 8, *qbar = bars + 16;
+    const int NS = p.nslots;
+    uint64_t *full = bars, *empty = bars + kPrefillMaxSlots;
+    uint64_t *sfull = bars + 2 * kPrefillMaxSlots, *sfree = sfull + 2;
+    uint64_t *pfull = sfree + 2, *odone = pfull + 1, *qfull = odone + 1, *fin = qfull + 1;
+    uint64_t *xchg = fin + 1;  // [lane quarter][parity]: the two softmax warps of the same rows
     volatile int *abort_flag = &abort_s;
 
+    if (smem_u32(smem_raw) & 1023u) {  // the 128-byte swizzle needs 1024-byte aligned tiles
+        if (tid == 0) set_error(p.error, PA_DEVERR_SMEM);
+        return;
+    }
     // ---- the tile: request, KV head, new tokens [t0, t0 + ntok) ----
     const int b = blockIdx.z, g = blockIdx.y;
     const int qt = p.num_qtiles - 1 - (int)blockIdx.x;  // latest (heaviest) tiles first
@@ -103,48 +121,48 @@ __global__ void __launch_bounds__(kPrefillThreads, 1) paged_prefill_kernel(const
     const int t0 = qt * p.QT;
     if (t0 >= n) return;
     const int ntok = min(p.QT, n - t0);
-    const int pos0 = L - n + t0;       // position of the tile's first token
-    const int kend = pos0 + ntok;      // keys 0 .. kend-1 are visible to some row
-    const int ntiles = (kend + p.KT - 1) >> p.kt_log2;
+    const int pos0 = L - n + t0;            // position of the tile's first token
+    const int kend = pos0 + ntok;           // keys 0 .. kend-1 are visible to some row
+    const int ntiles = (kend + KT - 1) / KT;
+    const int nk_last = kend - (ntiles - 1) * KT;  // keys of the last tile holding visible keys
+    const int n16_last = (nk_last + 15) >> 4;      // its 16-key groups
 
     if (tid == 0) {
-        for (int s = 0; s < S; ++s) {
+        for (int s = 0; s < NS; ++s) {
             mbar_init(&full[s], 1);
-            mbar_init(&empty[s], kPrefillConsumerWarps);
+            mbar_init(&empty[s], 1);
         }
-        mbar_init(qbar, 1);
+        for (int i = 0; i < 2; ++i) {
+            mbar_init(&sfull[i], 1);
+            mbar_init(&sfree[i], kPrefillSoftmaxWarps);
+        }
+        mbar_init(pfull, kPrefillSoftmaxWarps);
+        mbar_init(odone, 1);
+        mbar_init(qfull, kPrefillSoftmaxWarps);
+        mbar_init(fin, 1);
+        for (int i = 0; i < 8; ++i) mbar_init(&xchg[i], 2);
         abort_s = 0;
         fence_mbarrier_init();
     }
+    if (warp == 1) tmem_alloc(&tmem_base_s, kPrefillTmemCols);
+    tc_fence_before();
     __syncthreads();
-    unsigned char *qs = smem + p.off_q;
-    unsigned char *stage_base = smem + p.off_stage;
+    tc_fence_after();
+    const uint32_t tmem = tmem_base_s;
+    unsigned char *ring = smem + p.off_ring;
 
-    if (warp == kPrefillConsumerWarps) {
+    if (warp == 0) {
         // ================= producer =================
         const uint64_t policy = policy_evict_normal();  // K/V are read by every q-tile of the request
-        if (lane == 0) {
-            // q rows of the tile: token i, heads g*G .. g*G+G-1 are G*D contiguous elements
-            const uint32_t row_bytes = (uint32_t)p.G * D * E;
-            mbar_arrive_expect_tx(qbar, (uint32_t)ntok * row_bytes);
-            const unsigned char *qg = static_cast<const unsigned char *>(p.q);
-            for (int i = 0; i < ntok; ++i)
-                bulk_g2s(qs + (size_t)i * row_bytes,
-                         qg + (((size_t)(q0 + t0 + i)) * p.Hq + (size_t)g * p.G) * D * E, row_bytes, qbar);
-        }
         const int32_t *table = p.block_tables + (size_t)b * p.max_blocks;
         const int br = 1 << p.br_log2;
         const uint32_t box_bytes = 128u << p.br_log2;
-        int stage = 0;
+        int slot = 0;
         uint32_t phase = 0, issued = 0, issued_par = 0;
         bool ok = true;
-        for (int kt = 0; kt < ntiles && ok; ++kt) {
-            if (!mbar_wait(&empty[stage], phase ^ 1u, abort_flag)) {
-                ok = false;
-                break;
-            }
-            const int k0 = kt * p.KT;
-            const int nk = min(p.KT, kend - k0);
+        for (int j = 0; j < ntiles && ok; ++j) {
+            const int k0 = j * KT;
+            const int nk = min(KT, kend - k0);
             const int npc = (nk + br - 1) >> p.br_log2;  // box pieces holding visible keys
             int phys = -1;
             uint32_t bytes = 0;
@@ -155,29 +173,33 @@ __global__ void __launch_bounds__(kPrefillThreads, 1) paged_prefill_kernel(const
                     set_error(p.error, PA_DEVERR_BLOCK_ID);
                     phys = -1;
                 } else {
-                    bytes = 2u * NDC * box_bytes;
+                    bytes = NDC * box_bytes;
                 }
             }
 #pragma unroll
             for (int m = 16; m >= 1; m >>= 1) bytes += __shfl_xor_sync(0xffffffffu, bytes, m);
-            unsigned char *kdst = stage_base + (size_t)stage * 2 * p.half_bytes;
-            unsigned char *vdst = kdst + p.half_bytes;
-            if (lane == 0) mbar_arrive_expect_tx(&full[stage], bytes);
-            __syncwarp();
-            if (phys >= 0) {
-                const int32_t row = phys * p.bs + (tp & (p.bs - 1));
+            const int32_t row = phys * p.bs + (tp & (p.bs - 1));
 #pragma unroll
-                for (int c2 = 0; c2 < NDC; ++c2) {
-                    const size_t off = ((size_t)lane * NDC + c2) * box_bytes;
-                    tma_load_3d(kdst + off, &p.tmap_k, c2 * 64, row, g, &full[stage], policy);
-                    tma_load_3d(vdst + off, &p.tmap_v, c2 * 64, row, g, &full[stage], policy);
+            for (int mat = 0; mat < 2; ++mat) {  // K, then V
+                if (!mbar_wait(&empty[slot], phase ^ 1u, abort_flag)) {
+                    ok = false;
+                    break;
                 }
-            }
-            issued |= 1u << stage;
-            issued_par = (issued_par & ~(1u << stage)) | (phase << stage);
-            if (++stage == S) {
-                stage = 0;
-                phase ^= 1u;
+                if (lane == 0) mbar_arrive_expect_tx(&full[slot], bytes);
+                __syncwarp();
+                if (phys >= 0) {
+                    unsigned char *dst = ring + (size_t)slot * p.slot_bytes + (size_t)lane * box_bytes;
+#pragma unroll
+                    for (int c = 0; c < NDC; ++c)
+                        tma_load_3d(dst + c * kSlotBlk, mat ? &p.tmap_v : &p.tmap_k, c * 64, row, g, &full[slot],
+                                    policy);
+                }
+                issued |= 1u << slot;
+                issued_par = (issued_par & ~(1u << slot)) | (phase << slot);
+                if (++slot == NS) {
+                    slot = 0;
+                    phase ^= 1u;
+                }
             }
         }
         if (!ok) {
@@ -186,194 +208,265 @@ __global__ void __launch_bounds__(kPrefillThreads, 1) paged_prefill_kernel(const
         }
         // every copy issued lands before the CTA retires
         volatile int never = 0;
-        for (int st = 0; st < S; ++st)
+        for (int st = 0; st < NS; ++st)
             if (issued & (1u << st)) mbar_wait(&full[st], (issued_par >> st) & 1u, &never);
-        mbar_wait(qbar, 0u, &never);
-        return;
-    }
-
-    // ================= consumers: rows warp*16 .. warp*16+15 =================
-    const int g4 = lane >> 2, t4 = lane & 3;
-    const int rows = ntok * p.G;
-    const int r_lo = warp * 16 + g4, r_hi = r_lo + 8;  // this lane's two rows
-    const int qpos_lo = pos0 + r_lo / p.G, qpos_hi = pos0 + r_hi / p.G;
-    const int warp_last_pos = pos0 + min(warp * 16 + 15, rows - 1) / p.G;  // furthest key any row sees
-    const bool warp_live = warp * 16 < rows;
-
-    if (!mbar_wait(qbar, 0u, abort_flag)) {
-        *abort_flag = 1;
-        if (lane == 0) set_error(p.error, PA_DEVERR_TIMEOUT);
-    }
-    // Q as A fragments (m16 x k16 per k-step): row r at qs + r * D * E
-    uint32_t qa[KS][4];
-    {
-        const unsigned char *r0 = qs + (size_t)r_lo * D * E, *r1 = qs + (size_t)r_hi * D * E;
-        const bool v0 = r_lo < rows, v1 = r_hi < rows;
-#pragma unroll
-        for (int ks = 0; ks < KS; ++ks) {
-            const int c = ks * 16 + 2 * t4;
-            qa[ks][0] = v0 ? *reinterpret_cast<const uint32_t *>(r0 + c * E) : 0u;
-            qa[ks][1] = v1 ? *reinterpret_cast<const uint32_t *>(r1 + c * E) : 0u;
-            qa[ks][2] = v0 ? *reinterpret_cast<const uint32_t *>(r0 + (c + 8) * E) : 0u;
-            qa[ks][3] = v1 ? *reinterpret_cast<const uint32_t *>(r1 + (c + 8) * E) : 0u;
-        }
-    }
-    float o[NO][4];
-#pragma unroll
-    for (int j = 0; j < NO; ++j) o[j][0] = o[j][1] = o[j][2] = o[j][3] = 0.f;
-    float m_lo = -INFINITY, m_hi = -INFINITY, l_lo = 0.f, l_hi = 0.f;
-
-    // ldmatrix lane roles: K as B (non-transposed) and V as B (transposed)
-    const int kb_key = (lane & 7) + ((lane >> 4) & 1) * 8, kb_col = ((lane >> 3) & 1);
-    const int vb_key = (lane & 7) + ((lane >> 3) & 1) * 8, vb_col = (lane >> 4);
-
-    int stage = 0;
-    uint32_t phase = 0;
-    for (int kt = 0; kt < ntiles; ++kt) {
-        if (!*abort_flag && !mbar_wait(&full[stage], phase, abort_flag)) {
-            *abort_flag = 1;
-            set_error(p.error, PA_DEVERR_TIMEOUT);
-        }
-        const int k0 = kt * p.KT;
-        if (!*abort_flag && warp_live && k0 <= warp_last_pos) {
-            unsigned char *kst = stage_base + (size_t)stage * 2 * p.half_bytes;
-            unsigned char *vst = kst + p.half_bytes;
-            const int nk16 = (min(p.KT, kend - k0) + 15) >> 4;  // 16-key groups with visible keys
-            // V rows past the context end (unwritten pool slots in the last
-            // block) get zero weight, but may hold anything: zero them before
-            // they enter P V.  Every warp writes the same zeros before its own
-            // reads, so no warp can see a stale row.
-            const int vz0 = L - k0, vz1 = nk16 * 16;
-            if (vz0 < vz1) {
-                for (int i = lane; i < (vz1 - vz0) * (D / 8); i += 32)
-                    *reinterpret_cast<uint4 *>(kv_chunk<D>(vst, vz0 + i / (D / 8), i % (D / 8), p.br_log2)) =
-                        make_uint4(0u, 0u, 0u, 0u);
-                fence_async_smem();  // ordered before the next tensor-map fill of this stage
-                __syncwarp();
-            }
-            // One online-softmax step over NG groups of 16 keys (groups kg0 ..
-            // kg0 + NG - 1, all loaded): S, mask, one max / rescale / sum, P V.
-            auto step = [&](auto ng, int kg0) {
-                constexpr int NG = decltype(ng)::value;
-                // ---- S[16 rows x 16 NG keys] = Q K^T, one accumulation chain per 8 keys ----
-                float sc[2 * NG][4];
-#pragma unroll
-                for (int nt = 0; nt < 2 * NG; ++nt) sc[nt][0] = sc[nt][1] = sc[nt][2] = sc[nt][3] = 0.f;
+    } else if (warp == 1) {
+        // ================= MMA issue (one lane) =================
+        if (lane == 0) {
+            const uint32_t q_addr = smem_u32(smem), p_addr = smem_u32(smem + p.off_p), r_addr = smem_u32(ring);
+            bool ok = mbar_wait(qfull, 0u, abort_flag);
+            bool issued_any = false;
+            // O += P_i V_i for tile i (P high part, then low part)
+            auto pv = [&](int i) {
+                if (!ok) return;
+                const int sv = (2 * i + 1) % NS;
+                const uint32_t par = (uint32_t)((2 * i + 1) / NS) & 1u;
+                if (!mbar_wait(pfull, (uint32_t)i & 1u, abort_flag) || !mbar_wait(&full[sv], par, abort_flag)) {
+                    ok = false;
+                    return;
+                }
+                tc_fence_after();
+                const int n16 = i == ntiles - 1 ? n16_last : KT / 16;
+                const uint32_t vb = r_addr + (uint32_t)sv * p.slot_bytes;
+                for (int part = 0; part < 2; ++part) {
+                    const uint32_t pb = p_addr + (uint32_t)part * kPPart;
+                    for (int kk = 0; kk < n16; ++kk) {
+                        const uint64_t ad = umma_desc_sw128(pb + (kk >> 2) * kBlk + (kk & 3) * 32, 16, 1024);
+                        const uint64_t bd = umma_desc_sw128(vb + kk * 2048, kSlotBlk, 1024);
+                        umma_f16(tmem + kColO, ad, bd, kIdescPV, (i > 0 || part > 0 || kk > 0) ? 1u : 0u);
+                    }
+                }
+                umma_commit(odone);
+                umma_commit(&empty[sv]);
+                issued_any = true;
+            };
+            for (int j = 0; j < ntiles && ok; ++j) {
+                const int sk = (2 * j) % NS;
+                const uint32_t par = (uint32_t)((2 * j) / NS) & 1u;
+                if (!mbar_wait(&full[sk], par, abort_flag) ||
+                    (j >= 2 && !mbar_wait(&sfree[j & 1], (uint32_t)((j >> 1) - 1) & 1u, abort_flag))) {
+                    ok = false;
+                    break;
+                }
+                tc_fence_after();
+                const int N = j == ntiles - 1 ? n16_last * 16 : KT;
+                const uint32_t idesc = umma_idesc(kPrefillRows, N, false, false, kBf16);
+                const uint32_t kb = r_addr + (uint32_t)sk * p.slot_bytes;
 #pragma unroll
                 for (int ks = 0; ks < KS; ++ks) {
-#pragma unroll
-                    for (int gi = 0; gi < NG; ++gi) {
-                        uint32_t bf[4];
-                        ldmatrix_x4(bf, kv_chunk<D>(kst, (kg0 + gi) * 16 + kb_key, ks * 2 + kb_col, p.br_log2));
-                        Op::mma(sc[2 * gi], qa[ks], bf[0], bf[1]);
-                        Op::mma(sc[2 * gi + 1], qa[ks], bf[2], bf[3]);
-                    }
+                    const uint64_t ad = umma_desc_sw128(q_addr + (ks >> 2) * kBlk + (ks & 3) * 32, 16, 1024);
+                    const uint64_t bd = umma_desc_sw128(kb + (ks >> 2) * kSlotBlk + (ks & 3) * 32, 16, 1024);
+                    umma_f16(tmem + (uint32_t)(j & 1) * KT, ad, bd, idesc, ks > 0 ? 1u : 0u);
                 }
-                // ---- causal mask, scores in the base-2 domain ----
-                // sc[nt][0..1]: row lo, keys kc, kc+1 with kc = k0 + kg0*16 + nt*8 + 2*t4; [2..3]: row hi
-                float mx_lo = -INFINITY, mx_hi = -INFINITY;
-#pragma unroll
-                for (int nt = 0; nt < 2 * NG; ++nt) {
-                    const int kc = k0 + kg0 * 16 + nt * 8 + 2 * t4;
-#pragma unroll
-                    for (int i = 0; i < 2; ++i) {
-                        sc[nt][i] = kc + i <= qpos_lo ? sc[nt][i] * p.qscale : -INFINITY;
-                        sc[nt][2 + i] = kc + i <= qpos_hi ? sc[nt][2 + i] * p.qscale : -INFINITY;
-                        mx_lo = fmaxf(mx_lo, sc[nt][i]);
-                        mx_hi = fmaxf(mx_hi, sc[nt][2 + i]);
-                    }
-                }
-                mx_lo = fmaxf(mx_lo, __shfl_xor_sync(0xffffffffu, mx_lo, 1));
-                mx_lo = fmaxf(mx_lo, __shfl_xor_sync(0xffffffffu, mx_lo, 2));
-                mx_hi = fmaxf(mx_hi, __shfl_xor_sync(0xffffffffu, mx_hi, 1));
-                mx_hi = fmaxf(mx_hi, __shfl_xor_sync(0xffffffffu, mx_hi, 2));
-                const float mn_lo = fmaxf(m_lo, mx_lo), mn_hi = fmaxf(m_hi, mx_hi);
-                // a row with no visible key yet keeps m = -inf: its weights are 0
-                const float al_lo = mn_lo == -INFINITY ? 1.f : exp2_fast(m_lo - mn_lo);
-                const float al_hi = mn_hi == -INFINITY ? 1.f : exp2_fast(m_hi - mn_hi);
-                const float sub_lo = mn_lo == -INFINITY ? 0.f : mn_lo, sub_hi = mn_hi == -INFINITY ? 0.f : mn_hi;
-                float sum_lo = 0.f, sum_hi = 0.f;
-#pragma unroll
-                for (int nt = 0; nt < 2 * NG; ++nt) {
-#pragma unroll
-                    for (int i = 0; i < 2; ++i) {
-                        sc[nt][i] = exp2_fast(sc[nt][i] - sub_lo);  // masked: 2^-inf = 0
-                        sc[nt][2 + i] = exp2_fast(sc[nt][2 + i] - sub_hi);
-                        sum_lo += sc[nt][i];
-                        sum_hi += sc[nt][2 + i];
-                    }
-                }
-                sum_lo += __shfl_xor_sync(0xffffffffu, sum_lo, 1);
-                sum_lo += __shfl_xor_sync(0xffffffffu, sum_lo, 2);
-                sum_hi += __shfl_xor_sync(0xffffffffu, sum_hi, 1);
-                sum_hi += __shfl_xor_sync(0xffffffffu, sum_hi, 2);
-                l_lo = l_lo * al_lo + sum_lo;
-                l_hi = l_hi * al_hi + sum_hi;
-                m_lo = mn_lo;
-                m_hi = mn_hi;
-                if (al_lo != 1.f || al_hi != 1.f) {
-#pragma unroll
-                    for (int j = 0; j < NO; ++j) {
-                        o[j][0] *= al_lo;
-                        o[j][1] *= al_lo;
-                        o[j][2] *= al_hi;
-                        o[j][3] *= al_hi;
-                    }
-                }
-                // ---- O[16 rows x D] += P V, one 16-key group at a time ----
-#pragma unroll
-                for (int gi = 0; gi < NG; ++gi) {
-                    // P as the A operand (m16 x k16), high and low 16-bit parts
-                    const float *c0 = sc[2 * gi], *c1 = sc[2 * gi + 1];
-                    uint32_t ph[4], pl[4];
-                    ph[0] = Op::pack_p(c0[0], c0[1]);  // row lo, keys +2*t4
-                    ph[1] = Op::pack_p(c0[2], c0[3]);  // row hi
-                    ph[2] = Op::pack_p(c1[0], c1[1]);  // row lo, keys +8+2*t4
-                    ph[3] = Op::pack_p(c1[2], c1[3]);  // row hi
-                    {
-                        const float2 h0 = Op::unpack(ph[0]), h1 = Op::unpack(ph[1]);
-                        const float2 h2 = Op::unpack(ph[2]), h3 = Op::unpack(ph[3]);
-                        pl[0] = Op::pack_p(c0[0] - h0.x, c0[1] - h0.y);
-                        pl[1] = Op::pack_p(c0[2] - h1.x, c0[3] - h1.y);
-                        pl[2] = Op::pack_p(c1[0] - h2.x, c1[1] - h2.y);
-                        pl[3] = Op::pack_p(c1[2] - h3.x, c1[3] - h3.y);
-                    }
-                    const int vkey = (kg0 + gi) * 16 + vb_key;
-#pragma unroll
-                    for (int j2 = 0; j2 < NO / 2; ++j2) {
-                        uint32_t vf[4];
-                        ldmatrix_x4_trans(vf, kv_chunk<D>(vst, vkey, j2 * 2 + vb_col, p.br_log2));
-                        Op::mma(o[2 * j2], ph, vf[0], vf[1]);
-                        Op::mma(o[2 * j2 + 1], ph, vf[2], vf[3]);
-                        Op::mma(o[2 * j2], pl, vf[0], vf[1]);
-                        Op::mma(o[2 * j2 + 1], pl, vf[2], vf[3]);
-                    }
-                }
-            };
-            int kg = 0;
-            for (; kg + 1 < nk16; kg += 2) step(std::integral_constant<int, 2>{}, kg);
-            if (kg < nk16) step(std::integral_constant<int, 1>{}, kg);
+                umma_commit(&sfull[j & 1]);
+                umma_commit(&empty[sk]);
+                issued_any = true;
+                if (j >= 1) pv(j - 1);
+            }
+            if (ok) pv(ntiles - 1);
+            if (!ok) {
+                *abort_flag = 1;
+                set_error(p.error, PA_DEVERR_TIMEOUT);
+            }
+            if (issued_any) {
+                // every product issued completes before tensor memory is released
+                umma_commit(fin);
+                volatile int never = 0;
+                mbar_wait(fin, 0u, &never);
+            }
         }
-        __syncwarp();
-        if (lane == 0) mbar_arrive(&empty[stage]);
-        if (++stage == S) {
-            stage = 0;
-            phase ^= 1u;
+    } else {
+        // ================= softmax: two threads per row =================
+        constexpr int HC = KT / 2;            // S columns per thread
+        constexpr int HD = D / 2;             // O columns per thread
+        const int half = (warp - 2) >> 2;     // column half
+        const int quad = warp & 3;            // tensor-memory lane quarter of this warp
+        const int row = quad * 32 + lane;
+        const int sid = tid - 64;             // 0 .. 255 over the softmax warps
+        const uint32_t tl = tmem + ((uint32_t)(quad * 32) << 16);  // this warp's lanes
+        uint64_t *xb = xchg + quad * 2;
+        const int tok = row >> p.g_log2, hj = row & (p.G - 1);
+        const bool valid = tok < ntok;
+        const size_t grow = ((size_t)(q0 + t0 + tok) * p.Hq + (size_t)g * p.G + hj) * D;  // q / out row
+        // ---- Q tile: half of row `row`, K-major with the 128-byte swizzle ----
+        {
+            const uint4 *src = reinterpret_cast<const uint4 *>(static_cast<const unsigned char *>(p.q) + grow * E);
+#pragma unroll
+            for (int i = 0; i < D / 16; ++i) {
+                const int c = half * (D / 16) + i;
+                uint4 v = make_uint4(0u, 0u, 0u, 0u);
+                if (valid) {
+                    v = __ldg(src + c);
+                    v.x ^= p.qflip;
+                    v.y ^= p.qflip;
+                    v.z ^= p.qflip;
+                    v.w ^= p.qflip;
+                }
+                *reinterpret_cast<uint4 *>(smem + (c >> 3) * kBlk + row * 128 + (((c & 7) ^ (row & 7)) << 4)) = v;
+            }
+            fence_async_smem();
+            __syncwarp();
+            if (lane == 0) mbar_arrive(qfull);
+        }
+        const int pos_row = pos0 + (valid ? tok : ntok - 1);  // rows past the tokens mirror the last token
+        unsigned char *pst = smem + p.off_p + half * kBlk;    // this half's 64-key block of P
+        const float qs = p.qscale;
+        float m_used = -INFINITY, l = 0.f;
+        bool ok = true;
+        for (int j = 0; j < ntiles; ++j) {
+            const int k0 = j * KT;
+            if (!mbar_wait(&sfull[j & 1], (uint32_t)(j >> 1) & 1u, abort_flag)) {
+                ok = false;
+                break;
+            }
+            tc_fence_after();
+            float s[HC];
+            tmem_ld32(tl + (uint32_t)(j & 1) * KT + half * HC, s);
+            tmem_ld32(tl + (uint32_t)(j & 1) * KT + half * HC + 32, s + 32);
+            tmem_wait_ld();
+            tc_fence_before();
+            __syncwarp();
+            if (lane == 0) mbar_arrive(&sfree[j & 1]);
+            // keys past the row's position (or past the keys loaded) are out
+            const bool diag = k0 + KT - 1 > pos0;
+            const int lim = pos_row - k0 - half * HC;  // columns c <= lim are visible
+            float m4[4] = {-INFINITY, -INFINITY, -INFINITY, -INFINITY};
+            if (diag) {
+#pragma unroll
+                for (int c = 0; c < HC; ++c) {
+                    s[c] = c <= lim ? s[c] : -INFINITY;
+                    m4[c & 3] = fmaxf(m4[c & 3], s[c]);
+                }
+            } else {
+#pragma unroll
+                for (int c = 0; c < HC; ++c) m4[c & 3] = fmaxf(m4[c & 3], s[c]);
+            }
+            float mx = fmaxf(fmaxf(m4[0], m4[1]), fmaxf(m4[2], m4[3]));
+            // row maximum over both halves
+            red_s[j & 1][half][row] = mx;
+            __syncwarp();
+            if (lane == 0) mbar_arrive(&xb[j & 1]);
+            if (!mbar_wait(&xb[j & 1], (uint32_t)(j >> 1) & 1u, abort_flag)) {
+                ok = false;
+                break;
+            }
+            mx = fmaxf(mx, red_s[j & 1][half ^ 1][row]);
+            const float mt = mx == -INFINITY ? -INFINITY : mx * qs;  // base-2 domain
+            const bool move = mt > m_used + kPrefillRescaleLog2;
+            float alpha = 1.f;
+            if (move) {
+                alpha = exp2_fast(m_used - mt);  // 0 on the first tile
+                m_used = mt;
+            }
+            const float nm = -m_used;
+            float l4[4] = {0.f, 0.f, 0.f, 0.f};
+            if (diag) {
+#pragma unroll
+                for (int c = 0; c < HC; ++c) {
+                    s[c] = c <= lim ? exp2_fast(fmaf(s[c], qs, nm)) : 0.f;
+                    l4[c & 3] += s[c];
+                }
+            } else {
+#pragma unroll
+                for (int c = 0; c < HC; ++c) {
+                    s[c] = exp2_fast(fmaf(s[c], qs, nm));
+                    l4[c & 3] += s[c];
+                }
+            }
+            l = l * alpha + ((l4[0] + l4[1]) + (l4[2] + l4[3]));
+            if (j >= 1) {
+                // P V of the previous tile is done: P's buffer is free and O is current
+                if (!mbar_wait(odone, (uint32_t)(j - 1) & 1u, abort_flag)) {
+                    ok = false;
+                    break;
+                }
+                tc_fence_after();
+                if (__any_sync(0xffffffffu, move)) {
+#pragma unroll
+                    for (int c = 0; c < HD / 32; ++c) {
+                        float o[32];
+                        tmem_ld32(tl + kColO + half * HD + c * 32, o);
+                        tmem_wait_ld();
+#pragma unroll
+                        for (int i = 0; i < 32; ++i) o[i] *= alpha;
+                        tmem_st32(tl + kColO + half * HD + c * 32, o);
+                    }
+                    tmem_wait_st();
+                }
+            }
+            if (j == ntiles - 1) {
+                // V rows of the last 16-key group past the context end are
+                // unwritten pool slots: zero them (weight 0 times anything
+                // must stay 0) once their tensor-map fill has landed
+                const int z0 = L - k0, z1 = n16_last * 16;
+                if (z0 < z1) {
+                    const int sv = (2 * j + 1) % NS;
+                    if (!mbar_wait(&full[sv], (uint32_t)((2 * j + 1) / NS) & 1u, abort_flag)) {
+                        ok = false;
+                        break;
+                    }
+                    unsigned char *vs = ring + (size_t)sv * p.slot_bytes;
+                    for (int i = sid; i < (z1 - z0) * NDC * 8; i += 32 * kPrefillSoftmaxWarps) {
+                        const int r = z0 + i / (NDC * 8), c = i % (NDC * 8);
+                        *reinterpret_cast<uint4 *>(vs + (c >> 3) * kSlotBlk + r * 128 + ((c & 7) << 4)) =
+                            make_uint4(0u, 0u, 0u, 0u);
+                    }
+                }
+            }
+            // ---- P (high and low 16-bit parts), K-major with the 128-byte swizzle ----
+#pragma unroll
+            for (int c8 = 0; c8 < HC / 8; ++c8) {
+                uint32_t hi[4], lo[4];
+#pragma unroll
+                for (int i = 0; i < 4; ++i) Op::split_p(s[c8 * 8 + 2 * i], s[c8 * 8 + 2 * i + 1], hi[i], lo[i]);
+                const uint32_t off = row * 128 + ((c8 ^ (row & 7)) << 4);
+                *reinterpret_cast<uint4 *>(pst + off) = make_uint4(hi[0], hi[1], hi[2], hi[3]);
+                *reinterpret_cast<uint4 *>(pst + kPPart + off) = make_uint4(lo[0], lo[1], lo[2], lo[3]);
+            }
+            fence_async_smem();
+            tc_fence_before();
+            __syncwarp();
+            if (lane == 0) mbar_arrive(pfull);
+        }
+        if (ok && mbar_wait(odone, (uint32_t)(ntiles - 1) & 1u, abort_flag)) {
+            tc_fence_after();
+            // row sum over both halves
+            red_s[ntiles & 1][half][row] = l;
+            __syncwarp();
+            if (lane == 0) mbar_arrive(&xb[ntiles & 1]);
+            ok = mbar_wait(&xb[ntiles & 1], (uint32_t)(ntiles >> 1) & 1u, abort_flag);
+            if (ok) {
+                // ---- normalise and store this half of the rows of real tokens ----
+                const float inv = 1.f / (l + red_s[ntiles & 1][half ^ 1][row]);
+                uint4 *dst = reinterpret_cast<uint4 *>(static_cast<unsigned char *>(p.out) + (grow + half * HD) * E);
+#pragma unroll
+                for (int c = 0; c < HD / 32; ++c) {
+                    float o[32];
+                    tmem_ld32(tl + kColO + half * HD + c * 32, o);
+                    tmem_wait_ld();
+                    if (valid) {
+#pragma unroll
+                        for (int i = 0; i < 4; ++i)
+                            dst[c * 4 + i] = make_uint4(Op::pack(o[8 * i] * inv, o[8 * i + 1] * inv),
+                                                        Op::pack(o[8 * i + 2] * inv, o[8 * i + 3] * inv),
+                                                        Op::pack(o[8 * i + 4] * inv, o[8 * i + 5] * inv),
+                                                        Op::pack(o[8 * i + 6] * inv, o[8 * i + 7] * inv));
+                    }
+                }
+            }
+        } else {
+            ok = false;
+        }
+        if (!ok) {
+            *abort_flag = 1;
+            if (lane == 0) set_error(p.error, PA_DEVERR_TIMEOUT);
         }
     }
-    if (*abort_flag || !warp_live) return;
-    // ---- normalise and store the rows of real tokens ----
-    unsigned char *outb = static_cast<unsigned char *>(p.out);
-    const float inv_lo = 1.f / l_lo, inv_hi = 1.f / l_hi;
-    const size_t orow_lo = ((size_t)(q0 + t0 + r_lo / p.G) * p.Hq + (size_t)g * p.G + r_lo % p.G) * D;
-    const size_t orow_hi = ((size_t)(q0 + t0 + r_hi / p.G) * p.Hq + (size_t)g * p.G + r_hi % p.G) * D;
-#pragma unroll
-    for (int j = 0; j < NO; ++j) {
-        const int d = j * 8 + 2 * t4;
-        if (r_lo < rows)
-            *reinterpret_cast<uint32_t *>(outb + (orow_lo + d) * E) = Op::pack(o[j][0] * inv_lo, o[j][1] * inv_lo);
-        if (r_hi < rows)
-            *reinterpret_cast<uint32_t *>(outb + (orow_hi + d) * E) = Op::pack(o[j][2] * inv_hi, o[j][3] * inv_hi);
+    tc_fence_before();
+    __syncthreads();
+    if (warp == 1) {
+        tc_fence_after();
+        tmem_dealloc(tmem, kPrefillTmemCols);
     }
 }
 
