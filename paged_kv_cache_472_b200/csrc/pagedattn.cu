@@ -546,12 +546,11 @@ pa_status pa_prefill_plan(const pa_shape *s, int32_t max_new_tokens, pa_prefill_
     const int QT = pa::kPrefillRows / G;
     const int KT = pa::kPrefillKT;
     const uint32_t q_bytes = (uint32_t)pa::kPrefillRows * s->D * 2;
-    const uint32_t p_bytes = 2u * pa::kPrefillRows * KT * 2;  // P, high and low parts
     const uint32_t slot = (uint32_t)KT * s->D * 2;
     int nslots = pa::kPrefillMaxSlots;
     uint32_t total = 0;
     for (; nslots >= 2; nslots -= 2) {
-        total = q_bytes + p_bytes + (uint32_t)nslots * slot;  // the kernel checks its base is 1024-aligned
+        total = q_bytes + (uint32_t)nslots * slot;  // the kernel checks its base is 1024-aligned
         if (total + kPrefillStaticSmem <= (uint32_t)kSmemLimit) break;
     }
     memset(plan, 0, sizeof *plan);
@@ -604,8 +603,7 @@ pa_status pa_prefill(const void *q, const void *k_cache, const void *v_cache, co
     p.br_log2 = log2i(br);
     p.nslots = 2 * plan->stages;
     p.num_qtiles = plan->num_qtiles;
-    p.off_p = (uint32_t)pa::kPrefillRows * s->D * 2;
-    p.off_ring = p.off_p + 2u * pa::kPrefillRows * pa::kPrefillKT * 2;
+    p.off_ring = (uint32_t)pa::kPrefillRows * s->D * 2;
     p.slot_bytes = (uint32_t)pa::kPrefillKT * s->D * 2;
     if (pa_status st = encode_pool_map(&p.tmap_k, k_cache, s, br, 1)) return st;
     if (pa_status st = encode_pool_map(&p.tmap_v, v_cache, s, br, 1)) return st;

@@ -17,23 +17,30 @@
 // holding the latest tokens see the most keys; the grid runs them first.
 //
 // Inside a CTA (5th-generation tensor cores, accumulators in tensor memory):
-//   warp 0     producer: walks the block table and fills a ring of K and V
-//              slots with tensor-map boxes ([d-block][key][128 B], 128-byte
-//              swizzle: the canonical K-major layout for K, MN-major for V);
+//   warps 0,10 producers of K and of V: each walks the block table (one tile
+//              ahead) and fills its own ring of slots with tensor-map boxes
+//              ([d-block][key][128 B], 128-byte swizzle: the canonical K-major
+//              layout for K, MN-major for V), so K never queues behind a V
+//              slot that a product still holds;
 //   warp 1     allocates tensor memory; one lane issues every tcgen05.mma:
-//                S_j = Q K_j^T   (M 128 rows, N 128 keys, into one of two S
-//                                 buffers, so S_{j+1} runs while the softmax
-//                                 works on S_j),
-//                O  += P_j V_j   (M 128 rows, N = D, K = keys; P in two
-//                                 16-bit parts, high and low, as in decode);
+//                S_j = Q K_j^T   (M 128 rows, N 128 keys, into one of three
+//                                 S buffers, up to three tiles ahead of the
+//                                 softmax),
+//                O  += P_j V_j   (M 128 rows, N = D, K = keys; P read from
+//                                 tensor memory, where the softmax wrote it
+//                                 over S_j, in two 16-bit parts, high and
+//                                 low, as in decode);
 //   warps 2-9  softmax: two threads per row (tensor-memory lane = row), one
 //              for each half of the key columns (and of the O columns).  They
 //              copy the q rows into the swizzled Q tile, then per key tile
 //              read their half of the S row, mask, exchange the row maximum
 //              with the partner (a two-warp mbarrier), run the fp32 online
-//              softmax in the base-2 domain, write P (high and low parts) to
-//              shared memory, and at the end combine the two row sums, read
-//              O, divide and store the output row.
+//              softmax in the base-2 domain, write P (high and low parts) into
+//              the S buffer they read, and at the end combine the two row
+//              sums, read O, divide and store the output row.
+// The tensor pipe runs its products in issue order, so S_{j+3} (issued after
+// P_j V_j) never overwrites P_j before it is read, and the softmax of tile j
+// never waits for P_{j-1} V_{j-1}: only a rescale of O does.
 // The running maximum is moved only when a tile's maximum exceeds it by more
 // than 2^8 (weights stay below 256, exact in fp32 and safe in 16 bits); the
 // rescale of O in tensor memory is then rare.  The final division uses the
@@ -49,8 +56,10 @@ namespace pa {
 constexpr int kPrefillRows = 128;     // rows per CTA: M of every tensor-core product
 constexpr int kPrefillKT = 128;       // keys per tile: N of S, K of P V
 constexpr int kPrefillSoftmaxWarps = 8;
-constexpr int kPrefillThreads = (2 + kPrefillSoftmaxWarps) * 32;  // producer, MMA, softmax
-constexpr int kPrefillTmemCols = 512; // S buffers (2 x 128 columns) + O (D columns), power of two
+constexpr int kPrefillVWarp = 2 + kPrefillSoftmaxWarps;             // the V producer
+constexpr int kPrefillThreads = (3 + kPrefillSoftmaxWarps) * 32;  // K producer, MMA, softmax, V producer
+constexpr int kPrefillSBufs = 3;      // S / P buffers in tensor memory
+constexpr int kPrefillTmemCols = 512; // S / P buffers (3 x 128 columns) + O (D columns), power of two
 constexpr int kPrefillMaxSlots = 8;   // K / V ring slots
 constexpr float kPrefillRescaleLog2 = 8.f;
 
@@ -68,9 +77,9 @@ struct PrefillParams {
     int32_t B, Hq, Hkv, G, g_log2, bs, bs_log2, num_blocks, max_blocks;
     int32_t QT;          // new tokens per CTA (QT * G = kPrefillRows)
     int32_t br_log2;     // rows of one box = min(kPrefillKT, bs)
-    int32_t nslots;      // ring slots, even: K of tile j in slot 2j mod nslots, V in the next
+    int32_t nslots;      // ring slots, even: K of tile j in slot j mod (nslots/2), V of tile j in the second half
     int32_t num_qtiles;  // tiles of QT tokens the grid covers per request
-    uint32_t off_p, off_ring, slot_bytes;  // shared-memory layout (from the 1024-aligned base; Q at 0)
+    uint32_t off_ring, slot_bytes;  // shared-memory layout (from the 1024-aligned base; Q at 0)
 };
 static_assert(offsetof(PrefillParams, tmap_k) % 64 == 0 && offsetof(PrefillParams, tmap_v) % 64 == 0,
               "tensor maps must be 64-byte aligned");
@@ -83,24 +92,30 @@ __global__ void __launch_bounds__(kPrefillThreads, 1) paged_prefill_kernel(const
     constexpr int KS = D / 16;                         // k-steps of S over d
     constexpr int NDC = D / 64;                        // 64-wide d-blocks
     constexpr uint32_t kBlk = kPrefillRows * 128u;     // one 64-column block of a 128-row operand: 16 KB
-    constexpr uint32_t kPPart = kPrefillRows * KT * E; // one 16-bit part of P
     constexpr uint32_t kSlotBlk = KT * 128u;           // one d-block of a K / V slot
     constexpr bool kBf16 = std::is_same<T, __nv_bfloat16>::value;
     constexpr uint32_t kIdescPV = umma_idesc(kPrefillRows, D, false, true, kBf16);
-    constexpr uint32_t kColO = 2 * KT;                 // tensor-memory column of O
+    constexpr uint32_t kColO = kPrefillSBufs * KT;     // tensor-memory column of O
+    static_assert(kPrefillSBufs * KT + D <= kPrefillTmemCols, "tensor memory");
     extern __shared__ __align__(1024) unsigned char smem_raw[];
     unsigned char *smem = smem_raw;  // the plan leaves no room to realign: checked below
-    __shared__ uint64_t bars[2 * kPrefillMaxSlots + 16];
+    // mbarriers: full[], empty[] (ring), sfull[3], pfull[2], odone[2], qfull, fin, xchg[4][2]
+    constexpr int kOffSfull = 2 * kPrefillMaxSlots, kOffPfull = kOffSfull + kPrefillSBufs;
+    constexpr int kOffOdone = kOffPfull + 2, kOffQfull = kOffOdone + 2, kOffFin = kOffQfull + 1;
+    constexpr int kOffXchg = kOffFin + 1, kBars = kOffXchg + 8;
+    __shared__ uint64_t bars[kBars];
     __shared__ float red_s[2][2][kPrefillRows];  // [tile parity][column half][row]: row max / row sum
     __shared__ uint32_t tmem_base_s;
     __shared__ volatile int abort_s;
 
     const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
-    const int NS = p.nslots;
+    const int NH = p.nslots / 2;  // K slots 0 .. NH-1, V slots NH .. 2NH-1
     uint64_t *full = bars, *empty = bars + kPrefillMaxSlots;
-    uint64_t *sfull = bars + 2 * kPrefillMaxSlots, *sfree = sfull + 2;
-    uint64_t *pfull = sfree + 2, *odone = pfull + 1, *qfull = odone + 1, *fin = qfull + 1;
-    uint64_t *xchg = fin + 1;  // [lane quarter][parity]: the two softmax warps of the same rows
+    // sfull (one per S buffer), pfull and odone (one per tile parity): no
+    // barrier's phase can run two ahead of a thread that waits on it by parity
+    uint64_t *sfull = bars + kOffSfull, *pfull = bars + kOffPfull, *odone = bars + kOffOdone;
+    uint64_t *qfull = bars + kOffQfull, *fin = bars + kOffFin;
+    uint64_t *xchg = bars + kOffXchg;  // [lane quarter][parity]: the two softmax warps of the same rows
     volatile int *abort_flag = &abort_s;
 
     if (smem_u32(smem_raw) & 1023u) {  // the 128-byte swizzle needs 1024-byte aligned tiles
@@ -128,16 +143,15 @@ __global__ void __launch_bounds__(kPrefillThreads, 1) paged_prefill_kernel(const
     const int n16_last = (nk_last + 15) >> 4;      // its 16-key groups
 
     if (tid == 0) {
-        for (int s = 0; s < NS; ++s) {
+        for (int s = 0; s < 2 * NH; ++s) {
             mbar_init(&full[s], 1);
             mbar_init(&empty[s], 1);
         }
+        for (int i = 0; i < kPrefillSBufs; ++i) mbar_init(&sfull[i], 1);
         for (int i = 0; i < 2; ++i) {
-            mbar_init(&sfull[i], 1);
-            mbar_init(&sfree[i], kPrefillSoftmaxWarps);
+            mbar_init(&pfull[i], kPrefillSoftmaxWarps);
+            mbar_init(&odone[i], 1);
         }
-        mbar_init(pfull, kPrefillSoftmaxWarps);
-        mbar_init(odone, 1);
         mbar_init(qfull, kPrefillSoftmaxWarps);
         mbar_init(fin, 1);
         for (int i = 0; i < 8; ++i) mbar_init(&xchg[i], 2);
@@ -151,56 +165,55 @@ __global__ void __launch_bounds__(kPrefillThreads, 1) paged_prefill_kernel(const
     const uint32_t tmem = tmem_base_s;
     unsigned char *ring = smem + p.off_ring;
 
-    if (warp == 0) {
-        // ================= producer =================
+    if (warp == 0 || warp == kPrefillVWarp) {
+        // ================= producers: K (warp 0) and V =================
+        const int mat = warp == 0 ? 0 : 1;
+        const CUtensorMap *map = mat ? &p.tmap_v : &p.tmap_k;
+        const int base = mat * NH;  // this matrix's ring slots: base .. base + NH - 1
         const uint64_t policy = policy_evict_normal();  // K/V are read by every q-tile of the request
         const int32_t *table = p.block_tables + (size_t)b * p.max_blocks;
         const int br = 1 << p.br_log2;
         const uint32_t box_bytes = 128u << p.br_log2;
-        int slot = 0;
-        uint32_t phase = 0, issued = 0, issued_par = 0;
-        bool ok = true;
-        for (int j = 0; j < ntiles && ok; ++j) {
+        // physical block of this lane's box piece of tile j (-1: no piece, or a bad entry)
+        auto lookup = [&](int j) {
             const int k0 = j * KT;
-            const int nk = min(KT, kend - k0);
-            const int npc = (nk + br - 1) >> p.br_log2;  // box pieces holding visible keys
+            const int npc = (min(KT, kend - k0) + br - 1) >> p.br_log2;  // pieces holding visible keys
             int phys = -1;
-            uint32_t bytes = 0;
-            const int tp = k0 + lane * br;  // first key of this lane's piece
             if (lane < npc) {
-                phys = table[tp >> p.bs_log2];
+                phys = table[(k0 + lane * br) >> p.bs_log2];
                 if (phys < 0 || phys >= p.num_blocks) {
                     set_error(p.error, PA_DEVERR_BLOCK_ID);
                     phys = -1;
-                } else {
-                    bytes = NDC * box_bytes;
                 }
             }
+            return phys;
+        };
+        uint32_t issued = 0, issued_par = 0;
+        bool ok = true;
+        int phys = lookup(0);
+        for (int j = 0; j < ntiles; ++j) {
+            const int cur = phys;
+            if (j + 1 < ntiles) phys = lookup(j + 1);  // the next tile's entries load while this one waits
+            uint32_t bytes = cur >= 0 ? NDC * box_bytes : 0u;
 #pragma unroll
             for (int m = 16; m >= 1; m >>= 1) bytes += __shfl_xor_sync(0xffffffffu, bytes, m);
-            const int32_t row = phys * p.bs + (tp & (p.bs - 1));
-#pragma unroll
-            for (int mat = 0; mat < 2; ++mat) {  // K, then V
-                if (!mbar_wait(&empty[slot], phase ^ 1u, abort_flag)) {
-                    ok = false;
-                    break;
-                }
-                if (lane == 0) mbar_arrive_expect_tx(&full[slot], bytes);
-                __syncwarp();
-                if (phys >= 0) {
-                    unsigned char *dst = ring + (size_t)slot * p.slot_bytes + (size_t)lane * box_bytes;
-#pragma unroll
-                    for (int c = 0; c < NDC; ++c)
-                        tma_load_3d(dst + c * kSlotBlk, mat ? &p.tmap_v : &p.tmap_k, c * 64, row, g, &full[slot],
-                                    policy);
-                }
-                issued |= 1u << slot;
-                issued_par = (issued_par & ~(1u << slot)) | (phase << slot);
-                if (++slot == NS) {
-                    slot = 0;
-                    phase ^= 1u;
-                }
+            const int slot = base + j % NH;
+            const uint32_t par = (uint32_t)(j / NH) & 1u;
+            if (!mbar_wait(&empty[slot], par ^ 1u, abort_flag)) {
+                ok = false;
+                break;
             }
+            if (lane == 0) mbar_arrive_expect_tx(&full[slot], bytes);
+            __syncwarp();
+            if (cur >= 0) {
+                const int32_t row = cur * p.bs + ((j * KT + lane * br) & (p.bs - 1));
+                unsigned char *dst = ring + (size_t)slot * p.slot_bytes + (size_t)lane * box_bytes;
+#pragma unroll
+                for (int c = 0; c < NDC; ++c)
+                    tma_load_3d(dst + c * kSlotBlk, map, c * 64, row, g, &full[slot], policy);
+            }
+            issued |= 1u << slot;
+            issued_par = (issued_par & ~(1u << slot)) | (par << slot);
         }
         if (!ok) {
             *abort_flag = 1;
@@ -208,45 +221,47 @@ __global__ void __launch_bounds__(kPrefillThreads, 1) paged_prefill_kernel(const
         }
         // every copy issued lands before the CTA retires
         volatile int never = 0;
-        for (int st = 0; st < NS; ++st)
+        for (int st = base; st < base + NH; ++st)
             if (issued & (1u << st)) mbar_wait(&full[st], (issued_par >> st) & 1u, &never);
     } else if (warp == 1) {
         // ================= MMA issue (one lane) =================
         if (lane == 0) {
-            const uint32_t q_addr = smem_u32(smem), p_addr = smem_u32(smem + p.off_p), r_addr = smem_u32(ring);
+            const uint32_t q_addr = smem_u32(smem), r_addr = smem_u32(ring);
             bool ok = mbar_wait(qfull, 0u, abort_flag);
             bool issued_any = false;
             // O += P_i V_i for tile i (P high part, then low part)
             auto pv = [&](int i) {
                 if (!ok) return;
-                const int sv = (2 * i + 1) % NS;
-                const uint32_t par = (uint32_t)((2 * i + 1) / NS) & 1u;
-                if (!mbar_wait(pfull, (uint32_t)i & 1u, abort_flag) || !mbar_wait(&full[sv], par, abort_flag)) {
+                const int sv = NH + i % NH;
+                const uint32_t par = (uint32_t)(i / NH) & 1u;
+                if (!mbar_wait(&pfull[i & 1], (uint32_t)(i >> 1) & 1u, abort_flag) ||
+                    !mbar_wait(&full[sv], par, abort_flag)) {
                     ok = false;
                     return;
                 }
                 tc_fence_after();
                 const int n16 = i == ntiles - 1 ? n16_last : KT / 16;
                 const uint32_t vb = r_addr + (uint32_t)sv * p.slot_bytes;
+                // P_i: columns (i % 3) * KT + part * KT / 2 + key / 2 of tensor memory
                 for (int part = 0; part < 2; ++part) {
-                    const uint32_t pb = p_addr + (uint32_t)part * kPPart;
+                    const uint32_t pa = tmem + (uint32_t)(i % kPrefillSBufs) * KT + (uint32_t)part * (KT / 2);
                     for (int kk = 0; kk < n16; ++kk) {
-                        const uint64_t ad = umma_desc_sw128(pb + (kk >> 2) * kBlk + (kk & 3) * 32, 16, 1024);
                         const uint64_t bd = umma_desc_sw128(vb + kk * 2048, kSlotBlk, 1024);
-                        umma_f16(tmem + kColO, ad, bd, kIdescPV, (i > 0 || part > 0 || kk > 0) ? 1u : 0u);
+                        umma_f16_ts(tmem + kColO, pa + kk * 8, bd, kIdescPV, (i > 0 || part > 0 || kk > 0) ? 1u : 0u);
                     }
                 }
-                umma_commit(odone);
+                umma_commit(&odone[i & 1]);
                 umma_commit(&empty[sv]);
                 issued_any = true;
             };
-            for (int j = 0; j < ntiles && ok; ++j) {
-                const int sk = (2 * j) % NS;
-                const uint32_t par = (uint32_t)((2 * j) / NS) & 1u;
-                if (!mbar_wait(&full[sk], par, abort_flag) ||
-                    (j >= 2 && !mbar_wait(&sfree[j & 1], (uint32_t)((j >> 1) - 1) & 1u, abort_flag))) {
+            // S_j = Q K_j^T into buffer j % 3, which held P_{j-3}: issued after P_{j-3} V_{j-3}
+            auto s_issue = [&](int j) {
+                if (!ok) return;
+                const int sk = j % NH;
+                const uint32_t par = (uint32_t)(j / NH) & 1u;
+                if (!mbar_wait(&full[sk], par, abort_flag)) {
                     ok = false;
-                    break;
+                    return;
                 }
                 tc_fence_after();
                 const int N = j == ntiles - 1 ? n16_last * 16 : KT;
@@ -256,14 +271,17 @@ __global__ void __launch_bounds__(kPrefillThreads, 1) paged_prefill_kernel(const
                 for (int ks = 0; ks < KS; ++ks) {
                     const uint64_t ad = umma_desc_sw128(q_addr + (ks >> 2) * kBlk + (ks & 3) * 32, 16, 1024);
                     const uint64_t bd = umma_desc_sw128(kb + (ks >> 2) * kSlotBlk + (ks & 3) * 32, 16, 1024);
-                    umma_f16(tmem + (uint32_t)(j & 1) * KT, ad, bd, idesc, ks > 0 ? 1u : 0u);
+                    umma_f16(tmem + (uint32_t)(j % kPrefillSBufs) * KT, ad, bd, idesc, ks > 0 ? 1u : 0u);
                 }
-                umma_commit(&sfull[j & 1]);
+                umma_commit(&sfull[j % kPrefillSBufs]);
                 umma_commit(&empty[sk]);
                 issued_any = true;
-                if (j >= 1) pv(j - 1);
+            };
+            for (int j = 0; j < kPrefillSBufs && j < ntiles; ++j) s_issue(j);
+            for (int i = 0; i < ntiles && ok; ++i) {
+                pv(i);
+                if (i + kPrefillSBufs < ntiles) s_issue(i + kPrefillSBufs);
             }
-            if (ok) pv(ntiles - 1);
             if (!ok) {
                 *abort_flag = 1;
                 set_error(p.error, PA_DEVERR_TIMEOUT);
@@ -309,24 +327,32 @@ __global__ void __launch_bounds__(kPrefillThreads, 1) paged_prefill_kernel(const
             if (lane == 0) mbar_arrive(qfull);
         }
         const int pos_row = pos0 + (valid ? tok : ntok - 1);  // rows past the tokens mirror the last token
-        unsigned char *pst = smem + p.off_p + half * kBlk;    // this half's 64-key block of P
         const float qs = p.qscale;
         float m_used = -INFINITY, l = 0.f;
         bool ok = true;
+        // P V completions, confirmed per barrier in order: odone[i & 1] phase
+        // i >> 1 is P_i V_i, and P_{i+2} V_{i+2} cannot complete before the
+        // softmax of tile i+2 has run, so a parity wait never skips a phase
+        int od_next[2] = {0, 0};
+        auto od_wait = [&](int i) {
+            int &nx = od_next[i & 1];
+            for (; nx <= (i >> 1); ++nx)
+                if (!mbar_wait(&odone[i & 1], (uint32_t)nx & 1u, abort_flag)) return false;
+            tc_fence_after();
+            return true;
+        };
         for (int j = 0; j < ntiles; ++j) {
             const int k0 = j * KT;
-            if (!mbar_wait(&sfull[j & 1], (uint32_t)(j >> 1) & 1u, abort_flag)) {
+            const uint32_t sb = tl + (uint32_t)(j % kPrefillSBufs) * KT;  // S_j / P_j
+            if (!mbar_wait(&sfull[j % kPrefillSBufs], (uint32_t)(j / kPrefillSBufs) & 1u, abort_flag)) {
                 ok = false;
                 break;
             }
             tc_fence_after();
             float s[HC];
-            tmem_ld32(tl + (uint32_t)(j & 1) * KT + half * HC, s);
-            tmem_ld32(tl + (uint32_t)(j & 1) * KT + half * HC + 32, s + 32);
+            tmem_ld32(sb + half * HC, s);
+            tmem_ld32(sb + half * HC + 32, s + 32);
             tmem_wait_ld();
-            tc_fence_before();
-            __syncwarp();
-            if (lane == 0) mbar_arrive(&sfree[j & 1]);
             // keys past the row's position (or past the keys loaded) are out
             const bool diag = k0 + KT - 1 > pos0;
             const int lim = pos_row - k0 - half * HC;  // columns c <= lim are visible
@@ -342,7 +368,8 @@ __global__ void __launch_bounds__(kPrefillThreads, 1) paged_prefill_kernel(const
                 for (int c = 0; c < HC; ++c) m4[c & 3] = fmaxf(m4[c & 3], s[c]);
             }
             float mx = fmaxf(fmaxf(m4[0], m4[1]), fmaxf(m4[2], m4[3]));
-            // row maximum over both halves
+            // row maximum over both halves (after this exchange both threads
+            // of the row hold their S values, so P may overwrite S)
             red_s[j & 1][half][row] = mx;
             __syncwarp();
             if (lane == 0) mbar_arrive(&xb[j & 1]);
@@ -359,29 +386,14 @@ __global__ void __launch_bounds__(kPrefillThreads, 1) paged_prefill_kernel(const
                 m_used = mt;
             }
             const float nm = -m_used;
-            float l4[4] = {0.f, 0.f, 0.f, 0.f};
-            if (diag) {
-#pragma unroll
-                for (int c = 0; c < HC; ++c) {
-                    s[c] = c <= lim ? exp2_fast(fmaf(s[c], qs, nm)) : 0.f;
-                    l4[c & 3] += s[c];
-                }
-            } else {
-#pragma unroll
-                for (int c = 0; c < HC; ++c) {
-                    s[c] = exp2_fast(fmaf(s[c], qs, nm));
-                    l4[c & 3] += s[c];
-                }
-            }
-            l = l * alpha + ((l4[0] + l4[1]) + (l4[2] + l4[3]));
-            if (j >= 1) {
-                // P V of the previous tile is done: P's buffer is free and O is current
-                if (!mbar_wait(odone, (uint32_t)(j - 1) & 1u, abort_flag)) {
+            l *= alpha;
+            if (j >= 1 && __any_sync(0xffffffffu, move)) {
+                // rescale O: P_{j-1} V_{j-1} must be in it first
+                if (!od_wait(j - 1)) {
                     ok = false;
                     break;
                 }
-                tc_fence_after();
-                if (__any_sync(0xffffffffu, move)) {
+                {
 #pragma unroll
                     for (int c = 0; c < HD / 32; ++c) {
                         float o[32];
@@ -400,8 +412,8 @@ __global__ void __launch_bounds__(kPrefillThreads, 1) paged_prefill_kernel(const
                 // must stay 0) once their tensor-map fill has landed
                 const int z0 = L - k0, z1 = n16_last * 16;
                 if (z0 < z1) {
-                    const int sv = (2 * j + 1) % NS;
-                    if (!mbar_wait(&full[sv], (uint32_t)((2 * j + 1) / NS) & 1u, abort_flag)) {
+                    const int sv = NH + j % NH;
+                    if (!mbar_wait(&full[sv], (uint32_t)(j / NH) & 1u, abort_flag)) {
                         ok = false;
                         break;
                     }
@@ -413,23 +425,47 @@ __global__ void __launch_bounds__(kPrefillThreads, 1) paged_prefill_kernel(const
                     }
                 }
             }
-            // ---- P (high and low 16-bit parts), K-major with the 128-byte swizzle ----
+            // ---- weights and P over S_j: high parts in columns [0, KT/2), low parts
+            // in [KT/2, KT), two keys per column; two chunks of 32 keys, the
+            // first chunk's stores in flight while the second is computed ----
+            float l4[4] = {0.f, 0.f, 0.f, 0.f};
 #pragma unroll
-            for (int c8 = 0; c8 < HC / 8; ++c8) {
-                uint32_t hi[4], lo[4];
+            for (int ch = 0; ch < 2; ++ch) {
+                float *sc = s + ch * 32;
+                if (diag) {
 #pragma unroll
-                for (int i = 0; i < 4; ++i) Op::split_p(s[c8 * 8 + 2 * i], s[c8 * 8 + 2 * i + 1], hi[i], lo[i]);
-                const uint32_t off = row * 128 + ((c8 ^ (row & 7)) << 4);
-                *reinterpret_cast<uint4 *>(pst + off) = make_uint4(hi[0], hi[1], hi[2], hi[3]);
-                *reinterpret_cast<uint4 *>(pst + kPPart + off) = make_uint4(lo[0], lo[1], lo[2], lo[3]);
+                    for (int c = 0; c < 32; ++c) {
+                        sc[c] = ch * 32 + c <= lim ? exp2_fast(fmaf(sc[c], qs, nm)) : 0.f;
+                        l4[c & 3] += sc[c];
+                    }
+                } else {
+#pragma unroll
+                    for (int c = 0; c < 32; ++c) {
+                        sc[c] = exp2_fast(fmaf(sc[c], qs, nm));
+                        l4[c & 3] += sc[c];
+                    }
+                }
+                uint32_t hi[16], lo[16];
+#pragma unroll
+                for (int i = 0; i < 16; ++i) Op::split_p(sc[2 * i], sc[2 * i + 1], hi[i], lo[i]);
+                const uint32_t pb = sb + half * (HC / 2) + ch * 16;
+                tmem_st16u(pb, hi);
+                tmem_st16u(pb + KT / 2, lo);
             }
-            fence_async_smem();
+            l += (l4[0] + l4[1]) + (l4[2] + l4[3]);
+            // confirm P_{j-2} V_{j-2} (long done) before P_j is published: P_j V_j
+            // could otherwise complete and put odone[j & 1] two phases ahead
+            if (j >= 2 && !od_wait(j - 2)) {
+                ok = false;
+                break;
+            }
+            tmem_wait_st();
+            fence_async_smem();  // V rows zeroed above
             tc_fence_before();
             __syncwarp();
-            if (lane == 0) mbar_arrive(pfull);
+            if (lane == 0) mbar_arrive(&pfull[j & 1]);
         }
-        if (ok && mbar_wait(odone, (uint32_t)(ntiles - 1) & 1u, abort_flag)) {
-            tc_fence_after();
+        if (ok && od_wait(ntiles - 1)) {  // the last product: every earlier one is done too
             // row sum over both halves
             red_s[ntiles & 1][half][row] = l;
             __syncwarp();
