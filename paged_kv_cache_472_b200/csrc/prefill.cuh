@@ -242,13 +242,13 @@ __global__ void __launch_bounds__(kPrefillThreads, 1) paged_prefill_kernel(const
                 tc_fence_after();
                 const int n16 = i == ntiles - 1 ? n16_last : KT / 16;
                 const uint32_t vb = r_addr + (uint32_t)sv * p.slot_bytes;
-                // P_i: columns (i % 3) * KT + part * KT / 2 + key / 2 of tensor memory
-                for (int part = 0; part < 2; ++part) {
-                    const uint32_t pa = tmem + (uint32_t)(i % kPrefillSBufs) * KT + (uint32_t)part * (KT / 2);
-                    for (int kk = 0; kk < n16; ++kk) {
-                        const uint64_t bd = umma_desc_sw128(vb + kk * 2048, kSlotBlk, 1024);
-                        umma_f16_ts(tmem + kColO, pa + kk * 8, bd, kIdescPV, (i > 0 || part > 0 || kk > 0) ? 1u : 0u);
-                    }
+                // P_i in buffer i % 3: keys 16kk .. 16kk+15 in columns 16kk .. 16kk+7
+                // (high parts) and 16kk+8 .. 16kk+15 (low parts), two keys per column
+                const uint32_t pa = tmem + (uint32_t)(i % kPrefillSBufs) * KT;
+                for (int kk = 0; kk < n16; ++kk) {
+                    const uint64_t bd = umma_desc_sw128(vb + kk * 2048, kSlotBlk, 1024);
+                    umma_f16_ts(tmem + kColO, pa + kk * 16, bd, kIdescPV, (i > 0 || kk > 0) ? 1u : 0u);
+                    umma_f16_ts(tmem + kColO, pa + kk * 16 + 8, bd, kIdescPV, 1u);
                 }
                 umma_commit(&odone[i & 1]);
                 umma_commit(&empty[sv]);
@@ -343,7 +343,7 @@ __global__ void __launch_bounds__(kPrefillThreads, 1) paged_prefill_kernel(const
         };
         for (int j = 0; j < ntiles; ++j) {
             const int k0 = j * KT;
-            const uint32_t sb = tl + (uint32_t)(j % kPrefillSBufs) * KT;  // S_j / P_j
+            const uint32_t sb = tl + (uint32_t)(j % kPrefillSBufs) * KT;  // S_j, then P_j
             if (!mbar_wait(&sfull[j % kPrefillSBufs], (uint32_t)(j / kPrefillSBufs) & 1u, abort_flag)) {
                 ok = false;
                 break;
@@ -352,7 +352,6 @@ __global__ void __launch_bounds__(kPrefillThreads, 1) paged_prefill_kernel(const
             float s[HC];
             tmem_ld32(sb + half * HC, s);
             tmem_ld32(sb + half * HC + 32, s + 32);
-            tmem_wait_ld();
             // keys past the row's position (or past the keys loaded) are out
             const bool diag = k0 + KT - 1 > pos0;
             const int lim = pos_row - k0 - half * HC;  // columns c <= lim are visible
@@ -368,8 +367,7 @@ __global__ void __launch_bounds__(kPrefillThreads, 1) paged_prefill_kernel(const
                 for (int c = 0; c < HC; ++c) m4[c & 3] = fmaxf(m4[c & 3], s[c]);
             }
             float mx = fmaxf(fmaxf(m4[0], m4[1]), fmaxf(m4[2], m4[3]));
-            // row maximum over both halves (after this exchange both threads
-            // of the row hold their S values, so P may overwrite S)
+            // row maximum over both halves
             red_s[j & 1][half][row] = mx;
             __syncwarp();
             if (lane == 0) mbar_arrive(&xb[j & 1]);
@@ -398,7 +396,6 @@ __global__ void __launch_bounds__(kPrefillThreads, 1) paged_prefill_kernel(const
                     for (int c = 0; c < HD / 32; ++c) {
                         float o[32];
                         tmem_ld32(tl + kColO + half * HD + c * 32, o);
-                        tmem_wait_ld();
 #pragma unroll
                         for (int i = 0; i < 32; ++i) o[i] *= alpha;
                         tmem_st32(tl + kColO + half * HD + c * 32, o);
@@ -425,34 +422,38 @@ __global__ void __launch_bounds__(kPrefillThreads, 1) paged_prefill_kernel(const
                     }
                 }
             }
-            // ---- weights and P over S_j: high parts in columns [0, KT/2), low parts
-            // in [KT/2, KT), two keys per column; two chunks of 32 keys, the
-            // first chunk's stores in flight while the second is computed ----
-            float l4[4] = {0.f, 0.f, 0.f, 0.f};
+            // ---- weights and P over S_j, 16 keys at a time: the chunk's S
+            // columns are read back and its P parts written over them (high
+            // parts in the first 8 columns, low parts in the next 8), so no
+            // column is written before its S value is read.  A rolled loop
+            // keeps this warp's code (and the MMA warp's beside it) in the
+            // instruction cache. ----
+            float l4[2] = {0.f, 0.f};
+            {
+                const uint32_t hb = sb + half * HC;  // this half's 64 columns
+#pragma unroll 1
+                for (int c = 0; c < HC / 16; ++c) {
+                    float w[16];
+                    tmem_ld16(hb + c * 16, w);
+                    const int cl = lim - c * 16;
+                    float2 l2 = make_float2(0.f, 0.f);
+                    uint32_t pw[16];  // P high parts (words 0-7), low parts (words 8-15)
 #pragma unroll
-            for (int ch = 0; ch < 2; ++ch) {
-                float *sc = s + ch * 32;
-                if (diag) {
-#pragma unroll
-                    for (int c = 0; c < 32; ++c) {
-                        sc[c] = ch * 32 + c <= lim ? exp2_fast(fmaf(sc[c], qs, nm)) : 0.f;
-                        l4[c & 3] += sc[c];
+                    for (int i = 0; i < 8; ++i) {
+                        const float2 t = ffma2(make_float2(w[2 * i], w[2 * i + 1]), make_float2(qs, qs), make_float2(nm, nm));
+                        float2 e = make_float2(exp2_fast(t.x), exp2_fast(t.y));
+                        if (diag) {
+                            e.x = 2 * i <= cl ? e.x : 0.f;
+                            e.y = 2 * i + 1 <= cl ? e.y : 0.f;
+                        }
+                        l2 = fadd2(l2, e);
+                        Op::split_p(e.x, e.y, pw[i], pw[8 + i]);
                     }
-                } else {
-#pragma unroll
-                    for (int c = 0; c < 32; ++c) {
-                        sc[c] = exp2_fast(fmaf(sc[c], qs, nm));
-                        l4[c & 3] += sc[c];
-                    }
+                    l4[c & 1] += l2.x + l2.y;
+                    tmem_st16u(hb + c * 16, pw);
                 }
-                uint32_t hi[16], lo[16];
-#pragma unroll
-                for (int i = 0; i < 16; ++i) Op::split_p(sc[2 * i], sc[2 * i + 1], hi[i], lo[i]);
-                const uint32_t pb = sb + half * (HC / 2) + ch * 16;
-                tmem_st16u(pb, hi);
-                tmem_st16u(pb + KT / 2, lo);
             }
-            l += (l4[0] + l4[1]) + (l4[2] + l4[3]);
+            l += l4[0] + l4[1];
             // confirm P_{j-2} V_{j-2} (long done) before P_j is published: P_j V_j
             // could otherwise complete and put odone[j & 1] two phases ahead
             if (j >= 2 && !od_wait(j - 2)) {
@@ -479,7 +480,6 @@ __global__ void __launch_bounds__(kPrefillThreads, 1) paged_prefill_kernel(const
                 for (int c = 0; c < HD / 32; ++c) {
                     float o[32];
                     tmem_ld32(tl + kColO + half * HD + c * 32, o);
-                    tmem_wait_ld();
                     if (valid) {
 #pragma unroll
                         for (int i = 0; i < 4; ++i)
