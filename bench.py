@@ -86,9 +86,9 @@ def measured_tensor_peak():
 
 
 def profiled_traffic(workload: str):
-    """DRAM bytes per decode launch from the committed ncu summary, if it was
-    taken on the current kernel sources."""
-    path = os.path.join(ROOT, "profiles", "decode_traffic.json")
+    """DRAM bytes per launch of the workload's kernel from the committed ncu
+    summary, if it was taken on the current kernel sources."""
+    path = os.path.join(ROOT, "profiles", "dram_traffic.json")
     try:
         with open(path) as f:
             rec = json.load(f)
@@ -293,7 +293,8 @@ def run_prefill(args):
                        "flops_per_step": alg["flops"], "min_bytes_per_step": alg["bytes"],
                        "l2": f"{R} rotating input copies"},
             "roofline": {"bound": "tensor", "achieved": round(k_tflops, 2), "peak": peak, "unit": "TFLOP/s",
-                         "frac": round(k_tflops / peak, 4), "traffic": None, "kernel": "paged_prefill_kernel",
+                         "frac": round(k_tflops / peak, 4), "traffic": profiled_traffic(pc.name),
+                         "kernel": "paged_prefill_kernel",
                          "peak_kind": kind, "kernel_us": round(ms_kernel * 1e3, 3),
                          "engine": "tcgen05.mma, S and O in tensor memory, P split into two 16-bit parts"},
             "gpu_launches": 2 * K, "clocks": clk.summary()}
