@@ -487,6 +487,7 @@ struct CoreEngine {
     static constexpr int TPL = kSubTile / LPH;                   // tokens per softmax lane
     static constexpr int E = Elem<T>::kBytes;
     static constexpr bool kPaddedRows = false;
+    static constexpr bool kPairs = false;  // subtile_pair not provided
     static constexpr int kUnitsPerWarp = UPW;
     static constexpr int kCombFloats = HC * D + 8;
     static constexpr int kScratchFloats = 2 * kSubTile * HC;
@@ -724,14 +725,17 @@ struct CoreEngine {
 };
 
 // ===========================================================================
-// tensor-core engine (bf16 / fp16): tokens are the M dimension of every tile
+// tensor-core engine (bf16 / fp16): tokens are the M dimension of every tile.
+// PAIR: the instantiation for units whose subtiles are split between warps
+// (large head groups), which steps through two full subtiles at a time.
 // ===========================================================================
-template <typename T, int D, int UPW>
+template <typename T, int D, int UPW, bool PAIR = false>
 struct MmaEngine {
     using Op = Mma16<T>;
     static constexpr int KS = D / 16;  // k-steps of QK (over d) = m-tiles of PV (over d)
     static constexpr int E = 2;
     static constexpr bool kPaddedRows = true;
+    static constexpr bool kPairs = PAIR;  // subtile_pair: two full subtiles in one online-softmax step
     static constexpr int kUnitsPerWarp = UPW;
     static constexpr int kCombFloats = 4 * KS * 32 + 4 * 32;  // fragment-ordered o, then m, l
     static constexpr int kScratchFloats = 0;
@@ -870,6 +874,101 @@ struct MmaEngine {
             ldmatrix_x4_trans(a, va + chunk_off(mt * 2 + (v_col >> 3), vswz, p));
             Op::mma(u.o[mt], a, bh0, bh1);
             Op::mma(u.o[mt], a, bl0, bl1);
+        }
+    }
+
+    // Two full subtiles (sa, sb: 32 tokens, no row past the context) in one
+    // online-softmax step: both S^T products as four independent chains, one
+    // maximum / rescale / sum over the 32 tokens, then both O^T updates.  The
+    // result is that of two subtile() calls (one softmax step over a longer
+    // run of tokens), with twice the independent work between the waits.
+    __device__ __forceinline__ void subtile_pair(Unit &u, const unsigned char *tile_k, const unsigned char *tile_v,
+                                                 int sa, int sb, int g_local, const DecodeParams &p) const {
+        float s[2][4] = {}, t[2][4] = {};
+        const unsigned char *ka0 = row_ptr(tile_k, sa * kSubTile + a_tok, g_local, p);
+        const unsigned char *ka1 = row_ptr(tile_k, sb * kSubTile + a_tok, g_local, p);
+        const int swz = a_tok & 7;
+#pragma unroll
+        for (int ks = 0; ks < KS; ks += 2) {
+            uint32_t a0[4], b0[4], a1[4], b1[4];
+            ldmatrix_x4(a0, ka0 + chunk_off(ks * 2 + (a_col >> 3), swz, p));
+            ldmatrix_x4(a1, ka1 + chunk_off(ks * 2 + (a_col >> 3), swz, p));
+            ldmatrix_x4(b0, ka0 + chunk_off((ks + 1) * 2 + (a_col >> 3), swz, p));
+            ldmatrix_x4(b1, ka1 + chunk_off((ks + 1) * 2 + (a_col >> 3), swz, p));
+            Op::mma(s[0], a0, u.qb[ks][0], u.qb[ks][1]);
+            Op::mma(s[1], a1, u.qb[ks][0], u.qb[ks][1]);
+            Op::mma(t[0], b0, u.qb[ks + 1][0], u.qb[ks + 1][1]);
+            Op::mma(t[1], b1, u.qb[ks + 1][0], u.qb[ks + 1][1]);
+        }
+        float x[2][4];
+#pragma unroll
+        for (int k = 0; k < 2; ++k)
+#pragma unroll
+            for (int i = 0; i < 4; ++i) x[k][i] = (s[k][i] + t[k][i]) * qscale;
+        // head 2*t4 uses elements 0, 2 (tokens g4, g4 + 8); head 2*t4+1 uses 1, 3
+        float mx0 = fmaxf(fmaxf(x[0][0], x[0][2]), fmaxf(x[1][0], x[1][2]));
+        float mx1 = fmaxf(fmaxf(x[0][1], x[0][3]), fmaxf(x[1][1], x[1][3]));
+#pragma unroll
+        for (int m = 4; m < 32; m <<= 1) {
+            mx0 = fmaxf(mx0, __shfl_xor_sync(0xffffffffu, mx0, m));
+            mx1 = fmaxf(mx1, __shfl_xor_sync(0xffffffffu, mx1, m));
+        }
+        const float mn0 = fmaxf(u.m[0], mx0), mn1 = fmaxf(u.m[1], mx1);
+        const float al0 = exp2_fast(u.m[0] - mn0), al1 = exp2_fast(u.m[1] - mn1);
+        float pr[2][4];
+#pragma unroll
+        for (int k = 0; k < 2; ++k) {
+            pr[k][0] = exp2_fast(x[k][0] - mn0);
+            pr[k][1] = exp2_fast(x[k][1] - mn1);
+            pr[k][2] = exp2_fast(x[k][2] - mn0);
+            pr[k][3] = exp2_fast(x[k][3] - mn1);
+        }
+        float r0 = (pr[0][0] + pr[0][2]) + (pr[1][0] + pr[1][2]);
+        float r1 = (pr[0][1] + pr[0][3]) + (pr[1][1] + pr[1][3]);
+#pragma unroll
+        for (int m = 4; m < 32; m <<= 1) {
+            r0 += __shfl_xor_sync(0xffffffffu, r0, m);
+            r1 += __shfl_xor_sync(0xffffffffu, r1, m);
+        }
+        u.l[0] = u.l[0] * al0 + r0;
+        u.l[1] = u.l[1] * al1 + r1;
+        u.m[0] = mn0;
+        u.m[1] = mn1;
+        // P^T fragments (k = token, n = head), high and low 16-bit parts, per subtile
+        uint32_t bh[2][2], bl[2][2];
+#pragma unroll
+        for (int k = 0; k < 2; ++k) {
+            const uint32_t ph0 = Op::pack_p(pr[k][0], pr[k][1]), ph1 = Op::pack_p(pr[k][2], pr[k][3]);
+            const float2 h0 = Op::unpack(ph0), h1 = Op::unpack(ph1);
+            const uint32_t pl0 = Op::pack_p(pr[k][0] - h0.x, pr[k][1] - h0.y);
+            const uint32_t pl1 = Op::pack_p(pr[k][2] - h1.x, pr[k][3] - h1.y);
+            bh[k][0] = movmatrix_trans(ph0);
+            bh[k][1] = movmatrix_trans(ph1);
+            bl[k][0] = movmatrix_trans(pl0);
+            bl[k][1] = movmatrix_trans(pl1);
+        }
+        if (al0 != 1.f || al1 != 1.f) {
+#pragma unroll
+            for (int mt = 0; mt < KS; ++mt) {
+                u.o[mt][0] *= al0;
+                u.o[mt][1] *= al1;
+                u.o[mt][2] *= al0;
+                u.o[mt][3] *= al1;
+            }
+        }
+        // ---- O^T[d x heads] += V^T P^T over both subtiles ----
+        const unsigned char *va0 = row_ptr(tile_v, sa * kSubTile + v_tok, g_local, p);
+        const unsigned char *va1 = row_ptr(tile_v, sb * kSubTile + v_tok, g_local, p);
+        const int vswz = v_tok & 7;
+#pragma unroll
+        for (int mt = 0; mt < KS; ++mt) {
+            uint32_t a0[4], a1[4];
+            ldmatrix_x4_trans(a0, va0 + chunk_off(mt * 2 + (v_col >> 3), vswz, p));
+            ldmatrix_x4_trans(a1, va1 + chunk_off(mt * 2 + (v_col >> 3), vswz, p));
+            Op::mma(u.o[mt], a0, bh[0][0], bh[0][1]);
+            Op::mma(u.o[mt], a1, bh[1][0], bh[1][1]);
+            Op::mma(u.o[mt], a0, bl[0][0], bl[0][1]);
+            Op::mma(u.o[mt], a1, bl[1][0], bl[1][1]);
         }
     }
 
@@ -1882,7 +1981,19 @@ __global__ void __launch_bounds__(kDecodeThreads, 1) paged_decode_kernel(const _
                 unsigned char *kst = stage_base + (size_t)stage * 2 * p.half_bytes;
                 unsigned char *vst = kst + p.half_bytes;
                 const int ntok = min(p.ST, s.L - t * p.ST);
-                for (int st = split; st * kSubTile < ntok; st += tsplit) {
+                int st = split;
+                if constexpr (Engine::kPairs) {
+                    // two full subtiles per step where a unit's subtiles are split
+                    // between warps (large head groups: the MMA chain is the bound),
+                    // away from the tile holding the appended token
+                    if (t != patch_tile)
+                        for (; (st + tsplit + 1) * kSubTile <= ntok; st += 2 * tsplit) {
+#pragma unroll
+                            for (int k = 0; k < UPW; ++k)
+                                eng.subtile_pair(unit[k], kst, vst, st, st + tsplit, u_g[k], p);
+                        }
+                }
+                for (; st * kSubTile < ntok; st += tsplit) {
                     const int nvalid = min(kSubTile, ntok - st * kSubTile);
                     if (t == patch_tile && st == patch_tok / kSubTile) {
 #pragma unroll

@@ -82,17 +82,19 @@ KernelFn pick_core(int hc, int upw) {
 }
 
 template <typename T, int D>
-KernelFn pick_mma(int upw) {
+KernelFn pick_mma(int upw, int ts) {
+    if (upw == 1 && ts > 1) return pa::paged_decode_kernel<T, D, pa::MmaEngine<T, D, 1, true>>;
     if (upw == 1) return pa::paged_decode_kernel<T, D, pa::MmaEngine<T, D, 1>>;
     if (upw == 2) return pa::paged_decode_kernel<T, D, pa::MmaEngine<T, D, 2>>;
     return nullptr;
 }
 
-KernelFn pick_kernel(int dtype, int D, int hc, int upw) {
+KernelFn pick_kernel(int dtype, int D, int hc, int upw, int ts) {
     if (dtype == PA_DTYPE_BF16)
-        return D == 64 ? pick_mma<__nv_bfloat16, 64>(upw) : (D == 128 ? pick_mma<__nv_bfloat16, 128>(upw) : nullptr);
+        return D == 64 ? pick_mma<__nv_bfloat16, 64>(upw, ts)
+                       : (D == 128 ? pick_mma<__nv_bfloat16, 128>(upw, ts) : nullptr);
     if (dtype == PA_DTYPE_F16)
-        return D == 64 ? pick_mma<__half, 64>(upw) : (D == 128 ? pick_mma<__half, 128>(upw) : nullptr);
+        return D == 64 ? pick_mma<__half, 64>(upw, ts) : (D == 128 ? pick_mma<__half, 128>(upw, ts) : nullptr);
     return D == 64 ? pick_core<64>(hc, upw) : (D == 128 ? pick_core<128>(hc, upw) : nullptr);
 }
 
@@ -286,7 +288,7 @@ pa_status launch_decode(const void *q, const void *k_cache, const void *v_cache,
     const int HC = plan->heads_per_unit, UPW = plan->units_per_warp, TS = plan->warps_per_unit;
     const int G = s->Hq / s->Hkv;
     const int e = elem_bytes(s->dtype);
-    KernelFn fn = pick_kernel(s->dtype, s->D, HC, UPW);
+    KernelFn fn = pick_kernel(s->dtype, s->D, HC, UPW, TS);
     if (!fn) return fail(PA_ERR_INVALID_ARG, "plan names no kernel variant");
     const int HG = plan->head_group;
     const int NHvr = HG * G;
