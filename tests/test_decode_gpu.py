@@ -23,7 +23,7 @@ _REF = {}
 
 
 def oracle_out(orc, case):
-    key = (case.name, case.seed)
+    key = (case.name, case.seed, case.scale)
     if key not in _REF:
         _REF[key] = orc.decode(case)
     return _REF[key]
@@ -217,6 +217,14 @@ def test_fp16_workload_shape(orc):
     case = synth.build_case("qwen3-0.6b-fp16", dtype="f16", Hq=16, Hkv=8, D=128, block_size=16,
                             context_lens=lens, seed=2002)
     check_full(orc, case, 0)
+
+
+@pytest.mark.parametrize("scale", [-0.2, 0.0, 0.5])
+@pytest.mark.parametrize("cid,batch", [(2, 6), (4, 2)])
+def test_any_scale(orc, scale, cid, batch):
+    """Negative, zero and large scales (the balanced split, with the merge)."""
+    case = dataclasses.replace(synth.make_config(cid, batch=batch), scale=scale)
+    check_full(orc, case, 0, f"{case.name} scale {scale}")
 
 
 @pytest.mark.parametrize("cid,batch", [(2, None), (3, 32), (5, 48), (1, None)])

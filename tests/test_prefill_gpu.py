@@ -2,6 +2,8 @@
 oracle on the same seeded inputs: the new tokens' K/V are written with
 pa_kv_append (one row per new token), then every new token attends causally
 to its request's positions up to its own."""
+import dataclasses
+
 import numpy as np
 import pytest
 import torch
@@ -98,6 +100,17 @@ def test_prefill_edge_shapes(orc, name, dtype, Hq, Hkv, D, bs, lens, new):
     pc = synth.build_prefill_case(name, dtype=dtype, Hq=Hq, Hkv=Hkv, D=D, block_size=bs, context_lens=lens,
                                   new_tokens=new, seed=sum(lens) + 7, pool="factor", pool_factor=1.5)
     check(orc, pc, name)
+
+
+@pytest.mark.parametrize("scale", [-0.2, 0.0, 0.5])
+def test_prefill_any_scale(orc, scale):
+    """A negative scale (the kernel feeds q negated and uses |scale|), zero
+    (uniform weights over each row's visible keys) and a large one (peaked
+    rows, where the low part of each weight matters)."""
+    base = synth.build_prefill_case("scale", dtype="bf16", Hq=16, Hkv=4, D=128, block_size=16,
+                                    context_lens=[300, 40], new_tokens=[150, 40], seed=11, pool="factor",
+                                    pool_factor=1.5)
+    check(orc, dataclasses.replace(base, scale=scale, name=f"scale {scale}"), f"scale {scale}")
 
 
 def test_prefill_one_new_token_matches_decode(orc):
