@@ -150,11 +150,6 @@ __device__ __forceinline__ uint64_t policy_evict_first() {
     return p;
 }
 
-// Named barrier among `nthreads` threads (id 0 is __syncthreads).
-__device__ __forceinline__ void named_barrier(uint32_t id, uint32_t nthreads) {
-    asm volatile("bar.sync %0, %1;" ::"r"(id), "r"(nthreads) : "memory");
-}
-
 // Packed fp32x2 fused multiply-add (sm_100): d = a * b + c, lane-wise.
 __device__ __forceinline__ float2 ffma2(float2 a, float2 b, float2 c) {
     uint64_t d;
@@ -178,14 +173,6 @@ __device__ __forceinline__ float2 fadd2(float2 a, float2 b) {
     const uint64_t ua = *reinterpret_cast<const uint64_t *>(&a);
     const uint64_t ub = *reinterpret_cast<const uint64_t *>(&b);
     asm("add.rn.f32x2 %0, %1, %2;" : "=l"(d) : "l"(ua), "l"(ub));
-    return *reinterpret_cast<float2 *>(&d);
-}
-
-__device__ __forceinline__ float2 fsub2(float2 a, float2 b) {
-    uint64_t d;
-    const uint64_t ua = *reinterpret_cast<const uint64_t *>(&a);
-    const uint64_t ub = *reinterpret_cast<const uint64_t *>(&b);
-    asm("sub.rn.f32x2 %0, %1, %2;" : "=l"(d) : "l"(ua), "l"(ub));
     return *reinterpret_cast<float2 *>(&d);
 }
 
@@ -400,18 +387,6 @@ __device__ __forceinline__ void umma_f16_ts(uint32_t d_tmem, uint32_t a_tmem, ui
         : "memory");
 }
 
-// 32 consecutive 32-bit TMEM columns of this thread's lane, from raw words.
-__device__ __forceinline__ void tmem_st32u(uint32_t taddr, const uint32_t *v) {
-    asm volatile(
-        "tcgen05.st.sync.aligned.32x32b.x32.b32 [%0], {%1,%2,%3,%4,%5,%6,%7,%8,%9,%10,%11,%12,%13,%14,%15,%16,"
-        "%17,%18,%19,%20,%21,%22,%23,%24,%25,%26,%27,%28,%29,%30,%31,%32};" ::"r"(taddr),
-        "r"(v[0]), "r"(v[1]), "r"(v[2]), "r"(v[3]), "r"(v[4]), "r"(v[5]), "r"(v[6]), "r"(v[7]), "r"(v[8]),
-        "r"(v[9]), "r"(v[10]), "r"(v[11]), "r"(v[12]), "r"(v[13]), "r"(v[14]), "r"(v[15]), "r"(v[16]),
-        "r"(v[17]), "r"(v[18]), "r"(v[19]), "r"(v[20]), "r"(v[21]), "r"(v[22]), "r"(v[23]), "r"(v[24]),
-        "r"(v[25]), "r"(v[26]), "r"(v[27]), "r"(v[28]), "r"(v[29]), "r"(v[30]), "r"(v[31])
-        : "memory");
-}
-
 // 16 consecutive 32-bit TMEM columns of this thread's lane, from raw words.
 __device__ __forceinline__ void tmem_st16u(uint32_t taddr, const uint32_t *v) {
     asm volatile(
@@ -420,13 +395,6 @@ __device__ __forceinline__ void tmem_st16u(uint32_t taddr, const uint32_t *v) {
         "r"(v[0]), "r"(v[1]), "r"(v[2]), "r"(v[3]), "r"(v[4]), "r"(v[5]), "r"(v[6]), "r"(v[7]), "r"(v[8]),
         "r"(v[9]), "r"(v[10]), "r"(v[11]), "r"(v[12]), "r"(v[13]), "r"(v[14]), "r"(v[15])
         : "memory");
-}
-
-// 8 consecutive 32-bit TMEM columns of this thread's lane, from raw words.
-__device__ __forceinline__ void tmem_st8u(uint32_t taddr, const uint32_t *v) {
-    asm volatile("tcgen05.st.sync.aligned.32x32b.x8.b32 [%0], {%1,%2,%3,%4,%5,%6,%7,%8};" ::"r"(taddr), "r"(v[0]),
-                 "r"(v[1]), "r"(v[2]), "r"(v[3]), "r"(v[4]), "r"(v[5]), "r"(v[6]), "r"(v[7])
-                 : "memory");
 }
 
 // One arrival on `bar` once every tcgen05.mma this thread issued so far has completed.
@@ -455,19 +423,6 @@ __device__ __forceinline__ void tmem_ld16(uint32_t taddr, float (&v)[16]) {
         : "memory");
 #pragma unroll
     for (int i = 0; i < 16; ++i) v[i] = __uint_as_float(r[i]);
-}
-
-__device__ __forceinline__ void tmem_st16(uint32_t taddr, const float (&v)[16]) {
-    asm volatile(
-        "tcgen05.st.sync.aligned.32x32b.x16.b32 [%0], {%1,%2,%3,%4,%5,%6,%7,%8,%9,%10,%11,%12,%13,%14,%15,%16};" ::"r"(
-            taddr),
-        "r"(__float_as_uint(v[0])), "r"(__float_as_uint(v[1])), "r"(__float_as_uint(v[2])),
-        "r"(__float_as_uint(v[3])), "r"(__float_as_uint(v[4])), "r"(__float_as_uint(v[5])),
-        "r"(__float_as_uint(v[6])), "r"(__float_as_uint(v[7])), "r"(__float_as_uint(v[8])),
-        "r"(__float_as_uint(v[9])), "r"(__float_as_uint(v[10])), "r"(__float_as_uint(v[11])),
-        "r"(__float_as_uint(v[12])), "r"(__float_as_uint(v[13])), "r"(__float_as_uint(v[14])),
-        "r"(__float_as_uint(v[15]))
-        : "memory");
 }
 
 // 32 consecutive 32-bit TMEM columns of this thread's lane, waited for in the
