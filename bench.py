@@ -16,6 +16,13 @@ Under torchrun each rank runs its own batch (weak scaling, no collective on
 the data path).  The end-to-end leg stages each step's inputs in one pinned
 host buffer (one copy in) and reads the output back (one copy out) around the
 same C call.
+
+  python bench.py --prefill 1|2 [--steps K] [--warmup W]
+
+times the chunked prefill step instead (pa_kv_append of the new tokens, then
+pa_prefill): value = algorithmic causal TFLOP/s, roofline against the
+measured bf16 tensor peak, end-to-end leg with the step's inputs copied from
+pinned host memory and the output copied back every step.
 """
 from __future__ import annotations
 
@@ -280,6 +287,34 @@ def run_prefill(args):
     e1.record(stream)
     torch.cuda.synchronize()
     ms_kernel = e0.elapsed_time(e1) / K
+    # end to end: every step copies its inputs (q, the new tokens' K/V and
+    # slots, tables, lengths, row offsets) from pinned host memory and the
+    # output back; the KV pool is resident state
+    host = {k: copies[0][k].cpu().pin_memory() for k in ("q", "kn", "vn", "sm", "bt", "cl", "qs")}
+    host_out = torch.empty(copies[0]["out"].shape, dtype=copies[0]["out"].dtype).pin_memory()
+
+    def e2e_step(i):
+        c = copies[i % R]
+        for k, t in host.items():
+            c[k].copy_(t, non_blocking=True)
+        rc = step(i)
+        host_out.copy_(c["out"], non_blocking=True)
+        return rc
+
+    for i in range(3):
+        if e2e_step(i):
+            raise RuntimeError(pa.pa_last_error_message())
+    torch.cuda.synchronize()
+    KE = max(1, min(K, args.e2e_steps))
+    torch.cuda._sleep(20_000_000)
+    e0.record(stream)
+    for i in range(KE):
+        e2e_step(i)
+    e1.record(stream)
+    torch.cuda.synchronize()
+    ms_e2e = e0.elapsed_time(e1) / KE
+    h2d = sum(t.numel() * t.element_size() for t in host.values())
+    d2h = host_out.numel() * host_out.element_size()
     if int(err.item()):
         raise RuntimeError(f"device error word {int(err.item()):#x}")
     peak, kind = measured_tensor_peak()
@@ -297,6 +332,8 @@ def run_prefill(args):
                          "kernel": "paged_prefill_kernel",
                          "peak_kind": kind, "kernel_us": round(ms_kernel * 1e3, 3),
                          "engine": "tcgen05.mma, S and O in tensor memory, P split into two 16-bit parts"},
+            "e2e": {"value": round(alg["flops"] / (ms_e2e * 1e-3) / 1e12, 2), "unit": "TFLOP/s",
+                    "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h, "us_per_step": round(ms_e2e * 1e3, 3)},
             "gpu_launches": 2 * K, "clocks": clk.summary()}
     if not args.no_cpu_baseline:
         import oracle
