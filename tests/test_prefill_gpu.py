@@ -92,6 +92,8 @@ EDGE = [
     ("g2_bs64", "bf16", 8, 4, 64, 64, [257, 63, 64], [200, 63, 1]),
     ("fp16", "f16", 16, 8, 128, 16, [500, 33], [120, 33]),
     ("ragged_tail_tiles", "bf16", 8, 2, 128, 32, [65, 129, 191], [65, 65, 66]),
+    ("g64_bs128", "bf16", 64, 1, 64, 128, [700, 129, 5], [50, 129, 5]),
+    ("g128_one_token_tiles", "f16", 128, 1, 128, 16, [300, 40], [9, 40]),
 ]
 
 
