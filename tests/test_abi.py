@@ -194,3 +194,17 @@ def test_prefill_plan_shapes_and_rejections():
     with pytest.raises(pa.PagedAttnError) as ei:
         pa.pa_prefill_plan(s, 256 * 16 + 1)            # more new tokens than a table row holds
     assert ei.value.status == pa.PA_ERR_INVALID_ARG
+
+
+@pytest.mark.parametrize("D", [64, 128])
+@pytest.mark.parametrize("dtype", [pa.DTYPE_BF16, pa.DTYPE_F16])
+def test_prefill_plan_budget_over_supported_shapes(D, dtype):
+    """Every supported shape gets a plan that fits the 227 KB shared-memory limit
+    with at least one K and one V slot, and tiles of 128 rows."""
+    for G in (1, 2, 4, 8, 16, 32, 64, 128):
+        for bs in (16, 32, 64, 128, 256):
+            s = pa.Shape(3, G * 2, 2, D, bs, 64, 16, dtype)
+            plan = pa.pa_prefill_plan(s, 100)
+            assert plan.q_tile * G == 128 and plan.kv_tile == 128
+            assert 2 <= 2 * plan.stages and plan.smem_bytes + 3072 <= 232448
+            assert plan.num_qtiles == -(-100 // plan.q_tile)
