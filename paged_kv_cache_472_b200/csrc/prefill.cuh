@@ -425,14 +425,13 @@ __global__ void __launch_bounds__(kPrefillThreads, 1) paged_prefill_kernel(const
             // ---- weights and P over S_j, 16 keys at a time: the chunk's S
             // columns are read back and its P parts written over them (high
             // parts in the first 8 columns, low parts in the next 8), so no
-            // column is written before its S value is read.  A rolled loop
-            // keeps this warp's code (and the MMA warp's beside it) in the
-            // instruction cache. ----
+            // column is written before its S value is read (rolled loops:
+            // small code for the warps that share a scheduler). ----
             float l4[2] = {0.f, 0.f};
             {
                 const uint32_t hb = sb + half * HC;  // this half's 64 columns
-#pragma unroll 1
-                for (int c = 0; c < HC / 16; ++c) {
+                // one chunk; the causal mask only on tiles that reach the diagonal
+                auto chunk = [&](int c, auto masked) {
                     float w[16];
                     tmem_ld16(hb + c * 16, w);
                     const int cl = lim - c * 16;
@@ -442,7 +441,7 @@ __global__ void __launch_bounds__(kPrefillThreads, 1) paged_prefill_kernel(const
                     for (int i = 0; i < 8; ++i) {
                         const float2 t = ffma2(make_float2(w[2 * i], w[2 * i + 1]), make_float2(qs, qs), make_float2(nm, nm));
                         float2 e = make_float2(exp2_fast(t.x), exp2_fast(t.y));
-                        if (diag) {
+                        if constexpr (decltype(masked)::value) {
                             e.x = 2 * i <= cl ? e.x : 0.f;
                             e.y = 2 * i + 1 <= cl ? e.y : 0.f;
                         }
@@ -451,6 +450,13 @@ __global__ void __launch_bounds__(kPrefillThreads, 1) paged_prefill_kernel(const
                     }
                     l4[c & 1] += l2.x + l2.y;
                     tmem_st16u(hb + c * 16, pw);
+                };
+                if (diag) {
+#pragma unroll 1
+                    for (int c = 0; c < HC / 16; ++c) chunk(c, std::true_type{});
+                } else {
+#pragma unroll 1
+                    for (int c = 0; c < HC / 16; ++c) chunk(c, std::false_type{});
                 }
             }
             l += l4[0] + l4[1];
