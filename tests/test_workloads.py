@@ -95,3 +95,35 @@ def test_prefill_config_structure(pid):
     assert len(set(pc.slot_mapping.tolist())) == pc.T          # distinct slots
     again = synth.make_prefill_config(pid, values=False)
     assert np.array_equal(again.context_lens, pc.context_lens) and np.array_equal(again.slot_mapping, pc.slot_mapping)
+
+
+def test_prefill_algorithmic_counts_by_brute_force():
+    """The prefill metric's flops and bytes, recounted pair by pair on a small case."""
+    pc = synth.build_prefill_case("count", dtype="bf16", Hq=8, Hkv=2, D=64, block_size=16,
+                                  context_lens=[40, 7, 100], new_tokens=[40, 3, 17], seed=5, values=False,
+                                  pool="factor", pool_factor=1.5)
+    pairs = 0
+    for b in range(pc.B):
+        L, n = int(pc.context_lens[b]), int(pc.query_start[b + 1] - pc.query_start[b])
+        for j in range(n):
+            pos = L - n + j
+            pairs += sum(1 for t in range(L) if t <= pos)
+    alg = synth.prefill_algorithmic(pc)
+    assert alg["flops"] == 4 * pairs * pc.Hq * pc.D
+    assert alg["bytes"] == int(sum(pc.context_lens)) * pc.Hkv * pc.D * 2 * 2 + 2 * pc.T * pc.Hq * pc.D * 2
+
+
+@pytest.mark.parametrize("cid", [1, 2, 3, 4, 5])
+def test_decode_algorithmic_bytes_by_definition(cid):
+    """The decode metric's bytes recounted from the lengths: K and V of every
+    position each request reads, q in and out, one table entry per block used
+    and one length per request."""
+    case = synth.make_config(cid, values=False)
+    e = {"f32": 4, "bf16": 2, "f16": 2}[case.dtype]
+    L = [int(x) for x in case.context_lens]
+    kv = sum(l * case.Hkv * case.D * e * 2 for l in L)
+    qo = 2 * case.B * case.Hq * case.D * e
+    tables = 4 * sum(-(-l // case.block_size) for l in L) + 4 * case.B
+    a = synth.algorithmic_bytes(case)
+    assert a["kv"] == kv and a["q_out"] == qo and a["tables"] == tables
+    assert a["decode_total"] == kv + qo + tables
