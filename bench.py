@@ -1,9 +1,13 @@
 """Benchmark: one decode step = one pa_kv_append_decode launch (append + decode) over one batch.
 
-Default workload: the Qwen3-0.6B-shaped decode batch (B=32, Hq=16, Hkv=8,
-D=128, block_size=16, context lengths ~ U[128, 2048], bf16, shuffled pool).
-Metric: paged-decode attention HBM GB/s (algorithmic bytes of the step /
-device time of the step) and us per decode step.
+Default workload: the Qwen3-8B-shaped heavy mixed batch (B=256, Hq=32, Hkv=8,
+D=128, block_size=16, log-normal context lengths with median 1024 clipped to
+[16, 16384], the first full blocks of every 8 requests shared, bf16): the
+largest of the decode batches.  Metric: paged-decode attention HBM GB/s
+(algorithmic bytes of the decode / device time of the step) and us per
+decode step.  The algorithmic bytes count every K/V block once (a prefix
+block several tables name is read once), plus q, out, block-table entries
+and lengths; the append's bytes are reported beside them, not in them.
 
   python bench.py [--gpus N] [--steps K] [--warmup W] [--config 1..5] [--impl reference]
 
@@ -11,11 +15,17 @@ Timing: inputs resident in HBM; R copies of the whole step's inputs are used
 in rotation so that the working set of consecutive steps exceeds the L2
 cache; the K timed steps are bracketed by a barrier and a device synchronise
 and measured with CUDA events on the launching stream (max over ranks).  The
-decode kernel's own duration is taken with events around every launch.
-Under torchrun each rank runs its own batch (weak scaling, no collective on
-the data path).  The end-to-end leg stages each step's inputs in one pinned
-host buffer (one copy in) and reads the output back (one copy out) around the
-same C call.
+K-step region is timed several times, so that the timed kernels span at
+least --min-timed-ms in total and the clock samples see them; the median
+region is reported.  The decode kernel's own duration comes from
+back-to-back launches timed the same way.  The other decode batches
+(Qwen3-0.6B, Llama-3.2-1B, long-context MQA) are timed in regions of their
+own and reported under "workloads".  A further leg times the step behind a
+~100 MB copy kernel on the same stream (the decode's predecessor is then not
+another decode).  Under torchrun each rank runs its own batch (weak scaling,
+no collective on the data path).  The end-to-end leg stages each step's
+inputs in one pinned host buffer (one copy in) and reads the output back
+(one copy out) around the same C call.
 
   python bench.py --prefill 1|2 [--steps K] [--warmup W]
 
@@ -49,12 +59,16 @@ def parse():
     ap.add_argument("--gpus", type=int, default=1)
     ap.add_argument("--steps", type=int, default=4000)
     ap.add_argument("--warmup", type=int, default=50)
-    ap.add_argument("--config", type=int, default=2)
+    ap.add_argument("--config", type=int, default=5)
     ap.add_argument("--partition", type=int, default=-1, help="-1: the workload's own (0 = balanced)")
     ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--cpu-seconds", type=float, default=10.0)
     ap.add_argument("--e2e-steps", type=int, default=200)
+    ap.add_argument("--min-timed-ms", type=float, default=250.0,
+                    help="repeat the K-step region until the timed kernels span this long in total")
+    ap.add_argument("--extra", default="2,3,4",
+                    help="other decode workloads timed in regions of their own (comma list; '' = none)")
     ap.add_argument("--prefill", type=int, default=0,
                     help="time the chunked prefill step of prefill workload N (1, 2) instead of the decode step")
     ap.add_argument("--dynamic-share", type=int, default=-1,
@@ -117,6 +131,9 @@ class ClockSampler:
     def __init__(self, index: int, period_s: float = 0.01):
         self.samples, self.reasons, self.ok = [], 0, False
         self.period, self.stop_ev = period_s, threading.Event()
+        self.max_mhz = None
+        if index < 0:   # sampling off
+            return
         try:
             import pynvml
             pynvml.nvmlInit()
@@ -179,24 +196,51 @@ def job_throughput_gbs(step_bytes: int, world: int, ms_step: float) -> float:
 
 # ---------------------------------------------------------------------------
 def cpu_baseline(case, seconds: float):
-    """The float64 oracle as it stands (append + decode of the whole batch),
-    repeated for about `seconds` on the host cores."""
+    """The float64 oracle as it stands (append + decode), on the host cores.
+
+    All cores: whole steps of the batch, repeated for about `seconds`; the
+    median of three such runs is the value.  One core: the same oracle with
+    one thread on a sample of the batch (every eighth request; the others
+    get length 0 and cost nothing), median of three runs.  GB/s counts the
+    same algorithmic bytes as the GPU line (for the sample: its own)."""
     import oracle
     from synth import algorithmic_bytes
     orc = oracle.default()
-    nbytes = algorithmic_bytes(case)["step_total"]
-    steps, t0 = 0, time.perf_counter()
-    while True:
-        kc, vc = orc.kv_append(case)
-        orc.decode(case, kc, vc)
-        steps += 1
-        el = time.perf_counter() - t0
-        if el >= seconds:
-            break
-    cores = orc.max_threads()
-    return {"value": nbytes * steps / el / 1e9, "unit": "GB/s", "cores": cores, "kind": "oracle",
-            "sample": f"{steps} full steps (append + decode of all {case.B} requests) of {case.name} in {el:.1f} s",
-            "ms_per_step": el / steps * 1e3}
+    nbytes = algorithmic_bytes(case)["decode_unique"]
+    runs, steps_all = [], 0
+    for _ in range(3):
+        steps, t0 = 0, time.perf_counter()
+        while True:
+            kc, vc = orc.kv_append(case)
+            orc.decode(case, kc, vc)
+            steps += 1
+            el = time.perf_counter() - t0
+            if el >= seconds / 3:
+                break
+        runs.append(el / steps)
+        steps_all += steps
+    sec_all = statistics.median(runs)
+    # one core, every eighth request
+    lens = case.context_lens.copy()
+    keep = np.zeros(case.B, dtype=bool)
+    keep[::8] = True
+    lens[~keep] = 0
+    e = case.elem_bytes
+    s_bytes = (int(lens.astype(np.int64).sum()) * case.Hkv * case.D * e * 2 + 2 * int(keep.sum()) * case.Hq * case.D * e)
+    kc, vc = orc.kv_append(case)
+    one = []
+    for _ in range(3):
+        t0 = time.perf_counter()
+        orc.decode(case, kc, vc, context_lens=lens, nthreads=1)
+        one.append(time.perf_counter() - t0)
+    sec_one = statistics.median(one)
+    return {"value": nbytes / sec_all / 1e9, "unit": "GB/s", "cores": orc.max_threads(), "kind": "oracle",
+            "sample": f"median of 3 runs of {steps_all // 3}-{steps_all - steps_all // 3 * 2} full steps (append + "
+                      f"decode of all {case.B} requests) of {case.name}, {sec_all * 1e3:.1f} ms per step",
+            "ms_per_step": sec_all * 1e3,
+            "cores_1": {"value": s_bytes / sec_one / 1e9, "unit": "GB/s", "cores": 1,
+                        "sample": f"median of 3 single-thread runs over {int(keep.sum())} of {case.B} requests "
+                                  f"(every eighth), {sec_one:.2f} s each"}}
 
 
 def run_reference(args):
@@ -207,13 +251,14 @@ def run_reference(args):
     case = synth.make_config(args.config)
     from synth import algorithmic_bytes
     base = cpu_baseline(case, max(args.cpu_seconds, 1.0) if args.steps else args.cpu_seconds)
+    ab = algorithmic_bytes(case)
     line = {"impl": "reference", "metric": "paged-decode attention HBM GB/s (% of B200 peak); us/decode step",
             "value": base["value"], "unit": "GB/s", "n_gpus": args.gpus, "steps": args.steps,
             "warmup": args.warmup, "ms_per_step": base["ms_per_step"], "higher_is_better": True,
             "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic",
             "config": {"workload": case.name, "B": case.B, "Hq": case.Hq, "Hkv": case.Hkv, "D": case.D,
-                       "block_size": case.block_size, "bytes_per_step": algorithmic_bytes(case)["step_total"]},
-            "cpu_baseline": {k: base[k] for k in ("kind", "cores", "sample", "value", "unit")},
+                       "block_size": case.block_size, "bytes_per_step": ab["decode_unique"]},
+            "cpu_baseline": {k: base[k] for k in ("kind", "cores", "sample", "value", "unit", "cores_1")},
             "e2e": {"value": base["value"], "unit": "GB/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
             "gpu_launches": 0}
     print(json.dumps(line), flush=True)
@@ -233,7 +278,7 @@ def run_prefill(args):
     libbuild.build()
     import ctypes
     import paged_kv_cache_472_b200 as pa
-    from tests import gpu_harness as H
+    from synth.device import to_device
 
     torch.cuda.set_device(0)
     pc = synth.make_prefill_config(args.prefill)
@@ -243,7 +288,7 @@ def run_prefill(args):
     ashape = pa.Shape(pc.T, pc.Hq, pc.Hkv, pc.D, pc.block_size, pc.num_blocks, pc.max_blocks_per_seq, dt)
     plan = pa.pa_prefill_plan(shape, int(pc.new_tokens().max()))
     R = 3
-    v = lambda a: H._vals(a, pc.dtype, "cuda")
+    v = lambda a: to_device(a, pc.dtype, "cuda")
     i32 = lambda a: torch.from_numpy(np.ascontiguousarray(a, dtype=np.int32)).cuda()
     copies = []
     for _ in range(R):
@@ -351,6 +396,146 @@ def run_prefill(args):
     print(json.dumps(line), flush=True)
 
 
+def timed_regions(fn, K: int, stream, min_ms: float, world: int, est_ms_step: float, max_regions: int = 200):
+    """Time `fn(i)` for i in 0..K-1 as one region (barrier + synchronise on
+    both sides, CUDA events on `stream`), repeated until the regions span
+    `min_ms` in total; returns (median region ms, regions, all region ms)."""
+    import torch
+    import torch.distributed as dist
+    n = max(1, min(max_regions, math.ceil(min_ms / max(K * est_ms_step, 1e-3))))
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    times = []
+    base = 0
+    for _ in range(n):
+        torch.cuda.synchronize()
+        if world > 1:
+            dist.barrier()
+        torch.cuda.synchronize()
+        torch.cuda._sleep(int(min(50e6, 2e6 + K * 40_000)))   # keep the host ahead of the GPU (not timed)
+        e0.record(stream)
+        for i in range(K):
+            fn(base + i)
+        e1.record(stream)
+        torch.cuda.synchronize()
+        times.append(e0.elapsed_time(e1))
+        base += K
+    return statistics.median(times), n, times
+
+
+def decode_workload(cid, args, world, rank, local, stream, lib, pa, extra=False):
+    """Upload workload `cid` (rank-seeded) in rotating copies and time its
+    step (fused append + decode), the decode kernel alone and (main
+    workload) the step behind a copy kernel and the end-to-end step."""
+    import ctypes
+    import torch
+    import synth
+    from synth import algorithmic_bytes
+    from synth.device import shape_fields, upload
+    from paged_kv_cache_472_b200.session import PagedDecoder, StepStaging
+
+    case = synth.make_config(cid, seed=rank_seed(cid, rank))
+    pt = case.partition_tokens if args.partition < 0 else args.partition
+    ab = algorithmic_bytes(case)
+    l2 = torch.cuda.get_device_properties(local).L2_cache_size
+    R = max(3, math.ceil(3 * l2 / max(ab["step_total"], 1)))
+    copies = [upload(case) for _ in range(R)]
+    dec = PagedDecoder(pa.Shape(*shape_fields(case)), int(case.max_blocks_per_seq * case.block_size), pt)
+    if args.dynamic_share >= 0 and not extra:
+        dec.plan.dynamic_share = args.dynamic_share
+    byref = ctypes.byref
+    shp, pln = byref(dec.shape), byref(dec.plan)
+    ws, wsb = dec.workspace.data_ptr(), dec.workspace.numel()
+    ptrs = [(c.k_new.data_ptr(), c.v_new.data_ptr(), c.slot_mapping.data_ptr(), c.k_cache.data_ptr(),
+             c.v_cache.data_ptr(), c.q.data_ptr(), c.block_tables.data_ptr(), c.context_lens.data_ptr(),
+             c.out.data_ptr()) for c in copies]
+    scale = float(case.scale)
+    sp = stream.cuda_stream
+
+    def step(i):
+        # one decode step through the public C entry point: append + decode in one launch
+        kn, vn, sm, kc, vc, q, bt, cl, out = ptrs[i % R]
+        return lib.pa_kv_append_decode(kn, vn, sm, q, kc, vc, bt, cl, scale, out, shp, pln, ws, wsb, sp)
+
+    def decode_only(i):
+        kn, vn, sm, kc, vc, q, bt, cl, out = ptrs[i % R]
+        return lib.pa_decode(q, kc, vc, bt, cl, scale, out, shp, pln, ws, wsb, sp)
+
+    for i in range(max(args.warmup, 3)):
+        if step(i):
+            raise RuntimeError(pa.pa_last_error_message())
+    torch.cuda.synchronize()
+    # a first estimate of the step time sizes the number of regions
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    e0.record(stream)
+    for i in range(8):
+        step(i)
+    e1.record(stream)
+    torch.cuda.synchronize()
+    est = max_over_ranks(e0.elapsed_time(e1) / 8, world, "cuda")   # the same region count on every rank
+    K = args.steps
+    res = {"case": case, "ab": ab, "R": R, "pt": pt, "dec": dec, "l2": l2}
+    KD = max(min(K, 2000), 1)
+    # clocks are sampled while the main workload's timed regions run
+    with ClockSampler(local if not extra else -1) as clk:
+        ms_region, nreg, _ = timed_regions(step, K, stream, args.min_timed_ms, world, est)
+        # the decode kernel alone, back to back (events around each region, not between launches)
+        ms_dec, nreg_d, _ = timed_regions(decode_only, KD, stream, args.min_timed_ms, world, est)
+    res["clocks"] = clk.summary()
+    res["ms_step"] = max_over_ranks(ms_region / K, world, "cuda")
+    res["regions"] = nreg
+    res["ms_decode"] = max_over_ranks(ms_dec / KD, world, "cuda")
+    res["decode_regions"], res["decode_launches"] = nreg_d, KD
+    err = dec.device_error()
+    if err:
+        raise RuntimeError(f"{case.name}: device error word {err:#x}")
+    if extra:
+        return res
+
+    # ---- the step behind another kernel: a ~100 MB copy (50 MB read, 50 MB
+    # written) on the same stream before every step, as the projection GEMM
+    # before attention would be in an engine ----
+    src = torch.empty(25 << 20, dtype=torch.int16, device="cuda")
+    dst = torch.empty_like(src)
+    KO = max(1, min(K, 500))
+    ms_copy, _, _ = timed_regions(lambda i: dst.copy_(src), KO, stream, args.min_timed_ms / 4, world, 0.02)
+
+    def copy_then_step(i):
+        dst.copy_(src)
+        step(i)
+
+    ms_both, _, _ = timed_regions(copy_then_step, KO, stream, args.min_timed_ms / 2, world, est + 0.02)
+    res["us_after_copy"] = max_over_ranks((ms_both - ms_copy) / KO * 1e3, world, "cuda")
+    res["copy_us"] = ms_copy / KO * 1e3
+    del src, dst
+
+    # ---- end to end: host buffers through the same C call ----
+    # the step's inputs staged in one pinned host buffer, uploaded with one
+    # copy; the result read back with one copy; the KV pool is resident state
+    E = max(1, args.e2e_steps)
+    c0 = copies[0]
+    names = StepStaging.ORDER
+    stg = StepStaging({n: (tuple(getattr(c0, n).shape), getattr(c0, n).dtype) for n in names},
+                      tuple(c0.out.shape), c0.out.dtype)
+    for n in names:
+        stg.host[n].copy_(getattr(c0, n).cpu())
+    res["h2d"] = stg.upload_bytes
+    res["d2h"] = stg.out.numel() * stg.out.element_size()
+    sq, skn, svn, ssm, scl, sbt = (stg.dev[n].data_ptr() for n in names)
+    kc, vc, out = c0.k_cache.data_ptr(), c0.v_cache.data_ptr(), c0.out.data_ptr()
+
+    def e2e_step(i):
+        stg.upload(stream)
+        lib.pa_kv_append_decode(skn, svn, ssm, sq, kc, vc, sbt, scl, scale, out, shp, pln, ws, wsb, sp)
+        stg.download(c0.out, stream)
+
+    ms_e2e, _, _ = timed_regions(e2e_step, E, stream, args.min_timed_ms / 2, world, est * 2)
+    res["ms_e2e"] = max_over_ranks(ms_e2e / E, world, "cuda")
+    err = dec.device_error()
+    if err:
+        raise RuntimeError(f"{case.name}: device error word {err:#x}")
+    return res
+
+
 def main():
     args = parse()
     if args.impl == "reference":
@@ -360,9 +545,6 @@ def main():
 
     import torch
     import torch.distributed as dist
-
-    import synth
-    from synth import algorithmic_bytes
     import importlib.util
     spec = importlib.util.spec_from_file_location(
         "_pagedattn_build", os.path.join(ROOT, "paged_kv_cache_472_b200", "build.py"))
@@ -370,8 +552,6 @@ def main():
     spec.loader.exec_module(libbuild)
     libbuild.build()   # before the package import loads the library
     import paged_kv_cache_472_b200 as pa
-    from paged_kv_cache_472_b200.session import PagedDecoder
-    from tests import gpu_harness as H
 
     world = int(os.environ.get("WORLD_SIZE", "1"))
     rank = int(os.environ.get("RANK", "0"))
@@ -380,137 +560,68 @@ def main():
     if world > 1:
         from datetime import timedelta
         dist.init_process_group("nccl", timeout=timedelta(seconds=120))
-
-    # each rank decodes its own batch of the workload (distinct seed per rank)
-    base_case = synth.make_config(args.config, seed=rank_seed(args.config, rank))
-    pt = base_case.partition_tokens if args.partition < 0 else args.partition
-    ab = algorithmic_bytes(base_case)
-    step_bytes = ab["step_total"]
-    decode_bytes = ab["decode_total"]
-    l2 = torch.cuda.get_device_properties(local).L2_cache_size
-    R = max(3, math.ceil(3 * l2 / max(step_bytes, 1)))
-    copies = [H.upload(base_case) for _ in range(R)]
-    shape = H.shape_of(base_case)
-    dec = PagedDecoder(shape, int(base_case.max_blocks_per_seq * base_case.block_size), pt)
-    if args.dynamic_share >= 0:
-        dec.plan.dynamic_share = args.dynamic_share
     stream = torch.cuda.current_stream()
-    sp = stream.cuda_stream
+    peak, peak_kind = measured_peak()
+    extras = [int(x) for x in args.extra.split(",") if x.strip() and int(x) != args.config]
 
-    # raw pointers, so the launch loop is two plain C calls
-    lib, byref = pa.lib, __import__("ctypes").byref
-    shp, pln = byref(dec.shape), byref(dec.plan)
-    ws, wsb = dec.workspace.data_ptr(), dec.workspace.numel()
-    ptrs = [(c.k_new.data_ptr(), c.v_new.data_ptr(), c.slot_mapping.data_ptr(), c.k_cache.data_ptr(),
-             c.v_cache.data_ptr(), c.q.data_ptr(), c.block_tables.data_ptr(), c.context_lens.data_ptr(),
-             c.out.data_ptr()) for c in copies]
-    scale = float(base_case.scale)
-
-    def step(i):
-        # one decode step through the public C entry point: append + decode
-        kn, vn, sm, kc, vc, q, bt, cl, out = ptrs[i % R]
-        return lib.pa_kv_append_decode(kn, vn, sm, q, kc, vc, bt, cl, scale, out, shp, pln, ws, wsb, sp)
-
-    def decode_only(i):
-        kn, vn, sm, kc, vc, q, bt, cl, out = ptrs[i % R]
-        return lib.pa_decode(q, kc, vc, bt, cl, scale, out, shp, pln, ws, wsb, sp)
-
-    for i in range(args.warmup):
-        if step(i):
-            raise RuntimeError(pa.pa_last_error_message())
-    torch.cuda.synchronize()
-    if world > 1:
-        dist.barrier()
-    torch.cuda.synchronize()
-
-    K = args.steps
-    start, end = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
-    with ClockSampler(local) as clk:
-        torch.cuda._sleep(50_000_000)          # keep the queue ahead of the GPU (not timed)
-        start.record(stream)
-        for i in range(K):
-            step(i)
-        end.record(stream)
-        torch.cuda.synchronize()
-    if world > 1:
-        dist.barrier()
-    ms_total = max_over_ranks(start.elapsed_time(end), world, "cuda")
-
-    # the decode kernel alone: KD back-to-back launches on its stream, CUDA
-    # events around the whole region (events between launches would add their
-    # own gaps to every launch)
-    KD = max(min(K, 2000), 1)
-    d0, d1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
-    torch.cuda._sleep(50_000_000)
-    d0.record(stream)
-    for i in range(KD):
-        decode_only(i)
-    d1.record(stream)
-    torch.cuda.synchronize()
-    dec_avg_ms = d0.elapsed_time(d1) / KD
-    ms_step = ms_total / K
-    err = dec.device_error()
-    if err:
-        raise RuntimeError(f"device error word {err:#x}")
-
-    # ---- end to end: host buffers through the same C calls ----
-    # the step's inputs staged in one pinned host buffer, uploaded with one
-    # copy; the result read back with one copy; the KV pool is resident state
-    from paged_kv_cache_472_b200.session import StepStaging
-    E = args.e2e_steps
-    c0 = copies[0]
-    names = StepStaging.ORDER
-    stg = StepStaging({n: (tuple(getattr(c0, n).shape), getattr(c0, n).dtype) for n in names},
-                      tuple(c0.out.shape), c0.out.dtype)
-    for n in names:
-        stg.host[n].copy_(getattr(c0, n).cpu())
-    h2d = stg.upload_bytes
-    d2h = stg.out.numel() * stg.out.element_size()
-    sq, skn, svn, ssm, scl, sbt = (stg.dev[n].data_ptr() for n in names)
-    kc, vc, out = c0.k_cache.data_ptr(), c0.v_cache.data_ptr(), c0.out.data_ptr()
-    torch.cuda.synchronize()
-    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
-    e0.record(stream)
-    for i in range(E):
-        stg.upload(stream)
-        lib.pa_kv_append_decode(skn, svn, ssm, sq, kc, vc, sbt, scl, scale, out, shp, pln, ws, wsb, sp)
-        stg.download(c0.out, stream)
-    e1.record(stream)
-    torch.cuda.synchronize()
-    e2e_ms = max_over_ranks(e0.elapsed_time(e1) / E, world, "cuda")
+    m = decode_workload(args.config, args, world, rank, local, stream, pa.lib, pa)
+    others = {}
+    for cid in extras:
+        r = decode_workload(cid, args, world, rank, local, stream, pa.lib, pa, extra=True)
+        ab = r["ab"]
+        others[r["case"].name] = {
+            "step_us": round(r["ms_step"] * 1e3, 3), "decode_us": round(r["ms_decode"] * 1e3, 3),
+            "decode_gbs": round(ab["decode_unique"] / (r["ms_decode"] * 1e-3) / 1e9, 1),
+            "frac": round(ab["decode_unique"] / (r["ms_decode"] * 1e-3) / 1e9 / peak, 4),
+            "step_gbs": round(ab["decode_unique"] / (r["ms_step"] * 1e-3) / 1e9, 1),
+            "bytes": ab["decode_unique"], "regions": r["regions"], "partition_tokens": r["pt"]}
+        del r
+        torch.cuda.empty_cache()
 
     if rank == 0:
-        peak, peak_kind = measured_peak()
-        achieved = decode_bytes / (dec_avg_ms * 1e-3) / 1e9
-        value = job_throughput_gbs(step_bytes, world, ms_step)
+        case, ab = m["case"], m["ab"]
+        ms_step = m["ms_step"]
+        dbytes = ab["decode_unique"]
+        achieved = dbytes / (m["ms_decode"] * 1e-3) / 1e9
+        value = job_throughput_gbs(dbytes, world, ms_step)
         line = {
             "metric": "paged-decode attention HBM GB/s (% of B200 peak); us/decode step",
-            "value": round(value, 2), "unit": "GB/s", "n_gpus": world, "steps": K, "warmup": args.warmup,
-            "ms_per_step": round(ms_step, 6), "us_per_step": round(ms_step * 1e3, 3),
-            "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": base_case.dtype,
+            "value": round(value, 2), "unit": "GB/s", "n_gpus": world, "steps": args.steps,
+            "warmup": args.warmup, "ms_per_step": round(ms_step, 6), "us_per_step": round(ms_step * 1e3, 3),
+            "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": case.dtype,
             "data": "synthetic",
-            "config": {"workload": base_case.name, "B": base_case.B, "Hq": base_case.Hq, "Hkv": base_case.Hkv,
-                       "D": base_case.D, "block_size": base_case.block_size,
-                       "context_tokens": int(base_case.context_lens.sum()), "partition_tokens": pt,
-                       "dynamic_share": int(dec.plan.dynamic_share),
-                       "bytes_per_step": step_bytes, "decode_bytes_per_step": decode_bytes,
-                       "l2": f"{R} rotating input copies, {R * step_bytes / 1e6:.0f} MB > L2 {l2 / 1e6:.0f} MB",
+            "config": {"workload": case.name, "B": case.B, "Hq": case.Hq, "Hkv": case.Hkv, "D": case.D,
+                       "block_size": case.block_size, "context_tokens": int(case.context_lens.sum()),
+                       "partition_tokens": m["pt"], "dynamic_share": int(m["dec"].plan.dynamic_share),
+                       "bytes_per_step": dbytes, "bytes_kind": "algorithmic: K/V of every block once + q + out "
+                                                                 "+ tables + lengths",
+                       "logical_bytes_per_step": ab["decode_total"], "append_bytes_per_step": ab["append"],
+                       "logical_gbs": round(world * ab["decode_total"] / (ms_step * 1e-3) / 1e9, 2),
+                       "l2": f"{m['R']} rotating input copies, {m['R'] * ab['step_total'] / 1e6:.0f} MB > L2 "
+                             f"{m['l2'] / 1e6:.0f} MB",
+                       "timed_regions": m["regions"], "region_stat": "median",
                        "parallelism": f"replicas x{world}" if world > 1 else "1 GPU",
-                       "tokens_per_s": round(world * base_case.B / (ms_step * 1e-3), 1),
-                       "pct_of_peak": round(100 * value / world / peak, 2)},
+                       "tokens_per_s": round(world * case.B / (ms_step * 1e-3), 1),
+                       "pct_of_peak": round(100 * value / world / peak, 2),
+                       "step_us_after_copy": round(m["us_after_copy"], 3),
+                       "copy_us": round(m["copy_us"], 3)},
             "roofline": {"bound": "hbm", "achieved": round(achieved, 2), "peak": peak, "unit": "GB/s",
-                         "frac": round(achieved / peak, 4), "traffic": profiled_traffic(base_case.name),
+                         "frac": round(achieved / peak, 4), "traffic": profiled_traffic(case.name),
                          "kernel": "paged_decode_kernel", "peak_kind": peak_kind,
-                         "decode_us": round(dec_avg_ms * 1e3, 3), "decode_launches_timed": KD,
-                         "engine": "tensor-core mma" if base_case.dtype == "bf16" else "cuda-core fp32"},
-            "e2e": {"value": round(job_throughput_gbs(step_bytes, world, e2e_ms), 2), "unit": "GB/s",
-                    "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h, "us_per_step": round(e2e_ms * 1e3, 3)},
-            "gpu_launches": K,   # one fused append + decode launch per step
-            "clocks": clk.summary(),
+                         "decode_us": round(m["ms_decode"] * 1e3, 3), "decode_launches_timed": m["decode_launches"],
+                         "decode_regions": m["decode_regions"],
+                         "algorithmic_bytes_per_launch": dbytes,
+                         "engine": "tensor-core mma" if case.dtype != "f32" else "cuda-core fp32"},
+            "e2e": {"value": round(job_throughput_gbs(dbytes, world, m["ms_e2e"]), 2), "unit": "GB/s",
+                    "h2d_bytes_per_step": m["h2d"], "d2h_bytes_per_step": m["d2h"],
+                    "us_per_step": round(m["ms_e2e"] * 1e3, 3)},
+            "workloads": others,
+            "gpu_launches": args.steps,   # one fused append + decode launch per step of the reported region
+            "clocks": m["clocks"],
         }
         if not args.no_cpu_baseline:
-            cb = cpu_baseline(base_case, args.cpu_seconds)
-            line["cpu_baseline"] = {k: cb[k] for k in ("value", "unit", "cores", "kind", "sample")}
+            cb = cpu_baseline(case, args.cpu_seconds)
+            line["cpu_baseline"] = {k: cb[k] for k in ("value", "unit", "cores", "kind", "sample", "cores_1")}
         print(json.dumps(line), flush=True)
     if world > 1:
         dist.barrier()

@@ -109,9 +109,14 @@ typedef struct {
  * reads.  PA_PLAN_NO_SPECULATION turns the early reads off (useful when the
  * preceding kernel rewrites the metadata every step).  PA_PLAN_TEST_MISGUESS
  * makes every early guess wrong, so that the plan-again path runs (for
- * tests; slower). */
+ * tests; slower).  PA_PLAN_TEST_STALL is for tests of the failure path only:
+ * the first CTA publishes its first piece but never fills a pipeline stage
+ * for it, so its consumers' bounded wait (about 2 s) gives up, records
+ * PA_DEVERR_TIMEOUT and the whole CTA leaves cleanly (no copy outstanding);
+ * the output is then undefined and the workspace must be re-initialised. */
 #define PA_PLAN_NO_SPECULATION 0x1
 #define PA_PLAN_TEST_MISGUESS  0x2
+#define PA_PLAN_TEST_STALL     0x4
 
 /* Library version: major*10000 + minor*100 + patch. */
 int32_t pa_version(void);
@@ -138,7 +143,8 @@ pa_status pa_kv_append(const void *k_new, const void *v_new, const int32_t *slot
                        void *v_cache, const pa_shape *s, int32_t *device_error, void *stream);
 
 /*
- * Host-only planner (no device work, no allocation).
+ * Host-only planner (no device work, no allocation): the "host-side partition
+ * planner" of the problem statement, here sized for a persistent grid.
  *   max_context_len : the largest context_lens[b] any later call will pass
  *                     (at most max_blocks_per_seq*block_size); recorded in
  *                     the plan.
@@ -162,11 +168,16 @@ pa_status pa_kv_append(const void *k_new, const void *v_new, const int32_t *slot
 pa_status pa_plan(const pa_shape *s, int32_t max_context_len, int32_t partition_tokens, int32_t num_sms,
                   pa_plan_t *plan_out);
 
-/* Bytes of device workspace pa_decode needs for `plan` (== plan->workspace_bytes). */
+/* Bytes of device workspace pa_decode needs for `plan` (== plan->workspace_bytes).
+ * The size follows from the plan alone (the planner fixes it from the shape,
+ * the partition size and the CTA count), not from the context lengths. */
 size_t pa_decode_workspace_size(const pa_plan_t *plan);
 
-/* Zero a workspace before its first pa_decode (the kernels leave it ready
- * for the next call afterwards).  Queued on `stream`. */
+/* Zero a workspace before its first pa_decode.  A call that completes
+ * leaves the workspace ready for the next one; a call that recorded
+ * PA_DEVERR_TIMEOUT (a CTA gave up part-way) may leave its merge counters
+ * set, so re-initialise the workspace after such an error.  Queued on
+ * `stream`. */
 pa_status pa_workspace_init(void *workspace, size_t workspace_bytes, void *stream);
 
 /*
@@ -179,7 +190,11 @@ pa_status pa_workspace_init(void *workspace, size_t workspace_bytes, void *strea
  *   scale        : softmax scale (typically 1/sqrt(D))
  *   out          : device, [B, Hq, D], dtype s->dtype (fp32 results rounded
  *                  to nearest-even for bf16)
- *   plan         : from pa_plan for the same *s
+ *   plan         : from pa_plan for the same *s; a plan whose fields differ
+ *                  from what pa_plan gives for the shape, max_context_len,
+ *                  partition size and CTA count it records is rejected with
+ *                  PA_ERR_INVALID_ARG (only dynamic_share and flags are the
+ *                  caller's to change)
  *   workspace    : device, >= plan->workspace_bytes, 256-byte aligned,
  *                  zeroed once by pa_workspace_init; holds partial results,
  *                  merge counters and the device error word.  Two calls that
@@ -213,13 +228,14 @@ pa_status pa_kv_append_decode(const void *k_new, const void *v_new, const int32_
  * the library holds it until the process exits).  There is no counterpart
  * of this call in the pages: it only changes where the scratch lives.
  *   Arguments as in pa_decode, minus workspace and workspace_bytes.
- *   plan->workspace_bytes above 16 MiB returns PA_ERR_WORKSPACE.
+ *   plan->workspace_bytes above 16 MiB returns PA_ERR_WORKSPACE.  Every
+ *   argument is checked before anything is queued.
  *   Allocates nothing: no cudaMalloc, no cudaFree, no allocating library call.
  *   The first call on a device looks up the array's device address for that
  *   device (with it current); make that first call before any stream capture.
- *   Every call clears the array's error word and merge counters first (one
- *   cudaMemsetAsync on `stream`), so index errors recorded by one call are
- *   gone at the next and cannot be read back through this entry point.
+ *   Every call first zeroes the array's merge counters (one cudaMemsetAsync
+ *   on `stream`); the array's error word is not cleared by it: it gathers the
+ *   index errors of all calls until pa_no_alloc_device_error reads it.
  *   All calls share the one array: two calls that overlap on the GPU race.
  */
 pa_status pa_decode_no_alloc(const void *q, const void *k_cache, const void *v_cache, const int32_t *block_tables,
@@ -271,8 +287,17 @@ pa_status pa_prefill(const void *q, const void *k_cache, const void *v_cache, co
                      const pa_shape *s, const pa_prefill_plan_t *plan, int32_t *device_error, void *stream);
 
 /* Copy the device error word of `workspace` to *err_out (synchronises
- * `stream`; not for the hot path).  clear != 0 resets it to 0 afterwards. */
+ * `stream`; not for the hot path).  clear != 0 resets it to 0 afterwards.
+ * The word is the first four bytes of the workspace: pa_kv_append may be
+ * given the same workspace pointer as its device_error. */
 pa_status pa_get_device_error(void *workspace, int32_t clear, int32_t *err_out, void *stream);
+
+/* The error word of pa_decode_no_alloc's built-in array on the current
+ * device, as pa_get_device_error does for a workspace: the PA_DEVERR_* bits
+ * of every pa_decode_no_alloc call since the word was last cleared
+ * (synchronises `stream`; clear != 0 resets it afterwards).  Allocates
+ * nothing.  No counterpart in the pages. */
+pa_status pa_no_alloc_device_error(int32_t clear, int32_t *err_out, void *stream);
 
 #ifdef __cplusplus
 }

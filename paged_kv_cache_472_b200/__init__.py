@@ -15,7 +15,7 @@ from .build import LIB as _LIB_PATH
 
 __all__ = ["PagedAttnError", "Shape", "Plan", "DTYPE_F32", "DTYPE_BF16", "DTYPE_F16", "SPLIT_BALANCED", "SPLIT_FIXED",
            "DEVERR_BLOCK_ID", "DEVERR_CONTEXT_LEN", "DEVERR_TIMEOUT", "DEVERR_WORKSPACE", "DEVERR_SLOT", "DEVERR_SMEM",
-           "PLAN_NO_SPECULATION", "PLAN_TEST_MISGUESS",
+           "PLAN_NO_SPECULATION", "PLAN_TEST_MISGUESS", "PLAN_TEST_STALL", "pa_no_alloc_device_error",
            "pa_version", "pa_status_str", "pa_last_error_message", "pa_kv_append", "pa_plan",
            "pa_decode_workspace_size", "pa_workspace_init", "pa_decode", "pa_kv_append_decode", "pa_get_device_error",
            "pa_decode_no_alloc", "PrefillPlan", "pa_prefill_plan", "pa_prefill", "lib"]
@@ -25,7 +25,7 @@ DTYPE_F32, DTYPE_BF16, DTYPE_F16 = 0, 1, 2
 SPLIT_BALANCED, SPLIT_FIXED = 0, 1
 DEVERR_BLOCK_ID, DEVERR_CONTEXT_LEN, DEVERR_TIMEOUT, DEVERR_WORKSPACE, DEVERR_SLOT, DEVERR_SMEM = (
     0x1, 0x2, 0x4, 0x8, 0x10, 0x20)
-PLAN_NO_SPECULATION, PLAN_TEST_MISGUESS = 0x1, 0x2
+PLAN_NO_SPECULATION, PLAN_TEST_MISGUESS, PLAN_TEST_STALL = 0x1, 0x2, 0x4
 
 
 class Shape(ctypes.Structure):
@@ -84,10 +84,11 @@ lib.pa_get_device_error.argtypes = [_vp, _i32, _P(_i32), _vp]
 lib.pa_kv_append_decode.argtypes = [_vp, _vp, _vp, _vp, _vp, _vp, _vp, _vp, ctypes.c_float, _vp, _P(Shape), _P(Plan),
                                     _vp, _sz, _vp]
 lib.pa_decode_no_alloc.argtypes = [_vp, _vp, _vp, _vp, _vp, ctypes.c_float, _vp, _P(Shape), _P(Plan), _vp]
+lib.pa_no_alloc_device_error.argtypes = [_i32, _P(_i32), _vp]
 lib.pa_prefill_plan.argtypes = [_P(Shape), _i32, _P(PrefillPlan)]
 lib.pa_prefill.argtypes = [_vp, _vp, _vp, _vp, _vp, _vp, ctypes.c_float, _vp, _P(Shape), _P(PrefillPlan), _vp, _vp]
 for _f in ("pa_kv_append", "pa_plan", "pa_workspace_init", "pa_decode", "pa_get_device_error",
-           "pa_kv_append_decode", "pa_decode_no_alloc", "pa_prefill_plan", "pa_prefill"):
+           "pa_kv_append_decode", "pa_decode_no_alloc", "pa_no_alloc_device_error", "pa_prefill_plan", "pa_prefill"):
     getattr(lib, _f).restype = ctypes.c_int
 
 
@@ -171,6 +172,13 @@ def pa_get_device_error(workspace, clear: bool = False, stream=None) -> int:
     err = _i32(0)
     _check(lib.pa_get_device_error(_ptr(workspace), int(bool(clear)), ctypes.byref(err), _stream(stream)),
            "pa_get_device_error")
+    return err.value
+
+
+def pa_no_alloc_device_error(clear: bool = False, stream=None) -> int:
+    err = _i32(0)
+    _check(lib.pa_no_alloc_device_error(int(bool(clear)), ctypes.byref(err), _stream(stream)),
+           "pa_no_alloc_device_error")
     return err.value
 
 

@@ -113,6 +113,7 @@ struct DecodeParams {
     int32_t bs_log2;
     int32_t st_log2;      // ST = 1 << st_log2
     int32_t spec;         // 0: no speculation; 1: speculate; 2: speculate on wrong guesses (tests)
+    int32_t test_stall;   // tests: CTA 0 never fills the stages of its first piece (the bounded waits give up)
     int32_t lens_cached;  // context lengths were copied into shared memory
 };
 static_assert(offsetof(DecodeParams, tmap_k) % 64 == 0 && offsetof(DecodeParams, tmap_v) % 64 == 0,
@@ -1040,6 +1041,14 @@ struct MmaEngine {
 // ===========================================================================
 // producer warp
 // ===========================================================================
+
+// Wait (bounded: twice the pipeline limit) until another warp of the CTA has
+// given up and raised the abort flag.
+__device__ __forceinline__ void wait_for_abort(const volatile int *abort_flag) {
+    const uint64_t t0 = globaltimer_ns();
+    while (!*abort_flag && globaltimer_ns() - t0 < 2 * kWaitLimitNs) __nanosleep(100000);
+}
+
 struct ProducerState {
     int stage = 0;
     uint32_t phase = 0;
@@ -1280,6 +1289,13 @@ __device__ __forceinline__ void run_producer(const DecodeParams &p, const Cut &k
         fused_info(p, s, lane);
         publish(p, ps, s, ctl, qfull, qempty, qarea, abort_flag, D, E, lane);
         if (!ps.ok) break;
+        if (p.test_stall && blockIdx.x == 0) {
+            // failure-path test: no stage of this piece is ever filled, so the
+            // consumers' wait gives up; issue nothing and leave once they abort
+            wait_for_abort(abort_flag);
+            ps.ok = false;
+            break;
+        }
         issue_tiles<D, E>(p, ps, s, s.t_begin, s.t_end, win, k.dyn && it.cur >= it.hi, full, empty, stage_base,
                           abort_flag, policy, policy_keep, lane);
     }

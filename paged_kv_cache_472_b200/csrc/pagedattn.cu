@@ -257,158 +257,9 @@ int log2i(int x) {
     return l;
 }
 
-// The fused step (k_new != NULL) appends each request's new token in the
-// same launch.  Every launch may start while the preceding grid on the stream
-// finishes (programmatic dependent launch): the kernel waits for that grid
-// before its first global memory access.
-pa_status launch_decode(const void *q, const void *k_cache, const void *v_cache, const int32_t *block_tables,
-                        const int32_t *context_lens, float scale, void *out, const pa_shape *s,
-                        const pa_plan_t *plan, void *workspace, size_t workspace_bytes, cudaStream_t stream,
-                        const void *k_new, const void *v_new, const int32_t *slot_mapping) {
-    if (!plan) return fail(PA_ERR_INVALID_ARG, "plan is NULL");
-    if (memcmp(&plan->shape, s, sizeof *s) != 0) return fail(PA_ERR_INVALID_ARG, "plan was made for another shape");
-    if (plan->dynamic_share < 0 || plan->dynamic_share > kMaxDynamicShare ||
-        (plan->dynamic_share > 0 && (plan->mode != PA_SPLIT_BALANCED || s->B > pa::kPrefixCache)))
-        return fail(PA_ERR_INVALID_ARG, "dynamic_share=%d outside [0, %d] or not available for this plan",
-                    plan->dynamic_share, kMaxDynamicShare);
-    if (!std::isfinite(scale)) return fail(PA_ERR_INVALID_ARG, "scale is not finite");
-    if (plan->flags & ~(PA_PLAN_NO_SPECULATION | PA_PLAN_TEST_MISGUESS))
-        return fail(PA_ERR_INVALID_ARG, "unknown plan flags %#x", plan->flags);
-    if (!workspace) return fail(PA_ERR_WORKSPACE, "workspace is NULL");
-    if (workspace_bytes < plan->workspace_bytes)
-        return fail(PA_ERR_WORKSPACE, "workspace %zu bytes < %zu needed", workspace_bytes, plan->workspace_bytes);
-    if ((reinterpret_cast<uintptr_t>(workspace) & 255u) != 0)
-        return fail(PA_ERR_INVALID_ARG, "workspace must be 256-byte aligned");
-    if (s->B == 0) return PA_OK;
-    if (!q || !k_cache || !v_cache || !block_tables || !context_lens || !out)
-        return fail(PA_ERR_INVALID_ARG, "NULL tensor pointer");
-    if (!aligned16(q) || !aligned16(k_cache) || !aligned16(v_cache) || !aligned16(out))
-        return fail(PA_ERR_INVALID_ARG, "value tensors must be 16-byte aligned");
-
-    const int HC = plan->heads_per_unit, UPW = plan->units_per_warp, TS = plan->warps_per_unit;
-    const int G = s->Hq / s->Hkv;
-    const int e = elem_bytes(s->dtype);
-    KernelFn fn = pick_kernel(s->dtype, s->D, HC, UPW, TS);
-    if (!fn) return fail(PA_ERR_INVALID_ARG, "plan names no kernel variant");
-    const int HG = plan->head_group;
-    const int NHvr = HG * G;
-    const uint32_t row_bytes = (uint32_t)(HG * s->D * e);
-    const uint32_t pitch = row_pitch_of(s, row_bytes);
-    const uint32_t half = (uint32_t)plan->tile_tokens * pitch;
-    const uint32_t q_bytes = (uint32_t)(NHvr * s->D * e);
-    const Layout lay = smem_layout(s->dtype, s->D, plan->stages, q_bytes, half, HC, TS, NHvr);
-    if ((int)lay.total != plan->smem_bytes) return fail(PA_ERR_INVALID_ARG, "plan is inconsistent");
-
-    pa::DecodeParams p{};
-    p.q = q;
-    p.k_cache = k_cache;
-    p.v_cache = v_cache;
-    p.block_tables = block_tables;
-    p.context_lens = context_lens;
-    p.out = out;
-    unsigned char *ws = static_cast<unsigned char *>(workspace);
-    const size_t counters = round_up((size_t)s->B * (s->Hkv / HG) * 4, 256);
-    p.error = reinterpret_cast<int32_t *>(ws);
-    p.grab = reinterpret_cast<int32_t *>(ws + kWsGrab);
-    p.grab_done = reinterpret_cast<int32_t *>(ws + kWsGrabDone);
-    p.fused = k_new ? 1 : 0;
-    p.k_new = k_new;
-    p.v_new = v_new;
-    p.slot_mapping = slot_mapping;
-    p.dyn_num = plan->mode == PA_SPLIT_BALANCED ? plan->dynamic_share : 0;
-    p.counters = reinterpret_cast<int32_t *>(ws + kWsHeader);
-    p.partials = reinterpret_cast<float *>(ws + kWsHeader + counters);
-    p.qscale = scale * 1.4426950408889634f;
-    p.B = s->B;
-    p.Hq = s->Hq;
-    p.Hkv = s->Hkv;
-    p.bs = s->block_size;
-    p.num_blocks = s->num_blocks;
-    p.max_blocks = s->max_blocks_per_seq;
-    p.G = G;
-    p.HG = HG;
-    p.NHG = s->Hkv / HG;
-    p.NHvr = NHvr;
-    p.ST = plan->tile_tokens;
-    p.stages = plan->stages;
-    p.mode = plan->mode;
-    p.part_tiles = plan->mode == PA_SPLIT_FIXED ? plan->partition_tokens / plan->tile_tokens : 1;
-    p.num_ctas = plan->num_ctas;
-    p.tsplit = TS;
-    p.units = HG * (G / HC);
-    p.heads_per_unit = HC;
-    p.max_slots = plan->max_slots;
-    p.slot_floats = (int64_t)NHvr * s->D + (int64_t)round_up(2 * NHvr, 4);
-    p.off_bar = lay.off_bar;
-    p.off_q = lay.off_q;
-    p.off_stage = lay.off_stage;
-    p.off_scratch = lay.off_scratch;
-    p.off_comb = lay.off_comb;
-    p.row_bytes = row_bytes;
-    p.row_pitch = pitch;
-    p.half_bytes = half;
-    p.q_bytes = q_bytes;
-    p.comb_stride = lay.comb_stride;
-    p.bs_log2 = log2i(s->block_size);
-    p.st_log2 = log2i(plan->tile_tokens);
-    p.spec = (plan->flags & PA_PLAN_NO_SPECULATION) ? 0 : ((plan->flags & PA_PLAN_TEST_MISGUESS) ? 2 : 1);
-    p.lens_cached = s->B <= pa::kLensCache ? 1 : 0;
-    if (tensor_core_dtype(s->dtype)) {
-        const int br = plan->tile_tokens < s->block_size ? plan->tile_tokens : s->block_size;
-        p.use_tmap = 1;
-        p.br_log2 = log2i(br);
-        if (pa_status st = encode_pool_map(&p.tmap_k, k_cache, s, br, HG)) return st;
-        if (pa_status st = encode_pool_map(&p.tmap_v, v_cache, s, br, HG)) return st;
-    }
-
-    if (pa_status st = ensure_smem_attr(fn, plan->smem_bytes)) return st;
-    cudaLaunchConfig_t cfg = {};
-    cfg.gridDim = dim3((unsigned)plan->num_ctas);
-    cfg.blockDim = dim3(pa::kDecodeThreads);
-    cfg.dynamicSmemBytes = (size_t)plan->smem_bytes;
-    cfg.stream = stream;
-    cudaLaunchAttribute attr[1];
-    attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
-    attr[0].val.programmaticStreamSerializationAllowed = 1;
-    cfg.attrs = attr;
-    cfg.numAttrs = 1;
-    cudaError_t ce = cudaLaunchKernelEx(&cfg, fn, p);
-    if (ce == cudaSuccess) ce = cudaGetLastError();
-    if (ce != cudaSuccess) return fail(PA_ERR_CUDA, "decode launch: %s", cudaGetErrorString(ce));
-    return PA_OK;
-}
-
-}  // namespace
-
-extern "C" {
-
-int32_t pa_version(void) { return 200; }
-
-const char *pa_status_str(pa_status st) {
-    switch (st) {
-        case PA_OK: return "PA_OK";
-        case PA_ERR_INVALID_ARG: return "PA_ERR_INVALID_ARG";
-        case PA_ERR_UNSUPPORTED: return "PA_ERR_UNSUPPORTED";
-        case PA_ERR_CUDA: return "PA_ERR_CUDA";
-        case PA_ERR_WORKSPACE: return "PA_ERR_WORKSPACE";
-    }
-    return "PA_ERR_UNKNOWN";
-}
-
-const char *pa_last_error_message(void) { return g_msg; }
-
-pa_status pa_kv_append(const void *k_new, const void *v_new, const int32_t *slot_mapping, void *k_cache,
-                       void *v_cache, const pa_shape *s, int32_t *device_error, void *stream) {
-    if (pa_status st = check_shape(s)) return st;
-    if (s->B == 0) return ok();
-    if (pa_status st = launch_append(k_new, v_new, slot_mapping, k_cache, v_cache, s, device_error,
-                                     (cudaStream_t)stream))
-        return st;
-    return ok();
-}
-
-pa_status pa_plan(const pa_shape *s, int32_t max_context_len, int32_t partition_tokens, int32_t num_sms,
-                  pa_plan_t *plan) {
+// The planner proper (pa_plan without the status-message reset).
+pa_status plan_internal(const pa_shape *s, int32_t max_context_len, int32_t partition_tokens, int32_t num_sms,
+                        pa_plan_t *plan) {
     if (!plan) return fail(PA_ERR_INVALID_ARG, "plan_out is NULL");
     if (pa_status st = check_shape(s)) return st;
     const int cap = s->max_blocks_per_seq * s->block_size;
@@ -490,6 +341,221 @@ pa_status pa_plan(const pa_shape *s, int32_t max_context_len, int32_t partition_
     const size_t slot_floats = (size_t)NHvr * s->D + round_up(2 * NHvr, 4);
     const size_t counters = round_up((size_t)s->B * NHG * 4, 256);
     plan->workspace_bytes = kWsHeader + counters + (size_t)plan->max_slots * slot_floats * 4;
+    return PA_OK;
+}
+
+
+// A plan passed to a decode call must be what the planner gives for its own
+// recorded inputs (shape, max_context_len, partition size, CTA count); only
+// dynamic_share and flags are the caller's to set.  Everything the launch
+// derives from the plan (kernel variant, grid, shared-memory layout,
+// workspace offsets) is therefore consistent before anything is queued.
+pa_status check_plan(const pa_shape *s, const pa_plan_t *plan) {
+    if (!plan) return fail(PA_ERR_INVALID_ARG, "plan is NULL");
+    if (memcmp(&plan->shape, s, sizeof *s) != 0) return fail(PA_ERR_INVALID_ARG, "plan was made for another shape");
+    if (plan->num_ctas <= 0 || (plan->mode != PA_SPLIT_BALANCED && plan->mode != PA_SPLIT_FIXED))
+        return fail(PA_ERR_INVALID_ARG, "plan is inconsistent");
+    pa_plan_t ref;
+    const int pt = plan->mode == PA_SPLIT_FIXED ? plan->partition_tokens : 0;
+    if (plan->mode == PA_SPLIT_FIXED && pt <= 0) return fail(PA_ERR_INVALID_ARG, "plan is inconsistent");
+    if (plan_internal(s, plan->max_context_len, pt, plan->num_ctas, &ref) != PA_OK) {
+        char why[sizeof g_msg];
+        memcpy(why, g_msg, sizeof why);
+        return fail(PA_ERR_INVALID_ARG, "plan is inconsistent: %s", why);
+    }
+    if (ref.mode != plan->mode || ref.partition_tokens != plan->partition_tokens || ref.tile_tokens != plan->tile_tokens ||
+        ref.stages != plan->stages || ref.head_group != plan->head_group || ref.heads_per_unit != plan->heads_per_unit ||
+        ref.units_per_warp != plan->units_per_warp || ref.warps_per_unit != plan->warps_per_unit ||
+        ref.smem_bytes != plan->smem_bytes || ref.max_slots != plan->max_slots ||
+        ref.workspace_bytes != plan->workspace_bytes)
+        return fail(PA_ERR_INVALID_ARG, "plan is inconsistent with the planner's output for this shape");
+    return PA_OK;
+}
+
+// A decode launch, validated and ready to queue.
+struct DecodeLaunch {
+    pa::DecodeParams p;
+    KernelFn fn = nullptr;
+    int smem_bytes = 0;
+    int num_ctas = 0;
+    bool empty = true;  // nothing to launch (B == 0)
+};
+
+// Every host-side check of a decode call, and the kernel parameters it
+// implies.  Nothing is queued on the GPU here.  The fused step (k_new !=
+// NULL) appends each request's new token in the same launch.
+pa_status prepare_decode(const void *q, const void *k_cache, const void *v_cache, const int32_t *block_tables,
+                         const int32_t *context_lens, float scale, void *out, const pa_shape *s,
+                         const pa_plan_t *plan, void *workspace, size_t workspace_bytes, const void *k_new,
+                         const void *v_new, const int32_t *slot_mapping, DecodeLaunch &L) {
+    if (pa_status st = check_plan(s, plan)) return st;
+    if (plan->dynamic_share < 0 || plan->dynamic_share > kMaxDynamicShare ||
+        (plan->dynamic_share > 0 && (plan->mode != PA_SPLIT_BALANCED || s->B > pa::kPrefixCache)))
+        return fail(PA_ERR_INVALID_ARG, "dynamic_share=%d outside [0, %d] or not available for this plan",
+                    plan->dynamic_share, kMaxDynamicShare);
+    if (!std::isfinite(scale)) return fail(PA_ERR_INVALID_ARG, "scale is not finite");
+    if (plan->flags & ~(PA_PLAN_NO_SPECULATION | PA_PLAN_TEST_MISGUESS | PA_PLAN_TEST_STALL))
+        return fail(PA_ERR_INVALID_ARG, "unknown plan flags %#x", plan->flags);
+    if (!workspace) return fail(PA_ERR_WORKSPACE, "workspace is NULL");
+    if (workspace_bytes < plan->workspace_bytes)
+        return fail(PA_ERR_WORKSPACE, "workspace %zu bytes < %zu needed", workspace_bytes, plan->workspace_bytes);
+    if ((reinterpret_cast<uintptr_t>(workspace) & 255u) != 0)
+        return fail(PA_ERR_INVALID_ARG, "workspace must be 256-byte aligned");
+    L.empty = s->B == 0;
+    if (L.empty) return PA_OK;
+    if (!q || !k_cache || !v_cache || !block_tables || !context_lens || !out)
+        return fail(PA_ERR_INVALID_ARG, "NULL tensor pointer");
+    if (!aligned16(q) || !aligned16(k_cache) || !aligned16(v_cache) || !aligned16(out))
+        return fail(PA_ERR_INVALID_ARG, "value tensors must be 16-byte aligned");
+
+    const int HC = plan->heads_per_unit, UPW = plan->units_per_warp, TS = plan->warps_per_unit;
+    const int G = s->Hq / s->Hkv;
+    const int e = elem_bytes(s->dtype);
+    KernelFn fn = pick_kernel(s->dtype, s->D, HC, UPW, TS);
+    if (!fn) return fail(PA_ERR_INVALID_ARG, "plan names no kernel variant");
+    const int HG = plan->head_group;
+    const int NHvr = HG * G;
+    const uint32_t row_bytes = (uint32_t)(HG * s->D * e);
+    const uint32_t pitch = row_pitch_of(s, row_bytes);
+    const uint32_t half = (uint32_t)plan->tile_tokens * pitch;
+    const uint32_t q_bytes = (uint32_t)(NHvr * s->D * e);
+    const Layout lay = smem_layout(s->dtype, s->D, plan->stages, q_bytes, half, HC, TS, NHvr);
+    if ((int)lay.total != plan->smem_bytes) return fail(PA_ERR_INVALID_ARG, "plan is inconsistent");
+
+    pa::DecodeParams &p = L.p;
+    p = pa::DecodeParams{};
+    p.q = q;
+    p.k_cache = k_cache;
+    p.v_cache = v_cache;
+    p.block_tables = block_tables;
+    p.context_lens = context_lens;
+    p.out = out;
+    unsigned char *ws = static_cast<unsigned char *>(workspace);
+    const size_t counters = round_up((size_t)s->B * (s->Hkv / HG) * 4, 256);
+    p.error = reinterpret_cast<int32_t *>(ws);
+    p.grab = reinterpret_cast<int32_t *>(ws + kWsGrab);
+    p.grab_done = reinterpret_cast<int32_t *>(ws + kWsGrabDone);
+    p.fused = k_new ? 1 : 0;
+    p.k_new = k_new;
+    p.v_new = v_new;
+    p.slot_mapping = slot_mapping;
+    p.dyn_num = plan->mode == PA_SPLIT_BALANCED ? plan->dynamic_share : 0;
+    p.counters = reinterpret_cast<int32_t *>(ws + kWsHeader);
+    p.partials = reinterpret_cast<float *>(ws + kWsHeader + counters);
+    p.qscale = scale * 1.4426950408889634f;
+    p.B = s->B;
+    p.Hq = s->Hq;
+    p.Hkv = s->Hkv;
+    p.bs = s->block_size;
+    p.num_blocks = s->num_blocks;
+    p.max_blocks = s->max_blocks_per_seq;
+    p.G = G;
+    p.HG = HG;
+    p.NHG = s->Hkv / HG;
+    p.NHvr = NHvr;
+    p.ST = plan->tile_tokens;
+    p.stages = plan->stages;
+    p.mode = plan->mode;
+    p.part_tiles = plan->mode == PA_SPLIT_FIXED ? plan->partition_tokens / plan->tile_tokens : 1;
+    p.num_ctas = plan->num_ctas;
+    p.tsplit = TS;
+    p.units = HG * (G / HC);
+    p.heads_per_unit = HC;
+    p.max_slots = plan->max_slots;
+    p.slot_floats = (int64_t)NHvr * s->D + (int64_t)round_up(2 * NHvr, 4);
+    p.off_bar = lay.off_bar;
+    p.off_q = lay.off_q;
+    p.off_stage = lay.off_stage;
+    p.off_scratch = lay.off_scratch;
+    p.off_comb = lay.off_comb;
+    p.row_bytes = row_bytes;
+    p.row_pitch = pitch;
+    p.half_bytes = half;
+    p.q_bytes = q_bytes;
+    p.comb_stride = lay.comb_stride;
+    p.bs_log2 = log2i(s->block_size);
+    p.st_log2 = log2i(plan->tile_tokens);
+    p.spec = (plan->flags & PA_PLAN_NO_SPECULATION) ? 0 : ((plan->flags & PA_PLAN_TEST_MISGUESS) ? 2 : 1);
+    p.test_stall = (plan->flags & PA_PLAN_TEST_STALL) ? 1 : 0;
+    p.lens_cached = s->B <= pa::kLensCache ? 1 : 0;
+    if (tensor_core_dtype(s->dtype)) {
+        const int br = plan->tile_tokens < s->block_size ? plan->tile_tokens : s->block_size;
+        p.use_tmap = 1;
+        p.br_log2 = log2i(br);
+        if (pa_status st = encode_pool_map(&p.tmap_k, k_cache, s, br, HG)) return st;
+        if (pa_status st = encode_pool_map(&p.tmap_v, v_cache, s, br, HG)) return st;
+    }
+    if (pa_status st = ensure_smem_attr(fn, plan->smem_bytes)) return st;
+    L.fn = fn;
+    L.smem_bytes = plan->smem_bytes;
+    L.num_ctas = plan->num_ctas;
+    return PA_OK;
+}
+
+// Queue a prepared decode.  The launch may start while the preceding grid on
+// the stream finishes (programmatic dependent launch): the kernel waits for
+// that grid before its first read of anything it wrote.
+pa_status enqueue_decode(const DecodeLaunch &L, cudaStream_t stream) {
+    if (L.empty) return PA_OK;
+    cudaLaunchConfig_t cfg = {};
+    cfg.gridDim = dim3((unsigned)L.num_ctas);
+    cfg.blockDim = dim3(pa::kDecodeThreads);
+    cfg.dynamicSmemBytes = (size_t)L.smem_bytes;
+    cfg.stream = stream;
+    cudaLaunchAttribute attr[1];
+    attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+    attr[0].val.programmaticStreamSerializationAllowed = 1;
+    cfg.attrs = attr;
+    cfg.numAttrs = 1;
+    cudaError_t ce = cudaLaunchKernelEx(&cfg, L.fn, L.p);
+    if (ce == cudaSuccess) ce = cudaGetLastError();
+    if (ce != cudaSuccess) return fail(PA_ERR_CUDA, "decode launch: %s", cudaGetErrorString(ce));
+    return PA_OK;
+}
+
+pa_status launch_decode(const void *q, const void *k_cache, const void *v_cache, const int32_t *block_tables,
+                        const int32_t *context_lens, float scale, void *out, const pa_shape *s,
+                        const pa_plan_t *plan, void *workspace, size_t workspace_bytes, cudaStream_t stream,
+                        const void *k_new, const void *v_new, const int32_t *slot_mapping) {
+    DecodeLaunch L;
+    if (pa_status st = prepare_decode(q, k_cache, v_cache, block_tables, context_lens, scale, out, s, plan, workspace,
+                                      workspace_bytes, k_new, v_new, slot_mapping, L))
+        return st;
+    return enqueue_decode(L, stream);
+}
+
+}  // namespace
+
+extern "C" {
+
+int32_t pa_version(void) { return 200; }
+
+const char *pa_status_str(pa_status st) {
+    switch (st) {
+        case PA_OK: return "PA_OK";
+        case PA_ERR_INVALID_ARG: return "PA_ERR_INVALID_ARG";
+        case PA_ERR_UNSUPPORTED: return "PA_ERR_UNSUPPORTED";
+        case PA_ERR_CUDA: return "PA_ERR_CUDA";
+        case PA_ERR_WORKSPACE: return "PA_ERR_WORKSPACE";
+    }
+    return "PA_ERR_UNKNOWN";
+}
+
+const char *pa_last_error_message(void) { return g_msg; }
+
+pa_status pa_kv_append(const void *k_new, const void *v_new, const int32_t *slot_mapping, void *k_cache,
+                       void *v_cache, const pa_shape *s, int32_t *device_error, void *stream) {
+    if (pa_status st = check_shape(s)) return st;
+    if (s->B == 0) return ok();
+    if (pa_status st = launch_append(k_new, v_new, slot_mapping, k_cache, v_cache, s, device_error,
+                                     (cudaStream_t)stream))
+        return st;
+    return ok();
+}
+
+pa_status pa_plan(const pa_shape *s, int32_t max_context_len, int32_t partition_tokens, int32_t num_sms,
+                  pa_plan_t *plan) {
+    if (pa_status st = plan_internal(s, max_context_len, partition_tokens, num_sms, plan)) return st;
     return ok();
 }
 
@@ -674,22 +740,36 @@ pa_status no_alloc_workspace(void **out) {
 extern "C" pa_status pa_decode_no_alloc(const void *q, const void *k_cache, const void *v_cache,
                                         const int32_t *block_tables, const int32_t *context_lens, float scale,
                                         void *out, const pa_shape *s, const pa_plan_t *plan, void *stream) {
+    // every host-side check comes before anything touches the array
     if (pa_status st = check_shape(s)) return st;
-    if (!plan) return fail(PA_ERR_INVALID_ARG, "plan is NULL");
+    if (pa_status st = check_plan(s, plan)) return st;
     if (plan->workspace_bytes > kNoAllocWorkspaceBytes)
         return fail(PA_ERR_WORKSPACE, "this plan needs %zu workspace bytes; the built-in workspace holds %zu",
                     plan->workspace_bytes, kNoAllocWorkspaceBytes);
     if (s->B == 0) return ok();
     void *ws = nullptr;
     if (pa_status st = no_alloc_workspace(&ws)) return st;
-    // the array keeps the previous call's contents: the error word and the
-    // merge counters must start at zero
-    const size_t counters = round_up((size_t)s->B * (s->Hkv / (plan->head_group > 0 ? plan->head_group : 1)) * 4, 256);
-    cudaError_t e = cudaMemsetAsync(ws, 0, kWsHeader + counters, (cudaStream_t)stream);
-    if (e != cudaSuccess) return fail(PA_ERR_CUDA, "cudaMemsetAsync: %s", cudaGetErrorString(e));
-    if (pa_status st = launch_decode(q, k_cache, v_cache, block_tables, context_lens, scale, out, s, plan, ws,
-                                     kNoAllocWorkspaceBytes, (cudaStream_t)stream, nullptr, nullptr, nullptr))
+    DecodeLaunch L;
+    if (pa_status st = prepare_decode(q, k_cache, v_cache, block_tables, context_lens, scale, out, s, plan, ws,
+                                      kNoAllocWorkspaceBytes, nullptr, nullptr, nullptr, L))
         return st;
+    // The array keeps the previous call's contents.  The run-time counters
+    // and the merge counters must start at zero (a call that gave up leaves
+    // them as they were); the error word (the first four bytes) is left
+    // alone, so it gathers the errors of every call until it is read and
+    // cleared with pa_no_alloc_device_error.
+    const size_t counters = round_up((size_t)s->B * (s->Hkv / plan->head_group) * 4, 256);
+    if (kWsHeader + counters > plan->workspace_bytes) return fail(PA_ERR_INVALID_ARG, "plan is inconsistent");
+    cudaError_t e = cudaMemsetAsync(static_cast<unsigned char *>(ws) + kWsGrab, 0, kWsHeader - kWsGrab + counters,
+                                    (cudaStream_t)stream);
+    if (e != cudaSuccess) return fail(PA_ERR_CUDA, "cudaMemsetAsync: %s", cudaGetErrorString(e));
+    if (pa_status st = enqueue_decode(L, (cudaStream_t)stream)) return st;
     return ok();
 }
 
+extern "C" pa_status pa_no_alloc_device_error(int32_t clear, int32_t *err_out, void *stream) {
+    if (!err_out) return fail(PA_ERR_INVALID_ARG, "NULL pointer");
+    void *ws = nullptr;
+    if (pa_status st = no_alloc_workspace(&ws)) return st;
+    return pa_get_device_error(ws, clear, err_out, stream);
+}

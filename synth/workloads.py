@@ -165,6 +165,18 @@ class PagedDecodeCase:
         """K+V bytes a decode step reads, counting each request's own reads."""
         return int(self.context_lens.astype(np.int64).sum()) * self.Hkv * self.D * self.elem_bytes * 2
 
+    def kv_bytes_unique(self) -> int:
+        """K+V bytes a decode step must read at least: every physical block
+        once, as many of its rows as the request reading most of it reads
+        (prefix blocks that several tables name are counted once)."""
+        rows = {}
+        for b in range(self.B):
+            L = int(self.context_lens[b])
+            for j in range(-(-L // self.block_size)):
+                blk = int(self.block_tables[b, j])
+                rows[blk] = max(rows.get(blk, 0), min(self.block_size, L - j * self.block_size))
+        return sum(rows.values()) * self.Hkv * self.D * self.elem_bytes * 2
+
     def unique_blocks(self) -> int:
         ids = set()
         for b in range(self.B):
@@ -470,13 +482,16 @@ def prefill_algorithmic(pc: PagedPrefillCase) -> dict:
 
 def algorithmic_bytes(case: PagedDecodeCase) -> dict:
     """Bytes one decode step must move: K+V each request reads, q in, out
-    written, block-table entries and lengths read.  Append bytes (read
-    k_new/v_new, write the slot) are listed separately."""
+    written, block-table entries and lengths read (``decode_total``, each
+    request's own reads; ``decode_unique``, a block several requests share
+    counted once).  Append bytes (read k_new/v_new, write the slot) are
+    listed separately."""
     e = case.elem_bytes
     kv = case.kv_bytes_logical()
     qo = 2 * case.B * case.Hq * case.D * e
     tables = 4 * case.blocks_used() + 4 * case.B
     append = 4 * case.B * case.Hkv * case.D * e + 4 * case.B
-    unique_kv = case.unique_blocks() * case.block_size * case.Hkv * case.D * e * 2
+    unique_kv = case.kv_bytes_unique()
     return {"kv": kv, "q_out": qo, "tables": tables, "decode_total": kv + qo + tables,
-            "append": append, "step_total": kv + qo + tables + append, "unique_kv_upper": unique_kv}
+            "append": append, "step_total": kv + qo + tables + append, "kv_unique": unique_kv,
+            "decode_unique": unique_kv + qo + tables}

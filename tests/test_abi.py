@@ -208,3 +208,42 @@ def test_prefill_plan_budget_over_supported_shapes(D, dtype):
             assert plan.q_tile * G == 128 and plan.kv_tile == 128
             assert 2 <= 2 * plan.stages and plan.smem_bytes + 3072 <= 232448
             assert plan.num_qtiles == -(-100 // plan.q_tile)
+
+
+@pytest.mark.parametrize("field,value", [("head_group", 0), ("head_group", 3), ("stages", 9), ("tile_tokens", 48),
+                                         ("smem_bytes", 1024), ("workspace_bytes", 512), ("max_slots", 1),
+                                         ("num_ctas", 0), ("units_per_warp", 3), ("mode", 7),
+                                         ("max_context_len", 10**6)])
+def test_decode_rejects_a_tampered_plan(field, value):
+    """Every plan field the launch derives anything from is checked against the
+    planner's own output before anything is queued (host only, no GPU)."""
+    s = pa.Shape(4, 16, 8, 128, 16, 64, 16, pa.DTYPE_BF16)
+    plan = pa.pa_plan(s, 256, 0, 148)
+    setattr(plan, field, value)
+    assert _decode(s, plan, ws_bytes=1 << 30) == pa.PA_ERR_INVALID_ARG
+    assert "plan" in pa.pa_last_error_message()
+
+
+def test_no_alloc_rejects_a_stale_plan_before_touching_its_array():
+    """A plan made for one request passed with a 4096-request shape: rejected on
+    the host, before the built-in array is looked up or cleared (this runs
+    without a GPU, so any device call would fail with PA_ERR_CUDA instead)."""
+    s1 = pa.Shape(1, 32, 8, 128, 16, 70000, 64, pa.DTYPE_BF16)
+    plan = pa.pa_plan(s1, 1024, 0, 148)
+    big = pa.Shape(4096, 32, 8, 128, 16, 70000, 64, pa.DTYPE_BF16)
+    st = pa.lib.pa_decode_no_alloc(FAKE, FAKE, FAKE, FAKE, FAKE, ctypes.c_float(0.1), FAKE, ctypes.byref(big),
+                                   ctypes.byref(plan), None)
+    assert st == pa.PA_ERR_INVALID_ARG
+    plan.head_group = 0                                    # tampered: would divide by zero
+    st = pa.lib.pa_decode_no_alloc(FAKE, FAKE, FAKE, FAKE, FAKE, ctypes.c_float(0.1), FAKE, ctypes.byref(s1),
+                                   ctypes.byref(plan), None)
+    assert st == pa.PA_ERR_INVALID_ARG
+
+
+def test_stall_flag_is_a_known_flag():
+    s = pa.Shape(2, 8, 2, 128, 16, 8, 4, pa.DTYPE_BF16)
+    plan = pa.pa_plan(s, 64, 0, 148)
+    plan.flags = pa.PLAN_TEST_STALL
+    assert _decode(s, plan, ws=0) == pa.PA_ERR_WORKSPACE       # passes the flag check
+    plan.flags = 0x8
+    assert _decode(s, plan) == pa.PA_ERR_INVALID_ARG

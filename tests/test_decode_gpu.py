@@ -1,9 +1,9 @@
 """pa_decode against the float64 oracle on the same seeded inputs.
 
 Full outputs at sizes the oracle finishes in seconds (several tiles, ragged
-tails, every split mode); sampled (request, head) outputs at the full sizes
-of the five workloads, in the launch configuration the benchmark times
-(balanced split, one CTA per SM)."""
+tails, every split mode), and every output element at the full sizes of the
+five workloads, in the launch configuration the benchmark times (one fused
+append + decode launch, one CTA per SM)."""
 import dataclasses
 import zlib
 
@@ -12,8 +12,9 @@ import pytest
 import torch
 
 import synth
-from paged_kv_cache_472_b200 import (DEVERR_BLOCK_ID, DEVERR_CONTEXT_LEN, DEVERR_SLOT, PLAN_NO_SPECULATION,
-                                     PLAN_TEST_MISGUESS)
+import paged_kv_cache_472_b200 as pa
+from paged_kv_cache_472_b200 import (DEVERR_BLOCK_ID, DEVERR_CONTEXT_LEN, DEVERR_SLOT, DEVERR_TIMEOUT,
+                                     PLAN_NO_SPECULATION, PLAN_TEST_MISGUESS, PLAN_TEST_STALL)
 from tests import gpu_harness as H
 
 pytestmark = pytest.mark.gpu
@@ -47,23 +48,34 @@ def test_workloads_full_output(orc, cid, batch, partition):
     check_full(orc, case, pt, f"{case.name}/{partition}")
 
 
-# ---- full sizes, sampled outputs, launch configuration of the benchmark ----
-@pytest.mark.parametrize("cid", [2, 3, 4, 5])
-def test_workloads_full_size_sampled(orc, cid):
+# ---- full sizes, every output element, launch configuration of the benchmark ----
+def bench_step(case, partition_tokens, flags=0):
+    """One fused append + decode launch as bench.py times it: the plan for the
+    table's full capacity and the given split."""
+    dev = H.upload(case)
+    dec = H.PagedDecoder(H.shape_of(case), int(case.max_blocks_per_seq * case.block_size), partition_tokens)
+    dec.plan.flags = flags
+    dec.append_decode(dev.k_new, dev.v_new, dev.slot_mapping, dev.q, dev.k_cache, dev.v_cache, dev.block_tables,
+                      dev.context_lens, case.scale, dev.out)
+    torch.cuda.synchronize()
+    return dev, dec
+
+
+@pytest.mark.parametrize("cid", [1, 2, 3, 4, 5])
+def test_workloads_full_size_full_output(orc, cid):
+    """All B x Hq x D outputs of each workload at its full size against the
+    oracle, and the whole pool after the append bit for bit."""
     case = synth.make_config(cid)
-    dev, dec, err = H.run(case, case.partition_tokens)
-    assert err == 0
-    pairs = H.sample_pairs(case, 48, seed=cid)
+    dev, dec = bench_step(case, case.partition_tokens)
+    assert dec.device_error() == 0
     kc, vc = orc.kv_append(case)
-    ref = orc.decode_pairs(case, pairs, kc, vc)
-    got = H.out_f64(dev)[pairs[:, 0], pairs[:, 1]]
-    H.assert_close(got, ref, case.dtype, f"{case.name} sampled")
-    assert np.all(np.isfinite(H.out_f64(dev)))
-    if case.partition_tokens:   # also the balanced split on the same inputs
-        dev2, _, err2 = H.run(case, 0, dev=H.upload(case))
-        assert err2 == 0
-        got2 = H.out_f64(dev2)[pairs[:, 0], pairs[:, 1]]
-        H.assert_close(got2, ref, case.dtype, f"{case.name} sampled balanced")
+    assert H.pool_equal(dev.k_cache, kc, case.dtype) and H.pool_equal(dev.v_cache, vc, case.dtype)
+    ref = oracle_out(orc, case)
+    H.assert_close(H.out_f64(dev), ref, case.dtype, f"{case.name} full size")
+    if case.partition_tokens:   # the balanced split on the same inputs, too
+        dev2, dec2 = bench_step(case, 0)
+        assert dec2.device_error() == 0
+        H.assert_close(H.out_f64(dev2), ref, case.dtype, f"{case.name} full size balanced")
 
 
 def test_split_equals_unsplit(orc):
@@ -164,6 +176,28 @@ def test_context_longer_than_table_is_flagged():
     dev.context_lens = torch.from_numpy(lens).cuda()
     dev, dec, err = H.run(case, 0, dev=dev, max_context_len=80)
     assert err & DEVERR_CONTEXT_LEN
+
+
+def test_bounded_wait_gives_up_and_the_context_survives(orc):
+    """Failure detection on the device: with PA_PLAN_TEST_STALL the first CTA
+    never receives the tiles of its first piece.  Its consumers' bounded wait
+    gives up (about 2 s), PA_DEVERR_TIMEOUT is recorded, the call returns and
+    the CUDA context stays usable: after pa_workspace_init the same decoder
+    gives the oracle's result."""
+    import time
+    case = synth.make_config(2, batch=8)
+    dev, dec, err = H.run(case, 0, flags=PLAN_TEST_STALL)
+    assert err & DEVERR_TIMEOUT, f"device error word {err:#x}"
+    t0 = time.time()
+    torch.cuda.synchronize()                       # nothing is left running
+    assert time.time() - t0 < 1.0
+    dec.plan.flags = 0
+    pa.pa_workspace_init(dec.workspace, dec.workspace.numel())
+    dev.out.fill_(float("nan"))
+    dec.decode(dev.q, dev.k_cache, dev.v_cache, dev.block_tables, dev.context_lens, case.scale, dev.out)
+    torch.cuda.synchronize()
+    assert dec.device_error() == 0
+    H.assert_close(H.out_f64(dev), oracle_out(orc, case), case.dtype, "after a timeout")
 
 
 def test_repeated_calls_reuse_workspace(orc):
