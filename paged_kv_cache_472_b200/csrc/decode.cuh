@@ -58,6 +58,7 @@
 #pragma once
 
 #include <cstddef>
+#include <type_traits>
 
 #include "common.cuh"
 
@@ -73,6 +74,7 @@ constexpr int kPrefixCache = 512;  // requests whose static / dynamic prefix sum
 struct DecodeParams {
     CUtensorMap tmap_k;   // bf16 path: [d, token row, head] view of the pools, 128B swizzle,
     CUtensorMap tmap_v;   // box {64, br, HG}: one block piece of one head group, head-major in smem
+    CUtensorMap tmap_q;   // tensor-core (tcgen05) engine: [d, request*head] view of q, box {64, NHvr}
     const void *q;
     const void *k_cache;
     const void *v_cache;
@@ -115,8 +117,11 @@ struct DecodeParams {
     int32_t spec;         // 0: no speculation; 1: speculate; 2: speculate on wrong guesses (tests)
     int32_t test_stall;   // tests: CTA 0 never fills the stages of its first piece (the bounded waits give up)
     int32_t lens_cached;  // context lengths were copied into shared memory
+    int32_t use_qmap;     // 1: q is staged by tmap_q boxes (128-byte swizzle), one per 64-wide d-chunk
+    int32_t dchunk_major; // 1: a stage is [d-chunk][token row][128 B] (tcgen05 engine, HG = 1)
 };
-static_assert(offsetof(DecodeParams, tmap_k) % 64 == 0 && offsetof(DecodeParams, tmap_v) % 64 == 0,
+static_assert(offsetof(DecodeParams, tmap_k) % 64 == 0 && offsetof(DecodeParams, tmap_v) % 64 == 0 &&
+                  offsetof(DecodeParams, tmap_q) % 64 == 0,
               "tensor maps must be 64-byte aligned");
 
 // ---------------------------------------------------------------------------
@@ -429,6 +434,7 @@ struct __align__(16) DecodeCtl {
     Seg segs[2];               // published by the producer together with q
     Seg pending[kMaxPending];  // pieces whose partial is stored; b < 0 ends the list
     int last[kMaxPending];     // set by the arrival warp: this CTA completed the vr
+    uint32_t tmem_base;        // tcgen05 engine: tensor-memory address of the CTA's allocation
 };
 
 // Barrier of the eight consumer warps on an mbarrier, so that every wait is
@@ -488,6 +494,7 @@ struct CoreEngine {
     static constexpr int TPL = kSubTile / LPH;                   // tokens per softmax lane
     static constexpr int E = Elem<T>::kBytes;
     static constexpr bool kPaddedRows = false;
+    static constexpr bool kTcgen05 = false;
     static constexpr bool kPairs = false;  // subtile_pair not provided
     static constexpr int kUnitsPerWarp = UPW;
     static constexpr int kCombFloats = HC * D + 8;
@@ -736,6 +743,7 @@ struct MmaEngine {
     static constexpr int KS = D / 16;  // k-steps of QK (over d) = m-tiles of PV (over d)
     static constexpr int E = 2;
     static constexpr bool kPaddedRows = true;
+    static constexpr bool kTcgen05 = false;
     static constexpr bool kPairs = PAIR;  // subtile_pair: two full subtiles in one online-softmax step
     static constexpr int kUnitsPerWarp = UPW;
     static constexpr int kCombFloats = 4 * KS * 32 + 4 * 32;  // fragment-ordered o, then m, l
@@ -1139,9 +1147,17 @@ __device__ __forceinline__ void publish(const DecodeParams &p, ProducerState &ps
         ctl.segs[ps.qslot] = s;
         if (s.b >= 0) {
             mbar_arrive_expect_tx(&qfull[ps.qslot], p.q_bytes);
-            const unsigned char *qg = reinterpret_cast<const unsigned char *>(p.q);
-            bulk_g2s(qarea + ps.qslot * p.q_bytes, qg + ((size_t)s.b * p.Hq + (size_t)s.hg * p.NHvr) * D * E,
-                     p.q_bytes, &qfull[ps.qslot]);
+            if (p.use_qmap) {
+                // [d-chunk][head][128 B], 128-byte swizzle: the K-major layout of the S product's B operand
+                const int32_t row = s.b * p.Hq + s.hg * p.NHvr;
+                for (int c = 0; c < D / 64; ++c)
+                    tma_load_2d(qarea + ps.qslot * p.q_bytes + (size_t)c * p.NHvr * 128, &p.tmap_q, c * 64, row,
+                                &qfull[ps.qslot], policy_evict_first());
+            } else {
+                const unsigned char *qg = reinterpret_cast<const unsigned char *>(p.q);
+                bulk_g2s(qarea + ps.qslot * p.q_bytes, qg + ((size_t)s.b * p.Hq + (size_t)s.hg * p.NHvr) * D * E,
+                         p.q_bytes, &qfull[ps.qslot]);
+            }
         } else {
             mbar_arrive(&qfull[ps.qslot]);
         }
@@ -1206,7 +1222,9 @@ __device__ __forceinline__ void issue_tiles(const DecodeParams &p, ProducerState
                 const int32_t head0 = s.hg * p.HG;
 #pragma unroll
                 for (int c2 = 0; c2 < NDC; ++c2) {
-                    const size_t off = (size_t)(lane * NDC + c2) * box_bytes;
+                    // head-major stage: [piece][d-chunk][head][row]; d-chunk-major: [d-chunk][token row]
+                    const size_t off = p.dchunk_major ? (size_t)c2 * p.ST * 128 + (size_t)lane * box_bytes
+                                                      : (size_t)(lane * NDC + c2) * box_bytes;
                     tma_load_3d(kdst + off, &p.tmap_k, c2 * 64, row, head0, &full[ps.stage], pol);
                     tma_load_3d(vdst + off, &p.tmap_v, c2 * 64, row, head0, &full[ps.stage], pol);
                 }
@@ -1504,6 +1522,11 @@ __device__ __forceinline__ void run_arrivals(const DecodeParams &p, DecodeCtl &c
 template <int D, int E>
 __device__ __forceinline__ unsigned char *stage_chunk(unsigned char *tile, int tok, int g_local, int c,
                                                       const DecodeParams &p) {
+    if (p.dchunk_major) {
+        // [d-chunk][token row][128 B] (one KV head), 16-byte slots swizzled by row
+        const int c2 = c >> 3, cc = c & 7;
+        return tile + (size_t)c2 * p.ST * 128 + (size_t)tok * 128 + ((cc ^ (tok & 7)) << 4);
+    }
     if (p.use_tmap) {
         // [piece][d-chunk][head][row][128 B], 16-byte slots swizzled by row
         const int piece = tok >> p.br_log2, r = tok & ((1 << p.br_log2) - 1);
@@ -1704,11 +1727,46 @@ __device__ __forceinline__ void speculative_prefetch(const DecodeParams &p, cons
     }
 }
 
+// Requests with no tokens: out = 0 (the fused step still appends their new
+// token).  Run by the consumer warps, requests dealt round-robin over CTAs.
+template <typename T, int D>
+__device__ __forceinline__ void zero_empty_requests(const DecodeParams &p, const int *lens_s, int tid) {
+    constexpr int E = Elem<T>::kBytes;
+    constexpr int NTH = kConsumerWarps * 32;
+    for (int b = blockIdx.x; b < p.B; b += p.num_ctas) {
+        if (clamped_len(p, lens_s, b) != 0) continue;
+        unsigned char *o = reinterpret_cast<unsigned char *>(p.out) + (size_t)b * p.Hq * D * E;
+        for (int i = tid; i < p.Hq * D / 8; i += NTH) Elem<T>::store_zero8(o + (size_t)i * 8 * E);
+        if (p.fused) {
+            const int sm = p.slot_mapping[b];
+            if (sm >= 0 && (int64_t)sm >= (int64_t)p.num_blocks * p.bs) {
+                if (tid == 0) set_error(p.error, PA_DEVERR_SLOT);
+            } else if (sm >= 0) {
+                const int nvec = p.Hkv * D * E / 16;
+                for (int i = tid; i < 2 * nvec; i += NTH) {
+                    const bool kk = i < nvec;
+                    const uint4 *src = reinterpret_cast<const uint4 *>(kk ? p.k_new : p.v_new) + (size_t)b * nvec;
+                    uint4 *dst = reinterpret_cast<uint4 *>(const_cast<void *>(kk ? p.k_cache : p.v_cache)) +
+                                 (size_t)sm * nvec;
+                    dst[i % nvec] = __ldg(src + i % nvec);
+                }
+            }
+        }
+    }
+}
+
+}  // namespace pa
+
+// the tcgen05 consumer side (large query-head groups)
+#include "decode_tc.cuh"
+
+namespace pa {
+
 // ===========================================================================
 template <typename T, int D, class Engine>
 __global__ void __launch_bounds__(kDecodeThreads, 1) paged_decode_kernel(const __grid_constant__ DecodeParams p) {
     constexpr int E = Elem<T>::kBytes;
-    constexpr int UPW = Engine::kUnitsPerWarp;
+    constexpr bool kTC = Engine::kTcgen05;
     constexpr int NWARPS = kConsumerWarps + 2;
     extern __shared__ __align__(1024) unsigned char smem_raw[];
     __shared__ DecodeCtl ctl;
@@ -1732,18 +1790,31 @@ __global__ void __launch_bounds__(kDecodeThreads, 1) paged_decode_kernel(const _
     unsigned char *qarea = smem + p.off_q;
     unsigned char *stage_base = smem + p.off_stage;
 
+    uint64_t *tcb = cbar + 1;  // tcgen05 engine: sfull[2], pfull[2], odone[2], xchg[2], tdone, tfin
     if (tid == 0) {
         for (int s = 0; s < S; ++s) {
             mbar_init(&full[s], 1);
-            mbar_init(&empty[s], kConsumerWarps);
+            // tcgen05 engine: a stage is released by one commit after its P V product
+            mbar_init(&empty[s], kTC ? 1 : kConsumerWarps);
         }
         for (int i = 0; i < 2; ++i) {
             mbar_init(&qfull[i], 1);
+            // tcgen05 engine: seven warps arrive, the MMA warp's commit after the piece's last S product
             mbar_init(&qempty[i], kConsumerWarps);
         }
         for (int i = 0; i < kMaxPending; ++i) mbar_init(&pdone[i], kConsumerWarps);
         mbar_init(adone, 1);
         mbar_init(cbar, kConsumerWarps);
+        if constexpr (kTC) {
+            for (int i = 0; i < 2; ++i) {
+                mbar_init(&tcb[i], 1);                    // sfull: S product done
+                mbar_init(&tcb[2 + i], kTcSoftmaxWarps);  // pfull: P written
+                mbar_init(&tcb[4 + i], 1);                // odone: P V product done
+                mbar_init(&tcb[6 + i], kTcSoftmaxWarps);  // xchg: per-warp maxima / sums written
+            }
+            mbar_init(&tcb[8], kTcSoftmaxWarps);          // tdone: last tensor-memory read
+            mbar_init(&tcb[9], 1);                        // tfin: every product done
+        }
         ctl.abort = 0;
         ctl.found_b = -1;
         fence_mbarrier_init();
@@ -1751,6 +1822,7 @@ __global__ void __launch_bounds__(kDecodeThreads, 1) paged_decode_kernel(const _
     if (warp == kProducerWarp && lane == 0 && p.use_tmap) {
         prefetch_tensormap(&p.tmap_k);
         prefetch_tensormap(&p.tmap_v);
+        if (p.use_qmap) prefetch_tensormap(&p.tmap_q);
     }
     // ---- while the preceding grid may still run: nothing here reads its output ----
     // Warm the constant cache with the launch parameters, and pull the first
@@ -1896,7 +1968,12 @@ __global__ void __launch_bounds__(kDecodeThreads, 1) paged_decode_kernel(const _
             }
         }
     }
+    if constexpr (kTC) {
+        if (warp == kTcMmaWarp) tmem_alloc(&ctl.tmem_base, Engine::kTmemCols);
+        tc_fence_before();
+    }
     __syncthreads();
+    if constexpr (kTC) tc_fence_after();
 
     const SegIter it = slice_iter(p, ctl, cut, lo, hi, lens_s);
 
@@ -1911,29 +1988,13 @@ __global__ void __launch_bounds__(kDecodeThreads, 1) paged_decode_kernel(const _
     }
 
     // ================= consumer warps =================
-    constexpr int NTH = kConsumerWarps * 32;
-    // requests with no tokens: out = 0 (a fused step still appends their token)
-    for (int b = blockIdx.x; b < p.B; b += p.num_ctas) {
-        if (clamped_len(p, lens_s, b) != 0) continue;
-        unsigned char *o = reinterpret_cast<unsigned char *>(p.out) + (size_t)b * p.Hq * D * E;
-        for (int i = tid; i < p.Hq * D / 8; i += NTH) Elem<T>::store_zero8(o + (size_t)i * 8 * E);
-        if (p.fused) {
-            const int sm = p.slot_mapping[b];
-            if (sm >= 0 && (int64_t)sm >= (int64_t)p.num_blocks * p.bs) {
-                if (tid == 0) set_error(p.error, PA_DEVERR_SLOT);
-            } else if (sm >= 0) {
-                const int nvec = p.Hkv * D * E / 16;
-                for (int i = tid; i < 2 * nvec; i += NTH) {
-                    const bool kk = i < nvec;
-                    const uint4 *src = reinterpret_cast<const uint4 *>(kk ? p.k_new : p.v_new) + (size_t)b * nvec;
-                    uint4 *dst = reinterpret_cast<uint4 *>(const_cast<void *>(kk ? p.k_cache : p.v_cache)) +
-                                 (size_t)sm * nvec;
-                    dst[i % nvec] = __ldg(src + i % nvec);
-                }
-            }
-        }
-    }
-
+    zero_empty_requests<T, D>(p, lens_s, tid);
+    if constexpr (kTC) {
+        run_tc_consumers<T, D, Engine>(p, ctl, lens_s, full, empty, qfull, qempty, pdone, adone, cbar, tcb, qarea,
+                                       stage_base, reinterpret_cast<float *>(smem + p.off_scratch), abort_flag,
+                                       tid, warp, lane);
+    } else {
+    constexpr int UPW = Engine::kUnitsPerWarp;
     const int U = p.units;
     const int tsplit = p.tsplit;
     const int split = (tsplit > 1) ? warp / U : 0;
@@ -2084,6 +2145,7 @@ __global__ void __launch_bounds__(kDecodeThreads, 1) paged_decode_kernel(const _
     __syncwarp();
     if (lane == 0) mbar_arrive(&pdone[npend]);
     flush_pending<T, D>(p, ctl, npend, adone, adone_par, abort_flag, cb, false, tid);
+    }
 }
 
 }  // namespace pa

@@ -89,7 +89,23 @@ KernelFn pick_mma(int upw, int ts) {
     return nullptr;
 }
 
+// tcgen05 engine: one KV head per work item and all its G query heads in one
+// tensor-core tile (heads_per_unit = G >= 16 names it in the plan)
+template <typename T>
+KernelFn pick_tc(int G) {
+    if (G == 16) return pa::paged_decode_kernel<T, 128, pa::TcEngine<T, 16>>;
+    if (G == 32) return pa::paged_decode_kernel<T, 128, pa::TcEngine<T, 32>>;
+    if (G == 64) return pa::paged_decode_kernel<T, 128, pa::TcEngine<T, 64>>;
+    return nullptr;
+}
+
 KernelFn pick_kernel(int dtype, int D, int hc, int upw, int ts) {
+    if (hc >= 16) {
+        if (D != 128 || upw != 1 || ts != 1) return nullptr;
+        if (dtype == PA_DTYPE_BF16) return pick_tc<__nv_bfloat16>(hc);
+        if (dtype == PA_DTYPE_F16) return pick_tc<__half>(hc);
+        return nullptr;
+    }
     if (dtype == PA_DTYPE_BF16)
         return D == 64 ? pick_mma<__nv_bfloat16, 64>(upw, ts)
                        : (D == 128 ? pick_mma<__nv_bfloat16, 128>(upw, ts) : nullptr);
@@ -130,6 +146,20 @@ struct Layout {
 Layout smem_layout(int dtype, int D, int stages, uint32_t q_bytes, uint32_t half_bytes, int hc, int tsplit,
                    int nhvr) {
     Layout l;
+    if (hc >= 16) {
+        // tcgen05 engine: q slots and stages 1024-aligned (128-byte swizzled
+        // boxes), then the softmax warps' exchange area: red[2][4][G],
+        // running maxima [4][G] and rescale factors [4][G]
+        l.off_bar = 0;
+        const uint32_t bar_bytes = (uint32_t)round_up((2 * stages + 4 + pa::kMaxPending + 2 + pa::kTcBars) * 8, 128);
+        l.off_q = (uint32_t)round_up(bar_bytes, 1024);
+        l.off_stage = (uint32_t)round_up(l.off_q + 2 * q_bytes, 1024);
+        l.off_scratch = l.off_stage + (uint32_t)stages * 2 * half_bytes;
+        l.off_comb = (uint32_t)round_up(l.off_scratch + 16u * hc * 4u, 128);
+        l.comb_stride = 0;
+        l.total = l.off_comb + 1024;
+        return l;
+    }
     const bool mma = tensor_core_dtype(dtype);
     l.off_bar = 0;
     // full/empty per stage, q full/empty, piece-done per pending piece, arrivals done,
@@ -177,6 +207,15 @@ struct Mapping {
 
 // Head group HG (KV heads per work item), heads per warp unit HC, units per
 // warp UPW and warps per unit TS (token split) for one shape and engine.
+// The tcgen05 engine takes bf16 / fp16 shapes with D = 128 and a group of
+// 16, 32 or 64 query heads per KV head, with tiles of 128 tokens (so fixed
+// partitions must be multiples of 128).
+bool tc_engine_shape(const pa_shape *s, int partition_tokens) {
+    const int G = s->Hq / s->Hkv;
+    return tensor_core_dtype(s->dtype) && s->D == 128 && (G == 16 || G == 32 || G == 64) &&
+           partition_tokens % pa::kTcTile == 0;
+}
+
 bool choose_mapping(const pa_shape *s, Mapping &m) {
     const int G = s->Hq / s->Hkv;
     const int e = elem_bytes(s->dtype);
@@ -251,6 +290,23 @@ pa_status encode_pool_map(CUtensorMap *map, const void *pool, const pa_shape *s,
     return PA_OK;
 }
 
+// [d, request*head] view of q [B, Hq, D]; the box {64, nh} lands as
+// [head][128 B] with the 128-byte swizzle (one box per 64-wide d-chunk).
+pa_status encode_q_map(CUtensorMap *map, const void *q, const pa_shape *s, int nh) {
+    PFN_cuTensorMapEncodeTiled enc = encode_fn();
+    if (!enc) return fail(PA_ERR_CUDA, "cuTensorMapEncodeTiled is not available");
+    cuuint64_t dims[2] = {(cuuint64_t)s->D, (cuuint64_t)s->B * (cuuint64_t)s->Hq};
+    cuuint64_t strides[1] = {(cuuint64_t)s->D * 2};
+    cuuint32_t box[2] = {64, (cuuint32_t)nh};
+    cuuint32_t estr[2] = {1, 1};
+    const CUtensorMapDataType dt =
+        s->dtype == PA_DTYPE_F16 ? CU_TENSOR_MAP_DATA_TYPE_FLOAT16 : CU_TENSOR_MAP_DATA_TYPE_BFLOAT16;
+    CUresult r = enc(map, dt, 2, const_cast<void *>(q), dims, strides, box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE,
+                     CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+    if (r != CUDA_SUCCESS) return fail(PA_ERR_CUDA, "cuTensorMapEncodeTiled (q) failed (%d)", (int)r);
+    return PA_OK;
+}
+
 int log2i(int x) {
     int l = 0;
     while ((1 << l) < x) ++l;
@@ -281,8 +337,12 @@ pa_status plan_internal(const pa_shape *s, int32_t max_context_len, int32_t part
     }
 
     Mapping mp;
-    if (!choose_mapping(s, mp))
+    const bool tc = tc_engine_shape(s, partition_tokens);
+    if (tc) {
+        mp = {1, G, 1, 1};
+    } else if (!choose_mapping(s, mp)) {
         return fail(PA_ERR_UNSUPPORTED, "no warp mapping for Hq=%d Hkv=%d D=%d", s->Hq, s->Hkv, s->D);
+    }
     const int HG = mp.HG, HC = mp.HC, UPW = mp.UPW, TS = mp.TS;
     const int NHvr = HG * G;
     const int NHG = s->Hkv / HG;
@@ -292,6 +352,7 @@ pa_status plan_internal(const pa_shape *s, int32_t max_context_len, int32_t part
 
     int ST = 16;
     while (ST * 2 <= 256 && (uint32_t)(ST * 2) * row_bytes <= (uint32_t)kStageTargetBytes) ST *= 2;
+    if (tc) ST = pa::kTcTile;  // M of the S product
     int mode = PA_SPLIT_BALANCED;
     if (partition_tokens > 0) {
         if (partition_tokens % 16)
@@ -308,7 +369,7 @@ pa_status plan_internal(const pa_shape *s, int32_t max_context_len, int32_t part
             if (lay.total + kStaticSmem <= (uint32_t)kSmemLimit) break;
         }
         if (stages >= 2) break;
-        if (ST == 16) return fail(PA_ERR_UNSUPPORTED, "shared memory too small for this shape");
+        if (ST == 16 || tc) return fail(PA_ERR_UNSUPPORTED, "shared memory too small for this shape");
         ST /= 2;
     }
 
@@ -484,6 +545,12 @@ pa_status prepare_decode(const void *q, const void *k_cache, const void *v_cache
         p.br_log2 = log2i(br);
         if (pa_status st = encode_pool_map(&p.tmap_k, k_cache, s, br, HG)) return st;
         if (pa_status st = encode_pool_map(&p.tmap_v, v_cache, s, br, HG)) return st;
+    }
+    if (HC >= 16) {
+        // tcgen05 engine: stages [d-chunk][token row], q staged by its own tensor map
+        p.dchunk_major = 1;
+        p.use_qmap = 1;
+        if (pa_status st = encode_q_map(&p.tmap_q, q, s, NHvr)) return st;
     }
     if (pa_status st = ensure_smem_attr(fn, plan->smem_bytes)) return st;
     L.fn = fn;

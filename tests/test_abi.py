@@ -55,7 +55,10 @@ def test_plan_workloads(cid):
     assert plan.stages >= 2
     assert plan.head_group * plan.heads_per_unit >= 1
     units = plan.head_group * G // plan.heads_per_unit
-    assert units == 8 * plan.units_per_warp or units * plan.warps_per_unit == 8
+    if plan.heads_per_unit >= 16:      # tcgen05 engine: one KV head, all its query heads in one tile
+        assert (plan.head_group, plan.heads_per_unit, plan.tile_tokens) == (1, G, 128)
+    else:
+        assert units == 8 * plan.units_per_warp or units * plan.warps_per_unit == 8
     assert plan.tile_tokens >= 16 and plan.tile_tokens & (plan.tile_tokens - 1) == 0
     assert pa.pa_decode_workspace_size(plan) == plan.workspace_bytes
     if c.partition_tokens:
@@ -66,16 +69,19 @@ def test_plan_workloads(cid):
         NV = c.B * (c.Hkv // plan.head_group)
         assert plan.mode == pa.SPLIT_BALANCED and plan.dynamic_share == 0
         assert plan.max_slots == 2 * NV + 148 + 8 * 148 * 64 // 256 + 1
-    expect = {1: (2, 1, 2), 2: (8, 2, 1), 3: (8, 4, 1), 4: (1, 8, 2), 5: (8, 4, 1)}[cid]
+    expect = {1: (2, 1, 2), 2: (8, 2, 1), 3: (8, 4, 1), 4: (1, 32, 1), 5: (8, 4, 1)}[cid]
     assert (plan.head_group, plan.heads_per_unit, plan.warps_per_unit) == expect
 
 
 @pytest.mark.parametrize("Hq,Hkv,D,upw,hc,hg,ts", [
     (32, 32, 128, 1, 1, 8, 1), (16, 16, 64, 2, 1, 16, 1), (64, 16, 64, 2, 4, 16, 1), (32, 16, 64, 2, 2, 16, 1),
-    (64, 16, 128, 1, 4, 8, 1), (4, 1, 128, 1, 4, 1, 8), (8, 1, 128, 1, 8, 1, 8), (64, 1, 128, 1, 8, 1, 1),
-    (2, 2, 64, 1, 1, 2, 4), (1, 1, 64, 1, 1, 1, 8), (32, 1, 128, 1, 8, 1, 2)])
+    (64, 16, 128, 1, 4, 8, 1), (4, 1, 128, 1, 4, 1, 8), (8, 1, 128, 1, 8, 1, 8), (64, 1, 128, 1, 64, 1, 1),
+    (2, 2, 64, 1, 1, 2, 4), (1, 1, 64, 1, 1, 1, 8), (32, 1, 128, 1, 32, 1, 1), (32, 2, 128, 1, 16, 1, 1),
+    (32, 1, 64, 1, 8, 1, 2), (64, 1, 64, 1, 8, 1, 1)])
 def test_plan_head_mappings(Hq, Hkv, D, upw, hc, hg, ts):
-    """bf16 shapes use the tensor-core engine: a unit is one KV head with up to 8 query heads."""
+    """bf16 shapes use the tensor-core engines: with D = 128 and 16, 32 or 64 query heads per KV head,
+    the tcgen05 engine (one KV head per work item, all its query heads in one tile); otherwise warp-level
+    tiles, a unit being one KV head with up to 8 query heads."""
     s = pa.Shape(3, Hq, Hkv, D, 16, 64, 8, pa.DTYPE_BF16)
     plan = pa.pa_plan(s, 128, 0, 148)
     assert (plan.units_per_warp, plan.heads_per_unit, plan.head_group, plan.warps_per_unit) == (upw, hc, hg, ts)
@@ -114,6 +120,19 @@ def test_plan_rejects_bad_partition_and_context():
     with pytest.raises(pa.PagedAttnError) as ei:
         pa.pa_plan(s, 65, 0, 148)          # > max_blocks_per_seq * block_size
     assert ei.value.status == pa.PA_ERR_INVALID_ARG
+
+
+def test_tcgen05_engine_needs_whole_tiles_per_partition():
+    """Fixed partitions that are not a multiple of the 128-token tile keep the warp-level engine."""
+    s = pa.Shape(2, 32, 1, 128, 256, 64, 16, pa.DTYPE_BF16)
+    assert pa.pa_plan(s, 4096, 512, 148).heads_per_unit == 32
+    assert pa.pa_plan(s, 4096, 0, 148).heads_per_unit == 32
+    p64 = pa.pa_plan(s, 4096, 64, 148)
+    assert (p64.heads_per_unit, p64.warps_per_unit) == (8, 2)
+    for G, stages in ((16, 3), (32, 3), (64, 2)):
+        p = pa.pa_plan(pa.Shape(2, G, 1, 128, 16, 64, 16, pa.DTYPE_F16), 256, 0, 148)
+        assert (p.heads_per_unit, p.tile_tokens, p.stages) == (G, 128, stages)
+        assert p.smem_bytes <= 232448 - 10 * 1024
 
 
 def test_fixed_plan_workspace_formula():

@@ -114,11 +114,16 @@ EDGE = [
     ("f16_gqa2", "f16", 16, 8, 128, 16, [300, 17, 1, 1100]),
     ("f16_d64_gqa4", "f16", 32, 8, 64, 32, [513, 64, 2]),
     ("f16_mqa32", "f16", 32, 1, 128, 256, [2000, 255]),
+    # the tcgen05 engine (D = 128, 16 / 32 / 64 query heads per KV head): ragged tiles of 128 tokens
+    ("tc_g64", "bf16", 64, 1, 128, 16, [700, 129, 1, 128]),
+    ("tc_g16_ragged", "bf16", 64, 4, 128, 16, [1, 15, 16, 17, 127, 128, 129, 255, 257]),
+    ("tc_g32_f16_bs64", "f16", 64, 2, 128, 64, [1000, 2, 385]),
+    ("tc_g16_f16_bs256", "f16", 16, 1, 128, 256, [5000, 300, 17]),
 ]
 
 
 @pytest.mark.parametrize("name,dtype,Hq,Hkv,D,bs,lens", EDGE, ids=[e[0] for e in EDGE])
-@pytest.mark.parametrize("pt", [0, 64])
+@pytest.mark.parametrize("pt", [0, 64, 256])
 def test_edge_shapes(orc, name, dtype, Hq, Hkv, D, bs, lens, pt):
     case = synth.build_case(name, dtype=dtype, Hq=Hq, Hkv=Hkv, D=D, block_size=bs, context_lens=lens,
                             seed=zlib.crc32(name.encode()) % 100000, pool="factor", pool_factor=1.25)
@@ -178,15 +183,18 @@ def test_context_longer_than_table_is_flagged():
     assert err & DEVERR_CONTEXT_LEN
 
 
-def test_bounded_wait_gives_up_and_the_context_survives(orc):
+@pytest.mark.parametrize("cid,batch,pt", [(2, 8, 0), (4, 2, 512)])
+def test_bounded_wait_gives_up_and_the_context_survives(orc, cid, batch, pt):
     """Failure detection on the device: with PA_PLAN_TEST_STALL the first CTA
     never receives the tiles of its first piece.  Its consumers' bounded wait
     gives up (about 2 s), PA_DEVERR_TIMEOUT is recorded, the call returns and
     the CUDA context stays usable: after pa_workspace_init the same decoder
-    gives the oracle's result."""
+    gives the oracle's result.  Both consumer designs: warp-level tiles
+    (Qwen3-0.6B shape) and the tcgen05 engine (long-context MQA), which also
+    frees its tensor memory on the way out."""
     import time
-    case = synth.make_config(2, batch=8)
-    dev, dec, err = H.run(case, 0, flags=PLAN_TEST_STALL)
+    case = synth.make_config(cid, batch=batch)
+    dev, dec, err = H.run(case, pt, flags=PLAN_TEST_STALL)
     assert err & DEVERR_TIMEOUT, f"device error word {err:#x}"
     t0 = time.time()
     torch.cuda.synchronize()                       # nothing is left running
