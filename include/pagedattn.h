@@ -94,7 +94,11 @@ typedef struct {
                                  sets 0; a caller may set 1..64 when B <= 512 (the
                                  workspace is sized for 64) */
     int32_t flags;            /* PA_PLAN_* bits; pa_plan sets 0, a caller may set them */
-    int32_t reserved;
+    int32_t split_merge;      /* 1: the pieces of split requests are combined by a second grid
+                                 launched behind the decode grid (one CTA per request and query
+                                 head), chosen when the CTAs outnumber the (request, KV head
+                                 group) pairs 8 to 1, so that each request is spread over many
+                                 CTAs; 0: the CTA that delivers a request's last piece does it */
     int64_t max_slots;        /* partial-result slots in the workspace */
     pa_shape shape;           /* the shape this plan was made for */
     size_t workspace_bytes;   /* bytes pa_decode needs at `workspace` */

@@ -43,7 +43,7 @@ class Plan(ctypes.Structure):
                 ("heads_per_unit", ctypes.c_int32), ("units_per_warp", ctypes.c_int32),
                 ("warps_per_unit", ctypes.c_int32), ("max_context_len", ctypes.c_int32),
                 ("smem_bytes", ctypes.c_int32), ("dynamic_share", ctypes.c_int32), ("flags", ctypes.c_int32),
-                ("reserved", ctypes.c_int32), ("max_slots", ctypes.c_int64),
+                ("split_merge", ctypes.c_int32), ("max_slots", ctypes.c_int64),
                 ("shape", Shape), ("workspace_bytes", ctypes.c_size_t)]
 
     def as_dict(self):

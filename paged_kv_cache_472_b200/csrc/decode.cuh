@@ -117,6 +117,8 @@ struct DecodeParams {
     int32_t spec;         // 0: no speculation; 1: speculate; 2: speculate on wrong guesses (tests)
     int32_t test_stall;   // tests: CTA 0 never fills the stages of its first piece (the bounded waits give up)
     int32_t lens_cached;  // context lengths were copied into shared memory
+    int32_t split_merge;  // 1: split vrs are merged by a second grid (paged_merge_kernel), not in this one
+    struct MergeRecord *records;  // split_merge: per vr, how its pieces map to partial slots
     int32_t use_qmap;     // 1: q is staged by tmap_q boxes (128-byte swizzle), one per 64-wide d-chunk
     int32_t dchunk_major; // 1: a stage is [d-chunk][token row][128 B] (tcgen05 engine, HG = 1)
 };
@@ -321,6 +323,13 @@ __device__ __forceinline__ PieceSlots piece_slots(const DecodeParams &p, const C
     return r;
 }
 
+// What the merge grid needs of a vr: its pieces and their partial slots
+// (PieceSlots), written each launch by the CTA holding the vr's first unit.
+struct MergeRecord {
+    int32_t nparts, ns;
+    int64_t a, b;
+};
+
 // pieces of this CTA's static slice, in list order
 struct SegIter {
     int64_t cur, hi;
@@ -426,8 +435,10 @@ struct GrainIter {
 
 constexpr int kMaxPending = 16;  // split pieces a CTA holds before it merges
 
+constexpr int kMaxWarps = 12;  // the largest CTA of any engine, in warps
+
 struct __align__(16) DecodeCtl {
-    int64_t red[kConsumerWarps + 2][2];
+    int64_t red[kMaxWarps][2];
     Cut cut;
     int64_t found_b, found_excl, found_dexcl;
     int abort;
@@ -495,6 +506,7 @@ struct CoreEngine {
     static constexpr int E = Elem<T>::kBytes;
     static constexpr bool kPaddedRows = false;
     static constexpr bool kTcgen05 = false;
+    static constexpr int kThreads = kDecodeThreads;
     static constexpr bool kPairs = false;  // subtile_pair not provided
     static constexpr int kUnitsPerWarp = UPW;
     static constexpr int kCombFloats = HC * D + 8;
@@ -744,6 +756,7 @@ struct MmaEngine {
     static constexpr int E = 2;
     static constexpr bool kPaddedRows = true;
     static constexpr bool kTcgen05 = false;
+    static constexpr int kThreads = kDecodeThreads;
     static constexpr bool kPairs = PAIR;  // subtile_pair: two full subtiles in one online-softmax step
     static constexpr int kUnitsPerWarp = UPW;
     static constexpr int kCombFloats = 4 * KS * 32 + 4 * 32;  // fragment-ordered o, then m, l
@@ -1305,6 +1318,16 @@ __device__ __forceinline__ void run_producer(const DecodeParams &p, const Cut &k
     while (ps.ok && it.next(p, k, s)) {
         win.prime(p, s, lens_s, lane);  // in flight while q is published
         fused_info(p, s, lane);
+        if (p.split_merge && s.t_begin == 0 && lane == 0) {
+            // the vr's first unit: record how its pieces map to slots for the merge grid
+            const PieceSlots sl = piece_slots(p, k, s);
+            MergeRecord r;
+            r.nparts = s.nparts;
+            r.ns = sl.ns;
+            r.a = sl.a;
+            r.b = sl.b;
+            p.records[(int64_t)s.b * p.NHG + s.hg] = r;
+        }
         publish(p, ps, s, ctl, qfull, qempty, qarea, abort_flag, D, E, lane);
         if (!ps.ok) break;
         if (p.test_stall && blockIdx.x == 0) {
@@ -1368,17 +1391,35 @@ __device__ __forceinline__ void run_producer(const DecodeParams &p, const Cut &k
 //     M[h] = max_i m_i[h]  (base-2 domain; pieces with m = -inf contribute 0).
 // ===========================================================================
 
+// The pieces a merge combines: k -> the k-th piece of the list (first + k * stride
+// in PieceSlots order).
+struct MergeList {
+    PieceSlots slots;
+    int first, stride, n;
+    __device__ __forceinline__ int64_t operator()(int k) const { return slots(first + k * stride); }
+};
+
+// Where a merge writes: into `out` (normalised, dtype of the cache), or into
+// partial slot `slot` as (o, m, l) like a piece.
+struct MergeDst {
+    bool to_slot;
+    int64_t slot;
+    size_t out_head0;  // first head of the vr in out
+};
+
 // From registers: one pass per output element keeps a running maximum, so any
 // number of pieces is combined with eight pieces' loads (o, m, l) in flight.
+// Writing into a slot that is also an input (a group's first piece), every
+// thread's reads come first: o elements are read and written by the same
+// thread, and (m, l) are written after a barrier of the consumer warps.
 template <typename T, int D>
-__device__ __forceinline__ void merge_vr(const DecodeParams &p, const Cut &cut, const Seg &s, int tid) {
+__device__ __forceinline__ bool merge_parts(const DecodeParams &p, const MergeList &L, const MergeDst &dst, int tid,
+                                            ConsumerBarrier &cb, volatile int *abort_flag) {
     constexpr int E = Elem<T>::kBytes;
     constexpr int NTH = kConsumerWarps * 32;
     constexpr int KF = 8;  // pieces per batch of loads
     const int NH = p.NHvr;
-    const int nparts = s.nparts;
-    const size_t out_head0 = (size_t)s.b * p.Hq + (size_t)s.hg * NH;
-    const PieceSlots slots = piece_slots(p, cut, s);
+    const int nparts = L.n;
     const int nq = NH * (D / 4);
     for (int idx0 = tid; idx0 < nq; idx0 += 2 * NTH) {
         constexpr int IT = 2;  // output items per thread per batch
@@ -1403,7 +1444,7 @@ __device__ __forceinline__ void merge_vr(const DecodeParams &p, const Cut &cut, 
                 const int i = i0 + k;
                 int64_t slot = -1;
                 if (i < nparts) {
-                    slot = slots(i);
+                    slot = L(i);
                     if (slot < 0 || slot >= p.max_slots) slot = -1;
                 }
                 sl[k] = slot;
@@ -1452,33 +1493,266 @@ __device__ __forceinline__ void merge_vr(const DecodeParams &p, const Cut &cut, 
 #pragma unroll
         for (int j = 0; j < IT; ++j) {
             if (!act[j]) continue;
-            const float inv = 1.f / den[j];
-            unsigned char *dst =
-                reinterpret_cast<unsigned char *>(p.out) + ((out_head0 + hh[j]) * D + dd[j] * 4) * E;
-            Elem<T>::store2(dst, num[j].x * inv, num[j].y * inv);
-            Elem<T>::store2(dst + 2 * E, num[j].z * inv, num[j].w * inv);
+            if (dst.to_slot) {
+                float *base = p.partials + dst.slot * p.slot_floats;
+                reinterpret_cast<float4 *>(base + (size_t)hh[j] * D)[dd[j]] = num[j];
+            } else {
+                const float inv = 1.f / den[j];
+                unsigned char *o8 =
+                    reinterpret_cast<unsigned char *>(p.out) + ((dst.out_head0 + hh[j]) * D + dd[j] * 4) * E;
+                Elem<T>::store2(o8, num[j].x * inv, num[j].y * inv);
+                Elem<T>::store2(o8 + 2 * E, num[j].z * inv, num[j].w * inv);
+            }
         }
     }
+    if (!dst.to_slot) return true;
+    // (m, l) of the merged piece, once every thread has read the inputs' (m, l):
+    // per head the same maximum over the pieces the o elements were scaled by
+    const bool ok = cb.sync(abort_flag, tid & 31);
+    if (ok) {
+        float *base = p.partials + dst.slot * p.slot_floats;
+        for (int hh = tid; hh < NH; hh += NTH) {
+            float M = -INFINITY;
+            for (int k = 0; k < nparts; ++k) {
+                const int64_t slot = L(k);
+                if (slot >= 0 && slot < p.max_slots) M = fmaxf(M, __ldcg(p.partials + slot * p.slot_floats + NH * D + hh));
+            }
+            float den = 0.f;
+            for (int k = 0; k < nparts; ++k) {
+                const int64_t slot = L(k);
+                if (slot < 0 || slot >= p.max_slots) continue;
+                const float *b = p.partials + slot * p.slot_floats + NH * D;
+                if (b[hh] != -INFINITY) den += exp2f(b[hh] - M) * __ldcg(b + NH + hh);
+            }
+            base[NH * D + hh] = M;
+            base[NH * D + NH + hh] = den;
+        }
+    }
+    return ok;
+}
+
+// The same merge streamed through shared memory, for a CTA's final merges
+// (its pipeline stages are free by then):
+//   * a ring of up to kMergeRing buffers of one piece's o block each is kept
+//     filled by bulk asynchronous copies (one mbarrier per buffer), the first
+//     ones issued before anything else, so that about kMergeRing copies are
+//     in flight for the whole merge;
+//   * meanwhile every piece's (m, l) of every head is loaded; per head the
+//     maximum M and the weights w_i = 2^(m_i - M) (divided by
+//     sum_j 2^(m_j - M) l_j when the merge writes `out`), each thread taking
+//     every (NTH/NH)-th piece of one head;
+//   * each thread adds w_i o_i to its output elements as the buffers land;
+//     the last warp to finish with a buffer refills it with a later piece (a
+//     shared-memory counter per buffer), so no warp waits for another.
+// One exponential per (head, piece), and the merge runs at the copy rate of
+// one SM instead of one round trip per batch of pieces.  The query heads of a
+// vr are a power of two <= 128, so they divide the consumer threads.  Every
+// consumer thread calls it; `ring` holds the ring's mbarriers and `ring_par`
+// their phases (bit b: buffer b).  Returns false if a wait gave up.
+constexpr int kMergeRing = 12;
+
+template <int NTH>
+__host__ __device__ constexpr size_t staged_merge_head_bytes(int nparts, int NH) {
+    // weights and (m, l) [nparts][NH] x 2, two [NTH] reduction rows, the ring's counters
+    return ((size_t)2 * nparts * NH * 4 + 2 * NTH * 4 + kMergeRing * 4 + 1023) & ~(size_t)1023;
+}
+
+template <typename T, int D>
+__device__ __forceinline__ bool merge_parts_staged(const DecodeParams &p, const MergeList &L, const MergeDst &dst,
+                                                   int tid, unsigned char *buf, uint32_t buf_bytes, uint64_t *ring,
+                                                   uint32_t &ring_par, volatile int *abort_flag, ConsumerBarrier &cb) {
+    constexpr int E = Elem<T>::kBytes;
+    constexpr int NTH = kConsumerWarps * 32;
+    constexpr int kMaxItems = 8;  // (head, 4 d) items per thread: NHvr * D <= 8192
+    const int NH = p.NHvr;
+    const int nparts = L.n;
+    const int lane = tid & 31;
+    const uint32_t o_bytes = (uint32_t)NH * D * 4u;
+    const uint32_t o_off = (uint32_t)staged_merge_head_bytes<NTH>(nparts, NH);
+    int nb = o_off < buf_bytes ? (int)((buf_bytes - o_off) / o_bytes) : 0;
+    nb = min(min(nb, kMergeRing), nparts);
+    float *w_s = reinterpret_cast<float *>(buf);  // [nparts][NH]: m, then the weights
+    float *l_s = w_s + (size_t)nparts * NH;      // [nparts][NH]
+    float *red = l_s + (size_t)nparts * NH;      // [2][NTH]
+    int *cnt = reinterpret_cast<int *>(red + 2 * NTH);  // [kMergeRing] warps done with each buffer
+    const int nq = NH * (D / 4);
+    auto issue = [&](int i, int b) {  // piece i into buffer b (one thread)
+        const int64_t slot = L(i);
+        const bool valid = slot >= 0 && slot < p.max_slots;
+        if (valid) {
+            mbar_arrive_expect_tx(&ring[b], o_bytes);
+            bulk_g2s(buf + o_off + (size_t)b * o_bytes, p.partials + slot * p.slot_floats, o_bytes, &ring[b]);
+        } else {
+            mbar_arrive(&ring[b]);  // nothing to copy: the buffer is read as weight 0
+        }
+    };
+    // ---- the first copies, in flight while the weights are worked out ----
+    if (tid == 0) {
+        fence_async_smem();  // earlier reads and writes of buf before the copies overwrite it
+        for (int b = 0; b < nb; ++b) {
+            cnt[b] = 0;
+            issue(b, b);
+        }
+    }
+    // ---- the weights ----
+    for (int x = tid; x < nparts * NH; x += NTH) {
+        const int i = x / NH, h = x - (x / NH) * NH;
+        const int64_t slot = L(i);
+        const bool valid = slot >= 0 && slot < p.max_slots;
+        const float *base = p.partials + (valid ? slot : 0) * p.slot_floats;
+        w_s[x] = valid ? __ldcg(base + (size_t)NH * D + h) : -INFINITY;
+        l_s[x] = valid ? __ldcg(base + (size_t)NH * D + NH + h) : 0.f;
+    }
+    const int h = tid & (NH - 1), sub = tid / NH, nsub = NTH / NH;
+    bool ok = cb.sync(abort_flag, lane);
+    float mloc = -INFINITY;
+    for (int i = sub; i < nparts; i += nsub) mloc = fmaxf(mloc, w_s[i * NH + h]);
+    red[tid] = mloc;
+    if (!cb.sync(abort_flag, lane)) ok = false;
+    float M = -INFINITY;
+    for (int k = 0; k < nsub; ++k) M = fmaxf(M, red[k * NH + h]);
+    float dloc = 0.f;
+    for (int i = sub; i < nparts; i += nsub) {
+        const float m = w_s[i * NH + h];
+        const float w = m == -INFINITY ? 0.f : exp2_fast(m - M);  // pieces with no token: weight 0
+        w_s[i * NH + h] = (L(i) >= 0 && L(i) < p.max_slots) ? w : 0.f;
+        dloc += w * l_s[i * NH + h];
+    }
+    red[NTH + tid] = dloc;
+    if (!cb.sync(abort_flag, lane)) ok = false;
+    float den = 0.f;
+    for (int k = 0; k < nsub; ++k) den += red[NTH + k * NH + h];
+    if (!dst.to_slot) {
+        const float inv = 1.f / den;
+        for (int i = sub; i < nparts; i += nsub) w_s[i * NH + h] *= inv;
+    }
+    if (!cb.sync(abort_flag, lane)) ok = false;
+    // ---- sum_i w_i o_i as the buffers land ----
+    float4 acc[kMaxItems];
+#pragma unroll
+    for (int j = 0; j < kMaxItems; ++j) acc[j] = make_float4(0.f, 0.f, 0.f, 0.f);
+    for (int i = 0; i < nparts && ok; ++i) {
+        const int b = i % nb;
+        if (!mbar_wait(&ring[b], (ring_par >> b) & 1u, abort_flag)) {
+            ok = false;
+            break;
+        }
+        ring_par ^= 1u << b;
+        const float4 *ob = reinterpret_cast<const float4 *>(buf + o_off + (size_t)b * o_bytes);
+        const float *wi = w_s + (size_t)i * NH;
+        const bool filled = L(i) >= 0 && L(i) < p.max_slots;  // else the buffer holds nothing of piece i
+#pragma unroll
+        for (int j = 0; j < kMaxItems; ++j) {
+            const int idx = tid + j * NTH;
+            if (idx < nq && filled) {
+                const float w = wi[idx / (D / 4)];
+                const float4 o = ob[idx];  // o[h][d] at h * D + d: float4 index h * (D/4) + d/4 = idx
+                acc[j].x += w * o.x;
+                acc[j].y += w * o.y;
+                acc[j].z += w * o.z;
+                acc[j].w += w * o.w;
+            }
+        }
+        // the last warp done with buffer b refills it with piece i + nb
+        __syncwarp();
+        if (lane == 0) {
+            __threadfence_block();
+            const int done = atomicAdd(&cnt[b], 1);
+            if (done == kConsumerWarps - 1) {
+                __threadfence_block();
+                cnt[b] = 0;
+                if (i + nb < nparts) {
+                    fence_async_smem();
+                    issue(i + nb, b);
+                }
+            }
+        }
+    }
+    if (!ok && tid == 0) {
+        // a wait gave up: let every copy still in flight into the ring land before
+        // the stages are left (bounded; a buffer with no copy pending times out)
+        volatile int never = 0;
+        for (int b = 0; b < nb; ++b) mbar_wait(&ring[b], (ring_par >> b) & 1u, &never);
+    }
+    // every buffer's last copy has been waited for by every thread
+    if (!cb.sync(abort_flag, lane)) ok = false;
+    if (ok) {
+        if (dst.to_slot) {
+            // a partial: o unnormalised (relative to M), then M and the sum
+            float *base = p.partials + dst.slot * p.slot_floats;
+#pragma unroll
+            for (int j = 0; j < kMaxItems; ++j) {
+                const int idx = tid + j * NTH;
+                if (idx < nq) reinterpret_cast<float4 *>(base)[idx] = acc[j];
+            }
+            if (sub == 0) {
+                base[NH * D + h] = M;
+                base[NH * D + NH + h] = den;
+            }
+        } else {
+            const size_t out0 = dst.out_head0 * D;
+#pragma unroll
+            for (int j = 0; j < kMaxItems; ++j) {
+                const int idx = tid + j * NTH;
+                if (idx < nq) {
+                    unsigned char *o8 = reinterpret_cast<unsigned char *>(p.out) + (out0 + (size_t)idx * 4) * E;
+                    Elem<T>::store2(o8, acc[j].x, acc[j].y);
+                    Elem<T>::store2(o8 + 2 * E, acc[j].z, acc[j].w);
+                }
+            }
+        }
+    }
+    return ok;
+}
+
+// One merge: streamed through the stages when allowed and worth it, else from registers.
+template <typename T, int D>
+__device__ __forceinline__ bool merge_run(const DecodeParams &p, const MergeList &L, const MergeDst &dst, int tid,
+                                          ConsumerBarrier &cb, volatile int *abort_flag, unsigned char *stage_area,
+                                          uint32_t stage_bytes, uint64_t *ring, uint32_t &ring_par) {
+    const size_t need = staged_merge_head_bytes<kConsumerWarps * 32>(L.n, p.NHvr) + (size_t)2 * p.NHvr * D * 4;
+    if (stage_area != nullptr && L.n > 4 && need <= stage_bytes)
+        return merge_parts_staged<T, D>(p, L, dst, tid, stage_area, stage_bytes, ring, ring_par, abort_flag, cb);
+    return merge_parts<T, D>(p, L, dst, tid, cb, abort_flag);
 }
 
 // Merge every vr for which this CTA delivered the last piece.  The arrival
 // warp has counted the arrivals of pieces [0, npend) and signals `adone`
 // once it has; its counting atomics acquire what the other pieces' CTAs
 // released, so their partials are visible to the loads below.  `more`: more
-// pieces follow, so the pending list is handed back afterwards.
+// pieces follow, so the pending list is handed back afterwards.  The final
+// call (`more` false) finds the pipeline stages free and may stream the merge
+// through them (`stage_area`, `stage_bytes`, the ring mbarriers `ring`).
 template <typename T, int D>
 __device__ __forceinline__ bool flush_pending(const DecodeParams &p, DecodeCtl &ctl, int npend, uint64_t *adone,
                                               uint32_t adone_par, volatile int *abort_flag, ConsumerBarrier &cb,
-                                              bool more, int tid) {
-    const bool ok = mbar_wait(adone, adone_par, abort_flag);
+                                              bool more, int tid, unsigned char *stage_area = nullptr,
+                                              uint32_t stage_bytes = 0, uint64_t *ring = nullptr) {
+    bool ok = mbar_wait(adone, adone_par, abort_flag);
     if (ok) {
         const Cut cut = ctl.cut;
-        for (int k = 0; k < npend; ++k) {
+        unsigned char *area = more ? nullptr : stage_area;
+        uint32_t ring_par = 0;
+        // the streamed merge needs every consumer past its tiles (true once adone
+        // has completed for the final list) and its generic accesses to the
+        // stages ordered before the bulk copies
+        if (area) {
+            fence_async_smem();
+            if (!cb.sync(abort_flag, tid & 31)) ok = false;
+        }
+        for (int k = 0; k < npend && ok; ++k) {
             if (!ctl.last[k]) continue;
             const Seg sk = ctl.pending[k];
-            merge_vr<T, D>(p, cut, sk, tid);
+            const MergeDst to_out{false, 0, (size_t)sk.b * p.Hq + (size_t)sk.hg * p.NHvr};
+            ok = merge_run<T, D>(p, MergeList{piece_slots(p, cut, sk), 0, 1, sk.nparts}, to_out, tid, cb, abort_flag,
+                                 area, stage_bytes, ring, ring_par);
             if (tid == 0) p.counters[(int64_t)sk.b * p.NHG + sk.hg] = 0;
+            if (area && !cb.sync(abort_flag, tid & 31)) ok = false;  // the stages are free for the next merge
         }
+    }
+    if (!ok) {
+        *abort_flag = 1;
+        if (tid == 0) set_error(p.error, PA_DEVERR_TIMEOUT);
     }
     if (more) cb.sync(abort_flag, tid & 31);  // pending list free again
     return ok;
@@ -1503,8 +1777,7 @@ __device__ __forceinline__ void run_arrivals(const DecodeParams &p, DecodeCtl &c
             // release: the consumers' partial stores, seen through pdone, before the
             // count; acquire: every other piece's partial before the merge reads them
             const int prev = atomic_add_acq_rel(&p.counters[(int64_t)s.b * p.NHG + s.hg], 1);
-            const int last = prev == s.nparts - 1;
-            ctl.last[k] = last;
+            ctl.last[k] = prev == s.nparts - 1;
         }
         __syncwarp();
         if (++k == kMaxPending) {
@@ -1591,10 +1864,10 @@ struct NewToken {
 // the request holding the slice's first unit (ctl.found_*, which must be -1
 // on entry).  Contains one __syncthreads; the caller synchronises before
 // reading ctl.
+template <int NWARPS>
 __device__ __forceinline__ Cut scan_requests(const DecodeParams &p, int raw, DecodeCtl &ctl, int *lens_s, int *pre_s,
                                              int *pre_d, bool may_dyn, int64_t &lo, int64_t &hi, int tid, int lane,
                                              int warp) {
-    constexpr int NWARPS = kConsumerWarps + 2;
     const int cap = p.max_blocks * p.bs;
     const int b = tid;
     int nu = 0, du = 0;
@@ -1764,10 +2037,12 @@ namespace pa {
 
 // ===========================================================================
 template <typename T, int D, class Engine>
-__global__ void __launch_bounds__(kDecodeThreads, 1) paged_decode_kernel(const __grid_constant__ DecodeParams p) {
+__global__ void __launch_bounds__(Engine::kThreads, 1) paged_decode_kernel(const __grid_constant__ DecodeParams p) {
     constexpr int E = Elem<T>::kBytes;
     constexpr bool kTC = Engine::kTcgen05;
-    constexpr int NWARPS = kConsumerWarps + 2;
+    constexpr int kThreads = Engine::kThreads;
+    constexpr int NWARPS = kThreads / 32;
+    static_assert(NWARPS <= kMaxWarps, "control block");
     extern __shared__ __align__(1024) unsigned char smem_raw[];
     __shared__ DecodeCtl ctl;
     __shared__ int lens_s[kLensCache];
@@ -1786,11 +2061,12 @@ __global__ void __launch_bounds__(kDecodeThreads, 1) paged_decode_kernel(const _
     uint64_t *pdone = qempty + 2;
     uint64_t *adone = pdone + kMaxPending;
     uint64_t *cbar = adone + 1;
+    uint64_t *mbar = cbar + 1;  // the final merges' ring of bulk copies (kMergeRing)
     volatile int *abort_flag = &ctl.abort;
     unsigned char *qarea = smem + p.off_q;
     unsigned char *stage_base = smem + p.off_stage;
 
-    uint64_t *tcb = cbar + 1;  // tcgen05 engine: sfull[2], pfull[2], odone[2], xchg[2], tdone, tfin
+    uint64_t *tcb = mbar + kMergeRing;  // tcgen05 engine: sfull[2], pfull[2], odone[2], xchg[2][2], tdone, tfin
     if (tid == 0) {
         for (int s = 0; s < S; ++s) {
             mbar_init(&full[s], 1);
@@ -1799,21 +2075,24 @@ __global__ void __launch_bounds__(kDecodeThreads, 1) paged_decode_kernel(const _
         }
         for (int i = 0; i < 2; ++i) {
             mbar_init(&qfull[i], 1);
-            // tcgen05 engine: seven warps arrive, the MMA warp's commit after the piece's last S product
-            mbar_init(&qempty[i], kConsumerWarps);
+            // tcgen05 engine: the consumer warps and the P V warp arrive, and the S warp by a
+            // commit after the piece's last S product (Q is read until then)
+            mbar_init(&qempty[i], kTC ? kConsumerWarps + 2 : kConsumerWarps);
         }
         for (int i = 0; i < kMaxPending; ++i) mbar_init(&pdone[i], kConsumerWarps);
         mbar_init(adone, 1);
         mbar_init(cbar, kConsumerWarps);
+        for (int i = 0; i < kMergeRing; ++i) mbar_init(&mbar[i], 1);
         if constexpr (kTC) {
             for (int i = 0; i < 2; ++i) {
                 mbar_init(&tcb[i], 1);                    // sfull: S product done
-                mbar_init(&tcb[2 + i], kTcSoftmaxWarps);  // pfull: P written
+                mbar_init(&tcb[2 + i], kConsumerWarps);   // pfull: P written
                 mbar_init(&tcb[4 + i], 1);                // odone: P V product done
-                mbar_init(&tcb[6 + i], kTcSoftmaxWarps);  // xchg: per-warp maxima / sums written
+                mbar_init(&tcb[6 + i], 4);                // xchg, heads of the first half: four warps
+                mbar_init(&tcb[8 + i], 4);                // xchg, heads of the second half
             }
-            mbar_init(&tcb[8], kTcSoftmaxWarps);          // tdone: last tensor-memory read
-            mbar_init(&tcb[9], 1);                        // tfin: every product done
+            mbar_init(&tcb[10], kConsumerWarps);          // tdone: last tensor-memory read
+            mbar_init(&tcb[11], 2);                       // tfin: every product of both issuers done
         }
         ctl.abort = 0;
         ctl.found_b = -1;
@@ -1830,13 +2109,13 @@ __global__ void __launch_bounds__(kDecodeThreads, 1) paged_decode_kernel(const _
     // CTA its share of the block tables, q and (fused step) the new tokens.
     {
         if (tid == 0) warm_params(p);
-        prefetch_l2_share(p.context_lens, (size_t)p.B * 4, tid, kDecodeThreads, 4);
-        const size_t first = (size_t)blockIdx.x * kDecodeThreads + tid;
-        const size_t stride = (size_t)gridDim.x * kDecodeThreads;
+        prefetch_l2_share(p.context_lens, (size_t)p.B * 4, tid, kThreads, 4);
+        const size_t first = (size_t)blockIdx.x * kThreads + tid;
+        const size_t stride = (size_t)gridDim.x * kThreads;
         prefetch_l2_share(p.block_tables, (size_t)p.B * p.max_blocks * 4, first, stride, 2);
         prefetch_l2_share(p.q, (size_t)p.B * p.Hq * D * E, first, stride, 2);
         if (p.fused) {
-            prefetch_l2_share(p.slot_mapping, (size_t)p.B * 4, tid, kDecodeThreads, 4);
+            prefetch_l2_share(p.slot_mapping, (size_t)p.B * 4, tid, kThreads, 4);
             prefetch_l2_share(p.k_new, (size_t)p.B * p.Hkv * D * E, first, stride, 1);
             prefetch_l2_share(p.v_new, (size_t)p.B * p.Hkv * D * E, first, stride, 1);
         }
@@ -1853,7 +2132,7 @@ __global__ void __launch_bounds__(kDecodeThreads, 1) paged_decode_kernel(const _
     int guess = 0;
     if (speculate) {
         if (tid < p.B) guess = ld_hint(p.context_lens + tid) + (p.spec == 2 ? 1 + (tid & 1) : 0);
-        cut = scan_requests(p, guess, ctl, lens_s, pre_s, pre_d, may_dyn, lo, hi, tid, lane, warp);
+        cut = scan_requests<NWARPS>(p, guess, ctl, lens_s, pre_s, pre_d, may_dyn, lo, hi, tid, lane, warp);
         __syncthreads();
         if (warp == kProducerWarp && p.use_tmap) speculative_prefetch<D>(p, ctl, cut, lo, hi, lens_s, lane);
     }
@@ -1871,12 +2150,12 @@ __global__ void __launch_bounds__(kDecodeThreads, 1) paged_decode_kernel(const _
         if (blockIdx.x == 0 && tid < p.B && (raw < 0 || raw > cap)) set_error(p.error, PA_DEVERR_CONTEXT_LEN);
         if (!__syncthreads_and(speculate && raw == guess)) {
             if (tid == 0) ctl.found_b = -1;
-            cut = scan_requests(p, raw, ctl, lens_s, pre_s, pre_d, may_dyn, lo, hi, tid, lane, warp);
+            cut = scan_requests<NWARPS>(p, raw, ctl, lens_s, pre_s, pre_d, may_dyn, lo, hi, tid, lane, warp);
         }
     } else {
         // any batch size: the totals first, then the prefix sums chunk by chunk
         int64_t t_local = 0, d_local = 0;
-        for (int b = tid; b < p.B; b += kDecodeThreads) {
+        for (int b = tid; b < p.B; b += kThreads) {
             const int raw = p.context_lens[b];
             if (blockIdx.x == 0 && (raw < 0 || raw > cap)) set_error(p.error, PA_DEVERR_CONTEXT_LEN);
             if (p.lens_cached) lens_s[b] = raw;
@@ -1913,7 +2192,7 @@ __global__ void __launch_bounds__(kDecodeThreads, 1) paged_decode_kernel(const _
         // the grains are located with
         if (lo < hi || cut.dyn) {
             int64_t run_s = 0, run_d = 0;
-            for (int base = 0; base < p.B; base += kDecodeThreads) {
+            for (int base = 0; base < p.B; base += kThreads) {
                 const int b = base + tid;
                 int64_t us = 0, ud = 0;
                 if (b < p.B) {
@@ -1988,11 +2267,11 @@ __global__ void __launch_bounds__(kDecodeThreads, 1) paged_decode_kernel(const _
     }
 
     // ================= consumer warps =================
-    zero_empty_requests<T, D>(p, lens_s, tid);
+    if (warp < kConsumerWarps) zero_empty_requests<T, D>(p, lens_s, tid);
     if constexpr (kTC) {
-        run_tc_consumers<T, D, Engine>(p, ctl, lens_s, full, empty, qfull, qempty, pdone, adone, cbar, tcb, qarea,
-                                       stage_base, reinterpret_cast<float *>(smem + p.off_scratch), abort_flag,
-                                       tid, warp, lane);
+        run_tc_consumers<T, D, Engine>(p, ctl, lens_s, full, empty, qfull, qempty, pdone, adone, cbar, mbar, tcb,
+                                       qarea, stage_base, reinterpret_cast<float *>(smem + p.off_scratch),
+                                       abort_flag, tid, warp, lane);
     } else {
     constexpr int UPW = Engine::kUnitsPerWarp;
     const int U = p.units;
@@ -2123,7 +2402,8 @@ __global__ void __launch_bounds__(kDecodeThreads, 1) paged_decode_kernel(const _
         }
 
         // partial piece: leave (m, l, o) in the slot; the arrival warp counts
-        // it once every consumer warp has stored its part
+        // it once every consumer warp has stored its part (the merge grid
+        // combines the pieces instead when split_merge is set)
         const bool slot_ok = s.slot < p.max_slots;
         if (writer && slot_ok) {
             float *base = p.partials + s.slot * p.slot_floats;
@@ -2131,6 +2411,7 @@ __global__ void __launch_bounds__(kDecodeThreads, 1) paged_decode_kernel(const _
             for (int k = 0; k < UPW; ++k) eng.write_partial(unit[k], base, p.NHvr, u_h0[k]);
         }
         if (!slot_ok && tid == 0) set_error(p.error, PA_DEVERR_WORKSPACE);
+        if (p.split_merge) continue;
         __syncwarp();
         if (tid == 0) ctl.pending[npend] = s;
         if (lane == 0) mbar_arrive(&pdone[npend]);
@@ -2144,8 +2425,96 @@ __global__ void __launch_bounds__(kDecodeThreads, 1) paged_decode_kernel(const _
     if (tid == 0) ctl.pending[npend].b = -1;
     __syncwarp();
     if (lane == 0) mbar_arrive(&pdone[npend]);
-    flush_pending<T, D>(p, ctl, npend, adone, adone_par, abort_flag, cb, false, tid);
+    flush_pending<T, D>(p, ctl, npend, adone, adone_par, abort_flag, cb, false, tid, stage_base,
+                        (uint32_t)S * 2u * p.half_bytes, mbar);
     }
+}
+
+// ===========================================================================
+// The merge grid (plans with split_merge): one CTA per (vr, query head),
+// launched behind the decode grid as its programmatic dependent.  The pieces
+// of a vr are spread over the CTA's four warps (warp w takes pieces w, w+4,
+// ...; lane = four consecutive d), each warp keeps a running maximum, sum and
+// weighted o over its pieces with all its loads independent, and the four
+// warps' results are combined by log-sum-exp:
+//     out[h] = sum_i 2^(m_i - M) o_i / sum_i 2^(m_i - M) l_i,  M = max_i m_i
+// (base-2 domain; pieces with m = -inf contribute 0).  A long request split
+// over dozens of CTAs is then merged by as many CTAs as it has heads, all at
+// once, instead of by the one CTA that delivered its last piece.
+constexpr int kMergeThreads = 128;
+
+template <typename T, int D>
+__global__ void __launch_bounds__(kMergeThreads) paged_merge_kernel(const __grid_constant__ DecodeParams p) {
+    constexpr int E = Elem<T>::kBytes;
+    constexpr int NW = kMergeThreads / 32;
+    __shared__ float sm_m[NW], sm_l[NW];
+    __shared__ float4 sm_o[NW][D / 4];
+    grid_dependency_wait();       // the decode grid's partials, records and lengths
+    grid_launch_dependents();
+    const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+    const int64_t cta = blockIdx.x;
+    const int h = (int)(cta % p.NHvr);
+    const int64_t v = cta / p.NHvr;
+    const int b = (int)(v / p.NHG), hg = (int)(v % p.NHG);
+    const int cap = p.max_blocks * p.bs;
+    const int L = p.context_lens[b];
+    if (L <= 0 || L > cap) return;  // no pieces (out already zero, or the length was flagged)
+    const MergeRecord rec = p.records[v];
+    const int n = rec.nparts;
+    if (n <= 1) return;  // written directly by the decode grid
+    const bool act = lane < D / 4;
+    float M = -INFINITY, den = 0.f;
+    float4 num = make_float4(0.f, 0.f, 0.f, 0.f);
+#pragma unroll 4
+    for (int i = warp; i < n; i += NW) {
+        const int64_t slot = i < rec.ns ? rec.a + i : rec.b + (i - rec.ns);
+        if (slot < 0 || slot >= p.max_slots) {
+            if (lane == 0) set_error(p.error, PA_DEVERR_WORKSPACE);
+            continue;
+        }
+        const float *base = p.partials + slot * p.slot_floats;
+        const float mi = __ldcg(base + (size_t)p.NHvr * D + h);
+        const float li = __ldcg(base + (size_t)p.NHvr * D + p.NHvr + h);
+        const float4 o = act ? __ldcg(reinterpret_cast<const float4 *>(base + (size_t)h * D) + lane)
+                             : make_float4(0.f, 0.f, 0.f, 0.f);
+        if (mi == -INFINITY) continue;
+        const float cm = fmaxf(M, mi);
+        const float a = exp2f(M - cm), w = exp2f(mi - cm);  // M = -inf before the first piece: a = 0
+        num.x = num.x * a + w * o.x;
+        num.y = num.y * a + w * o.y;
+        num.z = num.z * a + w * o.z;
+        num.w = num.w * a + w * o.w;
+        den = den * a + w * li;
+        M = cm;
+    }
+    if (lane == 0) {
+        sm_m[warp] = M;
+        sm_l[warp] = den;
+    }
+    if (act) sm_o[warp][lane] = num;
+    __syncthreads();
+    if (warp != 0 || !act) return;
+    float Mx = -INFINITY;
+#pragma unroll
+    for (int w = 0; w < NW; ++w) Mx = fmaxf(Mx, sm_m[w]);
+    float dsum = 0.f;
+    float4 acc = make_float4(0.f, 0.f, 0.f, 0.f);
+#pragma unroll
+    for (int w = 0; w < NW; ++w) {
+        if (sm_m[w] == -INFINITY) continue;
+        const float c = exp2f(sm_m[w] - Mx);
+        const float4 o = sm_o[w][lane];
+        dsum += c * sm_l[w];
+        acc.x += c * o.x;
+        acc.y += c * o.y;
+        acc.z += c * o.z;
+        acc.w += c * o.w;
+    }
+    const float inv = 1.f / dsum;
+    unsigned char *dst = reinterpret_cast<unsigned char *>(p.out) +
+                         ((((size_t)b * p.Hq + (size_t)hg * p.NHvr + h) * D) + (size_t)lane * 4) * E;
+    Elem<T>::store2(dst, acc.x * inv, acc.y * inv);
+    Elem<T>::store2(dst + 2 * E, acc.z * inv, acc.w * inv);
 }
 
 }  // namespace pa

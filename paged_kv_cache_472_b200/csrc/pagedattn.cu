@@ -49,6 +49,11 @@ constexpr size_t kWsGrabDone = 128;    // header offset of the finished-CTA coun
 constexpr int kDynamicShare = 0;
 constexpr int kMaxDynamicShare = 64;
 constexpr int kStageTargetBytes = 32768;  // K bytes per stage (V the same)
+
+// Merge counters of the workspace: one int per (request, head group).
+size_t counters_bytes(int B, int NHG) { return round_up((size_t)B * NHG * 4, 256); }
+// Merge-grid records (plans with split_merge): one per (request, head group).
+size_t records_bytes(int B, int NHG) { return round_up((size_t)B * NHG * sizeof(pa::MergeRecord), 256); }
 constexpr int kMaxStages = 4;
 
 pa_status check_shape(const pa_shape *s) {
@@ -114,6 +119,13 @@ KernelFn pick_kernel(int dtype, int D, int hc, int upw, int ts) {
     return D == 64 ? pick_core<64>(hc, upw) : (D == 128 ? pick_core<128>(hc, upw) : nullptr);
 }
 
+KernelFn pick_merge(int dtype, int D) {
+    if (dtype == PA_DTYPE_BF16)
+        return D == 64 ? pa::paged_merge_kernel<__nv_bfloat16, 64> : pa::paged_merge_kernel<__nv_bfloat16, 128>;
+    if (dtype == PA_DTYPE_F16) return D == 64 ? pa::paged_merge_kernel<__half, 64> : pa::paged_merge_kernel<__half, 128>;
+    return D == 64 ? pa::paged_merge_kernel<float, 64> : pa::paged_merge_kernel<float, 128>;
+}
+
 std::mutex g_attr_mu;
 
 pa_status ensure_smem_attr(KernelFn fn, int bytes) {
@@ -151,7 +163,7 @@ Layout smem_layout(int dtype, int D, int stages, uint32_t q_bytes, uint32_t half
         // boxes), then the softmax warps' exchange area: red[2][4][G],
         // running maxima [4][G] and rescale factors [4][G]
         l.off_bar = 0;
-        const uint32_t bar_bytes = (uint32_t)round_up((2 * stages + 4 + pa::kMaxPending + 2 + pa::kTcBars) * 8, 128);
+        const uint32_t bar_bytes = (uint32_t)round_up((2 * stages + 4 + pa::kMaxPending + 2 + pa::kMergeRing + pa::kTcBars) * 8, 128);
         l.off_q = (uint32_t)round_up(bar_bytes, 1024);
         l.off_stage = (uint32_t)round_up(l.off_q + 2 * q_bytes, 1024);
         l.off_scratch = l.off_stage + (uint32_t)stages * 2 * half_bytes;
@@ -163,8 +175,8 @@ Layout smem_layout(int dtype, int D, int stages, uint32_t q_bytes, uint32_t half
     const bool mma = tensor_core_dtype(dtype);
     l.off_bar = 0;
     // full/empty per stage, q full/empty, piece-done per pending piece, arrivals done,
-    // consumer barrier
-    const uint32_t bar_bytes = (uint32_t)round_up((2 * stages + 4 + pa::kMaxPending + 2) * 8, 128);
+    // consumer barrier, the final merge's copy ring
+    const uint32_t bar_bytes = (uint32_t)round_up((2 * stages + 4 + pa::kMaxPending + 2 + pa::kMergeRing) * 8, 128);
     l.off_q = bar_bytes;
     l.off_stage = (uint32_t)round_up(l.off_q + 2 * q_bytes, 1024);
     l.off_scratch = (uint32_t)round_up(l.off_stage + (size_t)stages * 2 * half_bytes, 128);
@@ -399,9 +411,12 @@ pa_status plan_internal(const pa_shape *s, int32_t max_context_len, int32_t part
         // one partial per (vr, slice) it touches, as in the static list above
         plan->max_slots = (int64_t)s->B * NHG + num_sms;
     }
+    // a second grid merges the split requests when each is likely spread over many CTAs
+    plan->split_merge = (s->B > 0 && (int64_t)num_sms >= 8 * (int64_t)s->B * NHG) ? 1 : 0;
     const size_t slot_floats = (size_t)NHvr * s->D + round_up(2 * NHvr, 4);
-    const size_t counters = round_up((size_t)s->B * NHG * 4, 256);
-    plan->workspace_bytes = kWsHeader + counters + (size_t)plan->max_slots * slot_floats * 4;
+    const size_t counters = counters_bytes(s->B, NHG);
+    const size_t records = plan->split_merge ? records_bytes(s->B, NHG) : 0;
+    plan->workspace_bytes = kWsHeader + counters + records + (size_t)plan->max_slots * slot_floats * 4;
     return PA_OK;
 }
 
@@ -428,7 +443,7 @@ pa_status check_plan(const pa_shape *s, const pa_plan_t *plan) {
         ref.stages != plan->stages || ref.head_group != plan->head_group || ref.heads_per_unit != plan->heads_per_unit ||
         ref.units_per_warp != plan->units_per_warp || ref.warps_per_unit != plan->warps_per_unit ||
         ref.smem_bytes != plan->smem_bytes || ref.max_slots != plan->max_slots ||
-        ref.workspace_bytes != plan->workspace_bytes)
+        ref.split_merge != plan->split_merge || ref.workspace_bytes != plan->workspace_bytes)
         return fail(PA_ERR_INVALID_ARG, "plan is inconsistent with the planner's output for this shape");
     return PA_OK;
 }
@@ -437,8 +452,11 @@ pa_status check_plan(const pa_shape *s, const pa_plan_t *plan) {
 struct DecodeLaunch {
     pa::DecodeParams p;
     KernelFn fn = nullptr;
+    KernelFn merge_fn = nullptr;  // split_merge: the merge grid
+    int merge_ctas = 0;
     int smem_bytes = 0;
     int num_ctas = 0;
+    int threads = pa::kDecodeThreads;
     bool empty = true;  // nothing to launch (B == 0)
 };
 
@@ -492,7 +510,7 @@ pa_status prepare_decode(const void *q, const void *k_cache, const void *v_cache
     p.context_lens = context_lens;
     p.out = out;
     unsigned char *ws = static_cast<unsigned char *>(workspace);
-    const size_t counters = round_up((size_t)s->B * (s->Hkv / HG) * 4, 256);
+    const size_t counters = counters_bytes(s->B, s->Hkv / HG);
     p.error = reinterpret_cast<int32_t *>(ws);
     p.grab = reinterpret_cast<int32_t *>(ws + kWsGrab);
     p.grab_done = reinterpret_cast<int32_t *>(ws + kWsGrabDone);
@@ -502,7 +520,10 @@ pa_status prepare_decode(const void *q, const void *k_cache, const void *v_cache
     p.slot_mapping = slot_mapping;
     p.dyn_num = plan->mode == PA_SPLIT_BALANCED ? plan->dynamic_share : 0;
     p.counters = reinterpret_cast<int32_t *>(ws + kWsHeader);
-    p.partials = reinterpret_cast<float *>(ws + kWsHeader + counters);
+    const size_t records = plan->split_merge ? records_bytes(s->B, s->Hkv / HG) : 0;
+    p.split_merge = plan->split_merge;
+    p.records = reinterpret_cast<pa::MergeRecord *>(ws + kWsHeader + counters);
+    p.partials = reinterpret_cast<float *>(ws + kWsHeader + counters + records);
     p.qscale = scale * 1.4426950408889634f;
     p.B = s->B;
     p.Hq = s->Hq;
@@ -554,6 +575,14 @@ pa_status prepare_decode(const void *q, const void *k_cache, const void *v_cache
     }
     if (pa_status st = ensure_smem_attr(fn, plan->smem_bytes)) return st;
     L.fn = fn;
+    if (plan->split_merge) {
+        L.merge_fn = pick_merge(s->dtype, s->D);
+        const int64_t ctas = (int64_t)s->B * s->Hq;  // one per (request, query head)
+        if (ctas > INT32_MAX) return fail(PA_ERR_UNSUPPORTED, "B*Hq too large for the merge grid");
+        L.merge_ctas = (int)ctas;
+        if (!L.merge_fn) return fail(PA_ERR_INVALID_ARG, "plan names no merge kernel");
+    }
+    L.threads = HC >= 16 ? pa::kTcThreads : pa::kDecodeThreads;
     L.smem_bytes = plan->smem_bytes;
     L.num_ctas = plan->num_ctas;
     return PA_OK;
@@ -566,7 +595,7 @@ pa_status enqueue_decode(const DecodeLaunch &L, cudaStream_t stream) {
     if (L.empty) return PA_OK;
     cudaLaunchConfig_t cfg = {};
     cfg.gridDim = dim3((unsigned)L.num_ctas);
-    cfg.blockDim = dim3(pa::kDecodeThreads);
+    cfg.blockDim = dim3((unsigned)L.threads);
     cfg.dynamicSmemBytes = (size_t)L.smem_bytes;
     cfg.stream = stream;
     cudaLaunchAttribute attr[1];
@@ -577,6 +606,16 @@ pa_status enqueue_decode(const DecodeLaunch &L, cudaStream_t stream) {
     cudaError_t ce = cudaLaunchKernelEx(&cfg, L.fn, L.p);
     if (ce == cudaSuccess) ce = cudaGetLastError();
     if (ce != cudaSuccess) return fail(PA_ERR_CUDA, "decode launch: %s", cudaGetErrorString(ce));
+    if (L.merge_fn) {
+        // the merge grid, also a programmatic dependent: its CTAs wait for the
+        // decode grid's memory before reading any partial
+        cfg.gridDim = dim3((unsigned)L.merge_ctas);
+        cfg.blockDim = dim3(pa::kMergeThreads);
+        cfg.dynamicSmemBytes = 0;
+        ce = cudaLaunchKernelEx(&cfg, L.merge_fn, L.p);
+        if (ce == cudaSuccess) ce = cudaGetLastError();
+        if (ce != cudaSuccess) return fail(PA_ERR_CUDA, "merge launch: %s", cudaGetErrorString(ce));
+    }
     return PA_OK;
 }
 
@@ -825,7 +864,7 @@ extern "C" pa_status pa_decode_no_alloc(const void *q, const void *k_cache, cons
     // them as they were); the error word (the first four bytes) is left
     // alone, so it gathers the errors of every call until it is read and
     // cleared with pa_no_alloc_device_error.
-    const size_t counters = round_up((size_t)s->B * (s->Hkv / plan->head_group) * 4, 256);
+    const size_t counters = counters_bytes(s->B, s->Hkv / plan->head_group);
     if (kWsHeader + counters > plan->workspace_bytes) return fail(PA_ERR_INVALID_ARG, "plan is inconsistent");
     cudaError_t e = cudaMemsetAsync(static_cast<unsigned char *>(ws) + kWsGrab, 0, kWsHeader - kWsGrab + counters,
                                     (cudaStream_t)stream);

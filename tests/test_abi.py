@@ -69,6 +69,7 @@ def test_plan_workloads(cid):
         NV = c.B * (c.Hkv // plan.head_group)
         assert plan.mode == pa.SPLIT_BALANCED and plan.dynamic_share == 0
         assert plan.max_slots == 2 * NV + 148 + 8 * 148 * 64 // 256 + 1
+    assert plan.split_merge == (1 if cid in (1, 4) else 0)   # few (request, KV head group) pairs per CTA
     expect = {1: (2, 1, 2), 2: (8, 2, 1), 3: (8, 4, 1), 4: (1, 32, 1), 5: (8, 4, 1)}[cid]
     assert (plan.head_group, plan.heads_per_unit, plan.warps_per_unit) == expect
 
@@ -140,7 +141,8 @@ def test_fixed_plan_workspace_formula():
     plan = pa.pa_plan(s, 131072, 512, 148)
     assert plan.max_slots == 8 + 148          # one partial per (request, slice)
     slot_floats = 32 * 128 + 64
-    assert plan.workspace_bytes == 256 + 256 + plan.max_slots * slot_floats * 4
+    assert plan.split_merge == 1                # 148 CTAs over 8 requests: a merge grid combines the pieces
+    assert plan.workspace_bytes == 256 + 256 + 256 + plan.max_slots * slot_floats * 4   # + the merge records
 
 
 FAKE = 1 << 20  # aligned, never dereferenced: every call below fails validation first
