@@ -1705,13 +1705,14 @@ __device__ __forceinline__ bool merge_parts_staged(const DecodeParams &p, const 
     return ok;
 }
 
-// One merge: streamed through the stages when allowed and worth it, else from registers.
+// One merge: streamed through the stages when allowed and worth it (more
+// pieces than two batches of register loads), else from registers.
 template <typename T, int D>
 __device__ __forceinline__ bool merge_run(const DecodeParams &p, const MergeList &L, const MergeDst &dst, int tid,
                                           ConsumerBarrier &cb, volatile int *abort_flag, unsigned char *stage_area,
                                           uint32_t stage_bytes, uint64_t *ring, uint32_t &ring_par) {
     const size_t need = staged_merge_head_bytes<kConsumerWarps * 32>(L.n, p.NHvr) + (size_t)2 * p.NHvr * D * 4;
-    if (stage_area != nullptr && L.n > 4 && need <= stage_bytes)
+    if (stage_area != nullptr && L.n > 16 && need <= stage_bytes)
         return merge_parts_staged<T, D>(p, L, dst, tid, stage_area, stage_bytes, ring, ring_par, abort_flag, cb);
     return merge_parts<T, D>(p, L, dst, tid, cb, abort_flag);
 }
@@ -2433,15 +2434,18 @@ __global__ void __launch_bounds__(Engine::kThreads, 1) paged_decode_kernel(const
 // ===========================================================================
 // The merge grid (plans with split_merge): one CTA per (vr, query head),
 // launched behind the decode grid as its programmatic dependent.  The pieces
-// of a vr are spread over the CTA's four warps (warp w takes pieces w, w+4,
-// ...; lane = four consecutive d), each warp keeps a running maximum, sum and
-// weighted o over its pieces with all its loads independent, and the four
-// warps' results are combined by log-sum-exp:
+// of a vr are dealt to the CTA's eight warps (warp w takes pieces w, w+8, ...;
+// lane = four consecutive d); a warp issues the loads of up to kMergeBatch of
+// its pieces before it uses any, so a request split over as many as 64 CTAs
+// costs one round trip to memory.  Each warp keeps a running maximum, sum and
+// weighted o over its pieces, and the warps' results are combined by
+// log-sum-exp:
 //     out[h] = sum_i 2^(m_i - M) o_i / sum_i 2^(m_i - M) l_i,  M = max_i m_i
 // (base-2 domain; pieces with m = -inf contribute 0).  A long request split
 // over dozens of CTAs is then merged by as many CTAs as it has heads, all at
 // once, instead of by the one CTA that delivered its last piece.
-constexpr int kMergeThreads = 128;
+constexpr int kMergeThreads = 256;
+constexpr int kMergeBatch = 8;
 
 template <typename T, int D>
 __global__ void __launch_bounds__(kMergeThreads) paged_merge_kernel(const __grid_constant__ DecodeParams p) {
@@ -2465,26 +2469,40 @@ __global__ void __launch_bounds__(kMergeThreads) paged_merge_kernel(const __grid
     const bool act = lane < D / 4;
     float M = -INFINITY, den = 0.f;
     float4 num = make_float4(0.f, 0.f, 0.f, 0.f);
-#pragma unroll 4
-    for (int i = warp; i < n; i += NW) {
-        const int64_t slot = i < rec.ns ? rec.a + i : rec.b + (i - rec.ns);
-        if (slot < 0 || slot >= p.max_slots) {
-            if (lane == 0) set_error(p.error, PA_DEVERR_WORKSPACE);
-            continue;
+    for (int i0 = warp; i0 < n; i0 += NW * kMergeBatch) {
+        float mi[kMergeBatch], li[kMergeBatch];
+        float4 o[kMergeBatch];
+#pragma unroll
+        for (int k = 0; k < kMergeBatch; ++k) {
+            const int i = i0 + k * NW;
+            const int64_t slot = i < rec.ns ? rec.a + i : rec.b + (i - rec.ns);
+            const bool ok = i < n && slot >= 0 && slot < p.max_slots;
+            if (i < n && !ok && lane == 0) set_error(p.error, PA_DEVERR_WORKSPACE);
+            const float *base = p.partials + (ok ? slot : 0) * p.slot_floats;
+            mi[k] = ok ? __ldcg(base + (size_t)p.NHvr * D + h) : -INFINITY;
+            li[k] = ok ? __ldcg(base + (size_t)p.NHvr * D + p.NHvr + h) : 0.f;
+            o[k] = (ok && act) ? __ldcg(reinterpret_cast<const float4 *>(base + (size_t)h * D) + lane)
+                               : make_float4(0.f, 0.f, 0.f, 0.f);
         }
-        const float *base = p.partials + slot * p.slot_floats;
-        const float mi = __ldcg(base + (size_t)p.NHvr * D + h);
-        const float li = __ldcg(base + (size_t)p.NHvr * D + p.NHvr + h);
-        const float4 o = act ? __ldcg(reinterpret_cast<const float4 *>(base + (size_t)h * D) + lane)
-                             : make_float4(0.f, 0.f, 0.f, 0.f);
-        if (mi == -INFINITY) continue;
-        const float cm = fmaxf(M, mi);
-        const float a = exp2f(M - cm), w = exp2f(mi - cm);  // M = -inf before the first piece: a = 0
-        num.x = num.x * a + w * o.x;
-        num.y = num.y * a + w * o.y;
-        num.z = num.z * a + w * o.z;
-        num.w = num.w * a + w * o.w;
-        den = den * a + w * li;
+        float cm = M;
+#pragma unroll
+        for (int k = 0; k < kMergeBatch; ++k) cm = fmaxf(cm, mi[k]);
+        if (cm == -INFINITY) continue;
+        const float a = exp2f(M - cm);  // M = -inf before the first piece: 0
+        num.x *= a;
+        num.y *= a;
+        num.z *= a;
+        num.w *= a;
+        den *= a;
+#pragma unroll
+        for (int k = 0; k < kMergeBatch; ++k) {
+            const float w = exp2f(mi[k] - cm);  // missing pieces: exp2(-inf) = 0
+            num.x += w * o[k].x;
+            num.y += w * o[k].y;
+            num.z += w * o[k].z;
+            num.w += w * o[k].w;
+            den += w * li[k];
+        }
         M = cm;
     }
     if (lane == 0) {
