@@ -257,10 +257,10 @@ pa_status pa_decode_no_alloc(const void *q, const void *k_cache, const void *v_c
  * group Hq/Hkv that is a power of two <= 128.
  */
 typedef struct {
-    int32_t q_tile;          /* new tokens per CTA (q_tile * Hq/Hkv rows) */
+    int32_t q_tile;          /* new tokens per query tile (q_tile * Hq/Hkv rows); a CTA takes two */
     int32_t kv_tile;         /* keys per pipeline stage */
     int32_t stages;
-    int32_t num_qtiles;      /* tiles of q_tile tokens per request the grid covers */
+    int32_t num_qtiles;      /* CTA tiles (two query tiles) per request the grid covers */
     int32_t max_new_tokens;
     int32_t smem_bytes;
     pa_shape shape;

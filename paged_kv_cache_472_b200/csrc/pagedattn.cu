@@ -719,7 +719,7 @@ pa_status pa_prefill_plan(const pa_shape *s, int32_t max_new_tokens, pa_prefill_
     if (s->Hkv > 65535 || s->B > 65535) return fail(PA_ERR_UNSUPPORTED, "Hkv or B above 65535");
     const int QT = pa::kPrefillRows / G;
     const int KT = pa::kPrefillKT;
-    const uint32_t q_bytes = (uint32_t)pa::kPrefillRows * s->D * 2;
+    const uint32_t q_bytes = (uint32_t)pa::kPrefillQTiles * pa::kPrefillRows * s->D * 2;  // both query tiles
     const uint32_t slot = (uint32_t)KT * s->D * 2;
     int nslots = pa::kPrefillMaxSlots;
     uint32_t total = 0;
@@ -732,7 +732,7 @@ pa_status pa_prefill_plan(const pa_shape *s, int32_t max_new_tokens, pa_prefill_
     plan->kv_tile = KT;
     plan->stages = nslots / 2;
     plan->max_new_tokens = max_new_tokens;
-    plan->num_qtiles = (max_new_tokens + QT - 1) / QT;
+    plan->num_qtiles = (max_new_tokens + pa::kPrefillQTiles * QT - 1) / (pa::kPrefillQTiles * QT);
     plan->smem_bytes = (int32_t)total;
     plan->shape = *s;
     return ok();
@@ -761,7 +761,9 @@ pa_status pa_prefill(const void *q, const void *k_cache, const void *v_cache, co
     p.context_lens = context_lens;
     p.query_start = query_start;
     p.error = device_error;
-    p.qscale = std::fabs(scale) * 1.4426950408889634f;
+    // kept above zero: a masked score enters the kernel as -inf and must give
+    // weight 0; with scale 0 every score times 2^-100 still rounds 2^x to 1
+    p.qscale = std::fmax(std::fabs(scale) * 1.4426950408889634f, 0x1p-100f);
     p.qflip = scale < 0.f ? 0x80008000u : 0u;
     p.B = s->B;
     p.Hq = s->Hq;
@@ -777,7 +779,7 @@ pa_status pa_prefill(const void *q, const void *k_cache, const void *v_cache, co
     p.br_log2 = log2i(br);
     p.nslots = 2 * plan->stages;
     p.num_qtiles = plan->num_qtiles;
-    p.off_ring = (uint32_t)pa::kPrefillRows * s->D * 2;
+    p.off_ring = (uint32_t)pa::kPrefillQTiles * pa::kPrefillRows * s->D * 2;
     p.slot_bytes = (uint32_t)pa::kPrefillKT * s->D * 2;
     if (pa_status st = encode_pool_map(&p.tmap_k, k_cache, s, br, 1)) return st;
     if (pa_status st = encode_pool_map(&p.tmap_v, v_cache, s, br, 1)) return st;

@@ -9,40 +9,44 @@
 // head h / (Hq/Hkv).  This is the step before decode (the MinivLLM review's
 // prefill path), read straight from the pages like the decode.
 //
-// Work decomposition: one CTA per (request, KV head, tile of QT new tokens).
-// Its 128 rows are the QT tokens x G query heads of that KV head (row r =
-// token r / G, head r % G), so every K/V tile staged in shared memory serves
-// the whole head group.  The CTA streams keys 0 .. pos(last token) in tiles
-// of 128 and masks, per row, the keys past the row's own position.  Tiles
+// Work decomposition: one CTA per (request, KV head, tile of 2 QT new
+// tokens), as two query tiles A and B of QT tokens each.  A query tile's 128
+// rows are its QT tokens x the G query heads of the KV head (row r = token
+// r / G, head r % G), so every K/V tile staged in shared memory serves both
+// query tiles and the whole head group.  The CTA streams keys 0 .. pos(last
+// token of the tile) in tiles of 128 and masks, per row, the keys past the
+// row's own position; query tile A stops at its own last position.  Tiles
 // holding the latest tokens see the most keys; the grid runs them first.
 //
 // Inside a CTA (5th-generation tensor cores, accumulators in tensor memory):
 //   warps 0,10 producers of K and of V: each walks the block table (one tile
 //              ahead) and fills its own ring of slots with tensor-map boxes
 //              ([d-block][key][128 B], 128-byte swizzle: the canonical K-major
-//              layout for K, MN-major for V), so K never queues behind a V
-//              slot that a product still holds;
-//   warp 1     allocates tensor memory; one lane issues every tcgen05.mma:
-//                S_j = Q K_j^T   (M 128 rows, N 128 keys, into one of three
-//                                 S buffers, up to three tiles ahead of the
-//                                 softmax),
-//                O  += P_j V_j   (M 128 rows, N = D, K = keys; P read from
+//              layout for K, MN-major for V);
+//   warp 1     allocates tensor memory; one lane issues every tcgen05.mma,
+//              alternating between the query tiles so that the tensor core
+//              works on one while the softmax of the other runs:
+//                S_t = Q_t K_j^T (M 128 rows, N 128 keys, into query tile t's
+//                                 S buffer),
+//                O_t += P_t V_j  (M 128 rows, N = D, K = keys; P read from
 //                                 tensor memory, where the softmax wrote it
-//                                 over S_j, in two 16-bit parts, high and
+//                                 over S_t, in two 16-bit parts, high and
 //                                 low, as in decode);
-//   warps 2-9  softmax: two threads per row (tensor-memory lane = row), one
-//              for each half of the key columns (and of the O columns).  They
-//              copy the q rows into the swizzled Q tile, then per key tile
-//              read their half of the S row, mask, exchange the row maximum
-//              with the partner (a two-warp mbarrier), run the fp32 online
-//              softmax in the base-2 domain, write P (high and low parts) into
-//              the S buffer they read, and at the end combine the two row
-//              sums, read O, divide and store the output row.
-// The tensor pipe runs its products in issue order, so S_{j+3} (issued after
-// P_j V_j) never overwrites P_j before it is read, and the softmax of tile j
-// never waits for P_{j-1} V_{j-1}: only a rescale of O does.
-// The running maximum is moved only when a tile's maximum exceeds it by more
-// than 2^8 (weights stay below 256, exact in fp32 and safe in 16 bits); the
+//   warps 2-9  softmax: warps 2-5 take query tile A, warps 6-9 query tile B,
+//              one thread per row (tensor-memory lane = row, the warp's lane
+//              quarter fixed by its index), so a row's maximum and sum never
+//              leave the thread.  They copy their q rows into the swizzled Q
+//              tile, then per key tile load the whole S row into registers
+//              (one 128-column load), take its maximum, run the fp32 online
+//              softmax in the base-2 domain, write P (high and low parts)
+//              over S, and at the end read O, divide and store the row.
+// The issuing lane keeps every operand descriptor in registers and adds
+// offsets to it: the tensor core queues only a few products ahead, so the
+// issuer's own latency between products is idle tensor time.
+// The tensor pipe runs its products in issue order, so S_t of the next key
+// tile (issued after P_t V_j) never overwrites P_t before it is read.  The
+// running maximum is moved only when a tile's maximum exceeds it by more than
+// 2^8 (weights stay below 256, exact in fp32 and safe in 16 bits); the
 // rescale of O in tensor memory is then rare.  The final division uses the
 // same maximum as every weight, so the result is the plain softmax.
 #pragma once
@@ -53,13 +57,13 @@
 
 namespace pa {
 
-constexpr int kPrefillRows = 128;     // rows per CTA: M of every tensor-core product
+constexpr int kPrefillRows = 128;     // rows per query tile: M of every tensor-core product
+constexpr int kPrefillQTiles = 2;     // query tiles per CTA, sharing every K/V tile
 constexpr int kPrefillKT = 128;       // keys per tile: N of S, K of P V
 constexpr int kPrefillSoftmaxWarps = 8;
 constexpr int kPrefillVWarp = 2 + kPrefillSoftmaxWarps;             // the V producer
 constexpr int kPrefillThreads = (3 + kPrefillSoftmaxWarps) * 32;  // K producer, MMA, softmax, V producer
-constexpr int kPrefillSBufs = 3;      // S / P buffers in tensor memory
-constexpr int kPrefillTmemCols = 512; // S / P buffers (3 x 128 columns) + O (D columns), power of two
+constexpr int kPrefillTmemCols = 512; // S / P of both query tiles (2 x 128 columns) + O of both (2 x D)
 constexpr int kPrefillMaxSlots = 8;   // K / V ring slots
 constexpr float kPrefillRescaleLog2 = 8.f;
 
@@ -75,11 +79,11 @@ struct PrefillParams {
     float qscale;        // |scale| * log2(e)
     uint32_t qflip;      // 0x80008000 when scale < 0: q enters negated, so scores keep their order
     int32_t B, Hq, Hkv, G, g_log2, bs, bs_log2, num_blocks, max_blocks;
-    int32_t QT;          // new tokens per CTA (QT * G = kPrefillRows)
+    int32_t QT;          // new tokens per query tile (QT * G = kPrefillRows); a CTA takes 2 QT
     int32_t br_log2;     // rows of one box = min(kPrefillKT, bs)
     int32_t nslots;      // ring slots, even: K of tile j in slot j mod (nslots/2), V of tile j in the second half
-    int32_t num_qtiles;  // tiles of QT tokens the grid covers per request
-    uint32_t off_ring, slot_bytes;  // shared-memory layout (from the 1024-aligned base; Q at 0)
+    int32_t num_qtiles;  // CTA tiles of 2 QT tokens the grid covers per request
+    uint32_t off_ring, slot_bytes;  // shared-memory layout (from the 1024-aligned base; Q tiles at 0)
 };
 static_assert(offsetof(PrefillParams, tmap_k) % 64 == 0 && offsetof(PrefillParams, tmap_v) % 64 == 0,
               "tensor maps must be 64-byte aligned");
@@ -92,69 +96,77 @@ __global__ void __launch_bounds__(kPrefillThreads, 1) paged_prefill_kernel(const
     constexpr int KS = D / 16;                         // k-steps of S over d
     constexpr int NDC = D / 64;                        // 64-wide d-blocks
     constexpr uint32_t kBlk = kPrefillRows * 128u;     // one 64-column block of a 128-row operand: 16 KB
+    constexpr uint32_t kQTile = kPrefillRows * D * 2;  // one query tile in shared memory
     constexpr uint32_t kSlotBlk = KT * 128u;           // one d-block of a K / V slot
     constexpr bool kBf16 = std::is_same<T, __nv_bfloat16>::value;
     constexpr uint32_t kIdescPV = umma_idesc(kPrefillRows, D, false, true, kBf16);
-    constexpr uint32_t kColO = kPrefillSBufs * KT;     // tensor-memory column of O
-    static_assert(kPrefillSBufs * KT + D <= kPrefillTmemCols, "tensor memory");
+    constexpr uint32_t kColO = kPrefillQTiles * KT;    // tensor-memory column of O of query tile 0
+    static_assert(kPrefillQTiles * (KT + D) <= kPrefillTmemCols, "tensor memory");
+    static_assert(kBlk == kSlotBlk, "Q and K blocks share the k-step offsets");
     extern __shared__ __align__(1024) unsigned char smem_raw[];
     unsigned char *smem = smem_raw;  // the plan leaves no room to realign: checked below
-    // mbarriers: full[], empty[] (ring), sfull[3], pfull[2], odone[2], qfull, fin, xchg[4][2]
-    constexpr int kOffSfull = 2 * kPrefillMaxSlots, kOffPfull = kOffSfull + kPrefillSBufs;
-    constexpr int kOffOdone = kOffPfull + 2, kOffQfull = kOffOdone + 2, kOffFin = kOffQfull + 1;
-    constexpr int kOffXchg = kOffFin + 1, kBars = kOffXchg + 8;
+    // mbarriers: full[], empty[] (ring), sfull[2] (per query tile), pfull[2][2] and
+    // odone[2][2] (per query tile and key-tile parity), qfull, fin
+    constexpr int kOffSfull = 2 * kPrefillMaxSlots, kOffPfull = kOffSfull + 2;
+    constexpr int kOffOdone = kOffPfull + 4, kOffQfull = kOffOdone + 4, kOffFin = kOffQfull + 1;
+    constexpr int kBars = kOffFin + 1;
     __shared__ uint64_t bars[kBars];
-    __shared__ float red_s[2][2][kPrefillRows];  // [tile parity][column half][row]: row max / row sum
     __shared__ uint32_t tmem_base_s;
     __shared__ volatile int abort_s;
 
     const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
     const int NH = p.nslots / 2;  // K slots 0 .. NH-1, V slots NH .. 2NH-1
     uint64_t *full = bars, *empty = bars + kPrefillMaxSlots;
-    // sfull (one per S buffer), pfull and odone (one per tile parity): no
-    // barrier's phase can run two ahead of a thread that waits on it by parity
-    uint64_t *sfull = bars + kOffSfull, *pfull = bars + kOffPfull, *odone = bars + kOffOdone;
+    uint64_t *sfull = bars + kOffSfull;  // [query tile]: its S product done (one phase per key tile)
+    uint64_t *pfull = bars + kOffPfull;  // [query tile][key-tile parity]: P written
+    uint64_t *odone = bars + kOffOdone;  // [query tile][key-tile parity]: P V product done
     uint64_t *qfull = bars + kOffQfull, *fin = bars + kOffFin;
-    uint64_t *xchg = bars + kOffXchg;  // [lane quarter][parity]: the two softmax warps of the same rows
     volatile int *abort_flag = &abort_s;
 
     if (smem_u32(smem_raw) & 1023u) {  // the 128-byte swizzle needs 1024-byte aligned tiles
         if (tid == 0) set_error(p.error, PA_DEVERR_SMEM);
         return;
     }
-    // ---- the tile: request, KV head, new tokens [t0, t0 + ntok) ----
+    // ---- the CTA's tile: request, KV head, new tokens [t0, t0 + ntok) ----
     const int b = blockIdx.z, g = blockIdx.y;
     const int qt = p.num_qtiles - 1 - (int)blockIdx.x;  // latest (heaviest) tiles first
     const int cap = p.max_blocks * p.bs;
     const int L = p.context_lens[b];
     const int q0 = p.query_start[b];
     const int n = p.query_start[b + 1] - q0;
-    if (L < 0 || L > cap || n < 0 || n > L || n > p.num_qtiles * p.QT) {
+    if (L < 0 || L > cap || n < 0 || n > L || n > p.num_qtiles * kPrefillQTiles * p.QT) {
         if (tid == 0 && blockIdx.x == 0 && blockIdx.y == 0) set_error(p.error, PA_DEVERR_CONTEXT_LEN);
         return;
     }
-    const int t0 = qt * p.QT;
+    const int t0 = qt * kPrefillQTiles * p.QT;
     if (t0 >= n) return;
-    const int ntok = min(p.QT, n - t0);
-    const int pos0 = L - n + t0;            // position of the tile's first token
-    const int kend = pos0 + ntok;           // keys 0 .. kend-1 are visible to some row
-    const int ntiles = (kend + KT - 1) / KT;
-    const int nk_last = kend - (ntiles - 1) * KT;  // keys of the last tile holding visible keys
-    const int n16_last = (nk_last + 15) >> 4;      // its 16-key groups
+    // query tile t: tokens t0 + t QT .. + ntok_t - 1 (ntok_t may be 0 for tile B)
+    int ntok_q[kPrefillQTiles], nkt[kPrefillQTiles], n16_q[kPrefillQTiles];
+#pragma unroll
+    for (int t = 0; t < kPrefillQTiles; ++t) {
+        ntok_q[t] = max(0, min(p.QT, n - (t0 + t * p.QT)));
+        // keys 0 .. kend_t - 1 are visible to some row of query tile t
+        const int kend_t = ntok_q[t] > 0 ? L - n + t0 + t * p.QT + ntok_q[t] : 0;
+        nkt[t] = (kend_t + KT - 1) / KT;
+        n16_q[t] = nkt[t] > 0 ? (kend_t - (nkt[t] - 1) * KT + 15) >> 4 : 0;  // 16-key groups of its last tile
+    }
+    const int ntiles = max(nkt[0], nkt[1]);  // key tiles the CTA streams
+    const int kend = L - n + t0 + ntok_q[0] + ntok_q[1];
 
     if (tid == 0) {
         for (int s = 0; s < 2 * NH; ++s) {
             mbar_init(&full[s], 1);
             mbar_init(&empty[s], 1);
         }
-        for (int i = 0; i < kPrefillSBufs; ++i) mbar_init(&sfull[i], 1);
-        for (int i = 0; i < 2; ++i) {
-            mbar_init(&pfull[i], kPrefillSoftmaxWarps);
-            mbar_init(&odone[i], 1);
+        for (int t = 0; t < kPrefillQTiles; ++t) {
+            mbar_init(&sfull[t], 1);
+            for (int par = 0; par < 2; ++par) {
+                mbar_init(&pfull[t * 2 + par], 4);  // the four warps of query tile t
+                mbar_init(&odone[t * 2 + par], 1);
+            }
         }
         mbar_init(qfull, kPrefillSoftmaxWarps);
         mbar_init(fin, 1);
-        for (int i = 0; i < 8; ++i) mbar_init(&xchg[i], 2);
         abort_s = 0;
         fence_mbarrier_init();
     }
@@ -226,61 +238,111 @@ __global__ void __launch_bounds__(kPrefillThreads, 1) paged_prefill_kernel(const
     } else if (warp == 1) {
         // ================= MMA issue (one lane) =================
         if (lane == 0) {
-            const uint32_t q_addr = smem_u32(smem), r_addr = smem_u32(ring);
+            const uint32_t r_addr = smem_u32(ring);
+            // Operand descriptors are built once; a shared-memory offset (every
+            // address here is below 256 KB) adds to the start-address field as
+            // offset / 16, so each product below costs one add per operand.
+            const uint64_t qdesc = umma_desc_sw128(smem_u32(smem), 16, 1024);        // Q tiles, K-major
+            const uint64_t kdesc = umma_desc_sw128(r_addr, 16, 1024);                // K slots, K-major
+            const uint64_t vdesc = umma_desc_sw128(r_addr, kSlotBlk, 1024);          // V slots, MN-major
+            const uint32_t slot16 = p.slot_bytes >> 4;
             bool ok = mbar_wait(qfull, 0u, abort_flag);
             bool issued_any = false;
-            // O += P_i V_i for tile i (P high part, then low part)
-            auto pv = [&](int i) {
+            // Everything a product needs is in registers before the loop: the
+            // issuing thread's own latency between products is tensor-core idle
+            // time, since the core queues only a few products ahead.
+            const int nk0 = nkt[0], nk1 = nkt[1];
+            const uint32_t idesc_full = umma_idesc(kPrefillRows, KT, false, false, kBf16);
+            const uint32_t idesc_last0 = umma_idesc(kPrefillRows, n16_q[0] * 16, false, false, kBf16);
+            const uint32_t idesc_last1 = umma_idesc(kPrefillRows, n16_q[1] * 16, false, false, kBf16);
+            // S_t = Q_t K_j^T into query tile t's buffer (K of tile j in slot sk, fill
+            // parity par); the last user of the K slot releases it
+            auto s_issue = [&](auto tc, int j, int sk, uint32_t par) {
+                constexpr int t = decltype(tc)::value;
                 if (!ok) return;
-                const int sv = NH + i % NH;
-                const uint32_t par = (uint32_t)(i / NH) & 1u;
-                if (!mbar_wait(&pfull[i & 1], (uint32_t)(i >> 1) & 1u, abort_flag) ||
-                    !mbar_wait(&full[sv], par, abort_flag)) {
-                    ok = false;
-                    return;
-                }
-                tc_fence_after();
-                const int n16 = i == ntiles - 1 ? n16_last : KT / 16;
-                const uint32_t vb = r_addr + (uint32_t)sv * p.slot_bytes;
-                // P_i in buffer i % 3: keys 16kk .. 16kk+15 in columns 16kk .. 16kk+7
-                // (high parts) and 16kk+8 .. 16kk+15 (low parts), two keys per column
-                const uint32_t pa = tmem + (uint32_t)(i % kPrefillSBufs) * KT;
-                for (int kk = 0; kk < n16; ++kk) {
-                    const uint64_t bd = umma_desc_sw128(vb + kk * 2048, kSlotBlk, 1024);
-                    umma_f16_ts(tmem + kColO, pa + kk * 16, bd, kIdescPV, (i > 0 || kk > 0) ? 1u : 0u);
-                    umma_f16_ts(tmem + kColO, pa + kk * 16 + 8, bd, kIdescPV, 1u);
-                }
-                umma_commit(&odone[i & 1]);
-                umma_commit(&empty[sv]);
-                issued_any = true;
-            };
-            // S_j = Q K_j^T into buffer j % 3, which held P_{j-3}: issued after P_{j-3} V_{j-3}
-            auto s_issue = [&](int j) {
-                if (!ok) return;
-                const int sk = j % NH;
-                const uint32_t par = (uint32_t)(j / NH) & 1u;
                 if (!mbar_wait(&full[sk], par, abort_flag)) {
                     ok = false;
                     return;
                 }
                 tc_fence_after();
-                const int N = j == ntiles - 1 ? n16_last * 16 : KT;
-                const uint32_t idesc = umma_idesc(kPrefillRows, N, false, false, kBf16);
-                const uint32_t kb = r_addr + (uint32_t)sk * p.slot_bytes;
+                const uint32_t idesc = j == (t ? nk1 : nk0) - 1 ? (t ? idesc_last1 : idesc_last0) : idesc_full;
+                const uint64_t ad = qdesc + (uint64_t)(t * (kQTile >> 4));
+                const uint64_t bd = kdesc + (uint64_t)(sk * slot16);
+                const uint32_t ds = tmem + (uint32_t)t * KT;
 #pragma unroll
                 for (int ks = 0; ks < KS; ++ks) {
-                    const uint64_t ad = umma_desc_sw128(q_addr + (ks >> 2) * kBlk + (ks & 3) * 32, 16, 1024);
-                    const uint64_t bd = umma_desc_sw128(kb + (ks >> 2) * kSlotBlk + (ks & 3) * 32, 16, 1024);
-                    umma_f16(tmem + (uint32_t)(j % kPrefillSBufs) * KT, ad, bd, idesc, ks > 0 ? 1u : 0u);
+                    // k-step ks: 64-column block ks / 4 (16 KB apart), 32 bytes per step inside it
+                    const uint32_t off = (uint32_t)((ks >> 2) * (kBlk >> 4) + (ks & 3) * 2);
+                    umma_f16(ds, ad + off, bd + off, idesc, ks > 0 ? 1u : 0u);
                 }
-                umma_commit(&sfull[j % kPrefillSBufs]);
-                umma_commit(&empty[sk]);
+                umma_commit(&sfull[t]);
+                // K slot j is read for the last time by the last query tile that sees tile j
+                if (t == kPrefillQTiles - 1 || j >= nk1) umma_commit(&empty[sk]);
                 issued_any = true;
             };
-            for (int j = 0; j < kPrefillSBufs && j < ntiles; ++j) s_issue(j);
-            for (int i = 0; i < ntiles && ok; ++i) {
-                pv(i);
-                if (i + kPrefillSBufs < ntiles) s_issue(i + kPrefillSBufs);
+            // O_t += P_t V_j (P high part, then low part; V of tile j in slot NH + sk);
+            // the last user of the V slot releases it
+            auto pv = [&](auto tc, int j, int sk, uint32_t par) {
+                constexpr int t = decltype(tc)::value;
+                if (!ok) return;
+                const int sv = NH + sk;
+                if (!mbar_wait(&pfull[t * 2 + (j & 1)], (uint32_t)(j >> 1) & 1u, abort_flag) ||
+                    !mbar_wait(&full[sv], par, abort_flag)) {
+                    ok = false;
+                    return;
+                }
+                tc_fence_after();
+                const uint64_t bd = vdesc + (uint64_t)(sv * slot16);  // keys 16kk.. at +16kk rows of 128 B
+                // P_t in its S buffer: keys 16kk .. 16kk+15 in columns 16kk .. 16kk+7
+                // (high parts) and 16kk+8 .. 16kk+15 (low parts), two keys per column
+                constexpr uint32_t pa_off = (uint32_t)t * KT, od_off = kColO + (uint32_t)t * D;
+                const uint32_t acc0 = j > 0 ? 1u : 0u;
+                if (j != (t ? nk1 : nk0) - 1) {
+#pragma unroll
+                    for (int kk = 0; kk < KT / 16; ++kk) {
+                        umma_f16_ts(tmem + od_off, tmem + pa_off + kk * 16, bd + (uint64_t)(kk * 128), kIdescPV,
+                                    kk > 0 ? 1u : acc0);
+                        umma_f16_ts(tmem + od_off, tmem + pa_off + kk * 16 + 8, bd + (uint64_t)(kk * 128), kIdescPV,
+                                    1u);
+                    }
+                } else {
+                    const int n16 = t ? n16_q[1] : n16_q[0];
+                    for (int kk = 0; kk < n16; ++kk) {
+                        umma_f16_ts(tmem + od_off, tmem + pa_off + kk * 16, bd + (uint64_t)(kk * 128), kIdescPV,
+                                    kk > 0 ? 1u : acc0);
+                        umma_f16_ts(tmem + od_off, tmem + pa_off + kk * 16 + 8, bd + (uint64_t)(kk * 128), kIdescPV,
+                                    1u);
+                    }
+                }
+                umma_commit(&odone[t * 2 + (j & 1)]);
+                if (t == kPrefillQTiles - 1 || j >= nk1) umma_commit(&empty[sv]);
+                issued_any = true;
+            };
+            using T0 = std::integral_constant<int, 0>;
+            using T1 = std::integral_constant<int, 1>;
+            static_assert(kPrefillQTiles == 2, "the issue order below names the two query tiles");
+            // ring position of tile j (slot j mod NH, fill parity (j / NH) & 1) and of tile j + 1
+            int sc = 0, sn = NH > 1 ? 1 : 0;
+            uint32_t pc = 0u, pn = NH > 1 ? 0u : 1u;
+            if (nk0 > 0) s_issue(T0{}, 0, sc, pc);
+            if (nk1 > 0) s_issue(T1{}, 0, sc, pc);
+            // alternate between the query tiles: while one tile's softmax runs, the
+            // tensor core takes the other tile's P V and next S
+            for (int j = 0; j < ntiles && ok; ++j) {
+                if (j < nk0) {
+                    pv(T0{}, j, sc, pc);
+                    if (j + 1 < nk0) s_issue(T0{}, j + 1, sn, pn);
+                }
+                if (j < nk1) {
+                    pv(T1{}, j, sc, pc);
+                    if (j + 1 < nk1) s_issue(T1{}, j + 1, sn, pn);
+                }
+                sc = sn;
+                pc = pn;
+                if (++sn == NH) {
+                    sn = 0;
+                    pn ^= 1u;
+                }
             }
             if (!ok) {
                 *abort_flag = 1;
@@ -294,24 +356,27 @@ __global__ void __launch_bounds__(kPrefillThreads, 1) paged_prefill_kernel(const
             }
         }
     } else {
-        // ================= softmax: two threads per row =================
-        constexpr int HC = KT / 2;            // S columns per thread
-        constexpr int HD = D / 2;             // O columns per thread
-        const int half = (warp - 2) >> 2;     // column half
+        // ================= softmax: one thread per row =================
+        constexpr int HD = D;                 // O columns per thread
+        const int qtile = (warp - 2) >> 2;    // query tile of this warp
         const int quad = warp & 3;            // tensor-memory lane quarter of this warp
         const int row = quad * 32 + lane;
-        const int sid = tid - 64;             // 0 .. 255 over the softmax warps
         const uint32_t tl = tmem + ((uint32_t)(quad * 32) << 16);  // this warp's lanes
-        uint64_t *xb = xchg + quad * 2;
+        const uint32_t sb = tl + (uint32_t)qtile * KT;             // S / P of this query tile
+        const uint32_t ob = tl + kColO + (uint32_t)qtile * D;      // O of this query tile
+        uint64_t *pf = pfull + qtile * 2, *odn = odone + qtile * 2;
         const int tok = row >> p.g_log2, hj = row & (p.G - 1);
+        const int ntok = qtile ? ntok_q[1] : ntok_q[0];
+        const int n16_last = qtile ? n16_q[1] : n16_q[0];  // 16-key groups of the tile's last key tile
+        const int tq0 = t0 + qtile * p.QT;    // first new token of this query tile
         const bool valid = tok < ntok;
-        const size_t grow = ((size_t)(q0 + t0 + tok) * p.Hq + (size_t)g * p.G + hj) * D;  // q / out row
-        // ---- Q tile: half of row `row`, K-major with the 128-byte swizzle ----
+        const size_t grow = ((size_t)(q0 + tq0 + tok) * p.Hq + (size_t)g * p.G + hj) * D;  // q / out row
+        // ---- Q tile: row `row`, K-major with the 128-byte swizzle ----
         {
             const uint4 *src = reinterpret_cast<const uint4 *>(static_cast<const unsigned char *>(p.q) + grow * E);
+            unsigned char *qs = smem + (size_t)qtile * kQTile;
 #pragma unroll
-            for (int i = 0; i < D / 16; ++i) {
-                const int c = half * (D / 16) + i;
+            for (int c = 0; c < D / 8; ++c) {
                 uint4 v = make_uint4(0u, 0u, 0u, 0u);
                 if (valid) {
                     v = __ldg(src + c);
@@ -320,62 +385,56 @@ __global__ void __launch_bounds__(kPrefillThreads, 1) paged_prefill_kernel(const
                     v.z ^= p.qflip;
                     v.w ^= p.qflip;
                 }
-                *reinterpret_cast<uint4 *>(smem + (c >> 3) * kBlk + row * 128 + (((c & 7) ^ (row & 7)) << 4)) = v;
+                *reinterpret_cast<uint4 *>(qs + (c >> 3) * kBlk + row * 128 + (((c & 7) ^ (row & 7)) << 4)) = v;
             }
             fence_async_smem();
             __syncwarp();
             if (lane == 0) mbar_arrive(qfull);
         }
-        const int pos_row = pos0 + (valid ? tok : ntok - 1);  // rows past the tokens mirror the last token
+        const int nj = qtile ? nkt[1] : nkt[0];
+        const int pos0 = L - n + tq0;                               // position of the query tile's first token
+        const int pos_row = pos0 + (valid ? tok : max(ntok, 1) - 1);  // rows past the tokens mirror the last token
         const float qs = p.qscale;
         float m_used = -INFINITY, l = 0.f;
         bool ok = true;
-        // P V completions, confirmed per barrier in order: odone[i & 1] phase
-        // i >> 1 is P_i V_i, and P_{i+2} V_{i+2} cannot complete before the
-        // softmax of tile i+2 has run, so a parity wait never skips a phase
+        // P V completions, confirmed per barrier in order: odone[j & 1] phase
+        // j >> 1 is P_j V_j, and P_{j+2} V_{j+2} cannot complete before the
+        // softmax of tile j+2 has run, so a parity wait never skips a phase
         int od_next[2] = {0, 0};
         auto od_wait = [&](int i) {
             int &nx = od_next[i & 1];
             for (; nx <= (i >> 1); ++nx)
-                if (!mbar_wait(&odone[i & 1], (uint32_t)nx & 1u, abort_flag)) return false;
+                if (!mbar_wait(&odn[i & 1], (uint32_t)nx & 1u, abort_flag)) return false;
             tc_fence_after();
             return true;
         };
-        for (int j = 0; j < ntiles; ++j) {
+        for (int j = 0; j < nj; ++j) {
             const int k0 = j * KT;
-            const uint32_t sb = tl + (uint32_t)(j % kPrefillSBufs) * KT;  // S_j, then P_j
-            if (!mbar_wait(&sfull[j % kPrefillSBufs], (uint32_t)(j / kPrefillSBufs) & 1u, abort_flag)) {
+            if (!mbar_wait(&sfull[qtile], (uint32_t)j & 1u, abort_flag)) {
                 ok = false;
                 break;
             }
             tc_fence_after();
-            float s[HC];
-            tmem_ld32(sb + half * HC, s);
-            tmem_ld32(sb + half * HC + 32, s + 32);
             // keys past the row's position (or past the keys loaded) are out
             const bool diag = k0 + KT - 1 > pos0;
-            const int lim = pos_row - k0 - half * HC;  // columns c <= lim are visible
-            float m4[4] = {-INFINITY, -INFINITY, -INFINITY, -INFINITY};
+            const int lim = pos_row - k0;  // columns c <= lim are visible
+            // ---- the whole S row in registers (one load, one wait); masked keys
+            // become -inf, so their weights below come out 0 ----
+            float sr[KT];
+            tmem_ld128(sb, sr);
             if (diag) {
 #pragma unroll
-                for (int c = 0; c < HC; ++c) {
-                    s[c] = c <= lim ? s[c] : -INFINITY;
-                    m4[c & 3] = fmaxf(m4[c & 3], s[c]);
-                }
-            } else {
+                for (int c = 0; c < KT; ++c) sr[c] = c <= lim ? sr[c] : -INFINITY;
+            }
+            float mx;
+            {
+                float m4[4] = {sr[0], sr[1], sr[2], sr[3]};
 #pragma unroll
-                for (int c = 0; c < HC; ++c) m4[c & 3] = fmaxf(m4[c & 3], s[c]);
+                for (int c = 4; c < KT; c += 8)
+#pragma unroll
+                    for (int i = 0; i < 4; ++i) m4[i] = fmax3(m4[i], sr[c + i], sr[c + 4 + i]);
+                mx = fmax3(m4[0], m4[1], fmaxf(m4[2], m4[3]));
             }
-            float mx = fmaxf(fmaxf(m4[0], m4[1]), fmaxf(m4[2], m4[3]));
-            // row maximum over both halves
-            red_s[j & 1][half][row] = mx;
-            __syncwarp();
-            if (lane == 0) mbar_arrive(&xb[j & 1]);
-            if (!mbar_wait(&xb[j & 1], (uint32_t)(j >> 1) & 1u, abort_flag)) {
-                ok = false;
-                break;
-            }
-            mx = fmaxf(mx, red_s[j & 1][half ^ 1][row]);
             const float mt = mx == -INFINITY ? -INFINITY : mx * qs;  // base-2 domain
             const bool move = mt > m_used + kPrefillRescaleLog2;
             float alpha = 1.f;
@@ -385,29 +444,49 @@ __global__ void __launch_bounds__(kPrefillThreads, 1) paged_prefill_kernel(const
             }
             const float nm = -m_used;
             l *= alpha;
+            // ---- weights, written over S as P in 16-key groups: high parts of
+            // keys 16c .. 16c+15 in columns 16c .. 16c+7, low parts in 16c+8 .. 16c+15 ----
+            float2 l2[2] = {make_float2(0.f, 0.f), make_float2(0.f, 0.f)};
+            {
+                const float2 qs2 = make_float2(qs, qs), nm2 = make_float2(nm, nm);
+                const int nch = j == nj - 1 ? n16_last : KT / 16;  // 16-key groups the P V product reads
+#pragma unroll
+                for (int c = 0; c < KT / 16; ++c) {
+                    if (c < nch) {
+                        uint32_t pw[16];
+#pragma unroll
+                        for (int i = 0; i < 8; ++i) {
+                            const float2 t = ffma2(make_float2(sr[16 * c + 2 * i], sr[16 * c + 2 * i + 1]), qs2, nm2);
+                            const float2 e = make_float2(exp2_fast(t.x), exp2_fast(t.y));
+                            l2[i & 1] = fadd2(l2[i & 1], e);
+                            Op::split_p2(e, pw[i], pw[8 + i]);
+                        }
+                        tmem_st16u(sb + c * 16, pw);
+                    }
+                }
+            }
+            l += (l2[0].x + l2[0].y) + (l2[1].x + l2[1].y);
             if (j >= 1 && __any_sync(0xffffffffu, move)) {
                 // rescale O: P_{j-1} V_{j-1} must be in it first
                 if (!od_wait(j - 1)) {
                     ok = false;
                     break;
                 }
-                {
 #pragma unroll
-                    for (int c = 0; c < HD / 32; ++c) {
-                        float o[32];
-                        tmem_ld32(tl + kColO + half * HD + c * 32, o);
+                for (int c = 0; c < HD / 32; ++c) {
+                    float o[32];
+                    tmem_ld32(ob + c * 32, o);
 #pragma unroll
-                        for (int i = 0; i < 32; ++i) o[i] *= alpha;
-                        tmem_st32(tl + kColO + half * HD + c * 32, o);
-                    }
-                    tmem_wait_st();
+                    for (int i = 0; i < 32; ++i) o[i] *= alpha;
+                    tmem_st32(ob + c * 32, o);
                 }
+                tmem_wait_st();
             }
-            if (j == ntiles - 1) {
-                // V rows of the last 16-key group past the context end are
-                // unwritten pool slots: zero them (weight 0 times anything
-                // must stay 0) once their tensor-map fill has landed
-                const int z0 = L - k0, z1 = n16_last * 16;
+            if (j == nj - 1) {
+                // V rows of the last 16-key groups this tile's P V product reads that
+                // lie past the context end are unwritten pool rows: zero them
+                // (weight 0 times anything must stay 0) once their fill has landed
+                const int z0 = max(0, L - k0), z1 = n16_last * 16;
                 if (z0 < z1) {
                     const int sv = NH + j % NH;
                     if (!mbar_wait(&full[sv], (uint32_t)(j / NH) & 1u, abort_flag)) {
@@ -415,51 +494,13 @@ __global__ void __launch_bounds__(kPrefillThreads, 1) paged_prefill_kernel(const
                         break;
                     }
                     unsigned char *vs = ring + (size_t)sv * p.slot_bytes;
-                    for (int i = sid; i < (z1 - z0) * NDC * 8; i += 32 * kPrefillSoftmaxWarps) {
+                    for (int i = quad * 32 + lane; i < (z1 - z0) * NDC * 8; i += 128) {
                         const int r = z0 + i / (NDC * 8), c = i % (NDC * 8);
                         *reinterpret_cast<uint4 *>(vs + (c >> 3) * kSlotBlk + r * 128 + ((c & 7) << 4)) =
                             make_uint4(0u, 0u, 0u, 0u);
                     }
                 }
             }
-            // ---- weights and P over S_j, 16 keys at a time: the chunk's S
-            // columns are read back and its P parts written over them (high
-            // parts in the first 8 columns, low parts in the next 8), so no
-            // column is written before its S value is read (rolled loops:
-            // small code for the warps that share a scheduler). ----
-            float l4[2] = {0.f, 0.f};
-            {
-                const uint32_t hb = sb + half * HC;  // this half's 64 columns
-                // one chunk; the causal mask only on tiles that reach the diagonal
-                auto chunk = [&](int c, auto masked) {
-                    float w[16];
-                    tmem_ld16(hb + c * 16, w);
-                    const int cl = lim - c * 16;
-                    float2 l2 = make_float2(0.f, 0.f);
-                    uint32_t pw[16];  // P high parts (words 0-7), low parts (words 8-15)
-#pragma unroll
-                    for (int i = 0; i < 8; ++i) {
-                        const float2 t = ffma2(make_float2(w[2 * i], w[2 * i + 1]), make_float2(qs, qs), make_float2(nm, nm));
-                        float2 e = make_float2(exp2_fast(t.x), exp2_fast(t.y));
-                        if constexpr (decltype(masked)::value) {
-                            e.x = 2 * i <= cl ? e.x : 0.f;
-                            e.y = 2 * i + 1 <= cl ? e.y : 0.f;
-                        }
-                        l2 = fadd2(l2, e);
-                        Op::split_p(e.x, e.y, pw[i], pw[8 + i]);
-                    }
-                    l4[c & 1] += l2.x + l2.y;
-                    tmem_st16u(hb + c * 16, pw);
-                };
-                if (diag) {
-#pragma unroll 1
-                    for (int c = 0; c < HC / 16; ++c) chunk(c, std::true_type{});
-                } else {
-#pragma unroll 1
-                    for (int c = 0; c < HC / 16; ++c) chunk(c, std::false_type{});
-                }
-            }
-            l += l4[0] + l4[1];
             // confirm P_{j-2} V_{j-2} (long done) before P_j is published: P_j V_j
             // could otherwise complete and put odone[j & 1] two phases ahead
             if (j >= 2 && !od_wait(j - 2)) {
@@ -470,33 +511,26 @@ __global__ void __launch_bounds__(kPrefillThreads, 1) paged_prefill_kernel(const
             fence_async_smem();  // V rows zeroed above
             tc_fence_before();
             __syncwarp();
-            if (lane == 0) mbar_arrive(&pfull[j & 1]);
+            if (lane == 0) mbar_arrive(&pf[j & 1]);
         }
-        if (ok && od_wait(ntiles - 1)) {  // the last product: every earlier one is done too
-            // row sum over both halves
-            red_s[ntiles & 1][half][row] = l;
-            __syncwarp();
-            if (lane == 0) mbar_arrive(&xb[ntiles & 1]);
-            ok = mbar_wait(&xb[ntiles & 1], (uint32_t)(ntiles >> 1) & 1u, abort_flag);
-            if (ok) {
-                // ---- normalise and store this half of the rows of real tokens ----
-                const float inv = 1.f / (l + red_s[ntiles & 1][half ^ 1][row]);
-                uint4 *dst = reinterpret_cast<uint4 *>(static_cast<unsigned char *>(p.out) + (grow + half * HD) * E);
+        if (ok && nj > 0 && od_wait(nj - 1)) {  // the last product: every earlier one is done too
+            // ---- normalise and store the row (real tokens only) ----
+            const float inv = 1.f / l;
+            uint4 *dst = reinterpret_cast<uint4 *>(static_cast<unsigned char *>(p.out) + grow * E);
+#pragma unroll 1
+            for (int c = 0; c < HD / 32; ++c) {
+                float o[32];
+                tmem_ld32(ob + c * 32, o);
+                if (valid) {
 #pragma unroll
-                for (int c = 0; c < HD / 32; ++c) {
-                    float o[32];
-                    tmem_ld32(tl + kColO + half * HD + c * 32, o);
-                    if (valid) {
-#pragma unroll
-                        for (int i = 0; i < 4; ++i)
-                            dst[c * 4 + i] = make_uint4(Op::pack(o[8 * i] * inv, o[8 * i + 1] * inv),
-                                                        Op::pack(o[8 * i + 2] * inv, o[8 * i + 3] * inv),
-                                                        Op::pack(o[8 * i + 4] * inv, o[8 * i + 5] * inv),
-                                                        Op::pack(o[8 * i + 6] * inv, o[8 * i + 7] * inv));
-                    }
+                    for (int i = 0; i < 4; ++i)
+                        dst[c * 4 + i] = make_uint4(Op::pack(o[8 * i] * inv, o[8 * i + 1] * inv),
+                                                    Op::pack(o[8 * i + 2] * inv, o[8 * i + 3] * inv),
+                                                    Op::pack(o[8 * i + 4] * inv, o[8 * i + 5] * inv),
+                                                    Op::pack(o[8 * i + 6] * inv, o[8 * i + 7] * inv));
                 }
             }
-        } else {
+        } else if (nj > 0) {
             ok = false;
         }
         if (!ok) {

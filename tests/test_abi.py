@@ -203,7 +203,7 @@ def test_decode_rejects_bad_dynamic_share(share, mode_fixed):
 def test_prefill_plan_shapes_and_rejections():
     s = pa.Shape(8, 32, 8, 128, 16, 4096, 256, pa.DTYPE_BF16)
     plan = pa.pa_prefill_plan(s, 512)
-    assert plan.q_tile * 4 == 128 and plan.num_qtiles == 512 // plan.q_tile and plan.stages >= 2
+    assert plan.q_tile * 4 == 128 and plan.num_qtiles == 512 // (2 * plan.q_tile) and plan.stages >= 2
     assert plan.smem_bytes <= 232448
     for bad, status in ((pa.Shape(2, 8, 2, 128, 16, 64, 8, pa.DTYPE_F32), pa.PA_ERR_UNSUPPORTED),
                         (pa.Shape(2, 8, 2, 96, 16, 64, 8, pa.DTYPE_BF16), pa.PA_ERR_UNSUPPORTED),
@@ -228,7 +228,7 @@ def test_prefill_plan_budget_over_supported_shapes(D, dtype):
             plan = pa.pa_prefill_plan(s, 100)
             assert plan.q_tile * G == 128 and plan.kv_tile == 128
             assert 2 <= 2 * plan.stages and plan.smem_bytes + 3072 <= 232448
-            assert plan.num_qtiles == -(-100 // plan.q_tile)
+            assert plan.num_qtiles == -(-100 // (2 * plan.q_tile))   # two query tiles per CTA
 
 
 @pytest.mark.parametrize("field,value", [("head_group", 0), ("head_group", 3), ("stages", 9), ("tile_tokens", 48),
