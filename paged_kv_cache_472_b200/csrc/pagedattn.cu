@@ -792,7 +792,10 @@ pa_status pa_prefill(const void *q, const void *k_cache, const void *v_cache, co
         cudaError_t e = cudaFuncSetAttribute(fn, cudaFuncAttributeMaxDynamicSharedMemorySize, plan->smem_bytes);
         if (e != cudaSuccess) return fail(PA_ERR_CUDA, "cudaFuncSetAttribute: %s", cudaGetErrorString(e));
     }
-    dim3 grid((unsigned)plan->num_qtiles, (unsigned)s->Hkv, (unsigned)s->B);
+    // one CTA per (request, CTA tile, KV head); the kernel ranks the pairs by work
+    const long long nctas = (long long)plan->num_qtiles * s->Hkv * s->B;
+    if (nctas > 0x7FFFFFFFll) return fail(PA_ERR_INVALID_ARG, "too many prefill tiles for one grid");
+    dim3 grid((unsigned)nctas);
     fn<<<grid, pa::kPrefillThreads, (size_t)plan->smem_bytes, (cudaStream_t)stream>>>(p);
     cudaError_t e = cudaGetLastError();
     if (e != cudaSuccess) return fail(PA_ERR_CUDA, "prefill launch: %s", cudaGetErrorString(e));

@@ -15,8 +15,9 @@
 // r / G, head r % G), so every K/V tile staged in shared memory serves both
 // query tiles and the whole head group.  The CTA streams keys 0 .. pos(last
 // token of the tile) in tiles of 128 and masks, per row, the keys past the
-// row's own position; query tile A stops at its own last position.  Tiles
-// holding the latest tokens see the most keys; the grid runs them first.
+// row's own position; query tile A stops at its own last position.  Every
+// CTA ranks the (request, CTA tile) pairs by their key tiles, from the
+// lengths, and takes the pair of its own rank: heavy pairs start first.
 //
 // Inside a CTA (5th-generation tensor cores, accumulators in tensor memory):
 //   warps 0,10 producers of K and of V: each walks the block table (one tile
@@ -66,6 +67,7 @@ constexpr int kPrefillThreads = (3 + kPrefillSoftmaxWarps) * 32;  // K producer,
 constexpr int kPrefillTmemCols = 512; // S / P of both query tiles (2 x 128 columns) + O of both (2 x D)
 constexpr int kPrefillMaxSlots = 8;   // K / V ring slots
 constexpr float kPrefillRescaleLog2 = 8.f;
+constexpr int kPrefillMaxRankedPairs = 2048;  // (request, CTA tile) pairs ranked in-kernel
 
 struct PrefillParams {
     CUtensorMap tmap_k;  // box {64 d, br rows, 1 head} on [d, token row, head] views of the pools
@@ -105,8 +107,9 @@ __global__ void __launch_bounds__(kPrefillThreads, 1) paged_prefill_kernel(const
     static_assert(kBlk == kSlotBlk, "Q and K blocks share the k-step offsets");
     extern __shared__ __align__(1024) unsigned char smem_raw[];
     unsigned char *smem = smem_raw;  // the plan leaves no room to realign: checked below
-    // mbarriers: full[], empty[] (ring), sfull[2] (per query tile), pfull[2][2] and
-    // odone[2][2] (per query tile and key-tile parity), qfull, fin
+    // mbarriers: full[], empty[] (ring), sfull[2] (per query tile), pfull[2][2] (per
+    // query tile and half of the key tile), odone[2][2] (per query tile and key-tile
+    // parity), qfull, fin
     constexpr int kOffSfull = 2 * kPrefillMaxSlots, kOffPfull = kOffSfull + 2;
     constexpr int kOffOdone = kOffPfull + 4, kOffQfull = kOffOdone + 4, kOffFin = kOffQfull + 1;
     constexpr int kBars = kOffFin + 1;
@@ -118,7 +121,7 @@ __global__ void __launch_bounds__(kPrefillThreads, 1) paged_prefill_kernel(const
     const int NH = p.nslots / 2;  // K slots 0 .. NH-1, V slots NH .. 2NH-1
     uint64_t *full = bars, *empty = bars + kPrefillMaxSlots;
     uint64_t *sfull = bars + kOffSfull;  // [query tile]: its S product done (one phase per key tile)
-    uint64_t *pfull = bars + kOffPfull;  // [query tile][key-tile parity]: P written
+    uint64_t *pfull = bars + kOffPfull;  // [query tile][half]: P of keys 64h .. 64h+63 written
     uint64_t *odone = bars + kOffOdone;  // [query tile][key-tile parity]: P V product done
     uint64_t *qfull = bars + kOffQfull, *fin = bars + kOffFin;
     volatile int *abort_flag = &abort_s;
@@ -128,14 +131,91 @@ __global__ void __launch_bounds__(kPrefillThreads, 1) paged_prefill_kernel(const
         return;
     }
     // ---- the CTA's tile: request, KV head, new tokens [t0, t0 + ntok) ----
-    const int b = blockIdx.z, g = blockIdx.y;
-    const int qt = p.num_qtiles - 1 - (int)blockIdx.x;  // latest (heaviest) tiles first
+    // ---- the CTA's (request, CTA tile) pair: pairs ranked by their key tiles,
+    // heaviest first, so the hardware's in-order dispatch of CTAs to free SMs
+    // is a longest-first list schedule; the KV heads of a pair are consecutive ----
+    const int g = (int)(blockIdx.x % (unsigned)p.Hkv);
+    const int rank = (int)(blockIdx.x / (unsigned)p.Hkv);
+    int pair;
+    {
+        const int npairs = p.B * p.num_qtiles;
+        if (npairs <= kPrefillMaxRankedPairs) {
+            __shared__ int hist[256];
+            __shared__ uint8_t bucket_of[kPrefillMaxRankedPairs];
+            __shared__ int pick;
+            for (int i = tid; i < 256; i += kPrefillThreads) hist[i] = 0;
+            __syncthreads();
+            for (int i = tid; i < npairs; i += kPrefillThreads) {
+                const int bb = i / p.num_qtiles, qq = i - bb * p.num_qtiles;
+                const int Lb = p.context_lens[bb], nb = p.query_start[bb + 1] - p.query_start[bb];
+                const int tt0 = qq * kPrefillQTiles * p.QT;
+                int work = 0;  // key tiles of the pair's query tiles (0: no tokens, or a bad length)
+                if (nb > tt0 && nb <= Lb && Lb <= p.max_blocks * p.bs) {
+#pragma unroll
+                    for (int t = 0; t < kPrefillQTiles; ++t) {
+                        const int last = min(nb, tt0 + (t + 1) * p.QT);  // tokens up to the tile's last
+                        if (last > tt0 + t * p.QT) work += (Lb - nb + last + KT - 1) / KT;
+                    }
+                }
+                const int bk = work > 0 ? 1 + min(work, 254) : 0;
+                bucket_of[i] = (uint8_t)bk;
+                atomicAdd(&hist[bk], 1);
+            }
+            __syncthreads();
+            if (warp == 0) {
+                // lane l sums buckets 255 - 8l .. 248 - 8l; a prefix over the lanes gives
+                // the pairs heavier than each lane's range
+                int s8 = 0;
+#pragma unroll
+                for (int k = 0; k < 8; ++k) s8 += hist[255 - 8 * lane - k];
+                int incl = s8;
+#pragma unroll
+                for (int o = 1; o < 32; o <<= 1) {
+                    const int v = __shfl_up_sync(0xffffffffu, incl, o);
+                    if (lane >= o) incl += v;
+                }
+                const int holder = __ffs(__ballot_sync(0xffffffffu, rank < incl)) - 1;
+                int bk = 0, before = incl - s8;
+                if (lane == holder) {
+                    for (int k = 0; k < 8; ++k) {
+                        const int c = hist[255 - 8 * lane - k];
+                        if (rank < before + c) {
+                            bk = 255 - 8 * lane - k;
+                            break;
+                        }
+                        before += c;
+                    }
+                }
+                bk = __shfl_sync(0xffffffffu, bk, holder);
+                before = __shfl_sync(0xffffffffu, before, holder);
+                // the (rank - before)-th pair of bucket bk, in index order
+                int want = rank - before;
+                for (int base = 0; base < npairs; base += 32) {
+                    const int i = base + lane;
+                    const bool hit = i < npairs && bucket_of[i] == bk;
+                    const unsigned hm = __ballot_sync(0xffffffffu, hit);
+                    const int c = __popc(hm);
+                    if (want < c) {
+                        if (hit && __popc(hm & ((1u << lane) - 1u)) == want) pick = i;
+                        break;
+                    }
+                    want -= c;
+                }
+            }
+            __syncthreads();
+            pair = pick;
+        } else {
+            // too many pairs to rank: requests in order, each one's latest tiles first
+            pair = (rank / p.num_qtiles) * p.num_qtiles + (p.num_qtiles - 1 - rank % p.num_qtiles);
+        }
+    }
+    const int b = pair / p.num_qtiles, qt = pair - b * p.num_qtiles;
     const int cap = p.max_blocks * p.bs;
     const int L = p.context_lens[b];
     const int q0 = p.query_start[b];
     const int n = p.query_start[b + 1] - q0;
     if (L < 0 || L > cap || n < 0 || n > L || n > p.num_qtiles * kPrefillQTiles * p.QT) {
-        if (tid == 0 && blockIdx.x == 0 && blockIdx.y == 0) set_error(p.error, PA_DEVERR_CONTEXT_LEN);
+        if (tid == 0 && g == 0 && qt == 0) set_error(p.error, PA_DEVERR_CONTEXT_LEN);
         return;
     }
     const int t0 = qt * kPrefillQTiles * p.QT;
@@ -161,7 +241,7 @@ __global__ void __launch_bounds__(kPrefillThreads, 1) paged_prefill_kernel(const
         for (int t = 0; t < kPrefillQTiles; ++t) {
             mbar_init(&sfull[t], 1);
             for (int par = 0; par < 2; ++par) {
-                mbar_init(&pfull[t * 2 + par], 4);  // the four warps of query tile t
+                mbar_init(&pfull[t * 2 + par], 4);  // the four warps of query tile t, per half
                 mbar_init(&odone[t * 2 + par], 1);
             }
         }
@@ -280,14 +360,17 @@ __global__ void __launch_bounds__(kPrefillThreads, 1) paged_prefill_kernel(const
                 if (t == kPrefillQTiles - 1 || j >= nk1) umma_commit(&empty[sk]);
                 issued_any = true;
             };
-            // O_t += P_t V_j (P high part, then low part; V of tile j in slot NH + sk);
-            // the last user of the V slot releases it
-            auto pv = [&](auto tc, int j, int sk, uint32_t par) {
-                constexpr int t = decltype(tc)::value;
+            // O_t += P_t V_j over keys 64h .. 64h+63 (each 16-key group: P high part,
+            // then low part; V of tile j in slot NH + sk).  The softmax publishes P
+            // in two halves, so the first half's products overlap the second
+            // half's weights.  After the second half the last user of the V slot
+            // releases it.
+            auto pv = [&](auto tc, auto hc, int j, int sk, uint32_t par) {
+                constexpr int t = decltype(tc)::value, h = decltype(hc)::value;
                 if (!ok) return;
                 const int sv = NH + sk;
-                if (!mbar_wait(&pfull[t * 2 + (j & 1)], (uint32_t)(j >> 1) & 1u, abort_flag) ||
-                    !mbar_wait(&full[sv], par, abort_flag)) {
+                if (!mbar_wait(&pfull[t * 2 + h], (uint32_t)j & 1u, abort_flag) ||
+                    (h == 0 && !mbar_wait(&full[sv], par, abort_flag))) {
                     ok = false;
                     return;
                 }
@@ -296,30 +379,37 @@ __global__ void __launch_bounds__(kPrefillThreads, 1) paged_prefill_kernel(const
                 // P_t in its S buffer: keys 16kk .. 16kk+15 in columns 16kk .. 16kk+7
                 // (high parts) and 16kk+8 .. 16kk+15 (low parts), two keys per column
                 constexpr uint32_t pa_off = (uint32_t)t * KT, od_off = kColO + (uint32_t)t * D;
+                constexpr int kH = KT / 32;  // 16-key groups per half
                 const uint32_t acc0 = j > 0 ? 1u : 0u;
                 if (j != (t ? nk1 : nk0) - 1) {
 #pragma unroll
-                    for (int kk = 0; kk < KT / 16; ++kk) {
+                    for (int kk = h * kH; kk < (h + 1) * kH; ++kk) {
                         umma_f16_ts(tmem + od_off, tmem + pa_off + kk * 16, bd + (uint64_t)(kk * 128), kIdescPV,
                                     kk > 0 ? 1u : acc0);
                         umma_f16_ts(tmem + od_off, tmem + pa_off + kk * 16 + 8, bd + (uint64_t)(kk * 128), kIdescPV,
                                     1u);
                     }
                 } else {
-                    const int n16 = t ? n16_q[1] : n16_q[0];
-                    for (int kk = 0; kk < n16; ++kk) {
+                    const int n16 = min(t ? n16_q[1] : n16_q[0], (h + 1) * kH);
+                    for (int kk = h * kH; kk < n16; ++kk) {
                         umma_f16_ts(tmem + od_off, tmem + pa_off + kk * 16, bd + (uint64_t)(kk * 128), kIdescPV,
                                     kk > 0 ? 1u : acc0);
                         umma_f16_ts(tmem + od_off, tmem + pa_off + kk * 16 + 8, bd + (uint64_t)(kk * 128), kIdescPV,
                                     1u);
                     }
                 }
-                umma_commit(&odone[t * 2 + (j & 1)]);
-                if (t == kPrefillQTiles - 1 || j >= nk1) umma_commit(&empty[sv]);
+                if (h == 1) {
+                    umma_commit(&odone[t * 2 + (j & 1)]);
+                    if (t == kPrefillQTiles - 1 || j >= nk1) umma_commit(&empty[sv]);
+                }
                 issued_any = true;
             };
             using T0 = std::integral_constant<int, 0>;
             using T1 = std::integral_constant<int, 1>;
+            auto pv_both = [&](auto tc, int j, int sk, uint32_t par) {
+                pv(tc, T0{}, j, sk, par);
+                pv(tc, T1{}, j, sk, par);
+            };
             static_assert(kPrefillQTiles == 2, "the issue order below names the two query tiles");
             // ring position of tile j (slot j mod NH, fill parity (j / NH) & 1) and of tile j + 1
             int sc = 0, sn = NH > 1 ? 1 : 0;
@@ -330,11 +420,11 @@ __global__ void __launch_bounds__(kPrefillThreads, 1) paged_prefill_kernel(const
             // tensor core takes the other tile's P V and next S
             for (int j = 0; j < ntiles && ok; ++j) {
                 if (j < nk0) {
-                    pv(T0{}, j, sc, pc);
+                    pv_both(T0{}, j, sc, pc);
                     if (j + 1 < nk0) s_issue(T0{}, j + 1, sn, pn);
                 }
                 if (j < nk1) {
-                    pv(T1{}, j, sc, pc);
+                    pv_both(T1{}, j, sc, pc);
                     if (j + 1 < nk1) s_issue(T1{}, j + 1, sn, pn);
                 }
                 sc = sn;
@@ -444,41 +534,20 @@ __global__ void __launch_bounds__(kPrefillThreads, 1) paged_prefill_kernel(const
             }
             const float nm = -m_used;
             l *= alpha;
-            // ---- weights, written over S as P in 16-key groups: high parts of
-            // keys 16c .. 16c+15 in columns 16c .. 16c+7, low parts in 16c+8 .. 16c+15 ----
-            float2 l2[2] = {make_float2(0.f, 0.f), make_float2(0.f, 0.f)};
-            {
-                const float2 qs2 = make_float2(qs, qs), nm2 = make_float2(nm, nm);
-                const int nch = j == nj - 1 ? n16_last : KT / 16;  // 16-key groups the P V product reads
-#pragma unroll
-                for (int c = 0; c < KT / 16; ++c) {
-                    if (c < nch) {
-                        uint32_t pw[16];
-#pragma unroll
-                        for (int i = 0; i < 8; ++i) {
-                            const float2 t = ffma2(make_float2(sr[16 * c + 2 * i], sr[16 * c + 2 * i + 1]), qs2, nm2);
-                            const float2 e = make_float2(exp2_fast(t.x), exp2_fast(t.y));
-                            l2[i & 1] = fadd2(l2[i & 1], e);
-                            Op::split_p2(e, pw[i], pw[8 + i]);
-                        }
-                        tmem_st16u(sb + c * 16, pw);
-                    }
-                }
-            }
-            l += (l2[0].x + l2[0].y) + (l2[1].x + l2[1].y);
             if (j >= 1 && __any_sync(0xffffffffu, move)) {
                 // rescale O: P_{j-1} V_{j-1} must be in it first
                 if (!od_wait(j - 1)) {
                     ok = false;
                     break;
                 }
+#pragma unroll 1
+                for (int c = 0; c < HD / 16; ++c) {
+                    float o[16];
+                    tmem_ld16(ob + c * 16, o);
+                    uint32_t w[16];
 #pragma unroll
-                for (int c = 0; c < HD / 32; ++c) {
-                    float o[32];
-                    tmem_ld32(ob + c * 32, o);
-#pragma unroll
-                    for (int i = 0; i < 32; ++i) o[i] *= alpha;
-                    tmem_st32(ob + c * 32, o);
+                    for (int i = 0; i < 16; ++i) w[i] = __float_as_uint(o[i] * alpha);
+                    tmem_st16u(ob + c * 16, w);
                 }
                 tmem_wait_st();
             }
@@ -507,11 +576,36 @@ __global__ void __launch_bounds__(kPrefillThreads, 1) paged_prefill_kernel(const
                 ok = false;
                 break;
             }
-            tmem_wait_st();
-            fence_async_smem();  // V rows zeroed above
-            tc_fence_before();
-            __syncwarp();
-            if (lane == 0) mbar_arrive(&pf[j & 1]);
+            // ---- weights, written over S as P in 16-key groups: high parts of
+            // keys 16c .. 16c+15 in columns 16c .. 16c+7, low parts in 16c+8 ..
+            // 16c+15; each half of the tile is published as soon as it is written ----
+            float2 l2[2] = {make_float2(0.f, 0.f), make_float2(0.f, 0.f)};
+            {
+                const float2 qs2 = make_float2(qs, qs), nm2 = make_float2(nm, nm);
+                const int nch = j == nj - 1 ? n16_last : KT / 16;  // 16-key groups the P V product reads
+#pragma unroll
+                for (int c = 0; c < KT / 16; ++c) {
+                    if (c < nch) {
+                        uint32_t pw[16];
+#pragma unroll
+                        for (int i = 0; i < 8; ++i) {
+                            const float2 t = ffma2(make_float2(sr[16 * c + 2 * i], sr[16 * c + 2 * i + 1]), qs2, nm2);
+                            const float2 e = make_float2(exp2_fast(t.x), exp2_fast(t.y));
+                            l2[i & 1] = fadd2(l2[i & 1], e);
+                            Op::split_p2(e, pw[i], pw[8 + i]);
+                        }
+                        tmem_st16u(sb + c * 16, pw);
+                    }
+                    if (c == KT / 32 - 1 || c == KT / 16 - 1) {
+                        tmem_wait_st();
+                        if (c == KT / 32 - 1) fence_async_smem();  // V rows zeroed above
+                        tc_fence_before();
+                        __syncwarp();
+                        if (lane == 0) mbar_arrive(&pf[c == KT / 16 - 1 ? 1 : 0]);
+                    }
+                }
+            }
+            l += (l2[0].x + l2[0].y) + (l2[1].x + l2[1].y);
         }
         if (ok && nj > 0 && od_wait(nj - 1)) {  // the last product: every earlier one is done too
             // ---- normalise and store the row (real tokens only) ----
