@@ -67,8 +67,9 @@ def parse():
     ap.add_argument("--e2e-steps", type=int, default=200)
     ap.add_argument("--min-timed-ms", type=float, default=250.0,
                     help="repeat the K-step region until the timed kernels span this long in total")
-    ap.add_argument("--extra", default="2,3,4",
-                    help="other decode workloads timed in regions of their own (comma list; '' = none)")
+    ap.add_argument("--extra", default="2,3,4,4:0",
+                    help="other decode workloads timed in regions of their own (comma list of C or C:P, "
+                         "P = partition tokens, 0 = balanced split; '' = none)")
     ap.add_argument("--prefill", type=int, default=0,
                     help="time the chunked prefill step of prefill workload N (1, 2) instead of the decode step")
     ap.add_argument("--dynamic-share", type=int, default=-1,
@@ -422,7 +423,7 @@ def timed_regions(fn, K: int, stream, min_ms: float, world: int, est_ms_step: fl
     return statistics.median(times), n, times
 
 
-def decode_workload(cid, args, world, rank, local, stream, lib, pa, extra=False):
+def decode_workload(cid, args, world, rank, local, stream, lib, pa, extra=False, partition=None):
     """Upload workload `cid` (rank-seeded) in rotating copies and time its
     step (fused append + decode), the decode kernel alone and (main
     workload) the step behind a copy kernel and the end-to-end step."""
@@ -434,7 +435,8 @@ def decode_workload(cid, args, world, rank, local, stream, lib, pa, extra=False)
     from paged_kv_cache_472_b200.session import PagedDecoder, StepStaging
 
     case = synth.make_config(cid, seed=rank_seed(cid, rank))
-    pt = case.partition_tokens if args.partition < 0 else args.partition
+    part = args.partition if partition is None else partition
+    pt = case.partition_tokens if part < 0 else part
     ab = algorithmic_bytes(case)
     l2 = torch.cuda.get_device_properties(local).L2_cache_size
     R = max(3, math.ceil(3 * l2 / max(ab["step_total"], 1)))
@@ -562,14 +564,23 @@ def main():
         dist.init_process_group("nccl", timeout=timedelta(seconds=120))
     stream = torch.cuda.current_stream()
     peak, peak_kind = measured_peak()
-    extras = [int(x) for x in args.extra.split(",") if x.strip() and int(x) != args.config]
+    # extra workloads: "C" (its own partition size) or "C:P" (partition size P, 0 = balanced split)
+    extras = []
+    for x in args.extra.split(","):
+        if not x.strip():
+            continue
+        cid, _, part = x.partition(":")
+        if int(cid) == args.config and not part:
+            continue
+        extras.append((int(cid), int(part) if part else None))
 
     m = decode_workload(args.config, args, world, rank, local, stream, pa.lib, pa)
     others = {}
-    for cid in extras:
-        r = decode_workload(cid, args, world, rank, local, stream, pa.lib, pa, extra=True)
+    for cid, part in extras:
+        r = decode_workload(cid, args, world, rank, local, stream, pa.lib, pa, extra=True, partition=part)
         ab = r["ab"]
-        others[r["case"].name] = {
+        key = r["case"].name + ("" if part is None else ("-balanced" if part == 0 else f"-partition{part}"))
+        others[key] = {
             "step_us": round(r["ms_step"] * 1e3, 3), "decode_us": round(r["ms_decode"] * 1e3, 3),
             "decode_gbs": round(ab["decode_unique"] / (r["ms_decode"] * 1e-3) / 1e9, 1),
             "frac": round(ab["decode_unique"] / (r["ms_decode"] * 1e-3) / 1e9 / peak, 4),

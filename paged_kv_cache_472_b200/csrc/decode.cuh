@@ -2510,6 +2510,7 @@ __global__ void __launch_bounds__(kMergeThreads) paged_merge_kernel(const __grid
         sm_l[warp] = den;
     }
     if (act) sm_o[warp][lane] = num;
+    __syncwarp();  // each warp meets the CTA barrier whole
     __syncthreads();
     if (warp != 0 || !act) return;
     float Mx = -INFINITY;

@@ -632,6 +632,11 @@ __global__ void __launch_bounds__(kPrefillThreads, 1) paged_prefill_kernel(const
             if (lane == 0) set_error(p.error, PA_DEVERR_TIMEOUT);
         }
     }
+    // Every warp reaches the CTA barrier whole: one lane of warp 1 issued the
+    // products while the others went ahead, and a barrier met by part of a warp
+    // does not hold the rest of the CTA (tensor memory must outlive the last
+    // read of O).
+    __syncwarp();
     tc_fence_before();
     __syncthreads();
     if (warp == 1) {
