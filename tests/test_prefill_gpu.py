@@ -86,6 +86,24 @@ def test_prefill_edge_shapes(orc, name, dtype, Hq, Hkv, D, bs, lens, new):
     check(orc, pc, name)
 
 
+def test_prefill_more_pairs_than_ranked(orc):
+    """More (request, CTA tile) pairs than the kernel ranks in shared memory
+    (1100 requests x 2 tiles): the CTAs fall back to taking the pairs in
+    request order, every row still against the oracle."""
+    rng = np.random.default_rng(5)
+    B = 1100
+    new = rng.integers(1, 4, size=B)
+    new[7] = 200  # one long chunk: two CTA tiles of 2 x 64 tokens per request
+    lens = new + rng.integers(0, 40, size=B)
+    pc = synth.build_prefill_case("many_pairs", dtype="bf16", Hq=4, Hkv=2, D=64, block_size=16,
+                                  context_lens=lens.tolist(), new_tokens=new.tolist(), seed=23, pool="factor",
+                                  pool_factor=1.25)
+    dev, err, plan = run_prefill(pc)
+    assert pc.B * plan.num_qtiles > 2048
+    assert err == 0, f"device error word {err:#x}"
+    H.assert_close(out_f64(dev), orc.prefill(pc), pc.dtype, pc.name)
+
+
 @pytest.mark.parametrize("scale", [-0.2, 0.0, 0.5])
 def test_prefill_any_scale(orc, scale):
     """A negative scale (the kernel feeds q negated and uses |scale|), zero
