@@ -70,6 +70,9 @@ def parse():
     ap.add_argument("--extra", default="2,3,4,4:0",
                     help="other decode workloads timed in regions of their own (comma list of C or C:P, "
                          "P = partition tokens, 0 = balanced split; '' = none)")
+    ap.add_argument("--copies", type=int, default=0,
+                    help="rotating input copies of a decode workload (0: enough to exceed L2 three times; "
+                         "1 only for profiler captures, whose passes flush the caches themselves)")
     ap.add_argument("--prefill", type=int, default=0,
                     help="time the chunked prefill step of prefill workload N (1, 2) instead of the decode step")
     ap.add_argument("--dynamic-share", type=int, default=-1,
@@ -439,7 +442,7 @@ def decode_workload(cid, args, world, rank, local, stream, lib, pa, extra=False,
     pt = case.partition_tokens if part < 0 else part
     ab = algorithmic_bytes(case)
     l2 = torch.cuda.get_device_properties(local).L2_cache_size
-    R = max(3, math.ceil(3 * l2 / max(ab["step_total"], 1)))
+    R = max(3, math.ceil(3 * l2 / max(ab["step_total"], 1))) if args.copies <= 0 else args.copies
     copies = [upload(case) for _ in range(R)]
     dec = PagedDecoder(pa.Shape(*shape_fields(case)), int(case.max_blocks_per_seq * case.block_size), pt)
     if args.dynamic_share >= 0 and not extra:
