@@ -105,6 +105,12 @@ __global__ void __launch_bounds__(kPrefillThreads, 1) paged_prefill_kernel(const
     constexpr uint32_t kColO = kPrefillQTiles * KT;    // tensor-memory column of O of query tile 0
     static_assert(kPrefillQTiles * (KT + D) <= kPrefillTmemCols, "tensor memory");
     static_assert(kBlk == kSlotBlk, "Q and K blocks share the k-step offsets");
+    // At D = 64 the 512 columns leave 64 per query tile for the second half of P:
+    // the next S can then go over the S buffer as soon as the first half's P V is
+    // issued, while the softmax still computes the second half (it holds the
+    // whole S row in registers from its one load).
+    constexpr bool kP2Own = kPrefillQTiles * (KT + D) + kPrefillQTiles * (KT / 2) <= kPrefillTmemCols;
+    constexpr uint32_t kColP2 = kPrefillQTiles * (KT + D);  // second-half P of query tile 0, when kP2Own
     extern __shared__ __align__(1024) unsigned char smem_raw[];
     unsigned char *smem = smem_raw;  // the plan leaves no room to realign: checked below
     // mbarriers: full[], empty[] (ring), sfull[2] (per query tile), pfull[2][2] (per
@@ -378,8 +384,11 @@ __global__ void __launch_bounds__(kPrefillThreads, 1) paged_prefill_kernel(const
                 const uint64_t bd = vdesc + (uint64_t)(sv * slot16);  // keys 16kk.. at +16kk rows of 128 B
                 // P_t in its S buffer: keys 16kk .. 16kk+15 in columns 16kk .. 16kk+7
                 // (high parts) and 16kk+8 .. 16kk+15 (low parts), two keys per column
-                constexpr uint32_t pa_off = (uint32_t)t * KT, od_off = kColO + (uint32_t)t * D;
                 constexpr int kH = KT / 32;  // 16-key groups per half
+                // A of group kk at column pa_off + 16 kk (the second half from its own columns when kP2Own)
+                constexpr uint32_t pa_off = (kP2Own && h == 1) ? kColP2 + (uint32_t)(t * (KT / 2) - kH * 16)
+                                                               : (uint32_t)t * KT;
+                constexpr uint32_t od_off = kColO + (uint32_t)t * D;
                 const uint32_t acc0 = j > 0 ? 1u : 0u;
                 if (j != (t ? nk1 : nk0) - 1) {
 #pragma unroll
@@ -419,13 +428,27 @@ __global__ void __launch_bounds__(kPrefillThreads, 1) paged_prefill_kernel(const
             // alternate between the query tiles: while one tile's softmax runs, the
             // tensor core takes the other tile's P V and next S
             for (int j = 0; j < ntiles && ok; ++j) {
-                if (j < nk0) {
-                    pv_both(T0{}, j, sc, pc);
-                    if (j + 1 < nk0) s_issue(T0{}, j + 1, sn, pn);
-                }
-                if (j < nk1) {
-                    pv_both(T1{}, j, sc, pc);
-                    if (j + 1 < nk1) s_issue(T1{}, j + 1, sn, pn);
+                if constexpr (kP2Own) {
+                    // first half's P V, the next S over the S buffer, then the second half's P V
+                    if (j < nk0) {
+                        pv(T0{}, T0{}, j, sc, pc);
+                        if (j + 1 < nk0) s_issue(T0{}, j + 1, sn, pn);
+                        pv(T0{}, T1{}, j, sc, pc);
+                    }
+                    if (j < nk1) {
+                        pv(T1{}, T0{}, j, sc, pc);
+                        if (j + 1 < nk1) s_issue(T1{}, j + 1, sn, pn);
+                        pv(T1{}, T1{}, j, sc, pc);
+                    }
+                } else {
+                    if (j < nk0) {
+                        pv_both(T0{}, j, sc, pc);
+                        if (j + 1 < nk0) s_issue(T0{}, j + 1, sn, pn);
+                    }
+                    if (j < nk1) {
+                        pv_both(T1{}, j, sc, pc);
+                        if (j + 1 < nk1) s_issue(T1{}, j + 1, sn, pn);
+                    }
                 }
                 sc = sn;
                 pc = pn;
@@ -585,6 +608,8 @@ __global__ void __launch_bounds__(kPrefillThreads, 1) paged_prefill_kernel(const
                 const int nch = j == nj - 1 ? n16_last : KT / 16;  // 16-key groups the P V product reads
 #pragma unroll
                 for (int c = 0; c < KT / 16; ++c) {
+                    if (kP2Own && c == KT / 32 && j >= 1 && c < nch && !od_wait(j - 1))
+                        ok = false;  // the second half's columns are free once P_{j-1} V_{j-1} is done
                     if (c < nch) {
                         uint32_t pw[16];
 #pragma unroll
@@ -594,7 +619,10 @@ __global__ void __launch_bounds__(kPrefillThreads, 1) paged_prefill_kernel(const
                             l2[i & 1] = fadd2(l2[i & 1], e);
                             Op::split_p2(e, pw[i], pw[8 + i]);
                         }
-                        tmem_st16u(sb + c * 16, pw);
+                        if (kP2Own && c >= KT / 32)
+                            tmem_st16u(tl + kColP2 + (uint32_t)(qtile * (KT / 2) + (c - KT / 32) * 16), pw);
+                        else
+                            tmem_st16u(sb + c * 16, pw);
                     }
                     if (c == KT / 32 - 1 || c == KT / 16 - 1) {
                         tmem_wait_st();
@@ -606,6 +634,7 @@ __global__ void __launch_bounds__(kPrefillThreads, 1) paged_prefill_kernel(const
                 }
             }
             l += (l2[0].x + l2[0].y) + (l2[1].x + l2[1].y);
+            if (!ok) break;
         }
         if (ok && nj > 0 && od_wait(nj - 1)) {  // the last product: every earlier one is done too
             // ---- normalise and store the row (real tokens only) ----
